@@ -1,0 +1,49 @@
+"""The seeded input generator: determinism and the storage formats it writes."""
+import numpy as np
+import torch
+
+import csa_inputs as CI
+from oracle import csa_oracle as O
+
+
+def test_deterministic():
+    a = CI.make_workload(0)
+    b = CI.make_workload(0)
+    for k in a.tensors:
+        assert np.array_equal(a.tensors[k], b.tensors[k]), k
+
+
+def test_e4m3_rows_roundtrip():
+    x = torch.randn(64, 128, generator=torch.Generator().manual_seed(3))
+    codes, scale = CI.quant_e4m3_rows(x)
+    v = O.decode_e4m3(codes) * scale[:, None]
+    # every row uses the full range: its largest magnitude maps to 448
+    assert np.all(np.abs(O.decode_e4m3(codes)).max(axis=1) == 448.0)
+    # error within half an e4m3 ulp (relative 2^-4) of each value
+    err = np.abs(v - x.numpy()) / np.maximum(np.abs(x.numpy()), 2.0 ** -6 * scale[:, None])
+    assert err.max() <= 2.0 ** -4 + 1e-7
+
+
+def test_mxfp4_rows_rne_and_scales():
+    x = torch.tensor([[0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, -5.0] + [0.0] * 23 + [6.0]])
+    packed, sc = CI.quant_mxfp4_rows(x)
+    assert sc.tolist() == [[127]]                      # amax 6 -> scale 2^0
+    v = O.decode_e2m1_packed(packed)
+    assert v[0, :8].tolist() == [0.0, 1.0, 1.0, 2.0, 2.0, 4.0, 4.0, -4.0]   # ties to even codes
+    y = torch.randn(16, 128, generator=torch.Generator().manual_seed(4)) * 3
+    p, s = CI.quant_mxfp4_rows(y)
+    deq = O.decode_e2m1_packed(p) * np.repeat(O.decode_ue8m0(s), 32, axis=-1)
+    blk = y.numpy().reshape(16, 4, 32)
+    amax = np.abs(blk).max(axis=-1)
+    assert np.all(amax / O.decode_ue8m0(s) <= 6.0) and np.all(amax / O.decode_ue8m0(s) > 3.0)
+    assert np.abs(deq - y.numpy()).max() <= (O.decode_ue8m0(s).max() * 1.0)
+
+
+def test_workload_shapes_small():
+    w = CI.make_workload(1, scale={"B": 2, "T": 4096})
+    t, D = w.tensors, w.dims
+    assert t["cache"].shape == (2, 1024, 576) and t["cache"].dtype == np.uint16
+    assert t["kI"].shape == (2, 1024, 128) and t["kI_scale"].shape == (2, 1024)
+    assert D["entry0"] == 1023 and D["q_pos0"] == 4095
+    w4 = CI.make_workload(4, scale={"B": 1, "T": 8192})
+    assert w4.tensors["kI"].shape == (1, 2048, 64) and w4.tensors["kI_scale"].shape == (1, 2048, 4)
