@@ -1,0 +1,356 @@
+"""Throughput of the CSA / HCA hot path on B200.
+
+Default workload: CSA decode, batch 16 sequences at a 65,536-token context
+(16,384 compressed entries, m = 4), 128 query heads of width 576/512, FP8
+indexer with 64 heads of width 128, top-k 512, window 128, attention sink.  A
+step is one decode token for every sequence: csa_compress (the block the token
+completes) -> lightning_index (scores + exact top-k) -> sparse_attn_decode
+(+ split combine).  Inputs are synthetic (seeded) and resident in HBM; L2 is
+flushed before every timed step.
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded sample
+of the same workload.  Under torchrun each rank runs its own batch (independent
+sequences: weak scaling, no data-path collective); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOADS = {
+    "csa_decode_64k": 1,
+    "hca_decode_1m": 2,
+    "csa_prefill_4k": 3,
+    "hybrid_pair_1m": 4,
+}
+METRIC = "CSA/HCA decode tokens/s and HBM GB/s (% roofline) at 64K-1M ctx; prefill TFLOP/s"
+
+
+def algorithmic_bytes(wid, D):
+    """Bytes the method must move per step (each input / output byte once)."""
+    B = D["B"]
+    if wid in (1, 4):
+        N, d, k, W, H, dv, dI = D["N"], D["d"], D["k"], D["W"], D["H"], D["dv"], D["dI"]
+        kI_row = dI + 4 if D["ifmt"] == "e4m3" else dI // 2 + dI // 32
+        per = dict(
+            compress=(4 * 4 * d * 2 + 2 * 4 * d * 2 * 0) + 8 * 4 * d + d * 2,   # 4 series x 4 tokens + biases + entry
+            indexer=N * kI_row + 64 * (dI + 4) + 64 * 4,
+            attention=k * d * 2 + W * d * 2 + H * d * 2 + H * dv * 2,
+        )
+        tot = {kk: v * B for kk, v in per.items()}
+        if wid == 4:
+            Nh = D["Nh"]
+            tot["hca"] = B * (Nh * d * 2 + W * d * 2 + H * d * 2 + H * dv * 2 + 2 * 128 * d * 2)
+        return tot
+    if wid == 2:
+        N, d, W, H, dv = D["N"], D["d"], D["W"], D["H"], D["dv"]
+        return dict(compress=B * 2 * 128 * d * 2, attention=B * (N * d * 2 + W * d * 2 + H * d * 2 + H * dv * 2))
+    if wid == 3:
+        Tq, d, H, dv, N = D["Tq"], D["d"], D["H"], D["dv"], D["N"]
+        return dict(compress=4 * Tq * d * 2, indexer=N * 132 + Tq * 64 * 132,
+                    attention=Tq * H * d * 2 + Tq * H * dv * 2 + N * d * 2)
+    raise ValueError(wid)
+
+
+def sample_clocks(stop, out):
+    cmd = ["nvidia-smi", "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+           "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+           "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+           "--format=csv,noheader,nounits", "-lms", "100"]
+    try:
+        p = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+    except OSError:
+        return
+    dev = os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0]
+    try:
+        while not stop.is_set():
+            line = p.stdout.readline()
+            if not line:
+                break
+            out.append(line.strip())
+    finally:
+        p.terminate()
+        try:
+            p.wait(timeout=5)
+        except Exception:
+            p.kill()
+
+
+def summarize_clocks(lines, local_index=None):
+    sm, mx, reasons = [], None, set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for l in lines:
+        f = [x.strip() for x in l.split(",")]
+        if len(f) < 9:
+            continue
+        try:
+            sm.append(float(f[1])); mx = float(f[2])
+        except ValueError:
+            continue
+        for n, v in zip(names, f[5:9]):
+            if v.lower().startswith("active"):
+                reasons.add(n)
+    if not sm:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+    sm.sort()
+    return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons)}
+
+
+def run_reference(args, wid):
+    """Time the fp64 oracle on host cores on a bounded sample of the workload."""
+    import numpy as np
+    import csa_inputs as CI
+    from oracle import csa_oracle as O
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    scale = None
+    wl = CI.make_workload(wid, scale=scale)
+    D = wl.dims
+    cores = os.cpu_count()
+    sample_b = list(range(min(D["B"], 4)))
+    for _ in range(args.warmup and 1):
+        pass
+    t0 = time.perf_counter()
+    steps_done = 0
+    for _ in range(max(1, args.steps)):
+        if wid in (1, 4):
+            O.run_csa_decode(wl, batches=sample_b)
+            if wid == 4:
+                O.run_hca_decode(wl, batches=sample_b, prefix="h_")
+        elif wid == 2:
+            O.run_hca_decode(wl, batches=sample_b)
+        steps_done += 1
+    dt = time.perf_counter() - t0
+    tokens = steps_done * len(sample_b)
+    value = tokens / dt
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt / steps_done * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD_NAME, "batch_sampled": len(sample_b)},
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{len(sample_b)} of {D['B']} sequences per step, full context"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+WORKLOAD_NAME = "csa_decode_64k"
+
+
+def main():
+    global WORKLOAD_NAME
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="csa_decode_64k", choices=list(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    WORKLOAD_NAME = args.workload
+    wid = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wid)
+        return
+    run_ours(args, wid)
+
+
+def run_ours(args, wid):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    import compressed_sparse_long_csa_b200 as csa
+    from compressed_sparse_long_csa_b200 import steps
+    import csa_inputs as CI
+
+    wl = CI.make_workload(wid, seed=wid + 1000 * rank)
+    D = wl.dims
+    T = steps.upload(wl)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+
+    # per-call events to attribute time to kernels
+    def step_timed(evs):
+        if wid in (1, 4):
+            evs[0].record()
+            csa.csa_compress(T["Ca"], T["Cb"], T["Za"], T["Zb"], T["Ba"], T["Bb"], T["prev_Cb"], T["prev_Zb"],
+                             T["entry0"], T["cache"], m=D["m"])
+            evs[1].record()
+            csa.lightning_index(T["qI"], T.get("qI_scale"), T["w"], T["kI"], T.get("kI_scale"), T["n_entries"],
+                                T["q_pos"], D["k"], steps._ifmt(D), T["idx"], T["iws"], m=D["m"])
+            evs[2].record()
+            csa.sparse_attn_decode(T["q"][:, 0], T["cache"], T["idx"][:, 0], T["win"], T["win_len"], T["sink"],
+                                   D["sm_scale"], D["dv"], T["out"][:, 0], T["lse"][:, 0], T["aws"])
+            evs[3].record()
+            if wid == 4:
+                steps.hca_decode_step(T, D, prefix="h_")
+            evs[4].record()
+        else:
+            evs[0].record()
+            steps.run_step(wl.kind, T, D)
+            evs[1].record(); evs[2].record(); evs[3].record(); evs[4].record()
+
+    def mk():
+        return [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step_timed(mk())
+    torch.cuda.synchronize()
+    assert csa.read_device_error() == 0
+
+    clock_lines, stop = [], threading.Event()
+    th = threading.Thread(target=sample_clocks, args=(stop, clock_lines), daemon=True)
+    th.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev_list = []
+    for _ in range(args.steps):
+        flush.zero_()                        # L2 flush outside the timed events
+        evs = mk()
+        step_timed(evs)
+        ev_list.append(evs)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    stop.set()
+    th.join(timeout=10)
+    per = np.array([[ev[i].elapsed_time(ev[i + 1]) for i in range(4)] for ev in ev_list])   # ms
+    step_ms = per.sum(axis=1)
+    total_ms = float(step_ms.sum())
+    if world > 1:
+        t = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    tokens_per_step = D["B"] * (D["Tq"] if wid == 3 else 1)
+    value = tokens_per_step * world / (ms_per_step * 1e-3)
+
+    # ---- e2e through the public API with host buffers
+    e2e = measure_e2e(args, wid, wl, T, D, csa, steps)
+    ab = algorithmic_bytes(wid, D)
+    comp = ["compress", "indexer", "attention", "hca"]
+    mean_ms = per.mean(axis=0)
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except Exception:
+        pass
+    hbm_peak = peaks.get("hbm_gbs", 6650.0)
+    # dominant kernel: the indexer for CSA decode, the attention otherwise
+    dom = "indexer" if wid in (1, 4) else "attention"
+    dom_ms = mean_ms[comp.index(dom)]
+    achieved = ab[dom] / (dom_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "batch": D["B"], "context": D["T"], "entries": D["N"],
+                   "top_k": D.get("k"), "window": D["W"], "heads": D["H"], "l2": "flushed before every step"},
+        "hbm_gbs_step": sum(ab.values()) / (ms_per_step * 1e-3) / 1e9,
+        "breakdown_ms": {c: float(m) for c, m in zip(comp, mean_ms)},
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "peak_source": "measured" if peaks else "fallback",
+                     "traffic": None},
+        "e2e": e2e,
+        "gpu_launches": launches_per_step(wid, D) * args.steps,
+        "clocks": summarize_clocks(clock_lines),
+    }
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(wid, wl)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def launches_per_step(wid, D):
+    if wid == 1:
+        return 5       # compress, indexer scores, indexer select, attention, combine
+    if wid == 2:
+        return 3
+    if wid == 3:
+        return 4
+    return 8
+
+
+def measure_e2e(args, wid, wl, T, D, csa, steps):
+    """Same step through the public API, inputs copied from pinned host memory and
+    the result read back, all inside the timed region."""
+    import torch
+    per_step_in = {1: ["Ca", "Cb", "Za", "Zb", "q", "qI", "qI_scale", "w", "win"],
+                   2: ["C", "Z", "q", "win"], 3: ["Ca", "Cb", "Za", "Zb", "q", "qI", "qI_scale", "w"],
+                   4: ["Ca", "Cb", "Za", "Zb", "q", "qI", "qI_scale", "w", "win", "h_C", "h_Z", "h_q", "h_win"]}[wid]
+    host = {k: T[k].cpu().pin_memory() for k in per_step_in}
+    outs = ["out", "idx"] if wid != 2 else ["out"]
+    if wid == 4:
+        outs.append("h_out")
+    hout = {k: torch.empty_like(T[k], device="cpu").pin_memory() for k in outs}
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = sum(v.numel() * v.element_size() for v in hout.values())
+    n = max(5, min(args.steps, 20))
+    for _ in range(2):
+        for k, v in host.items():
+            T[k].copy_(v, non_blocking=True)
+        steps.run_step(wl.kind, T, D)
+        for k, v in hout.items():
+            v.copy_(T[k], non_blocking=True)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n):
+        for k, v in host.items():
+            T[k].copy_(v, non_blocking=True)
+        steps.run_step(wl.kind, T, D)
+        for k, v in hout.items():
+            v.copy_(T[k], non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    tokens = D["B"] * (D["Tq"] if wid == 3 else 1)
+    return {"value": tokens / (ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def cpu_baseline(wid, wl):
+    """The oracle as it stands on the host cores, on a bounded sample."""
+    from oracle import csa_oracle as O
+    D = wl.dims
+    sample = list(range(min(D["B"], 2)))
+    t0 = time.perf_counter()
+    if wid in (1, 4):
+        O.run_csa_decode(wl, batches=sample)
+        if wid == 4:
+            O.run_hca_decode(wl, batches=sample, prefix="h_")
+    elif wid == 2:
+        O.run_hca_decode(wl, batches=sample)
+    else:
+        O.run_csa_prefill(wl, rows=list(range(8)))
+    dt = time.perf_counter() - t0
+    toks = len(sample) if wid != 3 else 8
+    return {"value": toks / dt, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{toks} {'query rows' if wid == 3 else 'sequences'} of the workload, one step"}
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,144 @@
+"""ctypes binding of libcsa_b200.so (argument marshalling only)."""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_HERE, "libcsa_b200.so")
+if not os.path.exists(lib_path):
+    raise ImportError(f"{lib_path} is missing: build it with `python -m compressed_sparse_long_csa_b200.build`")
+lib = C.CDLL(lib_path)
+
+CSA_F32, CSA_BF16 = 0, 1
+CSA_IFMT_F32, CSA_IFMT_E4M3, CSA_IFMT_MXFP4 = 0, 1, 2
+
+_vp, _i32, _i64, _f32, _sz = C.c_void_p, C.c_int, C.c_int64, C.c_float, C.c_size_t
+
+_SIGS = {
+    "csa_abi_version": ([], _i32),
+    "csa_status_string": ([_i32], C.c_char_p),
+    "csa_read_device_error": ([_vp, C.POINTER(C.c_uint32)], _i32),
+    "csa_compress": ([_vp] * 10 + [_i64, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
+    "hca_compress": ([_vp] * 5 + [_i64, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
+    "lightning_index_workspace_size": ([_i32, _i32, _i64, _i32], _sz),
+    "lightning_index": ([_vp] * 7 + [_i32, _i32, _i32, _i32, _i32, _i64, _i32, _i32, _vp, _vp, _vp, _sz, _vp], _i32),
+    "topk_select_workspace_size": ([_i32, _i64, _i32], _sz),
+    "topk_select": ([_vp, _i64, _vp, _i32, _i64, _i32, _vp, _vp, _sz, _vp], _i32),
+    "attn_decode_workspace_size": ([_i32, _i32, _i32, _i64], _sz),
+    "sparse_attn_decode": ([_vp] * 6 + [_i32, _i32, _i32, _i32, _i64, _i32, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp], _i32),
+    "hca_attn_decode": ([_vp] * 6 + [_i32, _i32, _i32, _i32, _i64, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp], _i32),
+    "sparse_attn_prefill": ([_vp] * 5 + [_i64, _vp, _vp] + [_i32] * 5 + [_i64, _i32, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp], _i32),
+}
+for _name, (_args, _res) in _SIGS.items():
+    _f = getattr(lib, _name)
+    _f.argtypes = _args
+    _f.restype = _res
+
+
+class CsaError(RuntimeError):
+    pass
+
+
+def _check(status: int, name: str):
+    if status != 0:
+        raise CsaError(f"{name}: {lib.csa_status_string(status).decode()}")
+
+
+def _p(t):
+    """Device pointer of a tensor (None -> NULL)."""
+    if t is None:
+        return None
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dtype_code(t):
+    return CSA_BF16 if t.dtype == torch.bfloat16 else CSA_F32
+
+
+def read_device_error(stream=None) -> int:
+    v = C.c_uint32(0)
+    _check(lib.csa_read_device_error(_stream(stream), C.byref(v)), "csa_read_device_error")
+    return int(v.value)
+
+
+def csa_compress(Ca, Cb, Za, Zb, Ba, Bb, prev_Cb, prev_Zb, entry0, cache, m=4, stream=None):
+    B, T_new, d = Ca.shape
+    _check(lib.csa_compress(_p(Ca), _p(Cb), _p(Za), _p(Zb), _p(Ba), _p(Bb), _p(prev_Cb), _p(prev_Zb),
+                            _p(entry0), _p(cache), cache.shape[1], B, T_new, d, m, _dtype_code(Ca),
+                            _stream(stream)), "csa_compress")
+
+
+def hca_compress(C_, Z, bias, entry0, cache, m_prime=128, stream=None):
+    B, T_new, d = C_.shape
+    _check(lib.hca_compress(_p(C_), _p(Z), _p(bias), _p(entry0), _p(cache), cache.shape[1], B, T_new, d,
+                            m_prime, _dtype_code(C_), _stream(stream)), "hca_compress")
+
+
+def lightning_index_workspace_size(B, Tq, n_max, k):
+    return int(lib.lightning_index_workspace_size(B, Tq, n_max, k))
+
+
+def lightning_index(qI, qI_scale, w, kI, kI_scale, n_entries, q_pos, k, ifmt, idx_out, workspace,
+                    score_out=None, m=4, stream=None):
+    B, Tq, H_I = w.shape
+    n_max = kI.shape[1]
+    d_I = qI.shape[-1] * (2 if ifmt == CSA_IFMT_MXFP4 else 1)
+    _check(lib.lightning_index(_p(qI), _p(qI_scale), _p(w), _p(kI), _p(kI_scale), _p(n_entries), _p(q_pos), m,
+                               B, Tq, H_I, d_I, n_max, k, ifmt, _p(idx_out), _p(score_out), _p(workspace),
+                               workspace.numel() * workspace.element_size(), _stream(stream)), "lightning_index")
+
+
+def topk_select(scores, n_valid, k, idx_out, stream=None):
+    R, n = scores.shape
+    _check(lib.topk_select(_p(scores), scores.stride(0), _p(n_valid), R, n, k, _p(idx_out), None, 0,
+                           _stream(stream)), "topk_select")
+
+
+def attn_decode_workspace_size(B, H, d_v, rows_max):
+    return int(lib.attn_decode_workspace_size(B, H, d_v, rows_max))
+
+
+def _ws(workspace):
+    if workspace is None:
+        return None, 0
+    return workspace.data_ptr(), workspace.numel() * workspace.element_size()
+
+
+def sparse_attn_decode(q, cache, idx, win, win_len, sink, sm_scale, d_v, out, lse=None, workspace=None,
+                       stream=None):
+    B, H, d_k = q.shape
+    W = win.shape[1] if win is not None else 0
+    k = idx.shape[1] if idx is not None else 0
+    wp, wb = _ws(workspace)
+    _check(lib.sparse_attn_decode(_p(q), _p(cache), _p(idx), _p(win), _p(win_len), _p(sink), B, H, d_k, d_v,
+                                  cache.shape[1], k, W, sm_scale, _dtype_code(q), _p(out), _p(lse), wp, wb,
+                                  _stream(stream)), "sparse_attn_decode")
+
+
+def hca_attn_decode(q, cache, n_entries, win, win_len, sink, sm_scale, d_v, out, lse=None, workspace=None,
+                    stream=None):
+    B, H, d_k = q.shape
+    W = win.shape[1] if win is not None else 0
+    wp, wb = _ws(workspace)
+    _check(lib.hca_attn_decode(_p(q), _p(cache), _p(n_entries), _p(win), _p(win_len), _p(sink), B, H, d_k, d_v,
+                               cache.shape[1], W, sm_scale, _dtype_code(q), _p(out), _p(lse), wp, wb,
+                               _stream(stream)), "hca_attn_decode")
+
+
+def sparse_attn_prefill(q, q_pos, cache, idx, raw, raw_pos0, W, sink, sm_scale, d_v, out, lse=None,
+                        workspace=None, stream=None):
+    B, Tq, H, d_k = q.shape
+    k = idx.shape[2] if idx is not None else 0
+    wp, wb = _ws(workspace)
+    _check(lib.sparse_attn_prefill(_p(q), _p(q_pos), _p(cache), _p(idx), _p(raw), raw.shape[1], _p(raw_pos0),
+                                   _p(sink), B, Tq, H, d_k, d_v, cache.shape[1], k, W, sm_scale, _dtype_code(q),
+                                   _p(out), _p(lse), wp, wb, _stream(stream)), "sparse_attn_prefill")

@@ -1,0 +1,311 @@
+// extern "C" entry points of libcsa_b200: host-side validation, workspace layout
+// and dispatch to the kernels.  Nothing here allocates device memory or
+// synchronises (except csa_read_device_error, which is documented to).
+#include <math.h>
+#include <mutex>
+
+#include "attention.cuh"
+#include "indexer.cuh"
+
+namespace csa {
+cudaError_t launch_csa_compress(const void*, const void*, const void*, const void*, const float*, const float*,
+                                const void*, const void*, const int32_t*, void*, int64_t, int, int, int, int,
+                                int, cudaStream_t, unsigned*);
+cudaError_t launch_hca_compress(const void*, const void*, const float*, const int32_t*, void*, int64_t, int,
+                                int, int, int, int, cudaStream_t, unsigned*);
+}  // namespace csa
+
+using namespace csa;
+
+// Per-device error word (see CSA_DEVERR_* in csa.h).
+__device__ unsigned int g_csa_device_error = 0u;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+unsigned* g_err_ptr[kMaxDevices] = {nullptr};
+std::mutex g_err_mu;
+
+unsigned* device_error_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_err_mu);
+  if (!g_err_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_csa_device_error) != cudaSuccess) return nullptr;
+    g_err_ptr[dev] = (unsigned*)p;
+  }
+  return g_err_ptr[dev];
+}
+
+inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline cudaStream_t S(void* s) { return (cudaStream_t)s; }
+inline csa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? CSA_OK : CSA_ERR_CUDA; }
+inline int elem_size(int dtype) { return dtype == CSA_BF16 ? 2 : 4; }
+
+#define REQUIRE(cond, code) do { if (!(cond)) return (code); } while (0)
+#define REQUIRE_PTR(p) do { if (!(p)) return CSA_ERR_NULL; if (!aligned16(p)) return CSA_ERR_ALIGN; } while (0)
+
+// tensor-core paths may be disabled (for A/B testing) through this environment variable
+bool tc_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("CSA_B200_DISABLE_TC");
+    v = (e && e[0] == '1') ? 0 : 1;
+  }
+  return v == 1;
+}
+
+}  // namespace
+
+extern "C" {
+
+int csa_abi_version(void) { return CSA_ABI_VERSION; }
+
+const char* csa_status_string(int s) {
+  switch (s) {
+    case CSA_OK: return "CSA_OK";
+    case CSA_ERR_NULL: return "CSA_ERR_NULL: a required pointer is NULL";
+    case CSA_ERR_SHAPE: return "CSA_ERR_SHAPE: a size is out of range or sizes are inconsistent";
+    case CSA_ERR_DTYPE: return "CSA_ERR_DTYPE: unsupported storage or operand format";
+    case CSA_ERR_ALIGN: return "CSA_ERR_ALIGN: a device pointer is not 16-byte aligned";
+    case CSA_ERR_UNSUPPORTED: return "CSA_ERR_UNSUPPORTED: no kernel for this combination of sizes";
+    case CSA_ERR_WORKSPACE: return "CSA_ERR_WORKSPACE: workspace missing or too small";
+    case CSA_ERR_CUDA: return "CSA_ERR_CUDA: a CUDA runtime call or launch failed";
+    default: return "unknown csa_status";
+  }
+}
+
+csa_status csa_read_device_error(void* stream, uint32_t* out) {
+  REQUIRE(out, CSA_ERR_NULL);
+  unsigned* w = device_error_word();
+  REQUIRE(w, CSA_ERR_CUDA);
+  unsigned h = 0;
+  cudaError_t e = cudaMemcpyAsync(&h, w, sizeof(unsigned), cudaMemcpyDeviceToHost, S(stream));
+  if (e == cudaSuccess) e = cudaMemsetAsync(w, 0, sizeof(unsigned), S(stream));
+  if (e == cudaSuccess) e = cudaStreamSynchronize(S(stream));
+  if (e != cudaSuccess) return CSA_ERR_CUDA;
+  *out = h;
+  return CSA_OK;
+}
+
+// ----------------------------------------------------------------------------- compressors
+csa_status csa_compress(const void* Ca, const void* Cb, const void* Za, const void* Zb, const float* Ba,
+                        const float* Bb, const void* prev_Cb, const void* prev_Zb, const int32_t* entry0,
+                        void* cache, int64_t n_max, int B, int T_new, int d, int m, int dtype, void* stream) {
+  REQUIRE(dtype == CSA_F32 || dtype == CSA_BF16, CSA_ERR_DTYPE);
+  REQUIRE(B >= 1 && B <= 65535 && T_new >= 1 && d >= 1 && m >= 1 && m <= 16 && n_max >= 1, CSA_ERR_SHAPE);
+  REQUIRE(T_new % m == 0, CSA_ERR_SHAPE);
+  REQUIRE(d % (dtype == CSA_BF16 ? 8 : 4) == 0, CSA_ERR_SHAPE);
+  REQUIRE_PTR(Ca); REQUIRE_PTR(Cb); REQUIRE_PTR(Za); REQUIRE_PTR(Zb); REQUIRE_PTR(Ba); REQUIRE_PTR(Bb);
+  REQUIRE_PTR(prev_Cb); REQUIRE_PTR(prev_Zb); REQUIRE_PTR(cache);
+  REQUIRE(entry0, CSA_ERR_NULL);
+  unsigned* err = device_error_word();
+  REQUIRE(err, CSA_ERR_CUDA);
+  return cuda_status(launch_csa_compress(Ca, Cb, Za, Zb, Ba, Bb, prev_Cb, prev_Zb, entry0, cache, n_max, B,
+                                         T_new, d, m, dtype, S(stream), err));
+}
+
+csa_status hca_compress(const void* C, const void* Z, const float* bias, const int32_t* entry0, void* cache,
+                        int64_t n_max, int B, int T_new, int d, int m_prime, int dtype, void* stream) {
+  REQUIRE(dtype == CSA_F32 || dtype == CSA_BF16, CSA_ERR_DTYPE);
+  REQUIRE(B >= 1 && B <= 65535 && T_new >= 1 && d >= 1 && m_prime >= 1 && m_prime <= 1024 && n_max >= 1,
+          CSA_ERR_SHAPE);
+  REQUIRE(T_new % m_prime == 0 && T_new / m_prime <= 2147483647, CSA_ERR_SHAPE);
+  REQUIRE(d % (dtype == CSA_BF16 ? 8 : 4) == 0, CSA_ERR_SHAPE);
+  REQUIRE_PTR(C); REQUIRE_PTR(Z); REQUIRE_PTR(bias); REQUIRE_PTR(cache);
+  REQUIRE(entry0, CSA_ERR_NULL);
+  unsigned* err = device_error_word();
+  REQUIRE(err, CSA_ERR_CUDA);
+  return cuda_status(launch_hca_compress(C, Z, bias, entry0, cache, n_max, B, T_new, d, m_prime, dtype,
+                                         S(stream), err));
+}
+
+// ----------------------------------------------------------------------------- indexer / top-k
+static int64_t idx_ld(int64_t n_max) { return (int64_t)round_up((size_t)n_max, 64); }
+
+size_t lightning_index_workspace_size(int B, int Tq, int64_t n_max, int k) {
+  (void)k;
+  if (B < 1 || Tq < 1 || n_max < 1) return 0;
+  return round_up((size_t)B * Tq * idx_ld(n_max) * sizeof(float), 256) + round_up((size_t)B * sizeof(unsigned), 256);
+}
+
+csa_status lightning_index(const void* qI, const void* qI_scale, const float* w, const void* kI,
+                           const void* kI_scale, const int32_t* n_entries, const int32_t* q_pos, int m, int B,
+                           int Tq, int H_I, int d_I, int64_t n_max, int k, int ifmt, int32_t* idx_out,
+                           float* score_out, void* workspace, size_t ws_bytes, void* stream) {
+  REQUIRE(ifmt == CSA_IFMT_F32 || ifmt == CSA_IFMT_E4M3 || ifmt == CSA_IFMT_MXFP4, CSA_ERR_DTYPE);
+  REQUIRE(B >= 1 && Tq >= 1 && (int64_t)B * Tq <= 65535 && H_I >= 1 && H_I <= 64 && m >= 1, CSA_ERR_SHAPE);
+  REQUIRE(d_I == 32 || d_I == 64 || d_I == 128, CSA_ERR_SHAPE);
+  REQUIRE(k >= 1 && k <= 2048 && n_max >= 1 && n_max <= (1 << 24), CSA_ERR_SHAPE);
+  REQUIRE_PTR(qI); REQUIRE_PTR(w); REQUIRE_PTR(kI); REQUIRE_PTR(idx_out);
+  if (ifmt != CSA_IFMT_F32) { REQUIRE_PTR(qI_scale); REQUIRE_PTR(kI_scale); }
+  if (score_out) REQUIRE(aligned16(score_out), CSA_ERR_ALIGN);
+  REQUIRE(n_entries && q_pos, CSA_ERR_NULL);
+  const size_t need = lightning_index_workspace_size(B, Tq, n_max, k);
+  REQUIRE(workspace && ws_bytes >= need, CSA_ERR_WORKSPACE);
+  REQUIRE(aligned16(workspace), CSA_ERR_ALIGN);
+  unsigned* err = device_error_word();
+  REQUIRE(err, CSA_ERR_CUDA);
+
+  IndexerArgs a{};
+  a.qI = qI; a.qI_scale = qI_scale; a.w = w; a.kI = kI; a.kI_scale = kI_scale;
+  a.n_entries = n_entries; a.q_pos = q_pos; a.m = m;
+  a.B = B; a.Tq = Tq; a.H_I = H_I; a.d_I = d_I; a.n_max = n_max; a.k = k; a.ifmt = ifmt;
+  a.ld = idx_ld(n_max);
+  a.scores = (float*)workspace;
+  a.knmax = (unsigned*)((char*)workspace + round_up((size_t)B * Tq * a.ld * sizeof(float), 256));
+  a.idx_out = idx_out; a.score_out = score_out; a.err = err;
+  cudaError_t e = cudaMemsetAsync(a.knmax, 0, (size_t)B * sizeof(unsigned), S(stream));
+  if (e != cudaSuccess) return CSA_ERR_CUDA;
+  bool used_tc = false;
+  if (tc_enabled()) {
+    e = launch_indexer_scores_tc(a, S(stream), &used_tc);
+    if (e != cudaSuccess) return CSA_ERR_CUDA;
+  }
+  if (!used_tc) {
+    // sequential fp32 FMA accumulation of d_I exact products: |err| <= (d_I+2) u sum|q c k c|
+    a.eps_dot = (float)(d_I + 4) * 5.9604645e-08f * 1.25f;
+    e = launch_indexer_scores_cuda_core(a, S(stream));
+    if (e != cudaSuccess) return CSA_ERR_CUDA;
+  }
+  return cuda_status(launch_indexer_select(a, S(stream)));
+}
+
+size_t topk_select_workspace_size(int R, int64_t n, int k) {
+  (void)R; (void)n; (void)k;
+  return 0;
+}
+
+csa_status topk_select(const float* scores, int64_t ld, const int32_t* n_valid, int R, int64_t n, int k,
+                       int32_t* idx_out, void* workspace, size_t ws_bytes, void* stream) {
+  (void)workspace; (void)ws_bytes;
+  REQUIRE(R >= 1 && n >= 1 && n <= (1 << 24) && ld >= n && k >= 1 && k <= 2048, CSA_ERR_SHAPE);
+  REQUIRE_PTR(scores); REQUIRE_PTR(idx_out);
+  unsigned* err = device_error_word();
+  REQUIRE(err, CSA_ERR_CUDA);
+  return cuda_status(launch_topk_select(scores, ld, n_valid, R, n, k, idx_out, S(stream), err));
+}
+
+// ----------------------------------------------------------------------------- attention
+static bool attn_tc_shape(int dtype, int H, int dk, int dv) {
+  return dtype == CSA_BF16 && H == 128 && dk == 576 && dv == 512;
+}
+
+static int decode_splits(int B, int H, int64_t rows_max) {
+  const int s1 = attn_choose_splits(B, H, rows_max, false);
+  const int s2 = attn_choose_splits(B, H, rows_max, true);
+  return s1 > s2 ? s1 : s2;
+}
+
+size_t attn_decode_workspace_size(int B, int H, int d_v, int64_t rows_max) {
+  if (B < 1 || H < 1 || d_v < 1 || rows_max < 1) return 0;
+  const int s = decode_splits(B, H, rows_max);
+  return round_up((size_t)B * s * H * (d_v + 2) * sizeof(float), 256);
+}
+
+static csa_status attn_common_checks(const void* q, const void* cache, const void* win, const float* sink, int B,
+                                     int H, int d_k, int d_v, int64_t n_max, int W, int dtype, void* out,
+                                     float* lse) {
+  REQUIRE(dtype == CSA_F32 || dtype == CSA_BF16, CSA_ERR_DTYPE);
+  REQUIRE(B >= 1 && H >= 1 && H <= 128 && d_k >= 1 && d_k <= 576 && d_v >= 1 && d_v <= d_k, CSA_ERR_SHAPE);
+  REQUIRE(d_k % 8 == 0 && d_v % 4 == 0 && n_max >= 1 && W >= 0 && W <= 4096, CSA_ERR_SHAPE);
+  REQUIRE_PTR(q); REQUIRE_PTR(cache); REQUIRE_PTR(sink); REQUIRE_PTR(out);
+  if (W > 0) REQUIRE_PTR(win);
+  if (lse) REQUIRE(aligned16(lse), CSA_ERR_ALIGN);
+  return CSA_OK;
+}
+
+static csa_status run_attention(AttnArgs& a, int dtype, void* workspace, size_t ws_bytes, bool decode,
+                                cudaStream_t st) {
+  const int64_t rows = attn_virtual_rows(a);
+  const bool tc = tc_enabled() && attn_tc_shape(dtype, a.H, a.dk, a.dv);
+  if (decode) {
+    a.splits = attn_choose_splits(a.B * a.Tq, a.H, rows, tc);
+  } else {
+    a.splits = 1;
+  }
+  a.rows_per_split = (int)((rows + a.splits - 1) / a.splits);
+  a.part = (float*)workspace;
+  bool used = false;
+  cudaError_t e = cudaSuccess;
+  if (tc) e = launch_attention_tc(a, st, &used);
+  if (e != cudaSuccess) return CSA_ERR_CUDA;
+  if (!used) {
+    if (tc) {  // the tensor-core path declined: recompute the split plan for the CUDA-core path
+      a.splits = decode ? attn_choose_splits(a.B * a.Tq, a.H, rows, false) : 1;
+      a.rows_per_split = (int)((rows + a.splits - 1) / a.splits);
+    }
+    e = launch_attention_cuda_core(a, dtype, st);
+    if (e != cudaSuccess) return CSA_ERR_CUDA;
+  }
+  if (a.splits > 1) return cuda_status(launch_attn_combine(a, dtype, st));
+  return CSA_OK;
+}
+
+csa_status sparse_attn_decode(const void* q, const void* cache, const int32_t* idx, const void* win,
+                              const int32_t* win_len, const float* sink, int B, int H, int d_k, int d_v,
+                              int64_t n_max, int k, int W, float sm_scale, int dtype, void* out, float* lse,
+                              void* workspace, size_t ws_bytes, void* stream) {
+  csa_status s = attn_common_checks(q, cache, win, sink, B, H, d_k, d_v, n_max, W, dtype, out, lse);
+  if (s != CSA_OK) return s;
+  REQUIRE(k >= 0 && k <= 65536 && B <= 65535, CSA_ERR_SHAPE);
+  REQUIRE(k == 0 || idx, CSA_ERR_NULL);
+  REQUIRE(W == 0 || win_len, CSA_ERR_NULL);
+  REQUIRE(isfinite(sm_scale), CSA_ERR_SHAPE);
+  REQUIRE(workspace && ws_bytes >= attn_decode_workspace_size(B, H, d_v, (int64_t)k + W), CSA_ERR_WORKSPACE);
+  REQUIRE(aligned16(workspace), CSA_ERR_ALIGN);
+  unsigned* err = device_error_word();
+  REQUIRE(err, CSA_ERR_CUDA);
+  AttnArgs a{};
+  a.q = q; a.cache = cache; a.idx = idx; a.k = k; a.n_seg_a = k; a.win = win; a.win_len = win_len;
+  a.W = W; a.prefill = 0; a.sink = sink; a.B = B; a.Tq = 1; a.H = H; a.dk = d_k; a.dv = d_v; a.n_max = n_max;
+  a.sm_scale = sm_scale; a.out = out; a.lse = lse; a.err = err;
+  return run_attention(a, dtype, workspace, ws_bytes, true, S(stream));
+}
+
+csa_status hca_attn_decode(const void* q, const void* cache, const int32_t* n_entries, const void* win,
+                           const int32_t* win_len, const float* sink, int B, int H, int d_k, int d_v,
+                           int64_t n_max, int W, float sm_scale, int dtype, void* out, float* lse,
+                           void* workspace, size_t ws_bytes, void* stream) {
+  csa_status s = attn_common_checks(q, cache, win, sink, B, H, d_k, d_v, n_max, W, dtype, out, lse);
+  if (s != CSA_OK) return s;
+  REQUIRE(n_max <= (1 << 24) && B <= 65535, CSA_ERR_SHAPE);
+  REQUIRE(n_entries, CSA_ERR_NULL);
+  REQUIRE(W == 0 || win_len, CSA_ERR_NULL);
+  REQUIRE(isfinite(sm_scale), CSA_ERR_SHAPE);
+  REQUIRE(workspace && ws_bytes >= attn_decode_workspace_size(B, H, d_v, n_max + W), CSA_ERR_WORKSPACE);
+  REQUIRE(aligned16(workspace), CSA_ERR_ALIGN);
+  unsigned* err = device_error_word();
+  REQUIRE(err, CSA_ERR_CUDA);
+  AttnArgs a{};
+  a.q = q; a.cache = cache; a.idx = nullptr; a.n_entries = n_entries; a.n_seg_a = (int)n_max;
+  a.win = win; a.win_len = win_len; a.W = W; a.prefill = 0; a.sink = sink; a.B = B; a.Tq = 1; a.H = H;
+  a.dk = d_k; a.dv = d_v; a.n_max = n_max; a.sm_scale = sm_scale; a.out = out; a.lse = lse; a.err = err;
+  return run_attention(a, dtype, workspace, ws_bytes, true, S(stream));
+}
+
+csa_status sparse_attn_prefill(const void* q, const int32_t* q_pos, const void* cache, const int32_t* idx,
+                               const void* raw, int64_t t_raw, const int32_t* raw_pos0, const float* sink, int B,
+                               int Tq, int H, int d_k, int d_v, int64_t n_max, int k, int W, float sm_scale,
+                               int dtype, void* out, float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  csa_status s = attn_common_checks(q, cache, raw, sink, B, H, d_k, d_v, n_max, W, dtype, out, lse);
+  if (s != CSA_OK) return s;
+  REQUIRE(Tq >= 1 && (int64_t)B * Tq <= 65535 && k >= 0 && k <= 65536, CSA_ERR_SHAPE);
+  REQUIRE(k == 0 || idx, CSA_ERR_NULL);
+  REQUIRE(q_pos, CSA_ERR_NULL);
+  REQUIRE(W == 0 || (raw_pos0 && t_raw >= 1), CSA_ERR_NULL);
+  REQUIRE(isfinite(sm_scale), CSA_ERR_SHAPE);
+  REQUIRE(workspace && ws_bytes >= attn_decode_workspace_size(B, H, d_v, (int64_t)k + W), CSA_ERR_WORKSPACE);
+  REQUIRE(aligned16(workspace), CSA_ERR_ALIGN);
+  unsigned* err = device_error_word();
+  REQUIRE(err, CSA_ERR_CUDA);
+  AttnArgs a{};
+  a.q = q; a.cache = cache; a.idx = idx; a.k = k; a.n_seg_a = k; a.win = raw; a.q_pos = q_pos;
+  a.raw_pos0 = raw_pos0; a.t_raw = t_raw; a.W = W; a.prefill = 1; a.sink = sink; a.B = B; a.Tq = Tq; a.H = H;
+  a.dk = d_k; a.dv = d_v; a.n_max = n_max; a.sm_scale = sm_scale; a.out = out; a.lse = lse; a.err = err;
+  return run_attention(a, dtype, workspace, ws_bytes, false, S(stream));
+}
+
+}  // extern "C"

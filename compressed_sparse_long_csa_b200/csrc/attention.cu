@@ -1,0 +1,187 @@
+// Attention over selected / all compressed entries + raw sliding window + sink,
+// CUDA-core path, and the split-KV combine.
+//
+// "Техотчёт DeepSeek-V4 (2026): миллион токенов контекста", section "Гибридное
+// внимание: CSA и HCA": CSA step 3 (MQA: every compressed entry is key and value
+// for all query heads), the HCA paragraph (dense attention over the compressed
+// entries) and the 128-token window of uncompressed entries; "Технический отчёт
+// DeepSeek-V4 — часть 1/2": MLA latent (keys use all 576 dims, values the first
+// 512), sliding-window branch and attention sink.
+//
+// The CUDA-core path runs fp32 math for any head count / width (it is the only
+// path for fp32 storage); the tcgen05 path (attention_tc.cu) covers bf16 with
+// 128 heads of width 576/512.  Both write the same split partials
+// (m, l, unnormalised o) which attn_combine merges with the sink.
+#include "attention.cuh"
+
+namespace csa {
+
+constexpr int CC_ROWS = 32;    // rows per shared-memory tile
+constexpr int CC_HG = 8;       // heads per CTA (one warp each)
+constexpr int CC_MAXD = 576;
+
+// grid (splits, ceil(H/8), B*Tq), 256 threads.  dynamic smem: [32][dk] floats.
+template <typename T>
+__global__ void __launch_bounds__(256)
+attn_cuda_core_kernel(AttnArgs a) {
+  extern __shared__ float Ks[];               // [CC_ROWS][dk]
+  __shared__ const T* rowp[CC_ROWS];
+  const int split = blockIdx.x, hg = blockIdx.y, row = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = hg * CC_HG + warp;
+  const int dk = a.dk, dv = a.dv;
+  const bool hv = h < a.H;
+  const int nq = (dk + 31) / 32, nv = (dv + 31) / 32;
+
+  float qr[CC_MAXD / 32];
+  float o[CC_MAXD / 32];
+#pragma unroll
+  for (int i = 0; i < CC_MAXD / 32; ++i) {
+    const int c = lane + 32 * i;
+    qr[i] = (hv && i < nq && c < dk) ? Elem<T>::ld((const T*)a.q + ((size_t)row * a.H + h) * dk + c) : 0.f;
+    o[i] = 0.f;
+  }
+  float m_run = -INFINITY, l_run = 0.f;
+  const int64_t nrows = attn_virtual_rows(a);
+  const int64_t v0 = (int64_t)split * a.rows_per_split;
+  const int64_t v1 = min(nrows, v0 + a.rows_per_split);
+  const float scale = a.sm_scale;
+
+  for (int64_t t0 = v0; t0 < v1; t0 += CC_ROWS) {
+    __syncthreads();
+    if (threadIdx.x < CC_ROWS) {
+      const int64_t v = t0 + threadIdx.x;
+      rowp[threadIdx.x] = (v < v1) ? attn_row_ptr<T>(a, row, (int)v) : nullptr;
+    }
+    __syncthreads();
+    const int vecs = dk / Elem<T>::VEC;
+    for (int i = threadIdx.x; i < CC_ROWS * vecs; i += blockDim.x) {
+      const int r = i / vecs, c = (i % vecs) * Elem<T>::VEC;
+      float tmp[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      if (rowp[r]) Elem<T>::ld_vec(rowp[r] + c, tmp);
+#pragma unroll
+      for (int u = 0; u < Elem<T>::VEC; ++u) Ks[r * dk + c + u] = tmp[u];
+    }
+    __syncthreads();
+    if (!hv) continue;
+    float logit = -INFINITY;
+    for (int r = 0; r < CC_ROWS; ++r) {
+      float part = 0.f;
+#pragma unroll
+      for (int i = 0; i < CC_MAXD / 32; ++i) {
+        const int c = lane + 32 * i;
+        if (i < nq && c < dk) part = fmaf(qr[i], Ks[r * dk + c], part);
+      }
+      part = warp_sum(part) * scale;
+      if (lane == r) logit = rowp[r] ? part : -INFINITY;
+    }
+    const float mx = warp_max(logit);
+    const float m_new = fmaxf(m_run, mx);
+    if (m_new == -INFINITY) continue;
+    const float alpha = __expf(m_run - m_new);
+    const float p = __expf(logit - m_new);
+    l_run = l_run * alpha + warp_sum(p);
+#pragma unroll
+    for (int i = 0; i < CC_MAXD / 32; ++i) o[i] *= alpha;
+    for (int r = 0; r < CC_ROWS; ++r) {
+      const float pr = __shfl_sync(0xffffffffu, p, r);
+      if (pr == 0.f) continue;
+#pragma unroll
+      for (int i = 0; i < CC_MAXD / 32; ++i) {
+        const int c = lane + 32 * i;
+        if (i < nv && c < dv) o[i] = fmaf(pr, Ks[r * dk + c], o[i]);
+      }
+    }
+    m_run = m_new;
+  }
+  if (!hv) return;
+  if (a.splits == 1) {
+    const float sk = a.sink[h];
+    const float M = fmaxf(sk, m_run);
+    float den = 0.f, f = 0.f;
+    if (M != -INFINITY) {
+      f = (m_run == -INFINITY) ? 0.f : __expf(m_run - M);
+      den = __expf(sk - M) + l_run * f;
+    }
+    const float inv = den > 0.f ? f / den : 0.f;
+#pragma unroll
+    for (int i = 0; i < CC_MAXD / 32; ++i) {
+      const int c = lane + 32 * i;
+      if (i < nv && c < dv) Elem<T>::st((T*)a.out + ((size_t)row * a.H + h) * dv + c, o[i] * inv);
+    }
+    if (a.lse && lane == 0) a.lse[(size_t)row * a.H + h] = den > 0.f ? M + logf(den) : -INFINITY;
+  } else {
+    float* P = a.part + (((size_t)row * a.splits + split) * a.H + h) * (dv + 2);
+#pragma unroll
+    for (int i = 0; i < CC_MAXD / 32; ++i) {
+      const int c = lane + 32 * i;
+      if (i < nv && c < dv) P[c] = o[i];
+    }
+    if (lane == 0) { P[dv] = m_run; P[dv + 1] = l_run; }
+  }
+}
+
+// out = sum_s e^{m_s-M} o_s / (e^{sink-M} + sum_s e^{m_s-M} l_s), M = max(sink, max_s m_s).
+// grid (B*Tq, H), 128 threads.
+template <typename T>
+__global__ void __launch_bounds__(128)
+attn_combine_kernel(AttnArgs a) {
+  const int row = blockIdx.x, h = blockIdx.y;
+  const int dv = a.dv, S = a.splits;
+  const float* P0 = a.part + ((size_t)row * S * a.H + h) * (dv + 2);
+  const size_t sstride = (size_t)a.H * (dv + 2);
+  const float sk = a.sink[h];
+  float M = sk;
+  for (int s = 0; s < S; ++s) M = fmaxf(M, P0[s * sstride + dv]);
+  float den = 0.f;
+  if (M != -INFINITY) {
+    den = __expf(sk - M);
+    for (int s = 0; s < S; ++s) {
+      const float ms = P0[s * sstride + dv];
+      if (ms != -INFINITY) den += P0[s * sstride + dv + 1] * __expf(ms - M);
+    }
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  for (int c = threadIdx.x; c < dv; c += blockDim.x) {
+    float acc = 0.f;
+    for (int s = 0; s < S; ++s) {
+      const float ms = P0[s * sstride + dv];
+      if (ms != -INFINITY) acc = fmaf(P0[s * sstride + c], __expf(ms - M), acc);
+    }
+    Elem<T>::st((T*)a.out + ((size_t)row * a.H + h) * dv + c, acc * inv);
+  }
+  if (a.lse && threadIdx.x == 0) a.lse[(size_t)row * a.H + h] = den > 0.f ? M + logf(den) : -INFINITY;
+}
+
+int attn_choose_splits(int n_queries, int H, int64_t rows, bool tc_path) {
+  // aim for >= 2 waves of CTAs on 148 SMs; never split below 64 rows per split
+  const int64_t ctas_per_split = tc_path ? (int64_t)n_queries * 2 : (int64_t)n_queries * ((H + CC_HG - 1) / CC_HG);
+  int64_t s = (2 * 148 + ctas_per_split - 1) / ctas_per_split;
+  const int64_t max_s = (rows + 63) / 64;
+  if (s > max_s) s = max_s;
+  if (s < 1) s = 1;
+  if (s > 64) s = 64;
+  return (int)s;
+}
+
+cudaError_t launch_attention_cuda_core(AttnArgs a, int dtype, cudaStream_t st) {
+  const size_t smem = (size_t)CC_ROWS * a.dk * sizeof(float);
+  dim3 grid(a.splits, (a.H + CC_HG - 1) / CC_HG, a.B * a.Tq);
+  if (dtype == CSA_BF16) {
+    cudaFuncSetAttribute(attn_cuda_core_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+    attn_cuda_core_kernel<__nv_bfloat16><<<grid, 256, smem, st>>>(a);
+  } else {
+    cudaFuncSetAttribute(attn_cuda_core_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+    attn_cuda_core_kernel<float><<<grid, 256, smem, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_combine(const AttnArgs& a, int dtype, cudaStream_t st) {
+  dim3 grid(a.B * a.Tq, a.H);
+  if (dtype == CSA_BF16) attn_combine_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(a);
+  else attn_combine_kernel<float><<<grid, 128, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace csa

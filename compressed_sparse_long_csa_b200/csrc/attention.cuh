@@ -1,0 +1,76 @@
+// Internal arguments of the attention kernels.
+#pragma once
+#include "common.cuh"
+
+namespace csa {
+
+struct AttnArgs {
+  const void* q;              // [B*Tq, H, dk]
+  const void* cache;          // [B, n_max, dk]
+  const int32_t* idx;         // [B*Tq, k] (sparse) or null (dense: entries 0..n_entries[b]-1)
+  const int32_t* n_entries;   // [B] (dense)
+  int k;                      // sparse: index slots per query; dense: unused
+  const void* win;            // decode: [B, W, dk]; prefill: raw [B, t_raw, dk]
+  const int32_t* win_len;     // decode: [B]
+  const int32_t* q_pos;       // prefill: [B*Tq]
+  const int32_t* raw_pos0;    // prefill: [B]
+  int64_t t_raw;
+  int W;
+  int prefill;
+  const float* sink;          // [H]
+  int B, Tq, H, dk, dv;
+  int64_t n_max;
+  float sm_scale;
+  void* out;                  // [B*Tq, H, dv]
+  float* lse;                 // [B*Tq, H] or null
+  float* part;                // split partials [B*Tq, splits, H, dv + 2]
+  int splits;
+  int rows_per_split;
+  int n_seg_a;                // virtual rows in segment A (k or n_max)
+  unsigned* err;
+};
+
+// Number of virtual rows of a query: compressed segment + window segment.
+__host__ __device__ inline int64_t attn_virtual_rows(const AttnArgs& a) { return (int64_t)a.n_seg_a + a.W; }
+
+// Resolve virtual row v of query `row` to a latent row pointer (null = not a row).
+template <typename T>
+__device__ __forceinline__ const T* attn_row_ptr(const AttnArgs& a, int row, int v) {
+  const int b = row / a.Tq;
+  if (v < a.n_seg_a) {
+    int e;
+    if (a.idx) {
+      e = a.idx[(size_t)row * a.k + v];
+      if (e < 0) return nullptr;
+      if ((int64_t)e >= a.n_max) { raise_err(a.err, CSA_DEVERR_INDEX); return nullptr; }
+    } else {
+      int n = a.n_entries[b];
+      if ((int64_t)n > a.n_max) n = (int)a.n_max;
+      if (v >= n) return nullptr;
+      e = v;
+    }
+    return (const T*)a.cache + ((size_t)b * a.n_max + e) * a.dk;
+  }
+  const int w = v - a.n_seg_a;
+  if (!a.prefill) {
+    int wl = a.win_len[b];
+    if (wl > a.W) wl = a.W;
+    if (w >= wl) return nullptr;
+    return (const T*)a.win + ((size_t)b * a.W + w) * a.dk;
+  }
+  const int pos = a.q_pos[row];
+  const int lo = pos - a.W + 1 < 0 ? 0 : pos - a.W + 1;
+  const int p = lo + w;
+  if (p > pos) return nullptr;
+  const int64_t r = (int64_t)p - a.raw_pos0[b];
+  if (r < 0 || r >= a.t_raw) { raise_err(a.err, CSA_DEVERR_WINDOW); return nullptr; }
+  return (const T*)a.win + ((size_t)b * a.t_raw + r) * a.dk;
+}
+
+int attn_choose_splits(int n_queries, int H, int64_t rows, bool tc_path);
+
+cudaError_t launch_attention_cuda_core(AttnArgs a, int dtype, cudaStream_t st);
+cudaError_t launch_attention_tc(AttnArgs a, cudaStream_t st, bool* used);
+cudaError_t launch_attn_combine(const AttnArgs& a, int dtype, cudaStream_t st);
+
+}  // namespace csa

@@ -1,0 +1,196 @@
+// CSA and HCA gated-pooling compressors fused with the KV-cache append.
+//
+// "Техотчёт DeepSeek-V4 (2026): миллион токенов контекста", section "Гибридное
+// внимание: CSA и HCA", CSA step 1 (two value series C^a, C^b and two gate series
+// Z^a, Z^b; a per-component softmax over the 2m sources of gate + positional bias;
+// shifted, overlapping a/b windows so that each entry draws on 2m tokens) and the
+// HCA paragraph (m' = 128 tokens per entry, no overlap).
+//
+// Both kernels are HBM-bound: every input element is read exactly once and every
+// output element written once, with 16-byte vector accesses.  Softmax statistics
+// are kept per component in fp32 with a streaming (running max / sum) update.
+#include "common.cuh"
+
+namespace csa {
+
+// Streaming softmax-weighted sum over sources for VEC components at once.
+struct PoolAcc {
+  float M[8], S[8], A[8];
+  __device__ __forceinline__ void init(int vec) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) { M[i] = -INFINITY; S[i] = 0.f; A[i] = 0.f; }
+  }
+  __device__ __forceinline__ void add(const float* c, const float* z, const float* b, int vec) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (i < vec) {
+        const float l = z[i] + b[i];
+        const float Mn = fmaxf(M[i], l);
+        const float a = __expf(M[i] - Mn);
+        const float e = __expf(l - Mn);
+        S[i] = S[i] * a + e;
+        A[i] = A[i] * a + e * c[i];
+        M[i] = Mn;
+      }
+    }
+  }
+};
+
+// One thread per (entry, VEC-wide component group).  grid.y = batch.
+template <typename T>
+__global__ void __launch_bounds__(256)
+csa_compress_kernel(const T* __restrict__ Ca, const T* __restrict__ Cb, const T* __restrict__ Za,
+                    const T* __restrict__ Zb, const float* __restrict__ Ba, const float* __restrict__ Bb,
+                    const T* __restrict__ pCb, const T* __restrict__ pZb, const int32_t* __restrict__ entry0,
+                    T* __restrict__ cache, int64_t n_max, int T_new, int d, int m, unsigned* err) {
+  constexpr int VEC = Elem<T>::VEC;
+  const int b = blockIdx.y;
+  const int groups = d / VEC;
+  const int n_blk = T_new / m;
+  const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= (int64_t)n_blk * groups) return;
+  const int j = (int)(gid / groups);
+  const int c0 = (int)(gid % groups) * VEC;
+  const int e = entry0[b] + j;
+  if (e < 0 || (int64_t)e >= n_max) { raise_err(err, CSA_DEVERR_ENTRY); return; }
+
+  const size_t seq = (size_t)b * T_new * d;
+  PoolAcc acc;
+  acc.init(VEC);
+  float cv[VEC], zv[VEC], bv[8];
+  // b-half: previous block (in the chunk, or prev_* for the chunk's first entry; none for entry 0)
+  if (e > 0) {
+    for (int t = 0; t < m; ++t) {
+      const T* cp; const T* zp;
+      if (j > 0) {
+        const size_t off = seq + (size_t)((j - 1) * m + t) * d + c0;
+        cp = Cb + off; zp = Zb + off;
+      } else {
+        const size_t off = ((size_t)b * m + t) * d + c0;
+        cp = pCb + off; zp = pZb + off;
+      }
+      Elem<T>::ld_vec(cp, cv);
+      Elem<T>::ld_vec(zp, zv);
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) bv[i] = Bb[t * d + c0 + i];
+      acc.add(cv, zv, bv, VEC);
+    }
+  }
+  // a-half: own block
+  for (int t = 0; t < m; ++t) {
+    const size_t off = seq + (size_t)(j * m + t) * d + c0;
+    Elem<T>::ld_vec(Ca + off, cv);
+    Elem<T>::ld_vec(Za + off, zv);
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) bv[i] = Ba[t * d + c0 + i];
+    acc.add(cv, zv, bv, VEC);
+  }
+  float out[VEC];
+#pragma unroll
+  for (int i = 0; i < VEC; ++i) out[i] = acc.A[i] / acc.S[i];
+  Elem<T>::st_vec(cache + ((size_t)b * n_max + e) * d + c0, out);
+}
+
+// One CTA per (entry, slab of 8*VEC components, batch): 8 component groups x 32 token lanes.
+// Each thread pools tokens tl, tl+32, ... of its group; the 32 partial (M, S, A) are merged
+// in shared memory.
+template <typename T>
+__global__ void __launch_bounds__(256)
+hca_compress_kernel(const T* __restrict__ C, const T* __restrict__ Z, const float* __restrict__ bias,
+                    const int32_t* __restrict__ entry0, T* __restrict__ cache, int64_t n_max,
+                    int T_new, int d, int mp, unsigned* err) {
+  constexpr int VEC = Elem<T>::VEC;
+  constexpr int SLAB = 8 * VEC;
+  __shared__ float sM[32][SLAB + 1], sS[32][SLAB + 1], sA[32][SLAB + 1];
+  const int j = blockIdx.x;          // entry within chunk
+  const int slab = blockIdx.y;
+  const int b = blockIdx.z;
+  const int g = threadIdx.x & 7;     // component group inside slab
+  const int tl = threadIdx.x >> 3;   // token lane 0..31
+  const int c0 = slab * SLAB + g * VEC;
+  const int e = entry0[b] + j;
+  const bool valid_e = !(e < 0 || (int64_t)e >= n_max);
+  const bool active = c0 < d;
+
+  PoolAcc acc;
+  acc.init(VEC);
+  if (active && valid_e) {
+    float cv[VEC], zv[VEC], bv[8];
+    for (int t = tl; t < mp; t += 32) {
+      const size_t off = ((size_t)b * T_new + (size_t)j * mp + t) * d + c0;
+      Elem<T>::ld_vec(C + off, cv);
+      Elem<T>::ld_vec(Z + off, zv);
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) bv[i] = bias[(size_t)t * d + c0 + i];
+      acc.add(cv, zv, bv, VEC);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < VEC; ++i) {
+    sM[tl][g * VEC + i] = acc.M[i];
+    sS[tl][g * VEC + i] = acc.S[i];
+    sA[tl][g * VEC + i] = acc.A[i];
+  }
+  __syncthreads();
+  if (!valid_e) {
+    if (threadIdx.x == 0) raise_err(err, CSA_DEVERR_ENTRY);
+    return;
+  }
+  if (threadIdx.x < SLAB) {
+    const int col = threadIdx.x;
+    const int c = slab * SLAB + col;
+    if (c < d) {
+      float M = -INFINITY;
+      for (int l = 0; l < 32; ++l) M = fmaxf(M, sM[l][col]);
+      float S = 0.f, A = 0.f;
+      for (int l = 0; l < 32; ++l) {
+        const float a = (sS[l][col] > 0.f) ? __expf(sM[l][col] - M) : 0.f;
+        S += sS[l][col] * a;
+        A += sA[l][col] * a;
+      }
+      Elem<T>::st(cache + ((size_t)b * n_max + e) * d + c, A / S);
+    }
+  }
+}
+
+cudaError_t launch_csa_compress(const void* Ca, const void* Cb, const void* Za, const void* Zb,
+                                const float* Ba, const float* Bb, const void* pCb, const void* pZb,
+                                const int32_t* entry0, void* cache, int64_t n_max, int B, int T_new,
+                                int d, int m, int dtype, cudaStream_t st, unsigned* err) {
+  const int n_blk = T_new / m;
+  if (dtype == CSA_BF16) {
+    using T = __nv_bfloat16;
+    const int64_t work = (int64_t)n_blk * (d / 8);
+    dim3 grid((unsigned)((work + 255) / 256), B);
+    csa_compress_kernel<T><<<grid, 256, 0, st>>>((const T*)Ca, (const T*)Cb, (const T*)Za, (const T*)Zb,
+                                                 Ba, Bb, (const T*)pCb, (const T*)pZb, entry0, (T*)cache,
+                                                 n_max, T_new, d, m, err);
+  } else {
+    const int64_t work = (int64_t)n_blk * (d / 4);
+    dim3 grid((unsigned)((work + 255) / 256), B);
+    csa_compress_kernel<float><<<grid, 256, 0, st>>>((const float*)Ca, (const float*)Cb, (const float*)Za,
+                                                     (const float*)Zb, Ba, Bb, (const float*)pCb,
+                                                     (const float*)pZb, entry0, (float*)cache, n_max,
+                                                     T_new, d, m, err);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_hca_compress(const void* C, const void* Z, const float* bias, const int32_t* entry0,
+                                void* cache, int64_t n_max, int B, int T_new, int d, int mp, int dtype,
+                                cudaStream_t st, unsigned* err) {
+  const int n_blk = T_new / mp;
+  if (dtype == CSA_BF16) {
+    using T = __nv_bfloat16;
+    dim3 grid(n_blk, (d + 63) / 64, B);
+    hca_compress_kernel<T><<<grid, 256, 0, st>>>((const T*)C, (const T*)Z, bias, entry0, (T*)cache, n_max,
+                                                 T_new, d, mp, err);
+  } else {
+    dim3 grid(n_blk, (d + 31) / 32, B);
+    hca_compress_kernel<float><<<grid, 256, 0, st>>>((const float*)C, (const float*)Z, bias, entry0,
+                                                     (float*)cache, n_max, T_new, d, mp, err);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace csa

@@ -1,0 +1,46 @@
+// Internal arguments of the indexer / top-k kernels.
+#pragma once
+#include "common.cuh"
+
+namespace csa {
+
+struct IndexerArgs {
+  const void* qI;
+  const void* qI_scale;
+  const float* w;
+  const void* kI;
+  const void* kI_scale;
+  const int32_t* n_entries;   // [B]
+  const int32_t* q_pos;       // [B*Tq]
+  int m;
+  int B, Tq, H_I, d_I;
+  int64_t n_max;
+  int k;
+  int ifmt;
+  float* scores;              // workspace [B*Tq, ld] fp32 scores
+  int64_t ld;
+  unsigned* knmax;            // workspace [B]: bits of max_s ||k_s||_2 (dequantised)
+  int32_t* idx_out;           // [B*Tq, k]
+  float* score_out;           // [B*Tq, k] or null
+  unsigned* err;
+  float eps_dot;              // bound on |fp32 dot - exact| / (||q|| ||k||) of the scoring path
+};
+
+// Number of entries visible to query row `row` (= b*Tq + t): all m sources <= pos.
+__device__ __forceinline__ int row_eligible(const IndexerArgs& a, int row) {
+  const int b = row / a.Tq;
+  const int pos = a.q_pos[row];
+  int ne = pos < 0 ? 0 : (pos + 1) / a.m;
+  int n = a.n_entries[b];
+  if ((int64_t)n > a.n_max) n = (int)a.n_max;
+  if (n < 0) n = 0;
+  return ne < n ? ne : n;
+}
+
+cudaError_t launch_indexer_scores_cuda_core(const IndexerArgs& a, cudaStream_t st);
+cudaError_t launch_indexer_scores_tc(const IndexerArgs& a, cudaStream_t st, bool* used);
+cudaError_t launch_indexer_select(const IndexerArgs& a, cudaStream_t st);
+cudaError_t launch_topk_select(const float* scores, int64_t ld, const int32_t* n_valid, int R, int64_t n,
+                               int k, int32_t* idx_out, cudaStream_t st, unsigned* err);
+
+}  // namespace csa

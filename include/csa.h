@@ -1,0 +1,226 @@
+/*
+ * csa.h — C ABI of the B200 (sm_100a) CSA / HCA attention hot path.
+ *
+ * The operations follow the DeepSeek-V4 technical report as digested in
+ * "Техотчёт DeepSeek-V4 (2026): миллион токенов контекста" (ai.flicky.cc),
+ * section "Гибридное внимание: CSA и HCA" (CSA steps 1-3, the HCA paragraph,
+ * the 128-token sliding window), table "Конфигурации" (m = 4, m' = 128,
+ * top-k 512 / 1024, 128 heads of width 512) and section "FP4 с учётом
+ * квантования" (FP4 indexer path); plus "Технический отчёт DeepSeek-V4 — часть
+ * 1/2" (aifinder.ae) for the MLA latent (576 = 512 + 64 RoPE dims), the window
+ * branch and the attention sink.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Every pointer named as device memory must be a CUDA device pointer on the
+ *   current device; sizes are element counts.  All tensors are dense, row-major
+ *   (C order) with the shapes given; the library never allocates, frees or
+ *   synchronises: outputs and workspaces belong to the caller.
+ * - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *   NULL = the legacy default stream).  It returns CSA_OK once its kernels are
+ *   enqueued.  Arguments are validated on the host BEFORE any launch; an invalid
+ *   argument returns an error code and enqueues nothing.
+ * - Device-side checks (an index out of range, a window row outside the raw
+ *   buffer, a bounded wait that gave up, a top-k candidate band that overflowed)
+ *   never fault: the offending access is skipped and a bit is OR-ed into a
+ *   per-device error word that csa_read_device_error() returns and clears.
+ * - Latent rows (compressor inputs, KV cache, window, queries, outputs) are
+ *   stored as CSA_BF16 or CSA_F32 (dtype argument).  Biases, sinks, indexer
+ *   weights and FP8 scales are always fp32.
+ * - 16-byte alignment is required of every device pointer; row widths must keep
+ *   rows 16-byte aligned (d * element size % 16 == 0).
+ */
+#ifndef CSA_B200_H
+#define CSA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define CSA_ABI_VERSION 1
+
+typedef enum csa_status {
+  CSA_OK = 0,
+  CSA_ERR_NULL = 1,        /* a required pointer is NULL                              */
+  CSA_ERR_SHAPE = 2,       /* a size is out of range or sizes are inconsistent         */
+  CSA_ERR_DTYPE = 3,       /* unsupported storage / operand format                     */
+  CSA_ERR_ALIGN = 4,       /* a device pointer is not 16-byte aligned                  */
+  CSA_ERR_UNSUPPORTED = 5, /* no kernel for this combination of sizes                  */
+  CSA_ERR_WORKSPACE = 6,   /* workspace NULL or smaller than the *_workspace_size()    */
+  CSA_ERR_CUDA = 7         /* a CUDA runtime call or launch failed                     */
+} csa_status;
+
+typedef enum csa_dtype { CSA_F32 = 0, CSA_BF16 = 1 } csa_dtype;
+
+/* Operand format of the lightning indexer (queries and keys use the same one). */
+typedef enum csa_ifmt {
+  CSA_IFMT_F32 = 0,   /* fp32 values, no scales                                      */
+  CSA_IFMT_E4M3 = 1,  /* FP8 e4m3 codes (1 byte) + one fp32 scale per row             */
+  CSA_IFMT_MXFP4 = 2  /* e2m1 codes packed 2 per byte (element 2i in the low nibble) +
+                         one ue8m0 scale byte (2^(code-127)) per 32 consecutive elements */
+} csa_ifmt;
+
+/* Bits of the per-device error word. */
+#define CSA_DEVERR_INDEX    0x1u  /* a KV / entry index outside [0, n_max): row skipped   */
+#define CSA_DEVERR_WINDOW   0x2u  /* a window row outside the raw buffer: row skipped    */
+#define CSA_DEVERR_TIMEOUT  0x4u  /* a bounded device-side wait gave up                  */
+#define CSA_DEVERR_BAND     0x8u  /* top-k candidate band exceeded its capacity          */
+#define CSA_DEVERR_ENTRY    0x10u /* a compressor output entry outside [0, n_max): skipped */
+
+int csa_abi_version(void);
+const char* csa_status_string(int status);
+
+/* Reads the calling device's error word into *out (host pointer), then clears
+ * it.  Synchronises `stream` (the only call that does).                       */
+csa_status csa_read_device_error(void* stream, uint32_t* out);
+
+/* ---------------------------------------------------------------------------
+ * csa_compress — CSA token-axis compression fused with the KV-cache append.
+ * ("Гибридное внимание: CSA и HCA", CSA step 1: two KV series C^a, C^b and two
+ * gate series Z^a, Z^b; per component a softmax over the 2m sources of
+ * (Z + learnable positional bias), then the weighted sum; the a/b windows are
+ * shifted so that entry i draws on 2m tokens and the length still shrinks m×.)
+ *
+ * Entry e of a sequence pools, per component c, the b-series of tokens
+ * m*e-m .. m*e-1 (bias Bb[j]) and the a-series of tokens m*e .. m*e+m-1
+ * (bias Ba[j]), j = offset inside the block.  Entry 0 has no b-half.
+ *
+ *   Ca, Cb, Za, Zb  device [B, T_new, d] dtype: the chunk's tokens, which start
+ *                   at token m*entry0[b] of sequence b; T_new % m == 0
+ *   Ba, Bb          device [m, d] fp32 positional biases
+ *   prev_Cb, prev_Zb device [B, m, d] dtype: b-series of the block just before
+ *                   the chunk (read only where entry0[b] > 0)
+ *   entry0          device [B] int32: index of the chunk's first entry
+ *   cache           device [B, n_max, d] dtype: rows entry0[b] .. entry0[b]+T_new/m-1
+ *                   are written (outputs rounded to nearest-even for bf16)
+ * Supported: m in 1..16, d % 8 == 0 (bf16) or d % 4 == 0 (f32).
+ * ------------------------------------------------------------------------- */
+csa_status csa_compress(const void* Ca, const void* Cb, const void* Za, const void* Zb,
+                        const float* Ba, const float* Bb,
+                        const void* prev_Cb, const void* prev_Zb,
+                        const int32_t* entry0, void* cache, int64_t n_max,
+                        int B, int T_new, int d, int m, int dtype, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * hca_compress — HCA compression ("HCA: сжать в 128 раз, но смотреть на всё":
+ * the same gated pooling with m' tokens per entry and no overlap).
+ *
+ *   C, Z    device [B, T_new, d] dtype, T_new % m_prime == 0, starting at token
+ *           m_prime*entry0[b]
+ *   bias    device [m_prime, d] fp32
+ *   cache   device [B, n_max, d]: rows entry0[b] .. entry0[b]+T_new/m_prime-1 written
+ * Supported: m_prime in 1..1024.
+ * ------------------------------------------------------------------------- */
+csa_status hca_compress(const void* C, const void* Z, const float* bias,
+                        const int32_t* entry0, void* cache, int64_t n_max,
+                        int B, int T_new, int d, int m_prime, int dtype, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * lightning_index — indexer scores and top-k selection of compressed entries
+ * ("Гибридное внимание: CSA и HCA", CSA step 2: the DSA lightning indexer
+ * scores I[t,s] with a ReLU and keeps the top-k compressed blocks; FP4 Q·K
+ * path from "FP4 с учётом квантования").
+ *
+ *   I[t,s] = sum_j w[t,j] * max(0, <q[t,j], k[s]>)   (dequantised operands)
+ *
+ * Query t of sequence b at absolute position pos = q_pos[b*Tq+t] sees entries
+ * s < min(n_entries[b], (pos+1)/m) (all of an entry's tokens are <= pos).  The
+ * k entries with the largest I are returned, ties to the lower index, in
+ * ascending index order, padded with -1.  Selection is exact: tensor-core fp32
+ * scores pick a candidate band which is re-scored in fp64 on CUDA cores.
+ *
+ *   qI       device [B, Tq, H_I, d_I] (F32: fp32; E4M3: bytes; MXFP4: [.., d_I/2] bytes)
+ *   qI_scale E4M3: device [B, Tq, H_I] fp32; MXFP4: [B, Tq, H_I, d_I/32] bytes; F32: NULL
+ *   w        device [B, Tq, H_I] fp32 head weights
+ *   kI       device [B, n_max, d_I] (same format; MXFP4 [B, n_max, d_I/2])
+ *   kI_scale E4M3: device [B, n_max] fp32; MXFP4: [B, n_max, d_I/32] bytes; F32: NULL
+ *   n_entries device [B] int32, q_pos device [B, Tq] int32
+ *   idx_out  device [B, Tq, k] int32;  score_out device [B, Tq, k] fp32 or NULL
+ *            (the fp64 score of each selected entry rounded to fp32; 0 for pads)
+ *   workspace >= lightning_index_workspace_size(B, Tq, n_max, k) bytes
+ * Supported: B*Tq <= 65535, H_I <= 64, d_I in {32, 64, 128}, k <= 2048,
+ * n_max <= 2^24.
+ * ------------------------------------------------------------------------- */
+size_t lightning_index_workspace_size(int B, int Tq, int64_t n_max, int k);
+csa_status lightning_index(const void* qI, const void* qI_scale, const float* w,
+                           const void* kI, const void* kI_scale,
+                           const int32_t* n_entries, const int32_t* q_pos, int m,
+                           int B, int Tq, int H_I, int d_I, int64_t n_max, int k, int ifmt,
+                           int32_t* idx_out, float* score_out,
+                           void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * topk_select — exact top-k of fp32 scores (CSA step 2's selection on its own).
+ *   scores   device [R, ld] fp32; row r has n_valid[r] valid leading entries
+ *   idx_out  device [R, k] int32: the k largest, ties to the lower index,
+ *            ascending index order, -1 padding.  NaN ranks below every number.
+ * Supported: k <= 2048, n <= 2^24.
+ * ------------------------------------------------------------------------- */
+size_t topk_select_workspace_size(int R, int64_t n, int k);
+csa_status topk_select(const float* scores, int64_t ld, const int32_t* n_valid,
+                       int R, int64_t n, int k, int32_t* idx_out,
+                       void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Attention over compressed entries + raw window + sink ("Гибридное внимание:
+ * CSA и HCA", CSA step 3: every compressed entry is key and value for all query
+ * heads (MQA); the 128-token window of uncompressed entries; the attention sink
+ * and the 576 = 512 + 64 latent of "Технический отчёт DeepSeek-V4 — часть 1/2").
+ *
+ * For head h of a query, over the row set R (selected / all compressed entries
+ * plus window rows):  l_r = sm_scale * <q_h, row_r[0:d_k]>,
+ *   out_h = sum_r e^{l_r - M} row_r[0:d_v] / (e^{sink_h - M} + sum_r e^{l_r - M}),
+ *   M = max(sink_h, max_r l_r),   lse_h = M + log(e^{sink_h-M} + sum_r e^{l_r-M}).
+ * Pass sink = -INFINITY for no sink.  out is rounded to dtype; lse is fp32.
+ * Supported: H <= 128, d_v <= d_k <= 576, d_k % 8 == 0.  The tcgen05 path runs
+ * for bf16 with H == 128, d_k == 576, d_v == 512; other shapes run a CUDA-core path.
+ * ------------------------------------------------------------------------- */
+
+/* Workspace for the split-KV partials of the decode calls: sparse_attn_decode needs
+ * attn_decode_workspace_size(B, H, d_v, k + W) bytes and hca_attn_decode
+ * attn_decode_workspace_size(B, H, d_v, n_max + W); CSA_ERR_WORKSPACE otherwise.
+ * sparse_attn_prefill takes no workspace (pass NULL, 0).                         */
+size_t attn_decode_workspace_size(int B, int H, int d_v, int64_t rows_max);
+
+/* sparse_attn_decode — one query token per sequence.
+ *   q       device [B, H, d_k];  cache device [B, n_max, d_k]
+ *   idx     device [B, k] int32 entry ids (-1 = unused slot)
+ *   win     device [B, W, d_k]: raw latents of the last win_len[b] positions
+ *   win_len device [B] int32 (0..W)
+ *   sink    device [H] fp32
+ *   out     device [B, H, d_v];  lse device [B, H] fp32 or NULL                */
+csa_status sparse_attn_decode(const void* q, const void* cache, const int32_t* idx,
+                              const void* win, const int32_t* win_len, const float* sink,
+                              int B, int H, int d_k, int d_v, int64_t n_max, int k, int W,
+                              float sm_scale, int dtype, void* out, float* lse,
+                              void* workspace, size_t ws_bytes, void* stream);
+
+/* hca_attn_decode — dense attention over entries 0..n_entries[b]-1 + window.
+ *   n_entries device [B] int32 (<= n_max); other arguments as sparse_attn_decode. */
+csa_status hca_attn_decode(const void* q, const void* cache, const int32_t* n_entries,
+                           const void* win, const int32_t* win_len, const float* sink,
+                           int B, int H, int d_k, int d_v, int64_t n_max, int W,
+                           float sm_scale, int dtype, void* out, float* lse,
+                           void* workspace, size_t ws_bytes, void* stream);
+
+/* sparse_attn_prefill — Tq query tokens per sequence, each with its own index set.
+ *   q        device [B, Tq, H, d_k];  q_pos device [B, Tq] int32 absolute positions
+ *   idx      device [B, Tq, k] int32 (-1 = unused)
+ *   raw      device [B, t_raw, d_k]: raw latents of positions raw_pos0[b] ..
+ *            raw_pos0[b]+t_raw-1 (raw_pos0 device [B] int32)
+ *   The window of a query at pos is positions max(0, pos-W+1) .. pos.
+ *   out      device [B, Tq, H, d_v];  lse device [B, Tq, H] fp32 or NULL       */
+csa_status sparse_attn_prefill(const void* q, const int32_t* q_pos, const void* cache,
+                               const int32_t* idx, const void* raw, int64_t t_raw,
+                               const int32_t* raw_pos0, const float* sink,
+                               int B, int Tq, int H, int d_k, int d_v, int64_t n_max, int k,
+                               int W, float sm_scale, int dtype, void* out, float* lse,
+                               void* workspace, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA_B200_H */

@@ -199,6 +199,12 @@ def hca_compress(C, Z, bias, m_prime=128):
 # a3: lightning indexer  ([P1] CSA step 2 and "FP4 с учётом квантования"; [P3])
 # ---------------------------------------------------------------------------
 
+def _dots(qv, kv):
+    """D[t, j, s] = sum_c qv[t, j, c] * kv[s, c] (a library float64 matmul)."""
+    Tq, HI, dI = qv.shape
+    return (qv.reshape(Tq * HI, dI) @ kv.T).reshape(Tq, HI, kv.shape[0])
+
+
 def head_dots(q, k, fmt, q_scale=None, k_scale=None):
     """Per-head dot products D[t, j, s] = <q[t,j], k[s]> with dequantisation scales.
 
@@ -211,11 +217,11 @@ def head_dots(q, k, fmt, q_scale=None, k_scale=None):
     if fmt == "f32":
         qv = np.asarray(q, dtype=np.float64)
         kv = np.asarray(k, dtype=np.float64)
-        return np.einsum("tjc,sc->tjs", qv, kv)
+        return _dots(qv, kv)
     if fmt == "e4m3":
         qv = decode_e4m3(q)
         kv = decode_e4m3(k)
-        raw = np.einsum("tjc,sc->tjs", qv, kv)               # exact: 43-bit span < 53
+        raw = _dots(qv, kv)                                    # exact: 43-bit span < 53
         return (np.asarray(q_scale, np.float64)[:, :, None]
                 * np.asarray(k_scale, np.float64)[None, None, :]) * raw
     if fmt == "mxfp4":
@@ -228,7 +234,7 @@ def head_dots(q, k, fmt, q_scale=None, k_scale=None):
         ks = decode_ue8m0(k_scale)                             # [N, nb]
         D = np.zeros((Tq, HI, N), dtype=np.float64)
         for b in range(nb):
-            part = np.einsum("tjc,sc->tjs", qv[:, :, 32 * b:32 * (b + 1)], kv[:, 32 * b:32 * (b + 1)])
+            part = _dots(qv[:, :, 32 * b:32 * (b + 1)], kv[:, 32 * b:32 * (b + 1)])
             D += qs[:, :, b][:, :, None] * ks[:, b][None, None, :] * part
         return D
     raise ValueError(fmt)

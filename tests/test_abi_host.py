@@ -1,0 +1,114 @@
+"""Host-only checks of the C ABI: the library loads, exports every declared entry
+point, and rejects invalid arguments with the documented status codes before any
+device work (these calls never reach a kernel, so they run without a GPU)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+import compressed_sparse_long_csa_b200 as csa
+from compressed_sparse_long_csa_b200 import _native as N
+
+HDR = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "csa.h")
+OK, ERR_NULL, ERR_SHAPE, ERR_DTYPE, ERR_ALIGN, ERR_UNSUP, ERR_WS, ERR_CUDA = range(8)
+
+
+def declared_functions():
+    src = open(HDR).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\**\s+\**([a-z_0-9]+)\s*\(", src, flags=re.M)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert {"csa_compress", "hca_compress", "lightning_index", "topk_select", "sparse_attn_decode",
+            "sparse_attn_prefill", "hca_attn_decode"} <= set(names)
+    for n in names:
+        assert hasattr(N.lib, n), n
+
+
+def test_version_and_strings():
+    assert N.lib.csa_abi_version() == 1
+    for s in range(8):
+        assert N.lib.csa_status_string(s).startswith(b"CSA_")
+
+
+FAKE = 1 << 20          # a 16-byte aligned non-null address that is never dereferenced on the host
+
+
+def compress(**kw):
+    args = dict(Ca=FAKE, Cb=FAKE, Za=FAKE, Zb=FAKE, Ba=FAKE, Bb=FAKE, pCb=FAKE, pZb=FAKE, e0=FAKE, cache=FAKE,
+                n_max=64, B=1, T=16, d=64, m=4, dtype=0)
+    args.update(kw)
+    a = args
+    return N.lib.csa_compress(a["Ca"], a["Cb"], a["Za"], a["Zb"], a["Ba"], a["Bb"], a["pCb"], a["pZb"], a["e0"],
+                              a["cache"], a["n_max"], a["B"], a["T"], a["d"], a["m"], a["dtype"], None)
+
+
+def test_compress_validation():
+    assert compress(Ca=None) == ERR_NULL
+    assert compress(e0=None) == ERR_NULL
+    assert compress(Cb=FAKE + 4) == ERR_ALIGN
+    assert compress(dtype=7) == ERR_DTYPE
+    assert compress(T=15) == ERR_SHAPE          # not a multiple of m
+    assert compress(m=0) == ERR_SHAPE
+    assert compress(m=17) == ERR_SHAPE
+    assert compress(d=6) == ERR_SHAPE           # rows must stay 16-byte aligned
+    assert compress(dtype=1, d=12) == ERR_SHAPE
+
+
+def test_indexer_validation():
+    def call(**kw):
+        a = dict(qI=FAKE, qs=FAKE, w=FAKE, kI=FAKE, ks=FAKE, ne=FAKE, qp=FAKE, m=4, B=1, Tq=1, HI=64, dI=128,
+                 n_max=1024, k=64, ifmt=1, idx=FAKE, so=None, ws=FAKE, wsb=1 << 30)
+        a.update(kw)
+        return N.lib.lightning_index(a["qI"], a["qs"], a["w"], a["kI"], a["ks"], a["ne"], a["qp"], a["m"], a["B"],
+                                     a["Tq"], a["HI"], a["dI"], a["n_max"], a["k"], a["ifmt"], a["idx"], a["so"],
+                                     a["ws"], a["wsb"], None)
+    assert call(ifmt=9) == ERR_DTYPE
+    assert call(dI=48) == ERR_SHAPE
+    assert call(HI=65) == ERR_SHAPE
+    assert call(k=4096) == ERR_SHAPE
+    assert call(qs=None) == ERR_NULL
+    assert call(ifmt=0, qs=None, ks=None) != ERR_NULL      # fp32 operands need no scales
+    assert call(wsb=16) == ERR_WS
+    assert call(ws=None) == ERR_WS
+    need = N.lib.lightning_index_workspace_size(2, 3, 1000, 64)
+    assert need >= 2 * 3 * 1000 * 4
+
+
+def test_attention_validation():
+    def call(**kw):
+        a = dict(q=FAKE, cache=FAKE, idx=FAKE, win=FAKE, wl=FAKE, sink=FAKE, B=2, H=128, dk=576, dv=512,
+                 n_max=4096, k=512, W=128, scale=0.04, dtype=1, out=FAKE, lse=None, ws=FAKE, wsb=1 << 30)
+        a.update(kw)
+        return N.lib.sparse_attn_decode(a["q"], a["cache"], a["idx"], a["win"], a["wl"], a["sink"], a["B"], a["H"],
+                                        a["dk"], a["dv"], a["n_max"], a["k"], a["W"], a["scale"], a["dtype"],
+                                        a["out"], a["lse"], a["ws"], a["wsb"], None)
+    assert call(H=129) == ERR_SHAPE
+    assert call(dv=640) == ERR_SHAPE
+    assert call(dk=580) == ERR_SHAPE
+    assert call(dtype=3) == ERR_DTYPE
+    assert call(idx=None) == ERR_NULL
+    assert call(wl=None) == ERR_NULL
+    assert call(out=FAKE + 2) == ERR_ALIGN
+    assert call(scale=float("nan")) == ERR_SHAPE
+    assert call(ws=None, wsb=0) == ERR_WS
+    assert N.lib.attn_decode_workspace_size(16, 128, 512, 640) > 0
+
+
+def test_topk_validation():
+    assert N.lib.topk_select(FAKE, 100, None, 4, 100, 4096, FAKE, None, 0, None) == ERR_SHAPE
+    assert N.lib.topk_select(FAKE, 50, None, 4, 100, 8, FAKE, None, 0, None) == ERR_SHAPE   # ld < n
+    assert N.lib.topk_select(None, 100, None, 4, 100, 8, FAKE, None, 0, None) == ERR_NULL
+
+
+def test_package_has_no_cpu_fallback():
+    # the binding exposes only library calls; importing never pulls in the oracle
+    import sys
+    assert not any(m.startswith("oracle") for m in sys.modules if m.startswith("oracle") and
+                   getattr(sys.modules[m], "__file__", "").startswith(os.path.dirname(csa.__file__)))
+    src = open(os.path.join(os.path.dirname(csa.__file__), "_native.py")).read() + \
+        open(os.path.join(os.path.dirname(csa.__file__), "steps.py")).read()
+    assert "oracle" not in src
