@@ -297,8 +297,6 @@ csa_status sparse_attn_prefill(const void* q, const int32_t* q_pos, const void* 
   REQUIRE(q_pos, CSA_ERR_NULL);
   REQUIRE(W == 0 || (raw_pos0 && t_raw >= 1), CSA_ERR_NULL);
   REQUIRE(isfinite(sm_scale), CSA_ERR_SHAPE);
-  REQUIRE(workspace && ws_bytes >= attn_decode_workspace_size(B, H, d_v, (int64_t)k + W), CSA_ERR_WORKSPACE);
-  REQUIRE(aligned16(workspace), CSA_ERR_ALIGN);
   unsigned* err = device_error_word();
   REQUIRE(err, CSA_ERR_CUDA);
   AttnArgs a{};

@@ -154,9 +154,16 @@ attn_combine_kernel(AttnArgs a) {
 }
 
 int attn_choose_splits(int n_queries, int H, int64_t rows, bool tc_path) {
-  // aim for >= 2 waves of CTAs on 148 SMs; never split below 64 rows per split
-  const int64_t ctas_per_split = tc_path ? (int64_t)n_queries * 2 : (int64_t)n_queries * ((H + CC_HG - 1) / CC_HG);
-  int64_t s = (2 * 148 + ctas_per_split - 1) / ctas_per_split;
+  int64_t s;
+  if (tc_path) {
+    // one wave of CTA pairs (one CTA per SM): every split re-reads the 147 KB query
+    // from L2, so more splits than SMs cost more than they hide
+    s = 148 / (2 * (int64_t)n_queries);
+  } else {
+    // aim for >= 2 waves of CTAs on 148 SMs
+    const int64_t ctas_per_split = (int64_t)n_queries * ((H + CC_HG - 1) / CC_HG);
+    s = (2 * 148 + ctas_per_split - 1) / ctas_per_split;
+  }
   const int64_t max_s = (rows + 63) / 64;
   if (s > max_s) s = max_s;
   if (s < 1) s = 1;

@@ -258,3 +258,35 @@ def test_lightning_index_score_out_and_k_equals_n():
         I = O.indexer_scores(wl.tensors["qI"][b], wl.tensors["w"][b], wl.tensors["kI"][b], "e4m3",
                              wl.tensors["qI_scale"][b], wl.tensors["kI_scale"][b])[0]
         np.testing.assert_allclose(so[b, 0].cpu().numpy(), I, rtol=1e-6)
+
+
+@pytest.mark.parametrize("wid,sc", [(1, {"B": 4, "T": 65536}), (3, {"ctx": 16384, "Tq": 64, "k": 1024})])
+def test_indexer_fp32_score_error_within_band_bound(wid, sc):
+    """The exact top-k trusts |S32 - S| <= eps * U * knmax (U = sum_j w_j ||q_j||,
+    knmax >= max_s ||k_s||).  Measure the fp32 scores the scoring kernel leaves in
+    the workspace against the exact oracle scores and check the bound with margin."""
+    wl = CI.make_workload(wid, scale=sc)
+    D = wl.dims
+    T = steps.upload(wl)
+    csa.lightning_index(T["qI"], T["qI_scale"], T["w"], T["kI"], T["kI_scale"], T["n_entries"], T["q_pos"], D["k"],
+                        csa.CSA_IFMT_E4M3, T["idx"], T["iws"])
+    torch.cuda.synchronize()
+    B, Tq, N = D["B"], D["Tq"], D["N"]
+    ld = (N + 63) // 64 * 64
+    S32 = T["iws"][:B * Tq * ld * 4].view(torch.float32).view(B, Tq, ld).double().cpu().numpy()
+    off = (B * Tq * ld * 4 + 255) // 256 * 256
+    knmax = T["iws"][off:off + 4 * B].view(torch.float32).double().cpu().numpy()
+    worst = 0.0
+    for b in range(B):
+        qv = O.decode_e4m3(wl.tensors["qI"][b]) * wl.tensors["qI_scale"][b][..., None]
+        U = (wl.tensors["w"][b] * np.sqrt((qv ** 2).sum(-1))).sum(-1)                  # [Tq]
+        kn = np.sqrt(((O.decode_e4m3(wl.tensors["kI"][b]) * wl.tensors["kI_scale"][b][:, None]) ** 2).sum(-1))
+        assert knmax[b] >= kn.max() * (1 - 1e-6)
+        I = O.indexer_scores(wl.tensors["qI"][b], wl.tensors["w"][b], wl.tensors["kI"][b], "e4m3",
+                             wl.tensors["qI_scale"][b], wl.tensors["kI_scale"][b])
+        for t in range(Tq):
+            ne = O.n_eligible(D["q_pos0"] + t, D["m"], N)
+            err = np.abs(S32[b, t, :ne] - I[t, :ne]) / (U[t] * knmax[b])
+            worst = max(worst, float(err.max()))
+    print(f"max |S32-S| / (U knmax) = {worst:.3e}")
+    assert worst <= 1.0 / 4096 / 4          # the kernel's eps with a 4x margin
