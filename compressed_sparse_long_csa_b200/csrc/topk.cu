@@ -31,8 +31,8 @@ struct TopkShared {
   int32_t amb[AMB_CAP];
   double amb_s[AMB_CAP];
   double contrib[32][64];
-  float kf[32][128];
-  float qf[64 * 129];
+  double kd[32][128];          // per-warp key row being re-scored (exact fp64 values of the codes)
+  double qd[64 * 129];         // query row codes as fp64 (padded rows: conflict-free per-head reads)
   float qsc[64 * 4];
   float w[64];
   uint32_t digit, remaining, n_sel, n_amb;
@@ -179,7 +179,7 @@ __device__ double rescore_entry(const IndexerArgs& a, TopkShared& sh, int row, i
   const int b = row / a.Tq;
   const int HI = a.H_I, dI = a.d_I, nb = dI / 32;
   const size_t koff = (size_t)b * a.n_max + s;
-  float* kf = sh.kf[warp];
+  double* kd = sh.kd[warp];
   for (int c = lane; c < dI; c += 32) {
     float v;
     if (a.ifmt == CSA_IFMT_F32) v = ((const float*)a.kI)[koff * dI + c];
@@ -188,7 +188,7 @@ __device__ double rescore_entry(const IndexerArgs& a, TopkShared& sh, int row, i
       const uint8_t byte = ((const uint8_t*)a.kI)[koff * (dI / 2) + c / 2];
       v = e2m1_to_float((c & 1) ? (byte >> 4) : (byte & 0xF));
     }
-    kf[c] = v;
+    kd[c] = (double)v;
   }
   __syncwarp();
   double ks = 1.0;
@@ -197,18 +197,18 @@ __device__ double rescore_entry(const IndexerArgs& a, TopkShared& sh, int row, i
   if (a.ifmt == CSA_IFMT_MXFP4)
     for (int bb = 0; bb < nb; ++bb) kblk[bb] = (double)ue8m0_to_float(((const uint8_t*)a.kI_scale)[koff * nb + bb]);
   for (int j = lane; j < HI; j += 32) {
-    const float* qj = sh.qf + j * 129;
+    const double* qj = sh.qd + j * 129;
     double D;
     if (a.ifmt == CSA_IFMT_MXFP4) {
       D = 0.0;
       for (int bb = 0; bb < nb; ++bb) {
         double part = 0.0;
-        for (int c = bb * 32; c < bb * 32 + 32; ++c) part = fma((double)qj[c], (double)kf[c], part);
+        for (int c = bb * 32; c < bb * 32 + 32; ++c) part = fma(qj[c], kd[c], part);
         D += ((double)sh.qsc[j * nb + bb] * kblk[bb]) * part;
       }
     } else {
       double raw = 0.0;
-      for (int c = 0; c < dI; ++c) raw = fma((double)qj[c], (double)kf[c], raw);
+      for (int c = 0; c < dI; ++c) raw = fma(qj[c], kd[c], raw);
       D = (a.ifmt == CSA_IFMT_E4M3) ? ((double)sh.qsc[j] * ks) * raw : raw;
     }
     sh.contrib[warp][j] = (double)sh.w[j] * fmax(D, 0.0);
@@ -246,7 +246,7 @@ indexer_select_kernel(IndexerArgs a) {
       const uint8_t byte = ((const uint8_t*)a.qI)[qoff * (dI / 2) + c / 2];
       v = e2m1_to_float((c & 1) ? (byte >> 4) : (byte & 0xF));
     }
-    sh.qf[j * 129 + c] = v;
+    sh.qd[j * 129 + c] = (double)v;
   }
   for (int i = threadIdx.x; i < HI; i += blockDim.x) {
     sh.w[i] = a.w[(size_t)row * HI + i];
@@ -276,7 +276,7 @@ indexer_select_kernel(IndexerArgs a) {
     for (int j = lane; j < HI; j += 32) {
       float n2 = 0.f;
       for (int c = 0; c < dI; ++c) {
-        float v = sh.qf[j * 129 + c];
+        float v = (float)sh.qd[j * 129 + c];
         if (a.ifmt == CSA_IFMT_E4M3) v *= sh.qsc[j];
         if (a.ifmt == CSA_IFMT_MXFP4) v *= sh.qsc[j * nb + c / 32];
         n2 = fmaf(v, v, n2);
