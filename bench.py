@@ -186,26 +186,35 @@ def run_ours(args, wid):
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
 
-    # per-call events to attribute time to kernels
+    # per-call events to attribute time to the ABI calls (compress / indexer / attention / hca)
     def step_timed(evs):
-        if wid in (1, 4):
-            evs[0].record()
+        p = "h_"
+        evs[0].record()
+        if wid in (1, 3, 4):
             csa.csa_compress(T["Ca"], T["Cb"], T["Za"], T["Zb"], T["Ba"], T["Bb"], T["prev_Cb"], T["prev_Zb"],
                              T["entry0"], T["cache"], m=D["m"])
             evs[1].record()
             csa.lightning_index(T["qI"], T.get("qI_scale"), T["w"], T["kI"], T.get("kI_scale"), T["n_entries"],
                                 T["q_pos"], D["k"], steps._ifmt(D), T["idx"], T["iws"], m=D["m"])
             evs[2].record()
-            csa.sparse_attn_decode(T["q"][:, 0], T["cache"], T["idx"][:, 0], T["win"], T["win_len"], T["sink"],
-                                   D["sm_scale"], D["dv"], T["out"][:, 0], T["lse"][:, 0], T["aws"])
+            if wid == 3:
+                csa.sparse_attn_prefill(T["q"], T["q_pos"], T["cache"], T["idx"], T["raw"], T["raw_pos0"], D["W"],
+                                        T["sink"], D["sm_scale"], D["dv"], T["out"], T["lse"])
+            else:
+                csa.sparse_attn_decode(T["q"][:, 0], T["cache"], T["idx"][:, 0], T["win"], T["win_len"], T["sink"],
+                                       D["sm_scale"], D["dv"], T["out"][:, 0], T["lse"][:, 0], T["aws"])
             evs[3].record()
             if wid == 4:
-                steps.hca_decode_step(T, D, prefix="h_")
+                steps.hca_decode_step(T, D, prefix=p)
             evs[4].record()
         else:
-            evs[0].record()
-            steps.run_step(wl.kind, T, D)
-            evs[1].record(); evs[2].record(); evs[3].record(); evs[4].record()
+            csa.hca_compress(T["C"], T["Z"], T["bias"], T["entry0"], T["cache"], D["m_prime"])
+            evs[1].record()
+            evs[2].record()
+            csa.hca_attn_decode(T["q"][:, 0], T["cache"], T["n_entries"], T["win"], T["win_len"], T["sink"],
+                                D["sm_scale"], D["dv"], T["out"][:, 0], T["lse"][:, 0], T["aws"])
+            evs[3].record()
+            evs[4].record()
 
     def mk():
         return [torch.cuda.Event(enable_timing=True) for _ in range(5)]

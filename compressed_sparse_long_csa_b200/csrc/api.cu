@@ -202,7 +202,7 @@ static int decode_splits(int B, int H, int64_t rows_max) {
 size_t attn_decode_workspace_size(int B, int H, int d_v, int64_t rows_max) {
   if (B < 1 || H < 1 || d_v < 1 || rows_max < 1) return 0;
   const int s = decode_splits(B, H, rows_max);
-  return round_up((size_t)B * s * H * (d_v + 2) * sizeof(float), 256);
+  return round_up((size_t)B * s * H * attn_part_stride(d_v) * sizeof(float), 256);
 }
 
 static csa_status attn_common_checks(const void* q, const void* cache, const void* win, const float* sink, int B,

@@ -111,7 +111,7 @@ attn_cuda_core_kernel(AttnArgs a) {
     }
     if (a.lse && lane == 0) a.lse[(size_t)row * a.H + h] = den > 0.f ? M + logf(den) : -INFINITY;
   } else {
-    float* P = a.part + (((size_t)row * a.splits + split) * a.H + h) * (dv + 2);
+    float* P = a.part + (((size_t)row * a.splits + split) * a.H + h) * attn_part_stride(dv);
 #pragma unroll
     for (int i = 0; i < CC_MAXD / 32; ++i) {
       const int c = lane + 32 * i;
@@ -128,8 +128,8 @@ __global__ void __launch_bounds__(128)
 attn_combine_kernel(AttnArgs a) {
   const int row = blockIdx.x, h = blockIdx.y;
   const int dv = a.dv, S = a.splits;
-  const float* P0 = a.part + ((size_t)row * S * a.H + h) * (dv + 2);
-  const size_t sstride = (size_t)a.H * (dv + 2);
+  const float* P0 = a.part + ((size_t)row * S * a.H + h) * attn_part_stride(dv);
+  const size_t sstride = (size_t)a.H * attn_part_stride(dv);
   const float sk = a.sink[h];
   float M = sk;
   for (int s = 0; s < S; ++s) M = fmaxf(M, P0[s * sstride + dv]);

@@ -23,12 +23,16 @@ struct AttnArgs {
   float sm_scale;
   void* out;                  // [B*Tq, H, dv]
   float* lse;                 // [B*Tq, H] or null
-  float* part;                // split partials [B*Tq, splits, H, dv + 2]
+  float* part;                // split partials [B*Tq, splits, H, attn_part_stride(dv)]
   int splits;
   int rows_per_split;
   int n_seg_a;                // virtual rows in segment A (k or n_max)
   unsigned* err;
 };
+
+// Floats per (query, split, head) record of the split partials: o[dv], m, l, 2 pad,
+// so that every record starts on a 16-byte boundary (vector stores).
+__host__ __device__ inline int attn_part_stride(int dv) { return dv + 4; }
 
 // Number of virtual rows of a query: compressed segment + window segment.
 __host__ __device__ inline int64_t attn_virtual_rows(const AttnArgs& a) { return (int64_t)a.n_seg_a + a.W; }

@@ -422,7 +422,7 @@ attn_tc_kernel(AttnArgs a) {
       }
       if (a.lse && rank == 0) a.lse[(size_t)row * AT_H + h] = den > 0.f ? M + logf(den) : -INFINITY;
     } else {
-      float* P = a.part + (((size_t)row * a.splits + split) * AT_H + h) * (512 + 2);
+      float* P = a.part + (((size_t)row * a.splits + split) * AT_H + h) * attn_part_stride(512);
 #pragma unroll 1
       for (int c = 0; c < AT_VD / 16; ++c) {
         uint32_t v[16];
