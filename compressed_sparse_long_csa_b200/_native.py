@@ -30,6 +30,7 @@ _SIGS = {
     "attn_decode_workspace_size": ([_i32, _i32, _i32, _i64], _sz),
     "sparse_attn_decode": ([_vp] * 6 + [_i32, _i32, _i32, _i32, _i64, _i32, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp], _i32),
     "hca_attn_decode": ([_vp] * 6 + [_i32, _i32, _i32, _i32, _i64, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp], _i32),
+    "sparse_attn_decode_noalloc": ([_vp] * 6 + [_i32, _i32, _i32, _i32, _i64, _i32, _i32, _f32, _i32, _vp, _vp, _vp], _i32),
     "sparse_attn_prefill": ([_vp] * 5 + [_i64, _vp, _vp] + [_i32] * 5 + [_i64, _i32, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp], _i32),
 }
 for _name, (_args, _res) in _SIGS.items():
@@ -142,3 +143,18 @@ def sparse_attn_prefill(q, q_pos, cache, idx, raw, raw_pos0, W, sink, sm_scale, 
     _check(lib.sparse_attn_prefill(_p(q), _p(q_pos), _p(cache), _p(idx), _p(raw), raw.shape[1], _p(raw_pos0),
                                    _p(sink), B, Tq, H, d_k, d_v, cache.shape[1], k, W, sm_scale, _dtype_code(q),
                                    _p(out), _p(lse), wp, wb, _stream(stream)), "sparse_attn_prefill")
+
+
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
+
+
+def sparse_attn_decode_noalloc(q, cache, idx, win, win_len, sink, sm_scale, d_v, out, lse=None, stream=None):
+    """sparse_attn_decode for callers that cannot allocate: the split partials use the
+    library's own fixed device buffer (NOALLOC_SCRATCH_BYTES).  Calls that overlap on
+    the GPU race on that buffer; the first call on a device should precede capture."""
+    B, H, d_k = q.shape
+    W = win.shape[1] if win is not None else 0
+    k = idx.shape[1] if idx is not None else 0
+    _check(lib.sparse_attn_decode_noalloc(_p(q), _p(cache), _p(idx), _p(win), _p(win_len), _p(sink), B, H, d_k,
+                                          d_v, cache.shape[1], k, W, sm_scale, _dtype_code(q), _p(out), _p(lse),
+                                          _stream(stream)), "sparse_attn_decode_noalloc")

@@ -220,6 +220,36 @@ csa_status sparse_attn_prefill(const void* q, const int32_t* q_pos, const void* 
                                int W, float sm_scale, int dtype, void* out, float* lse,
                                void* workspace, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * sparse_attn_decode_noalloc — sparse_attn_decode without a caller workspace.
+ * The paper has no counterpart to this call; it exists for callers that cannot
+ * allocate device memory: code running inside another framework's memory pool,
+ * latency-critical paths that must never call cudaMalloc (which can synchronise
+ * the device), or deployments whose device memory is budgeted up front.
+ *
+ * Arguments, results and rules are those of sparse_attn_decode, minus the
+ * workspace.  The split-KV partials go to a buffer the library owns: a fixed
+ * array of CSA_NOALLOC_SCRATCH_BYTES in device memory, held by every GPU that
+ * loads the library until the process exits.
+ * - Limit: when attn_decode_workspace_size(B, H, d_v, k + W) exceeds
+ *   CSA_NOALLOC_SCRATCH_BYTES the call returns CSA_ERR_WORKSPACE and enqueues
+ *   nothing.  Example: batch 16 with 128 heads, d_v = 512 and k + W = 640 needs
+ *   about 17 MB.
+ * - The first call on each device looks up the buffer's device address
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   before any stream capture.  Later calls only read the cached address.
+ * - All calls on a device share the one buffer, and it keeps the last call's
+ *   contents.  Every call rewrites all it reads, so nothing must be cleared.
+ *   Calls that overlap on the GPU (different streams, or different host threads
+ *   on the same device) race on the buffer: serialise them.
+ * - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ * ------------------------------------------------------------------------- */
+#define CSA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+csa_status sparse_attn_decode_noalloc(const void* q, const void* cache, const int32_t* idx,
+                                      const void* win, const int32_t* win_len, const float* sink,
+                                      int B, int H, int d_k, int d_v, int64_t n_max, int k, int W,
+                                      float sm_scale, int dtype, void* out, float* lse, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
