@@ -128,7 +128,8 @@ static int64_t idx_ld(int64_t n_max) { return (int64_t)round_up((size_t)n_max, 6
 size_t lightning_index_workspace_size(int B, int Tq, int64_t n_max, int k) {
   (void)k;
   if (B < 1 || Tq < 1 || n_max < 1) return 0;
-  return round_up((size_t)B * Tq * idx_ld(n_max) * sizeof(float), 256) + round_up((size_t)B * sizeof(unsigned), 256);
+  return round_up((size_t)B * Tq * idx_ld(n_max) * sizeof(float), 256) + round_up((size_t)B * sizeof(unsigned), 256) +
+         round_up((size_t)B * Tq * 2 * sizeof(unsigned), 256);
 }
 
 csa_status lightning_index(const void* qI, const void* qI_scale, const float* w, const void* kI,
@@ -157,7 +158,9 @@ csa_status lightning_index(const void* qI, const void* qI_scale, const float* w,
   a.scores = (float*)workspace;
   a.knmax = (unsigned*)((char*)workspace + round_up((size_t)B * Tq * a.ld * sizeof(float), 256));
   a.idx_out = idx_out; a.score_out = score_out; a.err = err;
-  cudaError_t e = cudaMemsetAsync(a.knmax, 0, (size_t)B * sizeof(unsigned), S(stream));
+  a.keyrange = a.knmax + round_up((size_t)B * sizeof(unsigned), 256) / sizeof(unsigned);
+  cudaError_t e = cudaMemsetAsync(a.knmax, 0, round_up((size_t)B * sizeof(unsigned), 256) +
+                                  (size_t)B * Tq * 2 * sizeof(unsigned), S(stream));
   if (e != cudaSuccess) return CSA_ERR_CUDA;
   bool used_tc = false;
   if (tc_enabled()) {

@@ -156,9 +156,12 @@ attn_combine_kernel(AttnArgs a) {
 int attn_choose_splits(int n_queries, int H, int64_t rows, bool tc_path) {
   int64_t s;
   if (tc_path) {
-    // one wave of CTA pairs (one CTA per SM): every split re-reads the 147 KB query
-    // from L2, so more splits than SMs cost more than they hide
+    // at most one wave of CTA pairs (one CTA per SM).  Each split also costs a 264 KB
+    // partial (o, m, l of 128 heads) written and read back, and re-reads the 147 KB query
+    // from L2, so a split should cover at least ~5 tiles of 64 rows.
     s = 148 / (2 * (int64_t)n_queries);
+    const int64_t by_rows = rows / 320;
+    if (s > by_rows) s = by_rows;
   } else {
     // aim for >= 2 waves of CTAs on 148 SMs
     const int64_t ctas_per_split = (int64_t)n_queries * ((H + CC_HG - 1) / CC_HG);

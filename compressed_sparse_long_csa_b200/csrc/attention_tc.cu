@@ -56,6 +56,7 @@ struct AtSmem {
   // partial logits received from the peer, double buffered
   alignas(16) float x[2][AT_H][AT_ROWS];
   uint8_t valid[AT_STAGES][AT_ROWS];
+  const __nv_bfloat16* rowp[2][AT_ROWS];   // resolved row pointers of the current / next tile
   alignas(8) uint64_t full[AT_STAGES];
   uint64_t empty[AT_STAGES];
   uint64_t sfull[2];
@@ -67,6 +68,7 @@ struct AtSmem {
   uint64_t qready;
   uint32_t tmem_base;
   int abort_flag;
+  int ld_stop;          // written only by loader threads, read by them after a named barrier
 };
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -172,6 +174,7 @@ attn_tc_kernel(AttnArgs a) {
     tc::mbar_init(&sm.pdone, 1);
     tc::mbar_init(&sm.qready, AT_LOADER_THREADS);
     sm.abort_flag = 0;
+    sm.ld_stop = 0;
     tc::fence_mbar_init();
   }
   if (warp == 1) { tc::tmem_alloc(&sm.tmem_base, TM_COLS); tc::tmem_relinquish(); }
@@ -203,14 +206,28 @@ attn_tc_kernel(AttnArgs a) {
     tc::fence_proxy_async_smem();
     tc::mbar_arrive(&sm.qready);
     bool ok = true;
+    // row pointers are resolved once per tile (one idx lookup per row, in parallel) and
+    // the next tile's are resolved while the current tile's copies are in flight
+    auto resolve = [&](int t, int buf) {
+      if (lt < AT_ROWS) {
+        const int64_t v = v0 + (int64_t)t * AT_ROWS + lt;
+        sm.rowp[buf][lt] = (v < v1) ? attn_row_ptr<__nv_bfloat16>(a, row, (int)v) : nullptr;
+      }
+    };
+    if (n_t > 0) resolve(0, 0);
+    named_bar(1, AT_LOADER_THREADS);
     for (int it = 0; it < n_t; ++it) {
       const int st = it % AT_STAGES;
       const uint32_t ph = (it / AT_STAGES) & 1;
-      if (!tc::mbar_wait(&sm.empty[st], ph ^ 1) || *(volatile int*)&sm.abort_flag) { ok = false; break; }
+      // all loader threads take the same decision: ld_stop is written only by loader
+      // threads before the barrier and read after it
+      const bool go = tc::mbar_wait(&sm.empty[st], ph ^ 1) && !*(volatile int*)&sm.abort_flag;
+      if (!go) sm.ld_stop = 1;
+      named_bar(1, AT_LOADER_THREADS);
+      if (*(volatile int*)&sm.ld_stop) { ok = false; break; }
       for (int p = lt; p < AT_ROWS * AT_CHUNKS; p += AT_LOADER_THREADS) {
         const int j = p / AT_CHUNKS, c = p % AT_CHUNKS;
-        const int64_t v = v0 + (int64_t)it * AT_ROWS + j;
-        const __nv_bfloat16* rp = (v < v1) ? attn_row_ptr<__nv_bfloat16>(a, row, (int)v) : nullptr;
+        const __nv_bfloat16* rp = sm.rowp[it & 1][j];
         if (c == 0) sm.valid[st][j] = rp != nullptr;
         uint32_t dst;
         const __nv_bfloat16* src;
@@ -224,9 +241,11 @@ attn_tc_kernel(AttnArgs a) {
         cp_async16(dst, src, rp != nullptr);
       }
       cp_async_commit();
+      if (it + 1 < n_t) resolve(it + 1, (it + 1) & 1);
       cp_async_wait<0>();
       tc::fence_proxy_async_smem();
       tc::mbar_arrive(&sm.full[st]);
+      named_bar(1, AT_LOADER_THREADS);               // next pointers visible; current buffer free
     }
     if (!ok) atomicExch(&sm.abort_flag, 1);
   } else if (warp == 1) {
@@ -303,13 +322,11 @@ attn_tc_kernel(AttnArgs a) {
       if (!w) { ok = false; break; }
       tc::fence_after_sync();
       float s[AT_ROWS];
+      {
+        uint32_t v[AT_ROWS];
+        tc::tmem_ld64(tmem + lane_base + TM_S + sb * AT_ROWS, v);
 #pragma unroll
-      for (int c = 0; c < AT_ROWS / 16; ++c) {
-        uint32_t v[16];
-        tc::tmem_ld16(tmem + lane_base + TM_S + sb * AT_ROWS + c * 16, v);
-        tc::tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 16; ++j) s[c * 16 + j] = __uint_as_float(v[j]);
+        for (int j = 0; j < AT_ROWS; ++j) s[j] = __uint_as_float(v[j]);
       }
       tc::fence_before_sync();
       __syncwarp();
@@ -359,13 +376,13 @@ attn_tc_kernel(AttnArgs a) {
       if (__any_sync(0xffffffffu, need_rescale)) {
         // O *= alpha for this row (alpha == 1 for lanes that did not need it)
 #pragma unroll 1
-        for (int c = 0; c < AT_VD / 16; ++c) {
-          uint32_t v[16];
-          tc::tmem_ld16(tmem + lane_base + TM_O + c * 16, v);
-          tc::tmem_ld_wait();
+        for (int c = 0; c < AT_VD / 64; ++c) {
+          uint32_t v[64];
+          tc::tmem_ld64(tmem + lane_base + TM_O + c * 64, v);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha);
-          tmem_st16(tmem + lane_base + TM_O + c * 16, v);
+          for (int j = 0; j < 64; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) tmem_st16(tmem + lane_base + TM_O + c * 64 + q * 16, v + q * 16);
         }
         tmem_st_wait();
       }
@@ -407,33 +424,34 @@ attn_tc_kernel(AttnArgs a) {
       const float inv = den > 0.f ? f / den : 0.f;
       __nv_bfloat16* o = (__nv_bfloat16*)a.out + ((size_t)row * AT_H + h) * 512 + dv0;
 #pragma unroll 1
-      for (int c = 0; c < AT_VD / 16; ++c) {
-        uint32_t v[16];
+      for (int c = 0; c < AT_VD / 64; ++c) {
+        uint32_t v[64];
         if (ok && n_t > 0) {
-          tc::tmem_ld16(tmem + lane_base + TM_O + c * 16, v);
-          tc::tmem_ld_wait();
+          tc::tmem_ld64(tmem + lane_base + TM_O + c * 64, v);
         } else {
-          for (int j = 0; j < 16; ++j) v[j] = 0u;
+          for (int j = 0; j < 64; ++j) v[j] = 0u;
         }
-        float f16v[16];
-        for (int j = 0; j < 16; ++j) f16v[j] = __uint_as_float(v[j]) * inv;
-        Elem<__nv_bfloat16>::st_vec(o + c * 16, f16v);
-        Elem<__nv_bfloat16>::st_vec(o + c * 16 + 8, f16v + 8);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          float f8[8];
+          for (int j = 0; j < 8; ++j) f8[j] = __uint_as_float(v[q * 8 + j]) * inv;
+          Elem<__nv_bfloat16>::st_vec(o + c * 64 + q * 8, f8);
+        }
       }
       if (a.lse && rank == 0) a.lse[(size_t)row * AT_H + h] = den > 0.f ? M + logf(den) : -INFINITY;
     } else {
       float* P = a.part + (((size_t)row * a.splits + split) * AT_H + h) * attn_part_stride(512);
 #pragma unroll 1
-      for (int c = 0; c < AT_VD / 16; ++c) {
-        uint32_t v[16];
+      for (int c = 0; c < AT_VD / 64; ++c) {
+        uint32_t v[64];
         if (ok && n_t > 0) {
-          tc::tmem_ld16(tmem + lane_base + TM_O + c * 16, v);
-          tc::tmem_ld_wait();
+          tc::tmem_ld64(tmem + lane_base + TM_O + c * 64, v);
         } else {
-          for (int j = 0; j < 16; ++j) v[j] = 0u;
+          for (int j = 0; j < 64; ++j) v[j] = 0u;
         }
-        float4* d4 = reinterpret_cast<float4*>(P + dv0 + c * 16);
-        for (int j = 0; j < 4; ++j)
+        float4* d4 = reinterpret_cast<float4*>(P + dv0 + c * 64);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
           d4[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]), __uint_as_float(v[4 * j + 2]),
                               __uint_as_float(v[4 * j + 3]));
       }

@@ -91,6 +91,73 @@ csa_compress_kernel(const T* __restrict__ Ca, const T* __restrict__ Cb, const T*
   Elem<T>::st_vec(cache + ((size_t)b * n_max + e) * d + c0, out);
 }
 
+// m = 4 (the CSA rate): all 16 source vectors and 8 bias vectors of a thread are
+// loaded before any arithmetic, so a thread waits for one memory round trip instead
+// of one per source.
+template <typename T>
+__global__ void __launch_bounds__(256)
+csa_compress_m4_kernel(const T* __restrict__ Ca, const T* __restrict__ Cb, const T* __restrict__ Za,
+                       const T* __restrict__ Zb, const float* __restrict__ Ba, const float* __restrict__ Bb,
+                       const T* __restrict__ pCb, const T* __restrict__ pZb, const int32_t* __restrict__ entry0,
+                       T* __restrict__ cache, int64_t n_max, int T_new, int d, unsigned* err) {
+  constexpr int VEC = Elem<T>::VEC;
+  constexpr int M = 4;
+  const int b = blockIdx.y;
+  const int groups = d / VEC;
+  const int n_blk = T_new / M;
+  const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= (int64_t)n_blk * groups) return;
+  const int j = (int)(gid / groups);
+  const int c0 = (int)(gid % groups) * VEC;
+  const int e = entry0[b] + j;
+  if (e < 0 || (int64_t)e >= n_max) { raise_err(err, CSA_DEVERR_ENTRY); return; }
+  const size_t seq = (size_t)b * T_new * d;
+  float c[2 * M][VEC], z[2 * M][VEC], bias[2 * M][VEC];
+  const bool has_b = e > 0;
+#pragma unroll
+  for (int t = 0; t < M; ++t) {
+    const T *cp, *zp;
+    if (j > 0) {
+      const size_t off = seq + (size_t)((j - 1) * M + t) * d + c0;
+      cp = Cb + off; zp = Zb + off;
+    } else {
+      const size_t off = ((size_t)b * M + t) * d + c0;
+      cp = pCb + off; zp = pZb + off;
+    }
+    if (has_b) { Elem<T>::ld_vec(cp, c[t]); Elem<T>::ld_vec(zp, z[t]); }
+    const size_t off = seq + (size_t)(j * M + t) * d + c0;
+    Elem<T>::ld_vec(Ca + off, c[M + t]);
+    Elem<T>::ld_vec(Za + off, z[M + t]);
+    const float4* bb = reinterpret_cast<const float4*>(Bb + t * d + c0);
+    const float4* ba = reinterpret_cast<const float4*>(Ba + t * d + c0);
+#pragma unroll
+    for (int q = 0; q < VEC / 4; ++q) {
+      const float4 x = bb[q], y = ba[q];
+      bias[t][4 * q] = x.x; bias[t][4 * q + 1] = x.y; bias[t][4 * q + 2] = x.z; bias[t][4 * q + 3] = x.w;
+      bias[M + t][4 * q] = y.x; bias[M + t][4 * q + 1] = y.y; bias[M + t][4 * q + 2] = y.z; bias[M + t][4 * q + 3] = y.w;
+    }
+  }
+  float out[VEC];
+#pragma unroll
+  for (int i = 0; i < VEC; ++i) {
+    float mx = -INFINITY;
+#pragma unroll
+    for (int t = 0; t < 2 * M; ++t)
+      if (has_b || t >= M) mx = fmaxf(mx, z[t][i] + bias[t][i]);
+    float S = 0.f, A = 0.f;
+#pragma unroll
+    for (int t = 0; t < 2 * M; ++t) {
+      if (has_b || t >= M) {
+        const float w = __expf(z[t][i] + bias[t][i] - mx);
+        S += w;
+        A = fmaf(w, c[t][i], A);
+      }
+    }
+    out[i] = A / S;
+  }
+  Elem<T>::st_vec(cache + ((size_t)b * n_max + e) * d + c0, out);
+}
+
 // One CTA per (entry, slab of 8*VEC components, batch): 8 component groups x 32 token lanes.
 // Each thread pools tokens tl, tl+32, ... of its group; the 32 partial (M, S, A) are merged
 // in shared memory.
@@ -158,6 +225,24 @@ cudaError_t launch_csa_compress(const void* Ca, const void* Cb, const void* Za, 
                                 const int32_t* entry0, void* cache, int64_t n_max, int B, int T_new,
                                 int d, int m, int dtype, cudaStream_t st, unsigned* err) {
   const int n_blk = T_new / m;
+  if (m == 4) {
+    const int vec = dtype == CSA_BF16 ? 8 : 4;
+    const int64_t work = (int64_t)n_blk * (d / vec);
+    const int threads = work < 256 ? (int)((work + 31) / 32 * 32) : 256;
+    dim3 grid((unsigned)((work + threads - 1) / threads), B);
+    if (dtype == CSA_BF16) {
+      using T = __nv_bfloat16;
+      csa_compress_m4_kernel<T><<<grid, threads, 0, st>>>((const T*)Ca, (const T*)Cb, (const T*)Za, (const T*)Zb, Ba,
+                                                          Bb, (const T*)pCb, (const T*)pZb, entry0, (T*)cache, n_max,
+                                                          T_new, d, err);
+    } else {
+      csa_compress_m4_kernel<float><<<grid, threads, 0, st>>>((const float*)Ca, (const float*)Cb, (const float*)Za,
+                                                              (const float*)Zb, Ba, Bb, (const float*)pCb,
+                                                              (const float*)pZb, entry0, (float*)cache, n_max, T_new,
+                                                              d, err);
+    }
+    return cudaGetLastError();
+  }
   if (dtype == CSA_BF16) {
     using T = __nv_bfloat16;
     const int64_t work = (int64_t)n_blk * (d / 8);

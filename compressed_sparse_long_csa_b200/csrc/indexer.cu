@@ -74,8 +74,8 @@ indexer_scores_cuda_core(IndexerArgs a) {
   __syncthreads();
 
   const int r = threadIdx.x;
-  if (r >= ntile) return;
-  const int s = s0 + r;
+  const bool has = r < ntile;
+  const int s = s0 + (has ? r : 0);
   const size_t koff = (size_t)b * a.n_max + s;
   const float* kr = ks + r * (dI + 1);
   float kscale = 1.f;
@@ -92,7 +92,7 @@ indexer_scores_cuda_core(IndexerArgs a) {
     if (a.ifmt == CSA_IFMT_MXFP4) v *= kblk[c / 32];
     kn2 = fmaf(v, v, kn2);
   }
-  atomicMax(a.knmax + b, __float_as_uint(sqrtf(kn2) * 1.0001f));
+  if (has) atomicMax(a.knmax + b, __float_as_uint(sqrtf(kn2) * 1.0001f));
 
   float score = 0.f;
   for (int j = 0; j < HI; ++j) {
@@ -112,7 +112,8 @@ indexer_scores_cuda_core(IndexerArgs a) {
     }
     score = fmaf(wsh[j], fmaxf(D, 0.f), score);
   }
-  a.scores[(size_t)row * a.ld + s] = score;
+  if (has) a.scores[(size_t)row * a.ld + s] = score;
+  record_key_range(a.keyrange, row, score, has);
 }
 
 cudaError_t launch_indexer_scores_cuda_core(const IndexerArgs& a, cudaStream_t st) {

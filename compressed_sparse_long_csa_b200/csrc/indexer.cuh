@@ -20,6 +20,7 @@ struct IndexerArgs {
   float* scores;              // workspace [B*Tq, ld] fp32 scores
   int64_t ld;
   unsigned* knmax;            // workspace [B]: bits of max_s ||k_s||_2 (dequantised)
+  unsigned* keyrange;         // workspace [B*Tq][2]: max order key, max of ~order key (= ~min) of the row's scores
   int32_t* idx_out;           // [B*Tq, k]
   float* score_out;           // [B*Tq, k] or null
   unsigned* err;
@@ -35,6 +36,19 @@ __device__ __forceinline__ int row_eligible(const IndexerArgs& a, int row) {
   if ((int64_t)n > a.n_max) n = (int)a.n_max;
   if (n < 0) n = 0;
   return ne < n ? ne : n;
+}
+
+// Record the order-key range of a warp's scores for `row` (one atomic pair per warp).
+// Lanes without a score pass valid = false.  All 32 lanes must call.
+__device__ __forceinline__ void record_key_range(unsigned* keyrange, int row, float score, bool valid) {
+  const uint32_t key = f32_order_key(score);
+  const uint32_t mx = __reduce_max_sync(0xffffffffu, valid ? key : 0u);
+  const uint32_t mn = __reduce_max_sync(0xffffffffu, valid ? ~key : 0u);
+  const bool any = __any_sync(0xffffffffu, valid);
+  if (any && (threadIdx.x & 31) == 0) {
+    atomicMax(keyrange + 2 * (size_t)row, mx);
+    atomicMax(keyrange + 2 * (size_t)row + 1, mn);
+  }
 }
 
 cudaError_t launch_indexer_scores_cuda_core(const IndexerArgs& a, cudaStream_t st);

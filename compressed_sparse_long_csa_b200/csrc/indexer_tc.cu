@@ -55,7 +55,7 @@ struct IdxSmem {
 };
 
 template <int G, int STAGES>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(256, G == 1 ? 2 : 1)
 indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ, IdxTcParams p) {
   extern __shared__ uint8_t smem_raw[];
   using Sm = IdxSmem<G, STAGES>;
@@ -160,30 +160,35 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     const int r = quarter * 32 + lane;
     const float* kscale = (const float*)a.kI_scale;
     float kmax = 0.f;
+    // the key scale of the next tile is loaded before waiting for the current accumulator
+    auto load_scale = [&](int it) {
+      const int s = (t_begin + it) * IT_ROWS + r;
+      return (it < n_t && s < a.n_max) ? __ldg(kscale + (size_t)b * a.n_max + s) : 0.f;
+    };
+    float sk_next = load_scale(0);
     for (int it = 0; it < n_t; ++it) {
       const int acc = it & 1;
       const uint32_t aph = (it >> 1) & 1;
+      const float sk = sk_next;
+      sk_next = load_scale(it + 1);
       bool ok = tc::mbar_wait(&sm.tfull[acc], aph) && !*(volatile int*)&sm.abort_flag;
       ok = __all_sync(0xffffffffu, ok);               // the TMEM loads below are warp-collective
       if (!ok) { atomicExch(&sm.abort_flag, 1); break; }
       tc::fence_after_sync();
       const int s = (t_begin + it) * IT_ROWS + r;
-      const float sk = (s < a.n_max) ? kscale[(size_t)b * a.n_max + s] : 0.f;
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         float val = 0.f;
+        uint32_t v[64];
+        tc::tmem_ld64(tmem + ((uint32_t)(quarter * 32) << 16) + acc * N + g * 64, v);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t v[16];
-          tc::tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + acc * N + g * 64 + c * 16, v);
-          tc::tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) val = fmaf(sm.wq[g][c * 16 + j], fmaxf(__uint_as_float(v[j]), 0.f), val);
-        }
-        if (s < sm.n_elig[g]) {
+        for (int j = 0; j < 64; ++j) val = fmaf(sm.wq[g][j], fmaxf(__uint_as_float(v[j]), 0.f), val);
+        const bool valid = s < sm.n_elig[g];
+        if (valid) {
           a.scores[(size_t)sm.row[g] * a.ld + s] = val * sk;
           kmax = fmaxf(kmax, sk);
         }
+        record_key_range(a.keyrange, sm.row[g], val * sk, valid);
       }
       tc::fence_before_sync();
       __syncwarp();
@@ -199,6 +204,204 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
   if (warp == 1) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, NCOLS);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// MXFP4 operands ("FP4 с учётом квантования": the indexer's Q·K path in FP4).  Same
+// structure as the E4M3 kernel, with the native block-scaled MMA: packed e2m1 key tiles
+// (64-byte rows, 64-byte swizzle) and one ue8m0 scale per 32 elements applied inside the
+// tensor core.  The scale factors go to TMEM with tcgen05.st: for M rows, row m's four
+// scale bytes (k-blocks 0..3) sit in 32-bit column m/32 of lane m%32, replicated in all
+// four lane quarters; warps 8..11 (one per quarter) write them for every tile.  Each tile
+// is two MMAs of K = 64 (k-blocks 0-1, then 2-3: scale byte 0, then byte 2).
+constexpr int MX_KB = 64;                 // bytes per packed key row (128 e2m1)
+constexpr int MX_TILE_BYTES = IT_ROWS * MX_KB;
+
+template <int STAGES>
+struct MxSmem {
+  alignas(1024) uint8_t q[64 * MX_KB];
+  alignas(1024) uint8_t k[STAGES][MX_TILE_BYTES];
+  alignas(8) uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t sfa_full[STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t qfull;
+  uint64_t sfb_ready;
+  uint32_t tmem_base;
+  int abort_flag;
+  int t_begin, t_end;
+  int n_elig;
+  float w[64];
+};
+
+// TMEM columns: two accumulators [0, 128), q scales at 128, key-scale ring at 136 + 4 * stage
+constexpr uint32_t MX_SFB = 128, MX_SFA = 136, MX_COLS = 256;
+
+template <int STAGES>
+__global__ void __launch_bounds__(384, 1)
+indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ, IdxTcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  using Sm = MxSmem<STAGES>;
+  Sm& sm = *reinterpret_cast<Sm*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const IndexerArgs& a = p.a;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.x, t = blockIdx.y, b = blockIdx.z;     // one query per CTA
+  const int row = b * a.Tq + t;
+  constexpr int N = 64;
+  const uint32_t* ksc = (const uint32_t*)a.kI_scale;                  // 4 ue8m0 bytes per entry
+  const uint32_t* qsc = (const uint32_t*)a.qI_scale;                  // 4 ue8m0 bytes per head
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      tc::mbar_init(&sm.full[s], 1); tc::mbar_init(&sm.empty[s], 1); tc::mbar_init(&sm.sfa_full[s], 4);
+    }
+    for (int s = 0; s < 2; ++s) { tc::mbar_init(&sm.tfull[s], 1); tc::mbar_init(&sm.tempty[s], 4); }
+    tc::mbar_init(&sm.qfull, 1);
+    tc::mbar_init(&sm.sfb_ready, 4);
+    tc::fence_mbar_init();
+    sm.abort_flag = 0;
+    const int ne = row_eligible(a, row);
+    sm.n_elig = ne;
+    const int t_lim = (ne + IT_ROWS - 1) / IT_ROWS;
+    int t0 = split * p.tiles_per_split, t1 = t0 + p.tiles_per_split;
+    if (t1 > t_lim) t1 = t_lim;
+    sm.t_begin = t0;
+    sm.t_end = t1 > t0 ? t1 : t0;
+  }
+  if (threadIdx.x < 64) sm.w[threadIdx.x] = threadIdx.x < a.H_I ? a.w[(size_t)row * a.H_I + threadIdx.x] : 0.f;
+  if (warp == 1) { tc::tmem_alloc(&sm.tmem_base, MX_COLS); tc::tmem_relinquish(); }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = sm.tmem_base;
+  const int t_begin = sm.t_begin, n_t = sm.t_end - sm.t_begin;
+
+  if (warp == 0) {
+    if (lane == 0 && n_t > 0) {
+      tc::prefetch_tmap(&tmK);
+      tc::prefetch_tmap(&tmQ);
+      tc::mbar_arrive_expect_tx(&sm.qfull, 64 * MX_KB);
+      tc::tma_load_2d(sm.q, &tmQ, &sm.qfull, 0, row * 64);
+      int issued = 0;
+      for (int it = 0; it < n_t; ++it) {
+        const int st = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (!tc::mbar_wait(&sm.empty[st], ph ^ 1)) { atomicExch(&sm.abort_flag, 1); break; }
+        if (*(volatile int*)&sm.abort_flag) break;
+        tc::mbar_arrive_expect_tx(&sm.full[st], MX_TILE_BYTES);
+        tc::tma_load_2d(sm.k[st], &tmK, &sm.full[st], 0, (int)(b * a.n_max) + (t_begin + it) * IT_ROWS);
+        ++issued;
+      }
+      tc::mbar_wait(&sm.qfull, 0);
+      for (int it = (issued > STAGES ? issued - STAGES : 0); it < issued; ++it)
+        tc::mbar_wait(&sm.full[it % STAGES], (it / STAGES) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && n_t > 0) {
+      constexpr uint32_t ID0 = tc::idesc_mxf4(IT_ROWS, N, 0, 0);
+      constexpr uint32_t ID1 = tc::idesc_mxf4(IT_ROWS, N, 2, 2);
+      bool ok = tc::mbar_wait(&sm.qfull, 0) && tc::mbar_wait(&sm.sfb_ready, 0);
+      int last_issued = -1;
+      const uint32_t q_addr = tc::smem_u32(sm.q);
+      for (int it = 0; ok && it < n_t; ++it) {
+        const int st = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        const int acc = it & 1;
+        const uint32_t aph = (it >> 1) & 1;
+        if (!tc::mbar_wait(&sm.tempty[acc], aph ^ 1) || !tc::mbar_wait(&sm.full[st], ph) ||
+            !tc::mbar_wait(&sm.sfa_full[st], ph) || *(volatile int*)&sm.abort_flag) { ok = false; break; }
+        tc::fence_after_sync();
+        const uint32_t k_addr = tc::smem_u32(sm.k[st]);
+        const uint32_t sfa = tmem + MX_SFA + 4 * st, sfb = tmem + MX_SFB;
+        tc::mma_mxf4(tmem + acc * N, tc::desc_k_sw64(k_addr), tc::desc_k_sw64(q_addr), ID0, sfa, sfb, 0u);
+        tc::mma_mxf4(tmem + acc * N, tc::desc_k_sw64(k_addr + 32), tc::desc_k_sw64(q_addr + 32), ID1, sfa, sfb, 1u);
+        tc::mma_commit(&sm.empty[st]);
+        tc::mma_commit(&sm.tfull[acc]);
+        last_issued = it;
+      }
+      if (!ok) {
+        atomicExch(&sm.abort_flag, 1);
+        if (last_issued >= 0) tc::mbar_wait(&sm.tfull[last_issued & 1], (last_issued >> 1) & 1);
+      }
+    }
+  } else if (warp >= 8) {
+    // scale-factor writers, one warp per lane quarter (all quarters hold the same data)
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    if (n_t > 0) {
+      // query scales: heads lane and lane + 32
+      tc::tmem_st2(tmem + lane_base + MX_SFB, __ldg(qsc + (size_t)row * 64 + lane), __ldg(qsc + (size_t)row * 64 + 32 + lane));
+      tc::tmem_st_wait();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&sm.sfb_ready);
+    }
+    auto load4 = [&](int it, uint32_t* v) {
+      const int s0 = (t_begin + it) * IT_ROWS + lane;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int s = s0 + 32 * c;
+        v[c] = (it < n_t && s < a.n_max) ? __ldg(ksc + (size_t)b * a.n_max + s) : 0u;
+      }
+    };
+    uint32_t nxt[4];
+    load4(0, nxt);
+    for (int it = 0; it < n_t; ++it) {
+      const int st = it % STAGES;
+      const uint32_t ph = (it / STAGES) & 1;
+      uint32_t cur[4] = {nxt[0], nxt[1], nxt[2], nxt[3]};
+      load4(it + 1, nxt);
+      bool ok = tc::mbar_wait(&sm.empty[st], ph ^ 1) && !*(volatile int*)&sm.abort_flag;
+      if (!__all_sync(0xffffffffu, ok)) { atomicExch(&sm.abort_flag, 1); break; }
+      tc::fence_after_sync();
+      tc::tmem_st4(tmem + lane_base + MX_SFA + 4 * st, cur[0], cur[1], cur[2], cur[3]);
+      tc::tmem_st_wait();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&sm.sfa_full[st]);
+    }
+  } else if (warp >= 4) {
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    float kb = 0.f;
+    for (int it = 0; it < n_t; ++it) {
+      const int acc = it & 1;
+      const uint32_t aph = (it >> 1) & 1;
+      const int s = (t_begin + it) * IT_ROWS + r;
+      const bool valid = s < sm.n_elig;
+      // ||k_s|| <= 6 * sqrt(32 * sum_b scale_b^2): |e2m1| <= 6
+      if (valid) {
+        const uint32_t sc = __ldg(ksc + (size_t)b * a.n_max + s);
+        float ss = 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) { const float f = ue8m0_to_float((sc >> (8 * q)) & 0xFFu); ss = fmaf(f, f, ss); }
+        kb = fmaxf(kb, 6.f * sqrtf(32.f * ss));
+      }
+      bool ok = tc::mbar_wait(&sm.tfull[acc], aph) && !*(volatile int*)&sm.abort_flag;
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) { atomicExch(&sm.abort_flag, 1); break; }
+      tc::fence_after_sync();
+      float val = 0.f;
+      uint32_t v[64];
+      tc::tmem_ld64(tmem + ((uint32_t)(quarter * 32) << 16) + acc * N, v);
+#pragma unroll
+      for (int j = 0; j < 64; ++j) val = fmaf(sm.w[j], fmaxf(__uint_as_float(v[j]), 0.f), val);
+      if (valid) a.scores[(size_t)row * a.ld + s] = val;
+      record_key_range(a.keyrange, row, val, valid);
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&sm.tempty[acc]);
+    }
+    kb = warp_max(kb);
+    if (lane == 0 && kb > 0.f) atomicMax(a.knmax + b, __float_as_uint(kb * 1.0001f));
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (sm.abort_flag && threadIdx.x == 0) raise_err(a.err, CSA_DEVERR_TIMEOUT);
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, MX_COLS);
   }
 }
 
@@ -228,15 +431,56 @@ bool make_map_rows128(CUtensorMap* m, const void* base, uint64_t rows, uint32_t 
   return r == CUDA_SUCCESS;
 }
 
+// 2D byte tensor: rows of 64 bytes, box = box_rows x 64 bytes, 64-byte swizzle.
+bool make_map_rows64(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {64, rows};
+  cuuint64_t strides[1] = {64};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+cudaError_t launch_mxf4(const IndexerArgs& a, cudaStream_t st, bool* used) {
+  constexpr int STAGES = 8;
+  IdxTcParams p{};
+  p.a = a;
+  p.n_qg = a.Tq;
+  p.tiles = (int)((a.n_max + IT_ROWS - 1) / IT_ROWS);
+  const int64_t ctas = (int64_t)a.B * a.Tq;
+  int splits = (int)((148 + ctas - 1) / ctas);
+  if (splits > p.tiles) splits = p.tiles;
+  if (splits < 1) splits = 1;
+  p.tiles_per_split = (p.tiles + splits - 1) / splits;
+  splits = (p.tiles + p.tiles_per_split - 1) / p.tiles_per_split;
+  CUtensorMap mk, mq;
+  if (!make_map_rows64(&mk, a.kI, (uint64_t)a.B * a.n_max, IT_ROWS)) return cudaSuccess;
+  if (!make_map_rows64(&mq, a.qI, (uint64_t)a.B * a.Tq * 64, 64)) return cudaSuccess;
+  const size_t smem = sizeof(MxSmem<STAGES>) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(indexer_mxf4_kernel<STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(splits, a.Tq, a.B);
+  indexer_mxf4_kernel<STAGES><<<grid, 384, smem, st>>>(mk, mq, p);
+  *used = true;
+  return cudaGetLastError();
+}
+
 template <int G, int STAGES>
 cudaError_t launch_g(const IndexerArgs& a, cudaStream_t st, bool* used) {
   IdxTcParams p{};
   p.a = a;
   p.n_qg = (a.Tq + G - 1) / G;
   p.tiles = (int)((a.n_max + IT_ROWS - 1) / IT_ROWS);
-  // decode-like shapes: split the entry tiles so that the grid covers the 148 SMs
+  // decode-like shapes: split the entry tiles so that the grid fills the SMs once
+  // (two CTAs per SM for the one-query variant, one for the four-query variant)
   const int64_t ctas = (int64_t)a.B * p.n_qg;
-  int splits = (int)((148 + ctas - 1) / ctas);
+  const int64_t slots = G == 1 ? 2 * 148 : 148;
+  int splits = (int)(slots / ctas);
   if (splits > p.tiles) splits = p.tiles;
   if (splits < 1) splits = 1;
   p.tiles_per_split = (p.tiles + splits - 1) / splits;
@@ -260,6 +504,14 @@ cudaError_t launch_g(const IndexerArgs& a, cudaStream_t st, bool* used) {
 // return *used = false and run on the CUDA-core path.
 cudaError_t launch_indexer_scores_tc(const IndexerArgs& a, cudaStream_t st, bool* used) {
   *used = false;
+  if (a.ifmt == CSA_IFMT_MXFP4 && a.H_I == 64 && a.d_I == 128) {
+    if (((uintptr_t)a.kI & 15) || ((uintptr_t)a.qI & 15) || ((uintptr_t)a.kI_scale & 3) || ((uintptr_t)a.qI_scale & 3))
+      return cudaSuccess;
+    if ((int64_t)a.B * a.n_max > 0x7fffffffLL || (int64_t)a.B * a.Tq * 64 > 0x7fffffffLL) return cudaSuccess;
+    // same bound as the E4M3 kernel: twice the worst case of a 128-term fp32 accumulation
+    const_cast<IndexerArgs&>(a).eps_dot = 1.0f / 65536.0f;
+    return launch_mxf4(a, st, used);
+  }
   if (a.ifmt != CSA_IFMT_E4M3 || a.H_I != 64 || a.d_I != 128) return cudaSuccess;
   if (((uintptr_t)a.kI & 15) || ((uintptr_t)a.qI & 15)) return cudaSuccess;
   if ((int64_t)a.B * a.n_max > 0x7fffffffLL || (int64_t)a.B * a.Tq * 64 > 0x7fffffffLL) return cudaSuccess;
@@ -268,7 +520,7 @@ cudaError_t launch_indexer_scores_tc(const IndexerArgs& a, cudaStream_t st, bool
   // bound's scale (test_indexer_fp32_score_error_within_band_bound).
   const_cast<IndexerArgs&>(a).eps_dot = 1.0f / 65536.0f;
   if (a.Tq >= 4) return launch_g<4, 6>(a, st, used);
-  return launch_g<1, 8>(a, st, used);
+  return launch_g<1, 6>(a, st, used);
 }
 
 }  // namespace csa

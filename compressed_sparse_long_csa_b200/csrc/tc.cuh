@@ -106,6 +106,14 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {
       : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// 64 consecutive columns: four loads issued back to back, one wait
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t* r) {
+  tmem_ld16(taddr, r);
+  tmem_ld16(taddr + 16, r + 16);
+  tmem_ld16(taddr + 32, r + 32);
+  tmem_ld16(taddr + 48, r + 48);
+  tmem_ld_wait();
+}
 
 // ---------------------------------------------------------------- descriptors
 // Shared-memory matrix descriptor, K-major operand with the 128-byte swizzle:
@@ -132,6 +140,48 @@ __device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t smem_addr, uint32_t l
   d |= (uint64_t)2u << 61;
   return d;
 }
+// K-major operand with the 64-byte swizzle: rows of 64 bytes, 8-row groups 512 bytes apart.
+__device__ __forceinline__ uint64_t desc_k_sw64(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;
+  d |= (uint64_t)(512u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)4u << 61;                        // SWIZZLE_64B
+  return d;
+}
+
+// 32 lanes x 32-bit, 2 / 4 consecutive columns from registers
+__device__ __forceinline__ void tmem_st2(uint32_t taddr, uint32_t a, uint32_t b) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1, %2};" ::"r"(taddr), "r"(a), "r"(b) : "memory");
+}
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(a), "r"(b), "r"(c),
+               "r"(d) : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// D[tmem] (+)= (A x 2^sfa) * (B x 2^sfb)^T, MXFP4 operands (packed e2m1, ue8m0 scale per 32
+// elements along K), K = 64 per instruction; scale factors are read from TMEM.
+__device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+// Block-scaled instruction descriptor: E2M1 x E2M1, UE8M0 scales, K-major, D f32,
+// sf_id = byte of the 32-bit scale column used for this instruction's first 32-block.
+__host__ __device__ constexpr uint32_t idesc_mxf4(uint32_t M, uint32_t N, uint32_t a_sf_id, uint32_t b_sf_id) {
+  return (b_sf_id << 4)
+       | (1u << 7) | (1u << 10)          // A, B format E2M1
+       | ((N >> 3) << 17)
+       | (1u << 23)                      // scale format UE8M0
+       | ((M >> 4) << 24)
+       | (a_sf_id << 29);
+}
+
 // Instruction descriptor: D f32, A/B formats, K-major unless stated, M and N.
 __host__ __device__ constexpr uint32_t idesc(uint32_t a_fmt, uint32_t b_fmt, uint32_t M, uint32_t N,
                                              uint32_t a_mn_major = 0, uint32_t b_mn_major = 0) {

@@ -24,8 +24,10 @@ constexpr int TK_THREADS = 1024;
 constexpr int TK_KMAX = 2048;
 constexpr int AMB_CAP = 2048;
 
+constexpr int HB = 2048;          // histogram bins of the range-aware select (11-bit digits)
+
 struct TopkShared {
-  uint32_t hist[256];
+  uint32_t hist[HB];
   uint32_t wtot[32];
   int32_t sel[TK_KMAX];
   int32_t amb[AMB_CAP];
@@ -36,6 +38,7 @@ struct TopkShared {
   float qsc[64 * 4];
   float w[64];
   uint32_t digit, remaining, n_sel, n_amb;
+  uint32_t hT, hcgt, hcT, kmax_s, kmin_s;
   float U;
 };
 
@@ -54,6 +57,88 @@ __device__ __forceinline__ int block_excl_scan_flag(bool f, uint32_t* wtot, int*
   __syncthreads();
   *total = tot;
   return wpre + pre;
+}
+
+// Histogram select over the range of the keys.  All keys share the bits above the
+// highest bit h where kmin and kmax differ, so the digit is bits [lo, h] of the key
+// (lo = max(0, h-10)): at most 2048 bins, spread over the keys' actual range.  Bins
+// are counted with warp-aggregated shared-memory atomics.  Returns the bin T that
+// holds the k-th largest key: key_lo..key_hi are the bin's key bounds, *c_gt the
+// number of keys above the bin and *c_T the number inside it.
+struct BinSel {
+  uint32_t key_lo, key_hi;
+  int c_gt, c_T;
+  bool exact;                     // every key of the bin is the same key
+};
+
+template <typename KeyFn>
+__device__ BinSel hist_select(TopkShared& sh, int n, int k, KeyFn key, uint32_t kmin, uint32_t kmax) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  BinSel r;
+  const uint32_t diff = kmin ^ kmax;
+  if (diff == 0u) {
+    r.key_lo = r.key_hi = kmax; r.c_gt = 0; r.c_T = n; r.exact = true;
+    return r;
+  }
+  const int h = 31 - __clz(diff);
+  const int lo = h >= 10 ? h - 10 : 0;
+  const uint32_t nbm = (1u << (h - lo + 1)) - 1u;
+  for (int i = tid; i < HB; i += blockDim.x) sh.hist[i] = 0u;
+  __syncthreads();
+  const int iters = (n + (int)blockDim.x - 1) / (int)blockDim.x;
+  for (int it = 0; it < iters; ++it) {
+    const int i = it * blockDim.x + tid;
+    const uint32_t dg = i < n ? (key(i) >> lo) & nbm : 0xFFFFFFFFu;
+    const unsigned peers = __match_any_sync(0xffffffffu, dg);
+    if (dg != 0xFFFFFFFFu && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[dg], (uint32_t)__popc(peers));
+  }
+  __syncthreads();
+  // suffix sums over bins: thread t owns bins 2t (lower) and 2t+1 (upper)
+  const uint32_t b0 = sh.hist[2 * tid], b1 = sh.hist[2 * tid + 1];
+  uint32_t v = b0 + b1;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t x = __shfl_down_sync(0xffffffffu, v, o);
+    if (lane + o < 32) v += x;
+  }
+  if (lane == 0) sh.wtot[warp] = v;                 // warp total (suffix from lane 0)
+  __syncthreads();
+  uint32_t above_w = 0;
+  for (int w = warp + 1; w < (int)(blockDim.x >> 5); ++w) above_w += sh.wtot[w];
+  const uint32_t after = v - (b0 + b1) + above_w;  // keys in bins above this thread's pair
+  const uint32_t kk = (uint32_t)k;
+  if (after < kk && kk <= after + b1) { sh.hT = 2 * tid + 1; sh.hcgt = after; sh.hcT = b1; }
+  if (after + b1 < kk && kk <= after + b1 + b0) { sh.hT = 2 * tid; sh.hcgt = after + b1; sh.hcT = b0; }
+  __syncthreads();
+  const uint32_t T = sh.hT;
+  const uint32_t pre = (h + 1 >= 32) ? 0u : (kmax & ~((2u << h) - 1u));
+  r.key_lo = pre | (T << lo);
+  r.key_hi = r.key_lo | ((1u << lo) - 1u);
+  r.c_gt = (int)sh.hcgt;
+  r.c_T = (int)sh.hcT;
+  r.exact = lo == 0;
+  __syncthreads();
+  return r;
+}
+
+// Block min / max of the keys.
+template <typename KeyFn>
+__device__ void key_range(TopkShared& sh, int n, KeyFn key, uint32_t* kmin, uint32_t* kmax) {
+  uint32_t mx = 0u, mn = 0xFFFFFFFFu;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const uint32_t x = key(i);
+    mx = max(mx, x);
+    mn = min(mn, x);
+  }
+  mx = __reduce_max_sync(0xffffffffu, mx);
+  mn = __reduce_min_sync(0xffffffffu, mn);
+  if (threadIdx.x == 0) { sh.kmax_s = 0u; sh.kmin_s = 0xFFFFFFFFu; }
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) { atomicMax(&sh.kmax_s, mx); atomicMin(&sh.kmin_s, mn); }
+  __syncthreads();
+  *kmin = sh.kmin_s;
+  *kmax = sh.kmax_s;
+  __syncthreads();
 }
 
 // Radix select: the k-th largest key among key(0..n-1).  Returns tau; *remaining =
@@ -131,6 +216,72 @@ __device__ void write_sorted(TopkShared& sh, int cnt, int k, int32_t* out) {
 }
 
 // ------------------------------------------------------------------ topk_select (fp32 keys)
+// Exact top-k of one row held in global memory (all threads of the CTA call it).
+__device__ void topk_select_global_row(TopkShared& sh, const float* S, int n, int k, int32_t* out) {
+  auto key = [&](int i) { return f32_order_key(S[i]); };
+  if (threadIdx.x == 0) sh.n_sel = 0;
+  __syncthreads();
+  uint32_t kmin, kmax;
+  key_range(sh, n, key, &kmin, &kmax);
+  const BinSel bs = hist_select(sh, n, k, key, kmin, kmax);
+  if (bs.c_T <= AMB_CAP) {
+    // keys above the bin are in; the bin's keys are ranked exactly in shared memory
+    if (threadIdx.x == 0) { sh.n_sel = 0; sh.n_amb = 0; }
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const uint32_t x = key(i);
+      if (x > bs.key_hi) {
+        const uint32_t slot = atomicAdd(&sh.n_sel, 1u);
+        if (slot < (uint32_t)k) sh.sel[slot] = i;
+      } else if (x >= bs.key_lo) {
+        const uint32_t slot = atomicAdd(&sh.n_amb, 1u);
+        if (slot < AMB_CAP) sh.amb[slot] = i;
+      }
+    }
+    __syncthreads();
+    const int n_gt = min((int)sh.n_sel, k), nc = min((int)sh.n_amb, AMB_CAP), need = k - n_gt;
+    for (int c = threadIdx.x; c < nc; c += blockDim.x) sh.hist[c] = key(sh.amb[c]);   // bin keys, staged
+    __syncthreads();
+    for (int c = threadIdx.x; c < nc; c += blockDim.x) {
+      const int ic = sh.amb[c];
+      const uint32_t xc = sh.hist[c];
+      int rank = 0;
+      for (int j = 0; j < nc; ++j) {
+        const uint32_t xj = sh.hist[j];
+        rank += (xj > xc) || (xj == xc && sh.amb[j] < ic);
+      }
+      if (rank < need) sh.sel[n_gt + rank] = ic;
+    }
+    __syncthreads();
+    write_sorted(sh, k, k, out);
+    return;
+  }
+  // many keys in one bin (heavy ties): exact multi-pass radix select over the row
+  if (threadIdx.x == 0) sh.n_sel = 0;
+  __syncthreads();
+  uint32_t remaining;
+  const uint32_t tau = radix_select(sh, n, (uint32_t)k, key, &remaining);
+  for (int i = threadIdx.x; i < n; i += blockDim.x)
+    if (key(i) > tau) {
+      const uint32_t slot = atomicAdd(&sh.n_sel, 1u);
+      if (slot < (uint32_t)k) sh.sel[slot] = i;
+    }
+  __syncthreads();
+  const int n_gt = min((int)sh.n_sel, k);
+  // ties at tau: the `remaining` lowest indices, found by an ordered pass
+  int taken = 0;
+  for (int base = 0; base < n && taken < (int)remaining; base += blockDim.x) {
+    const int i = base + threadIdx.x;
+    const bool f = i < n && key(i) == tau;
+    int tot;
+    const int pos = block_excl_scan_flag(f, sh.wtot, &tot);
+    if (f && taken + pos < (int)remaining) sh.sel[n_gt + taken + pos] = i;
+    taken += tot;
+  }
+  __syncthreads();
+  write_sorted(sh, k, k, out);
+}
+
 __global__ void __launch_bounds__(TK_THREADS)
 topk_select_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_valid,
                    int64_t n_cap, int k, int32_t* __restrict__ idx_out) {
@@ -142,33 +293,11 @@ topk_select_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* 
   if ((int64_t)n > n_cap) n = (int)n_cap;
   if (n < 0) n = 0;
   int32_t* out = idx_out + (size_t)row * k;
-  if (threadIdx.x == 0) sh.n_sel = 0;
-  __syncthreads();
   if (n <= k) {
     for (int i = threadIdx.x; i < k; i += blockDim.x) out[i] = i < n ? i : -1;
     return;
   }
-  uint32_t remaining;
-  const uint32_t tau = radix_select(sh, n, (uint32_t)k, [&](int i) { return f32_order_key(S[i]); }, &remaining);
-  for (int i = threadIdx.x; i < n; i += blockDim.x)
-    if (f32_order_key(S[i]) > tau) {
-      const uint32_t slot = atomicAdd(&sh.n_sel, 1u);
-      if (slot < (uint32_t)k) sh.sel[slot] = i;
-    }
-  __syncthreads();
-  const int n_gt = min((int)sh.n_sel, k);
-  // ties at tau: the `remaining` lowest indices, found by an ordered pass
-  int taken = 0;
-  for (int base = 0; base < n && taken < (int)remaining; base += blockDim.x) {
-    const int i = base + threadIdx.x;
-    const bool f = i < n && f32_order_key(S[i]) == tau;
-    int tot;
-    const int pos = block_excl_scan_flag(f, sh.wtot, &tot);
-    if (f && taken + pos < (int)remaining) sh.sel[n_gt + taken + pos] = i;
-    taken += tot;
-  }
-  __syncthreads();
-  write_sorted(sh, k, k, out);
+  topk_select_global_row(sh, S, n, k, out);
 }
 
 // ------------------------------------------------------------------ indexer selection
@@ -287,12 +416,16 @@ indexer_select_kernel(IndexerArgs a) {
     if (lane == 0) sh.U = u * 1.0001f;
   }
   const float* S = a.scores + (size_t)row * a.ld;
-  uint32_t remaining;
-  const uint32_t tau_key = radix_select(sh, n, (uint32_t)k, [&](int i) { return f32_order_key(S[i]); }, &remaining);
-  const float tau = f32_from_order_key(tau_key);
+  // the scoring kernel recorded this row's key range; the k-th largest fp32 score
+  // lies in histogram bin [f_lo, f_hi]
+  const uint32_t kmax = a.keyrange[2 * (size_t)row], kmin = ~a.keyrange[2 * (size_t)row + 1];
+  const BinSel bs = hist_select(sh, n, k, [&](int i) { return f32_order_key(S[i]); }, kmin, kmax);
+  const float f_lo = f32_from_order_key(bs.key_lo), f_hi = f32_from_order_key(bs.key_hi);
   const float knmax = __uint_as_float(a.knmax[b]);
-  const float E = a.eps_dot * sh.U * knmax + 1.52587890625e-05f * fabsf(tau);   // 2^-16 |tau|
-  const float hi = tau + 2.f * E, lo = tau - 2.f * E;
+  const float E = a.eps_dot * sh.U * knmax + 1.52587890625e-05f * fmaxf(fabsf(f_lo), fabsf(f_hi));  // 2^-16 |tau|
+  // every score is within E of its exact value, so entries above f_hi + 2E are in and
+  // entries below f_lo - 2E are out; the band between is re-scored exactly
+  const float hi = f_hi + 2.f * E, lo = f_lo - 2.f * E;
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
     const float v = S[i];
     if (v > hi) {
@@ -339,11 +472,333 @@ indexer_select_kernel(IndexerArgs a) {
   }
 }
 
+// ------------------------------------------------------------------ register-resident rows
+// For rows of at most 1024 * NPT scores, thread t holds scores [t*NPT, t*NPT+NPT) in
+// registers: the row is read from memory once, the key range, histogram and
+// classification run from registers, and the ascending output is one block-wide scan
+// of per-thread counts (each thread's chunk is contiguous).
+struct RegShared {
+  uint32_t chosen[65536 / 32];   // bitmap of candidates chosen by exact ranking
+  uint32_t tscan[32];
+};
+
+__device__ __forceinline__ int block_excl_scan(int v, uint32_t* wtot, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int x = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += x;
+  }
+  if (lane == 31) wtot[warp] = (uint32_t)incl;
+  __syncthreads();
+  int wpre = 0, tot = 0;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+    const int x = (int)wtot[w];
+    if (w < warp) wpre += x;
+    tot += x;
+  }
+  __syncthreads();
+  *total = tot;
+  return wpre + incl - v;
+}
+
+template <int NPT>
+__device__ __forceinline__ void load_row(const float* S, int n, float* v) {
+  const int base = threadIdx.x * NPT;
+  if (base + NPT <= n) {
+#pragma unroll
+    for (int e = 0; e < NPT; e += 4) {
+      const float4 x = *reinterpret_cast<const float4*>(S + base + e);
+      v[e] = x.x; v[e + 1] = x.y; v[e + 2] = x.z; v[e + 3] = x.w;
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < NPT; ++e) v[e] = (base + e < n) ? S[base + e] : 0.f;
+  }
+}
+
+// Histogram select from registers (same contract as hist_select).
+template <int NPT>
+__device__ BinSel hist_select_reg(TopkShared& sh, int n, int k, const float* val) {
+  const int tid = threadIdx.x, base = tid * NPT;
+  uint32_t mx = 0u, mn = 0xFFFFFFFFu;
+#pragma unroll
+  for (int e = 0; e < NPT; ++e)
+    if (base + e < n) { const uint32_t x = f32_order_key(val[e]); mx = max(mx, x); mn = min(mn, x); }
+  mx = __reduce_max_sync(0xffffffffu, mx);
+  mn = __reduce_min_sync(0xffffffffu, mn);
+  if (tid == 0) { sh.kmax_s = 0u; sh.kmin_s = 0xFFFFFFFFu; }
+  for (int i = tid; i < HB; i += blockDim.x) sh.hist[i] = 0u;
+  __syncthreads();
+  if ((tid & 31) == 0) { atomicMax(&sh.kmax_s, mx); atomicMin(&sh.kmin_s, mn); }
+  __syncthreads();
+  const uint32_t kmax = sh.kmax_s, kmin = sh.kmin_s;
+  BinSel r;
+  const uint32_t diff = kmin ^ kmax;
+  if (diff == 0u) {
+    r.key_lo = r.key_hi = kmax; r.c_gt = 0; r.c_T = n; r.exact = true;
+    return r;
+  }
+  const int h = 31 - __clz(diff);
+  const int lo = h >= 10 ? h - 10 : 0;
+  const uint32_t nbm = (1u << (h - lo + 1)) - 1u;
+#pragma unroll
+  for (int e = 0; e < NPT; ++e)
+    if (base + e < n) atomicAdd(&sh.hist[(f32_order_key(val[e]) >> lo) & nbm], 1u);
+  __syncthreads();
+  const int lane = tid & 31, warp = tid >> 5;
+  const uint32_t b0 = sh.hist[2 * tid], b1 = sh.hist[2 * tid + 1];
+  uint32_t v = b0 + b1;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t x = __shfl_down_sync(0xffffffffu, v, o);
+    if (lane + o < 32) v += x;
+  }
+  if (lane == 0) sh.wtot[warp] = v;
+  __syncthreads();
+  uint32_t above_w = 0;
+  for (int w = warp + 1; w < (int)(blockDim.x >> 5); ++w) above_w += sh.wtot[w];
+  const uint32_t after = v - (b0 + b1) + above_w;
+  const uint32_t kk = (uint32_t)k;
+  if (after < kk && kk <= after + b1) { sh.hT = 2 * tid + 1; sh.hcgt = after; sh.hcT = b1; }
+  if (after + b1 < kk && kk <= after + b1 + b0) { sh.hT = 2 * tid; sh.hcgt = after + b1; sh.hcT = b0; }
+  __syncthreads();
+  const uint32_t T = sh.hT;
+  const uint32_t pre = (h + 1 >= 32) ? 0u : (kmax & ~((2u << h) - 1u));
+  r.key_lo = pre | (T << lo);
+  r.key_hi = r.key_lo | ((1u << lo) - 1u);
+  r.c_gt = (int)sh.hcgt;
+  r.c_T = (int)sh.hcT;
+  r.exact = lo == 0;
+  __syncthreads();
+  return r;
+}
+
+// Writes the selected entries of this thread's chunk (sel bit e set) in ascending order.
+template <int NPT>
+__device__ void write_selected_reg(TopkShared& sh, uint64_t selmask, int k, int32_t* out) {
+  const int base = threadIdx.x * NPT;
+  int total;
+  int pos = block_excl_scan(__popcll(selmask), sh.wtot, &total);
+#pragma unroll
+  for (int e = 0; e < NPT; ++e)
+    if ((selmask >> e) & 1ull) { if (pos < k) out[pos] = base + e; ++pos; }
+  for (int i = total + threadIdx.x; i < k; i += blockDim.x) out[i] = -1;
+}
+
+template <int NPT>
+__global__ void __launch_bounds__(TK_THREADS)
+indexer_select_reg_kernel(IndexerArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  TopkShared& sh = *reinterpret_cast<TopkShared*>(smem_raw);
+  RegShared& rs = *reinterpret_cast<RegShared*>(smem_raw + ((sizeof(TopkShared) + 15) & ~size_t(15)));
+  const int row = blockIdx.x;
+  const int b = row / a.Tq;
+  const int HI = a.H_I, dI = a.d_I, nb = dI / 32;
+  const int k = a.k;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int n = row_eligible(a, row);
+  int32_t* out = a.idx_out + (size_t)row * k;
+  float* sout = a.score_out ? a.score_out + (size_t)row * k : nullptr;
+  const float* S = a.scores + (size_t)row * a.ld;
+  float v[NPT];
+  if (n > k) load_row<NPT>(S, n, v);               // issued first: its latency overlaps the staging below
+
+  for (int i = threadIdx.x; i < HI * dI; i += blockDim.x) {
+    const int j = i / dI, c = i - j * dI;
+    const size_t qoff = (size_t)row * HI + j;
+    float x;
+    if (a.ifmt == CSA_IFMT_F32) x = ((const float*)a.qI)[qoff * dI + c];
+    else if (a.ifmt == CSA_IFMT_E4M3) x = e4m3_to_float(((const uint8_t*)a.qI)[qoff * dI + c]);
+    else {
+      const uint8_t byte = ((const uint8_t*)a.qI)[qoff * (dI / 2) + c / 2];
+      x = e2m1_to_float((c & 1) ? (byte >> 4) : (byte & 0xF));
+    }
+    sh.qd[j * 129 + c] = (double)x;
+  }
+  for (int i = threadIdx.x; i < HI; i += blockDim.x) {
+    sh.w[i] = a.w[(size_t)row * HI + i];
+    if (a.ifmt == CSA_IFMT_E4M3) sh.qsc[i] = ((const float*)a.qI_scale)[(size_t)row * HI + i];
+    if (a.ifmt == CSA_IFMT_MXFP4)
+      for (int bb = 0; bb < nb; ++bb)
+        sh.qsc[i * nb + bb] = ue8m0_to_float(((const uint8_t*)a.qI_scale)[((size_t)row * HI + i) * nb + bb]);
+  }
+  if (threadIdx.x == 0) { sh.n_sel = 0; sh.n_amb = 0; }
+  for (int i = threadIdx.x; i < (NPT * TK_THREADS + 31) / 32; i += blockDim.x) rs.chosen[i] = 0u;
+  __syncthreads();
+
+  if (n <= k) {
+    for (int i = threadIdx.x; i < k; i += blockDim.x) out[i] = i < n ? i : -1;
+    if (sout) {
+      for (int i = warp; i < k; i += (int)(blockDim.x >> 5)) {
+        float x = 0.f;
+        if (i < n) x = (float)rescore_entry(a, sh, row, i);
+        if (lane == 0) sout[i] = x;
+      }
+    }
+    return;
+  }
+  // U = sum_j w_j ||q_j|| : one warp per head pair, lanes over dims
+  {
+    float u = 0.f;
+    for (int j = warp; j < HI; j += (int)(blockDim.x >> 5)) {
+      float n2 = 0.f;
+      for (int c = lane; c < dI; c += 32) {
+        float x = (float)sh.qd[j * 129 + c];
+        if (a.ifmt == CSA_IFMT_E4M3) x *= sh.qsc[j];
+        if (a.ifmt == CSA_IFMT_MXFP4) x *= sh.qsc[j * nb + c / 32];
+        n2 = fmaf(x, x, n2);
+      }
+      n2 = warp_sum(n2);
+      u += sh.w[j] * sqrtf(n2);
+    }
+    if (threadIdx.x == 0) sh.U = 0.f;
+    __syncthreads();
+    if (lane == 0) atomicAdd(&sh.U, u);
+  }
+  const BinSel bs = hist_select_reg<NPT>(sh, n, k, v);         // contains barriers: U is complete after it
+  const float f_lo = f32_from_order_key(bs.key_lo), f_hi = f32_from_order_key(bs.key_hi);
+  const float knmax = __uint_as_float(a.knmax[b]);
+  const float E = a.eps_dot * sh.U * 1.0001f * knmax + 1.52587890625e-05f * fmaxf(fabsf(f_lo), fabsf(f_hi));
+  const float hi = f_hi + 2.f * E, lo = f_lo - 2.f * E;
+  const int base = threadIdx.x * NPT;
+  uint64_t sure = 0ull, amb = 0ull;
+#pragma unroll
+  for (int e = 0; e < NPT; ++e) {
+    if (base + e >= n) continue;
+    if (v[e] > hi) { sure |= 1ull << e; }
+    else if (v[e] >= lo) {
+      amb |= 1ull << e;
+      const uint32_t slot = atomicAdd(&sh.n_amb, 1u);
+      if (slot < AMB_CAP) sh.amb[slot] = base + e;
+    }
+  }
+  int n_in_total;
+  block_excl_scan(__popcll(sure), sh.wtot, &n_in_total);
+  int n_amb = (int)sh.n_amb;
+  if (n_amb > AMB_CAP) {
+    if (threadIdx.x == 0) raise_err(a.err, CSA_DEVERR_BAND);
+    n_amb = AMB_CAP;
+  }
+  const int need = k - n_in_total;
+  for (int i = warp; i < n_amb; i += (int)(blockDim.x >> 5)) {
+    const double x = rescore_entry(a, sh, row, sh.amb[i]);
+    if (lane == 0) sh.amb_s[i] = x;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < n_amb; i += blockDim.x) {
+    const double si = sh.amb_s[i];
+    const int ii = sh.amb[i];
+    int rank = 0;
+    for (int j = 0; j < n_amb; ++j) {
+      const double sj = sh.amb_s[j];
+      rank += (sj > si) || (sj == si && sh.amb[j] < ii);
+    }
+    if (rank < need) atomicOr(&rs.chosen[ii >> 5], 1u << (ii & 31));
+  }
+  __syncthreads();
+  uint64_t sel = sure;
+#pragma unroll
+  for (int e = 0; e < NPT; ++e)
+    if ((amb >> e) & 1ull) {
+      const int i = base + e;
+      if ((rs.chosen[i >> 5] >> (i & 31)) & 1u) sel |= 1ull << e;
+    }
+  write_selected_reg<NPT>(sh, sel, k, out);
+  if (sout) {
+    __syncthreads();
+    // fp64 scores of the selected entries (in output order)
+    for (int i = warp; i < k; i += (int)(blockDim.x >> 5)) {
+      const int e = out[i];
+      float x = 0.f;
+      if (e >= 0) x = (float)rescore_entry(a, sh, row, e);
+      if (lane == 0) sout[i] = x;
+    }
+  }
+}
+
+template <int NPT>
+__global__ void __launch_bounds__(TK_THREADS)
+topk_select_reg_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_valid,
+                       int64_t n_cap, int k, int32_t* __restrict__ idx_out) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  TopkShared& sh = *reinterpret_cast<TopkShared*>(smem_raw);
+  RegShared& rs = *reinterpret_cast<RegShared*>(smem_raw + ((sizeof(TopkShared) + 15) & ~size_t(15)));
+  const int row = blockIdx.x;
+  const float* S = scores + (size_t)row * ld;
+  int n = n_valid ? n_valid[row] : (int)n_cap;
+  if ((int64_t)n > n_cap) n = (int)n_cap;
+  if (n < 0) n = 0;
+  int32_t* out = idx_out + (size_t)row * k;
+  if (n <= k) {
+    for (int i = threadIdx.x; i < k; i += blockDim.x) out[i] = i < n ? i : -1;
+    return;
+  }
+  float v[NPT];
+  load_row<NPT>(S, n, v);
+  if (threadIdx.x == 0) sh.n_amb = 0;
+  for (int i = threadIdx.x; i < (NPT * TK_THREADS + 31) / 32; i += blockDim.x) rs.chosen[i] = 0u;
+  const BinSel bs = hist_select_reg<NPT>(sh, n, k, v);
+  if (bs.c_T > AMB_CAP) {                            // heavy ties: exact multi-pass select from global memory
+    topk_select_global_row(sh, S, n, k, out);
+    return;
+  }
+  const int base = threadIdx.x * NPT;
+  uint64_t sure = 0ull, cand = 0ull;
+#pragma unroll
+  for (int e = 0; e < NPT; ++e) {
+    if (base + e >= n) continue;
+    const uint32_t x = f32_order_key(v[e]);
+    if (x > bs.key_hi) sure |= 1ull << e;
+    else if (x >= bs.key_lo) {
+      cand |= 1ull << e;
+      const uint32_t slot = atomicAdd(&sh.n_amb, 1u);
+      if (slot < AMB_CAP) { sh.amb[slot] = base + e; sh.hist[slot] = x; }
+    }
+  }
+  int n_gt;
+  block_excl_scan(__popcll(sure), sh.wtot, &n_gt);
+  const int nc = min((int)sh.n_amb, AMB_CAP), need = k - n_gt;
+  for (int c = threadIdx.x; c < nc; c += blockDim.x) {
+    const int ic = sh.amb[c];
+    const uint32_t xc = sh.hist[c];
+    int rank = 0;
+    for (int j = 0; j < nc; ++j) {
+      const uint32_t xj = sh.hist[j];
+      rank += (xj > xc) || (xj == xc && sh.amb[j] < ic);
+    }
+    if (rank < need) atomicOr(&rs.chosen[ic >> 5], 1u << (ic & 31));
+  }
+  __syncthreads();
+  uint64_t sel = sure;
+#pragma unroll
+  for (int e = 0; e < NPT; ++e)
+    if ((cand >> e) & 1ull) {
+      const int i = base + e;
+      if ((rs.chosen[i >> 5] >> (i & 31)) & 1u) sel |= 1ull << e;
+    }
+  write_selected_reg<NPT>(sh, sel, k, out);
+}
+
 static void set_smem_attr(const void* fn) {
   cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(TopkShared));
 }
 
+constexpr size_t REG_SMEM = ((sizeof(TopkShared) + 15) & ~size_t(15)) + sizeof(RegShared);
+
+template <int NPT>
+static cudaError_t launch_sel_reg(const IndexerArgs& a, cudaStream_t st) {
+  cudaFuncSetAttribute(indexer_select_reg_kernel<NPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)REG_SMEM);
+  indexer_select_reg_kernel<NPT><<<a.B * a.Tq, TK_THREADS, REG_SMEM, st>>>(a);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_indexer_select(const IndexerArgs& a, cudaStream_t st) {
+  const int64_t per = (a.n_max + TK_THREADS - 1) / TK_THREADS;
+  if (per <= 16) return launch_sel_reg<16>(a, st);
+  if (per <= 32) return launch_sel_reg<32>(a, st);
+  if (per <= 36) return launch_sel_reg<36>(a, st);
   set_smem_attr((const void*)indexer_select_kernel);
   indexer_select_kernel<<<a.B * a.Tq, TK_THREADS, sizeof(TopkShared), st>>>(a);
   return cudaGetLastError();
@@ -352,6 +807,18 @@ cudaError_t launch_indexer_select(const IndexerArgs& a, cudaStream_t st) {
 cudaError_t launch_topk_select(const float* scores, int64_t ld, const int32_t* n_valid, int R, int64_t n,
                                int k, int32_t* idx_out, cudaStream_t st, unsigned* err) {
   (void)err;
+  const int64_t per = (n + TK_THREADS - 1) / TK_THREADS;
+  const bool vec_ok = (ld % 4 == 0) && (((uintptr_t)scores & 15) == 0);   // float4 row loads
+  if (vec_ok && per <= 36) {
+#define CSA_TOPK_REG(NPT)                                                                              \
+    cudaFuncSetAttribute(topk_select_reg_kernel<NPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)REG_SMEM); \
+    topk_select_reg_kernel<NPT><<<R, TK_THREADS, REG_SMEM, st>>>(scores, ld, n_valid, n, k, idx_out);   \
+    return cudaGetLastError();
+    if (per <= 16) { CSA_TOPK_REG(16) }
+    if (per <= 32) { CSA_TOPK_REG(32) }
+    CSA_TOPK_REG(36)
+#undef CSA_TOPK_REG
+  }
   set_smem_attr((const void*)topk_select_kernel);
   topk_select_kernel<<<R, TK_THREADS, sizeof(TopkShared), st>>>(scores, ld, n_valid, n, k, idx_out);
   return cudaGetLastError();

@@ -263,7 +263,15 @@ def test_lightning_index_score_out_and_k_equals_n():
         np.testing.assert_allclose(so[b, 0].cpu().numpy(), I, rtol=1e-6)
 
 
-@pytest.mark.parametrize("wid,sc", [(1, {"B": 4, "T": 65536}), (3, {"ctx": 16384, "Tq": 64, "k": 1024})])
+def _dequant_rows(codes, scale, fmt):
+    if fmt == "e4m3":
+        return O.decode_e4m3(codes) * np.asarray(scale, np.float64)[..., None]
+    v = O.decode_e2m1_packed(codes)
+    return v * np.repeat(O.decode_ue8m0(scale), 32, axis=-1)
+
+
+@pytest.mark.parametrize("wid,sc", [(1, {"B": 4, "T": 65536}), (3, {"ctx": 16384, "Tq": 64, "k": 1024}),
+                                    (4, {"B": 2, "T": 262144})])
 def test_indexer_fp32_score_error_within_band_bound(wid, sc):
     """The exact top-k trusts |S32 - S| <= eps * U * knmax (U = sum_j w_j ||q_j||,
     knmax >= max_s ||k_s||).  Measure the fp32 scores the scoring kernel leaves in
@@ -271,8 +279,9 @@ def test_indexer_fp32_score_error_within_band_bound(wid, sc):
     wl = CI.make_workload(wid, scale=sc)
     D = wl.dims
     T = steps.upload(wl)
+    fmt = D["ifmt"]
     csa.lightning_index(T["qI"], T["qI_scale"], T["w"], T["kI"], T["kI_scale"], T["n_entries"], T["q_pos"], D["k"],
-                        csa.CSA_IFMT_E4M3, T["idx"], T["iws"])
+                        csa.CSA_IFMT_E4M3 if fmt == "e4m3" else csa.CSA_IFMT_MXFP4, T["idx"], T["iws"])
     torch.cuda.synchronize()
     B, Tq, N = D["B"], D["Tq"], D["N"]
     ld = (N + 63) // 64 * 64
@@ -281,11 +290,11 @@ def test_indexer_fp32_score_error_within_band_bound(wid, sc):
     knmax = T["iws"][off:off + 4 * B].view(torch.float32).double().cpu().numpy()
     worst = 0.0
     for b in range(B):
-        qv = O.decode_e4m3(wl.tensors["qI"][b]) * wl.tensors["qI_scale"][b][..., None]
+        qv = _dequant_rows(wl.tensors["qI"][b], wl.tensors["qI_scale"][b], fmt)
         U = (wl.tensors["w"][b] * np.sqrt((qv ** 2).sum(-1))).sum(-1)                  # [Tq]
-        kn = np.sqrt(((O.decode_e4m3(wl.tensors["kI"][b]) * wl.tensors["kI_scale"][b][:, None]) ** 2).sum(-1))
+        kn = np.sqrt((_dequant_rows(wl.tensors["kI"][b], wl.tensors["kI_scale"][b], fmt) ** 2).sum(-1))
         assert knmax[b] >= kn.max() * (1 - 1e-6)
-        I = O.indexer_scores(wl.tensors["qI"][b], wl.tensors["w"][b], wl.tensors["kI"][b], "e4m3",
+        I = O.indexer_scores(wl.tensors["qI"][b], wl.tensors["w"][b], wl.tensors["kI"][b], fmt,
                              wl.tensors["qI_scale"][b], wl.tensors["kI_scale"][b])
         for t in range(Tq):
             ne = O.n_eligible(D["q_pos0"] + t, D["m"], N)
