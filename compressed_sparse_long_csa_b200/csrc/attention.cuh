@@ -71,6 +71,44 @@ __device__ __forceinline__ const T* attn_row_ptr(const AttnArgs& a, int row, int
   return (const T*)a.win + ((size_t)b * a.t_raw + r) * a.dk;
 }
 
+// Same resolution as attn_row_ptr, as (tensor, row) for TMA: which = 0 for the cache
+// ([B*n_max] rows), 1 for the window / raw buffer ([B*W] or [B*t_raw] rows), -1 when
+// virtual row v of query `row` is not a row.
+__device__ __forceinline__ int attn_row_coord(const AttnArgs& a, int row, int v, int* y) {
+  const int b = row / a.Tq;
+  if (v < a.n_seg_a) {
+    int e;
+    if (a.idx) {
+      e = a.idx[(size_t)row * a.k + v];
+      if (e < 0) return -1;
+      if ((int64_t)e >= a.n_max) { raise_err(a.err, CSA_DEVERR_INDEX); return -1; }
+    } else {
+      int n = a.n_entries[b];
+      if ((int64_t)n > a.n_max) n = (int)a.n_max;
+      if (v >= n) return -1;
+      e = v;
+    }
+    *y = (int)((int64_t)b * a.n_max + e);
+    return 0;
+  }
+  const int w = v - a.n_seg_a;
+  if (!a.prefill) {
+    int wl = a.win_len[b];
+    if (wl > a.W) wl = a.W;
+    if (w >= wl) return -1;
+    *y = b * a.W + w;
+    return 1;
+  }
+  const int pos = a.q_pos[row];
+  const int lo = pos - a.W + 1 < 0 ? 0 : pos - a.W + 1;
+  const int p = lo + w;
+  if (p > pos) return -1;
+  const int64_t r = (int64_t)p - a.raw_pos0[b];
+  if (r < 0 || r >= a.t_raw) { raise_err(a.err, CSA_DEVERR_WINDOW); return -1; }
+  *y = (int)((int64_t)b * a.t_raw + r);
+  return 1;
+}
+
 int attn_choose_splits(int n_queries, int H, int64_t rows, bool tc_path);
 
 cudaError_t launch_attention_cuda_core(AttnArgs a, int dtype, cudaStream_t st);

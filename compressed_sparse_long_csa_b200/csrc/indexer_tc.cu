@@ -508,17 +508,17 @@ cudaError_t launch_indexer_scores_tc(const IndexerArgs& a, cudaStream_t st, bool
     if (((uintptr_t)a.kI & 15) || ((uintptr_t)a.qI & 15) || ((uintptr_t)a.kI_scale & 3) || ((uintptr_t)a.qI_scale & 3))
       return cudaSuccess;
     if ((int64_t)a.B * a.n_max > 0x7fffffffLL || (int64_t)a.B * a.Tq * 64 > 0x7fffffffLL) return cudaSuccess;
-    // same bound as the E4M3 kernel: twice the worst case of a 128-term fp32 accumulation
-    const_cast<IndexerArgs&>(a).eps_dot = 1.0f / 65536.0f;
+    // same bound as the E4M3 kernel
+    const_cast<IndexerArgs&>(a).eps_dot = 1.0f / 131072.0f;
     return launch_mxf4(a, st, used);
   }
   if (a.ifmt != CSA_IFMT_E4M3 || a.H_I != 64 || a.d_I != 128) return cudaSuccess;
   if (((uintptr_t)a.kI & 15) || ((uintptr_t)a.qI & 15)) return cudaSuccess;
   if ((int64_t)a.B * a.n_max > 0x7fffffffLL || (int64_t)a.B * a.Tq * 64 > 0x7fffffffLL) return cudaSuccess;
-  // Bound on |fp32 MMA dot - exact| relative to ||q|| ||k||: twice the worst case of a
-  // 128-term fp32 accumulation (128 * 2^-24).  Measured on B200: <= 5e-9 relative to the
-  // bound's scale (test_indexer_fp32_score_error_within_band_bound).
-  const_cast<IndexerArgs&>(a).eps_dot = 1.0f / 65536.0f;
+  // Bound on |fp32 MMA dot - exact| relative to ||q|| ||k||: the worst case of a 128-term
+  // fp32 accumulation of exact products (128 * 2^-24 = 2^-17).  Measured on B200: <= 5e-9
+  // relative to the bound's scale (test_indexer_fp32_score_error_within_band_bound).
+  const_cast<IndexerArgs&>(a).eps_dot = 1.0f / 131072.0f;
   if (a.Tq >= 4) return launch_g<4, 6>(a, st, used);
   return launch_g<1, 6>(a, st, used);
 }

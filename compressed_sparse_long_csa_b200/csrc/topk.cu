@@ -33,7 +33,8 @@ struct TopkShared {
   int32_t amb[AMB_CAP];
   double amb_s[AMB_CAP];
   double contrib[32][64];
-  double kd[32][128];          // per-warp key row being re-scored (exact fp64 values of the codes)
+  double kd[32][128];          // key rows being re-scored (exact fp64 values of the codes)
+  double ksd[32][4];           // their scales: E4M3 row scale in [0], MXFP4 block scales in [0..3]
   double qd[64 * 129];         // query row codes as fp64 (padded rows: conflict-free per-head reads)
   float qsc[64 * 4];
   float w[64];
@@ -351,6 +352,74 @@ __device__ double rescore_entry(const IndexerArgs& a, TopkShared& sh, int row, i
   return S;
 }
 
+// Exact fp64 scores of the entries ids[0..n) of query row `row`, into out[0..n),
+// computed by the whole CTA: key rows are staged 32 at a time, then every thread
+// computes (candidate, head) dot products with four independent accumulators (the
+// partial sums of FP8 / FP4 products are exact in fp64, so their order does not
+// matter), and one thread per candidate adds the head terms in order j = 0..H_I-1.
+__device__ void rescore_block(const IndexerArgs& a, TopkShared& sh, int row, const int32_t* ids, int n,
+                              double* out) {
+  const int b = row / a.Tq;
+  const int HI = a.H_I, dI = a.d_I, nb = dI / 32;
+  for (int base = 0; base < n; base += 32) {
+    const int cnt = min(32, n - base);
+    for (int i = threadIdx.x; i < cnt * dI; i += blockDim.x) {
+      const int c = i / dI, d = i - c * dI;
+      const size_t koff = (size_t)b * a.n_max + ids[base + c];
+      float v;
+      if (a.ifmt == CSA_IFMT_F32) v = ((const float*)a.kI)[koff * dI + d];
+      else if (a.ifmt == CSA_IFMT_E4M3) v = e4m3_to_float(((const uint8_t*)a.kI)[koff * dI + d]);
+      else {
+        const uint8_t byte = ((const uint8_t*)a.kI)[koff * (dI / 2) + d / 2];
+        v = e2m1_to_float((d & 1) ? (byte >> 4) : (byte & 0xF));
+      }
+      sh.kd[c][d] = (double)v;
+    }
+    for (int c = threadIdx.x; c < cnt; c += blockDim.x) {
+      const size_t koff = (size_t)b * a.n_max + ids[base + c];
+      if (a.ifmt == CSA_IFMT_E4M3) sh.ksd[c][0] = (double)((const float*)a.kI_scale)[koff];
+      else if (a.ifmt == CSA_IFMT_MXFP4)
+        for (int bb = 0; bb < nb; ++bb) sh.ksd[c][bb] = (double)ue8m0_to_float(((const uint8_t*)a.kI_scale)[koff * nb + bb]);
+      else sh.ksd[c][0] = 1.0;
+    }
+    __syncthreads();
+    for (int p = threadIdx.x; p < cnt * HI; p += blockDim.x) {
+      const int c = p / HI, j = p - c * HI;
+      const double* qj = sh.qd + j * 129;
+      const double* kc = sh.kd[c];
+      double D;
+      if (a.ifmt == CSA_IFMT_MXFP4) {
+        D = 0.0;
+        for (int bb = 0; bb < nb; ++bb) {
+          double p0 = 0.0, p1 = 0.0, p2 = 0.0, p3 = 0.0;
+#pragma unroll
+          for (int d = bb * 32; d < bb * 32 + 32; d += 4) {
+            p0 = fma(qj[d], kc[d], p0); p1 = fma(qj[d + 1], kc[d + 1], p1);
+            p2 = fma(qj[d + 2], kc[d + 2], p2); p3 = fma(qj[d + 3], kc[d + 3], p3);
+          }
+          D += ((double)sh.qsc[j * nb + bb] * sh.ksd[c][bb]) * ((p0 + p1) + (p2 + p3));
+        }
+      } else {
+        double p0 = 0.0, p1 = 0.0, p2 = 0.0, p3 = 0.0;
+        for (int d = 0; d < dI; d += 4) {
+          p0 = fma(qj[d], kc[d], p0); p1 = fma(qj[d + 1], kc[d + 1], p1);
+          p2 = fma(qj[d + 2], kc[d + 2], p2); p3 = fma(qj[d + 3], kc[d + 3], p3);
+        }
+        const double raw = (p0 + p1) + (p2 + p3);
+        D = (a.ifmt == CSA_IFMT_E4M3) ? ((double)sh.qsc[j] * sh.ksd[c][0]) * raw : raw;
+      }
+      sh.contrib[c][j] = (double)sh.w[j] * fmax(D, 0.0);
+    }
+    __syncthreads();
+    for (int c = threadIdx.x; c < cnt; c += blockDim.x) {
+      double S = 0.0;
+      for (int j = 0; j < HI; ++j) S += sh.contrib[c][j];
+      out[base + c] = S;
+    }
+    __syncthreads();
+  }
+}
+
 __global__ void __launch_bounds__(TK_THREADS)
 indexer_select_kernel(IndexerArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -444,11 +513,7 @@ indexer_select_kernel(IndexerArgs a) {
     n_amb = AMB_CAP;
   }
   const int need = k - n_in;
-  for (int i = warp; i < n_amb; i += (int)(blockDim.x >> 5)) {
-    const double v = rescore_entry(a, sh, row, sh.amb[i]);
-    if (lane == 0) sh.amb_s[i] = v;
-  }
-  __syncthreads();
+  rescore_block(a, sh, row, sh.amb, n_amb, sh.amb_s);
   for (int i = threadIdx.x; i < n_amb; i += blockDim.x) {
     const double si = sh.amb_s[i];
     const int ii = sh.amb[i];
@@ -464,11 +529,8 @@ indexer_select_kernel(IndexerArgs a) {
   write_sorted(sh, cnt, k, out);
   if (sout) {
     __syncthreads();
-    for (int i = warp; i < k; i += (int)(blockDim.x >> 5)) {
-      float v = 0.f;
-      if (i < cnt) v = (float)rescore_entry(a, sh, row, sh.sel[i]);
-      if (lane == 0) sout[i] = v;
-    }
+    rescore_block(a, sh, row, sh.sel, cnt, sh.amb_s);
+    for (int i = threadIdx.x; i < k; i += blockDim.x) sout[i] = i < cnt ? (float)sh.amb_s[i] : 0.f;
   }
 }
 
@@ -658,11 +720,33 @@ indexer_select_reg_kernel(IndexerArgs a) {
     if (lane == 0) atomicAdd(&sh.U, u);
   }
   const BinSel bs = hist_select_reg<NPT>(sh, n, k, v);         // contains barriers: U is complete after it
-  const float f_lo = f32_from_order_key(bs.key_lo), f_hi = f32_from_order_key(bs.key_hi);
-  const float knmax = __uint_as_float(a.knmax[b]);
-  const float E = a.eps_dot * sh.U * 1.0001f * knmax + 1.52587890625e-05f * fmaxf(fabsf(f_lo), fabsf(f_hi));
-  const float hi = f_hi + 2.f * E, lo = f_lo - 2.f * E;
   const int base = threadIdx.x * NPT;
+  // the exact k-th largest fp32 score tau: rank the threshold bin's keys (stored in the
+  // free histogram) when they fit; otherwise fall back to the bin bounds
+  float tau_lo = f32_from_order_key(bs.key_lo), tau_hi = f32_from_order_key(bs.key_hi);
+  if (bs.c_T <= HB) {
+    if (threadIdx.x == 0) sh.n_sel = 0;
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < NPT; ++e) {
+      if (base + e >= n) continue;
+      const uint32_t x = f32_order_key(v[e]);
+      if (x >= bs.key_lo && x <= bs.key_hi) sh.hist[atomicAdd(&sh.n_sel, 1u)] = x;
+    }
+    __syncthreads();
+    const int nb_ = (int)sh.n_sel, want = k - bs.c_gt;           // tau = want-th largest key of the bin
+    for (int i = threadIdx.x; i < nb_; i += blockDim.x) {
+      const uint32_t xi = sh.hist[i];
+      int gt = 0, ge = 0;
+      for (int j = 0; j < nb_; ++j) { const uint32_t xj = sh.hist[j]; gt += xj > xi; ge += xj >= xi; }
+      if (gt < want && want <= ge) sh.digit = xi;               // every such xi is the same key
+    }
+    __syncthreads();
+    tau_lo = tau_hi = f32_from_order_key(sh.digit);
+  }
+  const float knmax = __uint_as_float(a.knmax[b]);
+  const float E = a.eps_dot * sh.U * 1.0001f * knmax + 1.52587890625e-05f * fmaxf(fabsf(tau_lo), fabsf(tau_hi));
+  const float hi = tau_hi + 2.f * E, lo = tau_lo - 2.f * E;
   uint64_t sure = 0ull, amb = 0ull;
 #pragma unroll
   for (int e = 0; e < NPT; ++e) {
@@ -682,11 +766,7 @@ indexer_select_reg_kernel(IndexerArgs a) {
     n_amb = AMB_CAP;
   }
   const int need = k - n_in_total;
-  for (int i = warp; i < n_amb; i += (int)(blockDim.x >> 5)) {
-    const double x = rescore_entry(a, sh, row, sh.amb[i]);
-    if (lane == 0) sh.amb_s[i] = x;
-  }
-  __syncthreads();
+  rescore_block(a, sh, row, sh.amb, n_amb, sh.amb_s);
   for (int i = threadIdx.x; i < n_amb; i += blockDim.x) {
     const double si = sh.amb_s[i];
     const int ii = sh.amb[i];
@@ -707,13 +787,15 @@ indexer_select_reg_kernel(IndexerArgs a) {
     }
   write_selected_reg<NPT>(sh, sel, k, out);
   if (sout) {
+    // fp64 scores of the selected entries (in output order), 32 at a time
     __syncthreads();
-    // fp64 scores of the selected entries (in output order)
-    for (int i = warp; i < k; i += (int)(blockDim.x >> 5)) {
-      const int e = out[i];
-      float x = 0.f;
-      if (e >= 0) x = (float)rescore_entry(a, sh, row, e);
-      if (lane == 0) sout[i] = x;
+    for (int base2 = 0; base2 < k; base2 += 32) {
+      const int cnt = min(32, k - base2);
+      if (threadIdx.x < cnt) sh.sel[threadIdx.x] = out[base2 + threadIdx.x];
+      __syncthreads();
+      rescore_block(a, sh, row, sh.sel, cnt, sh.amb_s);
+      if (threadIdx.x < cnt) sout[base2 + threadIdx.x] = (float)sh.amb_s[threadIdx.x];
+      __syncthreads();
     }
   }
 }
