@@ -229,7 +229,9 @@ static csa_status run_attention(AttnArgs& a, int dtype, void* workspace, size_t 
   } else {
     a.splits = 1;
   }
-  a.rows_per_split = (int)((rows + a.splits - 1) / a.splits);
+  a.rows_per_split = attn_rows_per_split(rows, a.splits, tc);
+  a.splits = (int)((rows + a.rows_per_split - 1) / a.rows_per_split);
+  if (a.splits < 1) a.splits = 1;
   a.part = (float*)workspace;
   bool used = false;
   cudaError_t e = cudaSuccess;
@@ -238,7 +240,7 @@ static csa_status run_attention(AttnArgs& a, int dtype, void* workspace, size_t 
   if (!used) {
     if (tc) {  // the tensor-core path declined: recompute the split plan for the CUDA-core path
       a.splits = decode ? attn_choose_splits(a.B * a.Tq, a.H, rows, false) : 1;
-      a.rows_per_split = (int)((rows + a.splits - 1) / a.splits);
+      a.rows_per_split = attn_rows_per_split(rows, a.splits, false);
     }
     e = launch_attention_cuda_core(a, dtype, st);
     if (e != cudaSuccess) return CSA_ERR_CUDA;

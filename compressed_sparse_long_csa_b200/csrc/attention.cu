@@ -155,23 +155,30 @@ attn_combine_kernel(AttnArgs a) {
 
 int attn_choose_splits(int n_queries, int H, int64_t rows, bool tc_path) {
   int64_t s;
+  const int64_t tiles = (rows + 63) / 64;
   if (tc_path) {
-    // at most one wave of CTA pairs (one CTA per SM).  Each split also costs a 264 KB
-    // partial (o, m, l of 128 heads) written and read back, and re-reads the 147 KB query
-    // from L2, so a split should cover at least ~5 tiles of 64 rows.
+    // one wave of CTAs (two per query and split, one CTA per SM), splits of at least two
+    // 64-row tiles, and the tiles spread as evenly as whole tiles allow
     s = 148 / (2 * (int64_t)n_queries);
-    const int64_t by_rows = rows / 320;
-    if (s > by_rows) s = by_rows;
+    if (s > tiles / 2) s = tiles / 2;
+    if (s < 1) s = 1;
+    const int64_t per = (tiles + s - 1) / s;
+    s = (tiles + per - 1) / per;
   } else {
     // aim for >= 2 waves of CTAs on 148 SMs
     const int64_t ctas_per_split = (int64_t)n_queries * ((H + CC_HG - 1) / CC_HG);
     s = (2 * 148 + ctas_per_split - 1) / ctas_per_split;
   }
-  const int64_t max_s = (rows + 63) / 64;
-  if (s > max_s) s = max_s;
+  if (s > tiles) s = tiles;
   if (s < 1) s = 1;
   if (s > 64) s = 64;
   return (int)s;
+}
+
+int attn_rows_per_split(int64_t rows, int splits, bool tc_path) {
+  int64_t r = (rows + splits - 1) / splits;
+  if (tc_path) r = (r + 63) / 64 * 64;     // the tensor-core kernel takes whole 64-row tiles
+  return (int)(r < 1 ? 1 : r);
 }
 
 cudaError_t launch_attention_cuda_core(AttnArgs a, int dtype, cudaStream_t st) {

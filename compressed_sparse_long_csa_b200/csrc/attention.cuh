@@ -110,6 +110,8 @@ __device__ __forceinline__ int attn_row_coord(const AttnArgs& a, int row, int v,
 }
 
 int attn_choose_splits(int n_queries, int H, int64_t rows, bool tc_path);
+// Rows of each split (the last split takes the rest); a multiple of 64 on the tensor-core path.
+int attn_rows_per_split(int64_t rows, int splits, bool tc_path);
 
 cudaError_t launch_attention_cuda_core(AttnArgs a, int dtype, cudaStream_t st);
 cudaError_t launch_attention_tc(AttnArgs a, cudaStream_t st, bool* used);
