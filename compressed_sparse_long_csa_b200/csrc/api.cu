@@ -143,6 +143,7 @@ csa_status lightning_index(const void* qI, const void* qI_scale, const float* w,
   REQUIRE_PTR(qI); REQUIRE_PTR(w); REQUIRE_PTR(kI); REQUIRE_PTR(idx_out);
   if (ifmt != CSA_IFMT_F32) { REQUIRE_PTR(qI_scale); REQUIRE_PTR(kI_scale); }
   if (score_out) REQUIRE(aligned16(score_out), CSA_ERR_ALIGN);
+  REQUIRE(aligned16(qI) && aligned16(kI), CSA_ERR_ALIGN);
   REQUIRE(n_entries && q_pos, CSA_ERR_NULL);
   const size_t need = lightning_index_workspace_size(B, Tq, n_max, k);
   REQUIRE(workspace && ws_bytes >= need, CSA_ERR_WORKSPACE);

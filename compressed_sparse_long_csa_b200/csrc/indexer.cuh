@@ -56,5 +56,9 @@ cudaError_t launch_indexer_scores_tc(const IndexerArgs& a, cudaStream_t st, bool
 cudaError_t launch_indexer_select(const IndexerArgs& a, cudaStream_t st);
 cudaError_t launch_topk_select(const float* scores, int64_t ld, const int32_t* n_valid, int R, int64_t n,
                                int k, int32_t* idx_out, cudaStream_t st, unsigned* err);
+// Cluster paths (select.cu); cudaErrorNotSupported when a row does not fit one cluster.
+cudaError_t launch_indexer_select_cluster(const IndexerArgs& a, cudaStream_t st);
+cudaError_t launch_topk_select_cluster(const float* scores, int64_t ld, const int32_t* n_valid, int R, int64_t n,
+                                       int k, int32_t* idx_out, cudaStream_t st);
 
 }  // namespace csa

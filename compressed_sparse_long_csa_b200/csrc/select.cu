@@ -1,0 +1,793 @@
+// Exact top-k selection of compressed entries on a thread-block cluster per query row.
+//
+// "Техотчёт DeepSeek-V4 (2026): миллион токенов контекста", section "Гибридное
+// внимание: CSA и HCA", CSA step 2 (the indexer keeps the top-k compressed blocks;
+// k = 512 / 1024 from table "Конфигурации").  Ties go to the lower entry index and
+// the selected set is written in ascending index order, padded with -1.
+//
+// A row of n scores is split over the C CTAs (C <= 8) of one cluster: CTA r holds
+// entries [r*chunk, (r+1)*chunk) in shared memory.  The CTAs combine their partial
+// results through distributed shared memory:
+//  1. the key range [kmin, kmax] of the row (monotone fp32 order keys);
+//  2. 2048-bin histograms whose bins split the current key range evenly (a multiply
+//     and a shift per key, monotone in the key); the bin holding the k-th largest key
+//     becomes the next range until it holds at most SL_CAP keys or one key value;
+//  3. topk_select: the keys of that bin, gathered by every CTA, give the exact k-th
+//     largest fp32 key tau (lightning_index refines the bin to at most 64 keys and
+//     uses its bounds [tau_lo, tau_hi] instead);
+//  4a. topk_select: keys above tau are in; of the keys equal to tau, the lowest
+//      indices complete the set (CTA rank order is index order);
+//  4b. lightning_index: the fp32 scores carry a bounded error E (accumulation in the
+//      scoring kernel), so the k-th largest exact score lies in [tau_lo - E, tau_hi + E].
+//      Entries above tau_hi + 2E are certainly in, entries below tau_lo - 2E certainly
+//      out.  The key range comes from the scoring kernel, which records it.  Every CTA re-scores its own band entries exactly in
+//      fp64 from the quantised operands (FP8 / FP4 products and their sums are exact
+//      in fp64; the per-head terms are then added in head order, as the definition
+//      does), and the band is ranked by (exact score desc, index asc).
+//  5. selections are kept as bitmaps (one ballot per 32 entries); cluster-wide prefix
+//     counts give each CTA its output offset and a scan over the bitmap words writes
+//     the indices in ascending order.
+// Every pass over the entries is a rolled loop: this kernel runs its code once per
+// row, and code that runs once costs its instruction fetch, so the code is kept small.
+#include "indexer.cuh"
+
+#include <algorithm>
+#include <cooperative_groups.h>
+#include <map>
+#include <mutex>
+#include <tuple>
+
+namespace csa {
+
+namespace cg = cooperative_groups;
+
+namespace {
+
+constexpr int SL_T = 512;              // threads per CTA (128 registers each: no spills)
+constexpr int SL_W = SL_T / 32;
+constexpr int SL_BINS = 2048;          // histogram bins
+constexpr int SL_CAP = 1024;           // threshold-bin keys / band entries gathered per row
+constexpr int SL_CMAX = 8;             // CTAs per cluster (portable cluster size)
+constexpr int SL_CHUNK = 34 * 1024;    // entries per CTA at most
+constexpr int SL_QPT = 8192 / SL_T;    // query-row elements per thread (H_I * d_I <= 8192)
+constexpr int SL_BAND_CT = 64;         // the indexer refines the threshold bin down to this many keys
+constexpr int SL_WORDS = SL_CHUNK / 32;
+constexpr int SL_RW = 4;               // warps that re-score band entries, 8 entries each at a time
+constexpr int SL_QLD = 132;            // padded row length (doubles) of the staged query / key rows
+
+struct SelFixed {
+  uint32_t hist[2][SL_BINS];           // read by peers (double-buffered across refinement rounds)
+  uint32_t keys[SL_CAP];               // read by peers: this CTA's keys of the threshold bin
+  uint32_t gkeys[SL_CAP];              // all keys of the threshold bin
+  uint32_t bits_a[SL_WORDS];           // selected (indexer: sure, then also chosen band) / above tau
+  uint32_t bits_b[SL_WORDS];           // plain select: equal to tau
+  int32_t band_id[SL_CAP];             // read by peers: this CTA's band entries
+  double band_s[SL_CAP];               // read by peers: their exact scores
+  int32_t gband_id[SL_CAP];
+  double gband_s[SL_CAP];
+  uint32_t wtot[SL_W];
+  uint32_t red[2];
+  uint32_t pub[4];                     // read by peers
+  uint32_t pcnt[SL_CMAX][2];
+  int goff[SL_CMAX + 1];               // start of each CTA's part in a gathered list
+  uint32_t cgt, cT, tau, tlo, thi, cnt, n_sure;
+  unsigned long long mult;
+  float n2[64];
+  float qsc[64 * 4];
+  float w[64];
+  float U;
+};
+
+// Re-scoring scratch: overlays the score array once the scores have been classified.
+struct Resc {
+  double qd[64 * SL_QLD];              // query row codes as fp64 (rows padded: conflict-free fragment reads)
+  double kd[SL_RW][8][SL_QLD];         // key rows being re-scored
+  double contrib[SL_RW][8][64];        // their per-head terms
+  float ksc[SL_RW][8][4];              // their scales (E4M3 row scale in [0], MXFP4 block scales)
+};
+
+constexpr size_t SL_FIXED = (sizeof(SelFixed) + 127) & ~size_t(127);
+
+// What the exact re-scoring reads of the key side, passed by value: taking the address of
+// a kernel parameter would copy the whole argument block to local memory.
+struct RescKeys {
+  const void* kI;
+  const void* kI_scale;
+  int64_t n_max;
+  int ifmt, HI, dI;
+};
+
+__device__ __forceinline__ void sl_sync(cg::cluster_group cl, unsigned C) {
+  if (C == 1) __syncthreads();
+  else cl.sync();
+}
+
+// Block-wide exclusive scan of one int per thread (all threads call).
+__device__ __forceinline__ int sl_excl_scan(int v, uint32_t* wtot, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int x = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += x;
+  }
+  if (lane == 31) wtot[warp] = (uint32_t)incl;
+  __syncthreads();
+  int wpre = 0, tot = 0;
+  if (lane < SL_W) {
+    const int x = (int)wtot[lane];
+    wpre = (lane < warp) ? x : 0;
+    tot = x;
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    wpre += __shfl_xor_sync(0xffffffffu, wpre, o);
+    tot += __shfl_xor_sync(0xffffffffu, tot, o);
+  }
+  __syncthreads();
+  *total = tot;
+  return wpre + incl - v;
+}
+
+// Word `slot` of CTA p's published values, p < C.
+__device__ __forceinline__ uint32_t sl_peer(cg::cluster_group cl, const uint32_t* pub, int slot, int p) {
+  return cl.map_shared_rank(pub, p)[slot];
+}
+
+// Concatenate every CTA's list (CTA p's count in its pub[slot]) into dst in rank order;
+// returns the total (at most cap).
+// The offsets are set by sl_gather_offsets (one thread, then a barrier).
+__device__ __forceinline__ void sl_gather_offsets(SelFixed& sh, cg::cluster_group cl, unsigned C, int slot) {
+  if (threadIdx.x == 0) {
+    int total = 0;
+    for (int p = 0; p < (int)C; ++p) {
+      sh.goff[p] = total;
+      total += (int)sl_peer(cl, sh.pub, slot, p);
+    }
+    for (int p = (int)C; p <= SL_CMAX; ++p) sh.goff[p] = total;
+  }
+}
+template <typename T>
+__device__ __forceinline__ int sl_gather(SelFixed& sh, cg::cluster_group cl, unsigned C, T* list, T* dst, int cap) {
+  const int total = min(sh.goff[SL_CMAX], cap);
+  for (int i = threadIdx.x; i < total; i += SL_T) {
+    int p = 0;
+    while (p + 1 < (int)C && sh.goff[p + 1] <= i) ++p;
+    dst[i] = cl.map_shared_rank(list, p)[i - sh.goff[p]];
+  }
+  return total;
+}
+
+// Key range [lo, hi] of the row over every CTA's entries sv[0..m).
+__device__ __forceinline__ void sl_key_range(SelFixed& sh, const float* sv, int m, cg::cluster_group cluster,
+                                          uint32_t* lo_out, uint32_t* hi_out) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  const unsigned C = cluster.num_blocks();
+  uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+  for (int i = tid; i < m; i += SL_T) {
+    const uint32_t x = f32_order_key(sv[i]);
+    mn = min(mn, x);
+    mx = max(mx, x);
+  }
+  mn = __reduce_min_sync(0xffffffffu, mn);
+  mx = __reduce_max_sync(0xffffffffu, mx);
+  if (tid == 0) { sh.red[0] = 0xFFFFFFFFu; sh.red[1] = 0u; }
+  __syncthreads();
+  if (lane == 0) { atomicMin(&sh.red[0], mn); atomicMax(&sh.red[1], mx); }
+  __syncthreads();
+  if (tid == 0) { sh.pub[0] = sh.red[0]; sh.pub[1] = sh.red[1]; }
+  sl_sync(cluster, C);
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+  for (int p = 0; p < (int)C; ++p) {
+    lo = min(lo, sl_peer(cluster, sh.pub, 0, p));
+    hi = max(hi, sl_peer(cluster, sh.pub, 1, p));
+  }
+  *lo_out = lo;
+  *hi_out = hi;
+}
+
+// Histogram refinement (step 2): [*lo, *hi] holds the k-th largest key of the row; on
+// return it is a bin of at most stop_ct keys (or one key value), *want is the rank of
+// the k-th largest key from the top among the keys inside it and *cT their number.
+// Every CTA of the cluster calls it with the same arguments and gets the same results.
+__device__ __forceinline__ void sl_refine(SelFixed& sh, const float* sv, int m, int k, int stop_ct,
+                                       cg::cluster_group cluster, uint32_t* lo_io, uint32_t* hi_io, int* want_out,
+                                       uint32_t* ct_out) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned C = cluster.num_blocks();
+  uint32_t lo = *lo_io, hi = *hi_io;
+  int want = k;
+  uint32_t cT = 0;
+  for (int round = 0; round < 6; ++round) {
+    uint32_t* H = sh.hist[round & 1];
+    reinterpret_cast<uint4*>(H)[tid] = make_uint4(0u, 0u, 0u, 0u);   // 4 bins per thread
+    if (tid == 0) sh.mult = (hi - lo) < (uint32_t)SL_BINS ? 0ull : (1ull << 43) / ((uint64_t)(hi - lo) + 1ull);
+    __syncthreads();
+    const uint32_t mult = (uint32_t)sh.mult;              // < 2^32 whenever it is used
+#pragma unroll 4
+    for (int i = tid; i < m; i += SL_T) {
+      const uint32_t x = f32_order_key(sv[i]);
+      if (x >= lo && x <= hi) atomicAdd(&H[mult ? __umulhi(x - lo, mult) : x - lo], 1u);
+    }
+    sl_sync(cluster, C);
+    uint4 hb = make_uint4(0u, 0u, 0u, 0u);
+    for (int p = 0; p < (int)C; ++p) {
+      const uint4 x = reinterpret_cast<const uint4*>(cluster.map_shared_rank(H, p))[tid];
+      hb.x += x.x; hb.y += x.y; hb.z += x.z; hb.w += x.w;
+    }
+    // suffix counts: bins above 4*tid+3 belong to higher threads
+    const uint32_t mine = hb.x + hb.y + hb.z + hb.w;
+    uint32_t vsum = mine;
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t x = __shfl_down_sync(0xffffffffu, vsum, o);
+      if (lane + o < 32) vsum += x;
+    }
+    if (lane == 0) sh.wtot[warp] = vsum;
+    __syncthreads();
+    uint32_t above_w = 0;
+    if (lane < SL_W && lane > warp) above_w = sh.wtot[lane];
+    above_w = __reduce_add_sync(0xffffffffu, above_w);
+    uint32_t after = vsum - mine + above_w;                 // keys in bins > 4*tid+3
+    const uint32_t kk = (uint32_t)want;
+    const uint32_t cb[4] = {hb.w, hb.z, hb.y, hb.x};        // bins 4t+3, 4t+2, 4t+1, 4t
+    int bin = -1;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (bin < 0 && after < kk && kk <= after + cb[q]) { bin = 4 * tid + 3 - q; sh.cgt = after; sh.cT = cb[q]; }
+      after += cb[q];
+    }
+    if (bin >= 0) {
+      // key bounds of bin T (one thread does the 64-bit divisions)
+      const uint64_t T = (uint64_t)bin, M = sh.mult;
+      if (!M) {
+        sh.tlo = sh.thi = lo + (uint32_t)T;
+      } else {
+        // bin T holds the keys x - lo in [ceil(T 2^32 / M), ceil((T+1) 2^32 / M) - 1]
+        const uint64_t a0 = ((T << 32) + M - 1) / M, a1 = (((T + 1) << 32) + M - 1) / M;
+        sh.tlo = lo + (uint32_t)a0;
+        const uint64_t top = (uint64_t)lo + a1 - 1;
+        sh.thi = top < (uint64_t)hi ? (uint32_t)top : hi;
+      }
+    }
+    __syncthreads();
+    want -= (int)sh.cgt;
+    cT = sh.cT;
+    lo = sh.tlo;
+    hi = sh.thi;
+    __syncthreads();                                       // sh.* is rewritten next round
+    if (lo == hi || cT <= (uint32_t)stop_ct) break;
+  }
+  *lo_io = lo;
+  *hi_io = hi;
+  *want_out = want;
+  *ct_out = cT;
+}
+
+// Step 3: the exact k-th largest key, given the bin [lo, hi] that holds it at rank
+// `want` from the top (the bin holds at most SL_CAP keys).
+__device__ __forceinline__ uint32_t sl_exact_tau(SelFixed& sh, const float* sv, int m, cg::cluster_group cluster,
+                                              uint32_t lo, uint32_t hi, int want) {
+  const int tid = threadIdx.x;
+  const unsigned C = cluster.num_blocks();
+  if (lo == hi) return lo;
+  if (tid == 0) { sh.cnt = 0; sh.tau = lo; }
+  __syncthreads();
+  for (int i = tid; i < m; i += SL_T) {
+    const uint32_t x = f32_order_key(sv[i]);
+    if (x >= lo && x <= hi) {
+      const uint32_t s = atomicAdd(&sh.cnt, 1u);
+      if (s < (uint32_t)SL_CAP) sh.keys[s] = x;
+    }
+  }
+  __syncthreads();
+  if (tid == 0) sh.pub[2] = min(sh.cnt, (uint32_t)SL_CAP);
+  sl_sync(cluster, C);
+  sl_gather_offsets(sh, cluster, C, 2);
+  __syncthreads();
+  const int ng = sl_gather(sh, cluster, C, sh.keys, sh.gkeys, SL_CAP);
+  __syncthreads();
+  for (int i = tid; i < ng; i += SL_T) {
+    const uint32_t xi = sh.gkeys[i];
+    int gt = 0, ge = 0;
+    for (int j = 0; j < ng; ++j) {
+      const uint32_t xj = sh.gkeys[j];
+      gt += xj > xi;
+      ge += xj >= xi;
+    }
+    if (gt < want && want <= ge) sh.tau = xi;             // every such xi is the same key
+  }
+  __syncthreads();
+  return sh.tau;
+}
+
+// Load this CTA's scores S[0, m) into sv (16-byte vectors when aligned).
+__device__ __forceinline__ void sl_load(const float* __restrict__ S, int m, bool vec, float* sv) {
+  if (vec) {
+    const int m4 = m & ~3;
+#pragma unroll 4
+    for (int i = threadIdx.x * 4; i < m4; i += SL_T * 4)
+      *reinterpret_cast<float4*>(sv + i) = *reinterpret_cast<const float4*>(S + i);
+    for (int i = m4 + threadIdx.x; i < m; i += SL_T) sv[i] = S[i];
+  } else {
+#pragma unroll 4
+    for (int i = threadIdx.x; i < m; i += SL_T) sv[i] = S[i];
+  }
+}
+
+// Writes this CTA's selected entries (bitmap sel over nwords words, entry ids base + bit
+// index) at out[off ...] in ascending order; returns the CTA's count.
+__device__ __forceinline__ int sl_write(SelFixed& sh, const uint32_t* sel, int nwords, int base, int off, int k, int32_t* out) {
+  const int wpt = (nwords + SL_T - 1) / SL_T;            // words per thread (contiguous)
+  const int w0 = threadIdx.x * wpt, w1 = min(nwords, w0 + wpt);
+  int cnt = 0;
+  for (int w = w0; w < w1; ++w) cnt += __popc(sel[w]);
+  int tot;
+  int pos = off + sl_excl_scan(cnt, sh.wtot, &tot);
+  for (int w = w0; w < w1; ++w)
+    for (uint32_t bits = sel[w]; bits; bits &= bits - 1) {
+      if (pos < k) out[pos] = base + 32 * w + __ffs(bits) - 1;
+      ++pos;
+    }
+  return tot;
+}
+
+// ------------------------------------------------------------------ plain top-k
+__global__ void __launch_bounds__(SL_T, 1)
+topk_cluster_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_valid, int64_t n_cap,
+                    int k, int32_t* __restrict__ idx_out, int chunk, int vec) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  SelFixed& sh = *reinterpret_cast<SelFixed*>(smem_raw);
+  float* sv = reinterpret_cast<float*>(smem_raw + SL_FIXED);
+  cg::cluster_group cluster = cg::this_cluster();
+  const unsigned C = cluster.num_blocks(), r = cluster.block_rank();
+  const int row = blockIdx.x / C;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int n = n_valid ? n_valid[row] : (int)n_cap;
+  if ((int64_t)n > n_cap) n = (int)n_cap;
+  if (n < 0) n = 0;
+  int32_t* out = idx_out + (size_t)row * k;
+  if (n <= k) {
+    if (r == 0)
+      for (int i = tid; i < k; i += SL_T) out[i] = i < n ? i : -1;
+    return;                                                // uniform over the cluster: no DSMEM use
+  }
+  const int lo = (int)r * chunk;
+  const int m = max(0, min(n - lo, chunk));
+  sl_load(scores + (size_t)row * ld + lo, m, vec != 0, sv);
+  __syncthreads();
+  uint32_t lo_k, hi_k, cT;
+  int want;
+  sl_key_range(sh, sv, m, cluster, &lo_k, &hi_k);
+  sl_refine(sh, sv, m, k, SL_CAP, cluster, &lo_k, &hi_k, &want, &cT);
+  const uint32_t tau = sl_exact_tau(sh, sv, m, cluster, lo_k, hi_k, want);
+  // bitmaps: above tau, equal to tau
+  const int nwords = (m + 31) / 32;
+  int gt = 0, eq = 0;
+  for (int w = warp; w < nwords; w += SL_W) {
+    const int i = 32 * w + lane;
+    const uint32_t x = i < m ? f32_order_key(sv[i]) : 0u;
+    const uint32_t ba = __ballot_sync(0xffffffffu, i < m && x > tau);
+    const uint32_t bb = __ballot_sync(0xffffffffu, i < m && x == tau);
+    if (lane == 0) { sh.bits_a[w] = ba; sh.bits_b[w] = bb; gt += __popc(ba); eq += __popc(bb); }
+  }
+  int gt_tot, eq_tot;
+  sl_excl_scan(gt, sh.wtot, &gt_tot);
+  sl_excl_scan(eq, sh.wtot, &eq_tot);
+  if (tid == 0) { sh.pub[0] = (uint32_t)gt_tot; sh.pub[1] = (uint32_t)eq_tot; }
+  sl_sync(cluster, C);
+  int all_gt = 0;
+  for (int p = 0; p < (int)C; ++p) all_gt += (int)sl_peer(cluster, sh.pub, 0, p);
+  const int eq_need = k - all_gt;
+  int eqp = 0, off = 0, quota = 0;
+  for (int p = 0; p < (int)C; ++p) {
+    const int g = (int)sl_peer(cluster, sh.pub, 0, p), e = (int)sl_peer(cluster, sh.pub, 1, p);
+    const int q = max(0, min(eq_need - eqp, e));
+    if (p < (int)r) off += g + q;
+    if (p == (int)r) quota = q;
+    eqp += e;
+  }
+  // keep the first `quota` entries equal to tau (index order)
+  {
+    const int wpt = (nwords + SL_T - 1) / SL_T;
+    const int w0 = tid * wpt, w1 = min(nwords, w0 + wpt);
+    int c = 0;
+    for (int w = w0; w < w1; ++w) c += __popc(sh.bits_b[w]);
+    int tot;
+    int seen = sl_excl_scan(c, sh.wtot, &tot);
+    for (int w = w0; w < w1; ++w) {
+      uint32_t keep = 0u;
+      for (uint32_t bits = sh.bits_b[w]; bits; bits &= bits - 1) {
+        if (seen < quota) keep |= bits & (0u - bits);
+        ++seen;
+      }
+      sh.bits_a[w] |= keep;
+    }
+  }
+  __syncthreads();
+  sl_write(sh, sh.bits_a, nwords, lo, off, k, out);
+  sl_sync(cluster, C);                                     // peers may still read pub
+}
+
+// ------------------------------------------------------------------ indexer selection
+// D (8x8) += A (8x4, row-major) * B (4x8, column-major), fp64 tensor-core MMA.  Lane l
+// holds A[l/4][l%4], B[l%4][l/4] and D[l/4][2(l%4)], D[l/4][2(l%4)+1].
+__device__ __forceinline__ void dmma_884(double& d0, double& d1, double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+               : "+d"(d0), "+d"(d1) : "d"(a), "d"(b));
+}
+
+// Exact fp64 scores of entries ids[0..cnt) (cnt <= 8), by one warp (re-scoring slot rw);
+// the query row is staged in rs.qd / sh.qsc / sh.w.  The per-head dot products of FP8 /
+// FP4 codes are exact in fp64 in any order, so they run on the fp64 tensor cores (heads x
+// entries, K = d_I, one accumulator chain per 8-head block); each head's term
+// w_j * max(D_j, 0) is formed as the definition does, and the terms are added in order
+// j = 0..H_I-1.
+__device__ __noinline__ void sl_rescore8(const RescKeys a, SelFixed& sh, Resc& rs, int rw, int b,
+                                         const int32_t* ids, int cnt, double* out) {
+  const int lane = threadIdx.x & 31;
+  const int HI = a.HI, dI = a.dI, nb = dI / 32;
+  // key rows (zeros past cnt): all loads first.  Lane l holds elements [4l, 4l+4) (E4M3,
+  // fp32) or [8l, 8l+8) (MXFP4) of each row (row starts are 16-byte aligned).
+  const bool lane_in = (a.ifmt == CSA_IFMT_MXFP4) ? lane * 8 < dI : lane * 4 < dI;
+  uint4 raw[8];
+  float scl[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    raw[c] = make_uint4(0u, 0u, 0u, 0u);
+    scl[c] = 0.f;
+    if (c < cnt) {
+      const size_t koff = (size_t)b * a.n_max + ids[c];
+      if (lane_in) {
+        if (a.ifmt == CSA_IFMT_E4M3) raw[c].x = reinterpret_cast<const uint32_t*>((const uint8_t*)a.kI + koff * dI)[lane];
+        else if (a.ifmt == CSA_IFMT_MXFP4) raw[c].x = reinterpret_cast<const uint32_t*>((const uint8_t*)a.kI + koff * (dI / 2))[lane];
+        else raw[c] = reinterpret_cast<const uint4*>((const float*)a.kI + koff * dI)[lane];
+      }
+      if (a.ifmt == CSA_IFMT_E4M3) scl[c] = ((const float*)a.kI_scale)[koff];
+      else if (a.ifmt == CSA_IFMT_MXFP4 && lane < nb) scl[c] = ue8m0_to_float(((const uint8_t*)a.kI_scale)[koff * nb + lane]);
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    double* kd = rs.kd[rw][c];
+    if (lane_in) {
+      if (a.ifmt == CSA_IFMT_E4M3) {
+        for (int e = 0; e < 4; ++e) kd[lane * 4 + e] = (double)e4m3_to_float((raw[c].x >> (8 * e)) & 0xFFu);
+      } else if (a.ifmt == CSA_IFMT_MXFP4) {
+        for (int e = 0; e < 8; ++e) kd[lane * 8 + e] = (double)e2m1_to_float((raw[c].x >> (4 * e)) & 0xFu);
+      } else {
+        kd[lane * 4] = (double)__uint_as_float(raw[c].x); kd[lane * 4 + 1] = (double)__uint_as_float(raw[c].y);
+        kd[lane * 4 + 2] = (double)__uint_as_float(raw[c].z); kd[lane * 4 + 3] = (double)__uint_as_float(raw[c].w);
+      }
+    }
+    if (a.ifmt == CSA_IFMT_E4M3 && lane == 0) rs.ksc[rw][c][0] = scl[c];
+    if (a.ifmt == CSA_IFMT_MXFP4 && lane < nb) rs.ksc[rw][c][lane] = scl[c];
+  }
+  __syncwarp();
+  const int g = lane >> 2, t = lane & 3;
+  const double* brow = rs.kd[rw][g];           // B[k][n]: entry n = g, dim k = t of each step
+  const int n_blk = (a.ifmt == CSA_IFMT_MXFP4) ? nb : 1;     // scale blocks along K
+  const int ks_blk = dI / 4 / n_blk;
+  double D[8][2];
+#pragma unroll
+  for (int h = 0; h < 8; ++h) D[h][0] = D[h][1] = 0.0;
+  for (int bb = 0; bb < n_blk; ++bb) {
+    double P[8][2];
+#pragma unroll
+    for (int h = 0; h < 8; ++h) P[h][0] = P[h][1] = 0.0;
+    for (int ks = bb * ks_blk; ks < (bb + 1) * ks_blk; ++ks) {
+      const double bf = brow[4 * ks + t];
+#pragma unroll
+      for (int h = 0; h < 8; ++h) dmma_884(P[h][0], P[h][1], rs.qd[(8 * h + g) * SL_QLD + 4 * ks + t], bf);
+    }
+    if (a.ifmt == CSA_IFMT_MXFP4) {
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        const int j = 8 * h + g;
+        const double qs = (j < HI) ? (double)sh.qsc[j * nb + bb] : 0.0;
+        D[h][0] += (qs * (double)rs.ksc[rw][2 * t][bb]) * P[h][0];
+        D[h][1] += (qs * (double)rs.ksc[rw][2 * t + 1][bb]) * P[h][1];
+      }
+    } else {
+#pragma unroll
+      for (int h = 0; h < 8; ++h) { D[h][0] = P[h][0]; D[h][1] = P[h][1]; }
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < 8; ++h) {
+    const int j = 8 * h + g;
+    if (j < HI) {
+      double d0 = D[h][0], d1 = D[h][1];
+      if (a.ifmt == CSA_IFMT_E4M3) {
+        d0 = ((double)sh.qsc[j] * (double)rs.ksc[rw][2 * t][0]) * d0;
+        d1 = ((double)sh.qsc[j] * (double)rs.ksc[rw][2 * t + 1][0]) * d1;
+      }
+      rs.contrib[rw][2 * t][j] = (double)sh.w[j] * fmax(d0, 0.0);
+      rs.contrib[rw][2 * t + 1][j] = (double)sh.w[j] * fmax(d1, 0.0);
+    }
+  }
+  __syncwarp();
+  if (lane < cnt) {
+    double S = 0.0;
+    for (int j = 0; j < HI; ++j) S += rs.contrib[rw][lane][j];
+    out[lane] = S;
+  }
+  __syncwarp();
+}
+
+// Exact scores of ids[0..n) into out[0..n): warps 0..SL_RW-1 take groups of 8.  All
+// threads of the CTA call (the function ends with a CTA barrier).
+__device__ __noinline__ void sl_rescore_list(const RescKeys a, SelFixed& sh, Resc& rs, int b, const int32_t* ids, int n,
+                                double* out) {
+  const int warp = threadIdx.x >> 5;
+  if (warp < SL_RW)
+    for (int g0 = warp * 8; g0 < n; g0 += SL_RW * 8) sl_rescore8(a, sh, rs, warp, b, ids + g0, min(8, n - g0), out + g0);
+  __syncthreads();
+}
+
+// Stage the query row codes (held in registers, element tid + SL_T*e) as fp64:
+// consecutive threads store consecutive doubles; rows up to the next multiple of 8 heads
+// are zero (fp64 MMA fragments read them).
+__device__ __forceinline__ void sl_stage_query(Resc& rs, const float (&qx)[SL_QPT], int total, int lgd, int HI, int dI) {
+  const int tid = threadIdx.x;
+#pragma unroll
+  for (int e = 0; e < SL_QPT; ++e) {
+    const int i = tid + SL_T * e;
+    if (i < total) rs.qd[(i >> lgd) * SL_QLD + (i & (dI - 1))] = (double)qx[e];
+  }
+  const int hpad = (HI + 7) / 8 * 8;
+  for (int i = total + tid; i < hpad * dI; i += SL_T) rs.qd[(i >> lgd) * SL_QLD + (i & (dI - 1))] = 0.0;
+}
+
+__global__ void __launch_bounds__(SL_T, 1)
+indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  SelFixed& sh = *reinterpret_cast<SelFixed*>(smem_raw);
+  float* sv = reinterpret_cast<float*>(smem_raw + SL_FIXED);
+  Resc& rs = *reinterpret_cast<Resc*>(smem_raw + SL_FIXED);      // overlays sv after classification
+  cg::cluster_group cluster = cg::this_cluster();
+  const unsigned C = cluster.num_blocks(), r = cluster.block_rank();
+  const int row = blockIdx.x / C;
+  const int b = row / a.Tq;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int k = a.k;
+  const int HI = a.H_I, dI = a.d_I, nb = dI / 32;
+  const int n = row_eligible(a, row);
+  int32_t* out = a.idx_out + (size_t)row * k;
+  float* sout = a.score_out ? a.score_out + (size_t)row * k : nullptr;
+  const RescKeys rk{a.kI, a.kI_scale, a.n_max, a.ifmt, a.H_I, a.d_I};
+  const int lo = (int)r * chunk;
+  const int m = max(0, min(n - lo, chunk));
+  // ---- the query row: codes into registers (staged into shared memory once the scores
+  // are classified), scales and weights, and U = sum_j w_j ||q_j|| for the error bound
+  const int total = HI * dI, lgd = __ffs(dI) - 1;
+  const size_t r0 = (size_t)row * total;
+  float qx[SL_QPT];
+#pragma unroll
+  for (int e = 0; e < SL_QPT; ++e) {
+    const int i = tid + SL_T * e;
+    qx[e] = 0.f;
+    if (i < total) {
+      if (a.ifmt == CSA_IFMT_E4M3) qx[e] = e4m3_to_float(((const uint8_t*)a.qI)[r0 + i]);
+      else if (a.ifmt == CSA_IFMT_MXFP4) {
+        const uint8_t byte = ((const uint8_t*)a.qI)[(r0 + i) >> 1];
+        qx[e] = e2m1_to_float((i & 1) ? (byte >> 4) : (byte & 0xF));
+      } else qx[e] = ((const float*)a.qI)[r0 + i];
+    }
+  }
+  if (tid < HI) {
+    sh.w[tid] = a.w[(size_t)row * HI + tid];
+    sh.n2[tid] = 0.f;
+    if (a.ifmt == CSA_IFMT_E4M3) sh.qsc[tid] = ((const float*)a.qI_scale)[(size_t)row * HI + tid];
+    if (a.ifmt == CSA_IFMT_MXFP4)
+      for (int bb = 0; bb < nb; ++bb)
+        sh.qsc[tid * nb + bb] = ue8m0_to_float(((const uint8_t*)a.qI_scale)[((size_t)row * HI + tid) * nb + bb]);
+  }
+  const float knmax = __uint_as_float(a.knmax[b]);
+  // the key range the scoring kernel recorded (exact min / max over the row's eligible entries)
+  uint32_t lo_k = ~a.keyrange[2 * (size_t)row + 1], hi_k = a.keyrange[2 * (size_t)row];
+  if (n > k) sl_load(a.scores + (size_t)row * a.ld + lo, m, true, sv);
+  __syncthreads();
+  // squared norms per head: a warp's 32 elements of one e lie in one head (d_I >= 32)
+#pragma unroll
+  for (int e = 0; e < SL_QPT; ++e) {
+    const int i = tid + SL_T * e;
+    float x = qx[e];
+    if (i < total) {
+      const int j = i >> lgd;
+      if (a.ifmt == CSA_IFMT_E4M3) x *= sh.qsc[j];
+      if (a.ifmt == CSA_IFMT_MXFP4) x *= sh.qsc[j * nb + ((i & (dI - 1)) >> 5)];
+    }
+    const float s2 = warp_sum(x * x);
+    if (lane == 0 && i < total) atomicAdd(&sh.n2[i >> lgd], s2);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    float u = 0.f;
+    for (int j = lane; j < HI; j += 32) u += sh.w[j] * sqrtf(sh.n2[j]);
+    u = warp_sum(u);
+    if (lane == 0) sh.U = u;
+  }
+  // (sh.U is read after the barriers of the threshold search)
+  if (n <= k) {
+    // every eligible entry is selected; CTA r scores the slots [r*k/C, (r+1)*k/C)
+    if (r == 0)
+      for (int i = tid; i < k; i += SL_T) out[i] = i < n ? i : -1;
+    if (sout) {
+      __syncthreads();
+      sl_stage_query(rs, qx, total, lgd, HI, dI);
+      const int s0 = (int)((int64_t)k * r / C), s1 = (int)((int64_t)k * (r + 1) / C);
+      for (int c0 = s0; c0 < s1; c0 += SL_CAP) {
+        const int cnt = min(SL_CAP, s1 - c0);
+        __syncthreads();
+        for (int i = tid; i < cnt; i += SL_T) sh.band_id[i] = min(c0 + i, max(n - 1, 0));
+        __syncthreads();
+        sl_rescore_list(rk, sh, rs, b, sh.band_id, cnt, sh.band_s);
+        for (int i = tid; i < cnt; i += SL_T) sout[c0 + i] = (c0 + i < n) ? (float)sh.band_s[i] : 0.f;
+      }
+    }
+    return;                                                // uniform over the cluster: no DSMEM use
+  }
+  // the bin [tau_lo, tau_hi] that holds the k-th largest fp32 score (at most SL_BAND_CT
+  // scores, or one value); the band is that bin widened by 2E on both sides
+  uint32_t cT;
+  int want;
+  sl_refine(sh, sv, m, k, SL_BAND_CT, cluster, &lo_k, &hi_k, &want, &cT);
+  const float tau_lo = f32_from_order_key(lo_k), tau_hi = f32_from_order_key(hi_k);
+  const float E = a.eps_dot * sh.U * 1.0001f * knmax + 1.52587890625e-05f * fmaxf(fabsf(tau_lo), fabsf(tau_hi));
+  const float band_hi = tau_hi + 2.f * E, band_lo = tau_lo - 2.f * E;
+  // ---- classify: sure (above the band) as a bitmap, band entries as a list
+  if (tid == 0) { sh.cnt = 0; sh.n_sure = 0; }
+  __syncthreads();
+  const int nwords = (m + 31) / 32;
+  int my_sure = 0;
+  for (int w = warp; w < nwords; w += SL_W) {
+    const int i = 32 * w + lane;
+    const float v = i < m ? sv[i] : 0.f;
+    const bool sure = i < m && v > band_hi;
+    const bool band = i < m && !sure && v >= band_lo;
+    const uint32_t ba = __ballot_sync(0xffffffffu, sure);
+    if (lane == 0) { sh.bits_a[w] = ba; my_sure += __popc(ba); }
+    if (band) {
+      const uint32_t s = atomicAdd(&sh.cnt, 1u);
+      if (s < (uint32_t)SL_CAP) sh.band_id[s] = lo + i;
+    }
+  }
+  if (lane == 0 && my_sure) atomicAdd(&sh.n_sure, (uint32_t)my_sure);
+  __syncthreads();                                         // sv is dead from here on
+  const uint32_t nb_raw = sh.cnt;
+  const int n_band = (int)min(nb_raw, (uint32_t)SL_CAP);
+  if (nb_raw > (uint32_t)SL_CAP && tid == 0) raise_err(a.err, CSA_DEVERR_BAND);
+  sl_stage_query(rs, qx, total, lgd, HI, dI);
+  __syncthreads();
+  // ---- exact scores of this CTA's band entries
+  sl_rescore_list(rk, sh, rs, b, sh.band_id, n_band, sh.band_s);
+  if (tid == 0) { sh.pub[0] = sh.n_sure; sh.pub[1] = (uint32_t)n_band; }
+  sl_sync(cluster, C);
+  // ---- gather every CTA's band and rank all of it (each CTA reaches the same verdicts)
+  sl_gather_offsets(sh, cluster, C, 1);
+  __syncthreads();
+  const int ng = sl_gather(sh, cluster, C, sh.band_id, sh.gband_id, SL_CAP);
+  sl_gather(sh, cluster, C, sh.band_s, sh.gband_s, SL_CAP);
+  int all_sure = 0;
+  for (int p = 0; p < (int)C; ++p) all_sure += (int)sl_peer(cluster, sh.pub, 0, p);
+  if (tid < SL_CMAX) {
+    sh.pcnt[tid][0] = (unsigned)tid < C ? sl_peer(cluster, sh.pub, 0, tid) : 0u;
+    sh.pcnt[tid][1] = 0u;
+  }
+  __syncthreads();
+  const int need = k - all_sure;
+  for (int i = tid; i < ng; i += SL_T) {
+    const double si = sh.gband_s[i];
+    const int ii = sh.gband_id[i];
+    int rank = 0;
+    for (int j = 0; j < ng; ++j) {
+      const double sj = sh.gband_s[j];
+      rank += (sj > si) || (sj == si && sh.gband_id[j] < ii);
+    }
+    if (rank < need) {
+      const int owner = ii / chunk;
+      atomicAdd(&sh.pcnt[owner][1], 1u);
+      if (owner == (int)r) atomicOr(&sh.bits_a[(ii - lo) >> 5], 1u << ((ii - lo) & 31));
+    }
+  }
+  __syncthreads();
+  int off = 0, tot_all = 0;
+  for (int p = 0; p < (int)C; ++p) {
+    const int c = (int)(sh.pcnt[p][0] + sh.pcnt[p][1]);
+    if (p < (int)r) off += c;
+    tot_all += c;
+  }
+  // ---- write the selected entries of this CTA in ascending order
+  const int mine = sl_write(sh, sh.bits_a, nwords, lo, off, k, out);
+  if (r == 0)
+    for (int i = tot_all + tid; i < k; i += SL_T) out[i] = -1;
+  if (sout) {
+    // this CTA's selected entries, SL_CAP at a time (the gathered band arrays as scratch)
+    const int p0 = off, p1 = min(k, off + mine);
+    for (int c0 = p0; c0 < p1; c0 += SL_CAP) {
+      const int cnt = min(SL_CAP, p1 - c0);
+      __syncthreads();
+      for (int i = tid; i < cnt; i += SL_T) sh.gband_id[i] = out[c0 + i];
+      __syncthreads();
+      sl_rescore_list(rk, sh, rs, b, sh.gband_id, cnt, sh.gband_s);
+      for (int i = tid; i < cnt; i += SL_T) sout[c0 + i] = (float)sh.gband_s[i];
+    }
+    if (r == 0)
+      for (int i = tot_all + tid; i < k; i += SL_T) sout[i] = 0.f;
+  }
+  sl_sync(cluster, C);                                     // peers may still read band_id / band_s / pub
+}
+
+// Cluster size and chunk: the fewest CTAs (at most SL_CMAX) whose shared memory holds
+// the row; chunk is a multiple of 1024 entries.
+bool sl_plan(int64_t n, int* C, int* chunk) {
+  const int64_t c = (n + SL_CHUNK - 1) / SL_CHUNK;
+  if (c > SL_CMAX) return false;
+  const int64_t cc = c < 1 ? 1 : c;
+  int64_t ch = (n + cc - 1) / cc;
+  ch = (ch + 1023) / 1024 * 1024;
+  if (ch < 1024) ch = 1024;
+  *C = (int)cc;
+  *chunk = (int)ch;
+  return true;
+}
+
+template <typename Kern, typename... Args>
+cudaError_t sl_launch(Kern kern, int rows, int C, size_t smem, cudaStream_t st, Args... args) {
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(rows * C);
+  cfg.blockDim = dim3(SL_T);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // a cluster of C CTAs of this size must fit on the GPU (checked once per kernel, C and size)
+  static std::mutex mu;
+  static std::map<std::tuple<const void*, int, size_t>, bool> fits;
+  {
+    std::lock_guard<std::mutex> g(mu);
+    const auto key = std::make_tuple((const void*)kern, C, smem);
+    auto it = fits.find(key);
+    if (it == fits.end()) {
+      int n_clusters = 0;
+      const bool ok = cudaOccupancyMaxActiveClusters(&n_clusters, kern, &cfg) == cudaSuccess && n_clusters > 0;
+      cudaGetLastError();
+      it = fits.emplace(key, ok).first;
+    }
+    if (!it->second) return cudaErrorNotSupported;
+  }
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+static_assert(SL_FIXED + sizeof(Resc) <= 232448 && SL_FIXED + (size_t)SL_CHUNK * 4 <= 232448,
+              "shared memory budget of one CTA (227 KB)");
+
+}  // namespace
+
+// Returns cudaErrorNotSupported when the row is too long for one cluster (the caller
+// then uses the single-CTA global-memory path).
+cudaError_t launch_indexer_select_cluster(const IndexerArgs& a, cudaStream_t st) {
+  int C, chunk;
+  const int rows = a.B * a.Tq;
+  if (a.H_I > 64 || a.d_I > 128 || a.H_I * a.d_I > SL_QPT * SL_T || !sl_plan(a.n_max, &C, &chunk) || (a.ld % 4) != 0 ||
+      ((uintptr_t)a.scores & 15) != 0 || (int64_t)rows * C > 0x7fffffffLL)
+    return cudaErrorNotSupported;
+  const size_t region = std::max((size_t)chunk * 4, sizeof(Resc));
+  return sl_launch(indexer_select_cluster_kernel, rows, C, SL_FIXED + region, st, a, chunk);
+}
+
+cudaError_t launch_topk_select_cluster(const float* scores, int64_t ld, const int32_t* n_valid, int R, int64_t n,
+                                       int k, int32_t* idx_out, cudaStream_t st) {
+  int C, chunk;
+  if (!sl_plan(n, &C, &chunk) || (int64_t)R * C > 0x7fffffffLL) return cudaErrorNotSupported;
+  const int vec = (ld % 4 == 0) && (((uintptr_t)scores & 15) == 0);
+  return sl_launch(topk_cluster_kernel, R, C, SL_FIXED + (size_t)chunk * 4, st, scores, ld, n_valid, n, k, idx_out,
+                   chunk, vec);
+}
+
+}  // namespace csa

@@ -1,13 +1,14 @@
-// Exact top-k selection of compressed entries.
+// Exact top-k selection of compressed entries: the single-CTA path for rows longer
+// than one thread-block cluster holds (select.cu has the cluster path used otherwise).
 //
 // "Техотчёт DeepSeek-V4 (2026): миллион токенов контекста", section "Гибридное
 // внимание: CSA и HCA", CSA step 2 (the indexer keeps the top-k compressed blocks;
 // k = 512 / 1024 from table "Конфигурации").  Ties go to the lower entry index and
 // the selected set is written in ascending index order, padded with -1.
 //
-// One CTA of 1024 threads per query row:
-//  1. MSB-first radix select (4 passes of 8 bits) over monotone fp32 keys gives the
-//     exact k-th largest fp32 score tau.
+// One CTA of 1024 threads per query row, scores read from global memory:
+//  1. range-aware histogram passes over monotone fp32 keys give the exact k-th
+//     largest fp32 score tau (MSB-first radix select as the fallback);
 //  2a. topk_select: entries with key > tau are in; the first `remaining` entries
 //     with key == tau (ascending index) complete the set.
 //  2b. lightning_index: the fp32 scores carry a bounded error E (accumulation in the
@@ -15,7 +16,7 @@
 //     tau - 2E certainly out; the band between is re-scored exactly in fp64 from
 //     the quantised operands (FP8/FP4 products and their sums are exact in fp64)
 //     and ranked by (score desc, index asc).
-//  3. The chosen indices are sorted ascending (bitonic sort in shared memory).
+//  3. The chosen indices are written in ascending order.
 #include "indexer.cuh"
 
 namespace csa {
@@ -534,353 +535,13 @@ indexer_select_kernel(IndexerArgs a) {
   }
 }
 
-// ------------------------------------------------------------------ register-resident rows
-// For rows of at most 1024 * NPT scores, thread t holds scores [t*NPT, t*NPT+NPT) in
-// registers: the row is read from memory once, the key range, histogram and
-// classification run from registers, and the ascending output is one block-wide scan
-// of per-thread counts (each thread's chunk is contiguous).
-struct RegShared {
-  uint32_t chosen[65536 / 32];   // bitmap of candidates chosen by exact ranking
-  uint32_t tscan[32];
-};
-
-__device__ __forceinline__ int block_excl_scan(int v, uint32_t* wtot, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int x = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += x;
-  }
-  if (lane == 31) wtot[warp] = (uint32_t)incl;
-  __syncthreads();
-  int wpre = 0, tot = 0;
-  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
-    const int x = (int)wtot[w];
-    if (w < warp) wpre += x;
-    tot += x;
-  }
-  __syncthreads();
-  *total = tot;
-  return wpre + incl - v;
-}
-
-template <int NPT>
-__device__ __forceinline__ void load_row(const float* S, int n, float* v) {
-  const int base = threadIdx.x * NPT;
-  if (base + NPT <= n) {
-#pragma unroll
-    for (int e = 0; e < NPT; e += 4) {
-      const float4 x = *reinterpret_cast<const float4*>(S + base + e);
-      v[e] = x.x; v[e + 1] = x.y; v[e + 2] = x.z; v[e + 3] = x.w;
-    }
-  } else {
-#pragma unroll
-    for (int e = 0; e < NPT; ++e) v[e] = (base + e < n) ? S[base + e] : 0.f;
-  }
-}
-
-// Histogram select from registers (same contract as hist_select).
-template <int NPT>
-__device__ BinSel hist_select_reg(TopkShared& sh, int n, int k, const float* val) {
-  const int tid = threadIdx.x, base = tid * NPT;
-  uint32_t mx = 0u, mn = 0xFFFFFFFFu;
-#pragma unroll
-  for (int e = 0; e < NPT; ++e)
-    if (base + e < n) { const uint32_t x = f32_order_key(val[e]); mx = max(mx, x); mn = min(mn, x); }
-  mx = __reduce_max_sync(0xffffffffu, mx);
-  mn = __reduce_min_sync(0xffffffffu, mn);
-  if (tid == 0) { sh.kmax_s = 0u; sh.kmin_s = 0xFFFFFFFFu; }
-  for (int i = tid; i < HB; i += blockDim.x) sh.hist[i] = 0u;
-  __syncthreads();
-  if ((tid & 31) == 0) { atomicMax(&sh.kmax_s, mx); atomicMin(&sh.kmin_s, mn); }
-  __syncthreads();
-  const uint32_t kmax = sh.kmax_s, kmin = sh.kmin_s;
-  BinSel r;
-  const uint32_t diff = kmin ^ kmax;
-  if (diff == 0u) {
-    r.key_lo = r.key_hi = kmax; r.c_gt = 0; r.c_T = n; r.exact = true;
-    return r;
-  }
-  const int h = 31 - __clz(diff);
-  const int lo = h >= 10 ? h - 10 : 0;
-  const uint32_t nbm = (1u << (h - lo + 1)) - 1u;
-#pragma unroll
-  for (int e = 0; e < NPT; ++e)
-    if (base + e < n) atomicAdd(&sh.hist[(f32_order_key(val[e]) >> lo) & nbm], 1u);
-  __syncthreads();
-  const int lane = tid & 31, warp = tid >> 5;
-  const uint32_t b0 = sh.hist[2 * tid], b1 = sh.hist[2 * tid + 1];
-  uint32_t v = b0 + b1;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t x = __shfl_down_sync(0xffffffffu, v, o);
-    if (lane + o < 32) v += x;
-  }
-  if (lane == 0) sh.wtot[warp] = v;
-  __syncthreads();
-  uint32_t above_w = 0;
-  for (int w = warp + 1; w < (int)(blockDim.x >> 5); ++w) above_w += sh.wtot[w];
-  const uint32_t after = v - (b0 + b1) + above_w;
-  const uint32_t kk = (uint32_t)k;
-  if (after < kk && kk <= after + b1) { sh.hT = 2 * tid + 1; sh.hcgt = after; sh.hcT = b1; }
-  if (after + b1 < kk && kk <= after + b1 + b0) { sh.hT = 2 * tid; sh.hcgt = after + b1; sh.hcT = b0; }
-  __syncthreads();
-  const uint32_t T = sh.hT;
-  const uint32_t pre = (h + 1 >= 32) ? 0u : (kmax & ~((2u << h) - 1u));
-  r.key_lo = pre | (T << lo);
-  r.key_hi = r.key_lo | ((1u << lo) - 1u);
-  r.c_gt = (int)sh.hcgt;
-  r.c_T = (int)sh.hcT;
-  r.exact = lo == 0;
-  __syncthreads();
-  return r;
-}
-
-// Writes the selected entries of this thread's chunk (sel bit e set) in ascending order.
-template <int NPT>
-__device__ void write_selected_reg(TopkShared& sh, uint64_t selmask, int k, int32_t* out) {
-  const int base = threadIdx.x * NPT;
-  int total;
-  int pos = block_excl_scan(__popcll(selmask), sh.wtot, &total);
-#pragma unroll
-  for (int e = 0; e < NPT; ++e)
-    if ((selmask >> e) & 1ull) { if (pos < k) out[pos] = base + e; ++pos; }
-  for (int i = total + threadIdx.x; i < k; i += blockDim.x) out[i] = -1;
-}
-
-template <int NPT>
-__global__ void __launch_bounds__(TK_THREADS)
-indexer_select_reg_kernel(IndexerArgs a) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  TopkShared& sh = *reinterpret_cast<TopkShared*>(smem_raw);
-  RegShared& rs = *reinterpret_cast<RegShared*>(smem_raw + ((sizeof(TopkShared) + 15) & ~size_t(15)));
-  const int row = blockIdx.x;
-  const int b = row / a.Tq;
-  const int HI = a.H_I, dI = a.d_I, nb = dI / 32;
-  const int k = a.k;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int n = row_eligible(a, row);
-  int32_t* out = a.idx_out + (size_t)row * k;
-  float* sout = a.score_out ? a.score_out + (size_t)row * k : nullptr;
-  const float* S = a.scores + (size_t)row * a.ld;
-  float v[NPT];
-  if (n > k) load_row<NPT>(S, n, v);               // issued first: its latency overlaps the staging below
-
-  for (int i = threadIdx.x; i < HI * dI; i += blockDim.x) {
-    const int j = i / dI, c = i - j * dI;
-    const size_t qoff = (size_t)row * HI + j;
-    float x;
-    if (a.ifmt == CSA_IFMT_F32) x = ((const float*)a.qI)[qoff * dI + c];
-    else if (a.ifmt == CSA_IFMT_E4M3) x = e4m3_to_float(((const uint8_t*)a.qI)[qoff * dI + c]);
-    else {
-      const uint8_t byte = ((const uint8_t*)a.qI)[qoff * (dI / 2) + c / 2];
-      x = e2m1_to_float((c & 1) ? (byte >> 4) : (byte & 0xF));
-    }
-    sh.qd[j * 129 + c] = (double)x;
-  }
-  for (int i = threadIdx.x; i < HI; i += blockDim.x) {
-    sh.w[i] = a.w[(size_t)row * HI + i];
-    if (a.ifmt == CSA_IFMT_E4M3) sh.qsc[i] = ((const float*)a.qI_scale)[(size_t)row * HI + i];
-    if (a.ifmt == CSA_IFMT_MXFP4)
-      for (int bb = 0; bb < nb; ++bb)
-        sh.qsc[i * nb + bb] = ue8m0_to_float(((const uint8_t*)a.qI_scale)[((size_t)row * HI + i) * nb + bb]);
-  }
-  if (threadIdx.x == 0) { sh.n_sel = 0; sh.n_amb = 0; }
-  for (int i = threadIdx.x; i < (NPT * TK_THREADS + 31) / 32; i += blockDim.x) rs.chosen[i] = 0u;
-  __syncthreads();
-
-  if (n <= k) {
-    for (int i = threadIdx.x; i < k; i += blockDim.x) out[i] = i < n ? i : -1;
-    if (sout) {
-      for (int i = warp; i < k; i += (int)(blockDim.x >> 5)) {
-        float x = 0.f;
-        if (i < n) x = (float)rescore_entry(a, sh, row, i);
-        if (lane == 0) sout[i] = x;
-      }
-    }
-    return;
-  }
-  // U = sum_j w_j ||q_j|| : one warp per head pair, lanes over dims
-  {
-    float u = 0.f;
-    for (int j = warp; j < HI; j += (int)(blockDim.x >> 5)) {
-      float n2 = 0.f;
-      for (int c = lane; c < dI; c += 32) {
-        float x = (float)sh.qd[j * 129 + c];
-        if (a.ifmt == CSA_IFMT_E4M3) x *= sh.qsc[j];
-        if (a.ifmt == CSA_IFMT_MXFP4) x *= sh.qsc[j * nb + c / 32];
-        n2 = fmaf(x, x, n2);
-      }
-      n2 = warp_sum(n2);
-      u += sh.w[j] * sqrtf(n2);
-    }
-    if (threadIdx.x == 0) sh.U = 0.f;
-    __syncthreads();
-    if (lane == 0) atomicAdd(&sh.U, u);
-  }
-  const BinSel bs = hist_select_reg<NPT>(sh, n, k, v);         // contains barriers: U is complete after it
-  const int base = threadIdx.x * NPT;
-  // the exact k-th largest fp32 score tau: rank the threshold bin's keys (stored in the
-  // free histogram) when they fit; otherwise fall back to the bin bounds
-  float tau_lo = f32_from_order_key(bs.key_lo), tau_hi = f32_from_order_key(bs.key_hi);
-  if (bs.c_T <= HB) {
-    if (threadIdx.x == 0) sh.n_sel = 0;
-    __syncthreads();
-#pragma unroll
-    for (int e = 0; e < NPT; ++e) {
-      if (base + e >= n) continue;
-      const uint32_t x = f32_order_key(v[e]);
-      if (x >= bs.key_lo && x <= bs.key_hi) sh.hist[atomicAdd(&sh.n_sel, 1u)] = x;
-    }
-    __syncthreads();
-    const int nb_ = (int)sh.n_sel, want = k - bs.c_gt;           // tau = want-th largest key of the bin
-    for (int i = threadIdx.x; i < nb_; i += blockDim.x) {
-      const uint32_t xi = sh.hist[i];
-      int gt = 0, ge = 0;
-      for (int j = 0; j < nb_; ++j) { const uint32_t xj = sh.hist[j]; gt += xj > xi; ge += xj >= xi; }
-      if (gt < want && want <= ge) sh.digit = xi;               // every such xi is the same key
-    }
-    __syncthreads();
-    tau_lo = tau_hi = f32_from_order_key(sh.digit);
-  }
-  const float knmax = __uint_as_float(a.knmax[b]);
-  const float E = a.eps_dot * sh.U * 1.0001f * knmax + 1.52587890625e-05f * fmaxf(fabsf(tau_lo), fabsf(tau_hi));
-  const float hi = tau_hi + 2.f * E, lo = tau_lo - 2.f * E;
-  uint64_t sure = 0ull, amb = 0ull;
-#pragma unroll
-  for (int e = 0; e < NPT; ++e) {
-    if (base + e >= n) continue;
-    if (v[e] > hi) { sure |= 1ull << e; }
-    else if (v[e] >= lo) {
-      amb |= 1ull << e;
-      const uint32_t slot = atomicAdd(&sh.n_amb, 1u);
-      if (slot < AMB_CAP) sh.amb[slot] = base + e;
-    }
-  }
-  int n_in_total;
-  block_excl_scan(__popcll(sure), sh.wtot, &n_in_total);
-  int n_amb = (int)sh.n_amb;
-  if (n_amb > AMB_CAP) {
-    if (threadIdx.x == 0) raise_err(a.err, CSA_DEVERR_BAND);
-    n_amb = AMB_CAP;
-  }
-  const int need = k - n_in_total;
-  rescore_block(a, sh, row, sh.amb, n_amb, sh.amb_s);
-  for (int i = threadIdx.x; i < n_amb; i += blockDim.x) {
-    const double si = sh.amb_s[i];
-    const int ii = sh.amb[i];
-    int rank = 0;
-    for (int j = 0; j < n_amb; ++j) {
-      const double sj = sh.amb_s[j];
-      rank += (sj > si) || (sj == si && sh.amb[j] < ii);
-    }
-    if (rank < need) atomicOr(&rs.chosen[ii >> 5], 1u << (ii & 31));
-  }
-  __syncthreads();
-  uint64_t sel = sure;
-#pragma unroll
-  for (int e = 0; e < NPT; ++e)
-    if ((amb >> e) & 1ull) {
-      const int i = base + e;
-      if ((rs.chosen[i >> 5] >> (i & 31)) & 1u) sel |= 1ull << e;
-    }
-  write_selected_reg<NPT>(sh, sel, k, out);
-  if (sout) {
-    // fp64 scores of the selected entries (in output order), 32 at a time
-    __syncthreads();
-    for (int base2 = 0; base2 < k; base2 += 32) {
-      const int cnt = min(32, k - base2);
-      if (threadIdx.x < cnt) sh.sel[threadIdx.x] = out[base2 + threadIdx.x];
-      __syncthreads();
-      rescore_block(a, sh, row, sh.sel, cnt, sh.amb_s);
-      if (threadIdx.x < cnt) sout[base2 + threadIdx.x] = (float)sh.amb_s[threadIdx.x];
-      __syncthreads();
-    }
-  }
-}
-
-template <int NPT>
-__global__ void __launch_bounds__(TK_THREADS)
-topk_select_reg_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_valid,
-                       int64_t n_cap, int k, int32_t* __restrict__ idx_out) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  TopkShared& sh = *reinterpret_cast<TopkShared*>(smem_raw);
-  RegShared& rs = *reinterpret_cast<RegShared*>(smem_raw + ((sizeof(TopkShared) + 15) & ~size_t(15)));
-  const int row = blockIdx.x;
-  const float* S = scores + (size_t)row * ld;
-  int n = n_valid ? n_valid[row] : (int)n_cap;
-  if ((int64_t)n > n_cap) n = (int)n_cap;
-  if (n < 0) n = 0;
-  int32_t* out = idx_out + (size_t)row * k;
-  if (n <= k) {
-    for (int i = threadIdx.x; i < k; i += blockDim.x) out[i] = i < n ? i : -1;
-    return;
-  }
-  float v[NPT];
-  load_row<NPT>(S, n, v);
-  if (threadIdx.x == 0) sh.n_amb = 0;
-  for (int i = threadIdx.x; i < (NPT * TK_THREADS + 31) / 32; i += blockDim.x) rs.chosen[i] = 0u;
-  const BinSel bs = hist_select_reg<NPT>(sh, n, k, v);
-  if (bs.c_T > AMB_CAP) {                            // heavy ties: exact multi-pass select from global memory
-    topk_select_global_row(sh, S, n, k, out);
-    return;
-  }
-  const int base = threadIdx.x * NPT;
-  uint64_t sure = 0ull, cand = 0ull;
-#pragma unroll
-  for (int e = 0; e < NPT; ++e) {
-    if (base + e >= n) continue;
-    const uint32_t x = f32_order_key(v[e]);
-    if (x > bs.key_hi) sure |= 1ull << e;
-    else if (x >= bs.key_lo) {
-      cand |= 1ull << e;
-      const uint32_t slot = atomicAdd(&sh.n_amb, 1u);
-      if (slot < AMB_CAP) { sh.amb[slot] = base + e; sh.hist[slot] = x; }
-    }
-  }
-  int n_gt;
-  block_excl_scan(__popcll(sure), sh.wtot, &n_gt);
-  const int nc = min((int)sh.n_amb, AMB_CAP), need = k - n_gt;
-  for (int c = threadIdx.x; c < nc; c += blockDim.x) {
-    const int ic = sh.amb[c];
-    const uint32_t xc = sh.hist[c];
-    int rank = 0;
-    for (int j = 0; j < nc; ++j) {
-      const uint32_t xj = sh.hist[j];
-      rank += (xj > xc) || (xj == xc && sh.amb[j] < ic);
-    }
-    if (rank < need) atomicOr(&rs.chosen[ic >> 5], 1u << (ic & 31));
-  }
-  __syncthreads();
-  uint64_t sel = sure;
-#pragma unroll
-  for (int e = 0; e < NPT; ++e)
-    if ((cand >> e) & 1ull) {
-      const int i = base + e;
-      if ((rs.chosen[i >> 5] >> (i & 31)) & 1u) sel |= 1ull << e;
-    }
-  write_selected_reg<NPT>(sh, sel, k, out);
-}
-
 static void set_smem_attr(const void* fn) {
   cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(TopkShared));
 }
 
-constexpr size_t REG_SMEM = ((sizeof(TopkShared) + 15) & ~size_t(15)) + sizeof(RegShared);
-
-template <int NPT>
-static cudaError_t launch_sel_reg(const IndexerArgs& a, cudaStream_t st) {
-  cudaFuncSetAttribute(indexer_select_reg_kernel<NPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)REG_SMEM);
-  indexer_select_reg_kernel<NPT><<<a.B * a.Tq, TK_THREADS, REG_SMEM, st>>>(a);
-  return cudaGetLastError();
-}
-
 cudaError_t launch_indexer_select(const IndexerArgs& a, cudaStream_t st) {
-  const int64_t per = (a.n_max + TK_THREADS - 1) / TK_THREADS;
-  if (per <= 16) return launch_sel_reg<16>(a, st);
-  if (per <= 32) return launch_sel_reg<32>(a, st);
-  if (per <= 36) return launch_sel_reg<36>(a, st);
+  const cudaError_t e = launch_indexer_select_cluster(a, st);
+  if (e != cudaErrorNotSupported) return e;
   set_smem_attr((const void*)indexer_select_kernel);
   indexer_select_kernel<<<a.B * a.Tq, TK_THREADS, sizeof(TopkShared), st>>>(a);
   return cudaGetLastError();
@@ -889,18 +550,8 @@ cudaError_t launch_indexer_select(const IndexerArgs& a, cudaStream_t st) {
 cudaError_t launch_topk_select(const float* scores, int64_t ld, const int32_t* n_valid, int R, int64_t n,
                                int k, int32_t* idx_out, cudaStream_t st, unsigned* err) {
   (void)err;
-  const int64_t per = (n + TK_THREADS - 1) / TK_THREADS;
-  const bool vec_ok = (ld % 4 == 0) && (((uintptr_t)scores & 15) == 0);   // float4 row loads
-  if (vec_ok && per <= 36) {
-#define CSA_TOPK_REG(NPT)                                                                              \
-    cudaFuncSetAttribute(topk_select_reg_kernel<NPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)REG_SMEM); \
-    topk_select_reg_kernel<NPT><<<R, TK_THREADS, REG_SMEM, st>>>(scores, ld, n_valid, n, k, idx_out);   \
-    return cudaGetLastError();
-    if (per <= 16) { CSA_TOPK_REG(16) }
-    if (per <= 32) { CSA_TOPK_REG(32) }
-    CSA_TOPK_REG(36)
-#undef CSA_TOPK_REG
-  }
+  const cudaError_t e = launch_topk_select_cluster(scores, ld, n_valid, R, n, k, idx_out, st);
+  if (e != cudaErrorNotSupported) return e;
   set_smem_attr((const void*)topk_select_kernel);
   topk_select_kernel<<<R, TK_THREADS, sizeof(TopkShared), st>>>(scores, ld, n_valid, n, k, idx_out);
   return cudaGetLastError();

@@ -142,7 +142,8 @@ csa_status hca_compress(const void* C, const void* Z, const float* bias,
  *            (the fp64 score of each selected entry rounded to fp32; 0 for pads)
  *   workspace >= lightning_index_workspace_size(B, Tq, n_max, k) bytes
  * Supported: B*Tq <= 65535, H_I <= 64, d_I in {32, 64, 128}, k <= 2048,
- * n_max <= 2^24.
+ * n_max <= 2^24.  qI, kI, score_out and workspace must be 16-byte aligned
+ * (CSA_ERR_ALIGN otherwise).
  * ------------------------------------------------------------------------- */
 size_t lightning_index_workspace_size(int B, int Tq, int64_t n_max, int k);
 csa_status lightning_index(const void* qI, const void* qI_scale, const float* w,

@@ -74,6 +74,8 @@ def test_indexer_validation():
     assert call(ifmt=0, qs=None, ks=None) != ERR_NULL      # fp32 operands need no scales
     assert call(wsb=16) == ERR_WS
     assert call(ws=None) == ERR_WS
+    assert call(qI=FAKE + 8) == ERR_ALIGN       # vector loads of the query and key rows
+    assert call(kI=FAKE + 4) == ERR_ALIGN
     need = N.lib.lightning_index_workspace_size(2, 3, 1000, 64)
     assert need >= 2 * 3 * 1000 * 4
 
