@@ -30,6 +30,7 @@
 // Every pass over the entries is a rolled loop: this kernel runs its code once per
 // row, and code that runs once costs its instruction fetch, so the code is kept small.
 #include "indexer.cuh"
+#include "tc.cuh"
 
 #include <algorithm>
 #include <cooperative_groups.h>
@@ -52,7 +53,7 @@ constexpr int SL_CHUNK = 34 * 1024;    // entries per CTA at most
 constexpr int SL_QPT = 8192 / SL_T;    // query-row elements per thread (H_I * d_I <= 8192)
 constexpr int SL_BAND_CT = 64;         // the indexer refines the threshold bin down to this many keys
 constexpr int SL_WORDS = SL_CHUNK / 32;
-constexpr int SL_RW = 4;               // warps that re-score band entries, 8 entries each at a time
+constexpr int SL_RR = 32;              // entries re-scored per round
 constexpr int SL_QLD = 132;            // padded row length (doubles) of the staged query / key rows
 
 struct SelFixed {
@@ -72,6 +73,7 @@ struct SelFixed {
   int goff[SL_CMAX + 1];               // start of each CTA's part in a gathered list
   uint32_t cgt, cT, tau, tlo, thi, cnt, n_sure;
   unsigned long long mult;
+  alignas(8) uint64_t ldbar;           // completion of the bulk copy of the scores
   float n2[64];
   float qsc[64 * 4];
   float w[64];
@@ -81,21 +83,13 @@ struct SelFixed {
 // Re-scoring scratch: overlays the score array once the scores have been classified.
 struct Resc {
   double qd[64 * SL_QLD];              // query row codes as fp64 (rows padded: conflict-free fragment reads)
-  double kd[SL_RW][8][SL_QLD];         // key rows being re-scored
-  double contrib[SL_RW][8][64];        // their per-head terms
-  float ksc[SL_RW][8][4];              // their scales (E4M3 row scale in [0], MXFP4 block scales)
+  double kd[SL_RR][SL_QLD];            // key rows being re-scored (one round)
+  double contrib[SL_RR][65];           // their per-head terms (rows padded)
+  float ksc[SL_RR][4];                 // their scales (E4M3 row scale in [0], MXFP4 block scales)
 };
 
 constexpr size_t SL_FIXED = (sizeof(SelFixed) + 127) & ~size_t(127);
 
-// What the exact re-scoring reads of the key side, passed by value: taking the address of
-// a kernel parameter would copy the whole argument block to local memory.
-struct RescKeys {
-  const void* kI;
-  const void* kI_scale;
-  int64_t n_max;
-  int ifmt, HI, dI;
-};
 
 __device__ __forceinline__ void sl_sync(cg::cluster_group cl, unsigned C) {
   if (C == 1) __syncthreads();
@@ -414,112 +408,124 @@ __device__ __forceinline__ void dmma_884(double& d0, double& d1, double a, doubl
                : "+d"(d0), "+d"(d1) : "d"(a), "d"(b));
 }
 
-// Exact fp64 scores of entries ids[0..cnt) (cnt <= 8), by one warp (re-scoring slot rw);
-// the query row is staged in rs.qd / sh.qsc / sh.w.  The per-head dot products of FP8 /
-// FP4 codes are exact in fp64 in any order, so they run on the fp64 tensor cores (heads x
-// entries, K = d_I, one accumulator chain per 8-head block); each head's term
-// w_j * max(D_j, 0) is formed as the definition does, and the terms are added in order
-// j = 0..H_I-1.
-__device__ __noinline__ void sl_rescore8(const RescKeys a, SelFixed& sh, Resc& rs, int rw, int b,
-                                         const int32_t* ids, int cnt, double* out) {
-  const int lane = threadIdx.x & 31;
+// What the exact re-scoring reads of the key side, passed by value: taking the address of
+// a kernel parameter would copy the whole argument block to local memory.
+struct RescKeys {
+  const void* kI;
+  const void* kI_scale;
+  int64_t n_max;
+  int HI, dI;
+};
+
+// Exact fp64 scores of entries ids[0..cnt) (cnt <= SL_RR) into out[0..cnt), by the whole
+// CTA (all threads call; barriers inside).  The query row is staged in rs.qd / sh.qsc /
+// sh.w.  The per-head dot products of FP8 / FP4 codes are exact in fp64 in any order, so
+// they run on the fp64 tensor cores: every warp takes (8 entries x 8 heads) tiles over
+// K = d_I.  Each head's term w_j * max(D_j, 0) is formed as the definition does, and the
+// terms are added in order j = 0..H_I-1.
+template <int F>
+__device__ __noinline__ void sl_rescore_round(const RescKeys a, SelFixed& sh, Resc& rs, int b, const int32_t* ids,
+                                              int cnt, double* out) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int HI = a.HI, dI = a.dI, nb = dI / 32;
-  // key rows (zeros past cnt): all loads first.  Lane l holds elements [4l, 4l+4) (E4M3,
-  // fp32) or [8l, 8l+8) (MXFP4) of each row (row starts are 16-byte aligned).
-  const bool lane_in = (a.ifmt == CSA_IFMT_MXFP4) ? lane * 8 < dI : lane * 4 < dI;
-  uint4 raw[8];
-  float scl[8];
+  // ---- key rows (zeros past cnt): element idx = tid + SL_T*u is (entry idx / d_I,
+  // dim idx % d_I); all loads first, then consecutive threads store consecutive doubles
+  const int lgd = __ffs(dI) - 1;
+  float xv[SL_RR * 128 / SL_T];
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    raw[c] = make_uint4(0u, 0u, 0u, 0u);
-    scl[c] = 0.f;
+  for (int u = 0; u < SL_RR * 128 / SL_T; ++u) {
+    const int idx = tid + SL_T * u;
+    const int c = idx >> lgd, d = idx & (dI - 1);
+    xv[u] = 0.f;
     if (c < cnt) {
       const size_t koff = (size_t)b * a.n_max + ids[c];
-      if (lane_in) {
-        if (a.ifmt == CSA_IFMT_E4M3) raw[c].x = reinterpret_cast<const uint32_t*>((const uint8_t*)a.kI + koff * dI)[lane];
-        else if (a.ifmt == CSA_IFMT_MXFP4) raw[c].x = reinterpret_cast<const uint32_t*>((const uint8_t*)a.kI + koff * (dI / 2))[lane];
-        else raw[c] = reinterpret_cast<const uint4*>((const float*)a.kI + koff * dI)[lane];
-      }
-      if (a.ifmt == CSA_IFMT_E4M3) scl[c] = ((const float*)a.kI_scale)[koff];
-      else if (a.ifmt == CSA_IFMT_MXFP4 && lane < nb) scl[c] = ue8m0_to_float(((const uint8_t*)a.kI_scale)[koff * nb + lane]);
+      if (F == CSA_IFMT_E4M3) xv[u] = e4m3_to_float(((const uint8_t*)a.kI)[koff * dI + d]);
+      else if (F == CSA_IFMT_MXFP4) {
+        const uint8_t byte = ((const uint8_t*)a.kI)[koff * (dI / 2) + (d >> 1)];
+        xv[u] = e2m1_to_float((d & 1) ? (byte >> 4) : (byte & 0xF));
+      } else xv[u] = ((const float*)a.kI)[koff * dI + d];
+    }
+  }
+  float scl = 0.f;
+  const int nsc = (F == CSA_IFMT_MXFP4) ? nb : 1;
+  if (tid < SL_RR * nsc) {
+    const int c = tid / nsc, q = tid - c * nsc;
+    if (c < cnt) {
+      const size_t koff = (size_t)b * a.n_max + ids[c];
+      if (F == CSA_IFMT_E4M3) scl = ((const float*)a.kI_scale)[koff];
+      if (F == CSA_IFMT_MXFP4) scl = ue8m0_to_float(((const uint8_t*)a.kI_scale)[koff * nb + q]);
     }
   }
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    double* kd = rs.kd[rw][c];
-    if (lane_in) {
-      if (a.ifmt == CSA_IFMT_E4M3) {
-        for (int e = 0; e < 4; ++e) kd[lane * 4 + e] = (double)e4m3_to_float((raw[c].x >> (8 * e)) & 0xFFu);
-      } else if (a.ifmt == CSA_IFMT_MXFP4) {
-        for (int e = 0; e < 8; ++e) kd[lane * 8 + e] = (double)e2m1_to_float((raw[c].x >> (4 * e)) & 0xFu);
-      } else {
-        kd[lane * 4] = (double)__uint_as_float(raw[c].x); kd[lane * 4 + 1] = (double)__uint_as_float(raw[c].y);
-        kd[lane * 4 + 2] = (double)__uint_as_float(raw[c].z); kd[lane * 4 + 3] = (double)__uint_as_float(raw[c].w);
-      }
-    }
-    if (a.ifmt == CSA_IFMT_E4M3 && lane == 0) rs.ksc[rw][c][0] = scl[c];
-    if (a.ifmt == CSA_IFMT_MXFP4 && lane < nb) rs.ksc[rw][c][lane] = scl[c];
+  for (int u = 0; u < SL_RR * 128 / SL_T; ++u) {
+    const int idx = tid + SL_T * u;
+    if (idx < SL_RR * dI) rs.kd[idx >> lgd][idx & (dI - 1)] = (double)xv[u];
   }
-  __syncwarp();
+  if (tid < SL_RR * nsc) rs.ksc[tid / nsc][tid % nsc] = scl;
+  __syncthreads();
+  // ---- (8 entries x 8 heads) tiles: tile = (group, head block)
   const int g = lane >> 2, t = lane & 3;
-  const double* brow = rs.kd[rw][g];           // B[k][n]: entry n = g, dim k = t of each step
-  const int n_blk = (a.ifmt == CSA_IFMT_MXFP4) ? nb : 1;     // scale blocks along K
+  const int n_hb = (HI + 7) / 8, n_grp = (cnt + 7) / 8;
+  const int n_blk = (F == CSA_IFMT_MXFP4) ? nb : 1;
   const int ks_blk = dI / 4 / n_blk;
-  double D[8][2];
-#pragma unroll
-  for (int h = 0; h < 8; ++h) D[h][0] = D[h][1] = 0.0;
-  for (int bb = 0; bb < n_blk; ++bb) {
-    double P[8][2];
-#pragma unroll
-    for (int h = 0; h < 8; ++h) P[h][0] = P[h][1] = 0.0;
-    for (int ks = bb * ks_blk; ks < (bb + 1) * ks_blk; ++ks) {
-      const double bf = brow[4 * ks + t];
-#pragma unroll
-      for (int h = 0; h < 8; ++h) dmma_884(P[h][0], P[h][1], rs.qd[(8 * h + g) * SL_QLD + 4 * ks + t], bf);
-    }
-    if (a.ifmt == CSA_IFMT_MXFP4) {
-#pragma unroll
-      for (int h = 0; h < 8; ++h) {
-        const int j = 8 * h + g;
+  for (int tile = warp; tile < n_grp * n_hb; tile += SL_W) {
+    const int grp = tile / n_hb, hb = tile - grp * n_hb;
+    const double* arow = rs.qd + (8 * hb + g) * SL_QLD;      // A[m][k]: head 8hb+g, dim k = t
+    const double* brow = rs.kd[8 * grp + g];                 // B[k][n]: entry 8grp+g, dim k = t
+    const int j = 8 * hb + g;
+    const int c0 = 8 * grp + 2 * t;
+    double D0 = 0.0, D1 = 0.0;
+    for (int bb = 0; bb < n_blk; ++bb) {
+      double P0 = 0.0, P1 = 0.0, Q0 = 0.0, Q1 = 0.0;         // two chains: even / odd k-steps
+      const int k0 = bb * ks_blk;
+#pragma unroll 4
+      for (int ks = 0; ks < ks_blk; ks += 2) {
+        dmma_884(P0, P1, arow[4 * (k0 + ks) + t], brow[4 * (k0 + ks) + t]);
+        dmma_884(Q0, Q1, arow[4 * (k0 + ks + 1) + t], brow[4 * (k0 + ks + 1) + t]);
+      }
+      P0 += Q0;                                              // exact: all partial sums are
+      P1 += Q1;                                              // multiples of the code grid
+      if (F == CSA_IFMT_MXFP4) {
         const double qs = (j < HI) ? (double)sh.qsc[j * nb + bb] : 0.0;
-        D[h][0] += (qs * (double)rs.ksc[rw][2 * t][bb]) * P[h][0];
-        D[h][1] += (qs * (double)rs.ksc[rw][2 * t + 1][bb]) * P[h][1];
+        D0 += (qs * (double)rs.ksc[c0][bb]) * P0;
+        D1 += (qs * (double)rs.ksc[c0 + 1][bb]) * P1;
+      } else {
+        D0 = P0;
+        D1 = P1;
       }
-    } else {
-#pragma unroll
-      for (int h = 0; h < 8; ++h) { D[h][0] = P[h][0]; D[h][1] = P[h][1]; }
     }
-  }
-#pragma unroll
-  for (int h = 0; h < 8; ++h) {
-    const int j = 8 * h + g;
     if (j < HI) {
-      double d0 = D[h][0], d1 = D[h][1];
-      if (a.ifmt == CSA_IFMT_E4M3) {
-        d0 = ((double)sh.qsc[j] * (double)rs.ksc[rw][2 * t][0]) * d0;
-        d1 = ((double)sh.qsc[j] * (double)rs.ksc[rw][2 * t + 1][0]) * d1;
+      if (F == CSA_IFMT_E4M3) {
+        D0 = ((double)sh.qsc[j] * (double)rs.ksc[c0][0]) * D0;
+        D1 = ((double)sh.qsc[j] * (double)rs.ksc[c0 + 1][0]) * D1;
       }
-      rs.contrib[rw][2 * t][j] = (double)sh.w[j] * fmax(d0, 0.0);
-      rs.contrib[rw][2 * t + 1][j] = (double)sh.w[j] * fmax(d1, 0.0);
+      rs.contrib[c0][j] = (double)sh.w[j] * fmax(D0, 0.0);
+      rs.contrib[c0 + 1][j] = (double)sh.w[j] * fmax(D1, 0.0);
     }
   }
-  __syncwarp();
-  if (lane < cnt) {
+  __syncthreads();
+  // ---- head terms added in order, one thread per entry
+  if (tid < cnt) {
+    const double* cr = rs.contrib[tid];
     double S = 0.0;
-    for (int j = 0; j < HI; ++j) S += rs.contrib[rw][lane][j];
-    out[lane] = S;
+    int j = 0;
+    for (; j + 8 <= HI; j += 8) {
+      double v[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = cr[j + q];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) S += v[q];
+    }
+    for (; j < HI; ++j) S += cr[j];
+    out[tid] = S;
   }
-  __syncwarp();
+  __syncthreads();
 }
 
-// Exact scores of ids[0..n) into out[0..n): warps 0..SL_RW-1 take groups of 8.  All
-// threads of the CTA call (the function ends with a CTA barrier).
-__device__ __noinline__ void sl_rescore_list(const RescKeys a, SelFixed& sh, Resc& rs, int b, const int32_t* ids, int n,
-                                double* out) {
-  const int warp = threadIdx.x >> 5;
-  if (warp < SL_RW)
-    for (int g0 = warp * 8; g0 < n; g0 += SL_RW * 8) sl_rescore8(a, sh, rs, warp, b, ids + g0, min(8, n - g0), out + g0);
-  __syncthreads();
+template <int F>
+__device__ __forceinline__ void sl_rescore_list(const RescKeys a, SelFixed& sh, Resc& rs, int b, const int32_t* ids,
+                                                int n, double* out) {
+  for (int c0 = 0; c0 < n; c0 += SL_RR) sl_rescore_round<F>(a, sh, rs, b, ids + c0, min(SL_RR, n - c0), out + c0);
 }
 
 // Stage the query row codes (held in registers, element tid + SL_T*e) as fp64:
@@ -536,6 +542,7 @@ __device__ __forceinline__ void sl_stage_query(Resc& rs, const float (&qx)[SL_QP
   for (int i = total + tid; i < hpad * dI; i += SL_T) rs.qd[(i >> lgd) * SL_QLD + (i & (dI - 1))] = 0.0;
 }
 
+template <int F>
 __global__ void __launch_bounds__(SL_T, 1)
 indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -552,9 +559,26 @@ indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
   const int n = row_eligible(a, row);
   int32_t* out = a.idx_out + (size_t)row * k;
   float* sout = a.score_out ? a.score_out + (size_t)row * k : nullptr;
-  const RescKeys rk{a.kI, a.kI_scale, a.n_max, a.ifmt, a.H_I, a.d_I};
+  const RescKeys rk{a.kI, a.kI_scale, a.n_max, a.H_I, a.d_I};
   const int lo = (int)r * chunk;
   const int m = max(0, min(n - lo, chunk));
+  // ---- this CTA's scores: one bulk copy into shared memory (the tail by plain loads)
+  const int m4 = (n > k) ? (m & ~3) : 0;
+  const float* srow = a.scores + (size_t)row * a.ld + lo;
+  if (tid == 0) {
+    tc::mbar_init(&sh.ldbar, 1);
+    tc::fence_mbar_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    tc::mbar_arrive_expect_tx(&sh.ldbar, (uint32_t)m4 * 4u);
+    for (int o = 0; o < m4; o += 8192) {
+      const uint32_t bytes = (uint32_t)min(8192, m4 - o) * 4u;
+      asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                   ::"r"(tc::smem_u32(sv + o)), "l"(srow + o), "r"(bytes), "r"(tc::smem_u32(&sh.ldbar)) : "memory");
+    }
+  }
+  if (n > k && tid < m - m4) sv[m4 + tid] = srow[m4 + tid];
   // ---- the query row: codes into registers (staged into shared memory once the scores
   // are classified), scales and weights, and U = sum_j w_j ||q_j|| for the error bound
   const int total = HI * dI, lgd = __ffs(dI) - 1;
@@ -565,8 +589,8 @@ indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
     const int i = tid + SL_T * e;
     qx[e] = 0.f;
     if (i < total) {
-      if (a.ifmt == CSA_IFMT_E4M3) qx[e] = e4m3_to_float(((const uint8_t*)a.qI)[r0 + i]);
-      else if (a.ifmt == CSA_IFMT_MXFP4) {
+      if (F == CSA_IFMT_E4M3) qx[e] = e4m3_to_float(((const uint8_t*)a.qI)[r0 + i]);
+      else if (F == CSA_IFMT_MXFP4) {
         const uint8_t byte = ((const uint8_t*)a.qI)[(r0 + i) >> 1];
         qx[e] = e2m1_to_float((i & 1) ? (byte >> 4) : (byte & 0xF));
       } else qx[e] = ((const float*)a.qI)[r0 + i];
@@ -575,28 +599,42 @@ indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
   if (tid < HI) {
     sh.w[tid] = a.w[(size_t)row * HI + tid];
     sh.n2[tid] = 0.f;
-    if (a.ifmt == CSA_IFMT_E4M3) sh.qsc[tid] = ((const float*)a.qI_scale)[(size_t)row * HI + tid];
-    if (a.ifmt == CSA_IFMT_MXFP4)
+    if (F == CSA_IFMT_E4M3) sh.qsc[tid] = ((const float*)a.qI_scale)[(size_t)row * HI + tid];
+    if (F == CSA_IFMT_MXFP4)
       for (int bb = 0; bb < nb; ++bb)
         sh.qsc[tid * nb + bb] = ue8m0_to_float(((const uint8_t*)a.qI_scale)[((size_t)row * HI + tid) * nb + bb]);
   }
   const float knmax = __uint_as_float(a.knmax[b]);
   // the key range the scoring kernel recorded (exact min / max over the row's eligible entries)
   uint32_t lo_k = ~a.keyrange[2 * (size_t)row + 1], hi_k = a.keyrange[2 * (size_t)row];
-  if (n > k) sl_load(a.scores + (size_t)row * a.ld + lo, m, true, sv);
   __syncthreads();
-  // squared norms per head: a warp's 32 elements of one e lie in one head (d_I >= 32)
+  // squared norms per head: a warp's 32 elements of one e lie in one head (d_I >= 32);
+  // the sixteen warp sums are independent, then one atomic each
+  {
+    float s2[SL_QPT];
 #pragma unroll
-  for (int e = 0; e < SL_QPT; ++e) {
-    const int i = tid + SL_T * e;
-    float x = qx[e];
-    if (i < total) {
-      const int j = i >> lgd;
-      if (a.ifmt == CSA_IFMT_E4M3) x *= sh.qsc[j];
-      if (a.ifmt == CSA_IFMT_MXFP4) x *= sh.qsc[j * nb + ((i & (dI - 1)) >> 5)];
+    for (int e = 0; e < SL_QPT; ++e) {
+      const int i = tid + SL_T * e;
+      float x = qx[e];
+      if (i < total) {
+        const int j = i >> lgd;
+        if (F == CSA_IFMT_E4M3) x *= sh.qsc[j];
+        if (F == CSA_IFMT_MXFP4) x *= sh.qsc[j * nb + ((i & (dI - 1)) >> 5)];
+      }
+      s2[e] = x * x;
     }
-    const float s2 = warp_sum(x * x);
-    if (lane == 0 && i < total) atomicAdd(&sh.n2[i >> lgd], s2);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+      for (int e = 0; e < SL_QPT; ++e) s2[e] += __shfl_xor_sync(0xffffffffu, s2[e], o);
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int e = 0; e < SL_QPT; ++e) {
+        const int i = tid + SL_T * e;
+        if (i < total) atomicAdd(&sh.n2[i >> lgd], s2[e]);
+      }
+    }
   }
   __syncthreads();
   if (warp == 0) {
@@ -605,13 +643,17 @@ indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
     u = warp_sum(u);
     if (lane == 0) sh.U = u;
   }
-  // (sh.U is read after the barriers of the threshold search)
+  // the scores have landed (bounded wait; on a timeout the error word is set)
+  if (n > k && m4 > 0) {
+    const bool ok = tc::mbar_wait(&sh.ldbar, 0);
+    if (!ok && tid == 0) raise_err(a.err, CSA_DEVERR_TIMEOUT);
+  }
+  __syncthreads();
   if (n <= k) {
     // every eligible entry is selected; CTA r scores the slots [r*k/C, (r+1)*k/C)
     if (r == 0)
       for (int i = tid; i < k; i += SL_T) out[i] = i < n ? i : -1;
     if (sout) {
-      __syncthreads();
       sl_stage_query(rs, qx, total, lgd, HI, dI);
       const int s0 = (int)((int64_t)k * r / C), s1 = (int)((int64_t)k * (r + 1) / C);
       for (int c0 = s0; c0 < s1; c0 += SL_CAP) {
@@ -619,7 +661,7 @@ indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
         __syncthreads();
         for (int i = tid; i < cnt; i += SL_T) sh.band_id[i] = min(c0 + i, max(n - 1, 0));
         __syncthreads();
-        sl_rescore_list(rk, sh, rs, b, sh.band_id, cnt, sh.band_s);
+        sl_rescore_list<F>(rk, sh, rs, b, sh.band_id, cnt, sh.band_s);
         for (int i = tid; i < cnt; i += SL_T) sout[c0 + i] = (c0 + i < n) ? (float)sh.band_s[i] : 0.f;
       }
     }
@@ -656,9 +698,8 @@ indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
   const int n_band = (int)min(nb_raw, (uint32_t)SL_CAP);
   if (nb_raw > (uint32_t)SL_CAP && tid == 0) raise_err(a.err, CSA_DEVERR_BAND);
   sl_stage_query(rs, qx, total, lgd, HI, dI);
-  __syncthreads();
-  // ---- exact scores of this CTA's band entries
-  sl_rescore_list(rk, sh, rs, b, sh.band_id, n_band, sh.band_s);
+  // ---- exact scores of this CTA's band entries (the first round's barrier covers the staging)
+  sl_rescore_list<F>(rk, sh, rs, b, sh.band_id, n_band, sh.band_s);
   if (tid == 0) { sh.pub[0] = sh.n_sure; sh.pub[1] = (uint32_t)n_band; }
   sl_sync(cluster, C);
   // ---- gather every CTA's band and rank all of it (each CTA reaches the same verdicts)
@@ -707,7 +748,7 @@ indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
       __syncthreads();
       for (int i = tid; i < cnt; i += SL_T) sh.gband_id[i] = out[c0 + i];
       __syncthreads();
-      sl_rescore_list(rk, sh, rs, b, sh.gband_id, cnt, sh.gband_s);
+      sl_rescore_list<F>(rk, sh, rs, b, sh.gband_id, cnt, sh.gband_s);
       for (int i = tid; i < cnt; i += SL_T) sout[c0 + i] = (float)sh.gband_s[i];
     }
     if (r == 0)
@@ -778,7 +819,9 @@ cudaError_t launch_indexer_select_cluster(const IndexerArgs& a, cudaStream_t st)
       ((uintptr_t)a.scores & 15) != 0 || (int64_t)rows * C > 0x7fffffffLL)
     return cudaErrorNotSupported;
   const size_t region = std::max((size_t)chunk * 4, sizeof(Resc));
-  return sl_launch(indexer_select_cluster_kernel, rows, C, SL_FIXED + region, st, a, chunk);
+  if (a.ifmt == CSA_IFMT_E4M3) return sl_launch(indexer_select_cluster_kernel<CSA_IFMT_E4M3>, rows, C, SL_FIXED + region, st, a, chunk);
+  if (a.ifmt == CSA_IFMT_MXFP4) return sl_launch(indexer_select_cluster_kernel<CSA_IFMT_MXFP4>, rows, C, SL_FIXED + region, st, a, chunk);
+  return sl_launch(indexer_select_cluster_kernel<CSA_IFMT_F32>, rows, C, SL_FIXED + region, st, a, chunk);
 }
 
 cudaError_t launch_topk_select_cluster(const float* scores, int64_t ld, const int32_t* n_valid, int R, int64_t n,
