@@ -9,8 +9,9 @@
 // entries [r*chunk, (r+1)*chunk) in shared memory.  The CTAs combine their partial
 // results through distributed shared memory:
 //  1. the key range [kmin, kmax] of the row (monotone fp32 order keys);
-//  2. 2048-bin histograms whose bins split the current key range evenly (a multiply
-//     and a shift per key, monotone in the key); the bin holding the k-th largest key
+//  2. 2048-bin histograms over the current key range [lo, hi]: bin = (key - lo) >> s
+//     with the smallest s that fits (at least half the bins are in use; no division);
+//     the bin holding the k-th largest key
 //     becomes the next range until it holds at most SL_CAP keys or one key value;
 //  3. topk_select: the keys of that bin, gathered by every CTA, give the exact k-th
 //     largest fp32 key tau (lightning_index refines the bin to at most 64 keys and
@@ -72,9 +73,7 @@ struct SelFixed {
   uint32_t pcnt[SL_CMAX][2];
   int goff[SL_CMAX + 1];               // start of each CTA's part in a gathered list
   uint32_t cgt, cT, tau, tlo, thi, cnt, n_sure;
-  unsigned long long mult;
   alignas(8) uint64_t ldbar;           // completion of the bulk copy of the scores
-  float n2[64];
   float qsc[64 * 4];
   float w[64];
   float U;
@@ -193,13 +192,14 @@ __device__ __forceinline__ void sl_refine(SelFixed& sh, const float* sv, int m, 
   for (int round = 0; round < 6; ++round) {
     uint32_t* H = sh.hist[round & 1];
     reinterpret_cast<uint4*>(H)[tid] = make_uint4(0u, 0u, 0u, 0u);   // 4 bins per thread
-    if (tid == 0) sh.mult = (hi - lo) < (uint32_t)SL_BINS ? 0ull : (1ull << 43) / ((uint64_t)(hi - lo) + 1ull);
+    // bins of 2^sh keys: the smallest shift with (hi - lo) >> sh < SL_BINS
+    const int range_bits = 32 - __clz(hi - lo);              // 0 when lo == hi
+    const int shf = range_bits > 11 ? range_bits - 11 : 0;
     __syncthreads();
-    const uint32_t mult = (uint32_t)sh.mult;              // < 2^32 whenever it is used
 #pragma unroll 4
     for (int i = tid; i < m; i += SL_T) {
       const uint32_t x = f32_order_key(sv[i]);
-      if (x >= lo && x <= hi) atomicAdd(&H[mult ? __umulhi(x - lo, mult) : x - lo], 1u);
+      if (x >= lo && x <= hi) atomicAdd(&H[(x - lo) >> shf], 1u);
     }
     sl_sync(cluster, C);
     uint4 hb = make_uint4(0u, 0u, 0u, 0u);
@@ -229,17 +229,10 @@ __device__ __forceinline__ void sl_refine(SelFixed& sh, const float* sv, int m, 
       after += cb[q];
     }
     if (bin >= 0) {
-      // key bounds of bin T (one thread does the 64-bit divisions)
-      const uint64_t T = (uint64_t)bin, M = sh.mult;
-      if (!M) {
-        sh.tlo = sh.thi = lo + (uint32_t)T;
-      } else {
-        // bin T holds the keys x - lo in [ceil(T 2^32 / M), ceil((T+1) 2^32 / M) - 1]
-        const uint64_t a0 = ((T << 32) + M - 1) / M, a1 = (((T + 1) << 32) + M - 1) / M;
-        sh.tlo = lo + (uint32_t)a0;
-        const uint64_t top = (uint64_t)lo + a1 - 1;
-        sh.thi = top < (uint64_t)hi ? (uint32_t)top : hi;
-      }
+      // key bounds of bin T
+      sh.tlo = lo + ((uint32_t)bin << shf);
+      const uint64_t top = (uint64_t)sh.tlo + ((1ull << shf) - 1ull);
+      sh.thi = top < (uint64_t)hi ? (uint32_t)top : hi;
     }
     __syncthreads();
     want -= (int)sh.cgt;
@@ -598,7 +591,6 @@ indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
   }
   if (tid < HI) {
     sh.w[tid] = a.w[(size_t)row * HI + tid];
-    sh.n2[tid] = 0.f;
     if (F == CSA_IFMT_E4M3) sh.qsc[tid] = ((const float*)a.qI_scale)[(size_t)row * HI + tid];
     if (F == CSA_IFMT_MXFP4)
       for (int bb = 0; bb < nb; ++bb)
@@ -608,40 +600,56 @@ indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
   // the key range the scoring kernel recorded (exact min / max over the row's eligible entries)
   uint32_t lo_k = ~a.keyrange[2 * (size_t)row + 1], hi_k = a.keyrange[2 * (size_t)row];
   __syncthreads();
-  // squared norms per head: a warp's 32 elements of one e lie in one head (d_I >= 32);
-  // the sixteen warp sums are independent, then one atomic each
+  // U = sum_j w_j ||q_j||: warp w takes heads w, w + SL_W, ...; lane l holds elements
+  // [epl*l, epl*l + epl) of the head (one 4- or 16-byte load, issued together)
+  if (tid == 0) sh.U = 0.f;
   {
-    float s2[SL_QPT];
+    constexpr int EPL = (F == CSA_IFMT_MXFP4) ? 8 : 4;
+    float uw = 0.f;
+    uint4 qv[64 / SL_W];
 #pragma unroll
-    for (int e = 0; e < SL_QPT; ++e) {
-      const int i = tid + SL_T * e;
-      float x = qx[e];
-      if (i < total) {
-        const int j = i >> lgd;
-        if (F == CSA_IFMT_E4M3) x *= sh.qsc[j];
-        if (F == CSA_IFMT_MXFP4) x *= sh.qsc[j * nb + ((i & (dI - 1)) >> 5)];
+    for (int h = 0; h < 64 / SL_W; ++h) {
+      const int j = warp + SL_W * h;
+      qv[h] = make_uint4(0u, 0u, 0u, 0u);
+      if (j < HI && lane * EPL < dI) {
+        const size_t e0 = r0 + (size_t)j * dI + lane * EPL;
+        if (F == CSA_IFMT_E4M3) qv[h].x = *reinterpret_cast<const uint32_t*>((const uint8_t*)a.qI + e0);
+        else if (F == CSA_IFMT_MXFP4) qv[h].x = *reinterpret_cast<const uint32_t*>((const uint8_t*)a.qI + e0 / 2);
+        else qv[h] = *reinterpret_cast<const uint4*>((const float*)a.qI + e0);
       }
-      s2[e] = x * x;
+    }
+    float n2[64 / SL_W];
+#pragma unroll
+    for (int h = 0; h < 64 / SL_W; ++h) {
+      const int j = warp + SL_W * h;
+      float acc = 0.f;
+      if (j < HI && lane * EPL < dI) {
+        if (F == CSA_IFMT_E4M3) {
+          for (int e = 0; e < 4; ++e) { const float x = e4m3_to_float((qv[h].x >> (8 * e)) & 0xFFu); acc = fmaf(x, x, acc); }
+          acc *= sh.qsc[j] * sh.qsc[j];
+        } else if (F == CSA_IFMT_MXFP4) {
+          for (int e = 0; e < 8; ++e) { const float x = e2m1_to_float((qv[h].x >> (4 * e)) & 0xFu); acc = fmaf(x, x, acc); }
+          const float sc = sh.qsc[j * nb + (lane * 8) / 32];
+          acc *= sc * sc;
+        } else {
+          acc = __uint_as_float(qv[h].x) * __uint_as_float(qv[h].x) + __uint_as_float(qv[h].y) * __uint_as_float(qv[h].y) +
+                __uint_as_float(qv[h].z) * __uint_as_float(qv[h].z) + __uint_as_float(qv[h].w) * __uint_as_float(qv[h].w);
+        }
+      }
+      n2[h] = acc;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
 #pragma unroll
-      for (int e = 0; e < SL_QPT; ++e) s2[e] += __shfl_xor_sync(0xffffffffu, s2[e], o);
+      for (int h = 0; h < 64 / SL_W; ++h) n2[h] += __shfl_xor_sync(0xffffffffu, n2[h], o);
     }
-    if (lane == 0) {
 #pragma unroll
-      for (int e = 0; e < SL_QPT; ++e) {
-        const int i = tid + SL_T * e;
-        if (i < total) atomicAdd(&sh.n2[i >> lgd], s2[e]);
-      }
+    for (int h = 0; h < 64 / SL_W; ++h) {
+      const int j = warp + SL_W * h;
+      if (j < HI) uw += sh.w[j] * sqrtf(n2[h]);
     }
-  }
-  __syncthreads();
-  if (warp == 0) {
-    float u = 0.f;
-    for (int j = lane; j < HI; j += 32) u += sh.w[j] * sqrtf(sh.n2[j]);
-    u = warp_sum(u);
-    if (lane == 0) sh.U = u;
+    __syncthreads();                                       // sh.U = 0 is visible
+    if (lane == 0) atomicAdd(&sh.U, uw);
   }
   // the scores have landed (bounded wait; on a timeout the error word is set)
   if (n > k && m4 > 0) {
@@ -703,10 +711,17 @@ indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
   if (tid == 0) { sh.pub[0] = sh.n_sure; sh.pub[1] = (uint32_t)n_band; }
   sl_sync(cluster, C);
   // ---- gather every CTA's band and rank all of it (each CTA reaches the same verdicts)
-  sl_gather_offsets(sh, cluster, C, 1);
-  __syncthreads();
-  const int ng = sl_gather(sh, cluster, C, sh.band_id, sh.gband_id, SL_CAP);
-  sl_gather(sh, cluster, C, sh.band_s, sh.gband_s, SL_CAP);
+  int ng = n_band;
+  const int32_t* gid = sh.band_id;
+  const double* gsc = sh.band_s;
+  if (C > 1) {
+    sl_gather_offsets(sh, cluster, C, 1);
+    __syncthreads();
+    ng = sl_gather(sh, cluster, C, sh.band_id, sh.gband_id, SL_CAP);
+    sl_gather(sh, cluster, C, sh.band_s, sh.gband_s, SL_CAP);
+    gid = sh.gband_id;
+    gsc = sh.gband_s;
+  }
   int all_sure = 0;
   for (int p = 0; p < (int)C; ++p) all_sure += (int)sl_peer(cluster, sh.pub, 0, p);
   if (tid < SL_CMAX) {
@@ -716,12 +731,12 @@ indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
   __syncthreads();
   const int need = k - all_sure;
   for (int i = tid; i < ng; i += SL_T) {
-    const double si = sh.gband_s[i];
-    const int ii = sh.gband_id[i];
+    const double si = gsc[i];
+    const int ii = gid[i];
     int rank = 0;
     for (int j = 0; j < ng; ++j) {
-      const double sj = sh.gband_s[j];
-      rank += (sj > si) || (sj == si && sh.gband_id[j] < ii);
+      const double sj = gsc[j];
+      rank += (sj > si) || (sj == si && gid[j] < ii);
     }
     if (rank < need) {
       const int owner = ii / chunk;
