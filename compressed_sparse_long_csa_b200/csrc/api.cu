@@ -234,9 +234,9 @@ static csa_status run_attention(AttnArgs& a, int dtype, void* workspace, size_t 
   a.splits = (int)((rows + a.rows_per_split - 1) / a.rows_per_split);
   if (a.splits < 1) a.splits = 1;
   a.part = (float*)workspace;
-  bool used = false;
+  bool used = false, combined = false;
   cudaError_t e = cudaSuccess;
-  if (tc) e = launch_attention_tc(a, st, &used);
+  if (tc) e = launch_attention_tc(a, st, &used, &combined);
   if (e != cudaSuccess) return CSA_ERR_CUDA;
   if (!used) {
     if (tc) {  // the tensor-core path declined: recompute the split plan for the CUDA-core path
@@ -246,7 +246,7 @@ static csa_status run_attention(AttnArgs& a, int dtype, void* workspace, size_t 
     e = launch_attention_cuda_core(a, dtype, st);
     if (e != cudaSuccess) return CSA_ERR_CUDA;
   }
-  if (a.splits > 1) return cuda_status(launch_attn_combine(a, dtype, st));
+  if (a.splits > 1 && !combined) return cuda_status(launch_attn_combine(a, dtype, st));
   return CSA_OK;
 }
 

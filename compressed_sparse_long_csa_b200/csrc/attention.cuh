@@ -27,6 +27,7 @@ struct AttnArgs {
   int splits;
   int rows_per_split;
   int n_seg_a;                // virtual rows in segment A (k or n_max)
+  int cluster_combine;        // tensor-core path: splits merged inside a thread-block cluster
   unsigned* err;
 };
 
@@ -114,7 +115,7 @@ int attn_choose_splits(int n_queries, int H, int64_t rows, bool tc_path);
 int attn_rows_per_split(int64_t rows, int splits, bool tc_path);
 
 cudaError_t launch_attention_cuda_core(AttnArgs a, int dtype, cudaStream_t st);
-cudaError_t launch_attention_tc(AttnArgs a, cudaStream_t st, bool* used);
+cudaError_t launch_attention_tc(AttnArgs a, cudaStream_t st, bool* used, bool* combined);
 cudaError_t launch_attn_combine(const AttnArgs& a, int dtype, cudaStream_t st);
 
 }  // namespace csa

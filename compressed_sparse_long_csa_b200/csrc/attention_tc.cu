@@ -20,12 +20,18 @@
 //   3. softmax threads (one per head, TMEM lanes 16-31) run an online softmax with a
 //      lazily raised running max and write P (bf16) to shared memory;
 //   4. O += P V (M=64, N=2x256, K=64; V is read MN-major from the same tile).
-// At the end, threads of TMEM lanes 0-15 normalise O (one split) or write a split
-// partial (o, m, l) for attn_combine.  Every wait is bounded (CSA_DEVERR_TIMEOUT).
+// At the end, threads of TMEM lanes 0-15 normalise O (one split), or the split partials
+// (o, m, l) are merged: the CTAs of one query's head half form a thread-block cluster,
+// stage their partials in shared memory and each merges a slice of the heads from all
+// of them through distributed shared memory (at most 8 splits), else the partials go to
+// global memory for attn_combine.  Every wait is bounded (CSA_DEVERR_TIMEOUT).
 #include "attention.cuh"
 #include "tc.cuh"
 
+#include <cooperative_groups.h>
 #include <cudaTypedefs.h>
+#include <map>
+#include <mutex>
 
 namespace csa {
 
@@ -41,6 +47,7 @@ constexpr int AT_THREADS = 5 * 32 + 2 * AT_GROUP;   // 4 softmax warps, 1 MMA wa
 constexpr float AT_RESCALE_THRESH = 8.0f;
 constexpr int ATOM = AT_ROWS * 128;      // one 64-row x 128-byte swizzle atom
 constexpr unsigned long long NO_RUN = ~0ull;
+constexpr int OST_LD = 516;              // staged partial row: 512 values + pad (16-byte aligned rows)
 
 struct AtSmem {
   alignas(1024) uint8_t q[AT_ATOMS][AT_HC * 128];          // 72 KB
@@ -100,7 +107,7 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   AtSmem& sm = *reinterpret_cast<AtSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = blockIdx.x >> 1, hh = blockIdx.x & 1;
+  const int hh = blockIdx.x / a.splits, split = blockIdx.x - hh * a.splits;   // a cluster spans the splits
   const int row = blockIdx.y;                       // query row b*Tq + t
   const int64_t nrows = attn_virtual_rows(a);
   const int64_t v0 = (int64_t)split * a.rows_per_split;
@@ -393,6 +400,31 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
         }
       }
       if (a.lse && !is_s) a.lse[(size_t)row * AT_H + h] = den > 0.f ? M + logf(den) : -INFINITY;
+    } else if (a.cluster_combine) {
+      // stage the partial in shared memory (the KV stages are idle: every PV has completed)
+      float* ost = reinterpret_cast<float*>(&sm.kv[0][0][0]);
+      float* ost_ml = ost + AT_HC * OST_LD;
+#pragma unroll 1
+      for (int c = 0; c < 512 / 64; ++c) {
+        uint32_t v[64];
+        if (have_o) {
+          tc::tmem_ld64(tmem + lane_base + c * 64, v);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 64; ++j) v[j] = 0u;
+        }
+        if (!is_s) {
+          float4* d4 = reinterpret_cast<float4*>(ost + hl * OST_LD + c * 64);
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            d4[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]), __uint_as_float(v[4 * j + 2]),
+                                __uint_as_float(v[4 * j + 3]));
+        }
+      }
+      if (!is_s) {
+        ost_ml[2 * hl] = have_o ? m_h : -INFINITY;
+        ost_ml[2 * hl + 1] = have_o ? l_h : 0.f;
+      }
     } else {
       float* P = a.part + (((size_t)row * a.splits + split) * AT_H + h) * attn_part_stride(512);
 #pragma unroll 1
@@ -425,6 +457,62 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, TM_COLS);
   }
+  if (a.cluster_combine) {
+    // merge heads [h0, h1) of this head half from every split's staged partial
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();
+    const int S = a.splits;
+    const int hp = (AT_HC + S - 1) / S;
+    const int h0 = split * hp, h1 = min(AT_HC, h0 + hp);
+    float* wts = reinterpret_cast<float*>(&sm.q[0][0]);          // [head][split] merge weights (Q is idle)
+    if ((int)threadIdx.x < h1 - h0) {
+      const int hl = h0 + threadIdx.x;
+      const float sk = a.sink[hh * AT_HC + hl];
+      float ms[8], ls[8];
+      float M = sk;
+      for (int p = 0; p < S; ++p) {
+        const float* ml = cluster.map_shared_rank(reinterpret_cast<float*>(&sm.kv[0][0][0]) + AT_HC * OST_LD, p);
+        ms[p] = ml[2 * hl];
+        ls[p] = ml[2 * hl + 1];
+        M = fmaxf(M, ms[p]);
+      }
+      float den = 0.f;
+      if (M != -INFINITY) {
+        den = __expf(sk - M);
+        for (int p = 0; p < S; ++p)
+          if (ms[p] != -INFINITY) den += ls[p] * __expf(ms[p] - M);
+      }
+      const float inv = den > 0.f ? 1.f / den : 0.f;
+      for (int p = 0; p < S; ++p)
+        wts[(hl - h0) * 8 + p] = (ms[p] == -INFINITY || M == -INFINITY) ? 0.f : __expf(ms[p] - M) * inv;
+      if (a.lse) a.lse[(size_t)row * AT_H + hh * AT_HC + hl] = den > 0.f ? M + logf(den) : -INFINITY;
+    }
+    __syncthreads();
+    const int items = (h1 - h0) * (512 / 4);
+    for (int it = threadIdx.x; it < items; it += AT_THREADS) {
+      const int hr = it >> 7, c4 = it & 127;
+      const int hl = h0 + hr;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int p = 0; p < S; ++p) {
+        const float wgt = wts[hr * 8 + p];
+        const float4 x = *reinterpret_cast<const float4*>(
+            cluster.map_shared_rank(reinterpret_cast<float*>(&sm.kv[0][0][0]), p) + hl * OST_LD + 4 * c4);
+        acc.x = fmaf(wgt, x.x, acc.x);
+        acc.y = fmaf(wgt, x.y, acc.y);
+        acc.z = fmaf(wgt, x.z, acc.z);
+        acc.w = fmaf(wgt, x.w, acc.w);
+      }
+      const float f4[4] = {acc.x, acc.y, acc.z, acc.w};
+      __nv_bfloat16* o = (__nv_bfloat16*)a.out + ((size_t)row * AT_H + hh * AT_HC + hl) * 512 + 4 * c4;
+      __nv_bfloat162 lo2 = __floats2bfloat162_rn(f4[0], f4[1]), hi2 = __floats2bfloat162_rn(f4[2], f4[3]);
+      uint2 pk;
+      pk.x = *reinterpret_cast<uint32_t*>(&lo2);
+      pk.y = *reinterpret_cast<uint32_t*>(&hi2);
+      *reinterpret_cast<uint2*>(o) = pk;
+    }
+    cluster.sync();                                  // peers may still read this CTA's staged partial
+  }
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_attn() {
@@ -454,8 +542,9 @@ bool make_latent_map(CUtensorMap* m, const void* base, uint64_t rows) {
 
 }  // namespace
 
-cudaError_t launch_attention_tc(AttnArgs a, cudaStream_t st, bool* used) {
+cudaError_t launch_attention_tc(AttnArgs a, cudaStream_t st, bool* used, bool* combined) {
   *used = false;
+  *combined = false;
   if (a.H != AT_H || a.dk != 576 || a.dv != 512) return cudaSuccess;
   if ((uintptr_t)a.q & 15 || (uintptr_t)a.cache & 15 || (a.win && ((uintptr_t)a.win & 15))) return cudaSuccess;
   if ((int64_t)a.B * a.n_max > 0x7fffffffLL || (int64_t)a.B * a.Tq * AT_H > 0x7fffffffLL) return cudaSuccess;
@@ -472,10 +561,38 @@ cudaError_t launch_attention_tc(AttnArgs a, cudaStream_t st, bool* used) {
   const size_t smem = sizeof(AtSmem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(2 * a.splits, a.B * a.Tq);
-  attn_tc_kernel<<<grid, AT_THREADS, smem, st>>>(maps, a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * a.splits, a.B * a.Tq);
+  cfg.blockDim = dim3(AT_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = a.splits;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  a.cluster_combine = 0;
+  if (a.splits >= 2 && a.splits <= 8) {
+    // merge the splits in a cluster when such clusters fit (checked once per split count)
+    static std::mutex mu;
+    static std::map<int, bool> fits;
+    std::lock_guard<std::mutex> g(mu);
+    auto it = fits.find(a.splits);
+    if (it == fits.end()) {
+      int n = 0;
+      const bool ok = cudaOccupancyMaxActiveClusters(&n, attn_tc_kernel, &cfg) == cudaSuccess && n > 0;
+      cudaGetLastError();
+      it = fits.emplace(a.splits, ok).first;
+    }
+    a.cluster_combine = it->second ? 1 : 0;
+  }
+  cfg.numAttrs = a.cluster_combine ? 1 : 0;
+  e = cudaLaunchKernelEx(&cfg, attn_tc_kernel, maps, a);
   *used = true;
-  return cudaGetLastError();
+  *combined = a.cluster_combine != 0;
+  return e;
 }
 
 }  // namespace csa
