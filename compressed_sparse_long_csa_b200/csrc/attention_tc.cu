@@ -43,7 +43,10 @@ constexpr int AT_HC = 64;                // heads per CTA (MMA M)
 constexpr int AT_ATOMS = 9;              // 576 dims = 9 atoms of 64 dims (128 bytes)
 constexpr int AT_CHUNKS = AT_ATOMS * 8;  // 16-byte chunks per row
 constexpr int AT_GROUP = 128;            // threads per loader group; group g fills stage g
-constexpr int AT_THREADS = 5 * 32 + 2 * AT_GROUP;   // 4 softmax warps, 1 MMA warp, 2 loader groups
+constexpr int AT_SMW = 8;                // softmax warps: two warpgroups, one per half of the tile's columns
+constexpr int AT_MMAW = AT_SMW;          // the MMA warp
+constexpr int AT_LDW = AT_SMW + 1;       // first loader warp
+constexpr int AT_THREADS = (AT_SMW + 1) * 32 + 2 * AT_GROUP;
 constexpr float AT_RESCALE_THRESH = 8.0f;
 constexpr int ATOM = AT_ROWS * 128;      // one 64-row x 128-byte swizzle atom
 constexpr unsigned long long NO_RUN = ~0ull;
@@ -67,6 +70,7 @@ struct AtSmem {
   uint32_t tmem_base;
   int abort_flag;
   int ld_stop[2];       // per loader group: 1 + the iteration at which it stops (0 = running)
+  float lx[2][AT_HC];   // softmax row sums of each warpgroup's columns
 };
 
 static_assert(sizeof(AtSmem) + 1024 <= 232448, "shared memory budget of one CTA (227 KB)");
@@ -120,27 +124,27 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
       tc::mbar_init(&sm.full[s], AT_GROUP);
       tc::mbar_init(&sm.empty[s], 1);
       tc::mbar_init(&sm.sfull[s], 1);
-      tc::mbar_init(&sm.sfree[s], 4);
+      tc::mbar_init(&sm.sfree[s], AT_SMW);
       sm.ld_stop[s] = 0;
     }
-    tc::mbar_init(&sm.pfull, 4);
+    tc::mbar_init(&sm.pfull, AT_SMW);
     tc::mbar_init(&sm.pdone, 1);
     tc::mbar_init(&sm.qfull, 1);
     tc::mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     tc::fence_mbar_init();
   }
-  if (warp == 4) { tc::tmem_alloc(&sm.tmem_base, TM_COLS); tc::tmem_relinquish(); }
+  if (warp == AT_MMAW) { tc::tmem_alloc(&sm.tmem_base, TM_COLS); tc::tmem_relinquish(); }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = sm.tmem_base;
 
-  if (warp >= 5) {
-    // ------------------------------------------------------------------ loader group g (128 threads)
+  if (warp >= AT_LDW) {
+    // ------------------------------------------------------------------ loader group g (64 threads)
     // Group g loads tiles g, g+2, ... into stage g; the two groups never wait on each other.
-    const int g = (warp - 5) / 4;
-    const int lg = threadIdx.x - 5 * 32 - g * AT_GROUP;
+    const int g = (warp - AT_LDW) / (AT_GROUP / 32);
+    const int lg = threadIdx.x - AT_LDW * 32 - g * AT_GROUP;
     if (g == 0 && lg == 0) {
       tc::prefetch_tmap(&maps.q);
       tc::prefetch_tmap(&maps.cache);
@@ -215,34 +219,40 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
       if (g == 0) tc::mbar_wait(&sm.qfull, 0);
       if (issued > 0) tc::mbar_wait(&sm.full[g], (issued - 1) & 1);
     }
-  } else if (warp == 4) {
+  } else if (warp == AT_MMAW) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t ID_S = tc::idesc(tc::FMT_BF16, tc::FMT_BF16, AT_HC, AT_ROWS);
       constexpr uint32_t ID_O = tc::idesc(tc::FMT_BF16, tc::FMT_BF16, AT_HC, 256, 0, 1);
       bool ok = n_t == 0 || tc::mbar_wait(&sm.qfull, 0);
-      for (int it = 0; ok && n_t > 0 && it <= n_t; ++it) {
-        if (it < n_t) {
-          const int st = it & 1;
-          const uint32_t ph = (it >> 1) & 1;
-          if (!tc::mbar_wait(&sm.full[st], ph) || !tc::mbar_wait(&sm.sfree[st], ph ^ 1) ||
-              *(volatile int*)&sm.abort_flag) { ok = false; break; }
-          tc::fence_after_sync();
-          const uint32_t d = tmem + TM_S_LANE + st * AT_ROWS;
-          for (int at = 0; at < AT_ATOMS; ++at) {
-            const uint32_t qa = tc::smem_u32(sm.q[at]), ka = tc::smem_u32(sm.kv[st][at]);
+      // Event-driven issue: S(ns) once its tile has landed and its S buffer is free, PV(np)
+      // once P(np) is ready, in order; a PV never waits behind the next tile's load.
+      int ns = 0, np = 0;
+      uint64_t t_idle = tc::now_ns();
+      uint32_t spins = 0;
+      while (ok && np < n_t) {
+        bool prog = false;
+        if (ns < n_t) {
+          const int st = ns & 1;
+          const uint32_t ph = (ns >> 1) & 1;
+          if (tc::mbar_try_wait(&sm.full[st], ph) && tc::mbar_try_wait(&sm.sfree[st], ph ^ 1)) {
+            tc::fence_after_sync();
+            const uint32_t d = tmem + TM_S_LANE + st * AT_ROWS;
+            for (int at = 0; at < AT_ATOMS; ++at) {
+              const uint32_t qa = tc::smem_u32(sm.q[at]), ka = tc::smem_u32(sm.kv[st][at]);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-              tc::mma_f16(d, tc::desc_k_sw128(qa + ks * 32), tc::desc_k_sw128(ka + ks * 32), ID_S,
-                          (at > 0 || ks > 0) ? 1u : 0u);
+              for (int ks = 0; ks < 4; ++ks)
+                tc::mma_f16(d, tc::desc_k_sw128(qa + ks * 32), tc::desc_k_sw128(ka + ks * 32), ID_S,
+                            (at > 0 || ks > 0) ? 1u : 0u);
+            }
+            tc::mma_commit(&sm.sfull[st]);
+            ++ns;
+            prog = true;
           }
-          tc::mma_commit(&sm.sfull[st]);
         }
-        if (it >= 1) {
-          // O += P_{it-1} V_{it-1}: value dims 0-255 (atoms 0-3) and 256-511 (atoms 4-7)
-          const int pt = it - 1;
-          const int st = pt & 1;
-          if (!tc::mbar_wait(&sm.pfull, pt & 1) || *(volatile int*)&sm.abort_flag) { ok = false; break; }
+        if (np < ns && tc::mbar_try_wait(&sm.pfull, np & 1)) {
+          // O += P_np V_np: value dims 0-255 (atoms 0-3) and 256-511 (atoms 4-7)
+          const int st = np & 1;
           tc::fence_after_sync();
           const uint32_t pa = tc::smem_u32(sm.p);
 #pragma unroll
@@ -251,10 +261,19 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
 #pragma unroll
             for (int ks = 0; ks < AT_ROWS / 16; ++ks)
               tc::mma_f16(tmem + 256 * half, tc::desc_k_sw128(pa + ks * 32),
-                          tc::desc_mn_sw128(va + ks * 16 * 128, ATOM, 1024), ID_O, (pt > 0 || ks > 0) ? 1u : 0u);
+                          tc::desc_mn_sw128(va + ks * 16 * 128, ATOM, 1024), ID_O, (np > 0 || ks > 0) ? 1u : 0u);
           }
           tc::mma_commit(&sm.empty[st]);
           tc::mma_commit(&sm.pdone);
+          ++np;
+          prog = true;
+        }
+        if (prog) {
+          spins = 0;
+        } else if ((++spins & 63u) == 0u) {
+          const uint64_t t = tc::now_ns();
+          if (spins == 64u) t_idle = t;
+          if (*(volatile int*)&sm.abort_flag || t - t_idle > tc::WAIT_LIMIT_NS) ok = false;
         }
       }
       if (!ok) atomicExch(&sm.abort_flag, 1);
@@ -263,16 +282,19 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
       tc::mbar_wait(&sm.drain, 0);
     }
   } else {
-    // ------------------------------------------------------------------ softmax + epilogue, warps 0-3
-    // TMEM quarter q = warp: lanes 16-31 hold the logits of heads 16q .. 16q+15 (S), lanes 0-15
-    // hold the output rows of the same heads (O).
-    const int quarter = warp;
+    // ------------------------------------------------------------------ softmax + epilogue, warps 0-7
+    // TMEM quarter q = warp % 4: lanes 16-31 hold the logits of heads 16q .. 16q+15 (S), lanes
+    // 0-15 the output rows of the same heads (O).  Warpgroup wg = warp / 4 exponentiates the
+    // tile's columns [32wg, 32wg+32): each S lane takes 16 of them and hands the other 16 to
+    // its O lane (lane - 16), which is otherwise idle here.  Both warpgroups read all 64
+    // logits, so they reach the same running max without exchanging it.
+    const int wg = warp >> 2, quarter = warp & 3;
     const bool is_s = lane >= 16;
     const int hl = quarter * 16 + (lane & 15);      // head within the CTA
     const int h = hh * AT_HC + hl;                  // head within the query
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const float scale = a.sm_scale;
-    float m_run = -INFINITY, l_run = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;           // S lanes: running max, this warpgroup's row sum
     bool ok = true;
     for (int it = 0; it < n_t; ++it) {
       const int st = it & 1;
@@ -306,7 +328,18 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
       }
       // the O row of head hl sits in lane (lane & 15) of the same warp
       const float alpha_o = __shfl_sync(0xffffffffu, alpha, (lane & 15) + 16);
+      const float m_use = __shfl_sync(0xffffffffu, m_run, (lane & 15) + 16);
       const bool rescale_any = __any_sync(0xffffffffu, need_rescale);
+      // this thread's 16 logits: S lanes keep the first 16 of the warpgroup's 32 columns,
+      // O lanes receive the second 16 from their S lane
+      float pv[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const float a0 = wg ? s[32 + q] : s[q];
+        const float a1 = wg ? s[48 + q] : s[16 + q];
+        const float moved = __shfl_down_sync(0xffffffffu, a1, 16);
+        pv[q] = is_s ? a0 : moved;
+      }
       // P and O are owned by the previous PV until it completes
       if (it >= 1) {
         if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.pdone, (it - 1) & 1))) { ok = false; break; }
@@ -315,13 +348,14 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
       if (rescale_any) {
         // A 32x32b store writes all 32 lanes, so the S lanes write back what they read.
         // That is harmless only while no MMA writes an S buffer: this tile's buffer is not
-        // released yet, and the next tile's S must have landed.
+        // released yet, and the next tile's S must have landed.  Warpgroup wg rescales O
+        // columns [256wg, 256wg+256).
         if (it + 1 < n_t) {
           if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.sfull[st ^ 1], ((it + 1) >> 1) & 1))) { ok = false; break; }
           tc::fence_after_sync();
         }
 #pragma unroll 1
-        for (int c = 0; c < 512 / 64; ++c) {
+        for (int c = 4 * wg; c < 4 * wg + 4; ++c) {
           uint32_t v[64];
           tc::tmem_ld64(tmem + lane_base + c * 64, v);
           const float f = is_s ? 1.f : alpha_o;
@@ -332,25 +366,26 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
         }
         tc::tmem_st_wait();
       }
-      if (is_s) {
-        l_run *= alpha;
+      {
         float psum = 0.f;
         const uint32_t pbase = tc::smem_u32(sm.p);
+        const int c0 = 4 * wg + (is_s ? 0 : 2);     // 16-byte chunks (8 columns) of the P row
 #pragma unroll
-        for (int c = 0; c < AT_ROWS / 8; ++c) {
+        for (int cc = 0; cc < 2; ++cc) {
           uint32_t w4[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const float p0 = (m_run == -INFINITY) ? 0.f : __expf(s[c * 8 + 2 * u] - m_run);
-            const float p1 = (m_run == -INFINITY) ? 0.f : __expf(s[c * 8 + 2 * u + 1] - m_run);
+            const float p0 = (m_use == -INFINITY) ? 0.f : __expf(pv[cc * 8 + 2 * u] - m_use);
+            const float p1 = (m_use == -INFINITY) ? 0.f : __expf(pv[cc * 8 + 2 * u + 1] - m_use);
             __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
             psum += __low2float(hb) + __high2float(hb);     // the normaliser uses the rounded P
             w4[u] = *reinterpret_cast<uint32_t*>(&hb);
           }
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pbase + sw128_off(hl, c)), "r"(w4[0]),
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pbase + sw128_off(hl, c0 + cc)), "r"(w4[0]),
                        "r"(w4[1]), "r"(w4[2]), "r"(w4[3]) : "memory");
         }
-        l_run += psum;
+        const float po = __shfl_up_sync(0xffffffffu, psum, 16);   // the O lane's part, to its S lane
+        if (is_s) l_run = l_run * alpha + psum + po;
       }
       // release this tile's S buffer and hand P (and a rescaled O) to the MMA thread
       tc::fence_proxy_async_smem();
@@ -366,9 +401,12 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
     if (!ok) atomicExch(&sm.abort_flag, 1);
     tc::fence_after_sync();
     const bool have_o = ok && n_t > 0;
-    // the O lanes take m and l of their head from the S lanes
+    // the row sum is the two warpgroups' parts; the O lanes take m and l from the S lanes
+    if (is_s) sm.lx[wg][hl] = l_run;
+    named_bar(3, AT_SMW * 32);
+    const float l_tot = sm.lx[0][hl] + sm.lx[1][hl];
     const float m_h = __shfl_sync(0xffffffffu, m_run, (lane & 15) + 16);
-    const float l_h = __shfl_sync(0xffffffffu, l_run, (lane & 15) + 16);
+    const float l_h = __shfl_sync(0xffffffffu, l_tot, (lane & 15) + 16);
     if (a.splits == 1) {
       const float sk = a.sink[h];
       const float mh = have_o ? m_h : -INFINITY;
@@ -381,7 +419,7 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
       const float inv = den > 0.f ? f / den : 0.f;
       __nv_bfloat16* o = (__nv_bfloat16*)a.out + ((size_t)row * AT_H + h) * 512;
 #pragma unroll 1
-      for (int c = 0; c < 512 / 64; ++c) {
+      for (int c = 4 * wg; c < 4 * wg + 4; ++c) {
         uint32_t v[64];
         if (have_o) {
           tc::tmem_ld64(tmem + lane_base + c * 64, v);
@@ -399,13 +437,13 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
           }
         }
       }
-      if (a.lse && !is_s) a.lse[(size_t)row * AT_H + h] = den > 0.f ? M + logf(den) : -INFINITY;
+      if (a.lse && !is_s && wg == 0) a.lse[(size_t)row * AT_H + h] = den > 0.f ? M + logf(den) : -INFINITY;
     } else if (a.cluster_combine) {
       // stage the partial in shared memory (the KV stages are idle: every PV has completed)
       float* ost = reinterpret_cast<float*>(&sm.kv[0][0][0]);
       float* ost_ml = ost + AT_HC * OST_LD;
 #pragma unroll 1
-      for (int c = 0; c < 512 / 64; ++c) {
+      for (int c = 4 * wg; c < 4 * wg + 4; ++c) {
         uint32_t v[64];
         if (have_o) {
           tc::tmem_ld64(tmem + lane_base + c * 64, v);
@@ -421,14 +459,14 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
                                 __uint_as_float(v[4 * j + 3]));
         }
       }
-      if (!is_s) {
+      if (!is_s && wg == 0) {
         ost_ml[2 * hl] = have_o ? m_h : -INFINITY;
         ost_ml[2 * hl + 1] = have_o ? l_h : 0.f;
       }
     } else {
       float* P = a.part + (((size_t)row * a.splits + split) * AT_H + h) * attn_part_stride(512);
 #pragma unroll 1
-      for (int c = 0; c < 512 / 64; ++c) {
+      for (int c = 4 * wg; c < 4 * wg + 4; ++c) {
         uint32_t v[64];
         if (have_o) {
           tc::tmem_ld64(tmem + lane_base + c * 64, v);
@@ -444,7 +482,7 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
                                 __uint_as_float(v[4 * j + 3]));
         }
       }
-      if (!is_s) {
+      if (!is_s && wg == 0) {
         P[512] = have_o ? m_h : -INFINITY;
         P[513] = have_o ? l_h : 0.f;
       }
@@ -453,7 +491,7 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
   tc::fence_before_sync();
   __syncthreads();
   if (sm.abort_flag && threadIdx.x == 0) raise_err(a.err, CSA_DEVERR_TIMEOUT);
-  if (warp == 4) {
+  if (warp == AT_MMAW) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, TM_COLS);
   }
