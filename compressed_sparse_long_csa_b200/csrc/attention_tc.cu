@@ -504,25 +504,37 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
     const int hp = (AT_HC + S - 1) / S;
     const int h0 = split * hp, h1 = min(AT_HC, h0 + hp);
     float* wts = reinterpret_cast<float*>(&sm.q[0][0]);          // [head][split] merge weights (Q is idle)
+    float* ost_local = reinterpret_cast<float*>(&sm.kv[0][0][0]);
+    // peer base addresses, all loads of a step issued before any is used (S <= 8)
+    const float* peer[8];
+#pragma unroll
+    for (int p = 0; p < 8; ++p) peer[p] = cluster.map_shared_rank(ost_local, p < S ? p : 0);
     if ((int)threadIdx.x < h1 - h0) {
       const int hl = h0 + threadIdx.x;
       const float sk = a.sink[hh * AT_HC + hl];
       float ms[8], ls[8];
-      float M = sk;
-      for (int p = 0; p < S; ++p) {
-        const float* ml = cluster.map_shared_rank(reinterpret_cast<float*>(&sm.kv[0][0][0]) + AT_HC * OST_LD, p);
-        ms[p] = ml[2 * hl];
-        ls[p] = ml[2 * hl + 1];
-        M = fmaxf(M, ms[p]);
+#pragma unroll
+      for (int p = 0; p < 8; ++p) {
+        ms[p] = -INFINITY;
+        ls[p] = 0.f;
+        if (p < S) {
+          ms[p] = peer[p][AT_HC * OST_LD + 2 * hl];
+          ls[p] = peer[p][AT_HC * OST_LD + 2 * hl + 1];
+        }
       }
+      float M = sk;
+#pragma unroll
+      for (int p = 0; p < 8; ++p) M = fmaxf(M, ms[p]);
       float den = 0.f;
       if (M != -INFINITY) {
         den = __expf(sk - M);
-        for (int p = 0; p < S; ++p)
+#pragma unroll
+        for (int p = 0; p < 8; ++p)
           if (ms[p] != -INFINITY) den += ls[p] * __expf(ms[p] - M);
       }
       const float inv = den > 0.f ? 1.f / den : 0.f;
-      for (int p = 0; p < S; ++p)
+#pragma unroll
+      for (int p = 0; p < 8; ++p)
         wts[(hl - h0) * 8 + p] = (ms[p] == -INFINITY || M == -INFINITY) ? 0.f : __expf(ms[p] - M) * inv;
       if (a.lse) a.lse[(size_t)row * AT_H + hh * AT_HC + hl] = den > 0.f ? M + logf(den) : -INFINITY;
     }
@@ -531,19 +543,21 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
     for (int it = threadIdx.x; it < items; it += AT_THREADS) {
       const int hr = it >> 7, c4 = it & 127;
       const int hl = h0 + hr;
+      float4 x[8];
+#pragma unroll
+      for (int p = 0; p < 8; ++p)
+        x[p] = p < S ? *reinterpret_cast<const float4*>(peer[p] + hl * OST_LD + 4 * c4) : make_float4(0.f, 0.f, 0.f, 0.f);
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int p = 0; p < S; ++p) {
+#pragma unroll
+      for (int p = 0; p < 8; ++p) {
         const float wgt = wts[hr * 8 + p];
-        const float4 x = *reinterpret_cast<const float4*>(
-            cluster.map_shared_rank(reinterpret_cast<float*>(&sm.kv[0][0][0]), p) + hl * OST_LD + 4 * c4);
-        acc.x = fmaf(wgt, x.x, acc.x);
-        acc.y = fmaf(wgt, x.y, acc.y);
-        acc.z = fmaf(wgt, x.z, acc.z);
-        acc.w = fmaf(wgt, x.w, acc.w);
+        acc.x = fmaf(wgt, x[p].x, acc.x);
+        acc.y = fmaf(wgt, x[p].y, acc.y);
+        acc.z = fmaf(wgt, x[p].z, acc.z);
+        acc.w = fmaf(wgt, x[p].w, acc.w);
       }
-      const float f4[4] = {acc.x, acc.y, acc.z, acc.w};
       __nv_bfloat16* o = (__nv_bfloat16*)a.out + ((size_t)row * AT_H + hh * AT_HC + hl) * 512 + 4 * c4;
-      __nv_bfloat162 lo2 = __floats2bfloat162_rn(f4[0], f4[1]), hi2 = __floats2bfloat162_rn(f4[2], f4[3]);
+      __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x, acc.y), hi2 = __floats2bfloat162_rn(acc.z, acc.w);
       uint2 pk;
       pk.x = *reinterpret_cast<uint32_t*>(&lo2);
       pk.y = *reinterpret_cast<uint32_t*>(&hi2);
