@@ -13,10 +13,11 @@
 //
 // CTA = (split of the entry tiles, group of G queries, sequence).  Warp roles:
 // warp 0 issues TMA loads of 128-entry x 128-byte key tiles (128-byte swizzle)
-// into a STAGES-deep ring; warp 1 owns the TMEM allocation and one lane issues the
-// tcgen05.mma (M = 128, N = 64 G, K = 32, four per tile) into a double-buffered
-// accumulator; warps 4..7 run the epilogue.  Every wait is bounded: on timeout the
-// CTA raises CSA_DEVERR_TIMEOUT, drains its own copies and exits.
+// into a STAGES-deep ring (the first ones before the CTA's setup barrier); warp 1 owns
+// the TMEM allocation and one lane issues the tcgen05.mma (M = 128, N = 64 G, K = 32,
+// four per tile) into a ring of accumulators; warps 4..11 run the epilogue as two
+// warpgroups that take alternate tiles.  Every wait is bounded: on timeout the CTA
+// raises CSA_DEVERR_TIMEOUT, drains its own copies and exits.
 #include "indexer.cuh"
 #include "tc.cuh"
 
@@ -37,25 +38,28 @@ struct IdxTcParams {
   int tiles_per_split;
 };
 
+constexpr int IT_THREADS = 384;  // warp 0 TMA, warp 1 MMA, warps 4..11 epilogue (two warpgroups)
+
 template <int G, int STAGES>
 struct IdxSmem {
   alignas(1024) uint8_t q[G * 64 * IT_KB];
   alignas(1024) uint8_t k[STAGES][IT_TILE_BYTES];
   alignas(8) uint64_t full[STAGES];
   uint64_t empty[STAGES];
-  uint64_t tfull[2];
-  uint64_t tempty[2];
+  uint64_t tfull[4];
+  uint64_t tempty[4];
   uint64_t qfull;
   uint32_t tmem_base;
   int abort_flag;
   int t_begin, t_end;
+  int issued0;          // tile loads issued before the setup barrier
   int n_elig[G];
   int row[G];
   float wq[G][64];
 };
 
 template <int G, int STAGES>
-__global__ void __launch_bounds__(256, G == 1 ? 2 : 1)
+__global__ void __launch_bounds__(IT_THREADS, G == 1 ? 2 : 1)
 indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ, IdxTcParams p) {
   extern __shared__ uint8_t smem_raw[];
   using Sm = IdxSmem<G, STAGES>;
@@ -64,11 +68,14 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x, qg = blockIdx.y, b = blockIdx.z;
   constexpr int N = 64 * G;
-  constexpr uint32_t NCOLS = 2 * N;          // two accumulators; power of two >= 32
+  constexpr int NACC = (G == 1) ? 4 : 2;     // accumulators in TMEM
+  constexpr uint32_t NCOLS = NACC * N;       // a power of two >= 32
 
   if (threadIdx.x == 0) {
+    tc::prefetch_tmap(&tmK);                 // descriptor fetches overlap the setup
+    tc::prefetch_tmap(&tmQ);
     for (int s = 0; s < STAGES; ++s) { tc::mbar_init(&sm.full[s], 1); tc::mbar_init(&sm.empty[s], 1); }
-    for (int s = 0; s < 2; ++s) { tc::mbar_init(&sm.tfull[s], 1); tc::mbar_init(&sm.tempty[s], 4); }
+    for (int s = 0; s < NACC; ++s) { tc::mbar_init(&sm.tfull[s], 1); tc::mbar_init(&sm.tempty[s], 4); }
     tc::mbar_init(&sm.qfull, 1);
     tc::fence_mbar_init();
     sm.abort_flag = 0;
@@ -86,6 +93,18 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     if (t1 > t_lim) t1 = t_lim;
     sm.t_begin = t0;
     sm.t_end = t1 > t0 ? t1 : t0;
+    // the query tile and the first key tiles go out before the setup barrier (a stage's
+    // first use needs no release)
+    const int n0 = sm.t_end - t0 < STAGES ? sm.t_end - t0 : STAGES;
+    if (n0 > 0) {
+      tc::mbar_arrive_expect_tx(&sm.qfull, G * 64 * IT_KB);
+      tc::tma_load_2d(sm.q, &tmQ, &sm.qfull, 0, (b * a.Tq + qg * G) * 64);
+      for (int it = 0; it < n0; ++it) {
+        tc::mbar_arrive_expect_tx(&sm.full[it], IT_TILE_BYTES);
+        tc::tma_load_2d(sm.k[it], &tmK, &sm.full[it], 0, (int)(b * a.n_max) + (t0 + it) * IT_ROWS);
+      }
+    }
+    sm.issued0 = n0;
   }
   for (int i = threadIdx.x; i < G * 64; i += blockDim.x) {
     const int g = i / 64, j = i % 64;
@@ -106,12 +125,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
 
   if (warp == 0) {
     if (lane == 0 && n_t > 0) {
-      tc::prefetch_tmap(&tmK);
-      tc::prefetch_tmap(&tmQ);
-      tc::mbar_arrive_expect_tx(&sm.qfull, G * 64 * IT_KB);
-      tc::tma_load_2d(sm.q, &tmQ, &sm.qfull, 0, (b * a.Tq + qg * G) * 64);
-      int issued = 0;
-      for (int it = 0; it < n_t; ++it) {
+      int issued = sm.issued0;
+      for (int it = issued; it < n_t; ++it) {
         const int st = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
         if (!tc::mbar_wait(&sm.empty[st], ph ^ 1)) { atomicExch(&sm.abort_flag, 1); break; }
@@ -134,8 +149,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
       for (int it = 0; ok && it < n_t; ++it) {
         const int st = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
-        const int acc = it & 1;
-        const uint32_t aph = (it >> 1) & 1;
+        const int acc = it % NACC;
+        const uint32_t aph = (it / NACC) & 1;
         if (!tc::mbar_wait(&sm.tempty[acc], aph ^ 1)) { ok = false; break; }
         if (!tc::mbar_wait(&sm.full[st], ph)) { ok = false; break; }
         if (*(volatile int*)&sm.abort_flag) { ok = false; break; }
@@ -152,25 +167,26 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
       if (!ok) {
         atomicExch(&sm.abort_flag, 1);
         // let the last issued MMA finish before the TMEM is released
-        if (last_issued >= 0) tc::mbar_wait(&sm.tfull[last_issued & 1], (last_issued >> 1) & 1);
+        if (last_issued >= 0) tc::mbar_wait(&sm.tfull[last_issued % NACC], (last_issued / NACC) & 1);
       }
     }
   } else if (warp >= 4) {
-    const int quarter = warp & 3;
+    // epilogue warpgroup e takes tiles e, e+2, ...; quarter q = warp % 4 reads TMEM lanes 32q..32q+31
+    const int e = (warp - 4) >> 2, quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const float* kscale = (const float*)a.kI_scale;
     float kmax = 0.f;
-    // the key scale of the next tile is loaded before waiting for the current accumulator
+    // the key scale of the group's next tile is loaded before waiting for the current accumulator
     auto load_scale = [&](int it) {
       const int s = (t_begin + it) * IT_ROWS + r;
       return (it < n_t && s < a.n_max) ? __ldg(kscale + (size_t)b * a.n_max + s) : 0.f;
     };
-    float sk_next = load_scale(0);
-    for (int it = 0; it < n_t; ++it) {
-      const int acc = it & 1;
-      const uint32_t aph = (it >> 1) & 1;
+    float sk_next = load_scale(e);
+    for (int it = e; it < n_t; it += 2) {
+      const int acc = it % NACC;
+      const uint32_t aph = (it / NACC) & 1;
       const float sk = sk_next;
-      sk_next = load_scale(it + 1);
+      sk_next = load_scale(it + 2);
       bool ok = tc::mbar_wait(&sm.tfull[acc], aph) && !*(volatile int*)&sm.abort_flag;
       ok = __all_sync(0xffffffffu, ok);               // the TMEM loads below are warp-collective
       if (!ok) { atomicExch(&sm.abort_flag, 1); break; }
@@ -178,11 +194,20 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
       const int s = (t_begin + it) * IT_ROWS + r;
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        float val = 0.f;
-        uint32_t v[64];
-        tc::tmem_ld64(tmem + ((uint32_t)(quarter * 32) << 16) + acc * N + g * 64, v);
+        // four partial sums over the heads (j mod 4)
+        float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int j = 0; j < 64; ++j) val = fmaf(sm.wq[g][j], fmaxf(__uint_as_float(v[j]), 0.f), val);
+        for (int hlf = 0; hlf < 2; ++hlf) {
+          uint32_t v[32];
+          const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + acc * N + g * 64 + hlf * 32;
+          tc::tmem_ld16(ta, v);
+          tc::tmem_ld16(ta + 16, v + 16);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            part[j & 3] = fmaf(sm.wq[g][hlf * 32 + j], fmaxf(__uint_as_float(v[j]), 0.f), part[j & 3]);
+        }
+        const float val = (part[0] + part[1]) + (part[2] + part[3]);
         const bool valid = s < sm.n_elig[g];
         if (valid) {
           a.scores[(size_t)sm.row[g] * a.ld + s] = val * sk;
@@ -493,7 +518,7 @@ cudaError_t launch_g(const IndexerArgs& a, cudaStream_t st, bool* used) {
                                        (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(splits, p.n_qg, a.B);
-  indexer_tc_kernel<G, STAGES><<<grid, 256, smem, st>>>(mk, mq, p);
+  indexer_tc_kernel<G, STAGES><<<grid, IT_THREADS, smem, st>>>(mk, mq, p);
   *used = true;
   return cudaGetLastError();
 }
