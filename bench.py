@@ -33,6 +33,33 @@ WORKLOADS = {
 }
 METRIC = "CSA/HCA decode tokens/s and HBM GB/s (% roofline) at 64K-1M ctx; prefill TFLOP/s"
 
+# DRAM bytes (read + write) per call of the dominant ABI call, summed over its kernels, from
+# the ncu captures summarised under profiles/ (None until a capture of the current kernels).
+TRAFFIC = {
+    # profiles/csa_decode_64k_dram_traffic.md: indexer_tc_kernel 34 767 872 + select 1 383 680 bytes
+    ("csa_decode_64k", "indexer"): 36151552,
+}
+
+
+def workload_config(name, D):
+    """The workload a line is measured on (shared by both arms)."""
+    return {"workload": name, "batch": D["B"], "context": D["T"], "entries": D["N"], "query_tokens": D.get("Tq", 1),
+            "top_k": D.get("k"), "window": D["W"], "heads": D["H"], "d_k": D["dk"], "d_v": D["dv"],
+            "indexer": D.get("ifmt"), "l2": "flushed before every step"}
+
+
+def algorithmic_flops(wid, D):
+    """Prefill multiply-adds x 2 of the tensor-core contractions (valid rows only)."""
+    if wid != 3:
+        return {}
+    import numpy as np
+    Tq, H, dk, dv, k, W, m = D["Tq"], D["H"], D["dk"], D["dv"], D["k"], D["W"], D["m"]
+    pos = D["q_pos0"] + np.arange(Tq)
+    n_elig = np.minimum(D["N"], (pos + 1) // m)
+    rows = np.minimum(n_elig, k) + np.minimum(pos + 1, W)
+    return {"attention": float(2 * H * (dk + dv) * rows.sum()),
+            "indexer": float(2 * D["HI"] * D["dI"] * n_elig.sum())}
+
 
 def algorithmic_bytes(wid, D):
     """Bytes the method must move per step (each input / output byte once)."""
@@ -117,8 +144,7 @@ def run_reference(args, wid):
     D = wl.dims
     cores = os.cpu_count()
     sample_b = list(range(min(D["B"], 4)))
-    for _ in range(args.warmup and 1):
-        pass
+    sample_rows = [int(r) for r in np.linspace(0, D["Tq"] - 1, 4)] if wid == 3 else []
     t0 = time.perf_counter()
     steps_done = 0
     for _ in range(max(1, args.steps)):
@@ -128,17 +154,20 @@ def run_reference(args, wid):
                 O.run_hca_decode(wl, batches=sample_b, prefix="h_")
         elif wid == 2:
             O.run_hca_decode(wl, batches=sample_b)
+        else:
+            O.run_csa_prefill(wl, rows=sample_rows)
         steps_done += 1
     dt = time.perf_counter() - t0
-    tokens = steps_done * len(sample_b)
+    tokens = steps_done * (len(sample_rows) if wid == 3 else len(sample_b))
+    sample = (f"{len(sample_rows)} of {D['Tq']} query tokens per step (compression of the whole chunk included)"
+              if wid == 3 else f"{len(sample_b)} of {D['B']} sequences per step, full context")
     value = tokens / dt
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dt / steps_done * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD_NAME, "batch_sampled": len(sample_b)},
+            "config": workload_config(WORKLOAD_NAME, D),
             "impl": "reference",
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                             "sample": f"{len(sample_b)} of {D['B']} sequences per step, full context"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -230,6 +259,11 @@ def run_ours(args, wid):
         for f in parts:
             f()
     torch.cuda.synchronize()
+    n0 = csa.launch_count()
+    for f in parts:                              # one more eager step: count the library's kernels
+        f()
+    launches_step = csa.launch_count() - n0
+    torch.cuda.synchronize()
     assert csa.read_device_error() == 0
     graphs = []
     for f in parts:
@@ -293,25 +327,35 @@ def run_ours(args, wid):
         peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
     except Exception:
         pass
+    src = "measured" if peaks else "fallback"
     hbm_peak = peaks.get("hbm_gbs", 6650.0)
-    # dominant kernel: the indexer for CSA decode, the attention otherwise
-    dom = "indexer" if wid in (1, 4) else "attention"
-    dom_ms = mean_ms[comp.index(dom)]
-    achieved = ab[dom] / (dom_ms * 1e-3) / 1e9
+    bf16_peak = peaks.get("bf16_tflops", 1590.0)
+    # the dominant ABI call by time; decode calls are HBM-bound, prefill calls tensor-bound
+    # (the FP8 indexer against twice the measured bf16 peak, the nominal dense ratio)
+    cand = [c for c in comp if c in ab]
+    dom = max(cand, key=lambda c: mean_ms[comp.index(c)])
+    dom_ms = float(mean_ms[comp.index(dom)])
+    fl = algorithmic_flops(wid, D)
+    if wid == 3 and dom in fl:
+        peak = bf16_peak * (2.0 if dom == "indexer" else 1.0)
+        achieved = fl[dom] / (dom_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "peak_source": src + (" bf16 x 2 (fp8)" if dom == "indexer" else " bf16 burst"),
+                "traffic": TRAFFIC.get((args.workload, dom))}
+    else:
+        achieved = ab[dom] / (dom_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "peak_source": src, "traffic": TRAFFIC.get((args.workload, dom))}
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": args.workload, "batch": D["B"], "context": D["T"], "entries": D["N"],
-                   "top_k": D.get("k"), "window": D["W"], "heads": D["H"], "l2": "flushed before every step",
-                   "launch": "one CUDA graph per ABI call"},
+        "config": dict(workload_config(args.workload, D), launch="one CUDA graph per ABI call"),
         "hbm_gbs_step": sum(ab.values()) / (ms_per_step * 1e-3) / 1e9,
         "breakdown_ms": {c: float(m) for c, m in zip(comp, mean_ms)},
-        "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "peak_source": "measured" if peaks else "fallback",
-                     "traffic": None},
+        "roofline": roof,
         "e2e": e2e,
-        "gpu_launches": launches_per_step(wid, D) * args.steps,
+        "gpu_launches": launches_step * args.steps,
         "clocks": summarize_clocks(clock_lines),
     }
     if rank == 0 and not args.no_cpu_baseline and world == 1:
@@ -321,16 +365,6 @@ def run_ours(args, wid):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
-
-
-def launches_per_step(wid, D):
-    if wid == 1:
-        return 5       # compress, indexer scores, indexer select, attention, combine
-    if wid == 2:
-        return 3
-    if wid == 3:
-        return 4
-    return 8
 
 
 def measure_e2e(args, wid, wl, T, D, csa, steps):

@@ -21,6 +21,7 @@ _SIGS = {
     "csa_abi_version": ([], _i32),
     "csa_status_string": ([_i32], C.c_char_p),
     "csa_read_device_error": ([_vp, C.POINTER(C.c_uint32)], _i32),
+    "csa_launch_count": ([], C.c_uint64),
     "csa_compress": ([_vp] * 10 + [_i64, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
     "hca_compress": ([_vp] * 5 + [_i64, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
     "lightning_index_workspace_size": ([_i32, _i32, _i64, _i32], _sz),
@@ -63,6 +64,11 @@ def _stream(stream):
 
 def _dtype_code(t):
     return CSA_BF16 if t.dtype == torch.bfloat16 else CSA_F32
+
+
+def launch_count() -> int:
+    """Kernels the library has enqueued in this process (a captured launch counts once)."""
+    return int(lib.csa_launch_count())
 
 
 def read_device_error(stream=None) -> int:

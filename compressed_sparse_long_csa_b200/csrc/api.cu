@@ -2,6 +2,7 @@
 // and dispatch to the kernels.  Nothing here allocates device memory or
 // synchronises (except csa_read_device_error, which is documented to).
 #include <math.h>
+#include <atomic>
 #include <mutex>
 
 #include "attention.cuh"
@@ -57,11 +58,17 @@ bool tc_enabled() {
   return v == 1;
 }
 
+std::atomic<uint64_t> g_launches{0};
+
 }  // namespace
+
+void csa::note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 extern "C" {
 
 int csa_abi_version(void) { return CSA_ABI_VERSION; }
+
+uint64_t csa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 const char* csa_status_string(int s) {
   switch (s) {

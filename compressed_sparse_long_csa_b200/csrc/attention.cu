@@ -186,9 +186,11 @@ cudaError_t launch_attention_cuda_core(AttnArgs a, int dtype, cudaStream_t st) {
   dim3 grid(a.splits, (a.H + CC_HG - 1) / CC_HG, a.B * a.Tq);
   if (dtype == CSA_BF16) {
     cudaFuncSetAttribute(attn_cuda_core_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+    note_launch();
     attn_cuda_core_kernel<__nv_bfloat16><<<grid, 256, smem, st>>>(a);
   } else {
     cudaFuncSetAttribute(attn_cuda_core_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+    note_launch();
     attn_cuda_core_kernel<float><<<grid, 256, smem, st>>>(a);
   }
   return cudaGetLastError();
@@ -196,8 +198,12 @@ cudaError_t launch_attention_cuda_core(AttnArgs a, int dtype, cudaStream_t st) {
 
 cudaError_t launch_attn_combine(const AttnArgs& a, int dtype, cudaStream_t st) {
   dim3 grid(a.B * a.Tq, a.H);
-  if (dtype == CSA_BF16) attn_combine_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(a);
-  else attn_combine_kernel<float><<<grid, 128, 0, st>>>(a);
+  note_launch();
+  if (dtype == CSA_BF16) {
+    attn_combine_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(a);
+  } else {
+    attn_combine_kernel<float><<<grid, 128, 0, st>>>(a);
+  }
   return cudaGetLastError();
 }
 

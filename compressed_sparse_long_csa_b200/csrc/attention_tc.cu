@@ -641,6 +641,7 @@ cudaError_t launch_attention_tc(AttnArgs a, cudaStream_t st, bool* used, bool* c
     a.cluster_combine = it->second ? 1 : 0;
   }
   cfg.numAttrs = a.cluster_combine ? 1 : 0;
+  note_launch();
   e = cudaLaunchKernelEx(&cfg, attn_tc_kernel, maps, a);
   *used = true;
   *combined = a.cluster_combine != 0;

@@ -8,6 +8,9 @@
 
 namespace csa {
 
+// Counts the kernels the library enqueues (defined in api.cu; read by csa_launch_count).
+void note_launch();
+
 // Error bits are OR-ed into a per-device word owned by api.cu; kernels get its address.
 __device__ __forceinline__ void raise_err(unsigned* err, unsigned bit) {
   if (err) atomicOr(err, bit);

@@ -232,10 +232,12 @@ cudaError_t launch_csa_compress(const void* Ca, const void* Cb, const void* Za, 
     dim3 grid((unsigned)((work + threads - 1) / threads), B);
     if (dtype == CSA_BF16) {
       using T = __nv_bfloat16;
+      note_launch();
       csa_compress_m4_kernel<T><<<grid, threads, 0, st>>>((const T*)Ca, (const T*)Cb, (const T*)Za, (const T*)Zb, Ba,
                                                           Bb, (const T*)pCb, (const T*)pZb, entry0, (T*)cache, n_max,
                                                           T_new, d, err);
     } else {
+      note_launch();
       csa_compress_m4_kernel<float><<<grid, threads, 0, st>>>((const float*)Ca, (const float*)Cb, (const float*)Za,
                                                               (const float*)Zb, Ba, Bb, (const float*)pCb,
                                                               (const float*)pZb, entry0, (float*)cache, n_max, T_new,
@@ -247,12 +249,14 @@ cudaError_t launch_csa_compress(const void* Ca, const void* Cb, const void* Za, 
     using T = __nv_bfloat16;
     const int64_t work = (int64_t)n_blk * (d / 8);
     dim3 grid((unsigned)((work + 255) / 256), B);
+    note_launch();
     csa_compress_kernel<T><<<grid, 256, 0, st>>>((const T*)Ca, (const T*)Cb, (const T*)Za, (const T*)Zb,
                                                  Ba, Bb, (const T*)pCb, (const T*)pZb, entry0, (T*)cache,
                                                  n_max, T_new, d, m, err);
   } else {
     const int64_t work = (int64_t)n_blk * (d / 4);
     dim3 grid((unsigned)((work + 255) / 256), B);
+    note_launch();
     csa_compress_kernel<float><<<grid, 256, 0, st>>>((const float*)Ca, (const float*)Cb, (const float*)Za,
                                                      (const float*)Zb, Ba, Bb, (const float*)pCb,
                                                      (const float*)pZb, entry0, (float*)cache, n_max,
@@ -268,10 +272,12 @@ cudaError_t launch_hca_compress(const void* C, const void* Z, const float* bias,
   if (dtype == CSA_BF16) {
     using T = __nv_bfloat16;
     dim3 grid(n_blk, (d + 63) / 64, B);
+    note_launch();
     hca_compress_kernel<T><<<grid, 256, 0, st>>>((const T*)C, (const T*)Z, bias, entry0, (T*)cache, n_max,
                                                  T_new, d, mp, err);
   } else {
     dim3 grid(n_blk, (d + 31) / 32, B);
+    note_launch();
     hca_compress_kernel<float><<<grid, 256, 0, st>>>((const float*)C, (const float*)Z, bias, entry0,
                                                      (float*)cache, n_max, T_new, d, mp, err);
   }

@@ -126,6 +126,7 @@ cudaError_t launch_indexer_scores_cuda_core(const IndexerArgs& a, cudaStream_t s
     attr_set[dev] = true;
   }
   dim3 grid((unsigned)((a.n_max + IDX_TILE - 1) / IDX_TILE), a.B * a.Tq);
+  note_launch();
   indexer_scores_cuda_core<<<grid, IDX_TILE, smem, st>>>(a);
   return cudaGetLastError();
 }

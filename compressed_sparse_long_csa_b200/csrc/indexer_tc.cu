@@ -490,6 +490,7 @@ cudaError_t launch_mxf4(const IndexerArgs& a, cudaStream_t st, bool* used) {
                                        (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(splits, a.Tq, a.B);
+  note_launch();
   indexer_mxf4_kernel<STAGES><<<grid, 384, smem, st>>>(mk, mq, p);
   *used = true;
   return cudaGetLastError();
@@ -518,6 +519,7 @@ cudaError_t launch_g(const IndexerArgs& a, cudaStream_t st, bool* used) {
                                        (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(splits, p.n_qg, a.B);
+  note_launch();
   indexer_tc_kernel<G, STAGES><<<grid, IT_THREADS, smem, st>>>(mk, mq, p);
   *used = true;
   return cudaGetLastError();

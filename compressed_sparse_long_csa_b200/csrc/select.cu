@@ -817,6 +817,7 @@ cudaError_t sl_launch(Kern kern, int rows, int C, size_t smem, cudaStream_t st, 
     }
     if (!it->second) return cudaErrorNotSupported;
   }
+  note_launch();
   return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 

@@ -543,6 +543,7 @@ cudaError_t launch_indexer_select(const IndexerArgs& a, cudaStream_t st) {
   const cudaError_t e = launch_indexer_select_cluster(a, st);
   if (e != cudaErrorNotSupported) return e;
   set_smem_attr((const void*)indexer_select_kernel);
+  note_launch();
   indexer_select_kernel<<<a.B * a.Tq, TK_THREADS, sizeof(TopkShared), st>>>(a);
   return cudaGetLastError();
 }
@@ -553,6 +554,7 @@ cudaError_t launch_topk_select(const float* scores, int64_t ld, const int32_t* n
   const cudaError_t e = launch_topk_select_cluster(scores, ld, n_valid, R, n, k, idx_out, st);
   if (e != cudaErrorNotSupported) return e;
   set_smem_attr((const void*)topk_select_kernel);
+  note_launch();
   topk_select_kernel<<<R, TK_THREADS, sizeof(TopkShared), st>>>(scores, ld, n_valid, n, k, idx_out);
   return cudaGetLastError();
 }

@@ -77,6 +77,11 @@ const char* csa_status_string(int status);
  * it.  Synchronises `stream` (the only call that does).                       */
 csa_status csa_read_device_error(void* stream, uint32_t* out);
 
+/* Number of kernels the library has enqueued in this process (all devices and
+ * streams; a launch captured into a CUDA graph counts once, at capture).  The
+ * paper has no counterpart: it lets a caller check which work ran on the GPU.  */
+uint64_t csa_launch_count(void);
+
 /* ---------------------------------------------------------------------------
  * csa_compress — CSA token-axis compression fused with the KV-cache append.
  * ("Гибридное внимание: CSA и HCA", CSA step 1: two KV series C^a, C^b and two

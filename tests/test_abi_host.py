@@ -28,6 +28,12 @@ def test_every_declared_symbol_is_exported():
         assert hasattr(N.lib, n), n
 
 
+def test_launch_counter_is_host_side_and_ignores_refused_calls():
+    before = N.lib.csa_launch_count()
+    assert N.lib.topk_select(None, 100, None, 4, 100, 8, FAKE, None, 0, None) == ERR_NULL
+    assert N.lib.csa_launch_count() == before
+
+
 def test_version_and_strings():
     assert N.lib.csa_abi_version() == 1
     for s in range(8):
