@@ -138,6 +138,9 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
+  // the setup above overlaps the previous kernel's tail; every input may come from it
+  tc::griddep_wait();
+  tc::griddep_launch_dependents();
   const uint32_t tmem = sm.tmem_base;
 
   if (warp >= AT_LDW) {
@@ -618,13 +621,15 @@ cudaError_t launch_attention_tc(AttnArgs a, cudaStream_t st, bool* used, bool* c
   cfg.blockDim = dim3(AT_THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = a.splits;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see griddep_wait in the kernel
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = a.splits;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   a.cluster_combine = 0;
   if (a.splits >= 2 && a.splits <= 8) {
     // merge the splits in a cluster when such clusters fit (checked once per split count)
@@ -640,7 +645,7 @@ cudaError_t launch_attention_tc(AttnArgs a, cudaStream_t st, bool* used, bool* c
     }
     a.cluster_combine = it->second ? 1 : 0;
   }
-  cfg.numAttrs = a.cluster_combine ? 1 : 0;
+  cfg.numAttrs = a.cluster_combine ? 2 : 1;
   note_launch();
   e = cudaLaunchKernelEx(&cfg, attn_tc_kernel, maps, a);
   *used = true;

@@ -120,6 +120,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
+  tc::griddep_launch_dependents();           // the selection kernel may start its prologue
   const uint32_t tmem = sm.tmem_base;
   const int t_begin = sm.t_begin, n_t = sm.t_end - sm.t_begin;
 

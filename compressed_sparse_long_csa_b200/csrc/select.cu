@@ -327,6 +327,7 @@ topk_cluster_kernel(const float* __restrict__ scores, int64_t ld, const int32_t*
   const unsigned C = cluster.num_blocks(), r = cluster.block_rank();
   const int row = blockIdx.x / C;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  tc::griddep_wait();                                      // every input may come from the previous kernel
   int n = n_valid ? n_valid[row] : (int)n_cap;
   if ((int64_t)n > n_cap) n = (int)n_cap;
   if (n < 0) n = 0;
@@ -555,25 +556,16 @@ indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
   const RescKeys rk{a.kI, a.kI_scale, a.n_max, a.H_I, a.d_I};
   const int lo = (int)r * chunk;
   const int m = max(0, min(n - lo, chunk));
-  // ---- this CTA's scores: one bulk copy into shared memory (the tail by plain loads)
+  tc::griddep_launch_dependents();
+  // ---- the query row (written before the scoring kernel started: read before waiting
+  // for it): codes into registers (staged into shared memory once the scores are
+  // classified), scales and weights, and U = sum_j w_j ||q_j|| for the error bound
   const int m4 = (n > k) ? (m & ~3) : 0;
   const float* srow = a.scores + (size_t)row * a.ld + lo;
   if (tid == 0) {
     tc::mbar_init(&sh.ldbar, 1);
     tc::fence_mbar_init();
   }
-  __syncthreads();
-  if (tid == 0) {
-    tc::mbar_arrive_expect_tx(&sh.ldbar, (uint32_t)m4 * 4u);
-    for (int o = 0; o < m4; o += 8192) {
-      const uint32_t bytes = (uint32_t)min(8192, m4 - o) * 4u;
-      asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                   ::"r"(tc::smem_u32(sv + o)), "l"(srow + o), "r"(bytes), "r"(tc::smem_u32(&sh.ldbar)) : "memory");
-    }
-  }
-  if (n > k && tid < m - m4) sv[m4 + tid] = srow[m4 + tid];
-  // ---- the query row: codes into registers (staged into shared memory once the scores
-  // are classified), scales and weights, and U = sum_j w_j ||q_j|| for the error bound
   const int total = HI * dI, lgd = __ffs(dI) - 1;
   const size_t r0 = (size_t)row * total;
   float qx[SL_QPT];
@@ -596,10 +588,7 @@ indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
       for (int bb = 0; bb < nb; ++bb)
         sh.qsc[tid * nb + bb] = ue8m0_to_float(((const uint8_t*)a.qI_scale)[((size_t)row * HI + tid) * nb + bb]);
   }
-  const float knmax = __uint_as_float(a.knmax[b]);
-  // the key range the scoring kernel recorded (exact min / max over the row's eligible entries)
-  uint32_t lo_k = ~a.keyrange[2 * (size_t)row + 1], hi_k = a.keyrange[2 * (size_t)row];
-  __syncthreads();
+  __syncthreads();                                         // w, scales and the barrier init are visible
   // U = sum_j w_j ||q_j||: warp w takes heads w, w + SL_W, ...; lane l holds elements
   // [epl*l, epl*l + epl) of the head (one 4- or 16-byte load, issued together)
   if (tid == 0) sh.U = 0.f;
@@ -651,6 +640,22 @@ indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
     __syncthreads();                                       // sh.U = 0 is visible
     if (lane == 0) atomicAdd(&sh.U, uw);
   }
+  // ---- the scoring kernel's outputs: scores (one bulk copy into shared memory, the tail
+  // by plain loads), key-norm bound and key range
+  tc::griddep_wait();
+  const float knmax = __uint_as_float(a.knmax[b]);
+  // the key range the scoring kernel recorded (exact min / max over the row's eligible entries)
+  uint32_t lo_k = ~a.keyrange[2 * (size_t)row + 1], hi_k = a.keyrange[2 * (size_t)row];
+  __syncthreads();
+  if (tid == 0) {
+    tc::mbar_arrive_expect_tx(&sh.ldbar, (uint32_t)m4 * 4u);
+    for (int o = 0; o < m4; o += 8192) {
+      const uint32_t bytes = (uint32_t)min(8192, m4 - o) * 4u;
+      asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                   ::"r"(tc::smem_u32(sv + o)), "l"(srow + o), "r"(bytes), "r"(tc::smem_u32(&sh.ldbar)) : "memory");
+    }
+  }
+  if (n > k && tid < m - m4) sv[m4 + tid] = srow[m4 + tid];
   // the scores have landed (bounded wait; on a timeout the error word is set)
   if (n > k && m4 > 0) {
     const bool ok = tc::mbar_wait(&sh.ldbar, 0);
@@ -795,13 +800,17 @@ cudaError_t sl_launch(Kern kern, int rows, int C, size_t smem, cudaStream_t st, 
   cfg.blockDim = dim3(SL_T);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = C;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // programmatic dependent launch: the prologue overlaps the previous kernel's tail; the
+  // kernels wait (griddepcontrol.wait) before reading anything that kernel writes
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   // a cluster of C CTAs of this size must fit on the GPU (checked once per kernel, C and size)
   static std::mutex mu;
   static std::map<std::tuple<const void*, int, size_t>, bool> fits;
