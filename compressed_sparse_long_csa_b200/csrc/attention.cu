@@ -126,31 +126,63 @@ attn_cuda_core_kernel(AttnArgs a) {
 template <typename T>
 __global__ void __launch_bounds__(128)
 attn_combine_kernel(AttnArgs a) {
+  __shared__ float wsh[64];            // per-split weight exp(m_s - M) / den
+  __shared__ float stat[2];            // M, den
   const int row = blockIdx.x, h = blockIdx.y;
   const int dv = a.dv, S = a.splits;
-  const float* P0 = a.part + ((size_t)row * S * a.H + h) * attn_part_stride(dv);
   const size_t sstride = (size_t)a.H * attn_part_stride(dv);
-  const float sk = a.sink[h];
-  float M = sk;
-  for (int s = 0; s < S; ++s) M = fmaxf(M, P0[s * sstride + dv]);
-  float den = 0.f;
-  if (M != -INFINITY) {
-    den = __expf(sk - M);
-    for (int s = 0; s < S; ++s) {
-      const float ms = P0[s * sstride + dv];
-      if (ms != -INFINITY) den += P0[s * sstride + dv + 1] * __expf(ms - M);
+  const float* P0 = a.part + ((size_t)row * S * a.H + h) * attn_part_stride(dv);
+  // the splits' (m, l) once, by the first warp
+  if (threadIdx.x < 32) {
+    float M = a.sink[h];
+    for (int s = threadIdx.x; s < S; s += 32) M = fmaxf(M, P0[s * sstride + dv]);
+    M = warp_max(M);
+    const float sk = a.sink[h];
+    float den = 0.f;
+    if (M != -INFINITY) {
+      for (int s = threadIdx.x; s < S; s += 32) {
+        const float ms = P0[s * sstride + dv];
+        if (ms != -INFINITY) den += P0[s * sstride + dv + 1] * __expf(ms - M);
+      }
+      den = warp_sum(den) + __expf(sk - M);
     }
-  }
-  const float inv = den > 0.f ? 1.f / den : 0.f;
-  for (int c = threadIdx.x; c < dv; c += blockDim.x) {
-    float acc = 0.f;
-    for (int s = 0; s < S; ++s) {
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    for (int s = threadIdx.x; s < S; s += 32) {
       const float ms = P0[s * sstride + dv];
-      if (ms != -INFINITY) acc = fmaf(P0[s * sstride + c], __expf(ms - M), acc);
+      wsh[s] = (ms == -INFINITY || M == -INFINITY) ? 0.f : __expf(ms - M) * inv;
     }
-    Elem<T>::st((T*)a.out + ((size_t)row * a.H + h) * dv + c, acc * inv);
+    if (threadIdx.x == 0) { stat[0] = M; stat[1] = den; }
   }
-  if (a.lse && threadIdx.x == 0) a.lse[(size_t)row * a.H + h] = den > 0.f ? M + logf(den) : -INFINITY;
+  __syncthreads();
+  // four values per thread and step, the splits' loads issued four at a time
+  for (int c = 4 * threadIdx.x; c < dv; c += 4 * blockDim.x) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    int s = 0;
+    for (; s + 4 <= S; s += 4) {
+      float4 x[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) x[u] = *reinterpret_cast<const float4*>(P0 + (s + u) * sstride + c);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float wgt = wsh[s + u];
+        acc.x = fmaf(wgt, x[u].x, acc.x); acc.y = fmaf(wgt, x[u].y, acc.y);
+        acc.z = fmaf(wgt, x[u].z, acc.z); acc.w = fmaf(wgt, x[u].w, acc.w);
+      }
+    }
+    for (; s < S; ++s) {
+      const float4 x = *reinterpret_cast<const float4*>(P0 + s * sstride + c);
+      const float wgt = wsh[s];
+      acc.x = fmaf(wgt, x.x, acc.x); acc.y = fmaf(wgt, x.y, acc.y);
+      acc.z = fmaf(wgt, x.z, acc.z); acc.w = fmaf(wgt, x.w, acc.w);
+    }
+    T* o = (T*)a.out + ((size_t)row * a.H + h) * dv + c;
+    Elem<T>::st(o, acc.x);
+    Elem<T>::st(o + 1, acc.y);
+    Elem<T>::st(o + 2, acc.z);
+    Elem<T>::st(o + 3, acc.w);
+  }
+  if (a.lse && threadIdx.x == 0)
+    a.lse[(size_t)row * a.H + h] = stat[1] > 0.f ? stat[0] + logf(stat[1]) : -INFINITY;
 }
 
 int attn_choose_splits(int n_queries, int H, int64_t rows, bool tc_path) {

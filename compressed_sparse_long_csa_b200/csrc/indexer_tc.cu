@@ -239,7 +239,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
 // (64-byte rows, 64-byte swizzle) and one ue8m0 scale per 32 elements applied inside the
 // tensor core.  The scale factors go to TMEM with tcgen05.st: for M rows, row m's four
 // scale bytes (k-blocks 0..3) sit in 32-bit column m/32 of lane m%32, replicated in all
-// four lane quarters; warps 8..11 (one per quarter) write them for every tile.  Each tile
+// four lane quarters; warps 12..15 (one per quarter) write them for every tile.  Each tile
 // is two MMAs of K = 64 (k-blocks 0-1, then 2-3: scale byte 0, then byte 2).
 constexpr int MX_KB = 64;                 // bytes per packed key row (128 e2m1)
 constexpr int MX_TILE_BYTES = IT_ROWS * MX_KB;
@@ -251,22 +251,25 @@ struct MxSmem {
   alignas(8) uint64_t full[STAGES];
   uint64_t empty[STAGES];
   uint64_t sfa_full[STAGES];
-  uint64_t tfull[2];
-  uint64_t tempty[2];
+  uint64_t tfull[4];
+  uint64_t tempty[4];
   uint64_t qfull;
   uint64_t sfb_ready;
   uint32_t tmem_base;
   int abort_flag;
   int t_begin, t_end;
+  int issued0;          // tile loads issued before the setup barrier
   int n_elig;
   float w[64];
 };
 
-// TMEM columns: two accumulators [0, 128), q scales at 128, key-scale ring at 136 + 4 * stage
-constexpr uint32_t MX_SFB = 128, MX_SFA = 136, MX_COLS = 256;
+// TMEM columns: four accumulators [0, 256), q scales at 256, key-scale ring at 264 + 4 * stage
+constexpr uint32_t MX_SFB = 256, MX_SFA = 264, MX_COLS = 512;
+constexpr int MX_NACC = 4;
+constexpr int MX_THREADS = 512;   // warp 0 TMA, 1 MMA, 4..11 epilogue (two warpgroups), 12..15 scale writers
 
 template <int STAGES>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(MX_THREADS, 1)
 indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ, IdxTcParams p) {
   extern __shared__ uint8_t smem_raw[];
   using Sm = MxSmem<STAGES>;
@@ -280,10 +283,12 @@ indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   const uint32_t* qsc = (const uint32_t*)a.qI_scale;                  // 4 ue8m0 bytes per head
 
   if (threadIdx.x == 0) {
+    tc::prefetch_tmap(&tmK);                 // descriptor fetches overlap the setup
+    tc::prefetch_tmap(&tmQ);
     for (int s = 0; s < STAGES; ++s) {
       tc::mbar_init(&sm.full[s], 1); tc::mbar_init(&sm.empty[s], 1); tc::mbar_init(&sm.sfa_full[s], 4);
     }
-    for (int s = 0; s < 2; ++s) { tc::mbar_init(&sm.tfull[s], 1); tc::mbar_init(&sm.tempty[s], 4); }
+    for (int s = 0; s < MX_NACC; ++s) { tc::mbar_init(&sm.tfull[s], 1); tc::mbar_init(&sm.tempty[s], 4); }
     tc::mbar_init(&sm.qfull, 1);
     tc::mbar_init(&sm.sfb_ready, 4);
     tc::fence_mbar_init();
@@ -295,23 +300,31 @@ indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     if (t1 > t_lim) t1 = t_lim;
     sm.t_begin = t0;
     sm.t_end = t1 > t0 ? t1 : t0;
+    // the query tile and the first key tiles go out before the setup barrier
+    const int n0 = sm.t_end - t0 < STAGES ? sm.t_end - t0 : STAGES;
+    if (n0 > 0) {
+      tc::mbar_arrive_expect_tx(&sm.qfull, 64 * MX_KB);
+      tc::tma_load_2d(sm.q, &tmQ, &sm.qfull, 0, row * 64);
+      for (int it = 0; it < n0; ++it) {
+        tc::mbar_arrive_expect_tx(&sm.full[it], MX_TILE_BYTES);
+        tc::tma_load_2d(sm.k[it], &tmK, &sm.full[it], 0, (int)(b * a.n_max) + (t0 + it) * IT_ROWS);
+      }
+    }
+    sm.issued0 = n0;
   }
   if (threadIdx.x < 64) sm.w[threadIdx.x] = threadIdx.x < a.H_I ? a.w[(size_t)row * a.H_I + threadIdx.x] : 0.f;
   if (warp == 1) { tc::tmem_alloc(&sm.tmem_base, MX_COLS); tc::tmem_relinquish(); }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
+  tc::griddep_launch_dependents();           // the selection kernel may start its prologue
   const uint32_t tmem = sm.tmem_base;
   const int t_begin = sm.t_begin, n_t = sm.t_end - sm.t_begin;
 
   if (warp == 0) {
     if (lane == 0 && n_t > 0) {
-      tc::prefetch_tmap(&tmK);
-      tc::prefetch_tmap(&tmQ);
-      tc::mbar_arrive_expect_tx(&sm.qfull, 64 * MX_KB);
-      tc::tma_load_2d(sm.q, &tmQ, &sm.qfull, 0, row * 64);
-      int issued = 0;
-      for (int it = 0; it < n_t; ++it) {
+      int issued = sm.issued0;
+      for (int it = issued; it < n_t; ++it) {
         const int st = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
         if (!tc::mbar_wait(&sm.empty[st], ph ^ 1)) { atomicExch(&sm.abort_flag, 1); break; }
@@ -334,8 +347,8 @@ indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       for (int it = 0; ok && it < n_t; ++it) {
         const int st = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
-        const int acc = it & 1;
-        const uint32_t aph = (it >> 1) & 1;
+        const int acc = it % MX_NACC;
+        const uint32_t aph = (it / MX_NACC) & 1;
         if (!tc::mbar_wait(&sm.tempty[acc], aph ^ 1) || !tc::mbar_wait(&sm.full[st], ph) ||
             !tc::mbar_wait(&sm.sfa_full[st], ph) || *(volatile int*)&sm.abort_flag) { ok = false; break; }
         tc::fence_after_sync();
@@ -349,10 +362,10 @@ indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       }
       if (!ok) {
         atomicExch(&sm.abort_flag, 1);
-        if (last_issued >= 0) tc::mbar_wait(&sm.tfull[last_issued & 1], (last_issued >> 1) & 1);
+        if (last_issued >= 0) tc::mbar_wait(&sm.tfull[last_issued % MX_NACC], (last_issued / MX_NACC) & 1);
       }
     }
-  } else if (warp >= 8) {
+  } else if (warp >= 12) {
     // scale-factor writers, one warp per lane quarter (all quarters hold the same data)
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     if (n_t > 0) {
@@ -388,17 +401,24 @@ indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       if (lane == 0) tc::mbar_arrive(&sm.sfa_full[st]);
     }
   } else if (warp >= 4) {
-    const int quarter = warp & 3;
+    // epilogue warpgroup e takes tiles e, e+2, ...; quarter q = warp % 4 reads TMEM lanes 32q..32q+31
+    const int e = (warp - 4) >> 2, quarter = warp & 3;
     const int r = quarter * 32 + lane;
     float kb = 0.f;
-    for (int it = 0; it < n_t; ++it) {
-      const int acc = it & 1;
-      const uint32_t aph = (it >> 1) & 1;
+    auto load_sc = [&](int it) {
+      const int s = (t_begin + it) * IT_ROWS + r;
+      return (it < n_t && s < a.n_max) ? __ldg(ksc + (size_t)b * a.n_max + s) : 0u;
+    };
+    uint32_t sc_next = load_sc(e);
+    for (int it = e; it < n_t; it += 2) {
+      const int acc = it % MX_NACC;
+      const uint32_t aph = (it / MX_NACC) & 1;
       const int s = (t_begin + it) * IT_ROWS + r;
       const bool valid = s < sm.n_elig;
+      const uint32_t sc = sc_next;
+      sc_next = load_sc(it + 2);
       // ||k_s|| <= 6 * sqrt(32 * sum_b scale_b^2): |e2m1| <= 6
       if (valid) {
-        const uint32_t sc = __ldg(ksc + (size_t)b * a.n_max + s);
         float ss = 0.f;
 #pragma unroll
         for (int q = 0; q < 4; ++q) { const float f = ue8m0_to_float((sc >> (8 * q)) & 0xFFu); ss = fmaf(f, f, ss); }
@@ -408,11 +428,18 @@ indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) { atomicExch(&sm.abort_flag, 1); break; }
       tc::fence_after_sync();
-      float val = 0.f;
-      uint32_t v[64];
-      tc::tmem_ld64(tmem + ((uint32_t)(quarter * 32) << 16) + acc * N, v);
+      float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int j = 0; j < 64; ++j) val = fmaf(sm.w[j], fmaxf(__uint_as_float(v[j]), 0.f), val);
+      for (int hlf = 0; hlf < 2; ++hlf) {
+        uint32_t v[32];
+        const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + acc * N + hlf * 32;
+        tc::tmem_ld16(ta, v);
+        tc::tmem_ld16(ta + 16, v + 16);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) part[j & 3] = fmaf(sm.w[hlf * 32 + j], fmaxf(__uint_as_float(v[j]), 0.f), part[j & 3]);
+      }
+      const float val = (part[0] + part[1]) + (part[2] + part[3]);
       if (valid) a.scores[(size_t)row * a.ld + s] = val;
       record_key_range(a.keyrange, row, val, valid);
       tc::fence_before_sync();
@@ -478,7 +505,7 @@ cudaError_t launch_mxf4(const IndexerArgs& a, cudaStream_t st, bool* used) {
   p.n_qg = a.Tq;
   p.tiles = (int)((a.n_max + IT_ROWS - 1) / IT_ROWS);
   const int64_t ctas = (int64_t)a.B * a.Tq;
-  int splits = (int)((148 + ctas - 1) / ctas);
+  int splits = (int)(148 / ctas);                   // one wave: one CTA per SM
   if (splits > p.tiles) splits = p.tiles;
   if (splits < 1) splits = 1;
   p.tiles_per_split = (p.tiles + splits - 1) / splits;
@@ -492,7 +519,7 @@ cudaError_t launch_mxf4(const IndexerArgs& a, cudaStream_t st, bool* used) {
   if (e != cudaSuccess) return e;
   dim3 grid(splits, a.Tq, a.B);
   note_launch();
-  indexer_mxf4_kernel<STAGES><<<grid, 384, smem, st>>>(mk, mq, p);
+  indexer_mxf4_kernel<STAGES><<<grid, MX_THREADS, smem, st>>>(mk, mq, p);
   *used = true;
   return cudaGetLastError();
 }
