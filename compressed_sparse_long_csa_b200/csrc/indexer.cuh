@@ -38,6 +38,27 @@ __device__ __forceinline__ int row_eligible(const IndexerArgs& a, int row) {
   return ne < n ? ne : n;
 }
 
+// Per-thread running order-key range of the scores a thread writes (flushed once, at
+// the end of a kernel, by flush_key_range).
+struct KeyRange {
+  uint32_t mx = 0u, nmn = 0u;           // max key, max of ~key (= ~min key)
+  __device__ __forceinline__ void add(float score) {
+    const uint32_t k = f32_order_key(score);
+    mx = max(mx, k);
+    nmn = max(nmn, ~k);
+  }
+};
+// Merge a warp's ranges for `row` into the workspace (one atomic pair per warp; all 32
+// lanes call; lanes that recorded nothing hold zeros, which change nothing).
+__device__ __forceinline__ void flush_key_range(unsigned* keyrange, int row, const KeyRange& r) {
+  const uint32_t mx = __reduce_max_sync(0xffffffffu, r.mx);
+  const uint32_t mn = __reduce_max_sync(0xffffffffu, r.nmn);
+  if ((threadIdx.x & 31) == 0 && (mx | mn) != 0u) {
+    atomicMax(keyrange + 2 * (size_t)row, mx);
+    atomicMax(keyrange + 2 * (size_t)row + 1, mn);
+  }
+}
+
 // Record the order-key range of a warp's scores for `row` (one atomic pair per warp).
 // Lanes without a score pass valid = false.  All 32 lanes must call.
 __device__ __forceinline__ void record_key_range(unsigned* keyrange, int row, float score, bool valid) {

@@ -183,6 +183,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
       return (it < n_t && s < a.n_max) ? __ldg(kscale + (size_t)b * a.n_max + s) : 0.f;
     };
     float sk_next = load_scale(e);
+    KeyRange kr[G];
     for (int it = e; it < n_t; it += 2) {
       const int acc = it % NACC;
       const uint32_t aph = (it / NACC) & 1;
@@ -213,13 +214,15 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         if (valid) {
           a.scores[(size_t)sm.row[g] * a.ld + s] = val * sk;
           kmax = fmaxf(kmax, sk);
+          kr[g].add(val * sk);
         }
-        record_key_range(a.keyrange, sm.row[g], val * sk, valid);
       }
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&sm.tempty[acc]);
     }
+#pragma unroll
+    for (int g = 0; g < G; ++g) flush_key_range(a.keyrange, sm.row[g], kr[g]);
     // |k8| <= 448 per element, so ||k_s|| <= sk * 448 * sqrt(d_I)
     kmax = warp_max(kmax);
     if (lane == 0 && kmax > 0.f) atomicMax(a.knmax + b, __float_as_uint(kmax * 448.f * 11.3137085f * 1.0001f));
@@ -410,6 +413,7 @@ indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       return (it < n_t && s < a.n_max) ? __ldg(ksc + (size_t)b * a.n_max + s) : 0u;
     };
     uint32_t sc_next = load_sc(e);
+    KeyRange kr;
     for (int it = e; it < n_t; it += 2) {
       const int acc = it % MX_NACC;
       const uint32_t aph = (it / MX_NACC) & 1;
@@ -440,12 +444,15 @@ indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         for (int j = 0; j < 32; ++j) part[j & 3] = fmaf(sm.w[hlf * 32 + j], fmaxf(__uint_as_float(v[j]), 0.f), part[j & 3]);
       }
       const float val = (part[0] + part[1]) + (part[2] + part[3]);
-      if (valid) a.scores[(size_t)row * a.ld + s] = val;
-      record_key_range(a.keyrange, row, val, valid);
+      if (valid) {
+        a.scores[(size_t)row * a.ld + s] = val;
+        kr.add(val);
+      }
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&sm.tempty[acc]);
     }
+    flush_key_range(a.keyrange, row, kr);
     kb = warp_max(kb);
     if (lane == 0 && kb > 0.f) atomicMax(a.knmax + b, __float_as_uint(kb * 1.0001f));
   }
