@@ -109,11 +109,9 @@ csa_compress_m4_kernel(const T* __restrict__ Ca, const T* __restrict__ Cb, const
   if (gid >= (int64_t)n_blk * groups) return;
   const int j = (int)(gid / groups);
   const int c0 = (int)(gid % groups) * VEC;
-  const int e = entry0[b] + j;
-  if (e < 0 || (int64_t)e >= n_max) { raise_err(err, CSA_DEVERR_ENTRY); return; }
+  const int e0 = entry0[b];                // in flight with the source loads below
   const size_t seq = (size_t)b * T_new * d;
   float c[2 * M][VEC], z[2 * M][VEC], bias[2 * M][VEC];
-  const bool has_b = e > 0;
 #pragma unroll
   for (int t = 0; t < M; ++t) {
     const T *cp, *zp;
@@ -124,7 +122,10 @@ csa_compress_m4_kernel(const T* __restrict__ Ca, const T* __restrict__ Cb, const
       const size_t off = ((size_t)b * M + t) * d + c0;
       cp = pCb + off; zp = pZb + off;
     }
-    if (has_b) { Elem<T>::ld_vec(cp, c[t]); Elem<T>::ld_vec(zp, z[t]); }
+    // the previous block's rows are read even for entry 0 (they exist; their terms are
+    // dropped below), so no load waits for entry0
+    Elem<T>::ld_vec(cp, c[t]);
+    Elem<T>::ld_vec(zp, z[t]);
     const size_t off = seq + (size_t)(j * M + t) * d + c0;
     Elem<T>::ld_vec(Ca + off, c[M + t]);
     Elem<T>::ld_vec(Za + off, z[M + t]);
@@ -137,6 +138,9 @@ csa_compress_m4_kernel(const T* __restrict__ Ca, const T* __restrict__ Cb, const
       bias[M + t][4 * q] = y.x; bias[M + t][4 * q + 1] = y.y; bias[M + t][4 * q + 2] = y.z; bias[M + t][4 * q + 3] = y.w;
     }
   }
+  const int e = e0 + j;
+  if (e < 0 || (int64_t)e >= n_max) { raise_err(err, CSA_DEVERR_ENTRY); return; }
+  const bool has_b = e > 0;
   float out[VEC];
 #pragma unroll
   for (int i = 0; i < VEC; ++i) {

@@ -72,13 +72,41 @@ def _ifmt(D):
     return {"f32": N.CSA_IFMT_F32, "e4m3": N.CSA_IFMT_E4M3, "mxfp4": N.CSA_IFMT_MXFP4}[D["ifmt"]]
 
 
-def csa_decode_step(T, D, stream=None):
+_SIDE = {}
+
+
+def _side_stream(device):
+    """A second stream per device for work that is independent of the main chain."""
+    key = torch.device(device).index
+    if key not in _SIDE:
+        _SIDE[key] = torch.cuda.Stream(device=device)
+    return _SIDE[key]
+
+
+def _csa_layer(T, D, stream, attend):
+    """One CSA layer: the compressor's cache append and the lightning indexer are
+    independent (the indexer scores the given indexer keys; the new cache entry is
+    read only by the attention), so the append runs on a side stream while the indexer
+    runs on the main one; the attention waits for both."""
+    main = stream if stream is not None else torch.cuda.current_stream()
+    side = _side_stream(main.device)
+    fork = torch.cuda.Event()
+    fork.record(main)
+    side.wait_event(fork)
     N.csa_compress(T["Ca"], T["Cb"], T["Za"], T["Zb"], T["Ba"], T["Bb"], T["prev_Cb"], T["prev_Zb"],
-                   T["entry0"], T["cache"], m=D["m"], stream=stream)
+                   T["entry0"], T["cache"], m=D["m"], stream=side)
+    join = torch.cuda.Event()
+    join.record(side)
     N.lightning_index(T["qI"], T.get("qI_scale"), T["w"], T["kI"], T.get("kI_scale"), T["n_entries"], T["q_pos"],
-                      D["k"], _ifmt(D), T["idx"], T["iws"], m=D["m"], stream=stream)
-    N.sparse_attn_decode(T["q"][:, 0], T["cache"], T["idx"][:, 0], T["win"], T["win_len"], T["sink"],
-                         D["sm_scale"], D["dv"], T["out"][:, 0], T["lse"][:, 0], T["aws"], stream=stream)
+                      D["k"], _ifmt(D), T["idx"], T["iws"], m=D["m"], stream=main)
+    main.wait_event(join)
+    attend(main)
+
+
+def csa_decode_step(T, D, stream=None):
+    _csa_layer(T, D, stream, lambda st: N.sparse_attn_decode(
+        T["q"][:, 0], T["cache"], T["idx"][:, 0], T["win"], T["win_len"], T["sink"], D["sm_scale"], D["dv"],
+        T["out"][:, 0], T["lse"][:, 0], T["aws"], stream=st))
 
 
 def hca_decode_step(T, D, stream=None, prefix=""):
@@ -91,12 +119,9 @@ def hca_decode_step(T, D, stream=None, prefix=""):
 
 
 def csa_prefill_step(T, D, stream=None):
-    N.csa_compress(T["Ca"], T["Cb"], T["Za"], T["Zb"], T["Ba"], T["Bb"], T["prev_Cb"], T["prev_Zb"],
-                   T["entry0"], T["cache"], m=D["m"], stream=stream)
-    N.lightning_index(T["qI"], T.get("qI_scale"), T["w"], T["kI"], T.get("kI_scale"), T["n_entries"], T["q_pos"],
-                      D["k"], _ifmt(D), T["idx"], T["iws"], m=D["m"], stream=stream)
-    N.sparse_attn_prefill(T["q"], T["q_pos"], T["cache"], T["idx"], T["raw"], T["raw_pos0"], D["W"], T["sink"],
-                          D["sm_scale"], D["dv"], T["out"], T["lse"], stream=stream)
+    _csa_layer(T, D, stream, lambda st: N.sparse_attn_prefill(
+        T["q"], T["q_pos"], T["cache"], T["idx"], T["raw"], T["raw_pos0"], D["W"], T["sink"], D["sm_scale"], D["dv"],
+        T["out"], T["lse"], stream=st))
 
 
 def hybrid_pair_step(T, D, stream=None):

@@ -97,7 +97,8 @@ uint64_t csa_launch_count(void);
  *                   at token m*entry0[b] of sequence b; T_new % m == 0
  *   Ba, Bb          device [m, d] fp32 positional biases
  *   prev_Cb, prev_Zb device [B, m, d] dtype: b-series of the block just before
- *                   the chunk (read only where entry0[b] > 0)
+ *                   the chunk (always allocated; its values count only where
+ *                   entry0[b] > 0)
  *   entry0          device [B] int32: index of the chunk's first entry
  *   cache           device [B, n_max, d] dtype: rows entry0[b] .. entry0[b]+T_new/m-1
  *                   are written (outputs rounded to nearest-even for bf16)
