@@ -581,32 +581,50 @@ indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
       } else qx[e] = ((const float*)a.qI)[r0 + i];
     }
   }
+  // weights and scales, and the words of this warp's heads for U = sum_j w_j ||q_j||
+  // (warp w takes heads w, w + SL_W, ...; lane l holds elements [epl*l, epl*l + epl)):
+  // every load of the prologue is issued before any is used
+  constexpr int EPL = (F == CSA_IFMT_MXFP4) ? 8 : 4;
+  float w_r = 0.f, qs_r[4] = {0.f, 0.f, 0.f, 0.f};
   if (tid < HI) {
-    sh.w[tid] = a.w[(size_t)row * HI + tid];
-    if (F == CSA_IFMT_E4M3) sh.qsc[tid] = ((const float*)a.qI_scale)[(size_t)row * HI + tid];
-    if (F == CSA_IFMT_MXFP4)
-      for (int bb = 0; bb < nb; ++bb)
-        sh.qsc[tid * nb + bb] = ue8m0_to_float(((const uint8_t*)a.qI_scale)[((size_t)row * HI + tid) * nb + bb]);
-  }
-  __syncthreads();                                         // w, scales and the barrier init are visible
-  // U = sum_j w_j ||q_j||: warp w takes heads w, w + SL_W, ...; lane l holds elements
-  // [epl*l, epl*l + epl) of the head (one 4- or 16-byte load, issued together)
-  if (tid == 0) sh.U = 0.f;
-  {
-    constexpr int EPL = (F == CSA_IFMT_MXFP4) ? 8 : 4;
-    float uw = 0.f;
-    uint4 qv[64 / SL_W];
+    w_r = a.w[(size_t)row * HI + tid];
+    if (F == CSA_IFMT_E4M3) qs_r[0] = ((const float*)a.qI_scale)[(size_t)row * HI + tid];
+    if (F == CSA_IFMT_MXFP4) {
 #pragma unroll
-    for (int h = 0; h < 64 / SL_W; ++h) {
-      const int j = warp + SL_W * h;
-      qv[h] = make_uint4(0u, 0u, 0u, 0u);
-      if (j < HI && lane * EPL < dI) {
-        const size_t e0 = r0 + (size_t)j * dI + lane * EPL;
-        if (F == CSA_IFMT_E4M3) qv[h].x = *reinterpret_cast<const uint32_t*>((const uint8_t*)a.qI + e0);
-        else if (F == CSA_IFMT_MXFP4) qv[h].x = *reinterpret_cast<const uint32_t*>((const uint8_t*)a.qI + e0 / 2);
-        else qv[h] = *reinterpret_cast<const uint4*>((const float*)a.qI + e0);
-      }
+      for (int bb = 0; bb < 4; ++bb)
+        if (bb < nb) qs_r[bb] = ue8m0_to_float(((const uint8_t*)a.qI_scale)[((size_t)row * HI + tid) * nb + bb]);
     }
+  }
+  uint4 qv[64 / SL_W];
+#pragma unroll
+  for (int h = 0; h < 64 / SL_W; ++h) {
+    const int j = warp + SL_W * h;
+    qv[h] = make_uint4(0u, 0u, 0u, 0u);
+    if (j < HI && lane * EPL < dI) {
+      const size_t e0 = r0 + (size_t)j * dI + lane * EPL;
+      if (F == CSA_IFMT_E4M3) qv[h].x = *reinterpret_cast<const uint32_t*>((const uint8_t*)a.qI + e0);
+      else if (F == CSA_IFMT_MXFP4) qv[h].x = *reinterpret_cast<const uint32_t*>((const uint8_t*)a.qI + e0 / 2);
+      else qv[h] = *reinterpret_cast<const uint4*>((const float*)a.qI + e0);
+    }
+  }
+  // ---- the scoring kernel's outputs: key-norm bound and key range (the scores follow
+  // by one bulk copy into shared memory, the tail by plain loads)
+  tc::griddep_wait();
+  const float knmax = __uint_as_float(a.knmax[b]);
+  // the key range the scoring kernel recorded (exact min / max over the row's eligible entries)
+  uint32_t lo_k = ~a.keyrange[2 * (size_t)row + 1], hi_k = a.keyrange[2 * (size_t)row];
+  if (tid < HI) {
+    sh.w[tid] = w_r;
+    if (F == CSA_IFMT_E4M3) sh.qsc[tid] = qs_r[0];
+    if (F == CSA_IFMT_MXFP4) {
+#pragma unroll
+      for (int bb = 0; bb < 4; ++bb)
+        if (bb < nb) sh.qsc[tid * nb + bb] = qs_r[bb];
+    }
+  }
+  if (tid == 0) sh.U = 0.f;
+  __syncthreads();                                         // w, scales, U = 0 and the barrier init are visible
+  {
     float n2[64 / SL_W];
 #pragma unroll
     for (int h = 0; h < 64 / SL_W; ++h) {
@@ -632,21 +650,14 @@ indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
 #pragma unroll
       for (int h = 0; h < 64 / SL_W; ++h) n2[h] += __shfl_xor_sync(0xffffffffu, n2[h], o);
     }
+    float uw = 0.f;
 #pragma unroll
     for (int h = 0; h < 64 / SL_W; ++h) {
       const int j = warp + SL_W * h;
       if (j < HI) uw += sh.w[j] * sqrtf(n2[h]);
     }
-    __syncthreads();                                       // sh.U = 0 is visible
-    if (lane == 0) atomicAdd(&sh.U, uw);
+    if (lane == 0) atomicAdd(&sh.U, uw);                   // read after the barriers below
   }
-  // ---- the scoring kernel's outputs: scores (one bulk copy into shared memory, the tail
-  // by plain loads), key-norm bound and key range
-  tc::griddep_wait();
-  const float knmax = __uint_as_float(a.knmax[b]);
-  // the key range the scoring kernel recorded (exact min / max over the row's eligible entries)
-  uint32_t lo_k = ~a.keyrange[2 * (size_t)row + 1], hi_k = a.keyrange[2 * (size_t)row];
-  __syncthreads();
   if (tid == 0) {
     tc::mbar_arrive_expect_tx(&sh.ldbar, (uint32_t)m4 * 4u);
     for (int o = 0; o < m4; o += 8192) {
