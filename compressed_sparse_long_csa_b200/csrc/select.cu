@@ -789,11 +789,19 @@ indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
 }
 
 // Cluster size and chunk: the fewest CTAs (at most SL_CMAX) whose shared memory holds
-// the row; chunk is a multiple of 1024 entries.
-bool sl_plan(int64_t n, int* C, int* chunk) {
+// the row, more when there are few rows; chunk is a multiple of 1024 entries.
+bool sl_plan(int64_t n, int rows, int* C, int* chunk) {
   const int64_t c = (n + SL_CHUNK - 1) / SL_CHUNK;
   if (c > SL_CMAX) return false;
-  const int64_t cc = c < 1 ? 1 : c;
+  int64_t cc = c < 1 ? 1 : c;
+  // few rows: up to four CTAs per row (their passes over the scores are shorter, their
+  // band re-scoring is shared), while each CTA keeps at least 4096 entries
+  if ((int64_t)rows * cc < 148) {
+    int64_t want = 148 / rows;
+    if (want > 4) want = 4;
+    while (want > cc && (n + want - 1) / want < 4096) --want;
+    if (want > cc) cc = want;
+  }
   int64_t ch = (n + cc - 1) / cc;
   ch = (ch + 1023) / 1024 * 1024;
   if (ch < 1024) ch = 1024;
@@ -851,7 +859,7 @@ static_assert(SL_FIXED + sizeof(Resc) <= 232448 && SL_FIXED + (size_t)SL_CHUNK *
 cudaError_t launch_indexer_select_cluster(const IndexerArgs& a, cudaStream_t st) {
   int C, chunk;
   const int rows = a.B * a.Tq;
-  if (a.H_I > 64 || a.d_I > 128 || a.H_I * a.d_I > SL_QPT * SL_T || !sl_plan(a.n_max, &C, &chunk) || (a.ld % 4) != 0 ||
+  if (a.H_I > 64 || a.d_I > 128 || a.H_I * a.d_I > SL_QPT * SL_T || !sl_plan(a.n_max, rows, &C, &chunk) || (a.ld % 4) != 0 ||
       ((uintptr_t)a.scores & 15) != 0 || (int64_t)rows * C > 0x7fffffffLL)
     return cudaErrorNotSupported;
   const size_t region = std::max((size_t)chunk * 4, sizeof(Resc));
@@ -863,7 +871,7 @@ cudaError_t launch_indexer_select_cluster(const IndexerArgs& a, cudaStream_t st)
 cudaError_t launch_topk_select_cluster(const float* scores, int64_t ld, const int32_t* n_valid, int R, int64_t n,
                                        int k, int32_t* idx_out, cudaStream_t st) {
   int C, chunk;
-  if (!sl_plan(n, &C, &chunk) || (int64_t)R * C > 0x7fffffffLL) return cudaErrorNotSupported;
+  if (!sl_plan(n, R, &C, &chunk) || (int64_t)R * C > 0x7fffffffLL) return cudaErrorNotSupported;
   const int vec = (ld % 4 == 0) && (((uintptr_t)scores & 15) == 0);
   return sl_launch(topk_cluster_kernel, R, C, SL_FIXED + (size_t)chunk * 4, st, scores, ld, n_valid, n, k, idx_out,
                    chunk, vec);
