@@ -243,8 +243,10 @@ static csa_status run_attention(AttnArgs& a, int dtype, void* workspace, size_t 
   a.part = (float*)workspace;
   bool used = false, combined = false;
   cudaError_t e = cudaSuccess;
+  a.part_fp16 = 0;
   if (tc) e = launch_attention_tc(a, st, &used, &combined);
   if (e != cudaSuccess) return CSA_ERR_CUDA;
+  if (used) a.part_fp16 = 1;                   // the tensor-core kernel's partial format
   if (!used) {
     if (tc) {  // the tensor-core path declined: recompute the split plan for the CUDA-core path
       a.splits = decode ? attn_choose_splits(a.B * a.Tq, a.H, rows, false) : 1;

@@ -126,52 +126,75 @@ attn_cuda_core_kernel(AttnArgs a) {
 template <typename T>
 __global__ void __launch_bounds__(128)
 attn_combine_kernel(AttnArgs a) {
-  __shared__ float wsh[64];            // per-split weight exp(m_s - M) / den
+  __shared__ float wsh[2][64];         // per split and half row: exp(m_s - M) / den (x l_s p_s in format 1)
   __shared__ float stat[2];            // M, den
   const int row = blockIdx.x, h = blockIdx.y;
-  const int dv = a.dv, S = a.splits;
-  const size_t sstride = (size_t)a.H * attn_part_stride(dv);
-  const float* P0 = a.part + ((size_t)row * S * a.H + h) * attn_part_stride(dv);
+  const int dv = a.dv, S = a.splits, H = a.H;
+  const size_t sstride = attn_part_block(H, dv);
+  const float* B0 = a.part + (size_t)row * S * sstride;     // block of split s: B0 + s * sstride
   // the splits' (m, l) once, by the first warp
   if (threadIdx.x < 32) {
+    auto rec_m = [&](int s) { return a.part_fp16 ? B0[s * sstride + attn_part16_rec(H, dv, h)]
+                                                 : B0[s * sstride + (size_t)h * attn_part_stride(dv) + dv]; };
+    auto rec_l = [&](int s) { return a.part_fp16 ? B0[s * sstride + attn_part16_rec(H, dv, h) + 1]
+                                                 : B0[s * sstride + (size_t)h * attn_part_stride(dv) + dv + 1]; };
     float M = a.sink[h];
-    for (int s = threadIdx.x; s < S; s += 32) M = fmaxf(M, P0[s * sstride + dv]);
+    for (int s = threadIdx.x; s < S; s += 32) M = fmaxf(M, rec_m(s));
     M = warp_max(M);
     const float sk = a.sink[h];
     float den = 0.f;
     if (M != -INFINITY) {
       for (int s = threadIdx.x; s < S; s += 32) {
-        const float ms = P0[s * sstride + dv];
-        if (ms != -INFINITY) den += P0[s * sstride + dv + 1] * __expf(ms - M);
+        const float ms = rec_m(s);
+        if (ms != -INFINITY) den += rec_l(s) * __expf(ms - M);
       }
       den = warp_sum(den) + __expf(sk - M);
     }
     const float inv = den > 0.f ? 1.f / den : 0.f;
     for (int s = threadIdx.x; s < S; s += 32) {
-      const float ms = P0[s * sstride + dv];
-      wsh[s] = (ms == -INFINITY || M == -INFINITY) ? 0.f : __expf(ms - M) * inv;
+      const float ms = rec_m(s);
+      const float w = (ms == -INFINITY || M == -INFINITY) ? 0.f : __expf(ms - M) * inv;
+      if (a.part_fp16) {
+        const float* r = B0 + s * sstride + attn_part16_rec(H, dv, h);
+        wsh[0][s] = w * r[1] * r[2];
+        wsh[1][s] = w * r[1] * r[3];
+      } else {
+        wsh[0][s] = w;
+        wsh[1][s] = w;
+      }
     }
     if (threadIdx.x == 0) { stat[0] = M; stat[1] = den; }
   }
   __syncthreads();
   // four values per thread and step, the splits' loads issued four at a time
   for (int c = 4 * threadIdx.x; c < dv; c += 4 * blockDim.x) {
+    const float* wc = wsh[(a.part_fp16 && 2 * c >= dv) ? 1 : 0];
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    auto load = [&](int s) -> float4 {
+      if (a.part_fp16) {
+        const uint2 u = *reinterpret_cast<const uint2*>(reinterpret_cast<const __half*>(B0 + s * sstride) +
+                                                        attn_part16_val(H, h, c));
+        const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
+        const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
+        return make_float4(lo.x, lo.y, hi.x, hi.y);
+      }
+      return *reinterpret_cast<const float4*>(B0 + s * sstride + (size_t)h * attn_part_stride(dv) + c);
+    };
     int s = 0;
     for (; s + 4 <= S; s += 4) {
       float4 x[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) x[u] = *reinterpret_cast<const float4*>(P0 + (s + u) * sstride + c);
+      for (int u = 0; u < 4; ++u) x[u] = load(s + u);
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const float wgt = wsh[s + u];
+        const float wgt = wc[s + u];
         acc.x = fmaf(wgt, x[u].x, acc.x); acc.y = fmaf(wgt, x[u].y, acc.y);
         acc.z = fmaf(wgt, x[u].z, acc.z); acc.w = fmaf(wgt, x[u].w, acc.w);
       }
     }
     for (; s < S; ++s) {
-      const float4 x = *reinterpret_cast<const float4*>(P0 + s * sstride + c);
-      const float wgt = wsh[s];
+      const float4 x = load(s);
+      const float wgt = wc[s];
       acc.x = fmaf(wgt, x.x, acc.x); acc.y = fmaf(wgt, x.y, acc.y);
       acc.z = fmaf(wgt, x.z, acc.z); acc.w = fmaf(wgt, x.w, acc.w);
     }
@@ -193,6 +216,7 @@ int attn_choose_splits(int n_queries, int H, int64_t rows, bool tc_path) {
     // 64-row tiles, and the tiles spread as evenly as whole tiles allow
     s = 148 / (2 * (int64_t)n_queries);
     if (s > tiles / 2) s = tiles / 2;
+    if (s > 64) s = 64;                      // attn_combine_kernel keeps 64 splits' weights
     if (s < 1) s = 1;
     const int64_t per = (tiles + s - 1) / s;
     s = (tiles + per - 1) / per;

@@ -2,6 +2,8 @@
 #pragma once
 #include "common.cuh"
 
+#include <cuda_fp16.h>
+
 namespace csa {
 
 struct AttnArgs {
@@ -23,9 +25,11 @@ struct AttnArgs {
   float sm_scale;
   void* out;                  // [B*Tq, H, dv]
   float* lse;                 // [B*Tq, H] or null
-  float* part;                // split partials [B*Tq, splits, H, attn_part_stride(dv)]
+  float* part;                // split partials: [B*Tq, splits] blocks of attn_part_block(H, dv) floats
+  int part_fp16;              // partial block format (see attn_part_block)
   int splits;
-  int rows_per_split;
+  int rows_per_split;         // CUDA-core path: contiguous virtual rows per split (the
+                              // tensor-core path deals 64-row tiles to the splits round-robin)
   int n_seg_a;                // virtual rows in segment A (k or n_max)
   int cluster_combine;        // tensor-core path: splits merged inside a thread-block cluster
   unsigned* err;
@@ -34,6 +38,17 @@ struct AttnArgs {
 // Floats per (query, split, head) record of the split partials: o[dv], m, l, 2 pad,
 // so that every record starts on a 16-byte boundary (vector stores).
 __host__ __device__ inline int attn_part_stride(int dv) { return dv + 4; }
+// Floats per (query, split) block of the split partials.  Two formats fit in it:
+//   0 (CUDA-core kernel): per head [H][attn_part_stride(dv)] fp32: o[dv], m, l, 2 pad;
+//   1 (tensor-core kernel): o as fp16 at [dv/8][H][8] (a warp's heads store contiguous
+//     16-byte pieces), each half row divided by l and by a power of two that puts its
+//     largest magnitude in [0.5, 1); then per head a float4 {m, l, p_lo, p_hi}, the powers
+//     of two of columns [0, dv/2) and [dv/2, dv).  o = stored * p * l.
+__host__ __device__ inline size_t attn_part_block(int H, int dv) { return (size_t)H * attn_part_stride(dv); }
+// format 1: offset (in halves) of values c..c+3 of head h (c a multiple of 4)
+__host__ __device__ inline size_t attn_part16_val(int H, int h, int c) { return ((size_t)(c >> 3) * H + h) * 8 + (c & 7); }
+// format 1: offset (in floats) of the record of head h
+__host__ __device__ inline size_t attn_part16_rec(int H, int dv, int h) { return (size_t)dv * H / 2 + 4 * (size_t)h; }
 
 // Number of virtual rows of a query: compressed segment + window segment.
 __host__ __device__ inline int64_t attn_virtual_rows(const AttnArgs& a) { return (int64_t)a.n_seg_a + a.W; }

@@ -20,11 +20,12 @@
 //   3. softmax threads (one per head, TMEM lanes 16-31) run an online softmax with a
 //      lazily raised running max and write P (bf16) to shared memory;
 //   4. O += P V (M=64, N=2x256, K=64; V is read MN-major from the same tile).
-// At the end, threads of TMEM lanes 0-15 normalise O (one split), or the split partials
-// (o, m, l) are merged: the CTAs of one query's head half form a thread-block cluster,
-// stage their partials in shared memory and each merges a slice of the heads from all
-// of them through distributed shared memory (at most 8 splits), else the partials go to
-// global memory for attn_combine.  Every wait is bounded (CSA_DEVERR_TIMEOUT).
+// At the end, threads of TMEM lanes 0-15 normalise O (one split), or write the split
+// partial (o, m, l) to the workspace.  The CTAs of one query's head half form a
+// thread-block cluster (at most 8 splits): after a cluster barrier each merges a slice
+// of the heads from every split's partial, read back from L2 (distributed shared memory
+// moved these partials at about 40 GB/s per SM, several times slower).  Without a
+// cluster attn_combine merges them.  Every wait is bounded (CSA_DEVERR_TIMEOUT).
 #include "attention.cuh"
 #include "tc.cuh"
 
@@ -50,7 +51,6 @@ constexpr int AT_THREADS = (AT_SMW + 1) * 32 + 2 * AT_GROUP;
 constexpr float AT_RESCALE_THRESH = 8.0f;
 constexpr int ATOM = AT_ROWS * 128;      // one 64-row x 128-byte swizzle atom
 constexpr unsigned long long NO_RUN = ~0ull;
-constexpr int OST_LD = 516;              // staged partial row: 512 values + pad (16-byte aligned rows)
 
 struct AtSmem {
   alignas(1024) uint8_t q[AT_ATOMS][AT_HC * 128];          // 72 KB
@@ -114,10 +114,11 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
   const int hh = blockIdx.x / a.splits, split = blockIdx.x - hh * a.splits;   // a cluster spans the splits
   const int row = blockIdx.y;                       // query row b*Tq + t
   const int64_t nrows = attn_virtual_rows(a);
-  const int64_t v0 = (int64_t)split * a.rows_per_split;
-  int64_t v1 = v0 + a.rows_per_split;
-  if (v1 > nrows) v1 = nrows;
-  const int n_t = v1 > v0 ? (int)((v1 - v0 + AT_ROWS - 1) / AT_ROWS) : 0;
+  // The 64-row tiles of the query's virtual rows are dealt to the splits round-robin
+  // (split s takes tiles s, s + S, ...), so the gathered top-k tiles and the contiguous
+  // window tiles (one TMA copy each, several times faster) spread evenly over the splits.
+  const int tiles_all = (int)((nrows + AT_ROWS - 1) / AT_ROWS);
+  const int n_t = split < tiles_all ? (tiles_all - split + a.splits - 1) / a.splits : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
@@ -142,6 +143,15 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
   tc::griddep_wait();
   tc::griddep_launch_dependents();
   const uint32_t tmem = sm.tmem_base;
+  // The sink logit, needed only at the end, is loaded now: with one split by every softmax
+  // thread for its head, else by threads [0, hp) for the heads they merge.
+  const int merge_hp = (AT_HC + a.splits - 1) / a.splits, merge_h0 = split * merge_hp;
+  float sink_pre = 0.f;
+  if (a.splits == 1) {
+    if (warp < AT_SMW) sink_pre = a.sink[hh * AT_HC + (warp & 3) * 16 + (lane & 15)];
+  } else if ((int)threadIdx.x < merge_hp && merge_h0 + (int)threadIdx.x < AT_HC) {
+    sink_pre = a.sink[hh * AT_HC + merge_h0 + threadIdx.x];
+  }
 
   if (warp >= AT_LDW) {
     // ------------------------------------------------------------------ loader group g (64 threads)
@@ -161,8 +171,8 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
       which = -1;
       y = 0;
       if (lg < AT_ROWS) {
-        const int64_t v = v0 + (int64_t)t * AT_ROWS + lg;
-        if (v < v1) which = attn_row_coord(a, row, (int)v, &y);
+        const int64_t v = (int64_t)(split + t * a.splits) * AT_ROWS + lg;
+        if (v < nrows) which = attn_row_coord(a, row, (int)v, &y);
       }
     };
     if (g < n_t) coord(g);
@@ -411,7 +421,7 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
     const float m_h = __shfl_sync(0xffffffffu, m_run, (lane & 15) + 16);
     const float l_h = __shfl_sync(0xffffffffu, l_tot, (lane & 15) + 16);
     if (a.splits == 1) {
-      const float sk = a.sink[h];
+      const float sk = sink_pre;
       const float mh = have_o ? m_h : -INFINITY;
       const float M = fmaxf(sk, mh);
       float den = 0.f, f = 0.f;
@@ -441,33 +451,25 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
         }
       }
       if (a.lse && !is_s && wg == 0) a.lse[(size_t)row * AT_H + h] = den > 0.f ? M + logf(den) : -INFINITY;
-    } else if (a.cluster_combine) {
-      // stage the partial in shared memory (the KV stages are idle: every PV has completed)
-      float* ost = reinterpret_cast<float*>(&sm.kv[0][0][0]);
-      float* ost_ml = ost + AT_HC * OST_LD;
-#pragma unroll 1
-      for (int c = 4 * wg; c < 4 * wg + 4; ++c) {
-        uint32_t v[64];
-        if (have_o) {
-          tc::tmem_ld64(tmem + lane_base + c * 64, v);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 64; ++j) v[j] = 0u;
-        }
-        if (!is_s) {
-          float4* d4 = reinterpret_cast<float4*>(ost + hl * OST_LD + c * 64);
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            d4[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]), __uint_as_float(v[4 * j + 2]),
-                                __uint_as_float(v[4 * j + 3]));
-        }
-      }
-      if (!is_s && wg == 0) {
-        ost_ml[2 * hl] = have_o ? m_h : -INFINITY;
-        ost_ml[2 * hl + 1] = have_o ? l_h : 0.f;
-      }
     } else {
-      float* P = a.part + (((size_t)row * a.splits + split) * AT_H + h) * attn_part_stride(512);
+      // Split partial, format 1 of attn_part_block: this thread's half row (256 values)
+      // divided by l and by the power of two that puts its largest magnitude in [0.5, 1),
+      // stored as fp16 at [512/8][128 heads][8], so that the 16 O lanes of a warp (16
+      // consecutive heads) store 256 contiguous bytes.
+      float* blk = a.part + ((size_t)row * a.splits + split) * attn_part_block(AT_H, 512);
+      float amax = 0.f;
+#pragma unroll 1
+      for (int c = 4 * wg; c < 4 * wg + 4 && have_o; ++c) {
+        uint32_t v[64];
+        tc::tmem_ld64(tmem + lane_base + c * 64, v);
+#pragma unroll
+        for (int j = 0; j < 64; ++j) amax = fmaxf(amax, fabsf(__uint_as_float(v[j])));
+      }
+      const float inv_l = (have_o && l_h > 0.f) ? 1.f / l_h : 0.f;
+      int e2 = 0;
+      frexpf(amax * inv_l, &e2);
+      const float f = inv_l * ldexpf(1.f, -e2);
+      uint4* d16 = reinterpret_cast<uint4*>(blk) + h;
 #pragma unroll 1
       for (int c = 4 * wg; c < 4 * wg + 4; ++c) {
         uint32_t v[64];
@@ -478,16 +480,26 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
           for (int j = 0; j < 64; ++j) v[j] = 0u;
         }
         if (!is_s) {
-          float4* d4 = reinterpret_cast<float4*>(P + c * 64);
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            d4[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]), __uint_as_float(v[4 * j + 2]),
-                                __uint_as_float(v[4 * j + 3]));
+          for (int q = 0; q < 8; ++q) {
+            uint32_t w4[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const __half2 hv = __floats2half2_rn(__uint_as_float(v[8 * q + 2 * u]) * f,
+                                                   __uint_as_float(v[8 * q + 2 * u + 1]) * f);
+              w4[u] = *reinterpret_cast<const uint32_t*>(&hv);
+            }
+            d16[(size_t)(c * 8 + q) * AT_H] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          }
         }
       }
-      if (!is_s && wg == 0) {
-        P[512] = have_o ? m_h : -INFINITY;
-        P[513] = have_o ? l_h : 0.f;
+      if (!is_s) {
+        float* rec = blk + 512 * AT_H / 2 + 4 * (size_t)h;
+        if (wg == 0) {
+          rec[0] = have_o ? m_h : -INFINITY;
+          rec[1] = have_o ? l_h : 0.f;
+        }
+        rec[2 + wg] = ldexpf(1.f, e2);
       }
     }
   }
@@ -499,74 +511,94 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
     tc::tmem_dealloc(tmem, TM_COLS);
   }
   if (a.cluster_combine) {
-    // merge heads [h0, h1) of this head half from every split's staged partial
+    // Merge heads [h0, h1) of this head half from every split's partial.  The partials are
+    // in the workspace (L2): a cluster barrier (release / acquire at cluster scope) orders
+    // their stores before these loads, which bypass L1.
     namespace cg = cooperative_groups;
-    cg::cluster_group cluster = cg::this_cluster();
-    cluster.sync();
+    cg::this_cluster().sync();
     const int S = a.splits;
-    const int hp = (AT_HC + S - 1) / S;
-    const int h0 = split * hp, h1 = min(AT_HC, h0 + hp);
-    float* wts = reinterpret_cast<float*>(&sm.q[0][0]);          // [head][split] merge weights (Q is idle)
-    float* ost_local = reinterpret_cast<float*>(&sm.kv[0][0][0]);
-    // peer base addresses, all loads of a step issued before any is used (S <= 8)
-    const float* peer[8];
+    const int hp = merge_hp, h0 = merge_h0, h1 = min(AT_HC, h0 + hp);
+    const size_t blkn = attn_part_block(AT_H, 512);
+    const float* blk0 = a.part + (size_t)row * S * blkn;      // split p: blk0 + p * blkn
+    const int hg0 = hh * AT_HC + h0;                          // first merged head within the query
+    const int nh = h1 > h0 ? h1 - h0 : 1;                     // heads merged here (the last slice may be short)
+    const int items = h1 > h0 ? nh * (512 / 8) : 0;           // (8-column piece, head), heads fastest
+    float* wts = reinterpret_cast<float*>(&sm.q[0][0]);       // [head][half][split] merge weights (Q is idle)
+    constexpr int OT_PITCH = 1040;                            // bytes per staged output row (16-byte multiple)
+    uint8_t* ot = &sm.q[0][0] + 4096;                         // [head][512] bf16 output rows
+    // the first item's partials are loaded before the weights are known
+    uint4 x[8];
+    int it = threadIdx.x;
+    auto load_item = [&](int i) {
+      const int hr = i % nh, c8 = i / nh;
 #pragma unroll
-    for (int p = 0; p < 8; ++p) peer[p] = cluster.map_shared_rank(ost_local, p < S ? p : 0);
+      for (int p = 0; p < 8; ++p)
+        x[p] = (p < S && i < items)
+                   ? __ldcg(reinterpret_cast<const uint4*>(blk0 + p * blkn) + (size_t)c8 * AT_H + hg0 + hr)
+                   : make_uint4(0u, 0u, 0u, 0u);
+    };
+    load_item(it);
     if ((int)threadIdx.x < h1 - h0) {
       const int hl = h0 + threadIdx.x;
-      const float sk = a.sink[hh * AT_HC + hl];
-      float ms[8], ls[8];
+      const float sk = sink_pre;
+      float4 rc[8];
 #pragma unroll
-      for (int p = 0; p < 8; ++p) {
-        ms[p] = -INFINITY;
-        ls[p] = 0.f;
-        if (p < S) {
-          ms[p] = peer[p][AT_HC * OST_LD + 2 * hl];
-          ls[p] = peer[p][AT_HC * OST_LD + 2 * hl + 1];
-        }
-      }
+      for (int p = 0; p < 8; ++p)
+        rc[p] = p < S ? __ldcg(reinterpret_cast<const float4*>(blk0 + p * blkn + 512 * AT_H / 2) + hh * AT_HC + hl)
+                      : make_float4(-INFINITY, 0.f, 0.f, 0.f);
       float M = sk;
 #pragma unroll
-      for (int p = 0; p < 8; ++p) M = fmaxf(M, ms[p]);
+      for (int p = 0; p < 8; ++p) M = fmaxf(M, rc[p].x);
       float den = 0.f;
       if (M != -INFINITY) {
         den = __expf(sk - M);
 #pragma unroll
         for (int p = 0; p < 8; ++p)
-          if (ms[p] != -INFINITY) den += ls[p] * __expf(ms[p] - M);
+          if (rc[p].x != -INFINITY) den += rc[p].y * __expf(rc[p].x - M);
       }
       const float inv = den > 0.f ? 1.f / den : 0.f;
 #pragma unroll
-      for (int p = 0; p < 8; ++p)
-        wts[(hl - h0) * 8 + p] = (ms[p] == -INFINITY || M == -INFINITY) ? 0.f : __expf(ms[p] - M) * inv;
+      for (int p = 0; p < 8; ++p) {
+        const float w = (rc[p].x == -INFINITY || M == -INFINITY) ? 0.f : __expf(rc[p].x - M) * inv * rc[p].y;
+        wts[(hl - h0) * 16 + p] = w * rc[p].z;
+        wts[(hl - h0) * 16 + 8 + p] = w * rc[p].w;
+      }
       if (a.lse) a.lse[(size_t)row * AT_H + hh * AT_HC + hl] = den > 0.f ? M + logf(den) : -INFINITY;
     }
     __syncthreads();
-    const int items = (h1 - h0) * (512 / 4);
-    for (int it = threadIdx.x; it < items; it += AT_THREADS) {
-      const int hr = it >> 7, c4 = it & 127;
-      const int hl = h0 + hr;
-      float4 x[8];
+    for (; it < items; it += AT_THREADS) {
+      const int hr = it % nh, c8 = it / nh;
+      const float* wr = wts + hr * 16 + (c8 >= 32 ? 8 : 0);
+      float acc[8];
 #pragma unroll
-      for (int p = 0; p < 8; ++p)
-        x[p] = p < S ? *reinterpret_cast<const float4*>(peer[p] + hl * OST_LD + 4 * c4) : make_float4(0.f, 0.f, 0.f, 0.f);
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int j = 0; j < 8; ++j) acc[j] = 0.f;
 #pragma unroll
       for (int p = 0; p < 8; ++p) {
-        const float wgt = wts[hr * 8 + p];
-        acc.x = fmaf(wgt, x[p].x, acc.x);
-        acc.y = fmaf(wgt, x[p].y, acc.y);
-        acc.z = fmaf(wgt, x[p].z, acc.z);
-        acc.w = fmaf(wgt, x[p].w, acc.w);
+        const float wgt = wr[p];
+        const uint32_t u[4] = {x[p].x, x[p].y, x[p].z, x[p].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&u[q]));
+          acc[2 * q] = fmaf(wgt, f2.x, acc[2 * q]);
+          acc[2 * q + 1] = fmaf(wgt, f2.y, acc[2 * q + 1]);
+        }
       }
-      __nv_bfloat16* o = (__nv_bfloat16*)a.out + ((size_t)row * AT_H + hh * AT_HC + hl) * 512 + 4 * c4;
-      __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x, acc.y), hi2 = __floats2bfloat162_rn(acc.z, acc.w);
-      uint2 pk;
-      pk.x = *reinterpret_cast<uint32_t*>(&lo2);
-      pk.y = *reinterpret_cast<uint32_t*>(&hi2);
-      *reinterpret_cast<uint2*>(o) = pk;
+      if (it + AT_THREADS < items) load_item(it + AT_THREADS);
+      uint32_t pk[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
+        pk[q] = *reinterpret_cast<uint32_t*>(&b2);
+      }
+      *reinterpret_cast<uint4*>(ot + hr * OT_PITCH + c8 * 16) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
-    cluster.sync();                                  // peers may still read this CTA's staged partial
+    __syncthreads();
+    // the merged rows leave in 16-byte pieces, 1 KB contiguous per head
+    for (int i = threadIdx.x; i < (h1 - h0) * 64; i += AT_THREADS) {
+      const int hr = i >> 6, ch = i & 63;
+      const uint4 v = *reinterpret_cast<const uint4*>(ot + hr * OT_PITCH + ch * 16);
+      *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(a.out) + ((size_t)row * AT_H + hg0 + hr) * 1024 + ch * 16) = v;
+    }
   }
 }
 
@@ -603,7 +635,6 @@ cudaError_t launch_attention_tc(AttnArgs a, cudaStream_t st, bool* used, bool* c
   if (a.H != AT_H || a.dk != 576 || a.dv != 512) return cudaSuccess;
   if ((uintptr_t)a.q & 15 || (uintptr_t)a.cache & 15 || (a.win && ((uintptr_t)a.win & 15))) return cudaSuccess;
   if ((int64_t)a.B * a.n_max > 0x7fffffffLL || (int64_t)a.B * a.Tq * AT_H > 0x7fffffffLL) return cudaSuccess;
-  if (a.rows_per_split % AT_ROWS != 0 && a.splits > 1) return cudaSuccess;
   AtMaps maps;
   const uint64_t win_rows = a.prefill ? (uint64_t)a.B * a.t_raw : (uint64_t)a.B * a.W;
   if (!make_latent_map(&maps.q, a.q, (uint64_t)a.B * a.Tq * AT_H)) return cudaSuccess;
