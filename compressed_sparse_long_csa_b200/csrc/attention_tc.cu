@@ -43,7 +43,8 @@ constexpr int AT_H = 128;                // heads per query
 constexpr int AT_HC = 64;                // heads per CTA (MMA M)
 constexpr int AT_ATOMS = 9;              // 576 dims = 9 atoms of 64 dims (128 bytes)
 constexpr int AT_CHUNKS = AT_ATOMS * 8;  // 16-byte chunks per row
-constexpr int AT_GROUP = 128;            // threads per loader group; group g fills stage g
+constexpr int AT_GROUP = 96;             // threads per loader group; group g fills stage g (15 warps in
+                                         // all: 128 registers per thread, where 17 warps get 96)
 constexpr int AT_SMW = 8;                // softmax warps: two warpgroups, one per half of the tile's columns
 constexpr int AT_MMAW = AT_SMW;          // the MMA warp
 constexpr int AT_LDW = AT_SMW + 1;       // first loader warp
@@ -58,7 +59,7 @@ struct AtSmem {
   alignas(1024) uint8_t p[AT_HC * 128];                    // P: 64 heads x 64 rows bf16
   const __nv_bfloat16* rowp[2][AT_ROWS];
   unsigned long long run_key[2][2];   // per stage and loader warp: (tensor << 32 | first row) or NO_RUN
-  uint8_t valid[2][AT_ROWS];
+  uint32_t vmask[2][2];  // per stage: bit j of word j / 32 set when row j of the tile is valid
   alignas(8) uint64_t full[2];
   uint64_t empty[2];
   uint64_t sfull[2];
@@ -154,7 +155,7 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
   }
 
   if (warp >= AT_LDW) {
-    // ------------------------------------------------------------------ loader group g (64 threads)
+    // ------------------------------------------------------------------ loader group g (96 threads)
     // Group g loads tiles g, g+2, ... into stage g; the two groups never wait on each other.
     const int g = (warp - AT_LDW) / (AT_GROUP / 32);
     const int lg = threadIdx.x - AT_LDW * 32 - g * AT_GROUP;
@@ -183,7 +184,8 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
       if (lg < AT_ROWS) {
         const __nv_bfloat16* base = which == 1 ? (const __nv_bfloat16*)a.win : (const __nv_bfloat16*)a.cache;
         sm.rowp[g][lg] = which >= 0 ? base + (size_t)y * 576 : nullptr;
-        sm.valid[g][lg] = which >= 0;
+        const uint32_t vb = __ballot_sync(0xffffffffu, which >= 0);
+        if ((lg & 31) == 0) sm.vmask[g][lg >> 5] = vb;
         // the tile is one contiguous run when all 64 rows are valid rows of one tensor
         // with y - lg the same everywhere; each warp checks its 32 rows
         const unsigned long long key =
@@ -234,66 +236,94 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
     }
   } else if (warp == AT_MMAW) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t ID_S = tc::idesc(tc::FMT_BF16, tc::FMT_BF16, AT_HC, AT_ROWS);
-      constexpr uint32_t ID_O = tc::idesc(tc::FMT_BF16, tc::FMT_BF16, AT_HC, 256, 0, 1);
-      bool ok = n_t == 0 || tc::mbar_wait(&sm.qfull, 0);
-      // Event-driven issue: S(ns) once its tile has landed and its S buffer is free, PV(np)
-      // once P(np) is ready, in order; a PV never waits behind the next tile's load.
-      int ns = 0, np = 0;
-      uint64_t t_idle = tc::now_ns();
-      uint32_t spins = 0;
-      while (ok && np < n_t) {
-        bool prog = false;
-        if (ns < n_t) {
-          const int st = ns & 1;
-          const uint32_t ph = (ns >> 1) & 1;
-          if (tc::mbar_try_wait(&sm.full[st], ph) && tc::mbar_try_wait(&sm.sfree[st], ph ^ 1)) {
-            tc::fence_after_sync();
-            const uint32_t d = tmem + TM_S_LANE + st * AT_ROWS;
-            for (int at = 0; at < AT_ATOMS; ++at) {
-              const uint32_t qa = tc::smem_u32(sm.q[at]), ka = tc::smem_u32(sm.kv[st][at]);
+    // The whole warp runs the loop (descriptors stay warp-uniform); lane 0 decides, one
+    // elected lane (always the same) issues every MMA and commit.
+    constexpr uint32_t ID_S = tc::idesc(tc::FMT_BF16, tc::FMT_BF16, AT_HC, AT_ROWS);
+    constexpr uint32_t ID_O = tc::idesc(tc::FMT_BF16, tc::FMT_BF16, AT_HC, 256, 0, 1);
+    bool ok = n_t == 0 || tc::mbar_wait(&sm.qfull, 0);
+    ok = __all_sync(0xffffffffu, ok);
+    // Descriptors are formed once; an MMA's operands are these plus compile-time offsets
+    // (the 14-bit address field of a descriptor cannot carry: shared memory < 256 KB).
+    const uint64_t q_d0 = tc::desc_k_sw128(tc::smem_u32(sm.q[0]));
+    const uint64_t k_d0 = tc::desc_k_sw128(tc::smem_u32(sm.kv[0][0])), k_d1 = tc::desc_k_sw128(tc::smem_u32(sm.kv[1][0]));
+    const uint64_t p_d0 = tc::desc_k_sw128(tc::smem_u32(sm.p));
+    const uint64_t v_d0 = tc::desc_mn_sw128(tc::smem_u32(sm.kv[0][0]), ATOM, 1024),
+                   v_d1 = tc::desc_mn_sw128(tc::smem_u32(sm.kv[1][0]), ATOM, 1024);
+    // Event-driven issue: S(ns) once its tile has landed and its S buffer is free, PV(np)
+    // once P(np) is ready, in order; a PV never waits behind the next tile's load.
+    int ns = 0, np = 0;
+    uint64_t t_idle = tc::now_ns();
+    uint32_t spins = 0;
+    while (ok && np < n_t) {
+      bool prog = false;
+      if (ns < n_t) {
+        const int st = ns & 1;
+        const uint32_t ph = (ns >> 1) & 1;
+        bool ready = false;
+        if (lane == 0) ready = tc::mbar_try_wait(&sm.full[st], ph) && tc::mbar_try_wait(&sm.sfree[st], ph ^ 1);
+        if (__shfl_sync(0xffffffffu, (int)ready, 0)) {
+          tc::fence_after_sync();
+          const uint32_t d = tmem + TM_S_LANE + st * AT_ROWS;
+          const uint64_t kd = st ? k_d1 : k_d0;
+          // S = Q K^T over 9 atoms x 4 k-steps of 16 (atoms of Q and of the tile are 8 KB apart)
+          if (tc::elect_one()) tc::mma_f16_c<false>(d, q_d0, kd, ID_S);
 #pragma unroll
-              for (int ks = 0; ks < 4; ++ks)
-                tc::mma_f16(d, tc::desc_k_sw128(qa + ks * 32), tc::desc_k_sw128(ka + ks * 32), ID_S,
-                            (at > 0 || ks > 0) ? 1u : 0u);
-            }
-            tc::mma_commit(&sm.sfull[st]);
-            ++ns;
-            prog = true;
+          for (int i = 1; i < AT_ATOMS * 4; ++i) {
+            const uint64_t off = (uint64_t)(((i >> 2) * ATOM + (i & 3) * 32) >> 4);
+            if (tc::elect_one()) tc::mma_f16_c<true>(d, q_d0 + off, kd + off, ID_S);
           }
+          if (tc::elect_one()) tc::mma_commit(&sm.sfull[st]);
+          __syncwarp();
+          ++ns;
+          prog = true;
         }
-        if (np < ns && tc::mbar_try_wait(&sm.pfull, np & 1)) {
+      }
+      if (np < ns) {
+        bool ready = false;
+        if (lane == 0) ready = tc::mbar_try_wait(&sm.pfull, np & 1);
+        if (__shfl_sync(0xffffffffu, (int)ready, 0)) {
           // O += P_np V_np: value dims 0-255 (atoms 0-3) and 256-511 (atoms 4-7)
           const int st = np & 1;
           tc::fence_after_sync();
-          const uint32_t pa = tc::smem_u32(sm.p);
+          const uint64_t vd = st ? v_d1 : v_d0;
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
-            const uint32_t va = tc::smem_u32(sm.kv[st][4 * half]);
+            const uint64_t vh = vd + (uint64_t)((4 * half * ATOM) >> 4);
+            if (tc::elect_one()) {
+              if (np > 0) tc::mma_f16_c<true>(tmem + 256 * half, p_d0, vh, ID_O);
+              else tc::mma_f16_c<false>(tmem + 256 * half, p_d0, vh, ID_O);
+            }
 #pragma unroll
-            for (int ks = 0; ks < AT_ROWS / 16; ++ks)
-              tc::mma_f16(tmem + 256 * half, tc::desc_k_sw128(pa + ks * 32),
-                          tc::desc_mn_sw128(va + ks * 16 * 128, ATOM, 1024), ID_O, (np > 0 || ks > 0) ? 1u : 0u);
+            for (int ks = 1; ks < AT_ROWS / 16; ++ks)
+              if (tc::elect_one())
+                tc::mma_f16_c<true>(tmem + 256 * half, p_d0 + (uint64_t)((ks * 32) >> 4), vh + (uint64_t)((ks * 16 * 128) >> 4), ID_O);
           }
-          tc::mma_commit(&sm.empty[st]);
-          tc::mma_commit(&sm.pdone);
+          if (tc::elect_one()) {
+            tc::mma_commit(&sm.empty[st]);
+            tc::mma_commit(&sm.pdone);
+          }
+          __syncwarp();
           ++np;
           prog = true;
         }
-        if (prog) {
-          spins = 0;
-        } else if ((++spins & 63u) == 0u) {
+      }
+      if (prog) {
+        spins = 0;
+      } else if ((++spins & 63u) == 0u) {
+        bool stop = false;
+        if (lane == 0) {
           const uint64_t t = tc::now_ns();
           if (spins == 64u) t_idle = t;
-          if (*(volatile int*)&sm.abort_flag || t - t_idle > tc::WAIT_LIMIT_NS) ok = false;
+          stop = *(volatile int*)&sm.abort_flag || t - t_idle > tc::WAIT_LIMIT_NS;
         }
+        if (__shfl_sync(0xffffffffu, (int)stop, 0)) ok = false;
       }
-      if (!ok) atomicExch(&sm.abort_flag, 1);
-      // every MMA this thread issued has completed before the CTA frees TMEM
-      tc::mma_commit(&sm.drain);
-      tc::mbar_wait(&sm.drain, 0);
     }
+    if (!ok && lane == 0) atomicExch(&sm.abort_flag, 1);
+    // every MMA the elected lane issued has completed before the CTA frees TMEM
+    if (tc::elect_one()) tc::mma_commit(&sm.drain);
+    __syncwarp();
+    tc::mbar_wait(&sm.drain, 0);
   } else {
     // ------------------------------------------------------------------ softmax + epilogue, warps 0-7
     // TMEM quarter q = warp % 4: lanes 16-31 hold the logits of heads 16q .. 16q+15 (S), lanes
@@ -323,13 +353,20 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
 #pragma unroll
         for (int j = 0; j < AT_ROWS; ++j) s[j] = __uint_as_float(v[j]);
       }
-      float mt = -INFINITY;
+      // scaled logits, invalid rows at -inf (a full tile skips the mask), and their max
+      // over four independent chains
+      const uint32_t vm0 = sm.vmask[st][0], vm1 = sm.vmask[st][1];
 #pragma unroll
-      for (int j = 0; j < AT_ROWS; ++j) {
-        const float l = sm.valid[st][j] ? s[j] * scale : -INFINITY;
-        s[j] = l;
-        mt = fmaxf(mt, l);
+      for (int j = 0; j < AT_ROWS; ++j) s[j] *= scale;
+      if ((vm0 & vm1) != 0xffffffffu) {
+#pragma unroll
+        for (int j = 0; j < AT_ROWS; ++j)
+          if (!((j < 32 ? vm0 >> j : vm1 >> (j - 32)) & 1u)) s[j] = -INFINITY;
       }
+      float mq[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+      for (int j = 4; j < AT_ROWS; ++j) mq[j & 3] = fmaxf(mq[j & 3], s[j]);
+      const float mt = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
       // online softmax with a lazily raised running max (S lanes decide; O lanes follow)
       bool need_rescale = false;
       float alpha = 1.f;

@@ -156,10 +156,10 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         if (!tc::mbar_wait(&sm.full[st], ph)) { ok = false; break; }
         if (*(volatile int*)&sm.abort_flag) { ok = false; break; }
         tc::fence_after_sync();
-        const uint32_t k_addr = tc::smem_u32(sm.k[st]);
+        const uint64_t kd = tc::desc_k_sw128(tc::smem_u32(sm.k[st])), qd = tc::desc_k_sw128(q_addr);
 #pragma unroll
         for (int ks = 0; ks < IT_KB / 32; ++ks)
-          tc::mma_f8f6f4(tmem + acc * N, tc::desc_k_sw128(k_addr + ks * 32), tc::desc_k_sw128(q_addr + ks * 32), ID,
+          tc::mma_f8f6f4(tmem + acc * N, kd + (uint64_t)((ks * 32) >> 4), qd + (uint64_t)((ks * 32) >> 4), ID,
                          ks > 0 ? 1u : 0u);
         tc::mma_commit(&sm.empty[st]);
         tc::mma_commit(&sm.tfull[acc]);
