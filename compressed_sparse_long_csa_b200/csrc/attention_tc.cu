@@ -49,7 +49,7 @@ constexpr int AT_SMW = 8;                // softmax warps: two warpgroups, one p
 constexpr int AT_MMAW = AT_SMW;          // the MMA warp
 constexpr int AT_LDW = AT_SMW + 1;       // first loader warp
 constexpr int AT_THREADS = (AT_SMW + 1) * 32 + 2 * AT_GROUP;
-constexpr float AT_RESCALE_THRESH = 8.0f;
+constexpr float AT_RESCALE_THRESH = 8.0f;  // base-2 units: O is rescaled once the max grows 256-fold
 constexpr int ATOM = AT_ROWS * 128;      // one 64-row x 128-byte swizzle atom
 constexpr unsigned long long NO_RUN = ~0ull;
 
@@ -99,6 +99,14 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
         "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
+}
+
+// 2^x by the MUFU.EX2 unit (ex2.approx; relative error about 2^-22, far below the bf16
+// rounding of P)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // byte offset of 16-byte chunk c of row j in a 128-byte-swizzled atom
@@ -336,7 +344,9 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
     const int hl = quarter * 16 + (lane & 15);      // head within the CTA
     const int h = hh * AT_HC + hl;                  // head within the query
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    const float scale = a.sm_scale;
+    // logits are kept in the base-2 domain (scale x log2 e): P = 2^(s - m); the running max
+    // and the partial's m leave it (x ln 2) at the end
+    const float scale2 = a.sm_scale * 1.4426950408889634f;
     float m_run = -INFINITY, l_run = 0.f;           // S lanes: running max, this warpgroup's row sum
     bool ok = true;
     for (int it = 0; it < n_t; ++it) {
@@ -357,7 +367,7 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
       // over four independent chains
       const uint32_t vm0 = sm.vmask[st][0], vm1 = sm.vmask[st][1];
 #pragma unroll
-      for (int j = 0; j < AT_ROWS; ++j) s[j] *= scale;
+      for (int j = 0; j < AT_ROWS; ++j) s[j] *= scale2;
       if ((vm0 & vm1) != 0xffffffffu) {
 #pragma unroll
         for (int j = 0; j < AT_ROWS; ++j)
@@ -372,7 +382,7 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
       float alpha = 1.f;
       if (is_s && (mt > m_run + AT_RESCALE_THRESH || (m_run == -INFINITY && mt != -INFINITY))) {
         const float m_new = fmaxf(mt, m_run);
-        alpha = (m_run == -INFINITY) ? 0.f : __expf(m_run - m_new);
+        alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_new);
         need_rescale = (m_run != -INFINITY);
         m_run = m_new;
       }
@@ -390,7 +400,20 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
         const float moved = __shfl_down_sync(0xffffffffu, a1, 16);
         pv[q] = is_s ? a0 : moved;
       }
-      // P and O are owned by the previous PV until it completes
+      // P in registers first (bf16, the normaliser sums the rounded values); it overlaps the
+      // previous PV, which owns the shared P tile and O until it completes
+      uint32_t w8[8];
+      float psum = 0.f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float p0 = (m_use == -INFINITY) ? 0.f : ex2_approx(pv[2 * u] - m_use);
+        const float p1 = (m_use == -INFINITY) ? 0.f : ex2_approx(pv[2 * u + 1] - m_use);
+        __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
+        psum += __low2float(hb) + __high2float(hb);
+        w8[u] = *reinterpret_cast<uint32_t*>(&hb);
+      }
+      const float po = __shfl_up_sync(0xffffffffu, psum, 16);   // the O lane's part, to its S lane
+      if (is_s) l_run = l_run * alpha + psum + po;
       if (it >= 1) {
         if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.pdone, (it - 1) & 1))) { ok = false; break; }
         tc::fence_after_sync();
@@ -417,25 +440,12 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
         tc::tmem_st_wait();
       }
       {
-        float psum = 0.f;
         const uint32_t pbase = tc::smem_u32(sm.p);
         const int c0 = 4 * wg + (is_s ? 0 : 2);     // 16-byte chunks (8 columns) of the P row
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          uint32_t w4[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float p0 = (m_use == -INFINITY) ? 0.f : __expf(pv[cc * 8 + 2 * u] - m_use);
-            const float p1 = (m_use == -INFINITY) ? 0.f : __expf(pv[cc * 8 + 2 * u + 1] - m_use);
-            __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
-            psum += __low2float(hb) + __high2float(hb);     // the normaliser uses the rounded P
-            w4[u] = *reinterpret_cast<uint32_t*>(&hb);
-          }
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pbase + sw128_off(hl, c0 + cc)), "r"(w4[0]),
-                       "r"(w4[1]), "r"(w4[2]), "r"(w4[3]) : "memory");
-        }
-        const float po = __shfl_up_sync(0xffffffffu, psum, 16);   // the O lane's part, to its S lane
-        if (is_s) l_run = l_run * alpha + psum + po;
+        for (int cc = 0; cc < 2; ++cc)
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pbase + sw128_off(hl, c0 + cc)), "r"(w8[4 * cc]),
+                       "r"(w8[4 * cc + 1]), "r"(w8[4 * cc + 2]), "r"(w8[4 * cc + 3]) : "memory");
       }
       // release this tile's S buffer and hand P (and a rescaled O) to the MMA thread
       tc::fence_proxy_async_smem();
@@ -455,7 +465,7 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
     if (is_s) sm.lx[wg][hl] = l_run;
     named_bar(3, AT_SMW * 32);
     const float l_tot = sm.lx[0][hl] + sm.lx[1][hl];
-    const float m_h = __shfl_sync(0xffffffffu, m_run, (lane & 15) + 16);
+    const float m_h = __shfl_sync(0xffffffffu, m_run, (lane & 15) + 16) * 0.6931471805599453f;
     const float l_h = __shfl_sync(0xffffffffu, l_tot, (lane & 15) + 16);
     if (a.splits == 1) {
       const float sk = sink_pre;
