@@ -266,13 +266,14 @@ struct MxSmem {
   float w[64];
 };
 
-// TMEM columns: four accumulators [0, 256), q scales at 256, key-scale ring at 264 + 4 * stage
-constexpr uint32_t MX_SFB = 256, MX_SFA = 264, MX_COLS = 512;
-constexpr int MX_NACC = 4;
+// TMEM columns (256: two CTAs share an SM): two accumulators [0, 128), q scales at 128,
+// key-scale ring at 136 + 4 * stage
+constexpr uint32_t MX_SFB = 128, MX_SFA = 136, MX_COLS = 256;
+constexpr int MX_NACC = 2;
 constexpr int MX_THREADS = 512;   // warp 0 TMA, 1 MMA, 4..11 epilogue (two warpgroups), 12..15 scale writers
 
 template <int STAGES>
-__global__ void __launch_bounds__(MX_THREADS, 1)
+__global__ void __launch_bounds__(MX_THREADS, 2)
 indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ, IdxTcParams p) {
   extern __shared__ uint8_t smem_raw[];
   using Sm = MxSmem<STAGES>;
@@ -512,7 +513,7 @@ cudaError_t launch_mxf4(const IndexerArgs& a, cudaStream_t st, bool* used) {
   p.n_qg = a.Tq;
   p.tiles = (int)((a.n_max + IT_ROWS - 1) / IT_ROWS);
   const int64_t ctas = (int64_t)a.B * a.Tq;
-  int splits = (int)(148 / ctas);                   // one wave: one CTA per SM
+  int splits = (int)(2 * 148 / ctas);               // one wave: two CTAs per SM
   if (splits > p.tiles) splits = p.tiles;
   if (splits < 1) splits = 1;
   p.tiles_per_split = (p.tiles + splits - 1) / splits;
