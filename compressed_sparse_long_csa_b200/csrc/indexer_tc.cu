@@ -55,7 +55,7 @@ struct IdxSmem {
   int issued0;          // tile loads issued before the setup barrier
   int n_elig[G];
   int row[G];
-  float wq[G][64];
+  alignas(16) float wq[G][64];
 };
 
 template <int G, int STAGES>
@@ -204,10 +204,20 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
           const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + acc * N + g * 64 + hlf * 32;
           tc::tmem_ld16(ta, v);
           tc::tmem_ld16(ta + 16, v + 16);
+          // the 32 weights as eight 16-byte loads, in flight with the TMEM loads (one load
+          // per weight exposed its latency 64 times per tile)
+          const float4* w4p = reinterpret_cast<const float4*>(&sm.wq[g][hlf * 32]);
+          float4 w4[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) w4[u] = w4p[u];
           tc::tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            part[j & 3] = fmaf(sm.wq[g][hlf * 32 + j], fmaxf(__uint_as_float(v[j]), 0.f), part[j & 3]);
+          for (int u = 0; u < 8; ++u) {
+            part[0] = fmaf(w4[u].x, fmaxf(__uint_as_float(v[4 * u]), 0.f), part[0]);
+            part[1] = fmaf(w4[u].y, fmaxf(__uint_as_float(v[4 * u + 1]), 0.f), part[1]);
+            part[2] = fmaf(w4[u].z, fmaxf(__uint_as_float(v[4 * u + 2]), 0.f), part[2]);
+            part[3] = fmaf(w4[u].w, fmaxf(__uint_as_float(v[4 * u + 3]), 0.f), part[3]);
+          }
         }
         const float val = (part[0] + part[1]) + (part[2] + part[3]);
         const bool valid = s < sm.n_elig[g];
@@ -263,7 +273,7 @@ struct MxSmem {
   int t_begin, t_end;
   int issued0;          // tile loads issued before the setup barrier
   int n_elig;
-  float w[64];
+  alignas(16) float w[64];
 };
 
 // TMEM columns (256: two CTAs share an SM): two accumulators [0, 128), q scales at 128,
@@ -434,15 +444,24 @@ indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       if (!ok) { atomicExch(&sm.abort_flag, 1); break; }
       tc::fence_after_sync();
       float part[4] = {0.f, 0.f, 0.f, 0.f};
+      // 16 heads at a time: their accumulator columns and weights (four 16-byte loads) in
+      // flight together (the kernel runs at 64 registers)
 #pragma unroll
-      for (int hlf = 0; hlf < 2; ++hlf) {
-        uint32_t v[32];
-        const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + acc * N + hlf * 32;
-        tc::tmem_ld16(ta, v);
-        tc::tmem_ld16(ta + 16, v + 16);
+      for (int q16 = 0; q16 < 4; ++q16) {
+        uint32_t v[16];
+        tc::tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + acc * N + q16 * 16, v);
+        const float4* w4p = reinterpret_cast<const float4*>(&sm.w[q16 * 16]);
+        float4 w4[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) w4[u] = w4p[u];
         tc::tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) part[j & 3] = fmaf(sm.w[hlf * 32 + j], fmaxf(__uint_as_float(v[j]), 0.f), part[j & 3]);
+        for (int u = 0; u < 4; ++u) {
+          part[0] = fmaf(w4[u].x, fmaxf(__uint_as_float(v[4 * u]), 0.f), part[0]);
+          part[1] = fmaf(w4[u].y, fmaxf(__uint_as_float(v[4 * u + 1]), 0.f), part[1]);
+          part[2] = fmaf(w4[u].z, fmaxf(__uint_as_float(v[4 * u + 2]), 0.f), part[2]);
+          part[3] = fmaf(w4[u].w, fmaxf(__uint_as_float(v[4 * u + 3]), 0.f), part[3]);
+        }
       }
       const float val = (part[0] + part[1]) + (part[2] + part[3]);
       if (valid) {
