@@ -208,6 +208,85 @@ attn_combine_kernel(AttnArgs a) {
     a.lse[(size_t)row * a.H + h] = stat[1] > 0.f ? stat[0] + logf(stat[1]) : -INFINITY;
 }
 
+// The tensor-core kernel's partials (format 1: fp16 values, 128 heads, d_v = 512) into bf16
+// outputs.  grid (B*Tq, 64): two heads per CTA, one 8-value piece per thread.  Every
+// split's piece is loaded before the weights are known (16 splits at a time).
+constexpr int C16_CHUNK = 16;
+__global__ void __launch_bounds__(128)
+attn_combine16_kernel(AttnArgs a) {
+  __shared__ float wsh[2][2][64];      // [head][half][split]
+  const int row = blockIdx.x, hp = threadIdx.x >> 6, c8 = threadIdx.x & 63;
+  const int h = blockIdx.y * 2 + hp;
+  const int S = a.splits;
+  const size_t sstride = attn_part_block(128, 512);
+  const float sk = a.sink[h];
+  const float* B0 = a.part + (size_t)row * S * sstride;
+  const uint4* v0 = reinterpret_cast<const uint4*>(B0) + (size_t)c8 * 128 + h;   // split s: + s * sstride / 4
+  uint4 x[C16_CHUNK];
+#pragma unroll
+  for (int u = 0; u < C16_CHUNK; ++u)
+    x[u] = u < S ? __ldcg(v0 + (size_t)u * (sstride / 4)) : make_uint4(0u, 0u, 0u, 0u);
+  // weights: the first warp of each head's pair of warps
+  if ((threadIdx.x & 63) < 32) {
+    const int lane = threadIdx.x & 31;
+    float4 rc[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int s2 = lane + 32 * q;
+      rc[q] = s2 < S ? __ldcg(reinterpret_cast<const float4*>(B0 + s2 * sstride + attn_part16_rec(128, 512, h)))
+                     : make_float4(-INFINITY, 0.f, 0.f, 0.f);
+    }
+    float M = fmaxf(sk, fmaxf(rc[0].x, rc[1].x));
+    M = warp_max(M);
+    float den = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int q = 0; q < 2; ++q)
+        if (rc[q].x != -INFINITY) den += rc[q].y * __expf(rc[q].x - M);
+      den = warp_sum(den) + __expf(sk - M);
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int s2 = lane + 32 * q;
+      const float w = (rc[q].x == -INFINITY || M == -INFINITY) ? 0.f : __expf(rc[q].x - M) * inv * rc[q].y;
+      wsh[hp][0][s2] = w * rc[q].z;
+      wsh[hp][1][s2] = w * rc[q].w;
+    }
+    if (a.lse && lane == 0) a.lse[(size_t)row * 128 + h] = den > 0.f ? M + logf(den) : -INFINITY;
+  }
+  __syncthreads();
+  const float* wr = wsh[hp][c8 >= 32 ? 1 : 0];
+  float acc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+  for (int s0 = 0; s0 < S; s0 += C16_CHUNK) {
+    if (s0 > 0) {
+#pragma unroll
+      for (int u = 0; u < C16_CHUNK; ++u)
+        x[u] = s0 + u < S ? __ldcg(v0 + (size_t)(s0 + u) * (sstride / 4)) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < C16_CHUNK; ++u) {
+      const float wgt = s0 + u < S ? wr[s0 + u] : 0.f;
+      const uint32_t q4[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&q4[q]));
+        acc[2 * q] = fmaf(wgt, f2.x, acc[2 * q]);
+        acc[2 * q + 1] = fmaf(wgt, f2.y, acc[2 * q + 1]);
+      }
+    }
+  }
+  uint32_t pk[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
+    pk[q] = *reinterpret_cast<uint32_t*>(&b2);
+  }
+  *reinterpret_cast<uint4*>((__nv_bfloat16*)a.out + ((size_t)row * 128 + h) * 512 + c8 * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+}
+
 int attn_choose_splits(int n_queries, int H, int64_t rows, bool tc_path) {
   int64_t s;
   const int64_t tiles = (rows + 63) / 64;
@@ -253,6 +332,13 @@ cudaError_t launch_attention_cuda_core(AttnArgs a, int dtype, cudaStream_t st) {
 }
 
 cudaError_t launch_attn_combine(const AttnArgs& a, int dtype, cudaStream_t st) {
+  if (a.part_fp16 && dtype == CSA_BF16 && a.H == 128 && a.dv == 512 && a.splits <= 64) {
+    // a plain launch: launched early, its CTAs would wait on the few SMs the attention
+    // grid leaves free and then run there
+    note_launch();
+    attn_combine16_kernel<<<dim3(a.B * a.Tq, 64), 128, 0, st>>>(a);
+    return cudaGetLastError();
+  }
   dim3 grid(a.B * a.Tq, a.H);
   note_launch();
   if (dtype == CSA_BF16) {
