@@ -79,7 +79,7 @@ struct SelFixed {
   float U;
 };
 
-// Re-scoring scratch: overlays the score array once the scores have been classified.
+// Re-scoring scratch (see sl_resc_sep for where it lives).
 struct Resc {
   double qd[64 * SL_QLD];              // query row codes as fp64 (rows padded: conflict-free fragment reads)
   double kd[SL_RR][SL_QLD];            // key rows being re-scored (one round)
@@ -88,6 +88,10 @@ struct Resc {
 };
 
 constexpr size_t SL_FIXED = (sizeof(SelFixed) + 127) & ~size_t(127);
+// The re-scoring scratch gets its own region after the scores when both fit (the query
+// row is then staged while the scores land), else it overlays them.
+__host__ __device__ constexpr size_t sl_score_bytes(int chunk) { return ((size_t)chunk * 4 + 127) & ~size_t(127); }
+__host__ __device__ constexpr bool sl_resc_sep(int chunk) { return SL_FIXED + sl_score_bytes(chunk) + sizeof(Resc) <= 232448; }
 
 
 __device__ __forceinline__ void sl_sync(cg::cluster_group cl, unsigned C) {
@@ -542,7 +546,8 @@ indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   SelFixed& sh = *reinterpret_cast<SelFixed*>(smem_raw);
   float* sv = reinterpret_cast<float*>(smem_raw + SL_FIXED);
-  Resc& rs = *reinterpret_cast<Resc*>(smem_raw + SL_FIXED);      // overlays sv after classification
+  const bool resc_sep = sl_resc_sep(chunk);
+  Resc& rs = *reinterpret_cast<Resc*>(smem_raw + SL_FIXED + (resc_sep ? sl_score_bytes(chunk) : 0));
   cg::cluster_group cluster = cg::this_cluster();
   const unsigned C = cluster.num_blocks(), r = cluster.block_rank();
   const int row = blockIdx.x / C;
@@ -667,6 +672,7 @@ indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
     }
   }
   if (n > k && tid < m - m4) sv[m4 + tid] = srow[m4 + tid];
+  if (resc_sep) sl_stage_query(rs, qx, total, lgd, HI, dI);   // covered by the barrier below
   // the scores have landed (bounded wait; on a timeout the error word is set)
   if (n > k && m4 > 0) {
     const bool ok = tc::mbar_wait(&sh.ldbar, 0);
@@ -678,7 +684,7 @@ indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
     if (r == 0)
       for (int i = tid; i < k; i += SL_T) out[i] = i < n ? i : -1;
     if (sout) {
-      sl_stage_query(rs, qx, total, lgd, HI, dI);
+      if (!resc_sep) sl_stage_query(rs, qx, total, lgd, HI, dI);
       const int s0 = (int)((int64_t)k * r / C), s1 = (int)((int64_t)k * (r + 1) / C);
       for (int c0 = s0; c0 < s1; c0 += SL_CAP) {
         const int cnt = min(SL_CAP, s1 - c0);
@@ -721,7 +727,7 @@ indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
   const uint32_t nb_raw = sh.cnt;
   const int n_band = (int)min(nb_raw, (uint32_t)SL_CAP);
   if (nb_raw > (uint32_t)SL_CAP && tid == 0) raise_err(a.err, CSA_DEVERR_BAND);
-  sl_stage_query(rs, qx, total, lgd, HI, dI);
+  if (!resc_sep) sl_stage_query(rs, qx, total, lgd, HI, dI);
   // ---- exact scores of this CTA's band entries (the first round's barrier covers the staging)
   sl_rescore_list<F>(rk, sh, rs, b, sh.band_id, n_band, sh.band_s);
   if (tid == 0) { sh.pub[0] = sh.n_sure; sh.pub[1] = (uint32_t)n_band; }
@@ -862,7 +868,7 @@ cudaError_t launch_indexer_select_cluster(const IndexerArgs& a, cudaStream_t st)
   if (a.H_I > 64 || a.d_I > 128 || a.H_I * a.d_I > SL_QPT * SL_T || !sl_plan(a.n_max, rows, &C, &chunk) || (a.ld % 4) != 0 ||
       ((uintptr_t)a.scores & 15) != 0 || (int64_t)rows * C > 0x7fffffffLL)
     return cudaErrorNotSupported;
-  const size_t region = std::max((size_t)chunk * 4, sizeof(Resc));
+  const size_t region = sl_resc_sep(chunk) ? sl_score_bytes(chunk) + sizeof(Resc) : std::max((size_t)chunk * 4, sizeof(Resc));
   if (a.ifmt == CSA_IFMT_E4M3) return sl_launch(indexer_select_cluster_kernel<CSA_IFMT_E4M3>, rows, C, SL_FIXED + region, st, a, chunk);
   if (a.ifmt == CSA_IFMT_MXFP4) return sl_launch(indexer_select_cluster_kernel<CSA_IFMT_MXFP4>, rows, C, SL_FIXED + region, st, a, chunk);
   return sl_launch(indexer_select_cluster_kernel<CSA_IFMT_F32>, rows, C, SL_FIXED + region, st, a, chunk);
