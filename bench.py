@@ -384,37 +384,85 @@ def run_ours(args, wid):
 
 
 def measure_e2e(args, wid, wl, T, D, csa, steps):
-    """Same step through the public API, inputs copied from pinned host memory and
-    the result read back, all inside the timed region."""
+    """Same step through the public API, every step's inputs copied from pinned host
+    memory and its results read back inside the timed region.  Two buffer sets: the
+    copies of step i+1's inputs and of step i-1's results run on their own streams while
+    step i computes (what a serving loop does); the region ends when the last result is
+    on the host.  The packed buffers hold exactly the tensors the step reads as input
+    and writes as result; every other tensor (caches, workspaces) stays resident."""
     import torch
     per_step_in = {1: ["Ca", "Cb", "Za", "Zb", "q", "qI", "qI_scale", "w", "win"],
                    2: ["C", "Z", "q", "win"], 3: ["Ca", "Cb", "Za", "Zb", "q", "qI", "qI_scale", "w"],
                    4: ["Ca", "Cb", "Za", "Zb", "q", "qI", "qI_scale", "w", "win", "h_C", "h_Z", "h_q", "h_win"]}[wid]
-    host = {k: T[k].cpu().pin_memory() for k in per_step_in}
     outs = ["out", "idx"] if wid != 2 else ["out"]
     if wid == 4:
         outs.append("h_out")
-    hout = {k: torch.empty_like(T[k], device="cpu").pin_memory() for k in outs}
-    h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = sum(v.numel() * v.element_size() for v in hout.values())
-    n = max(5, min(args.steps, 20))
-    for _ in range(2):
-        for k, v in host.items():
-            T[k].copy_(v, non_blocking=True)
-        steps.run_step(wl.kind, T, D)
-        for k, v in hout.items():
-            v.copy_(T[k], non_blocking=True)
+    # the step's inputs (and its results) are packed into one buffer each, so that a
+    # step moves one host-to-device and one device-to-host copy
+    def layout(names):
+        off, lay = 0, {}
+        for k in names:
+            nb = T[k].numel() * T[k].element_size()
+            lay[k] = (off, nb)
+            off += (nb + 255) // 256 * 256
+        return lay, off
+
+    def views(buf, lay):
+        return {k: buf[o:o + nb].view(T[k].dtype).view(T[k].shape) for k, (o, nb) in lay.items()}
+
+    lay_in, n_in = layout(per_step_in)
+    lay_out, n_out = layout(outs)
+    host_in = torch.empty(n_in, dtype=torch.uint8).pin_memory()
+    for k, v in views(host_in, lay_in).items():
+        v.copy_(T[k].cpu())
+    dev_in = [torch.empty(n_in, dtype=torch.uint8, device="cuda") for _ in range(2)]
+    dev_out = [torch.empty(n_out, dtype=torch.uint8, device="cuda") for _ in range(2)]
+    host_out = [torch.empty(n_out, dtype=torch.uint8).pin_memory() for _ in range(2)]
+    sets = [dict(T), dict(T)]
+    for j in range(2):
+        sets[j].update(views(dev_in[j], lay_in))
+        sets[j].update(views(dev_out[j], lay_out))
+    h2d = sum(nb for _, nb in lay_in.values())
+    d2h = sum(nb for _, nb in lay_out.values())
+    n = max(6, min(args.steps, 20))
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_comp = [torch.cuda.Event(), torch.cuda.Event()]
+    ev_out = [torch.cuda.Event(), torch.cuda.Event()]
+
+    def run(nsteps, e0=None, e1=None):
+        if e0 is not None:
+            e0.record(comp)
+        s_in.wait_stream(comp)
+        s_out.wait_stream(comp)
+        for i in range(nsteps):
+            j = i & 1
+            Tj = sets[j]
+            ev_in = torch.cuda.Event()
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_comp[j])          # step i-2 has read this set's inputs
+                dev_in[j].copy_(host_in, non_blocking=True)
+                ev_in.record(s_in)
+            comp.wait_event(ev_in)
+            if i >= 2:
+                comp.wait_event(ev_out[j])              # step i-2's results have left this set
+            steps.run_step(wl.kind, Tj, D)
+            ev_comp[j].record(comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_comp[j])
+                host_out[j].copy_(dev_out[j], non_blocking=True)
+                ev_out[j].record(s_out)
+        comp.wait_stream(s_out)
+        comp.wait_stream(s_in)
+        if e1 is not None:
+            e1.record(comp)
+
+    run(2)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(n):
-        for k, v in host.items():
-            T[k].copy_(v, non_blocking=True)
-        steps.run_step(wl.kind, T, D)
-        for k, v in hout.items():
-            v.copy_(T[k], non_blocking=True)
-    e1.record()
+    run(n, e0, e1)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / n
     tokens = D["B"] * (D["Tq"] if wid == 3 else 1)
