@@ -131,6 +131,27 @@ def summarize_clocks(lines, local_index=None):
     return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons)}
 
 
+def rank_seed(wid, rank):
+    """Each rank draws its own batch of the workload (independent sequences)."""
+    return wid + 1000 * rank
+
+
+def max_over_ranks(x, world, device):
+    """The slowest rank's value: every timing is taken per rank on its own device."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank, world, ms):
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return units_per_rank * world / (ms * 1e-3)
+
+
 def run_reference(args, wid):
     """Time the fp64 oracle on host cores on a bounded sample of the workload."""
     import numpy as np
@@ -209,7 +230,7 @@ def run_ours(args, wid):
     from compressed_sparse_long_csa_b200 import steps
     import csa_inputs as CI
 
-    wl = CI.make_workload(wid, seed=wid + 1000 * rank)
+    wl = CI.make_workload(wid, seed=rank_seed(wid, rank))
     D = wl.dims
     T = steps.upload(wl)
     stream = torch.cuda.current_stream()
@@ -324,17 +345,16 @@ def run_ours(args, wid):
     torch.cuda.synchronize()
     per = np.array([[ev[i].elapsed_time(ev[i + 1]) for i in range(4)] for ev in ev_list])   # ms
     step_ms = np.array([ev[0].elapsed_time(ev[1]) for ev in step_evs])
-    total_ms = float(step_ms.sum())
-    if world > 1:
-        t = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(float(step_ms.sum()), world, "cuda")
     ms_per_step = total_ms / args.steps
     tokens_per_step = D["B"] * (D["Tq"] if wid == 3 else 1)
-    value = tokens_per_step * world / (ms_per_step * 1e-3)
+    value = job_rate(tokens_per_step, world, ms_per_step)
 
-    # ---- e2e through the public API with host buffers
-    e2e = measure_e2e(args, wid, wl, T, D, csa, steps)
+    # ---- e2e through the public API with host buffers (max over ranks too)
+    e2e_ms, h2d, d2h = measure_e2e(args, wid, wl, T, D, csa, steps)
+    e2e_ms = max_over_ranks(e2e_ms, world, "cuda")
+    e2e = {"value": job_rate(tokens_per_step, world, e2e_ms), "unit": "tokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     ab = algorithmic_bytes(wid, D)
     comp = ["compress", "indexer", "attention", "hca"]
     mean_ms = per.mean(axis=0)
@@ -464,9 +484,7 @@ def measure_e2e(args, wid, wl, T, D, csa, steps):
     e1 = torch.cuda.Event(enable_timing=True)
     run(n, e0, e1)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / n
-    tokens = D["B"] * (D["Tq"] if wid == 3 else 1)
-    return {"value": tokens / (ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    return e0.elapsed_time(e1) / n, h2d, d2h
 
 
 def cpu_baseline(wid, wl):
