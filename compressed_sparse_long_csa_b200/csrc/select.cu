@@ -132,14 +132,16 @@ __device__ __forceinline__ uint32_t sl_peer(cg::cluster_group cl, const uint32_t
 // Concatenate every CTA's list (CTA p's count in its pub[slot]) into dst in rank order;
 // returns the total (at most cap).
 // The offsets are set by sl_gather_offsets (one thread, then a barrier).
+// Peer loads in these helpers are unrolled over SL_CMAX and predicated, so that all of
+// them are in flight at once (a loop over the runtime cluster size issued them one by one).
 __device__ __forceinline__ void sl_gather_offsets(SelFixed& sh, cg::cluster_group cl, unsigned C, int slot) {
-  if (threadIdx.x == 0) {
-    int total = 0;
-    for (int p = 0; p < (int)C; ++p) {
-      sh.goff[p] = total;
-      total += (int)sl_peer(cl, sh.pub, slot, p);
-    }
-    for (int p = (int)C; p <= SL_CMAX; ++p) sh.goff[p] = total;
+  const int t = threadIdx.x;
+  if (t <= SL_CMAX) {
+    int sum = 0;
+#pragma unroll
+    for (int p = 0; p < SL_CMAX; ++p)
+      if (p < t && p < (int)C) sum += (int)sl_peer(cl, sh.pub, slot, p);
+    sh.goff[t] = sum;
   }
 }
 template <typename T>
@@ -173,9 +175,12 @@ __device__ __forceinline__ void sl_key_range(SelFixed& sh, const float* sv, int 
   if (tid == 0) { sh.pub[0] = sh.red[0]; sh.pub[1] = sh.red[1]; }
   sl_sync(cluster, C);
   uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-  for (int p = 0; p < (int)C; ++p) {
-    lo = min(lo, sl_peer(cluster, sh.pub, 0, p));
-    hi = max(hi, sl_peer(cluster, sh.pub, 1, p));
+#pragma unroll
+  for (int p = 0; p < SL_CMAX; ++p) {
+    if (p < (int)C) {
+      lo = min(lo, sl_peer(cluster, sh.pub, 0, p));
+      hi = max(hi, sl_peer(cluster, sh.pub, 1, p));
+    }
   }
   *lo_out = lo;
   *hi_out = hi;
@@ -207,9 +212,13 @@ __device__ __forceinline__ void sl_refine(SelFixed& sh, const float* sv, int m, 
     }
     sl_sync(cluster, C);
     uint4 hb = make_uint4(0u, 0u, 0u, 0u);
-    for (int p = 0; p < (int)C; ++p) {
-      const uint4 x = reinterpret_cast<const uint4*>(cluster.map_shared_rank(H, p))[tid];
-      hb.x += x.x; hb.y += x.y; hb.z += x.z; hb.w += x.w;
+    {
+      uint4 xs[SL_CMAX];
+#pragma unroll
+      for (int p = 0; p < SL_CMAX; ++p)
+        xs[p] = p < (int)C ? reinterpret_cast<const uint4*>(cluster.map_shared_rank(H, p))[tid] : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int p = 0; p < SL_CMAX; ++p) { hb.x += xs[p].x; hb.y += xs[p].y; hb.z += xs[p].z; hb.w += xs[p].w; }
     }
     // suffix counts: bins above 4*tid+3 belong to higher threads
     const uint32_t mine = hb.x + hb.y + hb.z + hb.w;
@@ -365,16 +374,23 @@ topk_cluster_kernel(const float* __restrict__ scores, int64_t ld, const int32_t*
   sl_excl_scan(eq, sh.wtot, &eq_tot);
   if (tid == 0) { sh.pub[0] = (uint32_t)gt_tot; sh.pub[1] = (uint32_t)eq_tot; }
   sl_sync(cluster, C);
+  int gp[SL_CMAX], ep[SL_CMAX];
+#pragma unroll
+  for (int p = 0; p < SL_CMAX; ++p) {
+    gp[p] = p < (int)C ? (int)sl_peer(cluster, sh.pub, 0, p) : 0;
+    ep[p] = p < (int)C ? (int)sl_peer(cluster, sh.pub, 1, p) : 0;
+  }
   int all_gt = 0;
-  for (int p = 0; p < (int)C; ++p) all_gt += (int)sl_peer(cluster, sh.pub, 0, p);
+#pragma unroll
+  for (int p = 0; p < SL_CMAX; ++p) all_gt += gp[p];
   const int eq_need = k - all_gt;
   int eqp = 0, off = 0, quota = 0;
-  for (int p = 0; p < (int)C; ++p) {
-    const int g = (int)sl_peer(cluster, sh.pub, 0, p), e = (int)sl_peer(cluster, sh.pub, 1, p);
-    const int q = max(0, min(eq_need - eqp, e));
-    if (p < (int)r) off += g + q;
+#pragma unroll
+  for (int p = 0; p < SL_CMAX; ++p) {
+    const int q = max(0, min(eq_need - eqp, ep[p]));
+    if (p < (int)r) off += gp[p] + q;
     if (p == (int)r) quota = q;
-    eqp += e;
+    eqp += ep[p];
   }
   // keep the first `quota` entries equal to tau (index order)
   {
@@ -744,13 +760,14 @@ indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
     gid = sh.gband_id;
     gsc = sh.gband_s;
   }
-  int all_sure = 0;
-  for (int p = 0; p < (int)C; ++p) all_sure += (int)sl_peer(cluster, sh.pub, 0, p);
   if (tid < SL_CMAX) {
     sh.pcnt[tid][0] = (unsigned)tid < C ? sl_peer(cluster, sh.pub, 0, tid) : 0u;
     sh.pcnt[tid][1] = 0u;
   }
   __syncthreads();
+  int all_sure = 0;
+#pragma unroll
+  for (int p = 0; p < SL_CMAX; ++p) all_sure += (int)sh.pcnt[p][0];
   const int need = k - all_sure;
   for (int i = tid; i < ng; i += SL_T) {
     const double si = gsc[i];
