@@ -31,6 +31,8 @@ _SIGS = {
     "attn_decode_workspace_size": ([_i32, _i32, _i32, _i64], _sz),
     "sparse_attn_decode": ([_vp] * 6 + [_i32, _i32, _i32, _i32, _i64, _i32, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp], _i32),
     "hca_attn_decode": ([_vp] * 6 + [_i32, _i32, _i32, _i32, _i64, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp], _i32),
+    "hca_compress_attn_decode": ([_vp] * 4 + [_i32, _i32] + [_vp] * 6 + [_i32, _i32, _i32, _i32, _i64, _i32, _f32, _i32,
+                                                                      _vp, _vp, _vp, _sz, _vp], _i32),
     "sparse_attn_decode_noalloc": ([_vp] * 6 + [_i32, _i32, _i32, _i32, _i64, _i32, _i32, _f32, _i32, _vp, _vp, _vp], _i32),
     "sparse_attn_prefill": ([_vp] * 5 + [_i64, _vp, _vp] + [_i32] * 5 + [_i64, _i32, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp], _i32),
 }
@@ -139,6 +141,19 @@ def hca_attn_decode(q, cache, n_entries, win, win_len, sink, sm_scale, d_v, out,
     _check(lib.hca_attn_decode(_p(q), _p(cache), _p(n_entries), _p(win), _p(win_len), _p(sink), B, H, d_k, d_v,
                                cache.shape[1], W, sm_scale, _dtype_code(q), _p(out), _p(lse), wp, wb,
                                _stream(stream)), "hca_attn_decode")
+
+
+def hca_compress_attn_decode(C_, Z, bias, entry0, q, cache, n_entries, win, win_len, sink, sm_scale, d_v, out,
+                             lse=None, workspace=None, m_prime=128, stream=None):
+    """hca_compress of the fresh chunk (C_, Z) then hca_attn_decode, as one call."""
+    B, H, d_k = q.shape
+    T_new = C_.shape[1]
+    W = win.shape[1] if win is not None else 0
+    wp, wb = _ws(workspace)
+    _check(lib.hca_compress_attn_decode(_p(C_), _p(Z), _p(bias), _p(entry0), T_new, m_prime, _p(q), _p(cache),
+                                        _p(n_entries), _p(win), _p(win_len), _p(sink), B, H, d_k, d_v, cache.shape[1],
+                                        W, sm_scale, _dtype_code(q), _p(out), _p(lse), wp, wb, _stream(stream)),
+           "hca_compress_attn_decode")
 
 
 def sparse_attn_prefill(q, q_pos, cache, idx, raw, raw_pos0, W, sink, sm_scale, d_v, out, lse=None,

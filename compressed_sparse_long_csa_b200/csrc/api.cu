@@ -13,7 +13,7 @@ cudaError_t launch_csa_compress(const void*, const void*, const void*, const voi
                                 const void*, const void*, const int32_t*, void*, int64_t, int, int, int, int,
                                 int, cudaStream_t, unsigned*);
 cudaError_t launch_hca_compress(const void*, const void*, const float*, const int32_t*, void*, int64_t, int,
-                                int, int, int, int, cudaStream_t, unsigned*);
+                                int, int, int, int, cudaStream_t, unsigned*, int max_ctas);
 }  // namespace csa
 
 using namespace csa;
@@ -126,7 +126,7 @@ csa_status hca_compress(const void* C, const void* Z, const float* bias, const i
   unsigned* err = device_error_word();
   REQUIRE(err, CSA_ERR_CUDA);
   return cuda_status(launch_hca_compress(C, Z, bias, entry0, cache, n_max, B, T_new, d, m_prime, dtype,
-                                         S(stream), err));
+                                         S(stream), err, 0));
 }
 
 // ----------------------------------------------------------------------------- indexer / top-k
@@ -298,6 +298,39 @@ csa_status hca_attn_decode(const void* q, const void* cache, const int32_t* n_en
   a.q = q; a.cache = cache; a.idx = nullptr; a.n_entries = n_entries; a.n_seg_a = (int)n_max;
   a.win = win; a.win_len = win_len; a.W = W; a.prefill = 0; a.sink = sink; a.B = B; a.Tq = 1; a.H = H;
   a.dk = d_k; a.dv = d_v; a.n_max = n_max; a.sm_scale = sm_scale; a.out = out; a.lse = lse; a.err = err;
+  return run_attention(a, dtype, workspace, ws_bytes, true, S(stream));
+}
+
+csa_status hca_compress_attn_decode(const void* C, const void* Z, const float* bias, const int32_t* entry0, int T_new,
+                                    int m_prime, const void* q, void* cache, const int32_t* n_entries, const void* win,
+                                    const int32_t* win_len, const float* sink, int B, int H, int d_k, int d_v,
+                                    int64_t n_max, int W, float sm_scale, int dtype, void* out, float* lse,
+                                    void* workspace, size_t ws_bytes, void* stream) {
+  // every argument of both calls is checked before the first launch
+  csa_status s = attn_common_checks(q, cache, win, sink, B, H, d_k, d_v, n_max, W, dtype, out, lse);
+  if (s != CSA_OK) return s;
+  REQUIRE(n_max <= (1 << 24) && B <= 65535, CSA_ERR_SHAPE);
+  REQUIRE(n_entries, CSA_ERR_NULL);
+  REQUIRE(W == 0 || win_len, CSA_ERR_NULL);
+  REQUIRE(isfinite(sm_scale), CSA_ERR_SHAPE);
+  REQUIRE(workspace && ws_bytes >= attn_decode_workspace_size(B, H, d_v, n_max + W), CSA_ERR_WORKSPACE);
+  REQUIRE(aligned16(workspace), CSA_ERR_ALIGN);
+  REQUIRE(T_new >= 1 && m_prime >= 1 && m_prime <= 1024 && T_new % m_prime == 0, CSA_ERR_SHAPE);
+  REQUIRE(d_k % (dtype == CSA_BF16 ? 8 : 4) == 0, CSA_ERR_SHAPE);
+  REQUIRE_PTR(C); REQUIRE_PTR(Z); REQUIRE_PTR(bias);
+  REQUIRE(entry0, CSA_ERR_NULL);
+  unsigned* err = device_error_word();
+  REQUIRE(err, CSA_ERR_CUDA);
+  // the full compression grid: capping it (CTAs that loop over their slabs) left room for
+  // the whole attention grid but made the compression the longest chain
+  cudaError_t e = launch_hca_compress(C, Z, bias, entry0, cache, n_max, B, T_new, d_k, m_prime, dtype, S(stream), err, 0);
+  if (e != cudaSuccess) return CSA_ERR_CUDA;
+  AttnArgs a{};
+  a.q = q; a.cache = cache; a.idx = nullptr; a.n_entries = n_entries; a.n_seg_a = (int)n_max;
+  a.win = win; a.win_len = win_len; a.W = W; a.prefill = 0; a.sink = sink; a.B = B; a.Tq = 1; a.H = H;
+  a.dk = d_k; a.dv = d_v; a.n_max = n_max; a.sm_scale = sm_scale; a.out = out; a.lse = lse; a.err = err;
+  a.dep_entry0 = entry0;
+  a.dep_rows = T_new / m_prime;
   return run_attention(a, dtype, workspace, ws_bytes, true, S(stream));
 }
 

@@ -32,6 +32,8 @@ struct AttnArgs {
                               // tensor-core path deals 64-row tiles to the splits round-robin)
   int n_seg_a;                // virtual rows in segment A (k or n_max)
   int cluster_combine;        // tensor-core path: splits merged inside a thread-block cluster
+  const int32_t* dep_entry0;  // dense decode after a compression kernel in the same stream: it
+  int dep_rows;               // writes rows dep_entry0[b] .. +dep_rows-1 (null: wait for it at once)
   unsigned* err;
 };
 

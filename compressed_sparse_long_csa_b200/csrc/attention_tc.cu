@@ -148,8 +148,11 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  // the setup above overlaps the previous kernel's tail; every input may come from it
-  tc::griddep_wait();
+  // The setup above overlaps the previous kernel's tail; every input may come from it,
+  // except after a compression kernel that writes known rows (dep_entry0): then only the
+  // loader of a tile holding them waits, just before loading it.
+  const bool dep_rows_only = a.dep_entry0 != nullptr;
+  if (!dep_rows_only) tc::griddep_wait();
   tc::griddep_launch_dependents();
   const uint32_t tmem = sm.tmem_base;
   // The sink logit, needed only at the end, is loaded now: with one split by every softmax
@@ -185,6 +188,13 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
       }
     };
     if (g < n_t) coord(g);
+    // rows the preceding compression writes (dense decode): [dep0, dep1) of this sequence
+    int64_t dep0 = 0, dep1 = 0;
+    bool dep_done = !dep_rows_only;
+    if (dep_rows_only) {
+      dep0 = a.dep_entry0[row / a.Tq];
+      dep1 = dep0 + a.dep_rows;
+    }
     int issued = 0;                                   // tiles this group started (for the drain)
     for (int it = g, i = 0; it < n_t; it += 2, ++i) {
       const bool go = tc::mbar_wait(&sm.empty[g], (i & 1) ^ 1) && !*(volatile int*)&sm.abort_flag;
@@ -205,6 +215,13 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
       named_bar(1 + g, AT_GROUP);
       const int stop = *(volatile int*)&sm.ld_stop[g];
       if (stop != 0 && stop <= i + 1) break;
+      if (!dep_done) {
+        const int64_t r0 = (int64_t)(split + it * a.splits) * AT_ROWS;   // the tile's cache rows
+        if (r0 < dep1 && r0 + AT_ROWS > dep0) {
+          tc::griddep_wait();                         // every thread of the group loads
+          dep_done = true;
+        }
+      }
       const unsigned long long k0 = sm.run_key[g][0];
       const bool run = k0 != NO_RUN && k0 == sm.run_key[g][1];
       if (run) {

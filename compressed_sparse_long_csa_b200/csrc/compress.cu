@@ -173,54 +173,59 @@ hca_compress_kernel(const T* __restrict__ C, const T* __restrict__ Z, const floa
   constexpr int VEC = Elem<T>::VEC;
   constexpr int SLAB = 8 * VEC;
   __shared__ float sM[32][SLAB + 1], sS[32][SLAB + 1], sA[32][SLAB + 1];
+  // a dependent attention kernel (hca_compress_attn_decode) may start now: it reads the
+  // rows written here only after waiting for this grid
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int j = blockIdx.x;          // entry within chunk
-  const int slab = blockIdx.y;
   const int b = blockIdx.z;
   const int g = threadIdx.x & 7;     // component group inside slab
   const int tl = threadIdx.x >> 3;   // token lane 0..31
-  const int c0 = slab * SLAB + g * VEC;
   const int e = entry0[b] + j;
   const bool valid_e = !(e < 0 || (int64_t)e >= n_max);
-  const bool active = c0 < d;
-
-  PoolAcc acc;
-  acc.init(VEC);
-  if (active && valid_e) {
-    float cv[VEC], zv[VEC], bv[8];
-    for (int t = tl; t < mp; t += 32) {
-      const size_t off = ((size_t)b * T_new + (size_t)j * mp + t) * d + c0;
-      Elem<T>::ld_vec(C + off, cv);
-      Elem<T>::ld_vec(Z + off, zv);
-#pragma unroll
-      for (int i = 0; i < VEC; ++i) bv[i] = bias[(size_t)t * d + c0 + i];
-      acc.add(cv, zv, bv, VEC);
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < VEC; ++i) {
-    sM[tl][g * VEC + i] = acc.M[i];
-    sS[tl][g * VEC + i] = acc.S[i];
-    sA[tl][g * VEC + i] = acc.A[i];
-  }
-  __syncthreads();
   if (!valid_e) {
     if (threadIdx.x == 0) raise_err(err, CSA_DEVERR_ENTRY);
     return;
   }
-  if (threadIdx.x < SLAB) {
-    const int col = threadIdx.x;
-    const int c = slab * SLAB + col;
-    if (c < d) {
-      float M = -INFINITY;
-      for (int l = 0; l < 32; ++l) M = fmaxf(M, sM[l][col]);
-      float S = 0.f, A = 0.f;
-      for (int l = 0; l < 32; ++l) {
-        const float a = (sS[l][col] > 0.f) ? __expf(sM[l][col] - M) : 0.f;
-        S += sS[l][col] * a;
-        A += sA[l][col] * a;
+  // slabs of SLAB components: blockIdx.y, blockIdx.y + gridDim.y, ...
+  for (int slab = blockIdx.y; slab * SLAB < d; slab += gridDim.y) {
+    const int c0 = slab * SLAB + g * VEC;
+    const bool active = c0 < d;
+    PoolAcc acc;
+    acc.init(VEC);
+    if (active) {
+      float cv[VEC], zv[VEC], bv[8];
+      for (int t = tl; t < mp; t += 32) {
+        const size_t off = ((size_t)b * T_new + (size_t)j * mp + t) * d + c0;
+        Elem<T>::ld_vec(C + off, cv);
+        Elem<T>::ld_vec(Z + off, zv);
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) bv[i] = bias[(size_t)t * d + c0 + i];
+        acc.add(cv, zv, bv, VEC);
       }
-      Elem<T>::st(cache + ((size_t)b * n_max + e) * d + c, A / S);
     }
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) {
+      sM[tl][g * VEC + i] = acc.M[i];
+      sS[tl][g * VEC + i] = acc.S[i];
+      sA[tl][g * VEC + i] = acc.A[i];
+    }
+    __syncthreads();
+    if (threadIdx.x < SLAB) {
+      const int col = threadIdx.x;
+      const int c = slab * SLAB + col;
+      if (c < d) {
+        float M = -INFINITY;
+        for (int l = 0; l < 32; ++l) M = fmaxf(M, sM[l][col]);
+        float S = 0.f, A = 0.f;
+        for (int l = 0; l < 32; ++l) {
+          const float a = (sS[l][col] > 0.f) ? __expf(sM[l][col] - M) : 0.f;
+          S += sS[l][col] * a;
+          A += sA[l][col] * a;
+        }
+        Elem<T>::st(cache + ((size_t)b * n_max + e) * d + c, A / S);
+      }
+    }
+    __syncthreads();                 // the partials of the next slab reuse the shared arrays
   }
 }
 
@@ -271,16 +276,26 @@ cudaError_t launch_csa_compress(const void* Ca, const void* Cb, const void* Za, 
 
 cudaError_t launch_hca_compress(const void* C, const void* Z, const float* bias, const int32_t* entry0,
                                 void* cache, int64_t n_max, int B, int T_new, int d, int mp, int dtype,
-                                cudaStream_t st, unsigned* err) {
+                                cudaStream_t st, unsigned* err, int max_ctas) {
   const int n_blk = T_new / mp;
+  // slab groups per entry: every slab its own CTA, or fewer CTAs that loop over slabs
+  // when max_ctas bounds the grid (it runs beside an attention grid that fills the SMs)
+  auto groups = [&](int slabs) {
+    int gy = slabs;
+    if (max_ctas > 0) {
+      const int64_t per = (int64_t)max_ctas / ((int64_t)n_blk * B);
+      gy = (int)(per < 1 ? 1 : (per < slabs ? per : slabs));
+    }
+    return gy;
+  };
   if (dtype == CSA_BF16) {
     using T = __nv_bfloat16;
-    dim3 grid(n_blk, (d + 63) / 64, B);
+    dim3 grid(n_blk, groups((d + 63) / 64), B);
     note_launch();
     hca_compress_kernel<T><<<grid, 256, 0, st>>>((const T*)C, (const T*)Z, bias, entry0, (T*)cache, n_max,
                                                  T_new, d, mp, err);
   } else {
-    dim3 grid(n_blk, (d + 31) / 32, B);
+    dim3 grid(n_blk, groups((d + 31) / 32), B);
     note_launch();
     hca_compress_kernel<float><<<grid, 256, 0, st>>>((const float*)C, (const float*)Z, bias, entry0,
                                                      (float*)cache, n_max, T_new, d, mp, err);

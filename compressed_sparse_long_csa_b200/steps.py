@@ -110,12 +110,13 @@ def csa_decode_step(T, D, stream=None):
 
 
 def hca_decode_step(T, D, stream=None, prefix=""):
+    """The fresh chunk's compression and the dense attention as one call (the attention
+    streams the other entries while the compression runs)."""
     p = prefix
-    N.hca_compress(T[p + "C"], T[p + "Z"], T[p + "bias"], T[p + "entry0"], T[p + "cache"], D["m_prime"],
-                   stream=stream)
-    N.hca_attn_decode(T[p + "q"][:, 0], T[p + "cache"], T[p + "n_entries"], T[p + "win"], T[p + "win_len"],
-                      T[p + "sink"], D["sm_scale"], D["dv"], T[p + "out"][:, 0], T[p + "lse"][:, 0],
-                      T[p + "aws"], stream=stream)
+    N.hca_compress_attn_decode(T[p + "C"], T[p + "Z"], T[p + "bias"], T[p + "entry0"], T[p + "q"][:, 0],
+                               T[p + "cache"], T[p + "n_entries"], T[p + "win"], T[p + "win_len"], T[p + "sink"],
+                               D["sm_scale"], D["dv"], T[p + "out"][:, 0], T[p + "lse"][:, 0], T[p + "aws"],
+                               m_prime=D["m_prime"], stream=stream)
 
 
 def csa_prefill_step(T, D, stream=None):

@@ -213,6 +213,22 @@ csa_status hca_attn_decode(const void* q, const void* cache, const int32_t* n_en
                            float sm_scale, int dtype, void* out, float* lse,
                            void* workspace, size_t ws_bytes, void* stream);
 
+/* hca_compress_attn_decode — one HCA decode step: hca_compress of the fresh chunk
+ * into the cache, then hca_attn_decode over entries 0..n_entries[b]-1 (which include
+ * the fresh rows) + window + sink; the same results as the two calls in that order.
+ * The attention kernel starts while the compression runs: its CTAs stream the rows the
+ * compression does not write and wait for the compression only before the tile that
+ * holds rows entry0[b] .. entry0[b] + T_new/m_prime - 1.
+ *   C, Z, bias, entry0, T_new, m_prime  as hca_compress (d = d_k, same dtype as q)
+ *   other arguments                     as hca_attn_decode                          */
+csa_status hca_compress_attn_decode(const void* C, const void* Z, const float* bias,
+                                    const int32_t* entry0, int T_new, int m_prime,
+                                    const void* q, void* cache, const int32_t* n_entries,
+                                    const void* win, const int32_t* win_len, const float* sink,
+                                    int B, int H, int d_k, int d_v, int64_t n_max, int W,
+                                    float sm_scale, int dtype, void* out, float* lse,
+                                    void* workspace, size_t ws_bytes, void* stream);
+
 /* sparse_attn_prefill — Tq query tokens per sequence, each with its own index set.
  *   q        device [B, Tq, H, d_k];  q_pos device [B, Tq] int32 absolute positions
  *   idx      device [B, Tq, k] int32 (-1 = unused)

@@ -23,7 +23,7 @@ def declared_functions():
 def test_every_declared_symbol_is_exported():
     names = declared_functions()
     assert {"csa_compress", "hca_compress", "lightning_index", "topk_select", "sparse_attn_decode",
-            "sparse_attn_prefill", "hca_attn_decode"} <= set(names)
+            "sparse_attn_prefill", "hca_attn_decode", "hca_compress_attn_decode"} <= set(names)
     for n in names:
         assert hasattr(N.lib, n), n
 
@@ -104,6 +104,27 @@ def test_attention_validation():
     assert call(scale=float("nan")) == ERR_SHAPE
     assert call(ws=None, wsb=0) == ERR_WS
     assert N.lib.attn_decode_workspace_size(16, 128, 512, 640) > 0
+
+
+def test_fused_hca_step_validation_before_any_launch():
+    def call(**kw):
+        a = dict(C=FAKE, Z=FAKE, bias=FAKE, e0=FAKE, T_new=128, mp=128, q=FAKE, cache=FAKE, ne=FAKE, win=FAKE,
+                 wl=FAKE, sink=FAKE, B=2, H=128, dk=576, dv=512, n_max=8192, W=128, scale=0.04, dtype=1, out=FAKE,
+                 lse=None, ws=FAKE, wsb=1 << 30)
+        a.update(kw)
+        return N.lib.hca_compress_attn_decode(a["C"], a["Z"], a["bias"], a["e0"], a["T_new"], a["mp"], a["q"],
+                                              a["cache"], a["ne"], a["win"], a["wl"], a["sink"], a["B"], a["H"],
+                                              a["dk"], a["dv"], a["n_max"], a["W"], a["scale"], a["dtype"], a["out"],
+                                              a["lse"], a["ws"], a["wsb"], None)
+    before = N.lib.csa_launch_count()
+    assert call(T_new=100) == ERR_SHAPE        # not a multiple of m'
+    assert call(mp=2048) == ERR_SHAPE
+    assert call(e0=None) == ERR_NULL
+    assert call(C=FAKE + 8) == ERR_ALIGN
+    assert call(ne=None) == ERR_NULL
+    assert call(dv=640) == ERR_SHAPE
+    assert call(ws=None, wsb=0) == ERR_WS
+    assert N.lib.csa_launch_count() == before  # nothing was launched, not even the compression
 
 
 def test_topk_validation():

@@ -160,6 +160,32 @@ def test_hca_decode(case):
                                atol=2e-3, rtol=0)
 
 
+@pytest.mark.parametrize("case", list(HCA_CASES))
+def test_fused_hca_step_equals_separate_calls(case):
+    """hca_compress_attn_decode (attention started while the compression runs) gives
+    bit-for-bit the results of hca_compress followed by hca_attn_decode."""
+    i, sc = HCA_CASES[case]
+    wl = CI.make_workload(i, scale=sc)
+    D = wl.dims
+    T = steps.upload(wl)
+    cache0 = T["cache"].clone()
+    csa.hca_compress(T["C"], T["Z"], T["bias"], T["entry0"], T["cache"], D["m_prime"])
+    csa.hca_attn_decode(T["q"][:, 0], T["cache"], T["n_entries"], T["win"], T["win_len"], T["sink"], D["sm_scale"],
+                        D["dv"], T["out"][:, 0], T["lse"][:, 0], T["aws"])
+    torch.cuda.synchronize()
+    out_sep, lse_sep, cache_sep = T["out"].clone(), T["lse"].clone(), T["cache"].clone()
+    T["cache"].copy_(cache0)
+    T["out"].zero_()
+    csa.hca_compress_attn_decode(T["C"], T["Z"], T["bias"], T["entry0"], T["q"][:, 0], T["cache"], T["n_entries"],
+                                 T["win"], T["win_len"], T["sink"], D["sm_scale"], D["dv"], T["out"][:, 0],
+                                 T["lse"][:, 0], T["aws"], m_prime=D["m_prime"])
+    torch.cuda.synchronize()
+    assert csa.read_device_error() == 0
+    assert torch.equal(T["cache"], cache_sep)
+    assert torch.equal(T["out"], out_sep)
+    assert torch.equal(T["lse"], lse_sep)
+
+
 # ----------------------------------------------------------------------------- edge cases
 
 def test_decode_ragged_window_pad_indices_and_determinism():
