@@ -580,7 +580,7 @@ indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
   tc::griddep_launch_dependents();
   // ---- the query row (written before the scoring kernel started: read before waiting
   // for it): codes into registers (staged into shared memory once the scores are
-  // classified), scales and weights, and U = sum_j w_j ||q_j|| for the error bound
+  // classified), scales and weights, and U = sum_j |w_j| ||q_j|| for the error bound
   const int m4 = (n > k) ? (m & ~3) : 0;
   const float* srow = a.scores + (size_t)row * a.ld + lo;
   if (tid == 0) {
@@ -602,7 +602,7 @@ indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
       } else qx[e] = ((const float*)a.qI)[r0 + i];
     }
   }
-  // weights and scales, and the words of this warp's heads for U = sum_j w_j ||q_j||
+  // weights and scales, and the words of this warp's heads for U = sum_j |w_j| ||q_j||
   // (warp w takes heads w, w + SL_W, ...; lane l holds elements [epl*l, epl*l + epl)):
   // every load of the prologue is issued before any is used
   constexpr int EPL = (F == CSA_IFMT_MXFP4) ? 8 : 4;
@@ -631,6 +631,17 @@ indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
   // ---- the scoring kernel's outputs: key-norm bound and key range (the scores follow
   // by one bulk copy into shared memory, the tail by plain loads)
   tc::griddep_wait();
+  // the scores go into shared memory first (one bulk copy, the tail by plain loads); the
+  // head-norm bound below runs while they travel (tid 0 initialised the barrier itself)
+  if (tid == 0) {
+    tc::mbar_arrive_expect_tx(&sh.ldbar, (uint32_t)m4 * 4u);
+    for (int o = 0; o < m4; o += 8192) {
+      const uint32_t bytes = (uint32_t)min(8192, m4 - o) * 4u;
+      asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                   ::"r"(tc::smem_u32(sv + o)), "l"(srow + o), "r"(bytes), "r"(tc::smem_u32(&sh.ldbar)) : "memory");
+    }
+  }
+  if (n > k && tid < m - m4) sv[m4 + tid] = srow[m4 + tid];
   const float knmax = __uint_as_float(a.knmax[b]);
   // the key range the scoring kernel recorded (exact min / max over the row's eligible entries)
   uint32_t lo_k = ~a.keyrange[2 * (size_t)row + 1], hi_k = a.keyrange[2 * (size_t)row];
@@ -675,19 +686,10 @@ indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
 #pragma unroll
     for (int h = 0; h < 64 / SL_W; ++h) {
       const int j = warp + SL_W * h;
-      if (j < HI) uw += sh.w[j] * sqrtf(n2[h]);
+      if (j < HI) uw += fabsf(sh.w[j]) * sqrtf(n2[h]);     // |w|: the bound holds for any sign
     }
     if (lane == 0) atomicAdd(&sh.U, uw);                   // read after the barriers below
   }
-  if (tid == 0) {
-    tc::mbar_arrive_expect_tx(&sh.ldbar, (uint32_t)m4 * 4u);
-    for (int o = 0; o < m4; o += 8192) {
-      const uint32_t bytes = (uint32_t)min(8192, m4 - o) * 4u;
-      asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                   ::"r"(tc::smem_u32(sv + o)), "l"(srow + o), "r"(bytes), "r"(tc::smem_u32(&sh.ldbar)) : "memory");
-    }
-  }
-  if (n > k && tid < m - m4) sv[m4 + tid] = srow[m4 + tid];
   if (resc_sep) sl_stage_query(rs, qx, total, lgd, HI, dI);   // covered by the barrier below
   // the scores have landed (bounded wait; on a timeout the error word is set)
   if (n > k && m4 > 0) {

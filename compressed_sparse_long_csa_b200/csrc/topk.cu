@@ -480,7 +480,7 @@ indexer_select_kernel(IndexerArgs a) {
         if (a.ifmt == CSA_IFMT_MXFP4) v *= sh.qsc[j * nb + c / 32];
         n2 = fmaf(v, v, n2);
       }
-      u += sh.w[j] * sqrtf(n2);
+      u += fabsf(sh.w[j]) * sqrtf(n2);      // |w|: the bound holds for any sign
     }
     u = warp_sum(u);
     if (lane == 0) sh.U = u * 1.0001f;
