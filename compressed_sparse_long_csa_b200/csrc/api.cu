@@ -64,6 +64,18 @@ std::atomic<uint64_t> g_launches{0};
 
 void csa::note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
+int csa::num_sms() {
+  static const int n = [] {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+        v > 0)
+      return v;
+    cudaGetLastError();
+    return 148;
+  }();
+  return n;
+}
+
 extern "C" {
 
 int csa_abi_version(void) { return CSA_ABI_VERSION; }
@@ -172,7 +184,7 @@ csa_status lightning_index(const void* qI, const void* qI_scale, const float* w,
   if (e != cudaSuccess) return CSA_ERR_CUDA;
   bool used_tc = false;
   if (tc_enabled()) {
-    e = launch_indexer_scores_tc(a, S(stream), &used_tc);
+    e = launch_indexer_scores_tc(a, S(stream), &used_tc);       // sets a.eps_dot of its path
     if (e != cudaSuccess) return CSA_ERR_CUDA;
   }
   if (!used_tc) {

@@ -293,16 +293,16 @@ int attn_choose_splits(int n_queries, int H, int64_t rows, bool tc_path) {
   if (tc_path) {
     // one wave of CTAs (two per query and split, one CTA per SM), splits of at least two
     // 64-row tiles, and the tiles spread as evenly as whole tiles allow
-    s = 148 / (2 * (int64_t)n_queries);
+    s = num_sms() / (2 * (int64_t)n_queries);
     if (s > tiles / 2) s = tiles / 2;
     if (s > 64) s = 64;                      // attn_combine_kernel keeps 64 splits' weights
     if (s < 1) s = 1;
     const int64_t per = (tiles + s - 1) / s;
     s = (tiles + per - 1) / per;
   } else {
-    // aim for >= 2 waves of CTAs on 148 SMs
+    // aim for >= 2 waves of CTAs
     const int64_t ctas_per_split = (int64_t)n_queries * ((H + CC_HG - 1) / CC_HG);
-    s = (2 * 148 + ctas_per_split - 1) / ctas_per_split;
+    s = (2 * (int64_t)num_sms() + ctas_per_split - 1) / ctas_per_split;
   }
   if (s > tiles) s = tiles;
   if (s < 1) s = 1;

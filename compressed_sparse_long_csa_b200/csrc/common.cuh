@@ -10,6 +10,9 @@ namespace csa {
 
 // Counts the kernels the library enqueues (defined in api.cu; read by csa_launch_count).
 void note_launch();
+// SMs of the current device (148 on B200), read once; 148 when no device answers (the
+// host-only size queries of a machine without a GPU).  Grids are planned in its units.
+int num_sms();
 
 // Error bits are OR-ed into a per-device word owned by api.cu; kernels get its address.
 __device__ __forceinline__ void raise_err(unsigned* err, unsigned bit) {

@@ -73,7 +73,7 @@ __device__ __forceinline__ void record_key_range(unsigned* keyrange, int row, fl
 }
 
 cudaError_t launch_indexer_scores_cuda_core(const IndexerArgs& a, cudaStream_t st);
-cudaError_t launch_indexer_scores_tc(const IndexerArgs& a, cudaStream_t st, bool* used);
+cudaError_t launch_indexer_scores_tc(IndexerArgs& a, cudaStream_t st, bool* used);   // sets a.eps_dot
 cudaError_t launch_indexer_select(const IndexerArgs& a, cudaStream_t st);
 cudaError_t launch_topk_select(const float* scores, int64_t ld, const int32_t* n_valid, int R, int64_t n,
                                int k, int32_t* idx_out, cudaStream_t st, unsigned* err);

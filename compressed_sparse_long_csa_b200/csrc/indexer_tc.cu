@@ -532,7 +532,7 @@ cudaError_t launch_mxf4(const IndexerArgs& a, cudaStream_t st, bool* used) {
   p.n_qg = a.Tq;
   p.tiles = (int)((a.n_max + IT_ROWS - 1) / IT_ROWS);
   const int64_t ctas = (int64_t)a.B * a.Tq;
-  int splits = (int)(2 * 148 / ctas);               // one wave: two CTAs per SM
+  int splits = (int)(2 * num_sms() / ctas);         // one wave: two CTAs per SM
   if (splits > p.tiles) splits = p.tiles;
   if (splits < 1) splits = 1;
   p.tiles_per_split = (p.tiles + splits - 1) / splits;
@@ -560,7 +560,7 @@ cudaError_t launch_g(const IndexerArgs& a, cudaStream_t st, bool* used) {
   // decode-like shapes: split the entry tiles so that the grid fills the SMs once
   // (two CTAs per SM for the one-query variant, one for the four-query variant)
   const int64_t ctas = (int64_t)a.B * p.n_qg;
-  const int64_t slots = G == 1 ? 2 * 148 : 148;
+  const int64_t slots = G == 1 ? 2 * num_sms() : num_sms();
   int splits = (int)(slots / ctas);
   if (splits > p.tiles) splits = p.tiles;
   if (splits < 1) splits = 1;
@@ -584,14 +584,14 @@ cudaError_t launch_g(const IndexerArgs& a, cudaStream_t st, bool* used) {
 
 // Tensor-core scores for E4M3 operands with 64 heads of width 128; other shapes
 // return *used = false and run on the CUDA-core path.
-cudaError_t launch_indexer_scores_tc(const IndexerArgs& a, cudaStream_t st, bool* used) {
+cudaError_t launch_indexer_scores_tc(IndexerArgs& a, cudaStream_t st, bool* used) {
   *used = false;
   if (a.ifmt == CSA_IFMT_MXFP4 && a.H_I == 64 && a.d_I == 128) {
     if (((uintptr_t)a.kI & 15) || ((uintptr_t)a.qI & 15) || ((uintptr_t)a.kI_scale & 3) || ((uintptr_t)a.qI_scale & 3))
       return cudaSuccess;
     if ((int64_t)a.B * a.n_max > 0x7fffffffLL || (int64_t)a.B * a.Tq * 64 > 0x7fffffffLL) return cudaSuccess;
     // same bound as the E4M3 kernel
-    const_cast<IndexerArgs&>(a).eps_dot = 1.0f / 131072.0f;
+    a.eps_dot = 1.0f / 131072.0f;
     return launch_mxf4(a, st, used);
   }
   if (a.ifmt != CSA_IFMT_E4M3 || a.H_I != 64 || a.d_I != 128) return cudaSuccess;
@@ -600,7 +600,7 @@ cudaError_t launch_indexer_scores_tc(const IndexerArgs& a, cudaStream_t st, bool
   // Bound on |fp32 MMA dot - exact| relative to ||q|| ||k||: the worst case of a 128-term
   // fp32 accumulation of exact products (128 * 2^-24 = 2^-17).  Measured on B200: <= 5e-9
   // relative to the bound's scale (test_indexer_fp32_score_error_within_band_bound).
-  const_cast<IndexerArgs&>(a).eps_dot = 1.0f / 131072.0f;
+  a.eps_dot = 1.0f / 131072.0f;
   if (a.Tq >= 4) return launch_g<4, 6>(a, st, used);
   return launch_g<1, 6>(a, st, used);
 }

@@ -821,8 +821,8 @@ bool sl_plan(int64_t n, int rows, int* C, int* chunk) {
   int64_t cc = c < 1 ? 1 : c;
   // few rows: up to four CTAs per row (their passes over the scores are shorter, their
   // band re-scoring is shared), while each CTA keeps at least 4096 entries
-  if ((int64_t)rows * cc < 148) {
-    int64_t want = 148 / rows;
+  if ((int64_t)rows * cc < num_sms()) {
+    int64_t want = num_sms() / rows;
     if (want > 4) want = 4;
     while (want > cc && (n + want - 1) / want < 4096) --want;
     if (want > cc) cc = want;
