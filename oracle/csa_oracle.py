@@ -257,6 +257,96 @@ def n_eligible(pos, m, n_entries):
 
 
 # ---------------------------------------------------------------------------
+# indexer-key producer  ([P1] section "FP4 с учётом квантования": the indexer's
+# Q·K activations are cached and multiplied in FP4, MXFP4 with 1x32 tiles; the
+# keys of the compressed entries come from CSA step 1's gated pooling)
+#
+# Readings: the pooled value is quantised directly (no bf16 intermediate), and
+# every quantisation decision is taken on that value as an fp32 number, the
+# precision of the CUDA kernel: E4M3 scale = fp32(amax / 448) (1 for an
+# all-zero row) and y = fp32(x / scale); MXFP4 exponent e = the smallest integer
+# with amax <= 6 * 2^e over each 32-block (clamped to [-127, 127]; -127 for an
+# all-zero block) and y = x * 2^-e.  Codes round y to the nearest grid value,
+# ties to the even code, saturating at the largest finite value; a value that
+# rounds to zero gets the +0 code.
+# ---------------------------------------------------------------------------
+
+def _encode_nearest(y, mags, sign_bit):
+    """Codes of the grid values nearest to y; mags[c] is the magnitude of code c, increasing.
+
+    Ties go to the even code; |y| beyond the last magnitude saturates to it."""
+    a = np.minimum(np.abs(np.asarray(y, dtype=np.float64)), mags[-1])
+    hi = np.clip(np.searchsorted(mags, a, side="left"), 0, len(mags) - 1)
+    lo = np.maximum(hi - 1, 0)
+    dlo = a - mags[lo]
+    dhi = mags[hi] - a
+    pick_hi = (dhi < dlo) | ((dhi == dlo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo).astype(np.int64)
+    neg = (np.asarray(y) < 0) & (code != 0)
+    return (code | np.where(neg, sign_bit, 0)).astype(np.uint8)
+
+
+E4M3_MAGS = E4M3[:0x7F].copy()        # codes 0x00..0x7E: 0 .. 448, increasing
+E2M1_MAGS = E2M1[:8].copy()           # codes 0..7: 0, .5, 1, 1.5, 2, 3, 4, 6
+
+
+def encode_e4m3(y):
+    return _encode_nearest(y, E4M3_MAGS, 0x80)
+
+
+def encode_e2m1(y):
+    return _encode_nearest(y, E2M1_MAGS, 0x8)
+
+
+def mx_exponent(amax):
+    """Smallest integer e with amax <= 6 * 2^e (exact comparisons), clamped to [-127, 127];
+    -127 for amax == 0."""
+    amax = np.asarray(amax, dtype=np.float64)
+    out = np.full(amax.shape, -127, dtype=np.int64)
+    for idx in np.ndindex(amax.shape):
+        a = float(amax[idx])
+        if a == 0.0:
+            continue
+        e = math.frexp(a)[1] - 3                 # 6 * 2^e < a here
+        while 6.0 * 2.0 ** e < a:
+            e += 1
+        out[idx] = min(max(e, -127), 127)
+    return out
+
+
+def quantise_index_keys(x, fmt):
+    """Quantise pooled rows x [n, d] (float64) to the lightning indexer's key format.
+
+    Returns (codes, scales, y): E4M3 -> codes uint8 [n, d], scales float32 [n];
+    MXFP4 -> codes uint8 [n, d/2] (element 2i in the low nibble), scales ue8m0
+    uint8 [n, d/32].  y is the pre-rounding value on the code grid (float64)."""
+    x32 = np.asarray(x, dtype=np.float64).astype(np.float32)
+    n, d = x32.shape
+    if fmt == "e4m3":
+        amax = np.abs(x32).max(axis=1)
+        scale = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
+        y = (x32 / scale[:, None]).astype(np.float32).astype(np.float64)
+        return encode_e4m3(y), scale, y
+    if fmt == "mxfp4":
+        assert d % 32 == 0
+        blk = x32.reshape(n, d // 32, 32).astype(np.float64)
+        e = mx_exponent(np.abs(blk).max(axis=2))                        # [n, d/32]
+        y = (blk * np.ldexp(1.0, -e)[:, :, None]).reshape(n, d)
+        c = encode_e2m1(y)
+        packed = (c[:, 0::2] | (c[:, 1::2] << 4)).astype(np.uint8)
+        return packed, (e + 127).astype(np.uint8), y
+    raise ValueError(fmt)
+
+
+def index_key_compress(Ca, Cb, Za, Zb, Ba, Bb, fmt, prev_Cb=None, prev_Zb=None, first_entry=0, m=4):
+    """Indexer keys of the entries a chunk completes: csa_compress of the indexer
+    activations, then quantise_index_keys.  Returns (codes, scales, y, x)."""
+    x = csa_compress(Ca, Cb, Za, Zb, Ba, Bb, prev_Cb, prev_Zb, first_entry, m)
+    codes, scales, y = quantise_index_keys(x, fmt)
+    return codes, scales, y, x
+
+
+# ---------------------------------------------------------------------------
 # a4: top-k  ([P1] CSA step 2; k from table "Конфигурации")
 # ---------------------------------------------------------------------------
 

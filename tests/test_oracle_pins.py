@@ -370,3 +370,105 @@ def test_window_range():
     assert O.window_range(0, 16) == (0, 1)
     assert O.window_range(5, 16) == (0, 6)
     assert O.window_range(100, 16) == (85, 101)
+
+
+# ---------------------------------------------------------------- indexer-key producer
+# [P1] section "FP4 с учётом квантования": the indexer's Q·K activations are cached in
+# FP4 (MXFP4, 1x32 tiles); the keys of compressed entries come from CSA step 1's pooling.
+
+def _e4m3_cases():
+    mags = O.E4M3_MAGS
+    mids = (mags[1:] + mags[:-1]) / 2                       # every rounding tie
+    r = np.random.default_rng(7)
+    rand = np.exp(r.uniform(np.log(2.0 ** -12), np.log(448.0), 4000))
+    v = np.concatenate([mags, mids, rand, mids * (1 + 2.0 ** -20), mids * (1 - 2.0 ** -20)])
+    v = v[v <= 448.0]
+    return np.concatenate([v, -v])
+
+
+def test_e4m3_encoder_matches_torch_cast():
+    """torch's float8_e4m3fn cast (round to nearest even) is an independent encoder in the
+    finite range; it keeps the sign of a value that rounds to zero, the oracle writes +0."""
+    v = _e4m3_cases()
+    ref = torch.tensor(v, dtype=torch.float64).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    ref = np.where(ref == 0x80, 0, ref)
+    assert np.array_equal(O.encode_e4m3(v), ref)
+
+
+def test_e4m3_encoder_landmarks_and_saturation():
+    v = np.array([1.0, 17.0, 19.0, 2.0 ** -10, 3 * 2.0 ** -10, 448.0, 464.0, 1e6, -1e6, -1e-5, -2.0 ** -9])
+    # 17 ties 16 (even mantissa) / 18; 19 ties 18 / 20 (even); 2^-10 ties 0 / 2^-9
+    assert O.encode_e4m3(v).tolist() == [0x38, 0x58, 0x5A, 0x00, 0x02, 0x7E, 0x7E, 0x7E, 0xFE, 0x00, 0x81]
+
+
+def test_e2m1_encoder_ties_and_saturation():
+    # grid 0 .5 1 1.5 2 3 4 6 (codes 0..7); ties go to the even code
+    v = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 7.0, 0.26, 4.9, -0.1, -0.3, -6.0, -100.0])
+    assert O.encode_e2m1(v).tolist() == [0, 2, 2, 4, 4, 6, 6, 7, 1, 6, 0, 9, 15, 15]
+
+
+def test_mx_exponent_is_smallest_power_covering_amax():
+    f32_above_6 = float(np.nextafter(np.float32(6.0), np.float32(7.0)))
+    a = np.array([6.0, f32_above_6, 3.0, 0.0, 1.5, 1.5000001, 1e-45, 6.0 * 2.0 ** 100])
+    assert O.mx_exponent(a).tolist() == [0, 1, -1, -127, -2, -1, -127, 100]
+    r = np.random.default_rng(3)
+    amax = np.exp(r.uniform(-30, 30, 500))
+    e = O.mx_exponent(amax)
+    assert np.all(amax <= 6.0 * np.ldexp(1.0, e)) and np.all(amax > 6.0 * np.ldexp(1.0, e - 1))
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "mxfp4"])
+def test_quantised_keys_are_nearest_grid_values(fmt):
+    """Brute force: every code decodes to a grid value at least as close to y as any
+    other; the row (block) maximum lands at the top of the grid."""
+    r = np.random.default_rng(11)
+    x = r.normal(size=(24, 128)) * np.exp(r.uniform(-8, 8, size=(24, 1)))
+    x[3] = 0.0                                              # an all-zero row
+    codes, scales, y = O.quantise_index_keys(x, fmt)
+    if fmt == "e4m3":
+        grid = O.E4M3_MAGS
+        dq = O.decode_e4m3(codes)
+        assert scales[3] == 1.0 and not codes[3].any()
+        live = np.abs(x).max(axis=1) > 0
+        assert np.all(np.abs(y[live]).max(axis=1) == pytest.approx(448.0, rel=1e-6))
+        # half a step of the grid: 2^-4 relative for normals, 2^-10 absolute (in units of the
+        # scale) among subnormals, plus the fp32 rounding of x and y
+        s64 = scales[:, None].astype(np.float64)
+        assert np.all(np.abs(dq * s64 - x) <= 2.0 ** -4 * np.abs(x) + 2.0 ** -10 * s64 + 2.0 ** -22 * np.abs(x))
+    else:
+        grid = O.E2M1_MAGS
+        dq = O.decode_e2m1_packed(codes)
+        assert not codes[3].any() and np.all(scales[3] == 0)
+        top = np.abs(y).reshape(24, 4, 32).max(axis=2)
+        live = top > 0
+        assert np.all((top[live] > 3.0) & (top[live] <= 6.0))
+    dist = np.abs(np.abs(y)[..., None] - grid).min(axis=-1)
+    assert np.allclose(np.abs(np.abs(dq) - np.abs(y)), dist, rtol=0, atol=0)
+    assert np.all((np.sign(dq) == np.sign(y)) | (dq == 0))
+
+
+def test_index_key_compress_constant_rows_give_grid_codes():
+    """C constant along tokens: any gates give that constant (weights sum to one), so
+    rows that sit on the code grid come back as exactly those codes."""
+    r = np.random.default_rng(5)
+    m, d, n = 4, 64, 3
+    e4 = O.E4M3_MAGS[r.integers(1, 126, size=(n, d))] * np.where(r.random((n, d)) < 0.5, -1, 1)
+    e4[:, 0] = 448.0
+    row = np.repeat(e4, m, axis=0)                           # [n*m, d]: token 4i+t carries entry i's row
+    Z = lambda: r.normal(0, 2, size=(n * m, d))
+    B = lambda: r.normal(0, 0.1, size=(m, d))
+    prev = np.repeat(e4[:1], m, axis=0)
+    codes, scales, y, x = O.index_key_compress(row, np.concatenate([row[m:], prev]), Z(), Z(), B(), B(),
+                                               "e4m3", prev_Cb=prev, prev_Zb=r.normal(size=(m, d)),
+                                               first_entry=0)
+    # entry 0 pools only its own a-block; entries 1.. pool the b-series of block i-1,
+    # which carries row i here (Cb is shifted by one block), so every entry sees one value
+    assert np.array_equal(scales, np.ones(n, np.float32))
+    assert np.array_equal(O.decode_e4m3(codes), e4)
+    g = O.E2M1_MAGS[r.integers(0, 8, size=(n, d))] * np.where(r.random((n, d)) < 0.5, -1, 1)
+    g[:, ::32] = 6.0
+    rowg = np.repeat(g * 4.0, m, axis=0)
+    codes, scales, y, x = O.index_key_compress(rowg, np.concatenate([rowg[m:], rowg[:m]]), Z(), Z(), B(), B(),
+                                               "mxfp4")
+    assert np.all(scales == 129)                             # 2^2 covers 24 = 6 * 4
+    assert np.array_equal(O.decode_e2m1_packed(codes), g + 0.0)
