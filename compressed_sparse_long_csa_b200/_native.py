@@ -23,6 +23,7 @@ _SIGS = {
     "csa_read_device_error": ([_vp, C.POINTER(C.c_uint32)], _i32),
     "csa_launch_count": ([], C.c_uint64),
     "csa_compress": ([_vp] * 10 + [_i64, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
+    "index_key_compress": ([_vp] * 11 + [_i64, _i32, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
     "hca_compress": ([_vp] * 5 + [_i64, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
     "lightning_index_workspace_size": ([_i32, _i32, _i64, _i32], _sz),
     "lightning_index": ([_vp] * 7 + [_i32, _i32, _i32, _i32, _i32, _i64, _i32, _i32, _vp, _vp, _vp, _sz, _vp], _i32),
@@ -84,6 +85,13 @@ def csa_compress(Ca, Cb, Za, Zb, Ba, Bb, prev_Cb, prev_Zb, entry0, cache, m=4, s
     _check(lib.csa_compress(_p(Ca), _p(Cb), _p(Za), _p(Zb), _p(Ba), _p(Bb), _p(prev_Cb), _p(prev_Zb),
                             _p(entry0), _p(cache), cache.shape[1], B, T_new, d, m, _dtype_code(Ca),
                             _stream(stream)), "csa_compress")
+
+
+def index_key_compress(Ca, Cb, Za, Zb, Ba, Bb, prev_Cb, prev_Zb, entry0, kI, kI_scale, ifmt, m=4, stream=None):
+    B, T_new, d_I = Ca.shape
+    _check(lib.index_key_compress(_p(Ca), _p(Cb), _p(Za), _p(Zb), _p(Ba), _p(Bb), _p(prev_Cb), _p(prev_Zb),
+                                  _p(entry0), _p(kI), _p(kI_scale), kI.shape[1], B, T_new, d_I, m,
+                                  _dtype_code(Ca), ifmt, _stream(stream)), "index_key_compress")
 
 
 def hca_compress(C_, Z, bias, entry0, cache, m_prime=128, stream=None):

@@ -14,6 +14,9 @@ cudaError_t launch_csa_compress(const void*, const void*, const void*, const voi
                                 int, cudaStream_t, unsigned*);
 cudaError_t launch_hca_compress(const void*, const void*, const float*, const int32_t*, void*, int64_t, int,
                                 int, int, int, int, cudaStream_t, unsigned*, int max_ctas);
+cudaError_t launch_index_key_compress(const void*, const void*, const void*, const void*, const float*,
+                                      const float*, const void*, const void*, const int32_t*, void*, void*, int64_t,
+                                      int, int, int, int, int, cudaStream_t, unsigned*);
 }  // namespace csa
 
 using namespace csa;
@@ -139,6 +142,26 @@ csa_status hca_compress(const void* C, const void* Z, const float* bias, const i
   REQUIRE(err, CSA_ERR_CUDA);
   return cuda_status(launch_hca_compress(C, Z, bias, entry0, cache, n_max, B, T_new, d, m_prime, dtype,
                                          S(stream), err, 0));
+}
+
+csa_status index_key_compress(const void* Ca, const void* Cb, const void* Za, const void* Zb, const float* Ba,
+                              const float* Bb, const void* prev_Cb, const void* prev_Zb, const int32_t* entry0,
+                              void* kI, void* kI_scale, int64_t n_max, int B, int T_new, int d_I, int m, int dtype,
+                              int ifmt, void* stream) {
+  REQUIRE(dtype == CSA_F32 || dtype == CSA_BF16, CSA_ERR_DTYPE);
+  REQUIRE(ifmt == CSA_IFMT_E4M3 || ifmt == CSA_IFMT_MXFP4, CSA_ERR_DTYPE);
+  REQUIRE(B >= 1 && B <= 65535 && T_new >= 1 && n_max >= 1, CSA_ERR_SHAPE);
+  REQUIRE(m == 4, CSA_ERR_UNSUPPORTED);
+  REQUIRE(T_new % m == 0, CSA_ERR_SHAPE);
+  // d_I / (components per thread) threads share an entry: a power of two within a warp
+  REQUIRE(d_I == 32 || d_I == 64 || d_I == 128 || (d_I == 256 && dtype == CSA_BF16), CSA_ERR_UNSUPPORTED);
+  REQUIRE_PTR(Ca); REQUIRE_PTR(Cb); REQUIRE_PTR(Za); REQUIRE_PTR(Zb); REQUIRE_PTR(Ba); REQUIRE_PTR(Bb);
+  REQUIRE_PTR(prev_Cb); REQUIRE_PTR(prev_Zb); REQUIRE_PTR(kI); REQUIRE_PTR(kI_scale);
+  REQUIRE(entry0, CSA_ERR_NULL);
+  unsigned* err = device_error_word();
+  REQUIRE(err, CSA_ERR_CUDA);
+  return cuda_status(launch_index_key_compress(Ca, Cb, Za, Zb, Ba, Bb, prev_Cb, prev_Zb, entry0, kI, kI_scale,
+                                               n_max, B, T_new, d_I, dtype, ifmt, S(stream), err));
 }
 
 // ----------------------------------------------------------------------------- indexer / top-k

@@ -9,6 +9,8 @@
 // Both kernels are HBM-bound: every input element is read exactly once and every
 // output element written once, with 16-byte vector accesses.  Softmax statistics
 // are kept per component in fp32 with a streaming (running max / sum) update.
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace csa {
@@ -93,22 +95,18 @@ csa_compress_kernel(const T* __restrict__ Ca, const T* __restrict__ Cb, const T*
 
 // m = 4 (the CSA rate): all 16 source vectors and 8 bias vectors of a thread are
 // loaded before any arithmetic, so a thread waits for one memory round trip instead
-// of one per source.
+// of one per source.  Pools components c0 .. c0+VEC-1 of chunk entry j into out[];
+// returns the entry's index in the cache, or -1 (error word set) when it is outside
+// [0, n_max).
 template <typename T>
-__global__ void __launch_bounds__(256)
-csa_compress_m4_kernel(const T* __restrict__ Ca, const T* __restrict__ Cb, const T* __restrict__ Za,
-                       const T* __restrict__ Zb, const float* __restrict__ Ba, const float* __restrict__ Bb,
-                       const T* __restrict__ pCb, const T* __restrict__ pZb, const int32_t* __restrict__ entry0,
-                       T* __restrict__ cache, int64_t n_max, int T_new, int d, unsigned* err) {
+__device__ __forceinline__ int pool_m4(const T* __restrict__ Ca, const T* __restrict__ Cb,
+                                       const T* __restrict__ Za, const T* __restrict__ Zb,
+                                       const float* __restrict__ Ba, const float* __restrict__ Bb,
+                                       const T* __restrict__ pCb, const T* __restrict__ pZb,
+                                       const int32_t* __restrict__ entry0, int64_t n_max, int T_new, int d,
+                                       int b, int j, int c0, float* out, unsigned* err) {
   constexpr int VEC = Elem<T>::VEC;
   constexpr int M = 4;
-  const int b = blockIdx.y;
-  const int groups = d / VEC;
-  const int n_blk = T_new / M;
-  const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (gid >= (int64_t)n_blk * groups) return;
-  const int j = (int)(gid / groups);
-  const int c0 = (int)(gid % groups) * VEC;
   const int e0 = entry0[b];                // in flight with the source loads below
   const size_t seq = (size_t)b * T_new * d;
   float c[2 * M][VEC], z[2 * M][VEC], bias[2 * M][VEC];
@@ -139,9 +137,8 @@ csa_compress_m4_kernel(const T* __restrict__ Ca, const T* __restrict__ Cb, const
     }
   }
   const int e = e0 + j;
-  if (e < 0 || (int64_t)e >= n_max) { raise_err(err, CSA_DEVERR_ENTRY); return; }
+  if (e < 0 || (int64_t)e >= n_max) { raise_err(err, CSA_DEVERR_ENTRY); return -1; }
   const bool has_b = e > 0;
-  float out[VEC];
 #pragma unroll
   for (int i = 0; i < VEC; ++i) {
     float mx = -INFINITY;
@@ -159,7 +156,121 @@ csa_compress_m4_kernel(const T* __restrict__ Ca, const T* __restrict__ Cb, const
     }
     out[i] = A / S;
   }
+  return e;
+}
+
+// One thread per (entry, VEC-wide component group), m = 4.  grid.y = batch.
+template <typename T>
+__global__ void __launch_bounds__(256)
+csa_compress_m4_kernel(const T* __restrict__ Ca, const T* __restrict__ Cb, const T* __restrict__ Za,
+                       const T* __restrict__ Zb, const float* __restrict__ Ba, const float* __restrict__ Bb,
+                       const T* __restrict__ pCb, const T* __restrict__ pZb, const int32_t* __restrict__ entry0,
+                       T* __restrict__ cache, int64_t n_max, int T_new, int d, unsigned* err) {
+  constexpr int VEC = Elem<T>::VEC;
+  const int b = blockIdx.y;
+  const int groups = d / VEC;
+  const int n_blk = T_new / 4;
+  const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= (int64_t)n_blk * groups) return;
+  const int j = (int)(gid / groups);
+  const int c0 = (int)(gid % groups) * VEC;
+  float out[VEC];
+  const int e = pool_m4<T>(Ca, Cb, Za, Zb, Ba, Bb, pCb, pZb, entry0, n_max, T_new, d, b, j, c0, out, err);
+  if (e < 0) return;
   Elem<T>::st_vec(cache + ((size_t)b * n_max + e) * d + c0, out);
+}
+
+// ---- indexer-key producer -------------------------------------------------------------------
+// "Техотчёт DeepSeek-V4 (2026)", section "FP4 с учётом квантования": the indexer's Q·K path
+// caches its activations in FP4 (MXFP4, one scale per 1x32 tile).  The key of a compressed
+// entry is the CSA step-1 pooling (m = 4) of the indexer activations, quantised in this
+// kernel's epilogue to the format lightning_index reads:
+//   E4M3:  scale = amax(|row|) / 448 (1 for an all-zero row), code = RNE(x / scale), one fp32
+//          scale per row;
+//   MXFP4: per 32 components, e = the smallest integer with amax <= 6 * 2^e (clamped to
+//          [-127, 127]), code = RNE_e2m1(x * 2^-e), scale byte e + 127.
+// Every decision is taken on the fp32 pooled value (IEEE division for E4M3, an exact power
+// of two for MXFP4); the hardware conversion rounds to nearest even and saturates, and a
+// value that rounds to zero is written as +0.  The d / VEC threads of an entry (a power of
+// two <= 32, an aligned lane group) share the amax through shuffles.
+__device__ __forceinline__ uint32_t e4m3x2_rn(float lo, float hi) {
+  uint16_t h;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(hi), "f"(lo));
+  uint32_t v = h;
+  if ((v & 0x7Fu) == 0) v &= 0xFF00u;                    // +0, not -0
+  if ((v & 0x7F00u) == 0) v &= 0x00FFu;
+  return v;
+}
+
+__device__ __forceinline__ uint32_t e2m1x2_rn(float lo, float hi) {
+  uint32_t v;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+      : "=r"(v) : "f"(hi), "f"(lo));
+  if ((v & 0x7u) == 0) v &= 0xF0u;
+  if ((v & 0x70u) == 0) v &= 0x0Fu;
+  return v;
+}
+
+// The MX exponent of a block maximum, from its fp32 fields: amax = f * 2^E, f in [1, 2),
+// and 6 * 2^e = 1.5 * 2^(e+2), so e = E - 2 when f <= 1.5, else E - 1.
+__device__ __forceinline__ int mx_exponent(float amax) {
+  const uint32_t u = __float_as_uint(amax);
+  const int E = (int)((u >> 23) & 0xFFu);
+  if (E == 0) return -127;                                // zero or subnormal: below 2^-127 * 6
+  const int e = (u & 0x7FFFFFu) > 0x400000u ? E - 128 : E - 129;
+  return e < -127 ? -127 : e;
+}
+
+template <typename T, int FMT>
+__global__ void __launch_bounds__(256)
+index_key_compress_kernel(const T* __restrict__ Ca, const T* __restrict__ Cb, const T* __restrict__ Za,
+                          const T* __restrict__ Zb, const float* __restrict__ Ba, const float* __restrict__ Bb,
+                          const T* __restrict__ pCb, const T* __restrict__ pZb, const int32_t* __restrict__ entry0,
+                          uint8_t* __restrict__ kI, void* __restrict__ kI_scale, int64_t n_max, int T_new, int d,
+                          unsigned* err) {
+  constexpr int VEC = Elem<T>::VEC;
+  const int b = blockIdx.y;
+  const int tpe = d / VEC;                                // threads per entry
+  const int n_blk = T_new / 4;
+  const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= (int64_t)n_blk * tpe) return;               // whole lane groups leave together
+  const int j = (int)(gid / tpe);
+  const int g = (int)(gid % tpe);
+  const int c0 = g * VEC;
+  const int lane = threadIdx.x & 31;
+  const unsigned gmask = tpe == 32 ? 0xFFFFFFFFu : ((1u << tpe) - 1u) << (lane & ~(tpe - 1));
+  float x[VEC];
+  const int e = pool_m4<T>(Ca, Cb, Za, Zb, Ba, Bb, pCb, pZb, entry0, n_max, T_new, d, b, j, c0, x, err);
+  if (e < 0) return;                                      // the same for the whole group
+  const size_t row = (size_t)b * n_max + e;
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < VEC; ++i) amax = fmaxf(amax, fabsf(x[i]));
+  if (FMT == CSA_IFMT_E4M3) {
+    for (int o = tpe >> 1; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, o));
+    const float scale = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+    uint32_t w[VEC / 4];
+#pragma unroll
+    for (int q = 0; q < VEC / 4; ++q)
+      w[q] = e4m3x2_rn(__fdiv_rn(x[4 * q], scale), __fdiv_rn(x[4 * q + 1], scale)) |
+             (e4m3x2_rn(__fdiv_rn(x[4 * q + 2], scale), __fdiv_rn(x[4 * q + 3], scale)) << 16);
+    uint8_t* dst = kI + row * d + c0;
+    if (VEC == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[VEC / 4 - 1]);
+    else *reinterpret_cast<uint32_t*>(dst) = w[0];
+    if (g == 0) reinterpret_cast<float*>(kI_scale)[row] = scale;
+  } else {
+    constexpr int TPB = 32 / VEC;                         // threads per 32-component block
+    for (int o = TPB >> 1; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, o));
+    const int ex = mx_exponent(amax);
+    const float inv = __uint_as_float((uint32_t)(127 - ex) << 23);     // 2^-ex, exact: -ex in [-126, 127]
+    uint32_t w = 0;
+#pragma unroll
+    for (int q = 0; q < VEC / 2; ++q) w |= e2m1x2_rn(x[2 * q] * inv, x[2 * q + 1] * inv) << (8 * q);
+    uint8_t* dst = kI + row * (d / 2) + c0 / 2;
+    if (VEC == 8) *reinterpret_cast<uint32_t*>(dst) = w;
+    else *reinterpret_cast<uint16_t*>(dst) = (uint16_t)w;
+    if (g % TPB == 0) reinterpret_cast<uint8_t*>(kI_scale)[row * (d / 32) + c0 / 32] = (uint8_t)(ex + 127);
+  }
 }
 
 // One CTA per (entry, slab of 8*VEC components, batch): 8 component groups x 32 token lanes.
@@ -270,6 +381,31 @@ cudaError_t launch_csa_compress(const void* Ca, const void* Cb, const void* Za, 
                                                      (const float*)Zb, Ba, Bb, (const float*)pCb,
                                                      (const float*)pZb, entry0, (float*)cache, n_max,
                                                      T_new, d, m, err);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_index_key_compress(const void* Ca, const void* Cb, const void* Za, const void* Zb,
+                                     const float* Ba, const float* Bb, const void* pCb, const void* pZb,
+                                     const int32_t* entry0, void* kI, void* kI_scale, int64_t n_max, int B,
+                                     int T_new, int d, int dtype, int ifmt, cudaStream_t st, unsigned* err) {
+  const int vec = dtype == CSA_BF16 ? 8 : 4;
+  const int64_t work = (int64_t)(T_new / 4) * (d / vec);
+  const int threads = work < 256 ? (int)((work + 31) / 32 * 32) : 256;
+  dim3 grid((unsigned)((work + threads - 1) / threads), B);
+  auto go = [&](auto tag, auto fmt) {
+    using T = decltype(tag);
+    note_launch();
+    index_key_compress_kernel<T, decltype(fmt)::value><<<grid, threads, 0, st>>>(
+        (const T*)Ca, (const T*)Cb, (const T*)Za, (const T*)Zb, Ba, Bb, (const T*)pCb, (const T*)pZb, entry0,
+        (uint8_t*)kI, kI_scale, n_max, T_new, d, err);
+  };
+  using E4 = std::integral_constant<int, CSA_IFMT_E4M3>;
+  using MX = std::integral_constant<int, CSA_IFMT_MXFP4>;
+  if (dtype == CSA_BF16) {
+    if (ifmt == CSA_IFMT_E4M3) go(__nv_bfloat16(), E4()); else go(__nv_bfloat16(), MX());
+  } else {
+    if (ifmt == CSA_IFMT_E4M3) go(float(), E4()); else go(float(), MX());
   }
   return cudaGetLastError();
 }

@@ -36,7 +36,7 @@ import torch
 
 __all__ = [
     "WORKLOADS", "make_workload", "Workload",
-    "bf16_bits", "fp32", "quant_e4m3_rows", "quant_mxfp4_rows",
+    "bf16_bits", "fp32", "quant_e4m3_rows", "quant_mxfp4_rows", "index_key_inputs",
 ]
 
 # --------------------------------------------------------------------------
@@ -150,6 +150,22 @@ def _csa_compressor_inputs(r: _Rng, B, T_new, d, m, gate_std, to_store):
     t["Ba"] = fp32(r.normal((m, d), 0.1))
     t["Bb"] = fp32(r.normal((m, d), 0.1))
     return t
+
+
+def index_key_inputs(seed: int, B: int, T_new: int, d_I: int = 128, dtype: str = "bf16",
+                     gate_std: float = 2.0, spread: float = 0.0) -> dict:
+    """Indexer activations and gates for the indexer-key producer (the CSA pooling with
+    m = 4 over width d_I): Ca, Cb, prev_Cb ~ N(0, 1) times a per-token magnitude
+    2^u, u ~ U(-spread, spread) (spread = 0: plain N(0, 1)); Za, Zb, prev_Zb ~ N(0,
+    gate_std); Ba, Bb ~ N(0, 0.1) fp32.  Stored as bf16 bits or fp32 (``dtype``)."""
+    r = _Rng(seed)
+    to_store = bf16_bits if dtype == "bf16" else fp32
+    t = _csa_compressor_inputs(r, B, T_new, d_I, 4, gate_std, lambda x: x)
+    if spread > 0:
+        for name in ("Ca", "Cb", "prev_Cb"):
+            x = t[name]
+            t[name] = x * torch.exp2((r.uniform(x.shape[:-1] + (1,)) * 2 - 1) * spread)
+    return {k: (to_store(v) if isinstance(v, torch.Tensor) else v) for k, v in t.items()}
 
 
 def make_workload(i: int, seed: int | None = None, scale: dict | None = None) -> Workload:

@@ -125,6 +125,40 @@ csa_status hca_compress(const void* C, const void* Z, const float* bias,
                         int B, int T_new, int d, int m_prime, int dtype, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * index_key_compress — the indexer keys of the entries a chunk completes
+ * ("FP4 с учётом квантования": the indexer's Q·K activations are cached and
+ * multiplied in FP4, MXFP4 with 1x32 tiles; the keys belong to the compressed
+ * entries, so they come from the CSA step-1 pooling of the indexer activations).
+ *
+ * The pooling is csa_compress's with m = 4, over indexer activations of width
+ * d_I; the pooled fp32 row is quantised in the same kernel to the format that
+ * lightning_index reads:
+ *   CSA_IFMT_E4M3:  scale = amax(|row|)/448 (1 for an all-zero row), one fp32
+ *                   per row; code = round-to-nearest-even(x / scale) in e4m3;
+ *   CSA_IFMT_MXFP4: per 32 components e = the smallest integer with
+ *                   amax <= 6 * 2^e (clamped to [-127, 127]; -127 for zeros),
+ *                   scale byte e + 127; code = RNE e2m1 of x * 2^-e.
+ * Decisions are made on the fp32 pooled values; a value that rounds to zero is
+ * written as +0 (code 0).
+ *
+ *   Ca, Cb, Za, Zb   device [B, T_new, d_I] dtype (indexer activations and gates)
+ *   Ba, Bb           device [4, d_I] fp32 positional biases
+ *   prev_Cb, prev_Zb device [B, 4, d_I] dtype (as in csa_compress)
+ *   entry0           device [B] int32: index of the chunk's first entry
+ *   kI               device [B, n_max, d_I] bytes (E4M3) or [B, n_max, d_I/2] (MXFP4)
+ *   kI_scale         device [B, n_max] fp32 (E4M3) or [B, n_max, d_I/32] bytes (MXFP4)
+ *                    rows entry0[b] .. entry0[b]+T_new/4-1 are written; an entry
+ *                    outside [0, n_max) is skipped and sets CSA_DEVERR_ENTRY
+ * Supported: m == 4 (CSA_ERR_UNSUPPORTED otherwise), d_I in {32, 64, 128} (and
+ * 256 for bf16).  All pointers 16-byte aligned.
+ * ------------------------------------------------------------------------- */
+csa_status index_key_compress(const void* Ca, const void* Cb, const void* Za, const void* Zb,
+                              const float* Ba, const float* Bb,
+                              const void* prev_Cb, const void* prev_Zb,
+                              const int32_t* entry0, void* kI, void* kI_scale, int64_t n_max,
+                              int B, int T_new, int d_I, int m, int dtype, int ifmt, void* stream);
+
+/* ---------------------------------------------------------------------------
  * lightning_index — indexer scores and top-k selection of compressed entries
  * ("Гибридное внимание: CSA и HCA", CSA step 2: the DSA lightning indexer
  * scores I[t,s] with a ReLU and keeps the top-k compressed blocks; FP4 Q·K

@@ -23,7 +23,7 @@ def declared_functions():
 def test_every_declared_symbol_is_exported():
     names = declared_functions()
     assert {"csa_compress", "hca_compress", "lightning_index", "topk_select", "sparse_attn_decode",
-            "sparse_attn_prefill", "hca_attn_decode", "hca_compress_attn_decode"} <= set(names)
+            "sparse_attn_prefill", "hca_attn_decode", "hca_compress_attn_decode", "index_key_compress"} <= set(names)
     for n in names:
         assert hasattr(N.lib, n), n
 
@@ -62,6 +62,32 @@ def test_compress_validation():
     assert compress(m=17) == ERR_SHAPE
     assert compress(d=6) == ERR_SHAPE           # rows must stay 16-byte aligned
     assert compress(dtype=1, d=12) == ERR_SHAPE
+
+
+def index_keys(**kw):
+    a = dict(Ca=FAKE, Cb=FAKE, Za=FAKE, Zb=FAKE, Ba=FAKE, Bb=FAKE, pCb=FAKE, pZb=FAKE, e0=FAKE, kI=FAKE, ks=FAKE,
+             n_max=64, B=1, T=16, d=128, m=4, dtype=1, ifmt=1)
+    a.update(kw)
+    return N.lib.index_key_compress(a["Ca"], a["Cb"], a["Za"], a["Zb"], a["Ba"], a["Bb"], a["pCb"], a["pZb"],
+                                    a["e0"], a["kI"], a["ks"], a["n_max"], a["B"], a["T"], a["d"], a["m"],
+                                    a["dtype"], a["ifmt"], None)
+
+
+def test_index_key_compress_validation():
+    before = N.lib.csa_launch_count()
+    assert index_keys(kI=None) == ERR_NULL
+    assert index_keys(ks=None) == ERR_NULL
+    assert index_keys(e0=None) == ERR_NULL
+    assert index_keys(ks=FAKE + 4) == ERR_ALIGN
+    assert index_keys(ifmt=0) == ERR_DTYPE          # keys are quantised: E4M3 or MXFP4 only
+    assert index_keys(ifmt=3) == ERR_DTYPE
+    assert index_keys(dtype=2) == ERR_DTYPE
+    assert index_keys(m=8) == ERR_UNSUP             # the CSA rate only
+    assert index_keys(T=18) == ERR_SHAPE
+    assert index_keys(d=96) == ERR_UNSUP            # threads of an entry: a power of two within a warp
+    assert index_keys(d=256, dtype=0) == ERR_UNSUP
+    assert index_keys(B=0) == ERR_SHAPE
+    assert N.lib.csa_launch_count() == before
 
 
 def test_indexer_validation():
