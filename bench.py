@@ -391,6 +391,7 @@ def run_ours(args, wid):
         achieved = ab[dom] / (dom_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak, "peak_source": src, "traffic": TRAFFIC.get((args.workload, dom))}
+    extra = measure_index_keys(wid, D, csa, l2_flush, hbm_peak, src)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -403,6 +404,8 @@ def run_ours(args, wid):
         "gpu_launches": launches_step * args.steps,
         "clocks": summarize_clocks(clock_lines),
     }
+    if extra:
+        line["next_rows"] = extra
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(wid, wl)
     if rank == 0:
@@ -410,6 +413,58 @@ def run_ours(args, wid):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def measure_index_keys(wid, D, csa, l2_flush, hbm_peak, peak_src, reps=20):
+    """The indexer-key producer for the entries this workload's step completes (one per
+    sequence in decode, Tq/4 in the prefill chunk), timed alone: one call captured in a
+    CUDA graph, L2 flushed before each replay, CUDA events around it.  Not part of the
+    step's timed quantity."""
+    import numpy as np
+    import torch
+    import csa_inputs as CI
+    if wid not in (1, 3, 4):
+        return None
+    B, T_new, d_I = D["B"], (D["Tq"] if wid == 3 else D["m"]), D["dI"]
+    mx = D["ifmt"] == "mxfp4"
+    t = CI.index_key_inputs(977, B, T_new, d_I, "bf16")
+    dev = {k: (torch.from_numpy(v).cuda() if v.dtype == np.float32
+               else torch.from_numpy(v.view(np.int16)).cuda().view(torch.bfloat16)) for k, v in t.items()}
+    n_max = D["n_max"]
+    e0 = torch.full((B,), D["entry0"], dtype=torch.int32, device="cuda")
+    kI = torch.empty((B, n_max, d_I // 2 if mx else d_I), dtype=torch.uint8, device="cuda")
+    ks = (torch.empty((B, n_max, d_I // 32), dtype=torch.uint8, device="cuda") if mx
+          else torch.empty((B, n_max), dtype=torch.float32, device="cuda"))
+    fmt = csa.CSA_IFMT_MXFP4 if mx else csa.CSA_IFMT_E4M3
+
+    def call():
+        csa.index_key_compress(dev["Ca"], dev["Cb"], dev["Za"], dev["Zb"], dev["Ba"], dev["Bb"], dev["prev_Cb"],
+                               dev["prev_Zb"], e0, kI, ks, fmt)
+
+    for _ in range(3):
+        call()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call()
+    ms = []
+    for _ in range(reps):
+        l2_flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        ms.append((a, b))
+    torch.cuda.synchronize()
+    us = float(np.mean([a.elapsed_time(b) for a, b in ms])) * 1e3
+    n = B * (T_new // 4)
+    # algorithmic bytes: every source row read once (4 series of the chunk plus the two
+    # b-series rows before it), biases, and the key rows written
+    nbytes = (4 * B * T_new * d_I + 2 * B * 4 * d_I) * 2 + 2 * 4 * d_I * 4 + n * ((d_I // 2 + d_I // 32) if mx else (d_I + 4))
+    gbs = nbytes / (us * 1e-6) / 1e9
+    return {"index_key_compress": {"entries": n, "format": D["ifmt"], "us": us, "bytes": nbytes,
+                                   "achieved_gbs": gbs, "frac": gbs / hbm_peak, "peak_source": peak_src,
+                                   "l2": "flushed before every call",
+                                   "timing": "CUDA events around one graph replay of the call (launch included)"}}
 
 
 def measure_e2e(args, wid, wl, T, D, csa, steps):

@@ -390,9 +390,12 @@ cudaError_t launch_index_key_compress(const void* Ca, const void* Cb, const void
                                      const int32_t* entry0, void* kI, void* kI_scale, int64_t n_max, int B,
                                      int T_new, int d, int dtype, int ifmt, cudaStream_t st, unsigned* err) {
   const int vec = dtype == CSA_BF16 ? 8 : 4;
-  const int64_t work = (int64_t)(T_new / 4) * (d / vec);
-  const int threads = work < 256 ? (int)((work + 31) / 32 * 32) : 256;
-  dim3 grid((unsigned)((work + threads - 1) / threads), B);
+  const int64_t work = (int64_t)(T_new / 4) * (d / vec) * B;
+  // every thread waits for one round trip of its 16 source loads: spread small grids over
+  // more SMs with smaller CTAs
+  const int64_t per_seq = work / B;
+  const int threads = per_seq < 256 ? (int)((per_seq + 31) / 32 * 32) : (work < 256LL * num_sms() ? 128 : 256);
+  dim3 grid((unsigned)((per_seq + threads - 1) / threads), B);
   auto go = [&](auto tag, auto fmt) {
     using T = decltype(tag);
     note_launch();
