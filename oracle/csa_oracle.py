@@ -362,6 +362,14 @@ def topk(scores_row, n_elig, k):
     return out
 
 
+def topk_bf16(scores_row, n_elig, k):
+    """Top-k over bf16 keys ([P1] "FP4 с учётом квантования": the indexer's scores are
+    converted from FP32 to BF16 before the selection): each exact score rounded to the
+    nearest bf16 value (ties to even), then topk over those keys, so scores closer than
+    the bf16 resolution tie and the lower index wins."""
+    return topk(round_to_bf16(np.asarray(scores_row[:int(n_elig)], dtype=np.float64)), n_elig, k)
+
+
 # ---------------------------------------------------------------------------
 # a5 / a6: attention over compressed entries + window + sink  ([P1] CSA step 3,
 # HCA paragraph and sliding window; [P4] MLA latent, SWA, attention sink)

@@ -277,6 +277,20 @@ def test_topk_equals_full_sort():
         assert got.tolist() == exp
 
 
+def test_topk_bf16_rounds_before_selecting():
+    """Scores 1 + 2^-9 and 1 + 2^-8 round to the bf16 key 1.0 (ulp 2^-7), so they tie with
+    an exact 1.0 and the lowest indices win; 1 + 3 * 2^-8 rounds up to 1 + 2^-7."""
+    s = np.array([1.0, 1.0 + 2.0 ** -8, 0.5, 1.0 + 2.0 ** -9, 1.0 + 3 * 2.0 ** -8, 0.25])
+    assert O.topk(s, 6, 2).tolist() == [1, 4]                # exact: the two largest
+    assert O.topk(s, 6, 3).tolist() == [1, 3, 4]
+    assert O.topk_bf16(s, 6, 2).tolist() == [0, 4]           # bf16: 1+3*2^-8 -> 1+2^-7, then ties at 1.0
+    assert O.topk_bf16(s, 6, 3).tolist() == [0, 1, 4]
+    assert O.topk_bf16(s, 3, 5).tolist() == [0, 1, 2, -1, -1]
+    # keys already on the bf16 grid select exactly as topk does
+    g = O.round_to_bf16(np.random.default_rng(2).normal(size=300))
+    assert np.array_equal(O.topk_bf16(g, 300, 40), O.topk(g, 300, 40))
+
+
 def test_topk_invariant_to_positive_weight_scale():
     r = np.random.default_rng(11)
     q = r.standard_normal((2, 4, 8)); k = r.standard_normal((50, 8)); w = r.uniform(size=(2, 4))
