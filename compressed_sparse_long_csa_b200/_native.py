@@ -27,6 +27,7 @@ _SIGS = {
     "hca_compress": ([_vp] * 5 + [_i64, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
     "lightning_index_workspace_size": ([_i32, _i32, _i64, _i32], _sz),
     "lightning_index": ([_vp] * 7 + [_i32, _i32, _i32, _i32, _i32, _i64, _i32, _i32, _vp, _vp, _vp, _sz, _vp], _i32),
+    "lightning_index_bf16": ([_vp] * 7 + [_i32, _i32, _i32, _i32, _i32, _i64, _i32, _i32, _vp, _vp, _sz, _vp], _i32),
     "topk_select_workspace_size": ([_i32, _i64, _i32], _sz),
     "topk_select": ([_vp, _i64, _vp, _i32, _i64, _i32, _vp, _vp, _sz, _vp], _i32),
     "attn_decode_workspace_size": ([_i32, _i32, _i32, _i64], _sz),
@@ -112,6 +113,17 @@ def lightning_index(qI, qI_scale, w, kI, kI_scale, n_entries, q_pos, k, ifmt, id
     _check(lib.lightning_index(_p(qI), _p(qI_scale), _p(w), _p(kI), _p(kI_scale), _p(n_entries), _p(q_pos), m,
                                B, Tq, H_I, d_I, n_max, k, ifmt, _p(idx_out), _p(score_out), _p(workspace),
                                workspace.numel() * workspace.element_size(), _stream(stream)), "lightning_index")
+
+
+def lightning_index_bf16(qI, qI_scale, w, kI, kI_scale, n_entries, q_pos, k, ifmt, idx_out, workspace, m=4,
+                         stream=None):
+    B, Tq, H_I = w.shape
+    n_max = kI.shape[1]
+    d_I = qI.shape[-1] * (2 if ifmt == CSA_IFMT_MXFP4 else 1)
+    _check(lib.lightning_index_bf16(_p(qI), _p(qI_scale), _p(w), _p(kI), _p(kI_scale), _p(n_entries), _p(q_pos), m,
+                                    B, Tq, H_I, d_I, n_max, k, ifmt, _p(idx_out), _p(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream)),
+           "lightning_index_bf16")
 
 
 def topk_select(scores, n_valid, k, idx_out, stream=None):

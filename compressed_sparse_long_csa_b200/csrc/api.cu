@@ -174,10 +174,11 @@ size_t lightning_index_workspace_size(int B, int Tq, int64_t n_max, int k) {
          round_up((size_t)B * Tq * 2 * sizeof(unsigned), 256);
 }
 
-csa_status lightning_index(const void* qI, const void* qI_scale, const float* w, const void* kI,
-                           const void* kI_scale, const int32_t* n_entries, const int32_t* q_pos, int m, int B,
-                           int Tq, int H_I, int d_I, int64_t n_max, int k, int ifmt, int32_t* idx_out,
-                           float* score_out, void* workspace, size_t ws_bytes, void* stream) {
+static csa_status run_lightning_index(const void* qI, const void* qI_scale, const float* w, const void* kI,
+                                      const void* kI_scale, const int32_t* n_entries, const int32_t* q_pos, int m,
+                                      int B, int Tq, int H_I, int d_I, int64_t n_max, int k, int ifmt,
+                                      int32_t* idx_out, float* score_out, void* workspace, size_t ws_bytes,
+                                      void* stream, bool bf16_scores) {
   REQUIRE(ifmt == CSA_IFMT_F32 || ifmt == CSA_IFMT_E4M3 || ifmt == CSA_IFMT_MXFP4, CSA_ERR_DTYPE);
   REQUIRE(B >= 1 && Tq >= 1 && (int64_t)B * Tq <= 65535 && H_I >= 1 && H_I <= 64 && m >= 1, CSA_ERR_SHAPE);
   REQUIRE(d_I == 32 || d_I == 64 || d_I == 128, CSA_ERR_SHAPE);
@@ -201,6 +202,7 @@ csa_status lightning_index(const void* qI, const void* qI_scale, const float* w,
   a.scores = (float*)workspace;
   a.knmax = (unsigned*)((char*)workspace + round_up((size_t)B * Tq * a.ld * sizeof(float), 256));
   a.idx_out = idx_out; a.score_out = score_out; a.err = err;
+  a.score_bf16 = bf16_scores ? 1 : 0;
   a.keyrange = a.knmax + round_up((size_t)B * sizeof(unsigned), 256) / sizeof(unsigned);
   cudaError_t e = cudaMemsetAsync(a.knmax, 0, round_up((size_t)B * sizeof(unsigned), 256) +
                                   (size_t)B * Tq * 2 * sizeof(unsigned), S(stream));
@@ -216,7 +218,29 @@ csa_status lightning_index(const void* qI, const void* qI_scale, const float* w,
     e = launch_indexer_scores_cuda_core(a, S(stream));
     if (e != cudaSuccess) return CSA_ERR_CUDA;
   }
+  if (bf16_scores) {
+    // the stored keys are the selection's keys: a plain exact top-k over them
+    RowCount rc;
+    rc.q_pos = q_pos; rc.n_entries = n_entries; rc.m = m; rc.Tq = Tq;
+    return cuda_status(launch_topk_select(a.scores, a.ld, rc, B * Tq, n_max, k, idx_out, S(stream), err));
+  }
   return cuda_status(launch_indexer_select(a, S(stream)));
+}
+
+csa_status lightning_index(const void* qI, const void* qI_scale, const float* w, const void* kI,
+                           const void* kI_scale, const int32_t* n_entries, const int32_t* q_pos, int m, int B,
+                           int Tq, int H_I, int d_I, int64_t n_max, int k, int ifmt, int32_t* idx_out,
+                           float* score_out, void* workspace, size_t ws_bytes, void* stream) {
+  return run_lightning_index(qI, qI_scale, w, kI, kI_scale, n_entries, q_pos, m, B, Tq, H_I, d_I, n_max, k, ifmt,
+                             idx_out, score_out, workspace, ws_bytes, stream, false);
+}
+
+csa_status lightning_index_bf16(const void* qI, const void* qI_scale, const float* w, const void* kI,
+                                const void* kI_scale, const int32_t* n_entries, const int32_t* q_pos, int m, int B,
+                                int Tq, int H_I, int d_I, int64_t n_max, int k, int ifmt, int32_t* idx_out,
+                                void* workspace, size_t ws_bytes, void* stream) {
+  return run_lightning_index(qI, qI_scale, w, kI, kI_scale, n_entries, q_pos, m, B, Tq, H_I, d_I, n_max, k, ifmt,
+                             idx_out, nullptr, workspace, ws_bytes, stream, true);
 }
 
 size_t topk_select_workspace_size(int R, int64_t n, int k) {
@@ -231,7 +255,9 @@ csa_status topk_select(const float* scores, int64_t ld, const int32_t* n_valid, 
   REQUIRE_PTR(scores); REQUIRE_PTR(idx_out);
   unsigned* err = device_error_word();
   REQUIRE(err, CSA_ERR_CUDA);
-  return cuda_status(launch_topk_select(scores, ld, n_valid, R, n, k, idx_out, S(stream), err));
+  RowCount rc;
+  rc.n_valid = n_valid;
+  return cuda_status(launch_topk_select(scores, ld, rc, R, n, k, idx_out, S(stream), err));
 }
 
 // ----------------------------------------------------------------------------- attention

@@ -112,6 +112,7 @@ indexer_scores_cuda_core(IndexerArgs a) {
     }
     score = fmaf(wsh[j], fmaxf(D, 0.f), score);
   }
+  if (a.score_bf16) score = round_bf16(score);
   if (has) a.scores[(size_t)row * a.ld + s] = score;
   record_key_range(a.keyrange, row, score, has);
 }

@@ -25,7 +25,33 @@ struct IndexerArgs {
   float* score_out;           // [B*Tq, k] or null
   unsigned* err;
   float eps_dot;              // bound on |fp32 dot - exact| / (||q|| ||k||) of the scoring path
+  int score_bf16;             // 1: scores are rounded to bf16 before they are stored (lightning_index_bf16)
 };
+
+// Entries of one selection row: n_valid[row] (topk_select), else the indexer's
+// eligibility min(n_entries[b], (q_pos[row] + 1) / m) when q_pos is set, else n_cap;
+// always clamped to [0, n_cap].
+struct RowCount {
+  const int32_t* n_valid = nullptr;
+  const int32_t* q_pos = nullptr;
+  const int32_t* n_entries = nullptr;
+  int m = 1, Tq = 1;
+  __device__ __forceinline__ int operator()(int row, int64_t n_cap) const {
+    int n = (int)(n_cap < 0x7fffffff ? n_cap : 0x7fffffff);
+    if (n_valid) {
+      n = n_valid[row];
+    } else if (q_pos) {
+      const int pos = q_pos[row];
+      const int ne = pos < 0 ? 0 : (pos + 1) / m;
+      const int nb = n_entries[row / Tq];
+      n = ne < nb ? ne : nb;
+    }
+    if ((int64_t)n > n_cap) n = (int)n_cap;
+    return n < 0 ? 0 : n;
+  }
+};
+
+__device__ __forceinline__ float round_bf16(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
 
 // Number of entries visible to query row `row` (= b*Tq + t): all m sources <= pos.
 __device__ __forceinline__ int row_eligible(const IndexerArgs& a, int row) {
@@ -75,11 +101,11 @@ __device__ __forceinline__ void record_key_range(unsigned* keyrange, int row, fl
 cudaError_t launch_indexer_scores_cuda_core(const IndexerArgs& a, cudaStream_t st);
 cudaError_t launch_indexer_scores_tc(IndexerArgs& a, cudaStream_t st, bool* used);   // sets a.eps_dot
 cudaError_t launch_indexer_select(const IndexerArgs& a, cudaStream_t st);
-cudaError_t launch_topk_select(const float* scores, int64_t ld, const int32_t* n_valid, int R, int64_t n,
+cudaError_t launch_topk_select(const float* scores, int64_t ld, RowCount rc, int R, int64_t n,
                                int k, int32_t* idx_out, cudaStream_t st, unsigned* err);
 // Cluster paths (select.cu); cudaErrorNotSupported when a row does not fit one cluster.
 cudaError_t launch_indexer_select_cluster(const IndexerArgs& a, cudaStream_t st);
-cudaError_t launch_topk_select_cluster(const float* scores, int64_t ld, const int32_t* n_valid, int R, int64_t n,
+cudaError_t launch_topk_select_cluster(const float* scores, int64_t ld, RowCount rc, int R, int64_t n,
                                        int k, int32_t* idx_out, cudaStream_t st);
 
 }  // namespace csa

@@ -222,9 +222,10 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         const float val = (part[0] + part[1]) + (part[2] + part[3]);
         const bool valid = s < sm.n_elig[g];
         if (valid) {
-          a.scores[(size_t)sm.row[g] * a.ld + s] = val * sk;
+          const float sc = a.score_bf16 ? round_bf16(val * sk) : val * sk;
+          a.scores[(size_t)sm.row[g] * a.ld + s] = sc;
           kmax = fmaxf(kmax, sk);
-          kr[g].add(val * sk);
+          kr[g].add(sc);
         }
       }
       tc::fence_before_sync();
@@ -463,7 +464,8 @@ indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           part[3] = fmaf(w4[u].w, fmaxf(__uint_as_float(v[4 * u + 3]), 0.f), part[3]);
         }
       }
-      const float val = (part[0] + part[1]) + (part[2] + part[3]);
+      const float val = a.score_bf16 ? round_bf16((part[0] + part[1]) + (part[2] + part[3]))
+                                     : (part[0] + part[1]) + (part[2] + part[3]);
       if (valid) {
         a.scores[(size_t)row * a.ld + s] = val;
         kr.add(val);

@@ -331,7 +331,7 @@ __device__ __forceinline__ int sl_write(SelFixed& sh, const uint32_t* sel, int n
 
 // ------------------------------------------------------------------ plain top-k
 __global__ void __launch_bounds__(SL_T, 1)
-topk_cluster_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_valid, int64_t n_cap,
+topk_cluster_kernel(const float* __restrict__ scores, int64_t ld, RowCount rc, int64_t n_cap,
                     int k, int32_t* __restrict__ idx_out, int chunk, int vec) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   SelFixed& sh = *reinterpret_cast<SelFixed*>(smem_raw);
@@ -341,9 +341,7 @@ topk_cluster_kernel(const float* __restrict__ scores, int64_t ld, const int32_t*
   const int row = blockIdx.x / C;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   tc::griddep_wait();                                      // every input may come from the previous kernel
-  int n = n_valid ? n_valid[row] : (int)n_cap;
-  if ((int64_t)n > n_cap) n = (int)n_cap;
-  if (n < 0) n = 0;
+  const int n = rc(row, n_cap);
   int32_t* out = idx_out + (size_t)row * k;
   if (n <= k) {
     if (r == 0)
@@ -893,12 +891,12 @@ cudaError_t launch_indexer_select_cluster(const IndexerArgs& a, cudaStream_t st)
   return sl_launch(indexer_select_cluster_kernel<CSA_IFMT_F32>, rows, C, SL_FIXED + region, st, a, chunk);
 }
 
-cudaError_t launch_topk_select_cluster(const float* scores, int64_t ld, const int32_t* n_valid, int R, int64_t n,
+cudaError_t launch_topk_select_cluster(const float* scores, int64_t ld, RowCount rc, int R, int64_t n,
                                        int k, int32_t* idx_out, cudaStream_t st) {
   int C, chunk;
   if (!sl_plan(n, R, &C, &chunk) || (int64_t)R * C > 0x7fffffffLL) return cudaErrorNotSupported;
   const int vec = (ld % 4 == 0) && (((uintptr_t)scores & 15) == 0);
-  return sl_launch(topk_cluster_kernel, R, C, SL_FIXED + (size_t)chunk * 4, st, scores, ld, n_valid, n, k, idx_out,
+  return sl_launch(topk_cluster_kernel, R, C, SL_FIXED + (size_t)chunk * 4, st, scores, ld, rc, n, k, idx_out,
                    chunk, vec);
 }
 

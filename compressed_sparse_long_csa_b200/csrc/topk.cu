@@ -285,15 +285,13 @@ __device__ void topk_select_global_row(TopkShared& sh, const float* S, int n, in
 }
 
 __global__ void __launch_bounds__(TK_THREADS)
-topk_select_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_valid,
-                   int64_t n_cap, int k, int32_t* __restrict__ idx_out) {
+topk_select_kernel(const float* __restrict__ scores, int64_t ld, RowCount rc, int64_t n_cap, int k,
+                   int32_t* __restrict__ idx_out) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   TopkShared& sh = *reinterpret_cast<TopkShared*>(smem_raw);
   const int row = blockIdx.x;
   const float* S = scores + (size_t)row * ld;
-  int n = n_valid ? n_valid[row] : (int)n_cap;
-  if ((int64_t)n > n_cap) n = (int)n_cap;
-  if (n < 0) n = 0;
+  const int n = rc(row, n_cap);
   int32_t* out = idx_out + (size_t)row * k;
   if (n <= k) {
     for (int i = threadIdx.x; i < k; i += blockDim.x) out[i] = i < n ? i : -1;
@@ -548,14 +546,14 @@ cudaError_t launch_indexer_select(const IndexerArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_topk_select(const float* scores, int64_t ld, const int32_t* n_valid, int R, int64_t n,
+cudaError_t launch_topk_select(const float* scores, int64_t ld, RowCount rc, int R, int64_t n,
                                int k, int32_t* idx_out, cudaStream_t st, unsigned* err) {
   (void)err;
-  const cudaError_t e = launch_topk_select_cluster(scores, ld, n_valid, R, n, k, idx_out, st);
+  const cudaError_t e = launch_topk_select_cluster(scores, ld, rc, R, n, k, idx_out, st);
   if (e != cudaErrorNotSupported) return e;
   set_smem_attr((const void*)topk_select_kernel);
   note_launch();
-  topk_select_kernel<<<R, TK_THREADS, sizeof(TopkShared), st>>>(scores, ld, n_valid, n, k, idx_out);
+  topk_select_kernel<<<R, TK_THREADS, sizeof(TopkShared), st>>>(scores, ld, rc, n, k, idx_out);
   return cudaGetLastError();
 }
 

@@ -194,6 +194,23 @@ csa_status lightning_index(const void* qI, const void* qI_scale, const float* w,
                            void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * lightning_index_bf16 — the same scores rounded to bf16 before the top-k
+ * ("FP4 с учётом квантования": the indexer's scores are converted from FP32 to
+ * BF16, which makes the top-k selection faster while keeping nearly all of the
+ * needed entries).  Not the exact selection of lightning_index: the k largest
+ * bf16 keys bf16(I[t,s]) are kept, ties to the lower index, so entries whose
+ * scores differ by less than the bf16 resolution are ordered by index.  I is
+ * the scoring kernel's fp32 score (rounded to nearest even); a score within
+ * the fp32 accumulation error of a bf16 rounding midpoint may round either way.
+ * Arguments, layouts, workspace and errors as lightning_index (no score_out).
+ * ------------------------------------------------------------------------- */
+csa_status lightning_index_bf16(const void* qI, const void* qI_scale, const float* w,
+                                const void* kI, const void* kI_scale,
+                                const int32_t* n_entries, const int32_t* q_pos, int m,
+                                int B, int Tq, int H_I, int d_I, int64_t n_max, int k, int ifmt,
+                                int32_t* idx_out, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * topk_select — exact top-k of fp32 scores (CSA step 2's selection on its own).
  *   scores   device [R, ld] fp32; row r has n_valid[r] valid leading entries
  *   idx_out  device [R, k] int32: the k largest, ties to the lower index,

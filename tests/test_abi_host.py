@@ -23,7 +23,8 @@ def declared_functions():
 def test_every_declared_symbol_is_exported():
     names = declared_functions()
     assert {"csa_compress", "hca_compress", "lightning_index", "topk_select", "sparse_attn_decode",
-            "sparse_attn_prefill", "hca_attn_decode", "hca_compress_attn_decode", "index_key_compress"} <= set(names)
+            "sparse_attn_prefill", "hca_attn_decode", "hca_compress_attn_decode", "index_key_compress",
+            "lightning_index_bf16"} <= set(names)
     for n in names:
         assert hasattr(N.lib, n), n
 
@@ -110,6 +111,24 @@ def test_indexer_validation():
     assert call(kI=FAKE + 4) == ERR_ALIGN
     need = N.lib.lightning_index_workspace_size(2, 3, 1000, 64)
     assert need >= 2 * 3 * 1000 * 4
+
+
+def test_indexer_bf16_validation():
+    def call(**kw):
+        a = dict(qI=FAKE, qs=FAKE, w=FAKE, kI=FAKE, ks=FAKE, ne=FAKE, qp=FAKE, m=4, B=1, Tq=1, HI=64, dI=128,
+                 n_max=1024, k=64, ifmt=1, idx=FAKE, ws=FAKE, wsb=1 << 30)
+        a.update(kw)
+        return N.lib.lightning_index_bf16(a["qI"], a["qs"], a["w"], a["kI"], a["ks"], a["ne"], a["qp"], a["m"],
+                                          a["B"], a["Tq"], a["HI"], a["dI"], a["n_max"], a["k"], a["ifmt"], a["idx"],
+                                          a["ws"], a["wsb"], None)
+    before = N.lib.csa_launch_count()
+    assert call(ifmt=9) == ERR_DTYPE
+    assert call(k=0) == ERR_SHAPE
+    assert call(idx=None) == ERR_NULL
+    assert call(ks=None) == ERR_NULL
+    assert call(wsb=16) == ERR_WS
+    assert call(kI=FAKE + 4) == ERR_ALIGN
+    assert N.lib.csa_launch_count() == before
 
 
 def test_attention_validation():
