@@ -392,6 +392,9 @@ def run_ours(args, wid):
         roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak, "peak_source": src, "traffic": TRAFFIC.get((args.workload, dom))}
     extra = measure_index_keys(wid, D, csa, l2_flush, hbm_peak, src)
+    bf = measure_bf16_index(wid, D, T, csa, steps, l2_flush, float(mean_ms[comp.index("indexer")]))
+    if bf:
+        extra = dict(extra or {}, **bf)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -465,6 +468,45 @@ def measure_index_keys(wid, D, csa, l2_flush, hbm_peak, peak_src, reps=20):
                                    "achieved_gbs": gbs, "frac": gbs / hbm_peak, "peak_source": peak_src,
                                    "l2": "flushed before every call",
                                    "timing": "CUDA events around one graph replay of the call (launch included)"}}
+
+
+def measure_bf16_index(wid, D, T, csa, steps, l2_flush, exact_ms, reps=20):
+    """lightning_index_bf16 on this workload's indexer inputs, timed alone like the
+    per-call breakdown (one graph replay after an L2 flush), and its recall against the
+    exact selection of the same inputs (the step's own index output)."""
+    import numpy as np
+    import torch
+    if wid not in (1, 3, 4):
+        return None
+    exact = T["idx"].clone()
+    idx = torch.empty_like(T["idx"])
+    ws = torch.empty_like(T["iws"])
+
+    def call():
+        csa.lightning_index_bf16(T["qI"], T.get("qI_scale"), T["w"], T["kI"], T.get("kI_scale"), T["n_entries"],
+                                 T["q_pos"], D["k"], steps._ifmt(D), idx, ws, m=D["m"])
+
+    for _ in range(3):
+        call()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call()
+    evs = []
+    for _ in range(reps):
+        l2_flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    us = float(np.mean([a.elapsed_time(b) for a, b in evs])) * 1e3
+    e, f = exact.cpu().numpy().reshape(-1, D["k"]), idx.cpu().numpy().reshape(-1, D["k"])
+    hit = sum(np.intersect1d(f[r][f[r] >= 0], e[r][e[r] >= 0]).size for r in range(e.shape[0]))
+    recall = hit / max(int((e >= 0).sum()), 1)
+    return {"lightning_index_bf16": {"us": us, "exact_us": exact_ms * 1e3, "speedup": exact_ms * 1e3 / us,
+                                     "recall_vs_exact": recall, "l2": "flushed before every call",
+                                     "timing": "CUDA events around one graph replay of the call (launch included)"}}
 
 
 def measure_e2e(args, wid, wl, T, D, csa, steps):
