@@ -36,7 +36,7 @@ import torch
 
 __all__ = [
     "WORKLOADS", "make_workload", "Workload",
-    "bf16_bits", "fp32", "quant_e4m3_rows", "quant_mxfp4_rows", "index_key_inputs",
+    "bf16_bits", "fp32", "quant_e4m3_rows", "quant_mxfp4_rows", "index_key_inputs", "out_proj_inputs",
 ]
 
 # --------------------------------------------------------------------------
@@ -166,6 +166,19 @@ def index_key_inputs(seed: int, B: int, T_new: int, d_I: int = 128, dtype: str =
             x = t[name]
             t[name] = x * torch.exp2((r.uniform(x.shape[:-1] + (1,)) * 2 - 1) * spread)
     return {k: (to_store(v) if isinstance(v, torch.Tensor) else v) for k, v in t.items()}
+
+
+def out_proj_inputs(seed: int, T: int, H: int = 128, dv: int = 512, g: int = 16, d_mid: int = 1024,
+                    d: int = 7168) -> dict:
+    """Inputs of the grouped output projection, stored as bf16 bits: head outputs
+    o [T, H, dv] ~ N(0, 1), W1 [g*d_mid, (H/g)*dv] ~ N(0, 1/((H/g)*dv)) and
+    W2 [d, g*d_mid] ~ N(0, 1/(g*d_mid)) (random initialisation of that scale keeps the
+    outputs near unit size)."""
+    r = _Rng(seed)
+    k1, k2 = (H // g) * dv, g * d_mid
+    return {"o": bf16_bits(r.normal((T, H, dv))),
+            "W1": bf16_bits(r.normal((g * d_mid, k1), 1.0 / math.sqrt(k1))),
+            "W2": bf16_bits(r.normal((d, k2), 1.0 / math.sqrt(k2)))}
 
 
 def make_workload(i: int, seed: int | None = None, scale: dict | None = None) -> Workload:

@@ -347,6 +347,30 @@ def index_key_compress(Ca, Cb, Za, Zb, Ba, Bb, fmt, prev_Cb=None, prev_Zb=None, 
 
 
 # ---------------------------------------------------------------------------
+# grouped output projection  ([P1] CSA step 4: the head outputs are split into g
+# groups, each group is projected to an intermediate width, and the concatenation is
+# projected to the hidden size; table "Конфигурации": g = 16, width 1024, d = 7168)
+# ---------------------------------------------------------------------------
+
+def grouped_out_proj(o, W1, W2, g, dtype="bf16"):
+    """o [T, H, dv], W1 [g*d_mid, (H/g)*dv], W2 [d, g*d_mid] (float64 values).
+
+    Group j holds heads j*H/g .. (j+1)*H/g - 1; its outputs, concatenated in head order,
+    are multiplied by rows j*d_mid .. (j+1)*d_mid - 1 of W1.  The intermediate u is stored
+    (rounded to the storage format) before W2 reads it.  Returns (u, y), both stored."""
+    T, H, dv = o.shape
+    d_mid = W1.shape[0] // g
+    hg = H // g
+    u = np.empty((T, g * d_mid), dtype=np.float64)
+    for j in range(g):
+        xj = o[:, j * hg:(j + 1) * hg, :].reshape(T, hg * dv)
+        u[:, j * d_mid:(j + 1) * d_mid] = xj @ W1[j * d_mid:(j + 1) * d_mid].T
+    u = store(u, dtype)
+    y = store(u @ W2.T, dtype)
+    return u, y
+
+
+# ---------------------------------------------------------------------------
 # a4: top-k  ([P1] CSA step 2; k from table "Конфигурации")
 # ---------------------------------------------------------------------------
 

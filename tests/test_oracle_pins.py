@@ -486,3 +486,40 @@ def test_index_key_compress_constant_rows_give_grid_codes():
                                                "mxfp4")
     assert np.all(scales == 129)                             # 2^2 covers 24 = 6 * 4
     assert np.array_equal(O.decode_e2m1_packed(codes), g + 0.0)
+
+
+# ---------------------------------------------------------------- grouped output projection
+# [P1] CSA step 4 and table "Конфигурации" (g groups, intermediate width, hidden size d).
+
+def test_grouped_projection_is_a_block_diagonal_projection():
+    """The grouped first stage is one projection by the block-diagonal matrix of the group
+    matrices (built by scipy's block_diag) of the flattened head outputs."""
+    from scipy.linalg import block_diag
+    r = np.random.default_rng(21)
+    T, H, dv, g, d_mid, d = 3, 8, 4, 4, 5, 6
+    o = r.normal(size=(T, H, dv))
+    W1 = r.normal(size=(g * d_mid, (H // g) * dv))
+    W2 = r.normal(size=(d, g * d_mid))
+    u, y = O.grouped_out_proj(o, W1, W2, g, dtype="f64")
+    Bd = block_diag(*[W1[j * d_mid:(j + 1) * d_mid] for j in range(g)])     # [g*d_mid, H*dv]
+    np.testing.assert_allclose(u, o.reshape(T, H * dv) @ Bd.T, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(y, (o.reshape(T, H * dv) @ Bd.T) @ W2.T, rtol=1e-12, atol=1e-12)
+
+
+def test_grouped_projection_locality_and_rounding():
+    """A change to one head reaches only its group's intermediate columns; u is rounded to
+    bf16 before the second stage reads it."""
+    r = np.random.default_rng(22)
+    T, H, dv, g, d_mid, d = 2, 8, 4, 4, 3, 5
+    o = r.normal(size=(T, H, dv))
+    W1 = r.normal(size=(g * d_mid, (H // g) * dv))
+    W2 = r.normal(size=(d, g * d_mid))
+    u0, _ = O.grouped_out_proj(o, W1, W2, g, dtype="f64")
+    o2 = o.copy()
+    o2[:, 5] += 1.0                                          # head 5 is in group 2 (heads 4, 5)
+    u1, _ = O.grouped_out_proj(o2, W1, W2, g, dtype="f64")
+    changed = np.nonzero(np.any(u1 != u0, axis=0))[0]
+    assert changed.tolist() == list(range(2 * d_mid, 3 * d_mid))
+    ub, yb = O.grouped_out_proj(o, W1, W2, g, dtype="bf16")
+    assert np.array_equal(ub, O.round_to_bf16(u0))
+    assert np.array_equal(yb, O.round_to_bf16(O.round_to_bf16(u0) @ W2.T))
