@@ -24,6 +24,8 @@ _SIGS = {
     "csa_launch_count": ([], C.c_uint64),
     "csa_compress": ([_vp] * 10 + [_i64, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
     "index_key_compress": ([_vp] * 11 + [_i64, _i32, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
+    "grouped_out_proj_workspace_size": ([_i32, _i32, _i32, _i32], _sz),
+    "grouped_out_proj": ([_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp], _i32),
     "hca_compress": ([_vp] * 5 + [_i64, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
     "lightning_index_workspace_size": ([_i32, _i32, _i64, _i32], _sz),
     "lightning_index": ([_vp] * 7 + [_i32, _i32, _i32, _i32, _i32, _i64, _i32, _i32, _vp, _vp, _vp, _sz, _vp], _i32),
@@ -93,6 +95,20 @@ def index_key_compress(Ca, Cb, Za, Zb, Ba, Bb, prev_Cb, prev_Zb, entry0, kI, kI_
     _check(lib.index_key_compress(_p(Ca), _p(Cb), _p(Za), _p(Zb), _p(Ba), _p(Bb), _p(prev_Cb), _p(prev_Zb),
                                   _p(entry0), _p(kI), _p(kI_scale), kI.shape[1], B, T_new, d_I, m,
                                   _dtype_code(Ca), ifmt, _stream(stream)), "index_key_compress")
+
+
+def grouped_out_proj_workspace_size(T, g, d_mid, d):
+    return lib.grouped_out_proj_workspace_size(T, g, d_mid, d)
+
+
+def grouped_out_proj(o, W1, W2, g, u, y, workspace=None, stream=None):
+    """o [T, H, dv] bf16; W1 [g*d_mid, (H/g)*dv]; W2 [d, g*d_mid]; writes u [T, g*d_mid], y [T, d]."""
+    T, H, dv = o.shape
+    d_mid = W1.shape[0] // g
+    d = W2.shape[0]
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib.grouped_out_proj(_p(o), T, H, dv, g, d_mid, _p(W1), _p(W2), d, _p(u), _p(y), _p(workspace), ws_bytes,
+                                _stream(stream)), "grouped_out_proj")
 
 
 def hca_compress(C_, Z, bias, entry0, cache, m_prime=128, stream=None):

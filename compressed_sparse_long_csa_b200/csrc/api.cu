@@ -14,6 +14,10 @@ cudaError_t launch_csa_compress(const void*, const void*, const void*, const voi
                                 int, cudaStream_t, unsigned*);
 cudaError_t launch_hca_compress(const void*, const void*, const float*, const int32_t*, void*, int64_t, int,
                                 int, int, int, int, cudaStream_t, unsigned*, int max_ctas);
+size_t out_proj_partial_elems(int T, int R_max);
+cudaError_t launch_grouped_out_proj(const void* o, int T, int H, int dv, int g, int d_mid, const void* W1,
+                                    const void* W2, int d, void* u, void* y, float* part, size_t part_elems,
+                                    cudaStream_t st, unsigned* err);
 cudaError_t launch_index_key_compress(const void*, const void*, const void*, const void*, const float*,
                                       const float*, const void*, const void*, const int32_t*, void*, void*, int64_t,
                                       int, int, int, int, int, cudaStream_t, unsigned*);
@@ -258,6 +262,29 @@ csa_status topk_select(const float* scores, int64_t ld, const int32_t* n_valid, 
   RowCount rc;
   rc.n_valid = n_valid;
   return cuda_status(launch_topk_select(scores, ld, rc, R, n, k, idx_out, S(stream), err));
+}
+
+// ----------------------------------------------------------------------------- output projection
+size_t grouped_out_proj_workspace_size(int T, int g, int d_mid, int d) {
+  if (T < 1 || T > 256 || g < 1 || d_mid < 1 || d < 1) return 0;
+  const int R = g * d_mid > d ? g * d_mid : d;
+  return out_proj_partial_elems(T, R) * sizeof(float);
+}
+
+csa_status grouped_out_proj(const void* o, int T, int H, int dv, int g, int d_mid, const void* W1, const void* W2,
+                            int d, void* u, void* y, void* workspace, size_t ws_bytes, void* stream) {
+  REQUIRE(T >= 1 && H >= 1 && dv >= 1 && g >= 1 && d_mid >= 1 && d >= 1, CSA_ERR_SHAPE);
+  REQUIRE(H % g == 0, CSA_ERR_SHAPE);
+  REQUIRE(((int64_t)(H / g) * dv) % 64 == 0 && d_mid % 128 == 0 && d % 128 == 0, CSA_ERR_UNSUPPORTED);
+  REQUIRE((int64_t)H * dv <= (1 << 20) && (int64_t)g * d_mid <= (1 << 20) && d <= (1 << 20), CSA_ERR_SHAPE);
+  REQUIRE((int64_t)T * H * dv < (1LL << 40), CSA_ERR_SHAPE);
+  REQUIRE_PTR(o); REQUIRE_PTR(W1); REQUIRE_PTR(W2); REQUIRE_PTR(u); REQUIRE_PTR(y);
+  if (workspace) REQUIRE(aligned16(workspace), CSA_ERR_ALIGN);
+  unsigned* err = device_error_word();
+  REQUIRE(err, CSA_ERR_CUDA);
+  const size_t part_elems = workspace ? ws_bytes / sizeof(float) : 0;
+  return cuda_status(launch_grouped_out_proj(o, T, H, dv, g, d_mid, W1, W2, d, u, y, (float*)workspace, part_elems,
+                                             S(stream), err));
 }
 
 // ----------------------------------------------------------------------------- attention

@@ -159,6 +159,32 @@ csa_status index_key_compress(const void* Ca, const void* Cb, const void* Za, co
                               int B, int T_new, int d_I, int m, int dtype, int ifmt, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * grouped_out_proj — the grouped output projection after the attention
+ * ("Гибридное внимание: CSA и HCA", CSA step 4: the n_h head outputs are split
+ * into g groups, each group is projected to an intermediate width d_mid, and the
+ * concatenation of the groups is projected to the hidden size d; table
+ * "Конфигурации": g = 16, d_mid = 1024, head size 512, d = 7168 for Pro).
+ *
+ *   u[t, j*d_mid + i] = sum_k W1[j*d_mid + i, k] * o[t, j*(H/g)*dv + k],  k < (H/g)*dv
+ *   y[t, r]           = sum_k W2[r, k] * u[t, k],                          k < g*d_mid
+ *
+ *   o   device [T, H, dv] bf16 (the attention output; o[t] read as one row of H*dv)
+ *   W1  device [g*d_mid, (H/g)*dv] bf16 (group j's matrix is rows j*d_mid ..)
+ *   W2  device [d, g*d_mid] bf16
+ *   u   device [T, g*d_mid] bf16, written (the intermediate, rounded to bf16)
+ *   y   device [T, d] bf16, written (fp32 accumulation, rounded to nearest even)
+ *   workspace  NULL, or >= grouped_out_proj_workspace_size(T, g, d_mid, d) bytes:
+ *              with it, batches of at most 256 tokens split the weight stream
+ *              over more SMs (fp32 partials added in a fixed order)
+ * Supported: (H/g)*dv % 64 == 0, d_mid % 128 == 0, d % 128 == 0
+ * (CSA_ERR_UNSUPPORTED otherwise).  All pointers 16-byte aligned.
+ * ------------------------------------------------------------------------- */
+size_t grouped_out_proj_workspace_size(int T, int g, int d_mid, int d);
+csa_status grouped_out_proj(const void* o, int T, int H, int dv, int g, int d_mid,
+                            const void* W1, const void* W2, int d, void* u, void* y,
+                            void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * lightning_index — indexer scores and top-k selection of compressed entries
  * ("Гибридное внимание: CSA и HCA", CSA step 2: the DSA lightning indexer
  * scores I[t,s] with a ReLU and keeps the top-k compressed blocks; FP4 Q·K

@@ -24,7 +24,7 @@ def test_every_declared_symbol_is_exported():
     names = declared_functions()
     assert {"csa_compress", "hca_compress", "lightning_index", "topk_select", "sparse_attn_decode",
             "sparse_attn_prefill", "hca_attn_decode", "hca_compress_attn_decode", "index_key_compress",
-            "lightning_index_bf16"} <= set(names)
+            "lightning_index_bf16", "grouped_out_proj"} <= set(names)
     for n in names:
         assert hasattr(N.lib, n), n
 
@@ -129,6 +129,26 @@ def test_indexer_bf16_validation():
     assert call(wsb=16) == ERR_WS
     assert call(kI=FAKE + 4) == ERR_ALIGN
     assert N.lib.csa_launch_count() == before
+
+
+def test_grouped_out_proj_validation():
+    def call(**kw):
+        a = dict(o=FAKE, T=16, H=128, dv=512, g=16, dm=1024, W1=FAKE, W2=FAKE, d=7168, u=FAKE, y=FAKE, ws=None, wsb=0)
+        a.update(kw)
+        return N.lib.grouped_out_proj(a["o"], a["T"], a["H"], a["dv"], a["g"], a["dm"], a["W1"], a["W2"], a["d"],
+                                      a["u"], a["y"], a["ws"], a["wsb"], None)
+    before = N.lib.csa_launch_count()
+    assert call(o=None) == ERR_NULL
+    assert call(y=FAKE + 2) == ERR_ALIGN
+    assert call(T=0) == ERR_SHAPE
+    assert call(g=3) == ERR_SHAPE                   # heads split evenly into groups
+    assert call(dm=1000) == ERR_UNSUP               # intermediate rows in whole 128-row tiles
+    assert call(d=7000) == ERR_UNSUP
+    assert call(dv=4, H=16, g=16) == ERR_UNSUP      # K of a group: whole 64-element stages
+    assert call(ws=FAKE + 8, wsb=64) == ERR_ALIGN
+    assert N.lib.csa_launch_count() == before
+    assert N.lib.grouped_out_proj_workspace_size(16, 16, 1024, 7168) == 8 * 16 * 16384 * 4
+    assert N.lib.grouped_out_proj_workspace_size(4096, 16, 1024, 7168) == 0   # large batches need no split
 
 
 def test_attention_validation():
