@@ -395,6 +395,7 @@ def run_ours(args, wid):
     bf = measure_bf16_index(wid, D, T, csa, steps, l2_flush, float(mean_ms[comp.index("indexer")]))
     if bf:
         extra = dict(extra or {}, **bf)
+    extra = dict(extra or {}, **measure_out_proj(D, T, csa, l2_flush, hbm_peak, bf16_peak, src))
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -507,6 +508,56 @@ def measure_bf16_index(wid, D, T, csa, steps, l2_flush, exact_ms, reps=20):
     return {"lightning_index_bf16": {"us": us, "exact_us": exact_ms * 1e3, "speedup": exact_ms * 1e3 / us,
                                      "recall_vs_exact": recall, "l2": "flushed before every call",
                                      "timing": "CUDA events around one graph replay of the call (launch included)"}}
+
+
+def measure_out_proj(D, T, csa, l2_flush, hbm_peak, bf16_peak, peak_src, reps=10):
+    """The grouped output projection (16 groups -> 1024 -> 7168, the Pro sizes) applied to
+    this step's attention output, timed alone (one graph replay after an L2 flush).  Few
+    tokens stream 369 MB of weights (HBM-bound); a prefill chunk is tensor-bound."""
+    import numpy as np
+    import torch
+    import csa_inputs as CI
+    H, dv, g, d_mid, d = D["H"], D["dv"], 16, 1024, 7168
+    o = T["out"].reshape(-1, H, dv)
+    n_tok = o.shape[0]
+    x = CI.out_proj_inputs(4242, 1, H, dv, g, d_mid, d)
+    W1 = torch.from_numpy(x["W1"].view(np.int16)).cuda().view(torch.bfloat16)
+    W2 = torch.from_numpy(x["W2"].view(np.int16)).cuda().view(torch.bfloat16)
+    u = torch.empty((n_tok, g * d_mid), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((n_tok, d), dtype=torch.bfloat16, device="cuda")
+    nb = csa.grouped_out_proj_workspace_size(n_tok, g, d_mid, d)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda") if nb else None
+
+    def call():
+        csa.grouped_out_proj(o, W1, W2, g, u, y, ws)
+
+    for _ in range(3):
+        call()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr):
+        call()
+    evs = []
+    for _ in range(reps):
+        l2_flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        gr.replay()
+        b.record()
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    us = float(np.mean([a.elapsed_time(b) for a, b in evs])) * 1e3
+    wbytes = (W1.numel() + W2.numel()) * 2
+    nbytes = wbytes + n_tok * (H * dv + 2 * g * d_mid + d) * 2
+    flops = 2.0 * n_tok * (W1.numel() + W2.numel())
+    res = {"tokens": n_tok, "us": us, "bytes": nbytes, "achieved_gbs": nbytes / (us * 1e-6) / 1e9,
+           "tflops": flops / (us * 1e-6) / 1e12, "peak_source": peak_src, "l2": "flushed before every call",
+           "timing": "CUDA events around one graph replay of the call (launch included)"}
+    if n_tok <= 256:
+        res.update(bound="hbm", frac=res["achieved_gbs"] / hbm_peak)
+    else:
+        res.update(bound="tensor", frac=res["tflops"] / bf16_peak)
+    del W1, W2
+    return {"grouped_out_proj": res}
 
 
 def measure_e2e(args, wid, wl, T, D, csa, steps):
