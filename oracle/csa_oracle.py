@@ -347,6 +347,61 @@ def index_key_compress(Ca, Cb, Za, Zb, Ba, Bb, fmt, prev_Cb=None, prev_Zb=None, 
 
 
 # ---------------------------------------------------------------------------
+# FP8 KV storage  ([P3] section "Гибридный attention: CSA и HCA": KV entries are
+# stored in FP8, only the RoPE dimensions stay in BF16)
+#
+# Reading (the pages give no layout or scale): a 576-wide latent row is stored as
+# 656 bytes: its first 512 values as e4m3 codes of x * 2^-e, the 64 RoPE values as
+# bf16 (nearest even), then one byte e + 127 and 15 zero bytes.  e is the smallest
+# integer with max|x[:512]| <= 448 * 2^e, clamped to [-126, 127]; a power of two,
+# so every stored value times 2^e is exactly a bf16 value.  Decisions are taken on
+# the row as fp32 values, as for the indexer keys.
+# ---------------------------------------------------------------------------
+
+KV8_ROW_BYTES = 656
+
+
+def kv8_exponent(amax):
+    """Smallest integer e with amax <= 448 * 2^e (exact comparisons), clamped to [-126, 127]."""
+    amax = np.asarray(amax, dtype=np.float64)
+    out = np.full(amax.shape, -126, dtype=np.int64)
+    for idx in np.ndindex(amax.shape):
+        a = float(amax[idx])
+        if a == 0.0:
+            continue
+        e = math.frexp(a)[1] - 10                # 448 * 2^e < a here
+        while 448.0 * 2.0 ** e < a:
+            e += 1
+        out[idx] = min(max(e, -126), 127)
+    return out
+
+
+def quantise_latent_fp8(x):
+    """Rows x [n, 576] (float64) -> stored FP8 rows [n, 656] uint8."""
+    x32 = np.asarray(x, dtype=np.float64).astype(np.float32)
+    n = x32.shape[0]
+    assert x32.shape[1] == 576
+    nope = x32[:, :512].astype(np.float64)
+    e = kv8_exponent(np.abs(nope).max(axis=1))
+    codes = encode_e4m3(nope * np.ldexp(1.0, -e)[:, None])
+    rope = bf16_bits_of(round_to_bf16(x32[:, 512:].astype(np.float64)))
+    out = np.zeros((n, KV8_ROW_BYTES), dtype=np.uint8)
+    out[:, :512] = codes
+    out[:, 512:640] = rope.astype("<u2").view(np.uint8).reshape(n, 128)
+    out[:, 640] = (e + 127).astype(np.uint8)
+    return out
+
+
+def dequantise_latent_fp8(rows8):
+    """Stored FP8 rows [n, 656] -> the latent values [n, 576] they hold (float64, exact)."""
+    rows8 = np.asarray(rows8, dtype=np.uint8)
+    e = rows8[:, 640].astype(np.int64) - 127
+    nope = decode_e4m3(rows8[:, :512]) * np.ldexp(1.0, e)[:, None]
+    rope = decode_bf16(np.ascontiguousarray(rows8[:, 512:640]).view("<u2"))
+    return np.concatenate([nope, rope], axis=1)
+
+
+# ---------------------------------------------------------------------------
 # grouped output projection  ([P1] CSA step 4: the head outputs are split into g
 # groups, each group is projected to an intermediate width, and the concatenation is
 # projected to the hidden size; table "Конфигурации": g = 16, width 1024, d = 7168)

@@ -523,3 +523,46 @@ def test_grouped_projection_locality_and_rounding():
     ub, yb = O.grouped_out_proj(o, W1, W2, g, dtype="bf16")
     assert np.array_equal(ub, O.round_to_bf16(u0))
     assert np.array_equal(yb, O.round_to_bf16(O.round_to_bf16(u0) @ W2.T))
+
+
+# ---------------------------------------------------------------- FP8 KV storage
+# [P3] section "Гибридный attention: CSA и HCA": FP8 KV entries, BF16 RoPE dimensions.
+
+def test_kv8_rows_layout_scale_and_error_bound():
+    r = np.random.default_rng(41)
+    x = r.normal(size=(40, 576)) * np.exp(r.uniform(-6, 6, size=(40, 1)))
+    x[7] = 0.0
+    q = O.quantise_latent_fp8(x)
+    assert q.shape == (40, 656) and not q[:, 641:].any()
+    e = q[:, 640].astype(np.int64) - 127
+    amax = np.abs(x[:, :512].astype(np.float32).astype(np.float64)).max(axis=1)
+    live = amax > 0
+    assert np.all(amax[live] <= 448.0 * np.ldexp(1.0, e[live]))
+    assert np.all(amax[live] > 448.0 * np.ldexp(1.0, e[live] - 1))
+    assert e[7] == -126 and not q[7, :640].any()
+    dq = O.dequantise_latent_fp8(q)
+    # the codes are torch's float8 cast of x * 2^-e (up to the sign of zero)
+    y = x[:, :512].astype(np.float32).astype(np.float64) * np.ldexp(1.0, -e)[:, None]
+    ref = torch.tensor(y).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(np.where(ref == 0x80, 0, ref), q[:, :512])
+    # nope: within half an e4m3 step (2^-4 relative; 2^-10 * 2^e among subnormals)
+    s = np.ldexp(1.0, e)[:, None]
+    assert np.all(np.abs(dq[:, :512] - x[:, :512]) <= 2.0 ** -4 * np.abs(x[:, :512]) + 2.0 ** -10 * s + 1e-30)
+    # rope: torch's bf16 rounding of the fp32 value
+    rb = torch.tensor(x[:, 512:].astype(np.float32)).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(dq[:, 512:], rb)
+    # every dequantised value is a bf16 value (the attention kernel's exact operand)
+    assert np.array_equal(O.round_to_bf16(dq), dq)
+
+
+def test_kv8_rows_on_grid_round_trip_exactly():
+    r = np.random.default_rng(42)
+    codes = r.integers(0, 0x7F, size=(5, 512)).astype(np.uint8) | np.where(r.random((5, 512)) < 0.5, 0x80, 0).astype(np.uint8)
+    codes[:, 3] = 0x7E                                      # 448 somewhere in every row
+    e = np.array([-3, 0, 4, -126 + 9, 20])
+    x = np.zeros((5, 576))
+    x[:, :512] = O.decode_e4m3(codes) * np.ldexp(1.0, e)[:, None]
+    x[:, 512:] = O.round_to_bf16(r.normal(size=(5, 64)))
+    q = O.quantise_latent_fp8(x)
+    assert np.array_equal(q[:, 640].astype(np.int64) - 127, e)
+    assert np.array_equal(O.dequantise_latent_fp8(q), np.where(x == 0, 0.0, x))
