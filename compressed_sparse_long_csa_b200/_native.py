@@ -35,6 +35,8 @@ _SIGS = {
     "attn_decode_workspace_size": ([_i32, _i32, _i32, _i64], _sz),
     "sparse_attn_decode": ([_vp] * 6 + [_i32, _i32, _i32, _i32, _i64, _i32, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp], _i32),
     "hca_attn_decode": ([_vp] * 6 + [_i32, _i32, _i32, _i32, _i64, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp], _i32),
+    "sparse_attn_decode_kv8": ([_vp] * 6 + [_i32, _i32, _i32, _i32, _i64, _i32, _i32, _f32, _vp, _vp, _vp, _sz, _vp], _i32),
+    "hca_attn_decode_kv8": ([_vp] * 6 + [_i32, _i32, _i32, _i32, _i64, _i32, _f32, _vp, _vp, _vp, _sz, _vp], _i32),
     "hca_compress_attn_decode": ([_vp] * 4 + [_i32, _i32] + [_vp] * 6 + [_i32, _i32, _i32, _i32, _i64, _i32, _f32, _i32,
                                                                       _vp, _vp, _vp, _sz, _vp], _i32),
     "sparse_attn_decode_noalloc": ([_vp] * 6 + [_i32, _i32, _i32, _i32, _i64, _i32, _i32, _f32, _i32, _vp, _vp, _vp], _i32),
@@ -177,6 +179,28 @@ def hca_attn_decode(q, cache, n_entries, win, win_len, sink, sm_scale, d_v, out,
     _check(lib.hca_attn_decode(_p(q), _p(cache), _p(n_entries), _p(win), _p(win_len), _p(sink), B, H, d_k, d_v,
                                cache.shape[1], W, sm_scale, _dtype_code(q), _p(out), _p(lse), wp, wb,
                                _stream(stream)), "hca_attn_decode")
+
+
+def sparse_attn_decode_kv8(q, cache8, idx, win, win_len, sink, sm_scale, d_v, out, lse=None, workspace=None,
+                           stream=None):
+    """cache8: [B, n_max, 656] uint8 FP8 rows (see csa.h)."""
+    B, H, d_k = q.shape
+    W = win.shape[1] if win is not None else 0
+    k = idx.shape[1] if idx is not None else 0
+    wp, wb = _ws(workspace)
+    _check(lib.sparse_attn_decode_kv8(_p(q), _p(cache8), _p(idx), _p(win), _p(win_len), _p(sink), B, H, d_k, d_v,
+                                      cache8.shape[1], k, W, sm_scale, _p(out), _p(lse), wp, wb, _stream(stream)),
+           "sparse_attn_decode_kv8")
+
+
+def hca_attn_decode_kv8(q, cache8, n_entries, win, win_len, sink, sm_scale, d_v, out, lse=None, workspace=None,
+                        stream=None):
+    B, H, d_k = q.shape
+    W = win.shape[1] if win is not None else 0
+    wp, wb = _ws(workspace)
+    _check(lib.hca_attn_decode_kv8(_p(q), _p(cache8), _p(n_entries), _p(win), _p(win_len), _p(sink), B, H, d_k,
+                                   d_v, cache8.shape[1], W, sm_scale, _p(out), _p(lse), wp, wb, _stream(stream)),
+           "hca_attn_decode_kv8")
 
 
 def hca_compress_attn_decode(C_, Z, bias, entry0, q, cache, n_entries, win, win_len, sink, sm_scale, d_v, out,

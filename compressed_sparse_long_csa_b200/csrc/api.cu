@@ -332,8 +332,10 @@ static csa_status run_attention(AttnArgs& a, int dtype, void* workspace, size_t 
   bool used = false, combined = false;
   cudaError_t e = cudaSuccess;
   a.part_fp16 = 0;
+  if (a.kv8 && !tc) return CSA_ERR_UNSUPPORTED;
   if (tc) e = launch_attention_tc(a, st, &used, &combined);
   if (e != cudaSuccess) return CSA_ERR_CUDA;
+  if (a.kv8 && !used) return CSA_ERR_UNSUPPORTED;  // FP8 rows have no CUDA-core path
   if (used) a.part_fp16 = 1;                   // the tensor-core kernel's partial format
   if (!used) {
     if (tc) {  // the tensor-core path declined: recompute the split plan for the CUDA-core path
@@ -347,10 +349,10 @@ static csa_status run_attention(AttnArgs& a, int dtype, void* workspace, size_t 
   return CSA_OK;
 }
 
-csa_status sparse_attn_decode(const void* q, const void* cache, const int32_t* idx, const void* win,
-                              const int32_t* win_len, const float* sink, int B, int H, int d_k, int d_v,
-                              int64_t n_max, int k, int W, float sm_scale, int dtype, void* out, float* lse,
-                              void* workspace, size_t ws_bytes, void* stream) {
+static csa_status sparse_decode(const void* q, const void* cache, const int32_t* idx, const void* win,
+                                const int32_t* win_len, const float* sink, int B, int H, int d_k, int d_v,
+                                int64_t n_max, int k, int W, float sm_scale, int dtype, void* out, float* lse,
+                                void* workspace, size_t ws_bytes, void* stream, int kv8) {
   csa_status s = attn_common_checks(q, cache, win, sink, B, H, d_k, d_v, n_max, W, dtype, out, lse);
   if (s != CSA_OK) return s;
   REQUIRE(k >= 0 && k <= 65536 && B <= 65535, CSA_ERR_SHAPE);
@@ -364,14 +366,31 @@ csa_status sparse_attn_decode(const void* q, const void* cache, const int32_t* i
   AttnArgs a{};
   a.q = q; a.cache = cache; a.idx = idx; a.k = k; a.n_seg_a = k; a.win = win; a.win_len = win_len;
   a.W = W; a.prefill = 0; a.sink = sink; a.B = B; a.Tq = 1; a.H = H; a.dk = d_k; a.dv = d_v; a.n_max = n_max;
-  a.sm_scale = sm_scale; a.out = out; a.lse = lse; a.err = err;
+  a.sm_scale = sm_scale; a.out = out; a.lse = lse; a.err = err; a.kv8 = kv8;
   return run_attention(a, dtype, workspace, ws_bytes, true, S(stream));
 }
 
-csa_status hca_attn_decode(const void* q, const void* cache, const int32_t* n_entries, const void* win,
-                           const int32_t* win_len, const float* sink, int B, int H, int d_k, int d_v,
-                           int64_t n_max, int W, float sm_scale, int dtype, void* out, float* lse,
-                           void* workspace, size_t ws_bytes, void* stream) {
+csa_status sparse_attn_decode(const void* q, const void* cache, const int32_t* idx, const void* win,
+                              const int32_t* win_len, const float* sink, int B, int H, int d_k, int d_v,
+                              int64_t n_max, int k, int W, float sm_scale, int dtype, void* out, float* lse,
+                              void* workspace, size_t ws_bytes, void* stream) {
+  return sparse_decode(q, cache, idx, win, win_len, sink, B, H, d_k, d_v, n_max, k, W, sm_scale, dtype, out, lse,
+                       workspace, ws_bytes, stream, 0);
+}
+
+csa_status sparse_attn_decode_kv8(const void* q, const void* cache8, const int32_t* idx, const void* win,
+                                  const int32_t* win_len, const float* sink, int B, int H, int d_k, int d_v,
+                                  int64_t n_max, int k, int W, float sm_scale, void* out, float* lse,
+                                  void* workspace, size_t ws_bytes, void* stream) {
+  REQUIRE(attn_tc_shape(CSA_BF16, H, d_k, d_v), CSA_ERR_UNSUPPORTED);
+  return sparse_decode(q, cache8, idx, win, win_len, sink, B, H, d_k, d_v, n_max, k, W, sm_scale, CSA_BF16, out,
+                       lse, workspace, ws_bytes, stream, 1);
+}
+
+static csa_status hca_decode(const void* q, const void* cache, const int32_t* n_entries, const void* win,
+                             const int32_t* win_len, const float* sink, int B, int H, int d_k, int d_v,
+                             int64_t n_max, int W, float sm_scale, int dtype, void* out, float* lse,
+                             void* workspace, size_t ws_bytes, void* stream, int kv8) {
   csa_status s = attn_common_checks(q, cache, win, sink, B, H, d_k, d_v, n_max, W, dtype, out, lse);
   if (s != CSA_OK) return s;
   REQUIRE(n_max <= (1 << 24) && B <= 65535, CSA_ERR_SHAPE);
@@ -386,7 +405,25 @@ csa_status hca_attn_decode(const void* q, const void* cache, const int32_t* n_en
   a.q = q; a.cache = cache; a.idx = nullptr; a.n_entries = n_entries; a.n_seg_a = (int)n_max;
   a.win = win; a.win_len = win_len; a.W = W; a.prefill = 0; a.sink = sink; a.B = B; a.Tq = 1; a.H = H;
   a.dk = d_k; a.dv = d_v; a.n_max = n_max; a.sm_scale = sm_scale; a.out = out; a.lse = lse; a.err = err;
+  a.kv8 = kv8;
   return run_attention(a, dtype, workspace, ws_bytes, true, S(stream));
+}
+
+csa_status hca_attn_decode(const void* q, const void* cache, const int32_t* n_entries, const void* win,
+                           const int32_t* win_len, const float* sink, int B, int H, int d_k, int d_v,
+                           int64_t n_max, int W, float sm_scale, int dtype, void* out, float* lse,
+                           void* workspace, size_t ws_bytes, void* stream) {
+  return hca_decode(q, cache, n_entries, win, win_len, sink, B, H, d_k, d_v, n_max, W, sm_scale, dtype, out, lse,
+                    workspace, ws_bytes, stream, 0);
+}
+
+csa_status hca_attn_decode_kv8(const void* q, const void* cache8, const int32_t* n_entries, const void* win,
+                               const int32_t* win_len, const float* sink, int B, int H, int d_k, int d_v,
+                               int64_t n_max, int W, float sm_scale, void* out, float* lse, void* workspace,
+                               size_t ws_bytes, void* stream) {
+  REQUIRE(attn_tc_shape(CSA_BF16, H, d_k, d_v), CSA_ERR_UNSUPPORTED);
+  return hca_decode(q, cache8, n_entries, win, win_len, sink, B, H, d_k, d_v, n_max, W, sm_scale, CSA_BF16, out,
+                    lse, workspace, ws_bytes, stream, 1);
 }
 
 csa_status hca_compress_attn_decode(const void* C, const void* Z, const float* bias, const int32_t* entry0, int T_new,

@@ -34,6 +34,7 @@ struct AttnArgs {
   int cluster_combine;        // tensor-core path: splits merged inside a thread-block cluster
   const int32_t* dep_entry0;  // dense decode after a compression kernel in the same stream: it
   int dep_rows;               // writes rows dep_entry0[b] .. +dep_rows-1 (null: wait for it at once)
+  int kv8;                    // cache rows are 656-byte FP8 rows (tensor-core kernel only)
   unsigned* err;
 };
 

@@ -60,6 +60,7 @@ struct AtSmem {
   const __nv_bfloat16* rowp[2][AT_ROWS];
   unsigned long long run_key[2][2];   // per stage and loader warp: (tensor << 32 | first row) or NO_RUN
   uint32_t vmask[2][2];  // per stage: bit j of word j / 32 set when row j of the tile is valid
+  uint32_t k8mask[2][2]; // per stage: row j is an FP8 cache row, expanded to bf16 in place
   alignas(8) uint64_t full[2];
   uint64_t empty[2];
   uint64_t sfull[2];
@@ -111,6 +112,51 @@ __device__ __forceinline__ float ex2_approx(float x) {
 
 // byte offset of 16-byte chunk c of row j in a 128-byte-swizzled atom
 __device__ __forceinline__ uint32_t sw128_off(int j, int c) { return (j >> 3) * 1024 + (j & 7) * 128 + ((c ^ (j & 7)) << 4); }
+
+// ---- FP8 cache rows (656 bytes: 512 e4m3 codes of x / 2^e, 64 bf16 RoPE values, the byte
+// e + 127).  The gather puts a row's 64 codes of atom a into the second half of the row's
+// own 128-byte line of atom a (unswizzled), its RoPE values straight into atom 8, and its
+// exponent byte into the first bytes of its lines of atoms 0 and 4; a thread then expands
+// (row, atoms 0-3) or (row, atoms 4-7) in place: it reads the exponent and a line's codes
+// before it writes that line, and no other thread touches the line, so no barrier is needed
+// inside the expansion.  codes * 2^e are exact bf16 values: the MMA sees the stored row.
+constexpr int KV8_ROW = 656;
+
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t pair, float mult) {
+  uint32_t h2;
+  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h2) : "r"(pair));
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+  const __nv_bfloat162 b = __floats2bfloat162_rn(f.x * mult, f.y * mult);
+  return *reinterpret_cast<const uint32_t*>(&b);
+}
+
+__device__ __forceinline__ void kv8_expand(uint32_t kv0, const uint32_t* k8mask, int lg) {
+  for (int u = lg; u < 2 * AT_ROWS; u += AT_GROUP) {
+    const int j = u & (AT_ROWS - 1), h = u / AT_ROWS;
+    if (!((k8mask[j >> 5] >> (j & 31)) & 1u)) continue;
+    uint32_t sc;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(sc) : "r"(kv0 + 4 * h * ATOM + j * 128) : "memory");
+    const float mult = __uint_as_float((sc & 0xFFu) << 23);          // 2^e
+    for (int a4 = 0; a4 < 4; ++a4) {
+      const uint32_t atom = kv0 + (4 * h + a4) * ATOM;
+      const uint32_t line = atom + j * 128;
+      uint32_t cw[16];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(cw[4 * i]), "=r"(cw[4 * i + 1]), "=r"(cw[4 * i + 2]), "=r"(cw[4 * i + 3])
+                     : "r"(line + 64 + 16 * i) : "memory");
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {                                 // bf16 chunk i: codes 8i .. 8i+7
+        const uint32_t w0 = cw[2 * i], w1 = cw[2 * i + 1];
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                     ::"r"(atom + sw128_off(j, i)), "r"(e4m3x2_to_bf16x2(w0 & 0xFFFFu, mult)),
+                       "r"(e4m3x2_to_bf16x2(w0 >> 16, mult)), "r"(e4m3x2_to_bf16x2(w1 & 0xFFFFu, mult)),
+                       "r"(e4m3x2_to_bf16x2(w1 >> 16, mult)) : "memory");
+      }
+    }
+  }
+}
 
 // TMEM: O at lane offset 0, columns [0, 512); S buffers at lane offset 16, columns 0 and 64.
 constexpr uint32_t TM_S_LANE = 16u << 16, TM_COLS = 512;
@@ -200,14 +246,18 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
       const bool go = tc::mbar_wait(&sm.empty[g], (i & 1) ^ 1) && !*(volatile int*)&sm.abort_flag;
       if (!go) sm.ld_stop[g] = i + 1;      // the group leaves together at this iteration's barrier
       if (lg < AT_ROWS) {
+        const bool r8 = a.kv8 && which == 0;                 // an FP8 cache row
         const __nv_bfloat16* base = which == 1 ? (const __nv_bfloat16*)a.win : (const __nv_bfloat16*)a.cache;
-        sm.rowp[g][lg] = which >= 0 ? base + (size_t)y * 576 : nullptr;
+        sm.rowp[g][lg] = which < 0 ? nullptr
+                         : r8 ? reinterpret_cast<const __nv_bfloat16*>((const uint8_t*)a.cache + (size_t)y * KV8_ROW)
+                              : base + (size_t)y * 576;
         const uint32_t vb = __ballot_sync(0xffffffffu, which >= 0);
-        if ((lg & 31) == 0) sm.vmask[g][lg >> 5] = vb;
-        // the tile is one contiguous run when all 64 rows are valid rows of one tensor
+        const uint32_t kb = __ballot_sync(0xffffffffu, r8);
+        if ((lg & 31) == 0) { sm.vmask[g][lg >> 5] = vb; sm.k8mask[g][lg >> 5] = kb; }
+        // the tile is one contiguous run when all 64 rows are valid bf16 rows of one tensor
         // with y - lg the same everywhere; each warp checks its 32 rows
         const unsigned long long key =
-            which >= 0 ? ((unsigned long long)which << 32) | (unsigned)(y - lg) : NO_RUN;
+            which >= 0 && !r8 ? ((unsigned long long)which << 32) | (unsigned)(y - lg) : NO_RUN;
         int same = 0;
         __match_all_sync(0xffffffffu, key, &same);
         if ((lg & 31) == 0) sm.run_key[g][lg >> 5] = same ? key : NO_RUN;
@@ -235,9 +285,17 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
         }
       } else {
         const uint32_t kv0 = tc::smem_u32(sm.kv[g][0]);
+        const bool any8 = (sm.k8mask[g][0] | sm.k8mask[g][1]) != 0u;
         for (int p = lg; p < AT_ROWS * AT_CHUNKS; p += AT_GROUP) {
           const int j = p / AT_CHUNKS, c = p - j * AT_CHUNKS;
           const __nv_bfloat16* rp = sm.rowp[g][j];
+          if (any8 && ((sm.k8mask[g][j >> 5] >> (j & 31)) & 1u)) {
+            const uint8_t* rb = reinterpret_cast<const uint8_t*>(rp);
+            if (c < 32) cp_async16(kv0 + (c >> 2) * ATOM + j * 128 + 64 + (c & 3) * 16, rb + c * 16);
+            else if (c < 40) cp_async16(kv0 + 8 * ATOM + sw128_off(j, c - 32), rb + 512 + (c - 32) * 16);
+            else if (c < 42) cp_async16(kv0 + (c == 40 ? 0 : 4) * ATOM + j * 128, rb + 640);
+            continue;
+          }
           const uint32_t dst = kv0 + (c >> 3) * ATOM + sw128_off(j, c & 7);
           if (rp) cp_async16(dst, rp + c * 8);
           else cp_async_zero16(dst, a.cache);
@@ -249,6 +307,10 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
       if (it + 2 < n_t) coord(it + 2);
       if (!run) {
         cp_async_wait_all();
+        if ((sm.k8mask[g][0] | sm.k8mask[g][1]) != 0u) {   // the same for the whole group
+          named_bar(1 + g, AT_GROUP);                         // every thread's copies have landed
+          kv8_expand(tc::smem_u32(sm.kv[g][0]), sm.k8mask[g], lg);
+        }
         tc::fence_proxy_async_smem();
         tc::mbar_arrive(&sm.full[g]);
       }
@@ -702,7 +764,8 @@ cudaError_t launch_attention_tc(AttnArgs a, cudaStream_t st, bool* used, bool* c
   AtMaps maps;
   const uint64_t win_rows = a.prefill ? (uint64_t)a.B * a.t_raw : (uint64_t)a.B * a.W;
   if (!make_latent_map(&maps.q, a.q, (uint64_t)a.B * a.Tq * AT_H)) return cudaSuccess;
-  if (!make_latent_map(&maps.cache, a.cache, (uint64_t)a.B * a.n_max)) return cudaSuccess;
+  if (a.kv8) maps.cache = maps.q;                    // FP8 rows are gathered, never loaded by TMA
+  else if (!make_latent_map(&maps.cache, a.cache, (uint64_t)a.B * a.n_max)) return cudaSuccess;
   if (a.win && win_rows > 0) {
     if (!make_latent_map(&maps.win, a.win, win_rows)) return cudaSuccess;
   } else {

@@ -36,7 +36,7 @@ import torch
 
 __all__ = [
     "WORKLOADS", "make_workload", "Workload",
-    "bf16_bits", "fp32", "quant_e4m3_rows", "quant_mxfp4_rows", "index_key_inputs", "out_proj_inputs",
+    "bf16_bits", "fp32", "quant_e4m3_rows", "quant_mxfp4_rows", "index_key_inputs", "out_proj_inputs", "quant_latent_fp8_rows",
 ]
 
 # --------------------------------------------------------------------------
@@ -64,6 +64,29 @@ def quant_e4m3_rows(x: torch.Tensor):
     y = (x / scale.unsqueeze(-1)).clamp(-448.0, 448.0)
     codes = y.to(torch.float8_e4m3fn).view(torch.uint8)
     return codes.numpy().copy(), scale.numpy().astype(np.float32).copy()
+
+
+def quant_latent_fp8_rows(x: torch.Tensor) -> np.ndarray:
+    """576-wide latent rows -> 656-byte FP8 rows: bytes 0..511 the e4m3 codes (torch's
+    round-to-nearest-even cast, +0 for values that round to zero) of x[:512] / 2^e with e
+    the smallest integer such that max|x[:512]| <= 448 * 2^e (clamped to [-126, 127]);
+    bytes 512..639 x[512:] as bf16 (little endian); byte 640 = e + 127; the rest zero."""
+    x = x.to(torch.float32)
+    lead = x.shape[:-1]
+    nope = x[..., :512]
+    amax = nope.abs().amax(dim=-1)
+    e = torch.where(amax > 0, torch.ceil(torch.log2(amax / 448.0)), torch.full_like(amax, -126.0))
+    e = torch.where((amax > 0) & (amax > 448.0 * torch.exp2(e)), e + 1, e)
+    e = torch.where((amax > 0) & (amax <= 448.0 * torch.exp2(e - 1)), e - 1, e)
+    e = e.clamp(-126, 127)
+    codes = (nope / torch.exp2(e).unsqueeze(-1)).to(torch.float8_e4m3fn).view(torch.uint8)
+    codes = torch.where(codes == 0x80, torch.zeros_like(codes), codes)
+    out = torch.zeros(*lead, 656, dtype=torch.uint8)
+    out[..., :512] = codes
+    rope = x[..., 512:].to(torch.bfloat16).contiguous().view(torch.uint8)
+    out[..., 512:640] = rope.reshape(*lead, 128)
+    out[..., 640] = (e + 127).to(torch.uint8)
+    return out.numpy()
 
 
 def _e2m1_rne_codes(y: torch.Tensor) -> torch.Tensor:

@@ -290,6 +290,31 @@ csa_status hca_attn_decode(const void* q, const void* cache, const int32_t* n_en
                            float sm_scale, int dtype, void* out, float* lse,
                            void* workspace, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * sparse_attn_decode_kv8 / hca_attn_decode_kv8 — the same attention over an FP8
+ * cache ("Гибридный attention: CSA и HCA" of the aixai.ru digest: KV entries are
+ * stored in FP8, only the RoPE dimensions in BF16).
+ *
+ *   cache8  device [B, n_max, 656] bytes per entry: bytes 0..511 the e4m3 codes of
+ *           row[0:512] / 2^e, bytes 512..639 row[512:576] as bf16 (little endian),
+ *           byte 640 = e + 127 (e in [-126, 127]), bytes 641..655 zero.  The stored
+ *           row is codes * 2^e (exact) followed by the bf16 RoPE values.
+ * The window rows stay bf16 ([B, W, d_k]).  Each FP8 row is expanded to bf16 in
+ * shared memory as it is gathered; the arithmetic is that of the bf16 calls.
+ * Other arguments as sparse_attn_decode / hca_attn_decode with dtype bf16.
+ * Supported: H == 128, d_k == 576, d_v == 512 (CSA_ERR_UNSUPPORTED otherwise).
+ * ------------------------------------------------------------------------- */
+csa_status sparse_attn_decode_kv8(const void* q, const void* cache8, const int32_t* idx,
+                                  const void* win, const int32_t* win_len, const float* sink,
+                                  int B, int H, int d_k, int d_v, int64_t n_max, int k, int W,
+                                  float sm_scale, void* out, float* lse,
+                                  void* workspace, size_t ws_bytes, void* stream);
+csa_status hca_attn_decode_kv8(const void* q, const void* cache8, const int32_t* n_entries,
+                               const void* win, const int32_t* win_len, const float* sink,
+                               int B, int H, int d_k, int d_v, int64_t n_max, int W,
+                               float sm_scale, void* out, float* lse,
+                               void* workspace, size_t ws_bytes, void* stream);
+
 /* hca_compress_attn_decode — one HCA decode step: hca_compress of the fresh chunk
  * into the cache, then hca_attn_decode over entries 0..n_entries[b]-1 (which include
  * the fresh rows) + window + sink; the same results as the two calls in that order.

@@ -24,7 +24,8 @@ def test_every_declared_symbol_is_exported():
     names = declared_functions()
     assert {"csa_compress", "hca_compress", "lightning_index", "topk_select", "sparse_attn_decode",
             "sparse_attn_prefill", "hca_attn_decode", "hca_compress_attn_decode", "index_key_compress",
-            "lightning_index_bf16", "grouped_out_proj"} <= set(names)
+            "lightning_index_bf16", "grouped_out_proj", "sparse_attn_decode_kv8",
+            "hca_attn_decode_kv8"} <= set(names)
     for n in names:
         assert hasattr(N.lib, n), n
 
@@ -149,6 +150,21 @@ def test_grouped_out_proj_validation():
     assert N.lib.csa_launch_count() == before
     assert N.lib.grouped_out_proj_workspace_size(16, 16, 1024, 7168) == 8 * 16 * 16384 * 4
     assert N.lib.grouped_out_proj_workspace_size(4096, 16, 1024, 7168) == 0   # large batches need no split
+
+
+def test_kv8_attention_validation():
+    """FP8 rows exist only on the tensor-core shapes; the checks run before any launch."""
+    before = N.lib.csa_launch_count()
+    args = lambda H, dk, dv: (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, H, dk, dv, 1024, 64, 16, 0.05, FAKE, None,
+                              FAKE, 1 << 30, None)
+    assert N.lib.sparse_attn_decode_kv8(*args(64, 576, 512)) == ERR_UNSUP
+    assert N.lib.sparse_attn_decode_kv8(*args(128, 64, 64)) == ERR_UNSUP
+    a = list(args(128, 576, 512))
+    a[1] = None
+    assert N.lib.sparse_attn_decode_kv8(*a) == ERR_NULL
+    h = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 128, 576, 256, 1024, 16, 0.05, FAKE, None, FAKE, 1 << 30, None)
+    assert N.lib.hca_attn_decode_kv8(*h) == ERR_UNSUP
+    assert N.lib.csa_launch_count() == before
 
 
 def test_attention_validation():

@@ -47,3 +47,14 @@ def test_workload_shapes_small():
     assert D["entry0"] == 1023 and D["q_pos0"] == 4095
     w4 = CI.make_workload(4, scale={"B": 1, "T": 8192})
     assert w4.tensors["kI"].shape == (1, 2048, 64) and w4.tensors["kI_scale"].shape == (1, 2048, 4)
+
+
+def test_fp8_latent_rows_of_the_generator_match_the_oracle_format():
+    """The generator's FP8 cache rows (torch casts) equal the oracle's own quantiser (its
+    e4m3 encoder and exponent search) on rows of widely different magnitudes."""
+    import torch
+    from oracle import csa_oracle as O
+    g = torch.Generator().manual_seed(5)
+    x = torch.randn(64, 576, generator=g) * torch.exp(torch.randn(64, 1, generator=g) * 4)
+    x[9] = 0.0
+    assert np.array_equal(CI.quant_latent_fp8_rows(x), O.quantise_latent_fp8(x.double().numpy()))
