@@ -396,6 +396,9 @@ def run_ours(args, wid):
     if bf:
         extra = dict(extra or {}, **bf)
     extra = dict(extra or {}, **measure_out_proj(D, T, csa, l2_flush, hbm_peak, bf16_peak, src))
+    kv = measure_kv8_attention(wid, wl, D, T, csa, l2_flush, float(mean_ms[comp.index("attention")]), hbm_peak, src)
+    if kv:
+        extra.update(kv)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -558,6 +561,54 @@ def measure_out_proj(D, T, csa, l2_flush, hbm_peak, bf16_peak, peak_src, reps=10
         res.update(bound="tensor", frac=res["tflops"] / bf16_peak)
     del W1, W2
     return {"grouped_out_proj": res}
+
+
+def measure_kv8_attention(wid, wl, D, T, csa, l2_flush, bf16_ms, hbm_peak, peak_src, reps=20):
+    """The decode attention of this step over an FP8 copy of the cache (656-byte rows made
+    by the input generator from the same values), timed alone like the per-call breakdown,
+    beside the bf16 call's time."""
+    import numpy as np
+    import torch
+    import csa_inputs as CI
+    if wid not in (1, 2):
+        return None
+    bits = wl.tensors["cache"]
+    x = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).float()
+    c8 = torch.from_numpy(CI.quant_latent_fp8_rows(x)).cuda()
+    del x
+    B, H, dv, W = D["B"], D["H"], D["dv"], D["W"]
+    out = torch.empty(B, H, dv, dtype=torch.bfloat16, device="cuda")
+
+    def call():
+        if wid == 1:
+            csa.sparse_attn_decode_kv8(T["q"][:, 0], c8, T["idx"][:, 0], T["win"], T["win_len"], T["sink"],
+                                       D["sm_scale"], dv, out, workspace=T["aws"])
+        else:
+            csa.hca_attn_decode_kv8(T["q"][:, 0], c8, T["n_entries"], T["win"], T["win_len"], T["sink"],
+                                    D["sm_scale"], dv, out, workspace=T["aws"])
+
+    for _ in range(3):
+        call()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call()
+    evs = []
+    for _ in range(reps):
+        l2_flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    us = float(np.mean([a.elapsed_time(b) for a, b in evs])) * 1e3
+    rows = D["k"] if wid == 1 else D["N"]
+    nbytes = B * (rows * 656 + W * 1152 + H * 576 * 2 + H * dv * 2)
+    gbs = nbytes / (us * 1e-6) / 1e9
+    return {"attention_kv8": {"us": us, "bf16_us": bf16_ms * 1e3, "speedup": bf16_ms * 1e3 / us, "bytes": nbytes,
+                              "achieved_gbs": gbs, "frac": gbs / hbm_peak, "peak_source": peak_src,
+                              "l2": "flushed before every call",
+                              "timing": "CUDA events around one graph replay of the call (launch included)"}}
 
 
 def measure_e2e(args, wid, wl, T, D, csa, steps):

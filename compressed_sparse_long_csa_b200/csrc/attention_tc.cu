@@ -116,10 +116,11 @@ __device__ __forceinline__ uint32_t sw128_off(int j, int c) { return (j >> 3) * 
 // ---- FP8 cache rows (656 bytes: 512 e4m3 codes of x / 2^e, 64 bf16 RoPE values, the byte
 // e + 127).  The gather puts a row's 64 codes of atom a into the second half of the row's
 // own 128-byte line of atom a (unswizzled), its RoPE values straight into atom 8, and its
-// exponent byte into the first bytes of its lines of atoms 0 and 4; a thread then expands
-// (row, atoms 0-3) or (row, atoms 4-7) in place: it reads the exponent and a line's codes
-// before it writes that line, and no other thread touches the line, so no barrier is needed
-// inside the expansion.  codes * 2^e are exact bf16 values: the MMA sees the stored row.
+// exponent byte into the first bytes of each of its eight code lines; a thread then expands
+// one (row, atom) line in place: it reads the exponent and the line's codes before it writes
+// the line, and no other thread touches the line, so no barrier is needed inside the
+// expansion (512 lines per tile over the group's 96 threads).  codes * 2^e are exact bf16
+// values: the MMA sees the stored row.
 constexpr int KV8_ROW = 656;
 
 __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t pair, float mult) {
@@ -131,29 +132,26 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t pair, float mult) 
 }
 
 __device__ __forceinline__ void kv8_expand(uint32_t kv0, const uint32_t* k8mask, int lg) {
-  for (int u = lg; u < 2 * AT_ROWS; u += AT_GROUP) {
-    const int j = u & (AT_ROWS - 1), h = u / AT_ROWS;
+  for (int u = lg; u < 8 * AT_ROWS; u += AT_GROUP) {
+    const int j = u & (AT_ROWS - 1), a = u / AT_ROWS;
     if (!((k8mask[j >> 5] >> (j & 31)) & 1u)) continue;
-    uint32_t sc;
-    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(sc) : "r"(kv0 + 4 * h * ATOM + j * 128) : "memory");
+    const uint32_t atom = kv0 + a * ATOM;
+    const uint32_t line = atom + j * 128;
+    uint32_t sc, cw[16];
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(sc) : "r"(line) : "memory");
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(cw[4 * i]), "=r"(cw[4 * i + 1]), "=r"(cw[4 * i + 2]), "=r"(cw[4 * i + 3])
+                   : "r"(line + 64 + 16 * i) : "memory");
     const float mult = __uint_as_float((sc & 0xFFu) << 23);          // 2^e
-    for (int a4 = 0; a4 < 4; ++a4) {
-      const uint32_t atom = kv0 + (4 * h + a4) * ATOM;
-      const uint32_t line = atom + j * 128;
-      uint32_t cw[16];
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(cw[4 * i]), "=r"(cw[4 * i + 1]), "=r"(cw[4 * i + 2]), "=r"(cw[4 * i + 3])
-                     : "r"(line + 64 + 16 * i) : "memory");
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {                                 // bf16 chunk i: codes 8i .. 8i+7
-        const uint32_t w0 = cw[2 * i], w1 = cw[2 * i + 1];
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
-                     ::"r"(atom + sw128_off(j, i)), "r"(e4m3x2_to_bf16x2(w0 & 0xFFFFu, mult)),
-                       "r"(e4m3x2_to_bf16x2(w0 >> 16, mult)), "r"(e4m3x2_to_bf16x2(w1 & 0xFFFFu, mult)),
-                       "r"(e4m3x2_to_bf16x2(w1 >> 16, mult)) : "memory");
-      }
+    for (int i = 0; i < 8; ++i) {                                   // bf16 chunk i: codes 8i .. 8i+7
+      const uint32_t w0 = cw[2 * i], w1 = cw[2 * i + 1];
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                   ::"r"(atom + sw128_off(j, i)), "r"(e4m3x2_to_bf16x2(w0 & 0xFFFFu, mult)),
+                     "r"(e4m3x2_to_bf16x2(w0 >> 16, mult)), "r"(e4m3x2_to_bf16x2(w1 & 0xFFFFu, mult)),
+                     "r"(e4m3x2_to_bf16x2(w1 >> 16, mult)) : "memory");
     }
   }
 }
@@ -293,7 +291,7 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
             const uint8_t* rb = reinterpret_cast<const uint8_t*>(rp);
             if (c < 32) cp_async16(kv0 + (c >> 2) * ATOM + j * 128 + 64 + (c & 3) * 16, rb + c * 16);
             else if (c < 40) cp_async16(kv0 + 8 * ATOM + sw128_off(j, c - 32), rb + 512 + (c - 32) * 16);
-            else if (c < 42) cp_async16(kv0 + (c == 40 ? 0 : 4) * ATOM + j * 128, rb + 640);
+            else if (c < 48) cp_async16(kv0 + (c - 40) * ATOM + j * 128, rb + 640);   // exponent, per line
             continue;
           }
           const uint32_t dst = kv0 + (c >> 3) * ATOM + sw128_off(j, c & 7);
