@@ -23,6 +23,7 @@ _SIGS = {
     "csa_read_device_error": ([_vp, C.POINTER(C.c_uint32)], _i32),
     "csa_launch_count": ([], C.c_uint64),
     "csa_compress": ([_vp] * 10 + [_i64, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
+    "csa_compress_kv8": ([_vp] * 10 + [_i64, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
     "index_key_compress": ([_vp] * 11 + [_i64, _i32, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
     "grouped_out_proj_workspace_size": ([_i32, _i32, _i32, _i32], _sz),
     "grouped_out_proj": ([_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp], _i32),
@@ -111,6 +112,14 @@ def grouped_out_proj(o, W1, W2, g, u, y, workspace=None, stream=None):
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(lib.grouped_out_proj(_p(o), T, H, dv, g, d_mid, _p(W1), _p(W2), d, _p(u), _p(y), _p(workspace), ws_bytes,
                                 _stream(stream)), "grouped_out_proj")
+
+
+def csa_compress_kv8(Ca, Cb, Za, Zb, Ba, Bb, prev_Cb, prev_Zb, entry0, cache8, m=4, stream=None):
+    """cache8: [B, n_max, 656] uint8 FP8 rows (see csa.h)."""
+    B, T_new, d = Ca.shape
+    _check(lib.csa_compress_kv8(_p(Ca), _p(Cb), _p(Za), _p(Zb), _p(Ba), _p(Bb), _p(prev_Cb), _p(prev_Zb),
+                                _p(entry0), _p(cache8), cache8.shape[1], B, T_new, d, m, _dtype_code(Ca),
+                                _stream(stream)), "csa_compress_kv8")
 
 
 def hca_compress(C_, Z, bias, entry0, cache, m_prime=128, stream=None):

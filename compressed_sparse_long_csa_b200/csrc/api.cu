@@ -14,6 +14,9 @@ cudaError_t launch_csa_compress(const void*, const void*, const void*, const voi
                                 int, cudaStream_t, unsigned*);
 cudaError_t launch_hca_compress(const void*, const void*, const float*, const int32_t*, void*, int64_t, int,
                                 int, int, int, int, cudaStream_t, unsigned*, int max_ctas);
+cudaError_t launch_csa_compress_kv8(const void*, const void*, const void*, const void*, const float*, const float*,
+                                    const void*, const void*, const int32_t*, void*, int64_t, int, int, int,
+                                    cudaStream_t, unsigned*);
 size_t out_proj_partial_elems(int T, int R_max);
 cudaError_t launch_grouped_out_proj(const void* o, int T, int H, int dv, int g, int d_mid, const void* W1,
                                     const void* W2, int d, void* u, void* y, float* part, size_t part_elems,
@@ -131,6 +134,22 @@ csa_status csa_compress(const void* Ca, const void* Cb, const void* Za, const vo
   REQUIRE(err, CSA_ERR_CUDA);
   return cuda_status(launch_csa_compress(Ca, Cb, Za, Zb, Ba, Bb, prev_Cb, prev_Zb, entry0, cache, n_max, B,
                                          T_new, d, m, dtype, S(stream), err));
+}
+
+csa_status csa_compress_kv8(const void* Ca, const void* Cb, const void* Za, const void* Zb, const float* Ba,
+                            const float* Bb, const void* prev_Cb, const void* prev_Zb, const int32_t* entry0,
+                            void* cache8, int64_t n_max, int B, int T_new, int d, int m, int dtype, void* stream) {
+  REQUIRE(dtype == CSA_F32 || dtype == CSA_BF16, CSA_ERR_DTYPE);
+  REQUIRE(B >= 1 && B <= 65535 && T_new >= 1 && n_max >= 1, CSA_ERR_SHAPE);
+  REQUIRE(d == 576 && m == 4, CSA_ERR_UNSUPPORTED);
+  REQUIRE(T_new % m == 0, CSA_ERR_SHAPE);
+  REQUIRE_PTR(Ca); REQUIRE_PTR(Cb); REQUIRE_PTR(Za); REQUIRE_PTR(Zb); REQUIRE_PTR(Ba); REQUIRE_PTR(Bb);
+  REQUIRE_PTR(prev_Cb); REQUIRE_PTR(prev_Zb); REQUIRE_PTR(cache8);
+  REQUIRE(entry0, CSA_ERR_NULL);
+  unsigned* err = device_error_word();
+  REQUIRE(err, CSA_ERR_CUDA);
+  return cuda_status(launch_csa_compress_kv8(Ca, Cb, Za, Zb, Ba, Bb, prev_Cb, prev_Zb, entry0, cache8, n_max, B,
+                                             T_new, dtype, S(stream), err));
 }
 
 csa_status hca_compress(const void* C, const void* Z, const float* bias, const int32_t* entry0, void* cache,

@@ -340,6 +340,103 @@ hca_compress_kernel(const T* __restrict__ C, const T* __restrict__ Z, const floa
   }
 }
 
+// ---- CSA compression into an FP8 cache ----------------------------------------------------
+// "Гибридный attention: CSA и HCA" of the aixai.ru digest: KV entries are stored in FP8,
+// only the RoPE dimensions in BF16.  One warp per entry pools its 576 components (chunk
+// lane + 32 p of VEC components, p = 0, 1, ...) with the m = 4 pooling above and writes the
+// 656-byte row: the e4m3 codes of x[0:512] * 2^-e (round to nearest even, saturating, +0 for
+// values that round to zero), x[512:576] as bf16 and the byte e + 127, where e is the
+// smallest integer with max|x[0:512]| <= 448 * 2^e (clamped to [-126, 127]): from the fields
+// of amax = f * 2^E (f in [1, 2)), 448 * 2^e = 1.75 * 2^(e+8), so e = E - 8 when f <= 1.75,
+// else E - 7.  The decisions are taken on the fp32 pooled values.
+__device__ __forceinline__ int kv8_exponent(float amax) {
+  const uint32_t u = __float_as_uint(amax);
+  const int E = (int)((u >> 23) & 0xFFu);
+  if (E == 0) return -126;                                // zero or subnormal: the smallest exponent
+  const int e = (u & 0x7FFFFFu) > 0x600000u ? E - 134 : E - 135;
+  return e < -126 ? -126 : (e > 127 ? 127 : e);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+csa_compress_kv8_kernel(const T* __restrict__ Ca, const T* __restrict__ Cb, const T* __restrict__ Za,
+                        const T* __restrict__ Zb, const float* __restrict__ Ba, const float* __restrict__ Bb,
+                        const T* __restrict__ pCb, const T* __restrict__ pZb, const int32_t* __restrict__ entry0,
+                        uint8_t* __restrict__ cache8, int64_t n_max, int T_new, unsigned* err) {
+  constexpr int VEC = Elem<T>::VEC, D = 576, NCH = D / VEC, NOPE = 512 / VEC, PER = (NCH + 31) / 32;
+  const int b = blockIdx.y, lane = threadIdx.x & 31;
+  const int j = (int)(((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  if (j >= T_new / 4) return;                            // whole warps
+  float x[PER][VEC];
+  int e = -1;
+#pragma unroll
+  for (int p = 0; p < PER; ++p) {
+    const int ch = lane + 32 * p;
+    if (ch < NCH) {
+      const int ep = pool_m4<T>(Ca, Cb, Za, Zb, Ba, Bb, pCb, pZb, entry0, n_max, T_new, D, b, j, ch * VEC, x[p], err);
+      if (p == 0) e = ep;
+    }
+  }
+  if (e < 0) return;                                      // the same for the whole warp
+  float amax = 0.f;
+#pragma unroll
+  for (int p = 0; p < PER; ++p)
+    if (lane + 32 * p < NOPE)
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) amax = fmaxf(amax, fabsf(x[p][i]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+  const int ex = kv8_exponent(amax);
+  const float inv = __uint_as_float((uint32_t)(127 - ex) << 23);    // 2^-ex, exact: 127 - ex in [0, 253]
+  uint8_t* row = cache8 + ((size_t)b * n_max + e) * 656;
+#pragma unroll
+  for (int p = 0; p < PER; ++p) {
+    const int ch = lane + 32 * p;
+    if (ch < NOPE) {
+      uint32_t w[VEC / 4];
+#pragma unroll
+      for (int q = 0; q < VEC / 4; ++q)
+        w[q] = e4m3x2_rn(x[p][4 * q] * inv, x[p][4 * q + 1] * inv) |
+               (e4m3x2_rn(x[p][4 * q + 2] * inv, x[p][4 * q + 3] * inv) << 16);
+      if (VEC == 8) *reinterpret_cast<uint2*>(row + ch * VEC) = make_uint2(w[0], w[VEC / 4 - 1]);
+      else *reinterpret_cast<uint32_t*>(row + ch * VEC) = w[0];
+    } else if (ch < NCH) {
+      uint32_t w[VEC / 2];
+#pragma unroll
+      for (int q = 0; q < VEC / 2; ++q) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(x[p][2 * q], x[p][2 * q + 1]);
+        w[q] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      uint8_t* dst = row + 512 + (ch - NOPE) * VEC * 2;
+      if (VEC == 8) *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1 % (VEC / 2)], w[2 % (VEC / 2)], w[3 % (VEC / 2)]);
+      else *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1 % (VEC / 2)]);
+    }
+  }
+  if (lane == 0) *reinterpret_cast<uint4*>(row + 640) = make_uint4((uint32_t)(ex + 127), 0u, 0u, 0u);
+}
+
+cudaError_t launch_csa_compress_kv8(const void* Ca, const void* Cb, const void* Za, const void* Zb, const float* Ba,
+                                    const float* Bb, const void* pCb, const void* pZb, const int32_t* entry0,
+                                    void* cache8, int64_t n_max, int B, int T_new, int dtype, cudaStream_t st,
+                                    unsigned* err) {
+  const int64_t warps = T_new / 4;
+  const int threads = warps < 8 ? (int)warps * 32 : 256;
+  dim3 grid((unsigned)((warps * 32 + threads - 1) / threads), B);
+  note_launch();
+  if (dtype == CSA_BF16) {
+    using T = __nv_bfloat16;
+    csa_compress_kv8_kernel<T><<<grid, threads, 0, st>>>((const T*)Ca, (const T*)Cb, (const T*)Za, (const T*)Zb, Ba,
+                                                         Bb, (const T*)pCb, (const T*)pZb, entry0, (uint8_t*)cache8,
+                                                         n_max, T_new, err);
+  } else {
+    csa_compress_kv8_kernel<float><<<grid, threads, 0, st>>>((const float*)Ca, (const float*)Cb, (const float*)Za,
+                                                             (const float*)Zb, Ba, Bb, (const float*)pCb,
+                                                             (const float*)pZb, entry0, (uint8_t*)cache8, n_max,
+                                                             T_new, err);
+  }
+  return cudaGetLastError();
+}
+
 cudaError_t launch_csa_compress(const void* Ca, const void* Cb, const void* Za, const void* Zb,
                                 const float* Ba, const float* Bb, const void* pCb, const void* pZb,
                                 const int32_t* entry0, void* cache, int64_t n_max, int B, int T_new,

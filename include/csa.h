@@ -110,6 +110,19 @@ csa_status csa_compress(const void* Ca, const void* Cb, const void* Za, const vo
                         const int32_t* entry0, void* cache, int64_t n_max,
                         int B, int T_new, int d, int m, int dtype, void* stream);
 
+/* csa_compress_kv8 — csa_compress (m = 4, d = 576) writing the FP8 cache rows that
+ * sparse_attn_decode_kv8 reads ("Гибридный attention: CSA и HCA" of the aixai.ru
+ * digest: KV entries in FP8, RoPE dimensions in BF16).  Row entry0[b] + i of
+ * cache8 [B, n_max, 656] receives the 656-byte form of the pooled fp32 row (layout
+ * and exponent rule at sparse_attn_decode_kv8); codes round to nearest even and
+ * saturate, a value that rounds to zero gets code 0.  Other arguments as csa_compress.
+ * Supported: d == 576 and m == 4 (CSA_ERR_UNSUPPORTED otherwise).                   */
+csa_status csa_compress_kv8(const void* Ca, const void* Cb, const void* Za, const void* Zb,
+                            const float* Ba, const float* Bb,
+                            const void* prev_Cb, const void* prev_Zb,
+                            const int32_t* entry0, void* cache8, int64_t n_max,
+                            int B, int T_new, int d, int m, int dtype, void* stream);
+
 /* ---------------------------------------------------------------------------
  * hca_compress — HCA compression ("HCA: сжать в 128 раз, но смотреть на всё":
  * the same gated pooling with m' tokens per entry and no overlap).

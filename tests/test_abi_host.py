@@ -25,7 +25,7 @@ def test_every_declared_symbol_is_exported():
     assert {"csa_compress", "hca_compress", "lightning_index", "topk_select", "sparse_attn_decode",
             "sparse_attn_prefill", "hca_attn_decode", "hca_compress_attn_decode", "index_key_compress",
             "lightning_index_bf16", "grouped_out_proj", "sparse_attn_decode_kv8",
-            "hca_attn_decode_kv8"} <= set(names)
+            "hca_attn_decode_kv8", "csa_compress_kv8"} <= set(names)
     for n in names:
         assert hasattr(N.lib, n), n
 
@@ -150,6 +150,22 @@ def test_grouped_out_proj_validation():
     assert N.lib.csa_launch_count() == before
     assert N.lib.grouped_out_proj_workspace_size(16, 16, 1024, 7168) == 8 * 16 * 16384 * 4
     assert N.lib.grouped_out_proj_workspace_size(4096, 16, 1024, 7168) == 0   # large batches need no split
+
+
+def test_kv8_compress_validation():
+    def call(**kw):
+        a = dict(d=576, m=4, dtype=1, T=16, c8=FAKE)
+        a.update(kw)
+        return N.lib.csa_compress_kv8(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, a["c8"], 64, 2, a["T"],
+                                      a["d"], a["m"], a["dtype"], None)
+    before = N.lib.csa_launch_count()
+    assert call(d=512) == ERR_UNSUP
+    assert call(m=8) == ERR_UNSUP
+    assert call(T=18) == ERR_SHAPE
+    assert call(c8=None) == ERR_NULL
+    assert call(c8=FAKE + 8) == ERR_ALIGN
+    assert call(dtype=5) == ERR_DTYPE
+    assert N.lib.csa_launch_count() == before
 
 
 def test_kv8_attention_validation():

@@ -101,3 +101,80 @@ def test_hca_decode_kv8(B, T):
         rows = np.concatenate([deq[b][:n_entries[b]], winn[b][:win_len[b]]], axis=0)
         o, _ = O.attention(qn[b], rows, wl.tensors["sink"].astype(np.float64), D["sm_scale"], dv)
         _check(out8[b].float().cpu().numpy(), o, f"kv8 dense b={b}")
+
+
+# ----------------------------------------------------------------------------- the FP8 writer
+
+def _compare_rows(g8, o8, x, tol_x):
+    """Stored bytes must match, except where the fp32 pooling error (tol_x per component)
+    can carry a value across a rounding midpoint (codes, bf16 RoPE) or the row maximum
+    across an exponent boundary 448 * 2^e."""
+    x32 = x.astype(np.float32).astype(np.float64)
+    ge, oe = g8[:, 640].astype(np.int64) - 127, o8[:, 640].astype(np.int64) - 127
+    assert not g8[:, 641:].any()
+    amax = np.abs(x32[:, :512]).max(axis=1)
+    tol_a = tol_x[:, :512].max(axis=1)
+    bad = ge != oe
+    near = (np.abs(amax - 448.0 * np.ldexp(1.0, oe)) <= tol_a) | (np.abs(amax - 448.0 * np.ldexp(1.0, oe - 1)) <= tol_a)
+    assert np.all(near[bad]), "row exponent differs away from a boundary"
+    flips = int(bad.sum()) * 512
+    ok = ~bad
+    gc, oc = g8[ok, :512].astype(np.int64), o8[ok, :512].astype(np.int64)
+    mism = gc != oc
+    if mism.any():
+        y = x32[ok, :512] * np.ldexp(1.0, -oe[ok])[:, None]
+        ty = tol_x[ok, :512] * np.ldexp(1.0, -oe[ok])[:, None]
+        gm, om = gc[mism] & 0x7F, oc[mism] & 0x7F
+        assert np.all(np.abs(gm - om) == 1), "codes more than one step apart"
+        mid = (O.E4M3_MAGS[gm] + O.E4M3_MAGS[om]) / 2
+        assert np.all(np.abs(np.abs(y[mism]) - mid) <= ty[mism]), "a code differs away from a midpoint"
+        flips += int(mism.sum())
+    gr = O.decode_bf16(np.ascontiguousarray(g8[:, 512:640]).view("<u2"))
+    orr = O.decode_bf16(np.ascontiguousarray(o8[:, 512:640]).view("<u2"))
+    rm = gr != orr
+    if rm.any():
+        mid = (gr[rm] + orr[rm]) / 2
+        assert np.all(np.abs(x32[:, 512:][rm] - mid) <= tol_x[:, 512:][rm]), "a RoPE value differs away from a midpoint"
+        flips += int(rm.sum())
+    return flips
+
+
+@pytest.mark.parametrize("B,T_new,entry0,dtype", [
+    (16, 4, [0, 1, 63, 17, 2, 30, 31, 32, 5, 6, 62, 40, 41, 3, 9, 12], "bf16"),   # the decode append
+    (2, 1024, [8192, 0], "bf16"),                                               # a chunk of 256 entries
+    (3, 36, [0, 4, 100], "f32"),
+])
+def test_csa_compress_kv8(B, T_new, entry0, dtype):
+    n = T_new // 4
+    n_max = max(entry0) + n
+    t = CI.index_key_inputs(61 + B, B, T_new, 576, dtype, spread=4.0)
+    dev = {k: (torch.from_numpy(np.ascontiguousarray(v)).cuda() if v.dtype == np.float32
+               else _bf16_dev(v)) for k, v in t.items()}
+    c8 = torch.full((B, n_max, 656), 0xAB, dtype=torch.uint8, device="cuda")
+    e0 = torch.tensor(entry0, dtype=torch.int32, device="cuda")
+    csa.csa_compress_kv8(dev["Ca"], dev["Cb"], dev["Za"], dev["Zb"], dev["Ba"], dev["Bb"], dev["prev_Cb"],
+                         dev["prev_Zb"], e0, c8)
+    torch.cuda.synchronize()
+    assert csa.read_device_error() == 0
+    g = c8.cpu().numpy()
+    flips = 0
+    for b in range(B):
+        ld = lambda a: O.load(a, dtype)
+        x = O.csa_compress(ld(t["Ca"][b]), ld(t["Cb"][b]), ld(t["Za"][b]), ld(t["Zb"][b]),
+                           t["Ba"].astype(np.float64), t["Bb"].astype(np.float64), ld(t["prev_Cb"][b]),
+                           ld(t["prev_Zb"][b]), entry0[b])
+        srcmax = []
+        for j in range(n):
+            a = np.abs(ld(t["Ca"][b, 4 * j:4 * j + 4])).max(axis=0)
+            if j > 0:
+                a = np.maximum(a, np.abs(ld(t["Cb"][b, 4 * j - 4:4 * j])).max(axis=0))
+            elif entry0[b] > 0:
+                a = np.maximum(a, np.abs(ld(t["prev_Cb"][b])).max(axis=0))
+            srcmax.append(a)
+        tol_x = 4e-6 * np.stack(srcmax)
+        rows = slice(entry0[b], entry0[b] + n)
+        flips += _compare_rows(g[b, rows], O.quantise_latent_fp8(x), x, tol_x)
+        keep = np.ones(n_max, bool)
+        keep[rows] = False
+        assert np.all(g[b, keep] == 0xAB)
+    assert flips <= 1e-3 * B * n * 576, flips
