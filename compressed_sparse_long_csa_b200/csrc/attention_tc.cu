@@ -159,6 +159,9 @@ __device__ __forceinline__ void kv8_expand(uint32_t kv0, const uint32_t* k8mask,
 // TMEM: O at lane offset 0, columns [0, 512); S buffers at lane offset 16, columns 0 and 64.
 constexpr uint32_t TM_S_LANE = 16u << 16, TM_COLS = 512;
 
+// KV8: the cache rows are FP8 rows (a separate instance, so that the bf16 gather loop
+// carries no test for them).
+template <bool KV8>
 __global__ void __launch_bounds__(AT_THREADS, 1)
 attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -244,7 +247,7 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
       const bool go = tc::mbar_wait(&sm.empty[g], (i & 1) ^ 1) && !*(volatile int*)&sm.abort_flag;
       if (!go) sm.ld_stop[g] = i + 1;      // the group leaves together at this iteration's barrier
       if (lg < AT_ROWS) {
-        const bool r8 = a.kv8 && which == 0;                 // an FP8 cache row
+        const bool r8 = KV8 && which == 0;                   // an FP8 cache row
         const __nv_bfloat16* base = which == 1 ? (const __nv_bfloat16*)a.win : (const __nv_bfloat16*)a.cache;
         sm.rowp[g][lg] = which < 0 ? nullptr
                          : r8 ? reinterpret_cast<const __nv_bfloat16*>((const uint8_t*)a.cache + (size_t)y * KV8_ROW)
@@ -283,7 +286,7 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
         }
       } else {
         const uint32_t kv0 = tc::smem_u32(sm.kv[g][0]);
-        const bool any8 = (sm.k8mask[g][0] | sm.k8mask[g][1]) != 0u;
+        const bool any8 = KV8 && (sm.k8mask[g][0] | sm.k8mask[g][1]) != 0u;
         for (int p = lg; p < AT_ROWS * AT_CHUNKS; p += AT_GROUP) {
           const int j = p / AT_CHUNKS, c = p - j * AT_CHUNKS;
           const __nv_bfloat16* rp = sm.rowp[g][j];
@@ -305,7 +308,7 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
       if (it + 2 < n_t) coord(it + 2);
       if (!run) {
         cp_async_wait_all();
-        if ((sm.k8mask[g][0] | sm.k8mask[g][1]) != 0u) {   // the same for the whole group
+        if (KV8 && (sm.k8mask[g][0] | sm.k8mask[g][1]) != 0u) {   // the same for the whole group
           named_bar(1 + g, AT_GROUP);                         // every thread's copies have landed
           kv8_expand(tc::smem_u32(sm.kv[g][0]), sm.k8mask[g], lg);
         }
@@ -770,7 +773,8 @@ cudaError_t launch_attention_tc(AttnArgs a, cudaStream_t st, bool* used, bool* c
     maps.win = maps.cache;                           // no row is ever resolved to the window tensor
   }
   const size_t smem = sizeof(AtSmem) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = a.kv8 ? attn_tc_kernel<true> : attn_tc_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * a.splits, a.B * a.Tq);
@@ -790,20 +794,21 @@ cudaError_t launch_attention_tc(AttnArgs a, cudaStream_t st, bool* used, bool* c
   if (a.splits >= 2 && a.splits <= 8) {
     // merge the splits in a cluster when such clusters fit (checked once per split count)
     static std::mutex mu;
-    static std::map<int, bool> fits;
+    static std::map<std::pair<int, int>, bool> fits;
     std::lock_guard<std::mutex> g(mu);
-    auto it = fits.find(a.splits);
+    const auto key = std::make_pair(a.splits, a.kv8);
+    auto it = fits.find(key);
     if (it == fits.end()) {
       int n = 0;
-      const bool ok = cudaOccupancyMaxActiveClusters(&n, attn_tc_kernel, &cfg) == cudaSuccess && n > 0;
+      const bool ok = cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n > 0;
       cudaGetLastError();
-      it = fits.emplace(a.splits, ok).first;
+      it = fits.emplace(key, ok).first;
     }
     a.cluster_combine = it->second ? 1 : 0;
   }
   cfg.numAttrs = a.cluster_combine ? 2 : 1;
   note_launch();
-  e = cudaLaunchKernelEx(&cfg, attn_tc_kernel, maps, a);
+  e = cudaLaunchKernelEx(&cfg, kern, maps, a);
   *used = true;
   *combined = a.cluster_combine != 0;
   return e;
