@@ -36,10 +36,10 @@ METRIC = "CSA/HCA decode tokens/s and HBM GB/s (% roofline) at 64K-1M ctx; prefi
 # DRAM bytes (read + write) per call of the dominant ABI call, summed over its kernels, from
 # the ncu captures summarised under profiles/ (None until a capture of the current kernels).
 TRAFFIC = {
-    # profiles/csa_decode_64k_dram_traffic.md: indexer_tc_kernel 34 768 384 + select 1 378 304 bytes
-    ("csa_decode_64k", "indexer"): 36146688,
-    # profiles/hybrid_pair_1m_launches.md: indexer_mxf4_kernel 142 870 272 + 7 044 608, select 8 668 672
-    ("hybrid_pair_1m", "indexer"): 158583552,
+    # profiles/csa_decode_64k_dram_traffic.md: indexer_tc_kernel 34 768 896 + select 1 378 304 bytes
+    ("csa_decode_64k", "indexer"): 36147200,
+    # profiles/hybrid_pair_1m_launches.md: indexer_mxf4_kernel 144 098 816 + 7 310 592, select 8 669 952
+    ("hybrid_pair_1m", "indexer"): 160079360,
     # profiles/hca_decode_1m_launches.md: attn_tc_kernel 38 996 736 (the combine's reads are L2 hits
     # in the timed step; under ncu the caches are flushed before each kernel)
     ("hca_decode_1m", "attention"): 38996736,
