@@ -25,6 +25,8 @@ _SIGS = {
     "csa_compress": ([_vp] * 10 + [_i64, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
     "csa_compress_kv8": ([_vp] * 10 + [_i64, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
     "index_key_compress": ([_vp] * 11 + [_i64, _i32, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
+    "shard_topk_merge": ([_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp], _i32),
+    "attn_merge_shards": ([_vp, _vp, _i32, _i64, _i32, _i32, _vp, _vp, _vp], _i32),
     "grouped_out_proj_workspace_size": ([_i32, _i32, _i32, _i32], _sz),
     "grouped_out_proj": ([_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp], _i32),
     "hca_compress": ([_vp] * 5 + [_i64, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
@@ -98,6 +100,22 @@ def index_key_compress(Ca, Cb, Za, Zb, Ba, Bb, prev_Cb, prev_Zb, entry0, kI, kI_
     _check(lib.index_key_compress(_p(Ca), _p(Cb), _p(Za), _p(Zb), _p(Ba), _p(Bb), _p(prev_Cb), _p(prev_Zb),
                                   _p(entry0), _p(kI), _p(kI_scale), kI.shape[1], B, T_new, d_I, m,
                                   _dtype_code(Ca), ifmt, _stream(stream)), "index_key_compress")
+
+
+def shard_topk_merge(idx_parts, score_parts, bounds, local_idx_out, stream=None):
+    """idx_parts / score_parts [G, R, k]; bounds [G+1] int32; local_idx_out [G, R, k]."""
+    G, R, k = idx_parts.shape
+    _check(lib.shard_topk_merge(_p(idx_parts), _p(score_parts), _p(bounds), G, R, k, _p(local_idx_out),
+                                _stream(stream)), "shard_topk_merge")
+
+
+def attn_merge_shards(o_parts, lse_parts, out, lse_out=None, stream=None):
+    """o_parts [G, rows, dv] (any leading shape flattened to rows); lse_parts [G, rows]."""
+    G = o_parts.shape[0]
+    dv = o_parts.shape[-1]
+    rows = o_parts[0].numel() // dv
+    _check(lib.attn_merge_shards(_p(o_parts), _p(lse_parts), G, rows, dv, _dtype_code(o_parts), _p(out),
+                                 _p(lse_out), _stream(stream)), "attn_merge_shards")
 
 
 def grouped_out_proj_workspace_size(T, g, d_mid, d):

@@ -17,6 +17,9 @@ cudaError_t launch_hca_compress(const void*, const void*, const float*, const in
 cudaError_t launch_csa_compress_kv8(const void*, const void*, const void*, const void*, const float*, const float*,
                                     const void*, const void*, const int32_t*, void*, int64_t, int, int, int,
                                     cudaStream_t, unsigned*);
+cudaError_t launch_shard_topk_merge(const int32_t*, const float*, const int32_t*, int, int, int, int32_t*,
+                                    cudaStream_t);
+cudaError_t launch_attn_merge_shards(const void*, const float*, int, int64_t, int, int, void*, float*, cudaStream_t);
 size_t out_proj_partial_elems(int T, int R_max);
 cudaError_t launch_grouped_out_proj(const void* o, int T, int H, int dv, int g, int d_mid, const void* W1,
                                     const void* W2, int d, void* u, void* y, float* part, size_t part_elems,
@@ -281,6 +284,22 @@ csa_status topk_select(const float* scores, int64_t ld, const int32_t* n_valid, 
   RowCount rc;
   rc.n_valid = n_valid;
   return cuda_status(launch_topk_select(scores, ld, rc, R, n, k, idx_out, S(stream), err));
+}
+
+// ----------------------------------------------------------------------------- KV-sharded decode
+csa_status shard_topk_merge(const int32_t* idx_parts, const float* score_parts, const int32_t* bounds, int G, int R,
+                            int k, int32_t* local_idx_out, void* stream) {
+  REQUIRE(G >= 1 && G <= 8 && R >= 1 && R <= 65535 && k >= 1 && (int64_t)G * k <= 4096, CSA_ERR_SHAPE);
+  REQUIRE(idx_parts && score_parts && bounds && local_idx_out, CSA_ERR_NULL);
+  return cuda_status(launch_shard_topk_merge(idx_parts, score_parts, bounds, G, R, k, local_idx_out, S(stream)));
+}
+
+csa_status attn_merge_shards(const void* o_parts, const float* lse_parts, int G, int64_t rows, int dv, int dtype,
+                             void* out, float* lse_out, void* stream) {
+  REQUIRE(dtype == CSA_F32 || dtype == CSA_BF16, CSA_ERR_DTYPE);
+  REQUIRE(G >= 1 && G <= 64 && rows >= 1 && rows <= (1LL << 31) && dv >= 1 && dv <= 4096, CSA_ERR_SHAPE);
+  REQUIRE(o_parts && lse_parts && out, CSA_ERR_NULL);
+  return cuda_status(launch_attn_merge_shards(o_parts, lse_parts, G, rows, dv, dtype, out, lse_out, S(stream)));
 }
 
 // ----------------------------------------------------------------------------- output projection

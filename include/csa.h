@@ -172,6 +172,35 @@ csa_status index_key_compress(const void* Ca, const void* Cb, const void* Za, co
                               int B, int T_new, int d_I, int m, int dtype, int ifmt, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * KV-sharded decode of one sequence over G GPUs: the two merge steps.  The
+ * entries are split into G contiguous shards (shard g holds global entries
+ * bounds[g] .. bounds[g+1]-1).  Every GPU runs lightning_index on its shard with
+ * score_out, the candidates are all-gathered, and:
+ *
+ * shard_topk_merge — the global top-k ("Гибридное внимание: CSA и HCA", CSA step 2:
+ *   the k largest scores, ties to the lower entry id) of the G x k candidates.
+ *     idx_parts   device [G, R, k] int32 local ids (-1 = no candidate)
+ *     score_parts device [G, R, k] fp32 their scores (lightning_index score_out)
+ *     bounds      device [G + 1] int32 shard boundaries (global entry ids)
+ *     local_idx_out device [G, R, k] int32: for shard g, the selected entries of
+ *                 that shard as local ids in ascending order, -1 padded
+ *   Supported: G <= 8, G * k <= 4096, R <= 65535.
+ *
+ * attn_merge_shards — the attention over the union of the shards' rows from the
+ *   shards' outputs o_g (each normalised over its own rows) and their lse_g:
+ *   out = sum_g e^{lse_g - L} o_g, L = log sum_g e^{lse_g} (written to lse_out if
+ *   not NULL).  The sink and the window belong to one shard; the others pass a
+ *   very negative finite sink (e.g. -1e30), so that a shard without rows returns
+ *   o = 0 with lse = -1e30 and weighs nothing.
+ *     o_parts device [G, rows, dv] dtype;  lse_parts device [G, rows] fp32
+ *     out device [rows, dv] dtype (rows = B * H)
+ * ------------------------------------------------------------------------- */
+csa_status shard_topk_merge(const int32_t* idx_parts, const float* score_parts, const int32_t* bounds,
+                            int G, int R, int k, int32_t* local_idx_out, void* stream);
+csa_status attn_merge_shards(const void* o_parts, const float* lse_parts, int G, int64_t rows, int dv,
+                             int dtype, void* out, float* lse_out, void* stream);
+
+/* ---------------------------------------------------------------------------
  * grouped_out_proj — the grouped output projection after the attention
  * ("Гибридное внимание: CSA и HCA", CSA step 4: the n_h head outputs are split
  * into g groups, each group is projected to an intermediate width d_mid, and the

@@ -25,7 +25,7 @@ def test_every_declared_symbol_is_exported():
     assert {"csa_compress", "hca_compress", "lightning_index", "topk_select", "sparse_attn_decode",
             "sparse_attn_prefill", "hca_attn_decode", "hca_compress_attn_decode", "index_key_compress",
             "lightning_index_bf16", "grouped_out_proj", "sparse_attn_decode_kv8",
-            "hca_attn_decode_kv8", "csa_compress_kv8"} <= set(names)
+            "hca_attn_decode_kv8", "csa_compress_kv8", "shard_topk_merge", "attn_merge_shards"} <= set(names)
     for n in names:
         assert hasattr(N.lib, n), n
 
@@ -150,6 +150,17 @@ def test_grouped_out_proj_validation():
     assert N.lib.csa_launch_count() == before
     assert N.lib.grouped_out_proj_workspace_size(16, 16, 1024, 7168) == 8 * 16 * 16384 * 4
     assert N.lib.grouped_out_proj_workspace_size(4096, 16, 1024, 7168) == 0   # large batches need no split
+
+
+def test_shard_merge_validation():
+    before = N.lib.csa_launch_count()
+    assert N.lib.shard_topk_merge(FAKE, FAKE, FAKE, 9, 4, 64, FAKE, None) == ERR_SHAPE      # at most 8 shards
+    assert N.lib.shard_topk_merge(FAKE, FAKE, FAKE, 4, 4, 2048, FAKE, None) == ERR_SHAPE   # G * k <= 4096
+    assert N.lib.shard_topk_merge(FAKE, FAKE, None, 2, 4, 64, FAKE, None) == ERR_NULL
+    assert N.lib.attn_merge_shards(FAKE, FAKE, 2, 64, 512, 7, FAKE, None, None) == ERR_DTYPE
+    assert N.lib.attn_merge_shards(FAKE, None, 2, 64, 512, 1, FAKE, None, None) == ERR_NULL
+    assert N.lib.attn_merge_shards(FAKE, FAKE, 0, 64, 512, 1, FAKE, None, None) == ERR_SHAPE
+    assert N.lib.csa_launch_count() == before
 
 
 def test_kv8_compress_validation():
