@@ -391,14 +391,19 @@ def run_ours(args, wid):
         achieved = ab[dom] / (dom_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak, "peak_source": src, "traffic": TRAFFIC.get((args.workload, dom))}
-    extra = measure_index_keys(wid, D, csa, l2_flush, hbm_peak, src)
-    bf = measure_bf16_index(wid, D, T, csa, steps, l2_flush, float(mean_ms[comp.index("indexer")]))
-    if bf:
-        extra = dict(extra or {}, **bf)
-    extra = dict(extra or {}, **measure_out_proj(D, T, csa, l2_flush, hbm_peak, bf16_peak, src))
-    kv = measure_kv8_attention(wid, wl, D, T, csa, l2_flush, float(mean_ms[comp.index("attention")]), hbm_peak, src)
-    if kv:
-        extra.update(kv)
+    extra = None
+    if world == 1:
+        # the rows beyond the step, each timed alone on this GPU (single-GPU characterisations:
+        # a multi-rank run skips them)
+        extra = measure_index_keys(wid, D, csa, l2_flush, hbm_peak, src)
+        bf = measure_bf16_index(wid, D, T, csa, steps, l2_flush, float(mean_ms[comp.index("indexer")]))
+        if bf:
+            extra = dict(extra or {}, **bf)
+        extra = dict(extra or {}, **measure_out_proj(D, T, csa, l2_flush, hbm_peak, bf16_peak, src))
+        kv = measure_kv8_attention(wid, wl, D, T, csa, l2_flush, float(mean_ms[comp.index("attention")]), hbm_peak,
+                                   src)
+        if kv:
+            extra.update(kv)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
