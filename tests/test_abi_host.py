@@ -30,6 +30,20 @@ def test_every_declared_symbol_is_exported():
         assert hasattr(N.lib, n), n
 
 
+def test_header_is_plain_c(tmp_path):
+    """The boundary is a C ABI: the header compiles as C99 with no C++ in it."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "h.c"
+    src.write_text('#include "%s"\nint main(void) { return csa_abi_version() > 0 ? 0 : 1; }\n' % HDR)
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-fsyntax-only", str(src)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+
+
 def test_launch_counter_is_host_side_and_ignores_refused_calls():
     before = N.lib.csa_launch_count()
     assert N.lib.topk_select(None, 100, None, 4, 100, 8, FAKE, None, 0, None) == ERR_NULL
