@@ -58,3 +58,17 @@ def test_fp8_latent_rows_of_the_generator_match_the_oracle_format():
     x = torch.randn(64, 576, generator=g) * torch.exp(torch.randn(64, 1, generator=g) * 4)
     x[9] = 0.0
     assert np.array_equal(CI.quant_latent_fp8_rows(x), O.quantise_latent_fp8(x.double().numpy()))
+
+
+def test_added_generators_are_seeded_and_shaped():
+    a = CI.index_key_inputs(3, 2, 8, 128, "bf16", spread=4.0)
+    b = CI.index_key_inputs(3, 2, 8, 128, "bf16", spread=4.0)
+    assert all(np.array_equal(a[k], b[k]) for k in a)
+    assert a["Ca"].shape == (2, 8, 128) and a["Ca"].dtype == np.uint16
+    assert a["prev_Cb"].shape == (2, 4, 128) and a["Ba"].shape == (4, 128) and a["Ba"].dtype == np.float32
+    c = CI.index_key_inputs(4, 2, 8, 128, "bf16")
+    assert not np.array_equal(a["Ca"], c["Ca"])
+    x = CI.out_proj_inputs(5, 3, H=8, dv=16, g=4, d_mid=128, d=256)
+    assert x["o"].shape == (3, 8, 16) and x["W1"].shape == (512, 32) and x["W2"].shape == (256, 512)
+    y = CI.out_proj_inputs(5, 3, H=8, dv=16, g=4, d_mid=128, d=256)
+    assert all(np.array_equal(x[k], y[k]) for k in x)

@@ -149,3 +149,12 @@ def test_sharded_decode_equals_unsharded(tmp_path, world, dead_shard):
         np.testing.assert_allclose(out[b], o, rtol=1e-10, atol=1e-12)
     if dead_shard:
         assert not (sel[1] >= 0).any()                      # the second shard selected nothing
+
+
+def test_shard_bounds_cover_the_entries_contiguously():
+    from compressed_sparse_long_csa_b200 import sharded as S
+    for n, G in [(16384, 2), (16384, 3), (7, 4), (262144, 8)]:
+        b = S.shard_bounds(n, G)
+        assert b[0] == 0 and b[-1] == n and len(b) == G + 1
+        sizes = [b[g + 1] - b[g] for g in range(G)]
+        assert min(sizes) >= 0 and max(sizes) - min(sizes) <= 1
