@@ -44,6 +44,28 @@ def test_header_is_plain_c(tmp_path):
     assert r.returncode == 0, r.stderr
 
 
+def test_c_program_links_every_declared_call(tmp_path):
+    """A plain C program that takes the address of every declared call links against the
+    shared library and runs (csa_abi_version is host-only, so no GPU is needed)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    libdir = os.path.dirname(csa.lib_path)
+    names = declared_functions()
+    src = tmp_path / "link.c"
+    src.write_text('#include "%s"\nint main(void) {\n  const void* f[] = {%s};\n'
+                   '  unsigned i;\n  for (i = 0; i < sizeof f / sizeof f[0]; ++i) if (!f[i]) return 2;\n'
+                   '  return csa_abi_version() == %d ? 0 : 1;\n}\n'
+                   % (HDR, ", ".join("(const void*)%s" % n for n in names), N.lib.csa_abi_version()))
+    exe = tmp_path / "link"
+    r = subprocess.run([cc, "-std=c99", str(src), "-o", str(exe), "-L" + libdir, "-lcsa_b200",
+                        "-Wl,--allow-shlib-undefined", "-Wl,-rpath," + libdir], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    assert subprocess.run([str(exe)]).returncode == 0
+
+
 def test_launch_counter_is_host_side_and_ignores_refused_calls():
     before = N.lib.csa_launch_count()
     assert N.lib.topk_select(None, 100, None, 4, 100, 8, FAKE, None, 0, None) == ERR_NULL
