@@ -72,3 +72,25 @@ def test_added_generators_are_seeded_and_shaped():
     assert x["o"].shape == (3, 8, 16) and x["W1"].shape == (512, 32) and x["W2"].shape == (256, 512)
     y = CI.out_proj_inputs(5, 3, H=8, dv=16, g=4, d_mid=128, d=256)
     assert all(np.array_equal(x[k], y[k]) for k in x)
+
+
+def test_row_quantisers_of_the_generator_match_the_oracle():
+    """The generator's E4M3 and MXFP4 row quantisers (torch casts, its own e2m1 rounding)
+    and the oracle's key quantiser (its own nearest-grid encoders and exponent search)
+    agree on the same fp32 rows, up to the sign of a value that rounds to zero."""
+    import torch
+    from oracle import csa_oracle as O
+    g = torch.Generator().manual_seed(8)
+    x = torch.randn(40, 128, generator=g) * torch.exp(torch.randn(40, 1, generator=g) * 3)
+    x[3] = 0.0
+    c_gen, s_gen = CI.quant_e4m3_rows(x)
+    c_orc, s_orc, _ = O.quantise_index_keys(x.double().numpy(), "e4m3")
+    assert np.array_equal(s_gen, s_orc)
+    assert np.array_equal(np.where(c_gen == 0x80, 0, c_gen), c_orc)
+    p_gen, e_gen = CI.quant_mxfp4_rows(x)
+    p_orc, e_orc, _ = O.quantise_index_keys(x.double().numpy(), "mxfp4")
+    assert np.array_equal(e_gen, e_orc)
+    lo, hi = p_gen & 0xF, p_gen >> 4
+    lo = np.where(lo == 0x8, 0, lo)
+    hi = np.where(hi == 0x8, 0, hi)
+    assert np.array_equal((lo | (hi << 4)).astype(np.uint8), p_orc)
