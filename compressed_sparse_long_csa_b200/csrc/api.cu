@@ -289,7 +289,8 @@ csa_status topk_select(const float* scores, int64_t ld, const int32_t* n_valid, 
 // ----------------------------------------------------------------------------- KV-sharded decode
 csa_status shard_topk_merge(const int32_t* idx_parts, const float* score_parts, const int32_t* bounds, int G, int R,
                             int k, int32_t* local_idx_out, void* stream) {
-  REQUIRE(G >= 1 && G <= 8 && R >= 1 && R <= 65535 && k >= 1 && (int64_t)G * k <= 4096, CSA_ERR_SHAPE);
+  REQUIRE(G >= 1 && G <= CSA_SHARD_MAX_G && R >= 1 && R <= 65535 && k >= 1 && (int64_t)G * k <= CSA_SHARD_MAX_CANDIDATES,
+          CSA_ERR_SHAPE);
   REQUIRE(idx_parts && score_parts && bounds && local_idx_out, CSA_ERR_NULL);
   return cuda_status(launch_shard_topk_merge(idx_parts, score_parts, bounds, G, R, k, local_idx_out, S(stream)));
 }
@@ -297,7 +298,7 @@ csa_status shard_topk_merge(const int32_t* idx_parts, const float* score_parts, 
 csa_status attn_merge_shards(const void* o_parts, const float* lse_parts, int G, int64_t rows, int dv, int dtype,
                              void* out, float* lse_out, void* stream) {
   REQUIRE(dtype == CSA_F32 || dtype == CSA_BF16, CSA_ERR_DTYPE);
-  REQUIRE(G >= 1 && G <= 64 && rows >= 1 && rows <= (1LL << 31) && dv >= 1 && dv <= 4096, CSA_ERR_SHAPE);
+  REQUIRE(G >= 1 && G <= CSA_SHARD_MAX_G && rows >= 1 && rows <= (1LL << 31) && dv >= 1 && dv <= 4096, CSA_ERR_SHAPE);
   REQUIRE(o_parts && lse_parts && out, CSA_ERR_NULL);
   return cuda_status(launch_attn_merge_shards(o_parts, lse_parts, G, rows, dv, dtype, out, lse_out, S(stream)));
 }

@@ -13,13 +13,15 @@
 // which is the attention over the union of the rows (CSA step 3).
 #include <cuda_bf16.h>
 
+#include "../../include/csa.h"
 #include "common.cuh"
 
 namespace csa {
 namespace {
 
 constexpr int SM_THREADS = 512;
-constexpr int SM_CAP = 4096;          // G * k candidates per row at most
+constexpr int SM_CAP = CSA_SHARD_MAX_CANDIDATES;   // G * k candidates per row at most
+static_assert(CSA_SHARD_MAX_G <= 8, "per-shard counts cnt[] below hold G + 1 entries");
 
 // In-place ascending bitonic sort of n (a power of two, <= SM_CAP) keys in shared memory.
 __device__ void bitonic_sort(unsigned long long* key, int n) {
@@ -46,7 +48,7 @@ __global__ void __launch_bounds__(SM_THREADS)
 shard_topk_merge_kernel(const int32_t* __restrict__ idx_parts, const float* __restrict__ score_parts,
                         const int32_t* __restrict__ bounds, int G, int R, int k, int32_t* __restrict__ local_out) {
   __shared__ unsigned long long key[SM_CAP];
-  __shared__ int cnt[9];
+  __shared__ int cnt[CSA_SHARD_MAX_G + 1];
   const int row = blockIdx.x;
   const int n = G * k;
   int np = 1;

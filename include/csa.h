@@ -184,7 +184,7 @@ csa_status index_key_compress(const void* Ca, const void* Cb, const void* Za, co
  *     bounds      device [G + 1] int32 shard boundaries (global entry ids)
  *     local_idx_out device [G, R, k] int32: for shard g, the selected entries of
  *                 that shard as local ids in ascending order, -1 padded
- *   Supported: G <= 8, G * k <= 4096, R <= 65535.
+ *   Supported: G <= CSA_SHARD_MAX_G, G * k <= CSA_SHARD_MAX_CANDIDATES, R <= 65535.
  *
  * attn_merge_shards — the attention over the union of the shards' rows from the
  *   shards' outputs o_g (each normalised over its own rows) and their lse_g:
@@ -194,7 +194,10 @@ csa_status index_key_compress(const void* Ca, const void* Cb, const void* Za, co
  *   o = 0 with lse = -1e30 and weighs nothing.
  *     o_parts device [G, rows, dv] dtype;  lse_parts device [G, rows] fp32
  *     out device [rows, dv] dtype (rows = B * H)
+ * Both calls accept 1 <= G <= CSA_SHARD_MAX_G (CSA_ERR_SHAPE otherwise).
  * ------------------------------------------------------------------------- */
+#define CSA_SHARD_MAX_G 8                 /* shards G of one sequence, both merges       */
+#define CSA_SHARD_MAX_CANDIDATES 4096     /* G * k of shard_topk_merge                   */
 csa_status shard_topk_merge(const int32_t* idx_parts, const float* score_parts, const int32_t* bounds,
                             int G, int R, int k, int32_t* local_idx_out, void* stream);
 csa_status attn_merge_shards(const void* o_parts, const float* lse_parts, int G, int64_t rows, int dv,
@@ -404,7 +407,12 @@ csa_status sparse_attn_prefill(const void* q, const int32_t* q_pos, const void* 
  *   about 17 MB.
  * - The first call on each device looks up the buffer's device address
  *   (cudaGetSymbolAddress, with that device current); make that first call
- *   before any stream capture.  Later calls only read the cached address.
+ *   before any stream capture: inside a capture the lookup can fail, and the
+ *   call then returns CSA_ERR_CUDA.  Later calls only read the cached address.
+ * - The cached address belongs to the device's primary context: after
+ *   cudaDeviceReset on that device the address is stale, and so is the error
+ *   word every call uses.  Do not call the library after a reset in the same
+ *   process.
  * - All calls on a device share the one buffer, and it keeps the last call's
  *   contents.  Every call rewrites all it reads, so nothing must be cleared.
  *   Calls that overlap on the GPU (different streams, or different host threads
