@@ -1,16 +1,20 @@
 """Throughput of the CSA / HCA hot path on B200.
 
-Default workload: CSA decode, batch 16 sequences at a 65,536-token context
-(16,384 compressed entries, m = 4), 128 query heads of width 576/512, FP8
-indexer with 64 heads of width 128, top-k 512, window 128, attention sink.  A
-step is one decode token for every sequence: csa_compress (the block the token
-completes) -> lightning_index (scores + exact top-k) -> sparse_attn_decode
-(+ split combine).  Inputs are synthetic (seeded) and resident in HBM; L2 is
-flushed before every timed step.
+By default every workload runs in one invocation and prints one JSON line each:
+HCA decode at 1M context, the CSA prefill chunk, the hybrid pair at 1M context, and
+last the headline, CSA decode at a 64K context (batch 16 sequences, 16,384
+compressed entries, m = 4, 128 query heads of width 576/512, FP8 indexer with 64
+heads of width 128, top-k 512, window 128, attention sink).  A decode step is one
+token for every sequence: csa_compress (the block the token completes) ->
+lightning_index (scores + exact top-k) -> sparse_attn_decode (+ split combine);
+the HCA step compresses the fresh 128-token chunk and attends to every entry; the
+prefill step compresses the 4096-token chunk, selects per query and attends.
+Inputs are synthetic (seeded) and resident in HBM; L2 is flushed before every
+timed step.  ``--workload NAME`` runs one workload.
 
 --impl reference times the fp64 CPU oracle on the host cores on a bounded sample
-of the same workload.  Under torchrun each rank runs its own batch (independent
-sequences: weak scaling, no data-path collective); rank 0 prints one JSON line.
+of the same workloads.  Under torchrun each rank runs its own batch (independent
+sequences: weak scaling, no data-path collective); rank 0 prints the lines.
 """
 from __future__ import annotations
 
@@ -157,7 +161,7 @@ def job_rate(units_per_rank, world, ms):
     return units_per_rank * world / (ms * 1e-3)
 
 
-def run_reference(args, wid):
+def run_reference(args, wid, name):
     """Time the fp64 oracle on host cores on a bounded sample of the workload."""
     import numpy as np
     import csa_inputs as CI
@@ -169,7 +173,7 @@ def run_reference(args, wid):
     wl = CI.make_workload(wid, scale=scale)
     D = wl.dims
     cores = os.cpu_count()
-    sample_b = list(range(min(D["B"], 4)))
+    sample_b = list(range(min(D["B"], 1 if wid == 4 else 4)))   # the pair's MXFP4 decode costs ~1 s a sequence
     sample_rows = [int(r) for r in np.linspace(0, D["Tq"] - 1, 4)] if wid == 3 else []
     t0 = time.perf_counter()
     steps_done = 0
@@ -191,35 +195,35 @@ def run_reference(args, wid):
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dt / steps_done * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(WORKLOAD_NAME, D),
+            "config": workload_config(name, D),
             "impl": "reference",
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-WORKLOAD_NAME = "csa_decode_64k"
+# the order of the lines of a default run: the headline workload comes last
+ORDER = ["hca_decode_1m", "csa_prefill_4k", "hybrid_pair_1m", "csa_decode_64k"]
 
 
 def main():
-    global WORKLOAD_NAME
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="csa_decode_64k", choices=list(WORKLOADS))
+    ap.add_argument("--workload", default="all", choices=["all"] + list(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
-    WORKLOAD_NAME = args.workload
-    wid = WORKLOADS[args.workload]
-    if args.impl == "reference":
-        run_reference(args, wid)
-        return
-    run_ours(args, wid)
+    names = ORDER if args.workload == "all" else [args.workload]
+    for name in names:
+        if args.impl == "reference":
+            run_reference(args, WORKLOADS[name], name)
+        else:
+            run_ours(args, WORKLOADS[name], name)
 
 
-def run_ours(args, wid):
+def run_ours(args, wid, name):
     import numpy as np
     import torch
     import torch.distributed as dist
@@ -228,7 +232,7 @@ def run_ours(args, wid):
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
-    if world > 1:
+    if world > 1 and not dist.is_initialized():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
     import compressed_sparse_long_csa_b200 as csa
@@ -386,11 +390,11 @@ def run_ours(args, wid):
         achieved = fl[dom] / (dom_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "peak_source": src + (" bf16 x 2 (fp8)" if dom == "indexer" else " bf16 burst"),
-                "traffic": TRAFFIC.get((args.workload, dom))}
+                "traffic": TRAFFIC.get((name, dom))}
     else:
         achieved = ab[dom] / (dom_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved / hbm_peak, "peak_source": src, "traffic": TRAFFIC.get((args.workload, dom))}
+                "frac": achieved / hbm_peak, "peak_source": src, "traffic": TRAFFIC.get((name, dom))}
     extra = None
     if world == 1:
         # the rows beyond the step, each timed alone on this GPU (single-GPU characterisations:
@@ -408,7 +412,7 @@ def run_ours(args, wid):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": dict(workload_config(args.workload, D), launch="one CUDA graph per step"),
+        "config": dict(workload_config(name, D), launch="one CUDA graph per step"),
         "hbm_gbs_step": sum(ab.values()) / (ms_per_step * 1e-3) / 1e9,
         "breakdown_ms": {c: float(m) for c, m in zip(comp, mean_ms)},
         "roofline": roof,
@@ -422,9 +426,15 @@ def run_ours(args, wid):
         line["cpu_baseline"] = cpu_baseline(wid, wl)
     if rank == 0:
         print(json.dumps(line), flush=True)
+    # release this workload's graphs and buffers before the next one
+    del g_step, graphs, T
+    import gc
+    gc.collect()
+    torch.cuda.empty_cache()
     if world > 1:
         dist.barrier()
-        dist.destroy_process_group()
+        if name == ORDER[-1] or args.workload != "all":
+            dist.destroy_process_group()
 
 
 def measure_index_keys(wid, D, csa, l2_flush, hbm_peak, peak_src, reps=20):
@@ -700,24 +710,32 @@ def measure_e2e(args, wid, wl, T, D, csa, steps):
     return e0.elapsed_time(e1) / n, h2d, d2h
 
 
-def cpu_baseline(wid, wl):
-    """The oracle as it stands on the host cores, on a bounded sample."""
+def cpu_baseline(wid, wl, min_s=3.0, max_reps=20):
+    """The oracle as it stands on the host cores, on a bounded sample of the workload:
+    the sample (whole sequences of a decode step, query rows of the prefill chunk with
+    the chunk's compression) is repeated until at least min_s seconds have passed, and
+    the rate is taken over all repeats."""
     from oracle import csa_oracle as O
     D = wl.dims
     sample = list(range(min(D["B"], 2)))
-    t0 = time.perf_counter()
-    if wid in (1, 4):
-        O.run_csa_decode(wl, batches=sample)
-        if wid == 4:
-            O.run_hca_decode(wl, batches=sample, prefix="h_")
-    elif wid == 2:
-        O.run_hca_decode(wl, batches=sample)
-    else:
-        O.run_csa_prefill(wl, rows=list(range(8)))
+    rows = list(range(8))
+    reps, t0 = 0, time.perf_counter()
+    while reps < max_reps and (reps == 0 or time.perf_counter() - t0 < min_s):
+        if wid in (1, 4):
+            O.run_csa_decode(wl, batches=sample)
+            if wid == 4:
+                O.run_hca_decode(wl, batches=sample, prefix="h_")
+        elif wid == 2:
+            O.run_hca_decode(wl, batches=sample)
+        else:
+            O.run_csa_prefill(wl, rows=rows)
+        reps += 1
     dt = time.perf_counter() - t0
-    toks = len(sample) if wid != 3 else 8
+    toks = (len(sample) if wid != 3 else len(rows)) * reps
+    what = (f"{len(rows)} query rows of the chunk (with the chunk's compression)" if wid == 3
+            else f"{len(sample)} of {D['B']} sequences, full context")
     return {"value": toks / dt, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
-            "sample": f"{toks} {'query rows' if wid == 3 else 'sequences'} of the workload, one step"}
+            "sample": f"{what}, repeated {reps}x ({dt:.1f} s)"}
 
 
 if __name__ == "__main__":

@@ -22,6 +22,7 @@ _SIGS = {
     "csa_status_string": ([_i32], C.c_char_p),
     "csa_read_device_error": ([_vp, C.POINTER(C.c_uint32)], _i32),
     "csa_launch_count": ([], C.c_uint64),
+    "csa_wait_probe": ([C.c_uint64, _vp], _i32),
     "csa_compress": ([_vp] * 10 + [_i64, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
     "csa_compress_kv8": ([_vp] * 10 + [_i64, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
     "index_key_compress": ([_vp] * 11 + [_i64, _i32, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
@@ -75,6 +76,11 @@ def _stream(stream):
 
 def _dtype_code(t):
     return CSA_BF16 if t.dtype == torch.bfloat16 else CSA_F32
+
+
+def wait_probe(limit_ns: int, stream=None):
+    """One kernel whose wait can never end, bounded by limit_ns (sets CSA_DEVERR_TIMEOUT)."""
+    _check(lib.csa_wait_probe(int(limit_ns), _stream(stream)), "csa_wait_probe")
 
 
 def launch_count() -> int:

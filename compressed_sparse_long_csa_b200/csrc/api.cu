@@ -24,6 +24,7 @@ size_t out_proj_partial_elems(int T, int R_max);
 cudaError_t launch_grouped_out_proj(const void* o, int T, int H, int dv, int g, int d_mid, const void* W1,
                                     const void* W2, int d, void* u, void* y, float* part, size_t part_elems,
                                     cudaStream_t st, unsigned* err);
+cudaError_t launch_wait_probe(uint64_t limit_ns, cudaStream_t st, unsigned* err);
 cudaError_t launch_index_key_compress(const void*, const void*, const void*, const void*, const float*,
                                       const float*, const void*, const void*, const int32_t*, void*, void*, int64_t,
                                       int, int, int, int, int, cudaStream_t, unsigned*);
@@ -122,6 +123,13 @@ csa_status csa_read_device_error(void* stream, uint32_t* out) {
   return CSA_OK;
 }
 
+csa_status csa_wait_probe(uint64_t limit_ns, void* stream) {
+  REQUIRE(limit_ns >= 1000u && limit_ns <= 2000000000ull, CSA_ERR_SHAPE);
+  unsigned* err = device_error_word();
+  REQUIRE(err, CSA_ERR_CUDA);
+  return cuda_status(launch_wait_probe(limit_ns, S(stream), err));
+}
+
 // ----------------------------------------------------------------------------- compressors
 csa_status csa_compress(const void* Ca, const void* Cb, const void* Za, const void* Zb, const float* Ba,
                         const float* Bb, const void* prev_Cb, const void* prev_Zb, const int32_t* entry0,
@@ -193,11 +201,44 @@ csa_status index_key_compress(const void* Ca, const void* Cb, const void* Za, co
 // ----------------------------------------------------------------------------- indexer / top-k
 static int64_t idx_ld(int64_t n_max) { return (int64_t)round_up((size_t)n_max, 64); }
 
+// Decode rows (at most this many queries per sequence) select through the score histogram
+// (select_hist.cu), which needs its own workspace regions.
+constexpr int kHistMaxTq = 3;
+constexpr size_t kHistBins = 4096;
+
+// Workspace layout of lightning_index (each region 256-byte aligned):
+//   scores [R][ld] fp32 | knmax [B] | keyrange [R][2] | (decode rows:) hist [R][4096] |
+//   counters [R][4] | bitmap [R][ld/32] | cand [R][ld] (order key, id)
+// R = B * Tq.  knmax .. counters is one contiguous region, zeroed by one memset per call.
+struct IdxWs {
+  size_t scores, knmax, keyrange, hist, counters, bitmap, cand, end, zero_end;
+};
+static IdxWs idx_ws_layout(int B, int Tq, int64_t n_max) {
+  const size_t R = (size_t)B * Tq, ld = (size_t)idx_ld(n_max);
+  IdxWs L{};
+  L.scores = 0;
+  L.knmax = round_up(R * ld * sizeof(float), 256);
+  L.keyrange = L.knmax + round_up((size_t)B * sizeof(unsigned), 256);
+  L.hist = L.keyrange + round_up(R * 2 * sizeof(unsigned), 256);
+  L.counters = L.hist;
+  L.bitmap = L.hist;
+  L.cand = L.hist;
+  L.end = L.hist;
+  L.zero_end = L.hist;
+  if (Tq <= kHistMaxTq) {
+    L.counters = L.hist + round_up(R * kHistBins * sizeof(unsigned), 256);
+    L.zero_end = L.counters + R * 4 * sizeof(unsigned);
+    L.bitmap = L.counters + round_up(R * 4 * sizeof(unsigned), 256);
+    L.cand = L.bitmap + round_up(R * (ld / 32) * sizeof(unsigned), 256);
+    L.end = L.cand + round_up(R * ld * 2 * sizeof(unsigned), 256);
+  }
+  return L;
+}
+
 size_t lightning_index_workspace_size(int B, int Tq, int64_t n_max, int k) {
   (void)k;
   if (B < 1 || Tq < 1 || n_max < 1) return 0;
-  return round_up((size_t)B * Tq * idx_ld(n_max) * sizeof(float), 256) + round_up((size_t)B * sizeof(unsigned), 256) +
-         round_up((size_t)B * Tq * 2 * sizeof(unsigned), 256);
+  return idx_ws_layout(B, Tq, n_max).end;
 }
 
 static csa_status run_lightning_index(const void* qI, const void* qI_scale, const float* w, const void* kI,
@@ -225,19 +266,30 @@ static csa_status run_lightning_index(const void* qI, const void* qI_scale, cons
   a.n_entries = n_entries; a.q_pos = q_pos; a.m = m;
   a.B = B; a.Tq = Tq; a.H_I = H_I; a.d_I = d_I; a.n_max = n_max; a.k = k; a.ifmt = ifmt;
   a.ld = idx_ld(n_max);
-  a.scores = (float*)workspace;
-  a.knmax = (unsigned*)((char*)workspace + round_up((size_t)B * Tq * a.ld * sizeof(float), 256));
+  const IdxWs L = idx_ws_layout(B, Tq, n_max);
+  char* ws = (char*)workspace;
+  a.scores = (float*)(ws + L.scores);
+  a.knmax = (unsigned*)(ws + L.knmax);
+  a.keyrange = (unsigned*)(ws + L.keyrange);
   a.idx_out = idx_out; a.score_out = score_out; a.err = err;
   a.score_bf16 = bf16_scores ? 1 : 0;
-  a.keyrange = a.knmax + round_up((size_t)B * sizeof(unsigned), 256) / sizeof(unsigned);
-  cudaError_t e = cudaMemsetAsync(a.knmax, 0, round_up((size_t)B * sizeof(unsigned), 256) +
-                                  (size_t)B * Tq * 2 * sizeof(unsigned), S(stream));
+  // the histogram-seeded selection: decode rows of the exact call (the bf16-key call
+  // selects on the stored keys with the plain top-k)
+  const bool hist_path = Tq <= kHistMaxTq && !bf16_scores;
+  if (hist_path) {
+    a.hist = (unsigned*)(ws + L.hist);
+    a.counters = (unsigned*)(ws + L.counters);
+    a.bitmap = (unsigned*)(ws + L.bitmap);
+    a.cand = (uint2*)(ws + L.cand);
+  }
+  cudaError_t e = cudaMemsetAsync(ws + L.knmax, 0, L.zero_end - L.knmax, S(stream));
   if (e != cudaSuccess) return CSA_ERR_CUDA;
   bool used_tc = false;
   if (tc_enabled()) {
     e = launch_indexer_scores_tc(a, S(stream), &used_tc);       // sets a.eps_dot of its path
     if (e != cudaSuccess) return CSA_ERR_CUDA;
   }
+  if (!used_tc) a.hist = nullptr;                              // the CUDA-core scores come without a histogram
   if (!used_tc) {
     // sequential fp32 FMA accumulation of d_I exact products: |err| <= (d_I+2) u sum|q c k c|
     a.eps_dot = (float)(d_I + 4) * 5.9604645e-08f * 1.25f;

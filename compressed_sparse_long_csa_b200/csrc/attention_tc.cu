@@ -18,8 +18,10 @@
 //      fastest way to gather scattered rows that was measured on B200);
 //   2. one thread issues S = Q K^T (M=64, N=64, 36 steps of K=16) into TMEM;
 //   3. softmax threads (one per head, TMEM lanes 16-31) run an online softmax with a
-//      lazily raised running max and write P (bf16) to shared memory;
-//   4. O += P V (M=64, N=2x256, K=64; V is read MN-major from the same tile).
+//      lazily raised running max and write P to shared memory as two bf16 parts,
+//      P_hi = bf16(P) and P_lo = bf16(P - P_hi) (the second into the tile's RoPE atom,
+//      which only S reads);
+//   4. O += P_hi V + P_lo V (M=64, N=2x256, K=2x64; V is read MN-major from the same tile).
 // At the end, threads of TMEM lanes 0-15 normalise O (one split), or write the split
 // partial (o, m, l) to the workspace.  The CTAs of one query's head half form a
 // thread-block cluster (at most 8 splits): after a cluster barrier each merges a slice
@@ -335,6 +337,9 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
     const uint64_t q_d0 = tc::desc_k_sw128(tc::smem_u32(sm.q[0]));
     const uint64_t k_d0 = tc::desc_k_sw128(tc::smem_u32(sm.kv[0][0])), k_d1 = tc::desc_k_sw128(tc::smem_u32(sm.kv[1][0]));
     const uint64_t p_d0 = tc::desc_k_sw128(tc::smem_u32(sm.p));
+    // P's low part of tile st sits in the stage's RoPE atom (free once S has read it)
+    const uint64_t pl_d0 = tc::desc_k_sw128(tc::smem_u32(sm.kv[0][AT_ATOMS - 1])),
+                   pl_d1 = tc::desc_k_sw128(tc::smem_u32(sm.kv[1][AT_ATOMS - 1]));
     const uint64_t v_d0 = tc::desc_mn_sw128(tc::smem_u32(sm.kv[0][0]), ATOM, 1024),
                    v_d1 = tc::desc_mn_sw128(tc::smem_u32(sm.kv[1][0]), ATOM, 1024);
     // Event-driven issue: S(ns) once its tile has landed and its S buffer is free, PV(np)
@@ -370,10 +375,12 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
         bool ready = false;
         if (lane == 0) ready = tc::mbar_try_wait(&sm.pfull, np & 1);
         if (__shfl_sync(0xffffffffu, (int)ready, 0)) {
-          // O += P_np V_np: value dims 0-255 (atoms 0-3) and 256-511 (atoms 4-7)
+          // O += (P_hi + P_lo)_np V_np: value dims 0-255 (atoms 0-3) and 256-511 (atoms 4-7);
+          // the two bf16 parts of P are two K ranges over the same V rows
           const int st = np & 1;
           tc::fence_after_sync();
           const uint64_t vd = st ? v_d1 : v_d0;
+          const uint64_t pl = st ? pl_d1 : pl_d0;
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             const uint64_t vh = vd + (uint64_t)((4 * half * ATOM) >> 4);
@@ -385,6 +392,10 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
             for (int ks = 1; ks < AT_ROWS / 16; ++ks)
               if (tc::elect_one())
                 tc::mma_f16_c<true>(tmem + 256 * half, p_d0 + (uint64_t)((ks * 32) >> 4), vh + (uint64_t)((ks * 16 * 128) >> 4), ID_O);
+#pragma unroll
+            for (int ks = 0; ks < AT_ROWS / 16; ++ks)
+              if (tc::elect_one())
+                tc::mma_f16_c<true>(tmem + 256 * half, pl + (uint64_t)((ks * 32) >> 4), vh + (uint64_t)((ks * 16 * 128) >> 4), ID_O);
           }
           if (tc::elect_one()) {
             tc::mma_commit(&sm.empty[st]);
@@ -480,17 +491,22 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
         const float moved = __shfl_down_sync(0xffffffffu, a1, 16);
         pv[q] = is_s ? a0 : moved;
       }
-      // P in registers first (bf16, the normaliser sums the rounded values); it overlaps the
-      // previous PV, which owns the shared P tile and O until it completes
-      uint32_t w8[8];
+      // P in registers first, as two bf16 parts (hi = P rounded, lo = the remainder rounded:
+      // their sum carries P to about 2^-17 where bf16 alone gives 2^-9, which would use a
+      // third of the output's error budget); the normaliser sums the parts the MMA sees.
+      // This overlaps the previous PV, which owns the shared P tile and O until it completes.
+      uint32_t w8[8], l8[8];
       float psum = 0.f;
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const float p0 = (m_use == -INFINITY) ? 0.f : ex2_approx(pv[2 * u] - m_use);
         const float p1 = (m_use == -INFINITY) ? 0.f : ex2_approx(pv[2 * u + 1] - m_use);
-        __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
-        psum += __low2float(hb) + __high2float(hb);
-        w8[u] = *reinterpret_cast<uint32_t*>(&hb);
+        const __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
+        const float h0 = __low2float(hb), h1 = __high2float(hb);
+        const __nv_bfloat162 lb = __floats2bfloat162_rn(p0 - h0, p1 - h1);
+        psum += (h0 + __low2float(lb)) + (h1 + __high2float(lb));
+        w8[u] = *reinterpret_cast<const uint32_t*>(&hb);
+        l8[u] = *reinterpret_cast<const uint32_t*>(&lb);
       }
       const float po = __shfl_up_sync(0xffffffffu, psum, 16);   // the O lane's part, to its S lane
       if (is_s) l_run = l_run * alpha + psum + po;
@@ -520,12 +536,17 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
         tc::tmem_st_wait();
       }
       {
-        const uint32_t pbase = tc::smem_u32(sm.p);
+        // P_hi into the P tile, P_lo into this stage's RoPE atom (S of this tile, its only
+        // reader, has completed: sfull[st] was waited on above)
+        const uint32_t pbase = tc::smem_u32(sm.p), lbase = tc::smem_u32(sm.kv[st][AT_ATOMS - 1]);
         const int c0 = 4 * wg + (is_s ? 0 : 2);     // 16-byte chunks (8 columns) of the P row
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc)
+        for (int cc = 0; cc < 2; ++cc) {
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pbase + sw128_off(hl, c0 + cc)), "r"(w8[4 * cc]),
                        "r"(w8[4 * cc + 1]), "r"(w8[4 * cc + 2]), "r"(w8[4 * cc + 3]) : "memory");
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(lbase + sw128_off(hl, c0 + cc)), "r"(l8[4 * cc]),
+                       "r"(l8[4 * cc + 1]), "r"(l8[4 * cc + 2]), "r"(l8[4 * cc + 3]) : "memory");
+        }
       }
       // release this tile's S buffer and hand P (and a rescaled O) to the MMA thread
       tc::fence_proxy_async_smem();

@@ -26,6 +26,11 @@ struct IndexerArgs {
   unsigned* err;
   float eps_dot;              // bound on |fp32 dot - exact| / (||q|| ||k||) of the scoring path
   int score_bf16;             // 1: scores are rounded to bf16 before they are stored (lightning_index_bf16)
+  // decode rows (Tq <= 3) only, else null: the histogram-seeded selection (select_hist.cu)
+  unsigned* hist;             // [B*Tq][4096] score histogram (order key >> 20), zeroed per call
+  unsigned* counters;         // [B*Tq][4]: candidates, certain entries, CTAs done; zeroed per call
+  unsigned* bitmap;           // [B*Tq][ld/32] certain entries
+  uint2* cand;                // [B*Tq][ld] candidates (order key, entry id)
 };
 
 // Entries of one selection row: n_valid[row] (topk_select), else the indexer's
@@ -105,6 +110,9 @@ cudaError_t launch_topk_select(const float* scores, int64_t ld, RowCount rc, int
                                int k, int32_t* idx_out, cudaStream_t st, unsigned* err);
 // Cluster paths (select.cu); cudaErrorNotSupported when a row does not fit one cluster.
 cudaError_t launch_indexer_select_cluster(const IndexerArgs& a, cudaStream_t st);
+// Histogram-seeded selection of decode rows (select_hist.cu); cudaErrorNotSupported when
+// the scoring path wrote no histogram.
+cudaError_t launch_indexer_select_hist(const IndexerArgs& a, cudaStream_t st);
 cudaError_t launch_topk_select_cluster(const float* scores, int64_t ld, RowCount rc, int R, int64_t n,
                                        int k, int32_t* idx_out, cudaStream_t st);
 

@@ -40,10 +40,15 @@ struct IdxTcParams {
 
 constexpr int IT_THREADS = 384;  // warp 0 TMA, warp 1 MMA, warps 4..11 epilogue (two warpgroups)
 
-template <int G, int STAGES>
+// Level-1 bins of the score histogram that seeds the decode selection (select_hist.cu):
+// the top 12 bits of a score's monotone order key.
+constexpr int IT_HBINS = 4096;
+
+template <int G, int STAGES, bool HIST>
 struct IdxSmem {
   alignas(1024) uint8_t q[G * 64 * IT_KB];
   alignas(1024) uint8_t k[STAGES][IT_TILE_BYTES];
+  uint32_t hist[HIST ? IT_HBINS : 1];
   alignas(8) uint64_t full[STAGES];
   uint64_t empty[STAGES];
   uint64_t tfull[4];
@@ -58,11 +63,11 @@ struct IdxSmem {
   alignas(16) float wq[G][64];
 };
 
-template <int G, int STAGES>
+template <int G, int STAGES, bool HIST>
 __global__ void __launch_bounds__(IT_THREADS, G == 1 ? 2 : 1)
 indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ, IdxTcParams p) {
   extern __shared__ uint8_t smem_raw[];
-  using Sm = IdxSmem<G, STAGES>;
+  using Sm = IdxSmem<G, STAGES, HIST>;
   Sm& sm = *reinterpret_cast<Sm*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const IndexerArgs& a = p.a;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -106,6 +111,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     }
     sm.issued0 = n0;
   }
+  if (HIST)
+    for (int i = threadIdx.x; i < IT_HBINS; i += blockDim.x) sm.hist[i] = 0u;
   for (int i = threadIdx.x; i < G * 64; i += blockDim.x) {
     const int g = i / 64, j = i % 64;
     const int t = qg * G + g;
@@ -221,11 +228,17 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         }
         const float val = (part[0] + part[1]) + (part[2] + part[3]);
         const bool valid = s < sm.n_elig[g];
+        const float sc = a.score_bf16 ? round_bf16(val * sk) : val * sk;
         if (valid) {
-          const float sc = a.score_bf16 ? round_bf16(val * sk) : val * sk;
           a.scores[(size_t)sm.row[g] * a.ld + s] = sc;
           kmax = fmaxf(kmax, sk);
           kr[g].add(sc);
+        }
+        if (HIST) {
+          // one shared-memory atomic per distinct bin of the warp
+          const uint32_t bin = valid ? (f32_order_key(sc) >> 20) : 0xFFFFFFFFu;
+          const unsigned peers = __match_any_sync(0xffffffffu, bin);
+          if (valid && lane == __ffs(peers) - 1) atomicAdd(&sm.hist[bin], (uint32_t)__popc(peers));
         }
       }
       tc::fence_before_sync();
@@ -245,6 +258,14 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, NCOLS);
   }
+  if (HIST && a.hist) {
+    // this CTA's histogram into the row's (only the bins in use: a few dozen)
+    uint32_t* gh = a.hist + (size_t)sm.row[0] * IT_HBINS;
+    for (int i = threadIdx.x; i < IT_HBINS; i += blockDim.x) {
+      const uint32_t c = sm.hist[i];
+      if (c) atomicAdd(gh + i, c);
+    }
+  }
 }
 
 // ------------------------------------------------------------------------------------------
@@ -262,6 +283,7 @@ template <int STAGES>
 struct MxSmem {
   alignas(1024) uint8_t q[64 * MX_KB];
   alignas(1024) uint8_t k[STAGES][MX_TILE_BYTES];
+  uint32_t hist[IT_HBINS];
   alignas(8) uint64_t full[STAGES];
   uint64_t empty[STAGES];
   uint64_t sfa_full[STAGES];
@@ -328,6 +350,7 @@ indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     sm.issued0 = n0;
   }
   if (threadIdx.x < 64) sm.w[threadIdx.x] = threadIdx.x < a.H_I ? a.w[(size_t)row * a.H_I + threadIdx.x] : 0.f;
+  for (int i = threadIdx.x; i < IT_HBINS; i += blockDim.x) sm.hist[i] = 0u;
   if (warp == 1) { tc::tmem_alloc(&sm.tmem_base, MX_COLS); tc::tmem_relinquish(); }
   tc::fence_before_sync();
   __syncthreads();
@@ -470,6 +493,11 @@ indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         a.scores[(size_t)row * a.ld + s] = val;
         kr.add(val);
       }
+      {
+        const uint32_t bin = valid ? (f32_order_key(val) >> 20) : 0xFFFFFFFFu;
+        const unsigned peers = __match_any_sync(0xffffffffu, bin);
+        if (valid && lane == __ffs(peers) - 1) atomicAdd(&sm.hist[bin], (uint32_t)__popc(peers));
+      }
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&sm.tempty[acc]);
@@ -484,6 +512,13 @@ indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   if (warp == 1) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, MX_COLS);
+  }
+  if (a.hist) {
+    uint32_t* gh = a.hist + (size_t)row * IT_HBINS;
+    for (int i = threadIdx.x; i < IT_HBINS; i += blockDim.x) {
+      const uint32_t c = sm.hist[i];
+      if (c) atomicAdd(gh + i, c);
+    }
   }
 }
 
@@ -553,7 +588,7 @@ cudaError_t launch_mxf4(const IndexerArgs& a, cudaStream_t st, bool* used) {
   return cudaGetLastError();
 }
 
-template <int G, int STAGES>
+template <int G, int STAGES, bool HIST>
 cudaError_t launch_g(const IndexerArgs& a, cudaStream_t st, bool* used) {
   IdxTcParams p{};
   p.a = a;
@@ -571,13 +606,13 @@ cudaError_t launch_g(const IndexerArgs& a, cudaStream_t st, bool* used) {
   CUtensorMap mk, mq;
   if (!make_map_rows128(&mk, a.kI, (uint64_t)a.B * a.n_max, IT_ROWS)) return cudaSuccess;
   if (!make_map_rows128(&mq, a.qI, (uint64_t)a.B * a.Tq * 64, 64 * G)) return cudaSuccess;
-  const size_t smem = sizeof(IdxSmem<G, STAGES>) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<G, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const size_t smem = sizeof(IdxSmem<G, STAGES, HIST>) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<G, STAGES, HIST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(splits, p.n_qg, a.B);
   note_launch();
-  indexer_tc_kernel<G, STAGES><<<grid, IT_THREADS, smem, st>>>(mk, mq, p);
+  indexer_tc_kernel<G, STAGES, HIST><<<grid, IT_THREADS, smem, st>>>(mk, mq, p);
   *used = true;
   return cudaGetLastError();
 }
@@ -603,8 +638,11 @@ cudaError_t launch_indexer_scores_tc(IndexerArgs& a, cudaStream_t st, bool* used
   // fp32 accumulation of exact products (128 * 2^-24 = 2^-17).  Measured on B200: <= 5e-9
   // relative to the bound's scale (test_indexer_fp32_score_error_within_band_bound).
   a.eps_dot = 1.0f / 131072.0f;
-  if (a.Tq >= 4) return launch_g<4, 6>(a, st, used);
-  return launch_g<1, 6>(a, st, used);
+  if (a.Tq >= 4) return launch_g<4, 6, false>(a, st, used);
+  // decode rows: the score histogram for the selection (one fewer ring stage makes room
+  // for it at two CTAs per SM)
+  if (a.hist) return launch_g<1, 5, true>(a, st, used);
+  return launch_g<1, 6, false>(a, st, used);
 }
 
 }  // namespace csa

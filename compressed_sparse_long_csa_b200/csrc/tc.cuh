@@ -43,14 +43,17 @@ __device__ __forceinline__ uint64_t now_ns() {
 }
 // Every wait of the library gives up after this long (a healthy wait takes microseconds).
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
-// Bounded wait on a phase of a CTA-local mbarrier.  Returns false on timeout.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Bounded wait on a phase of a CTA-local mbarrier: false once limit_ns have passed.
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = now_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63u) == 0 && now_ns() - t0 > WAIT_LIMIT_NS) return false;
+    if ((i & 63u) == 0 && now_ns() - t0 > limit_ns) return false;
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  return mbar_wait_limit(bar, parity, WAIT_LIMIT_NS);
 }
 
 // ---------------------------------------------------------------- programmatic dependent launch

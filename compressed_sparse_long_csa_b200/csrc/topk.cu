@@ -538,6 +538,10 @@ static void set_smem_attr(const void* fn) {
 }
 
 cudaError_t launch_indexer_select(const IndexerArgs& a, cudaStream_t st) {
+  if (a.hist) {
+    const cudaError_t eh = launch_indexer_select_hist(a, st);
+    if (eh != cudaErrorNotSupported) return eh;
+  }
   const cudaError_t e = launch_indexer_select_cluster(a, st);
   if (e != cudaErrorNotSupported) return e;
   set_smem_attr((const void*)indexer_select_kernel);

@@ -82,6 +82,16 @@ csa_status csa_read_device_error(void* stream, uint32_t* out);
  * paper has no counterpart: it lets a caller check which work ran on the GPU.  */
 uint64_t csa_launch_count(void);
 
+/* Device-side waits.  Every kernel that waits (for a TMA copy, a tensor-core MMA or
+ * another warp of its CTA) waits on a CTA-local mbarrier with a time limit of 2 s; a
+ * wait that runs out sets CSA_DEVERR_TIMEOUT, the kernel waits (again bounded) for its
+ * own copies in flight, releases its tensor memory and returns.
+ * csa_wait_probe launches one CTA whose single wait nothing can complete, with the
+ * limit limit_ns (1e3 .. 2e9 ns, CSA_ERR_SHAPE otherwise): after it the error word
+ * holds CSA_DEVERR_TIMEOUT and the device stays usable.  The paper has no
+ * counterpart: it lets a caller check that a wait that cannot end returns an error. */
+csa_status csa_wait_probe(uint64_t limit_ns, void* stream);
+
 /* ---------------------------------------------------------------------------
  * csa_compress — CSA token-axis compression fused with the KV-cache append.
  * ("Гибридное внимание: CSA и HCA", CSA step 1: two KV series C^a, C^b and two

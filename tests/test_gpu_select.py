@@ -1,0 +1,115 @@
+"""GPU: the exact top-k of the lightning indexer on decode rows ("Техотчёт DeepSeek-V4
+(2026)", section "Гибридное внимание: CSA и HCA", CSA step 2), the cases the workload
+tests do not reach: rows of different eligible counts, just above and at k; every key
+identical (all scores tie: the lowest indices win); scores packed into one narrow range
+(more candidates than the selection stages on chip); the exact scores returned with the
+selection.  Expected values come from the oracle only.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import csa_inputs as CI
+from oracle import csa_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import compressed_sparse_long_csa_b200 as csa
+
+
+def _run(qI, qs, w, kI, ks, n_entries, q_pos, k, fmt, score_out=False):
+    """lightning_index on host arrays; returns (idx [B, k], scores or None, device error word)."""
+    B, n_max = kI.shape[0], kI.shape[1]
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    idx = torch.empty(B, 1, k, dtype=torch.int32, device="cuda")
+    so = torch.empty(B, 1, k, dtype=torch.float32, device="cuda") if score_out else None
+    ws = torch.empty(csa.lightning_index_workspace_size(B, 1, n_max, k), dtype=torch.uint8, device="cuda")
+    ifmt = csa.CSA_IFMT_E4M3 if fmt == "e4m3" else csa.CSA_IFMT_MXFP4
+    csa.lightning_index(dev(qI), dev(qs), dev(w), dev(kI), dev(ks), dev(n_entries.astype(np.int32)),
+                        dev(q_pos.astype(np.int32)), k, ifmt, idx, ws, score_out=so)
+    torch.cuda.synchronize()
+    err = csa.read_device_error()
+    return idx[:, 0].cpu().numpy(), (so[:, 0].cpu().numpy() if so is not None else None), err
+
+
+def _oracle(qI, qs, w, kI, ks, b, n, fmt):
+    return O.indexer_scores(qI[b], w[b], kI[b], fmt, qs[b], ks[b])[0][:n]
+
+
+def _keys(fmt, x):
+    return CI.quant_e4m3_rows(x) if fmt == "e4m3" else CI.quant_mxfp4_rows(x)
+
+
+def _check_exact(g, I, n, k):
+    """The selection must be the oracle's exactly: ascending, ties to the lower index."""
+    exp = O.topk(I, n, k)
+    assert np.array_equal(g, exp), (np.setdiff1d(g, exp)[:8], np.setdiff1d(exp, g)[:8])
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "mxfp4"])
+def test_decode_rows_of_different_eligible_counts(fmt):
+    g = torch.Generator().manual_seed(41)
+    B, N, k = 5, 6000, 512
+    qI, qs = _keys(fmt, torch.randn(B, 1, 64, 128, generator=g))
+    kI, ks = _keys(fmt, torch.randn(B, N, 128, generator=g))
+    w = torch.rand(B, 1, 64, generator=g).numpy()
+    n_entries = np.array([6000, 513, 512, 3001, 40])
+    q_pos = 4 * n_entries - 1                        # the current token completes entry n - 1
+    idx, _, err = _run(qI, qs, w, kI, ks, n_entries, q_pos, k, fmt)
+    assert err == 0
+    for b in range(B):
+        _check_exact(idx[b], _oracle(qI, qs, w, kI, ks, b, n_entries[b], fmt), n_entries[b], k)
+
+
+def test_all_scores_tie_and_lowest_indices_win():
+    """Every key identical: every score is the same, so the k lowest indices are the
+    selection (the candidate band outgrows its buffer here, which is flagged)."""
+    g = torch.Generator().manual_seed(42)
+    B, N, k = 2, 9000, 512
+    qI, qs = _keys("e4m3", torch.randn(B, 1, 64, 128, generator=g))
+    kI, ks = _keys("e4m3", torch.randn(1, 1, 128, generator=g).expand(B, N, 128).contiguous())
+    w = torch.rand(B, 1, 64, generator=g).numpy()
+    n_entries = np.array([N, N])
+    idx, _, err = _run(qI, qs, w, kI, ks, n_entries, 4 * n_entries - 1, k, "e4m3")
+    assert err & ~0x8 == 0                            # only CSA_DEVERR_BAND may be set
+    assert np.array_equal(idx, np.tile(np.arange(k), (B, 1)))
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "mxfp4"])
+def test_narrow_score_range_many_candidates(fmt):
+    """Keys = one shared direction plus a little noise: the scores of 40 000 entries fall
+    into one or two histogram bins, so the candidates outnumber the on-chip buffer and the
+    selection works from the list in L2."""
+    g = torch.Generator().manual_seed(43)
+    B, N, k = 2, 40000, 1024
+    qI, qs = _keys(fmt, torch.randn(B, 1, 64, 128, generator=g))
+    base = torch.randn(B, 1, 128, generator=g)
+    kI, ks = _keys(fmt, base + 0.1 * torch.randn(B, N, 128, generator=g))   # ~5000-27000 in bin T, band ~200
+    w = torch.rand(B, 1, 64, generator=g).numpy()
+    n_entries = np.array([N, N - 17])
+    idx, _, err = _run(qI, qs, w, kI, ks, n_entries, 4 * n_entries - 1, k, fmt)
+    assert err == 0
+    for b in range(B):
+        I = _oracle(qI, qs, w, kI, ks, b, n_entries[b], fmt)
+        _check_exact(idx[b], I, n_entries[b], k)
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "mxfp4"])
+def test_score_out_is_the_exact_score_of_each_selected_entry(fmt):
+    g = torch.Generator().manual_seed(44)
+    B, N, k = 3, 5000, 256
+    qI, qs = _keys(fmt, torch.randn(B, 1, 64, 128, generator=g))
+    kI, ks = _keys(fmt, torch.randn(B, N, 128, generator=g))
+    w = torch.rand(B, 1, 64, generator=g).numpy()
+    n_entries = np.array([N, 200, 2500])
+    idx, so, err = _run(qI, qs, w, kI, ks, n_entries, 4 * n_entries - 1, k, fmt, score_out=True)
+    assert err == 0
+    for b in range(B):
+        I = _oracle(qI, qs, w, kI, ks, b, n_entries[b], fmt)
+        _check_exact(idx[b], I, n_entries[b], k)
+        sel = idx[b][idx[b] >= 0]
+        assert np.array_equal(so[b][:sel.size], I[sel].astype(np.float32))
+        assert np.all(so[b][sel.size:] == 0)
