@@ -205,10 +205,11 @@ static int64_t idx_ld(int64_t n_max) { return (int64_t)round_up((size_t)n_max, 6
 // (select_hist.cu), which needs its own workspace regions.
 constexpr int kHistMaxTq = 3;
 constexpr size_t kHistBins = 4096;
+constexpr size_t kHistCounters = 256;     // per row: certain count, CTAs done, per-CTA candidate counts
 
 // Workspace layout of lightning_index (each region 256-byte aligned):
 //   scores [R][ld] fp32 | knmax [B] | keyrange [R][2] | (decode rows:) hist [R][4096] |
-//   counters [R][4] | bitmap [R][ld/32] | cand [R][ld] (order key, id)
+//   counters [R][256] | bitmap [R][ld/32] | cand [R][ld] (order key, id)
 // R = B * Tq.  knmax .. counters is one contiguous region, zeroed by one memset per call.
 struct IdxWs {
   size_t scores, knmax, keyrange, hist, counters, bitmap, cand, end, zero_end;
@@ -227,8 +228,8 @@ static IdxWs idx_ws_layout(int B, int Tq, int64_t n_max) {
   L.zero_end = L.hist;
   if (Tq <= kHistMaxTq) {
     L.counters = L.hist + round_up(R * kHistBins * sizeof(unsigned), 256);
-    L.zero_end = L.counters + R * 4 * sizeof(unsigned);
-    L.bitmap = L.counters + round_up(R * 4 * sizeof(unsigned), 256);
+    L.zero_end = L.counters + R * kHistCounters * sizeof(unsigned);
+    L.bitmap = L.counters + round_up(R * kHistCounters * sizeof(unsigned), 256);
     L.cand = L.bitmap + round_up(R * (ld / 32) * sizeof(unsigned), 256);
     L.end = L.cand + round_up(R * ld * 2 * sizeof(unsigned), 256);
   }

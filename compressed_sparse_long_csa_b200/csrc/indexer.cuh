@@ -28,7 +28,7 @@ struct IndexerArgs {
   int score_bf16;             // 1: scores are rounded to bf16 before they are stored (lightning_index_bf16)
   // decode rows (Tq <= 3) only, else null: the histogram-seeded selection (select_hist.cu)
   unsigned* hist;             // [B*Tq][4096] score histogram (order key >> 20), zeroed per call
-  unsigned* counters;         // [B*Tq][4]: candidates, certain entries, CTAs done; zeroed per call
+  unsigned* counters;         // [B*Tq][256]: certain entries, CTAs done, per-CTA candidate counts; zeroed per call
   unsigned* bitmap;           // [B*Tq][ld/32] certain entries
   uint2* cand;                // [B*Tq][ld] candidates (order key, entry id)
 };

@@ -47,11 +47,17 @@ constexpr int SH_BINS2 = 2048;           // refinement bins
 constexpr int SH_CCAP = 4096;            // candidates staged in shared memory (more stay in L2)
 constexpr int SH_BAND = 512;             // band entries re-scored exactly
 constexpr int SH_BMW = 8192;             // bitmap words handled per output pass (262 144 entries)
+constexpr int SH_RB = 32;                // entries re-scored per batch
+constexpr int SH_DLD = 132;              // bytes per staged digit row (128 dims + 4: conflict-free fragments)
+constexpr int SH_CTR0 = 4;               // row counters: [1] certain entries, [2] CTAs done, [4 + p] CTA p's candidates
+constexpr int SH_CTR_STRIDE = 256;       // words of counters per row (so at most 252 CTAs per row)
 
 struct ShSmem {
-  double qd[128][64];                    // query codes as fp64, [dim][head]: lanes read consecutive heads
-  double krow[SH_W][128];                // one key row per warp (re-scoring)
-  double contrib[SH_W][64];              // one entry's per-head terms per warp
+  int8_t qdig[3][64][SH_DLD];            // query codes as integer digits (see sh_digits), [plane][head][dim]
+  int8_t kdig[3][SH_RB][SH_DLD];         // key codes of one batch, [plane][entry][dim]
+  double contrib[SH_RB][65];             // the batch's per-head terms
+  double rs_out[SH_RB];                  // the batch's exact scores
+  float ksc[SH_RB][4];                   // their scales (E4M3 row scale in [0], MXFP4 block scales)
   uint2 cand[SH_CCAP];                   // (order key, entry id)
   uint32_t bm[SH_BMW];                   // output bitmap chunk
   uint32_t tie[SH_BMW];                  // fallback: band entries equal to tau
@@ -62,8 +68,8 @@ struct ShSmem {
   float w[64];
   float qsc[64 * 4];
   uint32_t wred[SH_W][4];
+  uint32_t coff[260];                    // gathered position of each classifying CTA's candidates
   uint32_t bins_above, bin_T, cnt, cnt2, ties, last, lo, hi;
-  int want;
   float U;
 };
 
@@ -122,63 +128,174 @@ struct KeySide {
   int HI, dI;
 };
 
-// Exact fp64 score of entry `id` of sequence b, by one warp; the query row is staged in
-// sm.qd / sm.qsc / sm.w.  Lane l forms the dot products of heads l and l + 32 over the key
-// row (exact: every partial sum is a multiple of the code grid's product unit and spans
-// fewer than 53 bits), applies the scales as the definition does, and lane 0 adds the
-// head terms w_j * max(D_j, 0) in order j = 0..H_I-1.  Returns the score on lane 0.
+// ---- exact dot products of quantised codes on the integer tensor cores
+//
+// An E4M3 value times 2^9 is an integer V with |V| < 2^18 (subnormals: the 3-bit mantissa;
+// normals: (8 + mantissa) << (exponent - 1)); V splits into three signed 7-bit digits,
+// V = d0 + 2^7 d1 + 2^14 d2.  For two code vectors of 128 dims,
+//   sum_c q_c k_c = 2^-18 sum_{a,b} 2^{7(a+b)} sum_c dq_{a,c} dk_{b,c},
+// where every inner sum (128 products of 7-bit digits, |.| < 2^21) is exact in an int32
+// accumulator of the int8 MMA, the weighted sum is exact in int64 (|.| < 2^53 since
+// sum_c |Vq Vk| < 2^43) and so is its conversion to fp64.  An e2m1 value times 2 is an
+// integer in [-12, 12]: one digit, and each 32-dim block's sum is 2^-2 times an exact int32.
+// So the per-head dot products equal the oracle's exact fp64 values bit for bit.
 template <int F>
-__device__ __noinline__ double sh_exact_score(const KeySide ks, ShSmem& sm, int b, int id) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  double* kr = sm.krow[warp];
-  const size_t koff = (size_t)b * ks.n_max + id;
-  const int dI = ks.dI, nb = dI / 32;
-  // key codes of the row as fp64
-  for (int c = lane; c < dI; c += 32) {
-    double v;
-    if (F == CSA_IFMT_E4M3) {
-      v = (double)e4m3_to_float(((const uint8_t*)ks.kI)[koff * dI + c]);
-    } else {
-      const uint8_t byte = ((const uint8_t*)ks.kI)[koff * (dI / 2) + (c >> 1)];
-      v = (double)e2m1_to_float((c & 1) ? (byte >> 4) : (byte & 0xF));
-    }
-    kr[c] = v;
-  }
-  double kscale[4] = {0.0, 0.0, 0.0, 0.0};
+__device__ __forceinline__ void sh_digits(uint32_t code, int (&d)[3]) {
+  int v, neg;
   if (F == CSA_IFMT_E4M3) {
-    kscale[0] = (double)((const float*)ks.kI_scale)[koff];
+    const int e = (code >> 3) & 0xF, mnt = code & 7;
+    v = e == 0 ? mnt : (8 + mnt) << (e - 1);
+    neg = (code >> 7) & 1;
   } else {
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      if (q < nb) kscale[q] = (double)ue8m0_to_float(((const uint8_t*)ks.kI_scale)[koff * nb + q]);
+    const int e = (code >> 1) & 3, mnt = code & 1;
+    v = e == 0 ? mnt : (2 + mnt) << (e - 1);
+    neg = (code >> 3) & 1;
   }
-  __syncwarp();
-  for (int h = 0; h < 2; ++h) {
-    const int j = lane + 32 * h;
-    if (j < ks.HI) {
-      double D = 0.0;
+  const int a = v & 127, b = (v >> 7) & 127, c = v >> 14;
+  d[0] = neg ? -a : a;
+  d[1] = neg ? -b : b;
+  d[2] = neg ? -c : c;
+}
+__device__ __forceinline__ uint32_t sh_pack4(int a, int b, int c, int d) {
+  return (uint32_t)(a & 0xFF) | ((uint32_t)(b & 0xFF) << 8) | ((uint32_t)(c & 0xFF) << 16) | ((uint32_t)(d & 0xFF) << 24);
+}
+// D (16x8 s32) += A (16x32 s8, row) * B (32x8 s8, col)
+__device__ __forceinline__ void mma_s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                       uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+               : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+               : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Digits of `cnt` rows of 128 codes (E4M3 bytes, or MXFP4 bytes of two codes) into
+// dst[plane][row][dim]; thread t converts 16 codes of row t / 8 per step.
+template <int F>
+__device__ __forceinline__ void sh_stage_digits(int8_t (*dst)[SH_DLD], size_t plane_stride, const uint8_t* const* rows,
+                                                int cnt, int dI) {
+  for (int u = threadIdx.x; u < cnt * 8; u += SH_T) {
+    const int r = u >> 3, seg = u & 7;
+    uint32_t wd[4] = {0u, 0u, 0u, 0u};
+    if (16 * seg < dI && rows[r]) {
       if (F == CSA_IFMT_E4M3) {
-        double acc = 0.0;
-#pragma unroll 8
-        for (int c = 0; c < dI; ++c) acc = fma(sm.qd[c][j], kr[c], acc);
-        D = ((double)sm.qsc[j] * kscale[0]) * acc;
+        const uint4 v = *reinterpret_cast<const uint4*>(rows[r] + 16 * seg);
+        wd[0] = v.x; wd[1] = v.y; wd[2] = v.z; wd[3] = v.w;
       } else {
-        for (int q = 0; q < nb; ++q) {
-          double part = 0.0;
-#pragma unroll 8
-          for (int c = 32 * q; c < 32 * q + 32; ++c) part = fma(sm.qd[c][j], kr[c], part);
-          D += ((double)sm.qsc[j * nb + q] * kscale[q]) * part;
-        }
+        const uint2 v = *reinterpret_cast<const uint2*>(rows[r] + 8 * seg);
+        wd[0] = v.x; wd[1] = v.y;
       }
-      sm.contrib[warp][j] = (double)sm.w[j] * fmax(D, 0.0);
+    }
+    int dg[16][3];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t code = F == CSA_IFMT_E4M3 ? (wd[i >> 2] >> (8 * (i & 3))) & 0xFFu : (wd[i >> 3] >> (4 * (i & 7))) & 0xFu;
+      sh_digits<F>(code, dg[i]);
+    }
+#pragma unroll
+    for (int p = 0; p < (F == CSA_IFMT_E4M3 ? 3 : 1); ++p) {
+      uint32_t* o = reinterpret_cast<uint32_t*>(&dst[r][16 * seg] + p * plane_stride);
+#pragma unroll
+      for (int w = 0; w < 4; ++w) o[w] = sh_pack4(dg[4 * w][p], dg[4 * w + 1][p], dg[4 * w + 2][p], dg[4 * w + 3][p]);
     }
   }
-  __syncwarp();
-  double S = 0.0;
-  if (lane == 0)
-    for (int j = 0; j < ks.HI; ++j) S += sm.contrib[warp][j];
-  __syncwarp();
-  return S;
+}
+
+// Exact fp64 scores of entries ids[0..cnt) (cnt <= SH_RB) of sequence b into sm.rs_out, by
+// the whole CTA (all threads call; barriers inside).  The query digits are in sm.qdig.  Warp w computes (16 heads x 8 entries) tiles with the int8 MMA; the
+// per-head values are then formed as the definition does (E4M3: (sq * sk) * raw; MXFP4: the
+// block terms (qs * ks) * P_b added in block order), each head's term w_j * max(D_j, 0) is
+// written, and one thread per entry adds the terms in order j = 0..H_I-1.
+template <int F>
+__device__ __noinline__ void sh_rescore(const KeySide ks, ShSmem& sm, const void* qI, size_t qrow, int b,
+                                        const int32_t* ids, int cnt) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int dI = ks.dI, nb = dI / 32, HI = ks.HI;
+  const int rowbytes = F == CSA_IFMT_E4M3 ? dI : dI / 2;
+  __shared__ const uint8_t* rowp[64];
+  (void)qI; (void)qrow;                                     // the query digits are staged in the prologue
+  __syncthreads();
+  if (tid < SH_RB) rowp[tid] = tid < cnt ? (const uint8_t*)ks.kI + ((size_t)b * ks.n_max + ids[tid]) * rowbytes : nullptr;
+  if (tid < SH_RB * 4) {
+    const int e2 = tid >> 2, q2 = tid & 3;
+    float v = 0.f;
+    if (e2 < cnt) {
+      const size_t koff = (size_t)b * ks.n_max + ids[e2];
+      if (F == CSA_IFMT_E4M3) v = q2 == 0 ? ((const float*)ks.kI_scale)[koff] : 0.f;
+      else v = q2 < nb ? ue8m0_to_float(((const uint8_t*)ks.kI_scale)[koff * nb + q2]) : 0.f;
+    }
+    sm.ksc[e2][q2] = v;
+  }
+  __syncthreads();
+  sh_stage_digits<F>(sm.kdig[0], sizeof(sm.kdig[0]), rowp, SH_RB, dI);
+  __syncthreads();
+  // ---- tiles: 4 head tiles x ceil(cnt / 8) entry tiles over the 8 warps
+  const int g = lane >> 2, tig = lane & 3;
+  const int ntile = (cnt + 7) / 8;
+  for (int job = warp; job < 4 * ntile; job += SH_W) {
+    const int mt = job & 3, nt = job >> 2;
+    // E4M3: one accumulator per digit pair (a, b), so that no MMA waits for another; MXFP4:
+    // one per 32-dim block
+    constexpr int NACC = F == CSA_IFMT_E4M3 ? 9 : 4;
+    int acc[NACC][4];
+#pragma unroll
+    for (int i = 0; i < NACC; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0;
+#pragma unroll
+    for (int kst = 0; kst < 4; ++kst) {
+      const int kc = 32 * kst + 4 * tig;
+      if (F == CSA_IFMT_E4M3) {
+        uint32_t bq[3][2];
+#pragma unroll
+        for (int pb = 0; pb < 3; ++pb) {
+          const int8_t* kb = &sm.kdig[pb][8 * nt + g][kc];
+          bq[pb][0] = *reinterpret_cast<const uint32_t*>(kb);
+          bq[pb][1] = *reinterpret_cast<const uint32_t*>(kb + 16);
+        }
+#pragma unroll
+        for (int pa = 0; pa < 3; ++pa) {
+          const int8_t* qa = &sm.qdig[pa][16 * mt + g][kc];
+          const uint32_t a0 = *reinterpret_cast<const uint32_t*>(qa);
+          const uint32_t a1 = *reinterpret_cast<const uint32_t*>(qa + 8 * SH_DLD);
+          const uint32_t a2 = *reinterpret_cast<const uint32_t*>(qa + 16);
+          const uint32_t a3 = *reinterpret_cast<const uint32_t*>(qa + 8 * SH_DLD + 16);
+#pragma unroll
+          for (int pb = 0; pb < 3; ++pb) mma_s8(acc[3 * pa + pb], a0, a1, a2, a3, bq[pb][0], bq[pb][1]);
+        }
+      } else {
+        const int8_t* qa = &sm.qdig[0][16 * mt + g][kc];
+        const int8_t* kb = &sm.kdig[0][8 * nt + g][kc];
+        mma_s8(acc[kst], *reinterpret_cast<const uint32_t*>(qa), *reinterpret_cast<const uint32_t*>(qa + 8 * SH_DLD),
+               *reinterpret_cast<const uint32_t*>(qa + 16), *reinterpret_cast<const uint32_t*>(qa + 8 * SH_DLD + 16),
+               *reinterpret_cast<const uint32_t*>(kb), *reinterpret_cast<const uint32_t*>(kb + 16));
+      }
+    }
+    // accumulator element i: head 16 mt + g + 8 (i >> 1), entry 8 nt + 2 tig + (i & 1)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int j = 16 * mt + g + 8 * (i >> 1), e = 8 * nt + 2 * tig + (i & 1);
+      if (j >= HI || e >= cnt) continue;
+      double D;
+      if (F == CSA_IFMT_E4M3) {
+        // sum over digit pairs of 2^(7 (a + b)) x the pair's exact int32 sum, exact in int64
+        const long long tot = (long long)acc[0][i] + (((long long)acc[1][i] + acc[3][i]) << 7) +
+                              (((long long)acc[2][i] + acc[4][i] + acc[6][i]) << 14) +
+                              (((long long)acc[5][i] + acc[7][i]) << 21) + ((long long)acc[8][i] << 28);
+        const double raw = (double)tot * 0x1p-18;                  // exact: |tot| < 2^53
+        D = ((double)sm.qsc[j] * (double)sm.ksc[e][0]) * raw;
+      } else {
+        D = 0.0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (q < nb) D += ((double)sm.qsc[j * nb + q] * (double)sm.ksc[e][q]) * ((double)acc[q][i] * 0.25);
+      }
+      sm.contrib[e][j] = (double)sm.w[j] * fmax(D, 0.0);
+    }
+  }
+  __syncthreads();
+  if (tid < cnt) {
+    double S = 0.0;
+    for (int jj = 0; jj < HI; ++jj) S += sm.contrib[tid][jj];
+    sm.rs_out[tid] = S;
+  }
+  __syncthreads();
 }
 
 template <int F>
@@ -194,13 +311,14 @@ indexer_select_hist_kernel(IndexerArgs a, int P, int chunk) {
   int32_t* out = a.idx_out + (size_t)row * k;
   float* sout = a.score_out ? a.score_out + (size_t)row * k : nullptr;
   uint32_t* hist = a.hist + (size_t)row * SH_BINS;
-  uint32_t* ctr = a.counters + (size_t)row * 4;              // [0] candidates, [1] certain, [2] CTAs done
+  uint32_t* ctr = a.counters + (size_t)row * SH_CTR_STRIDE;
   uint32_t* bitmap = a.bitmap + (size_t)row * (a.ld / 32);
   uint2* cand_g = a.cand + (size_t)row * a.ld;
   tc::griddep_launch_dependents();
 
-  // ---- prologue (inputs only; overlaps the scoring kernel): weights, query scales and
-  // U = sum_j |w_j| ||q_j||.  Thread t takes 32 elements of head t / 4.
+  // ---- prologue (inputs only; overlaps the scoring kernel): weights, query scales, the
+  // query row in registers as fp64 (thread t: head t / 4, dims [32 (t % 4), +32)) and
+  // U = sum_j |w_j| ||q_j||
   const size_t qrow = (size_t)row * HI * dI;
   if (tid < HI) {
     sm.w[tid] = a.w[(size_t)row * HI + tid];
@@ -209,32 +327,44 @@ indexer_select_hist_kernel(IndexerArgs a, int P, int chunk) {
       for (int q = 0; q < nb; ++q) sm.qsc[tid * nb + q] = ue8m0_to_float(((const uint8_t*)a.qI_scale)[((size_t)row * HI + tid) * nb + q]);
   }
   if (tid == 0) sm.U = 0.f;
-  __syncthreads();
   {
+    // thread t: head t / 4, dims [32 (t % 4), +32) (one MXFP4 scale block)
     const int j = tid >> 2, q = tid & 3;
     float ss = 0.f;
+    uint32_t wds[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
     if (j < HI && 32 * q < dI) {
       if (F == CSA_IFMT_E4M3) {
         const uint4* p = reinterpret_cast<const uint4*>((const uint8_t*)a.qI + qrow + (size_t)j * dI + 32 * q);
         const uint4 v0 = p[0], v1 = p[1];
-        const uint32_t wds[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-        for (int e = 0; e < 32; ++e) { const float x = e4m3_to_float((wds[e >> 2] >> (8 * (e & 3))) & 0xFFu); ss = fmaf(x, x, ss); }
-        ss *= sm.qsc[j] * sm.qsc[j];
+        wds[0] = v0.x; wds[1] = v0.y; wds[2] = v0.z; wds[3] = v0.w; wds[4] = v1.x; wds[5] = v1.y; wds[6] = v1.z; wds[7] = v1.w;
       } else {
         const uint4 v = *reinterpret_cast<const uint4*>((const uint8_t*)a.qI + (qrow + (size_t)j * dI + 32 * q) / 2);
-        const uint32_t wds[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 32; ++e) { const float x = e2m1_to_float((wds[e >> 3] >> (4 * (e & 7))) & 0xFu); ss = fmaf(x, x, ss); }
-        const float sc = sm.qsc[j * nb + q];
-        ss *= sc * sc;
+        wds[0] = v.x; wds[1] = v.y; wds[2] = v.z; wds[3] = v.w;
       }
+    }
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const float x = F == CSA_IFMT_E4M3 ? e4m3_to_float((wds[e >> 2] >> (8 * (e & 3))) & 0xFFu)
+                                         : e2m1_to_float((wds[e >> 3] >> (4 * (e & 7))) & 0xFu);
+      ss = fmaf(x, x, ss);
+    }
+    __syncthreads();                                         // w, scales, U = 0
+    if (j < HI && 32 * q < dI) {
+      const float sc = F == CSA_IFMT_E4M3 ? sm.qsc[j] : sm.qsc[j * nb + q];
+      ss *= sc * sc;
     }
     ss += __shfl_xor_sync(0xffffffffu, ss, 1);
     ss += __shfl_xor_sync(0xffffffffu, ss, 2);
     float u = (q == 0 && j < HI) ? fabsf(sm.w[j]) * sqrtf(ss) : 0.f;
     u = warp_sum(u);
     if (lane == 0) atomicAdd(&sm.U, u);
+  }
+  // the query row's integer digits for the exact re-scoring (inputs only: before the wait)
+  {
+    __shared__ const uint8_t* qrows[64];
+    if (tid < 64) qrows[tid] = tid < HI ? (const uint8_t*)a.qI + (F == CSA_IFMT_E4M3 ? qrow + (size_t)tid * dI : (qrow + (size_t)tid * dI) / 2) : nullptr;
+    __syncthreads();
+    sh_stage_digits<F>(sm.qdig[0], sizeof(sm.qdig[0]), qrows, 64, dI);
   }
   const int n = row_eligible(a, row);
   tc::griddep_wait();                                        // the scores, the histogram, knmax
@@ -244,23 +374,13 @@ indexer_select_hist_kernel(IndexerArgs a, int P, int chunk) {
     if (part == 0) {
       for (int i = tid; i < k; i += SH_T) out[i] = i < n ? i : -1;
       if (sout) {
-        // exact scores of entries 0..n-1 (one warp per entry) need the staged query row
-        for (int i = tid; i < 128 * 64; i += SH_T) {
-          const int c = i >> 6, j = i & 63;
-          double v = 0.0;
-          if (j < HI && c < dI) {
-            if (F == CSA_IFMT_E4M3) v = (double)e4m3_to_float(((const uint8_t*)a.qI)[qrow + (size_t)j * dI + c]);
-            else {
-              const uint8_t byte = ((const uint8_t*)a.qI)[(qrow + (size_t)j * dI + c) >> 1];
-              v = (double)e2m1_to_float((c & 1) ? (byte >> 4) : (byte & 0xF));
-            }
-          }
-          sm.qd[c][j] = v;
-        }
-        __syncthreads();
-        for (int i = warp; i < k; i += SH_W) {
-          const double s = i < n ? sh_exact_score<F>(ks, sm, b, i) : 0.0;
-          if (lane == 0) sout[i] = (float)s;
+        for (int i0 = 0; i0 < k; i0 += SH_RB) {
+          const int cnt = max(0, min(SH_RB, n - i0));
+          if (tid < SH_RB) sm.band_id[tid] = i0 + tid;
+          __syncthreads();
+          sh_rescore<F>(ks, sm, a.qI, qrow, b, sm.band_id, cnt);
+          if (tid < SH_RB && i0 + tid < k) sout[i0 + tid] = tid < cnt ? (float)sm.rs_out[tid] : 0.f;
+          __syncthreads();
         }
       }
     }
@@ -285,27 +405,45 @@ indexer_select_hist_kernel(IndexerArgs a, int P, int chunk) {
   const float E_max = (EU + 1.52587890625e-05f * fmaxf(fabsf(b_lo), fabsf(b_hi))) * 1.0001f;
   const float hi_thr = b_hi + 2.f * E_max, lo_thr = b_lo - 2.f * E_max;
 
-  // ---- A2: classify this CTA's chunk (whole bitmap words: chunk % 32 == 0)
+  // ---- A2: classify this CTA's chunk (whole bitmap words: chunk % 32 == 0): certain entries
+  // into the row's bitmap, candidates into this CTA's own region [c0, c0 + count) of the row's
+  // list (no place to reserve: the region holds the whole chunk), the count into ctr[4 + part]
   const int c0 = part * chunk, c1 = min(n, c0 + chunk);
   const float* srow = a.scores + (size_t)row * a.ld;
+  const int c_end = min(c0 + chunk, (int)a.ld);
+  constexpr int SH_WPT = 8;                                  // words per warp per round
+  uint2* my_cand = cand_g + c0;
+  if (tid == 0) sm.cnt = 0u;
+  __syncthreads();
   uint32_t n_sure = 0;
-  for (int base = c0 + 32 * warp; base < c0 + chunk && base < (int)a.ld; base += 32 * SH_W) {
-    const int i = base + lane;
-    const float s = i < c1 ? srow[i] : 0.f;
-    const bool sure = i < c1 && s > hi_thr;
-    const bool cnd = i < c1 && !sure && s >= lo_thr;
-    const uint32_t bs = __ballot_sync(0xffffffffu, sure);
-    const uint32_t bc = __ballot_sync(0xffffffffu, cnd);
-    if (lane == 0) bitmap[base >> 5] = bs;
-    n_sure += __popc(bs);
-    if (bc) {
-      uint32_t off = 0;
-      if (lane == 0) off = atomicAdd(&ctr[0], (uint32_t)__popc(bc));
-      off = __shfl_sync(0xffffffffu, off, 0);
-      if (cnd) cand_g[off + __popc(bc & ((1u << lane) - 1u))] = make_uint2(f32_order_key(s), (uint32_t)i);
+  for (int base0 = c0 + 32 * warp; base0 < c_end; base0 += SH_WPT * 32 * SH_W) {
+    float sv[SH_WPT];
+#pragma unroll
+    for (int u = 0; u < SH_WPT; ++u) {
+      const int i = base0 + u * 32 * SH_W + lane;
+      sv[u] = i < c1 ? __ldcg(srow + i) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < SH_WPT; ++u) {
+      const int base = base0 + u * 32 * SH_W;
+      const bool in = base < c_end && base + lane < c1;
+      const bool sure = in && sv[u] > hi_thr;
+      const bool cnd = in && !sure && sv[u] >= lo_thr;
+      const uint32_t bs = __ballot_sync(0xffffffffu, sure);
+      const uint32_t bc = __ballot_sync(0xffffffffu, cnd);
+      if (lane == 0 && base < c_end) bitmap[base >> 5] = bs;
+      n_sure += __popc(bs);
+      if (bc) {
+        uint32_t off = 0;
+        if (lane == 0) off = atomicAdd(&sm.cnt, (uint32_t)__popc(bc));
+        off = __shfl_sync(0xffffffffu, off, 0);
+        if (cnd) my_cand[off + __popc(bc & ((1u << lane) - 1u))] = make_uint2(f32_order_key(sv[u]), (uint32_t)(base + lane));
+      }
     }
   }
   if (lane == 0 && n_sure) atomicAdd(&ctr[1], n_sure);
+  __syncthreads();
+  if (tid == 0) ctr[SH_CTR0 + part] = sm.cnt;
   __threadfence();
   __syncthreads();
   if (tid == 0) sm.last = (atomicAdd(&ctr[2], 1u) == (uint32_t)(P - 1)) ? 1u : 0u;
@@ -313,50 +451,71 @@ indexer_select_hist_kernel(IndexerArgs a, int P, int chunk) {
   if (!sm.last) return;
   __threadfence();
 
-  // ---- B: the last CTA of the row.  Stage the query row as fp64 (for the re-scoring).
-  for (int i = tid; i < 128 * 64; i += SH_T) {
-    const int c = i >> 6, j = i & 63;
-    double v = 0.0;
-    if (j < HI && c < dI) {
-      if (F == CSA_IFMT_E4M3) v = (double)e4m3_to_float(((const uint8_t*)a.qI)[qrow + (size_t)j * dI + c]);
-      else {
-        const uint8_t byte = ((const uint8_t*)a.qI)[(qrow + (size_t)j * dI + c) >> 1];
-        v = (double)e2m1_to_float((c & 1) ? (byte >> 4) : (byte & 0xF));
+  // ---- B: the last CTA of the row.  The candidates' places: CTA p's count at ctr[4 + p],
+  // its list at p * chunk; sm.coff[p] = the first candidate of CTA p in the gathered order.
+  const uint32_t n_sure_all = __ldcg(&ctr[1]);
+  {
+    const uint32_t cp = tid < P ? __ldcg(&ctr[SH_CTR0 + tid]) : 0u;
+    uint32_t tot;
+    const uint32_t incl = sh_scan(cp, sm.wred, &tot);
+    if (tid < P) sm.coff[tid] = incl - cp;
+    if (tid == 0) { sm.coff[P] = tot; sm.cnt = tot; }
+  }
+  __syncthreads();
+  const uint32_t nc = sm.cnt;
+  const bool staged = nc <= (uint32_t)SH_CCAP;
+  // candidate i: staged in shared memory when they all fit, else found in its CTA's region
+  auto cget = [&](uint32_t i) -> uint2 {
+    if (staged) return sm.cand[i];
+    int lo_p = 0, hi_p = P;                                  // the last p with coff[p] <= i
+    while (hi_p - lo_p > 1) {
+      const int mid = (lo_p + hi_p) >> 1;
+      if (sm.coff[mid] <= i) lo_p = mid; else hi_p = mid;
+    }
+    return __ldcg(cand_g + (size_t)lo_p * chunk + (i - sm.coff[lo_p]));
+  };
+  // ---- B4: one histogram of the candidates over [lo_thr, hi_thr] (2048 bins of 2^shf keys,
+  // built while they are gathered); its bin [tau_lo, tau_hi] holding the want-th largest
+  // candidate is narrower than the error margin, so the band is that bin widened by 2E
+  uint32_t lo = f32_order_key(lo_thr), hi = f32_order_key(hi_thr);
+  uint32_t want = (uint32_t)k - n_sure_all;
+  int shf;
+  {
+    const int range_bits = 32 - __clz(hi - lo);
+    shf = range_bits > 11 ? range_bits - 11 : 0;
+  }
+  for (int i = tid; i < SH_BINS2; i += SH_T) sm.hist2[i] = 0u;
+  __syncthreads();
+  {
+    // every thread's candidates at once (their loads are independent): candidate i lives in
+    // the region of the last CTA p with coff[p] <= i
+    constexpr int GU = 4;
+    for (uint32_t i0 = 0; i0 < nc; i0 += GU * SH_T) {
+      uint2 c[GU];
+#pragma unroll
+      for (int u = 0; u < GU; ++u) {
+        const uint32_t i = i0 + u * SH_T + tid;
+        c[u] = make_uint2(0u, 0u);
+        if (i < nc) {
+          int lo_p = 0, hi_p = P;
+          while (hi_p - lo_p > 1) {
+            const int mid = (lo_p + hi_p) >> 1;
+            if (sm.coff[mid] <= i) lo_p = mid; else hi_p = mid;
+          }
+          c[u] = __ldcg(cand_g + (size_t)lo_p * chunk + (i - sm.coff[lo_p]));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < GU; ++u) {
+        const uint32_t i = i0 + u * SH_T + tid;
+        if (i >= nc) continue;
+        if (staged) sm.cand[i] = c[u];
+        if (c[u].x >= lo && c[u].x <= hi) atomicAdd(&sm.hist2[(c[u].x - lo) >> shf], 1u);
       }
     }
-    sm.qd[c][j] = v;
   }
-  const uint32_t nc = *(volatile uint32_t*)&ctr[0];
-  const uint32_t n_sure_all = *(volatile uint32_t*)&ctr[1];
-  const bool staged = nc <= (uint32_t)SH_CCAP;
-  // candidates: staged in shared memory when they fit, else read from L2 each pass
-  auto cget = [&](uint32_t i) { return staged ? sm.cand[i] : __ldcg(cand_g + i); };
-  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-  for (uint32_t i = tid; i < nc; i += SH_T) {
-    const uint2 c = __ldcg(cand_g + i);
-    if (staged) sm.cand[i] = c;
-    kmin = min(kmin, c.x);
-    kmax = max(kmax, c.x);
-  }
-  kmin = __reduce_min_sync(0xffffffffu, kmin);
-  kmax = __reduce_max_sync(0xffffffffu, kmax);
-  if (tid == 0) { sm.lo = 0xFFFFFFFFu; sm.hi = 0u; }
   __syncthreads();
-  if (lane == 0) { atomicMin(&sm.lo, kmin); atomicMax(&sm.hi, kmax); }
-  __syncthreads();
-  // ---- B4: tau = the exact want-th largest candidate key
-  uint32_t lo = sm.lo, hi = sm.hi;
-  uint32_t want = (uint32_t)k - n_sure_all;
-  for (int round = 0; round < 4 && lo != hi; ++round) {
-    const int range_bits = 32 - __clz(hi - lo);
-    const int shf = range_bits > 11 ? range_bits - 11 : 0;
-    for (int i = tid; i < SH_BINS2; i += SH_T) sm.hist2[i] = 0u;
-    __syncthreads();
-    for (uint32_t i = tid; i < nc; i += SH_T) {
-      const uint32_t x = cget(i).x;
-      if (x >= lo && x <= hi) atomicAdd(&sm.hist2[(x - lo) >> shf], 1u);
-    }
-    __syncthreads();
+  {
     uint32_t cnt[SH_BINS2 / SH_T];
 #pragma unroll
     for (int i = 0; i < SH_BINS2 / SH_T; ++i) cnt[i] = sm.hist2[(SH_BINS2 / SH_T) * tid + i];
@@ -368,35 +527,35 @@ indexer_select_hist_kernel(IndexerArgs a, int P, int chunk) {
     lo = nlo;
     __syncthreads();
   }
-  const float tau = f32_from_order_key(lo);
-  const float E = (EU + 1.52587890625e-05f * fabsf(tau)) * 1.0001f;
-  const float band_hi = tau + 2.f * E, band_lo = tau - 2.f * E;
+  const float tau_lo = f32_from_order_key(lo), tau_hi = f32_from_order_key(hi);
+  const float E = (EU + 1.52587890625e-05f * fmaxf(fabsf(tau_lo), fabsf(tau_hi))) * 1.0001f;
+  const float band_hi = tau_hi + 2.f * E, band_lo = tau_lo - 2.f * E;
   // ---- B5: in / band; the band is re-scored exactly and ranked
-  if (tid == 0) { sm.cnt = 0u; sm.cnt2 = 0u; sm.ties = 0u; }
+  if (tid == 0) { sm.cnt = 0u; sm.ties = 0u; }
   __syncthreads();
-  uint32_t my_in = 0, my_above = 0;
+  uint32_t my_in = 0;
   for (uint32_t i = tid; i < nc; i += SH_T) {
     const uint2 c = cget(i);
     const float s = f32_from_order_key(c.x);
     if (s > band_hi) {
       ++my_in;
     } else if (s >= band_lo) {
-      my_above += s > tau ? 1u : 0u;
       const uint32_t o = atomicAdd(&sm.cnt, 1u);
       if (o < (uint32_t)SH_BAND) sm.band_id[o] = (int32_t)c.y;
     }
   }
-  uint32_t n_in, n_above_tau;
+  uint32_t n_in;
   sh_scan(my_in, sm.wred, &n_in);
-  sh_scan(my_above, sm.wred, &n_above_tau);
   const uint32_t n_band = sm.cnt;
-  const uint32_t need = (uint32_t)k - n_sure_all - n_in;    // >= 1: tau itself is in the band
+  const uint32_t need = (uint32_t)k - n_sure_all - n_in;    // >= 1: the want-th candidate is in the band
   const bool exact = n_band <= (uint32_t)SH_BAND;
-  if (!exact && tid == 0) raise_err(a.err, CSA_DEVERR_BAND);
+  float tau = tau_lo;                                        // the fallback's exact fp32 k-th score
+  uint32_t n_above_tau = 0;
   if (exact) {
-    for (uint32_t i = warp; i < n_band; i += SH_W) {
-      const double s = sh_exact_score<F>(ks, sm, b, sm.band_id[i]);
-      if (lane == 0) sm.band_s[i] = s;
+    for (uint32_t i0 = 0; i0 < n_band; i0 += SH_RB) {
+      const int cnt = (int)min((uint32_t)SH_RB, n_band - i0);
+      sh_rescore<F>(ks, sm, a.qI, qrow, b, sm.band_id + i0, cnt);
+      if (tid < cnt) sm.band_s[i0 + tid] = sm.rs_out[tid];
     }
     __syncthreads();
     for (uint32_t i = tid; i < n_band; i += SH_T) {
@@ -410,6 +569,38 @@ indexer_select_hist_kernel(IndexerArgs a, int P, int chunk) {
       sm.band_take[i] = rank < need ? 1 : 0;
     }
     __syncthreads();
+  } else {
+    // the band outgrew its buffer (heavy ties): fall back to the fp32 order.  Refine the bin
+    // to the exact fp32 want-th largest candidate tau, then count the band entries above it.
+    if (tid == 0) raise_err(a.err, CSA_DEVERR_BAND);
+    for (int round = 0; round < 4 && lo != hi; ++round) {
+      const int range_bits = 32 - __clz(hi - lo);
+      const int sh2 = range_bits > 11 ? range_bits - 11 : 0;
+      for (int i = tid; i < SH_BINS2; i += SH_T) sm.hist2[i] = 0u;
+      __syncthreads();
+      for (uint32_t i = tid; i < nc; i += SH_T) {
+        const uint32_t x = cget(i).x;
+        if (x >= lo && x <= hi) atomicAdd(&sm.hist2[(x - lo) >> sh2], 1u);
+      }
+      __syncthreads();
+      uint32_t cnt[SH_BINS2 / SH_T];
+#pragma unroll
+      for (int i = 0; i < SH_BINS2 / SH_T; ++i) cnt[i] = sm.hist2[(SH_BINS2 / SH_T) * tid + i];
+      sh_find_bin<SH_BINS2 / SH_T>(sm, cnt, want);
+      want -= sm.bins_above;
+      const uint32_t nlo = lo + (sm.bin_T << sh2);
+      const uint64_t top = (uint64_t)nlo + ((1ull << sh2) - 1ull);
+      hi = top < (uint64_t)hi ? (uint32_t)top : hi;
+      lo = nlo;
+      __syncthreads();
+    }
+    tau = f32_from_order_key(lo);
+    uint32_t my_above = 0;
+    for (uint32_t i = tid; i < nc; i += SH_T) {
+      const float s = f32_from_order_key(cget(i).x);
+      my_above += (s > tau && s <= band_hi) ? 1u : 0u;
+    }
+    sh_scan(my_above, sm.wred, &n_above_tau);
   }
   // ---- B6: ascending write, SH_BMW bitmap words (32 * SH_BMW entries) per pass
   const int nwords = (n + 31) >> 5;
@@ -475,11 +666,15 @@ indexer_select_hist_kernel(IndexerArgs a, int P, int chunk) {
   for (uint32_t i = written + tid; i < (uint32_t)k; i += SH_T) out[i] = -1;
   if (written != (uint32_t)k && tid == 0) raise_err(a.err, CSA_DEVERR_BAND);
   if (sout) {
+    // the exact score of every selected entry (the output is written: read it back)
     __syncthreads();
-    for (int i = warp; i < k; i += SH_W) {
-      const int id = __ldcg(out + i);
-      const double s = id >= 0 ? sh_exact_score<F>(ks, sm, b, id) : 0.0;
-      if (lane == 0) sout[i] = (float)s;
+    for (int i0 = 0; i0 < k; i0 += SH_RB) {
+      const int cnt = min(SH_RB, (int)written - i0);
+      if (tid < SH_RB) sm.band_id[tid] = (i0 + tid < k) ? __ldcg(out + i0 + tid) : 0;
+      __syncthreads();
+      if (cnt > 0) sh_rescore<F>(ks, sm, a.qI, qrow, b, sm.band_id, cnt);
+      if (tid < SH_RB && i0 + tid < k) sout[i0 + tid] = tid < cnt ? (float)sm.rs_out[tid] : 0.f;
+      __syncthreads();
     }
   }
 }
@@ -501,7 +696,7 @@ cudaError_t launch_indexer_select_hist(const IndexerArgs& a, cudaStream_t st) {
   int64_t chunk = (a.n_max + P - 1) / P;
   chunk = (chunk + 31) / 32 * 32;
   P = (int)((a.n_max + chunk - 1) / chunk);
-  if ((int64_t)rows * P > 0x7fffffffLL) return cudaErrorNotSupported;
+  if ((int64_t)rows * P > 0x7fffffffLL || P > SH_CTR_STRIDE - SH_CTR0) return cudaErrorNotSupported;
   const size_t smem = sizeof(ShSmem);
   auto kern = a.ifmt == CSA_IFMT_E4M3 ? indexer_select_hist_kernel<CSA_IFMT_E4M3> : indexer_select_hist_kernel<CSA_IFMT_MXFP4>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -521,6 +716,6 @@ cudaError_t launch_indexer_select_hist(const IndexerArgs& a, cudaStream_t st) {
   return cudaLaunchKernelEx(&cfg, kern, a, P, (int)chunk);
 }
 
-static_assert(sizeof(ShSmem) <= 232448, "shared memory budget of one CTA (227 KB)");
+static_assert(sizeof(ShSmem) + 1024 <= 232448, "shared memory budget of one CTA (227 KB, with 1 KB of row pointers)");
 
 }  // namespace csa
