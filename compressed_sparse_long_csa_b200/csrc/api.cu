@@ -205,14 +205,15 @@ static int64_t idx_ld(int64_t n_max) { return (int64_t)round_up((size_t)n_max, 6
 // (select_hist.cu), which needs its own workspace regions.
 constexpr int kHistMaxTq = 3;
 constexpr size_t kHistBins = 4096;
+constexpr size_t kHistFine = 16;          // fine bins per coarse bin
 constexpr size_t kHistCounters = 256;     // per row: certain count, CTAs done, per-CTA candidate counts
 
 // Workspace layout of lightning_index (each region 256-byte aligned):
 //   scores [R][ld] fp32 | knmax [B] | keyrange [R][2] | (decode rows:) hist [R][4096] |
-//   counters [R][256] | bitmap [R][ld/32] | cand [R][ld] (order key, id)
+//   fhist [R][65536] | counters [R][256] | bitmap [R][ld/32] | band [R][ld] x 16 bytes
 // R = B * Tq.  knmax .. counters is one contiguous region, zeroed by one memset per call.
 struct IdxWs {
-  size_t scores, knmax, keyrange, hist, counters, bitmap, cand, end, zero_end;
+  size_t scores, knmax, keyrange, hist, fhist, counters, bitmap, cand, end, zero_end;
 };
 static IdxWs idx_ws_layout(int B, int Tq, int64_t n_max) {
   const size_t R = (size_t)B * Tq, ld = (size_t)idx_ld(n_max);
@@ -221,17 +222,14 @@ static IdxWs idx_ws_layout(int B, int Tq, int64_t n_max) {
   L.knmax = round_up(R * ld * sizeof(float), 256);
   L.keyrange = L.knmax + round_up((size_t)B * sizeof(unsigned), 256);
   L.hist = L.keyrange + round_up(R * 2 * sizeof(unsigned), 256);
-  L.counters = L.hist;
-  L.bitmap = L.hist;
-  L.cand = L.hist;
-  L.end = L.hist;
-  L.zero_end = L.hist;
+  L.fhist = L.counters = L.bitmap = L.cand = L.end = L.zero_end = L.hist;
   if (Tq <= kHistMaxTq) {
-    L.counters = L.hist + round_up(R * kHistBins * sizeof(unsigned), 256);
+    L.fhist = L.hist + round_up(R * kHistBins * sizeof(unsigned), 256);
+    L.counters = L.fhist + round_up(R * kHistBins * kHistFine * sizeof(unsigned), 256);
     L.zero_end = L.counters + R * kHistCounters * sizeof(unsigned);
     L.bitmap = L.counters + round_up(R * kHistCounters * sizeof(unsigned), 256);
     L.cand = L.bitmap + round_up(R * (ld / 32) * sizeof(unsigned), 256);
-    L.end = L.cand + round_up(R * ld * 2 * sizeof(unsigned), 256);
+    L.end = L.cand + round_up(R * ld * 16, 256);
   }
   return L;
 }
@@ -279,9 +277,10 @@ static csa_status run_lightning_index(const void* qI, const void* qI_scale, cons
   const bool hist_path = Tq <= kHistMaxTq && !bf16_scores;
   if (hist_path) {
     a.hist = (unsigned*)(ws + L.hist);
+    a.fhist = (unsigned*)(ws + L.fhist);
     a.counters = (unsigned*)(ws + L.counters);
     a.bitmap = (unsigned*)(ws + L.bitmap);
-    a.cand = (uint2*)(ws + L.cand);
+    a.cand = ws + L.cand;
   }
   cudaError_t e = cudaMemsetAsync(ws + L.knmax, 0, L.zero_end - L.knmax, S(stream));
   if (e != cudaSuccess) return CSA_ERR_CUDA;
@@ -290,7 +289,7 @@ static csa_status run_lightning_index(const void* qI, const void* qI_scale, cons
     e = launch_indexer_scores_tc(a, S(stream), &used_tc);       // sets a.eps_dot of its path
     if (e != cudaSuccess) return CSA_ERR_CUDA;
   }
-  if (!used_tc) a.hist = nullptr;                              // the CUDA-core scores come without a histogram
+  if (!used_tc) a.hist = a.fhist = nullptr;                    // the CUDA-core scores come without histograms
   if (!used_tc) {
     // sequential fp32 FMA accumulation of d_I exact products: |err| <= (d_I+2) u sum|q c k c|
     a.eps_dot = (float)(d_I + 4) * 5.9604645e-08f * 1.25f;

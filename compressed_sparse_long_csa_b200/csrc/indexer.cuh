@@ -27,10 +27,11 @@ struct IndexerArgs {
   float eps_dot;              // bound on |fp32 dot - exact| / (||q|| ||k||) of the scoring path
   int score_bf16;             // 1: scores are rounded to bf16 before they are stored (lightning_index_bf16)
   // decode rows (Tq <= 3) only, else null: the histogram-seeded selection (select_hist.cu)
-  unsigned* hist;             // [B*Tq][4096] score histogram (order key >> 20), zeroed per call
-  unsigned* counters;         // [B*Tq][256]: certain entries, CTAs done, per-CTA candidate counts; zeroed per call
+  unsigned* hist;             // [B*Tq][4096] coarse score histogram (order key >> 20), zeroed per call
+  unsigned* fhist;            // [B*Tq][65536] fine score histogram (order key >> 16), zeroed per call
+  unsigned* counters;         // [B*Tq][256]: certain entries, CTAs done, overflow, per-CTA band counts; zeroed
   unsigned* bitmap;           // [B*Tq][ld/32] certain entries
-  uint2* cand;                // [B*Tq][ld] candidates (order key, entry id)
+  void* cand;                 // [B*Tq][ld] band entries, 16 bytes each (order key, entry id, exact score)
 };
 
 // Entries of one selection row: n_valid[row] (topk_select), else the indexer's

@@ -40,15 +40,59 @@ struct IdxTcParams {
 
 constexpr int IT_THREADS = 384;  // warp 0 TMA, warp 1 MMA, warps 4..11 epilogue (two warpgroups)
 
-// Level-1 bins of the score histogram that seeds the decode selection (select_hist.cu):
-// the top 12 bits of a score's monotone order key.
+// The score histograms that seed the decode selection (select_hist.cu): coarse bins are the
+// top 12 bits of a score's monotone order key, fine bins the top 16.  A CTA counts its scores
+// in a window of IT_FWIN fine bins in shared memory (16-aligned, anchored on the first score
+// it sees: a row's scores span a few hundred fine bins) and adds the window to the row's
+// fine and coarse histograms once, at the end; a score outside the window goes to them
+// directly.
 constexpr int IT_HBINS = 4096;
+constexpr int IT_FWIN = 2048;
+constexpr uint32_t IT_FNONE = 0xFFFFFFFFu;
+
+// Count one score (order key) of row `row` (all lanes call; `valid` lanes count).
+__device__ __forceinline__ void hist_count(uint32_t* fwin, uint32_t* fbase, const IndexerArgs& a, size_t row,
+                                           uint32_t key, bool valid) {
+  if (!valid) return;
+  const uint32_t fb = key >> 16;
+  uint32_t base = *(volatile uint32_t*)fbase;
+  if (base == IT_FNONE) {
+    const uint32_t lo = fb > (uint32_t)(IT_FWIN / 2) ? ((fb - IT_FWIN / 2) & ~15u) : 0u;
+    const uint32_t want = lo < 65536u - IT_FWIN ? lo : 65536u - IT_FWIN;
+    const uint32_t old = atomicCAS(fbase, IT_FNONE, want);
+    base = old == IT_FNONE ? want : old;
+  }
+  const uint32_t o = fb - base;
+  if (o < (uint32_t)IT_FWIN) {
+    atomicAdd(fwin + o, 1u);
+  } else {
+    atomicAdd(a.fhist + row * (IT_HBINS * 16) + fb, 1u);
+    atomicAdd(a.hist + row * IT_HBINS + (fb >> 4), 1u);
+  }
+}
+
+// Add a CTA's window to the row's histograms (all threads of the CTA call, after a barrier).
+__device__ __forceinline__ void hist_flush(const uint32_t* fwin, uint32_t fbase, const IndexerArgs& a, size_t row) {
+  if (fbase == IT_FNONE) return;
+  uint32_t* gf = a.fhist + row * (IT_HBINS * 16) + fbase;
+  for (int i = threadIdx.x; i < IT_FWIN; i += blockDim.x) {
+    const uint32_t c = fwin[i];
+    if (c) atomicAdd(gf + i, c);
+  }
+  for (int g = threadIdx.x; g < IT_FWIN / 16; g += blockDim.x) {
+    uint32_t c = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) c += fwin[16 * g + i];
+    if (c) atomicAdd(a.hist + row * IT_HBINS + (fbase >> 4) + g, c);
+  }
+}
 
 template <int G, int STAGES, bool HIST>
 struct IdxSmem {
   alignas(1024) uint8_t q[G * 64 * IT_KB];
   alignas(1024) uint8_t k[STAGES][IT_TILE_BYTES];
-  uint32_t hist[HIST ? IT_HBINS : 1];
+  uint32_t fwin[HIST ? IT_FWIN : 1];
+  uint32_t fbase;
   alignas(8) uint64_t full[STAGES];
   uint64_t empty[STAGES];
   uint64_t tfull[4];
@@ -111,8 +155,10 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     }
     sm.issued0 = n0;
   }
-  if (HIST)
-    for (int i = threadIdx.x; i < IT_HBINS; i += blockDim.x) sm.hist[i] = 0u;
+  if (HIST) {
+    for (int i = threadIdx.x; i < IT_FWIN; i += blockDim.x) sm.fwin[i] = 0u;
+    if (threadIdx.x == 0) sm.fbase = IT_FNONE;
+  }
   for (int i = threadIdx.x; i < G * 64; i += blockDim.x) {
     const int g = i / 64, j = i % 64;
     const int t = qg * G + g;
@@ -206,20 +252,19 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         // four partial sums over the heads (j mod 4)
         float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int hlf = 0; hlf < 2; ++hlf) {
-          uint32_t v[32];
-          const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + acc * N + g * 64 + hlf * 32;
+        for (int q16 = 0; q16 < 4; ++q16) {
+          uint32_t v[16];
+          const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + acc * N + g * 64 + q16 * 16;
           tc::tmem_ld16(ta, v);
-          tc::tmem_ld16(ta + 16, v + 16);
-          // the 32 weights as eight 16-byte loads, in flight with the TMEM loads (one load
-          // per weight exposed its latency 64 times per tile)
-          const float4* w4p = reinterpret_cast<const float4*>(&sm.wq[g][hlf * 32]);
-          float4 w4[8];
+          // the 16 weights as four 16-byte loads, in flight with the TMEM load (one load per
+          // weight exposed its latency 64 times per tile)
+          const float4* w4p = reinterpret_cast<const float4*>(&sm.wq[g][q16 * 16]);
+          float4 w4[4];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) w4[u] = w4p[u];
+          for (int u = 0; u < 4; ++u) w4[u] = w4p[u];
           tc::tmem_ld_wait();
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
+          for (int u = 0; u < 4; ++u) {
             part[0] = fmaf(w4[u].x, fmaxf(__uint_as_float(v[4 * u]), 0.f), part[0]);
             part[1] = fmaf(w4[u].y, fmaxf(__uint_as_float(v[4 * u + 1]), 0.f), part[1]);
             part[2] = fmaf(w4[u].z, fmaxf(__uint_as_float(v[4 * u + 2]), 0.f), part[2]);
@@ -234,12 +279,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
           kmax = fmaxf(kmax, sk);
           kr[g].add(sc);
         }
-        if (HIST) {
-          // one shared-memory atomic per distinct bin of the warp
-          const uint32_t bin = valid ? (f32_order_key(sc) >> 20) : 0xFFFFFFFFu;
-          const unsigned peers = __match_any_sync(0xffffffffu, bin);
-          if (valid && lane == __ffs(peers) - 1) atomicAdd(&sm.hist[bin], (uint32_t)__popc(peers));
-        }
+        if (HIST && a.hist) hist_count(sm.fwin, &sm.fbase, a, (size_t)sm.row[g], f32_order_key(sc), valid);
       }
       tc::fence_before_sync();
       __syncwarp();
@@ -258,14 +298,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, NCOLS);
   }
-  if (HIST && a.hist) {
-    // this CTA's histogram into the row's (only the bins in use: a few dozen)
-    uint32_t* gh = a.hist + (size_t)sm.row[0] * IT_HBINS;
-    for (int i = threadIdx.x; i < IT_HBINS; i += blockDim.x) {
-      const uint32_t c = sm.hist[i];
-      if (c) atomicAdd(gh + i, c);
-    }
-  }
+  if (HIST && a.hist) hist_flush(sm.fwin, sm.fbase, a, (size_t)sm.row[0]);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -283,7 +316,8 @@ template <int STAGES>
 struct MxSmem {
   alignas(1024) uint8_t q[64 * MX_KB];
   alignas(1024) uint8_t k[STAGES][MX_TILE_BYTES];
-  uint32_t hist[IT_HBINS];
+  uint32_t fwin[IT_FWIN];
+  uint32_t fbase;
   alignas(8) uint64_t full[STAGES];
   uint64_t empty[STAGES];
   uint64_t sfa_full[STAGES];
@@ -350,7 +384,8 @@ indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     sm.issued0 = n0;
   }
   if (threadIdx.x < 64) sm.w[threadIdx.x] = threadIdx.x < a.H_I ? a.w[(size_t)row * a.H_I + threadIdx.x] : 0.f;
-  for (int i = threadIdx.x; i < IT_HBINS; i += blockDim.x) sm.hist[i] = 0u;
+  for (int i = threadIdx.x; i < IT_FWIN; i += blockDim.x) sm.fwin[i] = 0u;
+  if (threadIdx.x == 0) sm.fbase = IT_FNONE;
   if (warp == 1) { tc::tmem_alloc(&sm.tmem_base, MX_COLS); tc::tmem_relinquish(); }
   tc::fence_before_sync();
   __syncthreads();
@@ -493,11 +528,7 @@ indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         a.scores[(size_t)row * a.ld + s] = val;
         kr.add(val);
       }
-      {
-        const uint32_t bin = valid ? (f32_order_key(val) >> 20) : 0xFFFFFFFFu;
-        const unsigned peers = __match_any_sync(0xffffffffu, bin);
-        if (valid && lane == __ffs(peers) - 1) atomicAdd(&sm.hist[bin], (uint32_t)__popc(peers));
-      }
+      if (a.hist) hist_count(sm.fwin, &sm.fbase, a, (size_t)row, f32_order_key(val), valid);
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&sm.tempty[acc]);
@@ -513,13 +544,7 @@ indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, MX_COLS);
   }
-  if (a.hist) {
-    uint32_t* gh = a.hist + (size_t)row * IT_HBINS;
-    for (int i = threadIdx.x; i < IT_HBINS; i += blockDim.x) {
-      const uint32_t c = sm.hist[i];
-      if (c) atomicAdd(gh + i, c);
-    }
-  }
+  if (a.hist) hist_flush(sm.fwin, sm.fbase, a, (size_t)row);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
