@@ -79,7 +79,9 @@ def algorithmic_bytes(wid, D):
         N, d, k, W, H, dv, dI = D["N"], D["d"], D["k"], D["W"], D["H"], D["dv"], D["dI"]
         kI_row = dI + 4 if D["ifmt"] == "e4m3" else dI // 2 + dI // 32
         per = dict(
-            compress=(4 * 4 * d * 2 + 2 * 4 * d * 2 * 0) + 8 * 4 * d + d * 2,   # 4 series x 4 tokens + biases + entry
+            # the block's 4 series x 4 tokens + biases + the entry; its key's 4 x 4 indexer
+            # activations + key row; the raw row into the window
+            compress=(4 * 4 * d * 2) + 8 * 4 * d + d * 2 + (4 * 4 * dI * 2 + kI_row) + 2 * d * 2,
             indexer=N * kI_row + 64 * (dI + 4) + 64 * 4,
             attention=k * d * 2 + W * d * 2 + H * d * 2 + H * dv * 2,
         )
@@ -273,10 +275,14 @@ def run_ours(args, wid, name):
     p = "h_"
 
     def part_compress(T):
-        if wid in (1, 3, 4):
+        if "CaI" in T:
+            steps._decode_append(T, D, None)      # cache entry, its key and the window row, one launch
+        elif wid in (1, 3, 4):
             csa.csa_compress(T["Ca"], T["Cb"], T["Za"], T["Zb"], T["Ba"], T["Bb"], T["prev_Cb"], T["prev_Zb"],
                              T["entry0"], T["cache"], m=D["m"])
         else:
+            if "raw_new" in T:
+                csa.window_append(T["raw_new"], T["win"], T["win_slot"])
             csa.hca_compress(T["C"], T["Z"], T["bias"], T["entry0"], T["cache"], D["m_prime"])
 
     def part_indexer(T):
@@ -378,10 +384,11 @@ def run_ours(args, wid, name):
     value = job_rate(tokens_per_step, world, ms_per_step)
 
     # ---- e2e through the public API with host buffers (max over ranks too)
-    e2e_ms, h2d, d2h = measure_e2e(args, wid, wl, Ts, D, csa, steps)
+    e2e_ms, h2d, d2h, h2d_gbs = measure_e2e(args, wid, wl, Ts, D, csa, steps)
     e2e_ms = max_over_ranks(e2e_ms, world, "cuda")
     e2e = {"value": job_rate(tokens_per_step, world, e2e_ms), "unit": "tokens/s",
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "h2d_link_gbs": h2d_gbs, "h2d_copy_ms": h2d / h2d_gbs * 1e-6}
     ab = algorithmic_bytes(wid, D)
     comp = ["compress", "indexer", "attention", "hca"]
     mean_ms = per.mean(axis=0)
@@ -649,12 +656,17 @@ def measure_e2e(args, wid, wl, Ts, D, csa, steps):
     step i computes (what a serving loop does); the region ends when the last result is
     on the host.  The packed buffers hold exactly the tensors the step reads as input
     and writes as result; every other tensor (caches, workspaces) stays resident, and the
-    steps rotate over the resident copies as the device-timed steps do."""
+    steps rotate over the resident copies as the device-timed steps do.  Each step's calls
+    are one CUDA graph launch (captured per buffer set and resident copy)."""
     import torch
     T = Ts[0]
-    per_step_in = {1: ["Ca", "Cb", "Za", "Zb", "q", "qI", "qI_scale", "w", "win"],
-                   2: ["C", "Z", "q", "win"], 3: ["Ca", "Cb", "Za", "Zb", "q", "qI", "qI_scale", "w"],
-                   4: ["Ca", "Cb", "Za", "Zb", "q", "qI", "qI_scale", "w", "win", "h_C", "h_Z", "h_q", "h_win"]}[wid]
+    # a decode step brings its block's compressor and indexer activations, its query and its
+    # raw latent (appended to the resident window ring by the library); the window's other
+    # rows, the caches and the keys stay resident
+    fresh = ["CaI", "CbI", "ZaI", "ZbI", "raw_new"]
+    per_step_in = {1: ["Ca", "Cb", "Za", "Zb", "q", "qI", "qI_scale", "w"] + fresh,
+                   2: ["C", "Z", "q", "raw_new"], 3: ["Ca", "Cb", "Za", "Zb", "q", "qI", "qI_scale", "w"],
+                   4: ["Ca", "Cb", "Za", "Zb", "q", "qI", "qI_scale", "w"] + fresh + ["h_C", "h_Z", "h_q", "h_raw_new"]}[wid]
     outs = ["out", "idx"] if wid != 2 else ["out"]
     if wid == 4:
         outs.append("h_out")
@@ -687,6 +699,19 @@ def measure_e2e(args, wid, wl, Ts, D, csa, steps):
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
     ev_comp = [torch.cuda.Event(), torch.cuda.Event()]
     ev_out = [torch.cuda.Event(), torch.cuda.Event()]
+    # the step's calls, captured once per (buffer set, resident copy) into a CUDA graph, as a
+    # serving loop would: each step is then one launch from the host
+    step_graphs = {}
+    for j in range(2):
+        for c in range(len(Ts)):
+            Tjc = dict(Ts[c], **io[j])
+            steps.run_step(wl.kind, Tjc, D)                # warm (and resolve lazy set-up) outside capture
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                steps.run_step(wl.kind, Tjc, D)
+            step_graphs[(j, c)] = g
+    torch.cuda.synchronize()
 
     def run(nsteps, e0=None, e1=None):
         if e0 is not None:
@@ -695,7 +720,6 @@ def measure_e2e(args, wid, wl, Ts, D, csa, steps):
         s_out.wait_stream(comp)
         for i in range(nsteps):
             j = i & 1
-            Tj = dict(Ts[i % len(Ts)], **io[j])
             ev_in = torch.cuda.Event()
             with torch.cuda.stream(s_in):
                 if i >= 2:
@@ -705,7 +729,7 @@ def measure_e2e(args, wid, wl, Ts, D, csa, steps):
             comp.wait_event(ev_in)
             if i >= 2:
                 comp.wait_event(ev_out[j])              # step i-2's results have left this set
-            steps.run_step(wl.kind, Tj, D)
+            step_graphs[(j, i % len(Ts))].replay()      # the step's calls on set j and resident copy i
             ev_comp[j].record(comp)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_comp[j])
@@ -722,7 +746,19 @@ def measure_e2e(args, wid, wl, Ts, D, csa, steps):
     e1 = torch.cuda.Event(enable_timing=True)
     run(n, e0, e1)
     torch.cuda.synchronize()
-    return e0.elapsed_time(e1) / n, h2d, d2h
+    # the host link alone: the same packed input copy, back to back (the e2e roofline)
+    link = []
+    for _ in range(3):
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(s_in):
+            a.record(s_in)
+            for _ in range(n):
+                dev_in[0].copy_(host_in, non_blocking=True)
+            b_.record(s_in)
+        torch.cuda.synchronize()
+        link.append(a.elapsed_time(b_) / n)
+    h2d_gbs = h2d / (min(link) * 1e-3) / 1e9
+    return e0.elapsed_time(e1) / n, h2d, d2h, h2d_gbs
 
 
 def cpu_baseline(wid, wl, min_s=3.0, max_reps=20):

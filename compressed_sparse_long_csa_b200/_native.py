@@ -25,6 +25,8 @@ _SIGS = {
     "csa_wait_probe": ([C.c_uint64, _vp], _i32),
     "csa_compress": ([_vp] * 10 + [_i64, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
     "csa_compress_kv8": ([_vp] * 10 + [_i64, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
+    "csa_decode_append": ([_vp] * 10 + [_i64, _i32] + [_vp] * 10 + [_i32, _i32, _vp, _vp, _vp, _i32, _i32, _i32, _vp], _i32),
+    "window_append": ([_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp], _i32),
     "index_key_compress": ([_vp] * 11 + [_i64, _i32, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
     "shard_topk_merge": ([_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp], _i32),
     "attn_merge_shards": ([_vp, _vp, _i32, _i64, _i32, _i32, _vp, _vp, _vp], _i32),
@@ -76,6 +78,30 @@ def _stream(stream):
 
 def _dtype_code(t):
     return CSA_BF16 if t.dtype == torch.bfloat16 else CSA_F32
+
+
+def csa_decode_append(Ca, Cb, Za, Zb, Ba, Bb, prev_Cb, prev_Zb, entry0, cache, keys=None, window=None, stream=None):
+    """One decode step's appends in one launch (see csa.h).  keys = (CaI, CbI, ZaI, ZbI, BaI,
+    BbI, prev_CbI, prev_ZbI, kI, kI_scale, ifmt) or None; window = (raw_new, win, win_slot) or None."""
+    B, _, d = Ca.shape
+    kp = [None] * 10
+    d_I, ifmt = 0, CSA_IFMT_E4M3
+    if keys is not None:
+        kp = [_p(t) for t in keys[:10]]
+        d_I, ifmt = keys[0].shape[-1], keys[10]
+    raw_new, win, slot, W = None, None, None, 0
+    if window is not None:
+        raw_new, win, slot = window
+        W = win.shape[1]
+    _check(lib.csa_decode_append(_p(Ca), _p(Cb), _p(Za), _p(Zb), _p(Ba), _p(Bb), _p(prev_Cb), _p(prev_Zb), _p(entry0),
+                                 _p(cache), cache.shape[1], d, *kp, d_I, ifmt, _p(raw_new), _p(win), _p(slot), W, B,
+                                 _dtype_code(Ca), _stream(stream)), "csa_decode_append")
+
+
+def window_append(raw_new, win, win_slot, stream=None):
+    B, W, d = win.shape
+    _check(lib.window_append(_p(raw_new), _p(win), _p(win_slot), B, W, d, _dtype_code(win), _stream(stream)),
+           "window_append")
 
 
 def wait_probe(limit_ns: int, stream=None):

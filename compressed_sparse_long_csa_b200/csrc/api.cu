@@ -25,6 +25,12 @@ cudaError_t launch_grouped_out_proj(const void* o, int T, int H, int dv, int g, 
                                     const void* W2, int d, void* u, void* y, float* part, size_t part_elems,
                                     cudaStream_t st, unsigned* err);
 cudaError_t launch_wait_probe(uint64_t limit_ns, cudaStream_t st, unsigned* err);
+cudaError_t launch_decode_append(const void*, const void*, const void*, const void*, const float*, const float*,
+                                 const void*, const void*, const int32_t*, void*, int64_t, int, const void*,
+                                 const void*, const void*, const void*, const float*, const float*, const void*,
+                                 const void*, void*, void*, int, int, const void*, void*, const int32_t*, int, int,
+                                 int, cudaStream_t, unsigned*);
+cudaError_t launch_window_append(const void*, void*, const int32_t*, int, int, int, int, cudaStream_t, unsigned*);
 cudaError_t launch_index_key_compress(const void*, const void*, const void*, const void*, const float*,
                                       const float*, const void*, const void*, const int32_t*, void*, void*, int64_t,
                                       int, int, int, int, int, cudaStream_t, unsigned*);
@@ -161,6 +167,49 @@ csa_status csa_compress_kv8(const void* Ca, const void* Cb, const void* Za, cons
   REQUIRE(err, CSA_ERR_CUDA);
   return cuda_status(launch_csa_compress_kv8(Ca, Cb, Za, Zb, Ba, Bb, prev_Cb, prev_Zb, entry0, cache8, n_max, B,
                                              T_new, dtype, S(stream), err));
+}
+
+csa_status csa_decode_append(const void* Ca, const void* Cb, const void* Za, const void* Zb, const float* Ba,
+                             const float* Bb, const void* prev_Cb, const void* prev_Zb, const int32_t* entry0,
+                             void* cache, int64_t n_max, int d, const void* CaI, const void* CbI, const void* ZaI,
+                             const void* ZbI, const float* BaI, const float* BbI, const void* prev_CbI,
+                             const void* prev_ZbI, void* kI, void* kI_scale, int d_I, int ifmt, const void* raw_new,
+                             void* win, const int32_t* win_slot, int W, int B, int dtype, void* stream) {
+  REQUIRE(dtype == CSA_F32 || dtype == CSA_BF16, CSA_ERR_DTYPE);
+  const int vec = dtype == CSA_BF16 ? 8 : 4;
+  REQUIRE(B >= 1 && B <= 65535 && n_max >= 1 && d >= 1, CSA_ERR_SHAPE);
+  REQUIRE(d % vec == 0 && d / vec <= 96, CSA_ERR_UNSUPPORTED);
+  REQUIRE_PTR(Ca); REQUIRE_PTR(Cb); REQUIRE_PTR(Za); REQUIRE_PTR(Zb); REQUIRE_PTR(Ba); REQUIRE_PTR(Bb);
+  REQUIRE_PTR(prev_Cb); REQUIRE_PTR(prev_Zb); REQUIRE_PTR(cache);
+  REQUIRE(entry0, CSA_ERR_NULL);
+  if (CaI) {
+    REQUIRE(ifmt == CSA_IFMT_E4M3 || ifmt == CSA_IFMT_MXFP4, CSA_ERR_DTYPE);
+    REQUIRE(d_I == 32 || d_I == 64 || d_I == 128 || (d_I == 256 && dtype == CSA_BF16), CSA_ERR_UNSUPPORTED);
+    REQUIRE_PTR(CbI); REQUIRE_PTR(ZaI); REQUIRE_PTR(ZbI); REQUIRE_PTR(BaI); REQUIRE_PTR(BbI);
+    REQUIRE_PTR(prev_CbI); REQUIRE_PTR(prev_ZbI); REQUIRE_PTR(kI); REQUIRE_PTR(kI_scale);
+  }
+  if (raw_new) {
+    REQUIRE(W >= 1 && W <= 4096, CSA_ERR_SHAPE);
+    REQUIRE_PTR(win);
+    REQUIRE(win_slot, CSA_ERR_NULL);
+  }
+  unsigned* err = device_error_word();
+  REQUIRE(err, CSA_ERR_CUDA);
+  return cuda_status(launch_decode_append(Ca, Cb, Za, Zb, Ba, Bb, prev_Cb, prev_Zb, entry0, cache, n_max, d, CaI, CbI,
+                                          ZaI, ZbI, BaI, BbI, prev_CbI, prev_ZbI, kI, kI_scale, d_I, ifmt, raw_new, win,
+                                          win_slot, W, B, dtype, S(stream), err));
+}
+
+csa_status window_append(const void* raw_new, void* win, const int32_t* win_slot, int B, int W, int d, int dtype,
+                         void* stream) {
+  REQUIRE(dtype == CSA_F32 || dtype == CSA_BF16, CSA_ERR_DTYPE);
+  REQUIRE(B >= 1 && B <= 65535 && W >= 1 && W <= 4096 && d >= 1, CSA_ERR_SHAPE);
+  REQUIRE(d % (dtype == CSA_BF16 ? 8 : 4) == 0, CSA_ERR_SHAPE);
+  REQUIRE_PTR(raw_new); REQUIRE_PTR(win);
+  REQUIRE(win_slot, CSA_ERR_NULL);
+  unsigned* err = device_error_word();
+  REQUIRE(err, CSA_ERR_CUDA);
+  return cuda_status(launch_window_append(raw_new, win, win_slot, W, B, d, dtype, S(stream), err));
 }
 
 csa_status hca_compress(const void* C, const void* Z, const float* bias, const int32_t* entry0, void* cache,

@@ -221,6 +221,10 @@ __device__ __forceinline__ int mx_exponent(float amax) {
   return e < -127 ? -127 : e;
 }
 
+template <int VEC, int FMT>
+__device__ __forceinline__ void store_index_key(const float (&x)[VEC], size_t row, int d, int g, int tpe,
+                                                unsigned gmask, uint8_t* __restrict__ kI, void* __restrict__ kI_scale);
+
 template <typename T, int FMT>
 __global__ void __launch_bounds__(256)
 index_key_compress_kernel(const T* __restrict__ Ca, const T* __restrict__ Cb, const T* __restrict__ Za,
@@ -242,7 +246,15 @@ index_key_compress_kernel(const T* __restrict__ Ca, const T* __restrict__ Cb, co
   float x[VEC];
   const int e = pool_m4<T>(Ca, Cb, Za, Zb, Ba, Bb, pCb, pZb, entry0, n_max, T_new, d, b, j, c0, x, err);
   if (e < 0) return;                                      // the same for the whole group
-  const size_t row = (size_t)b * n_max + e;
+  store_index_key<VEC, FMT>(x, (size_t)b * n_max + e, d, g, tpe, gmask, kI, kI_scale);
+}
+
+// The quantised key of one pooled entry: thread g of the entry's tpe threads (an aligned lane
+// group, mask gmask) holds components [g * VEC, g * VEC + VEC) in x.
+template <int VEC, int FMT>
+__device__ __forceinline__ void store_index_key(const float (&x)[VEC], size_t row, int d, int g, int tpe,
+                                                unsigned gmask, uint8_t* __restrict__ kI, void* __restrict__ kI_scale) {
+  const int c0 = g * VEC;
   float amax = 0.f;
 #pragma unroll
   for (int i = 0; i < VEC; ++i) amax = fmaxf(amax, fabsf(x[i]));
@@ -270,6 +282,78 @@ index_key_compress_kernel(const T* __restrict__ Ca, const T* __restrict__ Cb, co
     if (VEC == 8) *reinterpret_cast<uint32_t*>(dst) = w;
     else *reinterpret_cast<uint16_t*>(dst) = (uint16_t)w;
     if (g % TPB == 0) reinterpret_cast<uint8_t*>(kI_scale)[row * (d / 32) + c0 / 32] = (uint8_t)(ex + 127);
+  }
+}
+
+// ---- one decode step's appends in one launch --------------------------------------------------
+// The token that completes block e = entry0[b] (m = 4) of sequence b brings three writes:
+//   warps 0..2  the CSA pooling of the block into cache row e (pool_m4, d / VEC threads);
+//   warp 3      the indexer key of the same block (pool_m4 of the indexer activations, then
+//               store_index_key; d_I / VEC threads), when CaI is given;
+//   warps 4..6  the token's raw latent into slot win_slot[b] of the window ring, when raw_new
+//               is given (the attention reads the window's rows in any order).
+// One CTA per sequence.
+template <typename T, int FMT>
+__global__ void __launch_bounds__(224)
+decode_append_kernel(const T* __restrict__ Ca, const T* __restrict__ Cb, const T* __restrict__ Za,
+                     const T* __restrict__ Zb, const float* __restrict__ Ba, const float* __restrict__ Bb,
+                     const T* __restrict__ pCb, const T* __restrict__ pZb, const int32_t* __restrict__ entry0,
+                     T* __restrict__ cache, int64_t n_max, int d,
+                     const T* __restrict__ CaI, const T* __restrict__ CbI, const T* __restrict__ ZaI,
+                     const T* __restrict__ ZbI, const float* __restrict__ BaI, const float* __restrict__ BbI,
+                     const T* __restrict__ pCbI, const T* __restrict__ pZbI, uint8_t* __restrict__ kI,
+                     void* __restrict__ kI_scale, int d_I,
+                     const T* __restrict__ raw_new, T* __restrict__ win, const int32_t* __restrict__ win_slot, int W,
+                     unsigned* err) {
+  constexpr int VEC = Elem<T>::VEC;
+  const int b = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp < 3) {
+    const int g = threadIdx.x;
+    if (g < d / VEC) {
+      float out[VEC];
+      const int e = pool_m4<T>(Ca, Cb, Za, Zb, Ba, Bb, pCb, pZb, entry0, n_max, 4, d, b, 0, g * VEC, out, err);
+      if (e >= 0) Elem<T>::st_vec(cache + ((size_t)b * n_max + e) * d + g * VEC, out);
+    }
+  } else if (warp == 3) {
+    const int tpe = d_I / VEC;
+    if (CaI && lane < tpe) {
+      const unsigned gmask = tpe == 32 ? 0xFFFFFFFFu : (1u << tpe) - 1u;
+      float x[VEC];
+      const int e = pool_m4<T>(CaI, CbI, ZaI, ZbI, BaI, BbI, pCbI, pZbI, entry0, n_max, 4, d_I, b, 0, lane * VEC, x, err);
+      if (e >= 0) store_index_key<VEC, FMT>(x, (size_t)b * n_max + e, d_I, lane, tpe, gmask, kI, kI_scale);
+    }
+  } else {
+    const int g = threadIdx.x - 128;
+    if (raw_new && g < d / VEC) {
+      const int slot = win_slot[b];
+      if (slot < 0 || slot >= W) {
+        if (g == 0) raise_err(err, CSA_DEVERR_WINDOW);
+      } else {
+        float v[VEC];
+        Elem<T>::ld_vec(raw_new + (size_t)b * d + g * VEC, v);
+        Elem<T>::st_vec(win + ((size_t)b * W + slot) * d + g * VEC, v);
+      }
+    }
+  }
+}
+
+// The raw latent of the current token into slot win_slot[b] of sequence b's window ring.
+template <typename T>
+__global__ void __launch_bounds__(96)
+window_append_kernel(const T* __restrict__ raw_new, T* __restrict__ win, const int32_t* __restrict__ win_slot, int W,
+                     int d, unsigned* err) {
+  constexpr int VEC = Elem<T>::VEC;
+  const int b = blockIdx.x;
+  for (int g = threadIdx.x; g < d / VEC; g += blockDim.x) {
+    const int slot = win_slot[b];
+    if (slot < 0 || slot >= W) {
+      if (g == 0) raise_err(err, CSA_DEVERR_WINDOW);
+      return;
+    }
+    float v[VEC];
+    Elem<T>::ld_vec(raw_new + (size_t)b * d + g * VEC, v);
+    Elem<T>::st_vec(win + ((size_t)b * W + slot) * d + g * VEC, v);
   }
 }
 
@@ -507,6 +591,42 @@ cudaError_t launch_index_key_compress(const void* Ca, const void* Cb, const void
   } else {
     if (ifmt == CSA_IFMT_E4M3) go(float(), E4()); else go(float(), MX());
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_append(const void* Ca, const void* Cb, const void* Za, const void* Zb, const float* Ba,
+                                 const float* Bb, const void* pCb, const void* pZb, const int32_t* entry0,
+                                 void* cache, int64_t n_max, int d, const void* CaI, const void* CbI,
+                                 const void* ZaI, const void* ZbI, const float* BaI, const float* BbI,
+                                 const void* pCbI, const void* pZbI, void* kI, void* kI_scale, int d_I, int ifmt,
+                                 const void* raw_new, void* win, const int32_t* win_slot, int W, int B, int dtype,
+                                 cudaStream_t st, unsigned* err) {
+  auto go = [&](auto tag, auto fmt) {
+    using T = decltype(tag);
+    note_launch();
+    decode_append_kernel<T, decltype(fmt)::value><<<B, 224, 0, st>>>(
+        (const T*)Ca, (const T*)Cb, (const T*)Za, (const T*)Zb, Ba, Bb, (const T*)pCb, (const T*)pZb, entry0,
+        (T*)cache, n_max, d, (const T*)CaI, (const T*)CbI, (const T*)ZaI, (const T*)ZbI, BaI, BbI, (const T*)pCbI,
+        (const T*)pZbI, (uint8_t*)kI, kI_scale, d_I, (const T*)raw_new, (T*)win, win_slot, W, err);
+  };
+  using E4 = std::integral_constant<int, CSA_IFMT_E4M3>;
+  using MX = std::integral_constant<int, CSA_IFMT_MXFP4>;
+  if (dtype == CSA_BF16) {
+    if (ifmt == CSA_IFMT_MXFP4) go(__nv_bfloat16(), MX()); else go(__nv_bfloat16(), E4());
+  } else {
+    if (ifmt == CSA_IFMT_MXFP4) go(float(), MX()); else go(float(), E4());
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_window_append(const void* raw_new, void* win, const int32_t* win_slot, int W, int B, int d,
+                                 int dtype, cudaStream_t st, unsigned* err) {
+  auto go = [&](auto tag) {
+    using T = decltype(tag);
+    note_launch();
+    window_append_kernel<T><<<B, 96, 0, st>>>((const T*)raw_new, (T*)win, win_slot, W, d, err);
+  };
+  if (dtype == CSA_BF16) go(__nv_bfloat16()); else go(float());
   return cudaGetLastError();
 }
 

@@ -21,7 +21,7 @@ import torch
 
 from . import _native as N
 
-_INT_META = ("entry0", "q_pos", "n_entries", "win_len", "raw_pos0", "h_entry0", "h_n_entries", "h_win_len")
+_INT_META = ("entry0", "q_pos", "n_entries", "win_len", "raw_pos0", "h_entry0", "h_n_entries", "h_win_len", "win_slot")
 
 
 def _to_device(name, arr, device):
@@ -53,10 +53,14 @@ def upload(wl, device="cuda"):
             T["raw_pos0"] = torch.full((B,), D["raw_pos0"], **i32)
         else:
             T["win_len"] = torch.full((B,), D["W"], **i32)
+            if "win_slot" in D:
+                T["win_slot"] = torch.full((B,), D["win_slot"], **i32)
             T["aws"] = torch.empty(max(1, N.attn_decode_workspace_size(B, D["H"], D["dv"], D["k"] + D["W"])),
                                    dtype=torch.uint8, device=device)
     if kind in ("hca_decode", "hybrid_pair"):
         p = "h_" if kind == "hybrid_pair" else ""
+        if "win_slot" in D and "win_slot" not in T:
+            T["win_slot"] = torch.full((B,), D["win_slot"], **i32)
         Nh = D["Nh"] if p else D["N"]
         T[p + "entry0"] = torch.full((B,), D["entry0_h"] if p else D["entry0"], **i32)
         T[p + "n_entries"] = torch.full((B,), Nh, **i32)
@@ -83,12 +87,31 @@ def _side_stream(device):
     return _SIDE[key]
 
 
+def _decode_append(T, D, stream):
+    """The decode token's appends in one launch: the block it completes pooled into the
+    cache, the indexer key of that block, and its raw latent into the window ring (the key
+    is read by the indexer, so this runs before it)."""
+    keys = (T["CaI"], T["CbI"], T["ZaI"], T["ZbI"], T["BaI"], T["BbI"], T["prev_CbI"], T["prev_ZbI"], T["kI"],
+            T["kI_scale"], _ifmt(D))
+    N.csa_decode_append(T["Ca"], T["Cb"], T["Za"], T["Zb"], T["Ba"], T["Bb"], T["prev_Cb"], T["prev_Zb"],
+                        T["entry0"], T["cache"], keys=keys, window=(T["raw_new"], T["win"], T["win_slot"]),
+                        stream=stream)
+
+
 def _csa_layer(T, D, stream, attend):
-    """One CSA layer: the compressor's cache append and the lightning indexer are
-    independent (the indexer scores the given indexer keys; the new cache entry is
-    read only by the attention), so the append runs on a side stream while the indexer
-    runs on the main one; the attention waits for both."""
+    """One CSA layer.  A decode token with its indexer activations and raw latent: one
+    launch appends the cache entry, its key and the window row, then the indexer and the
+    attention.  Otherwise the compressor's cache append and the lightning indexer are
+    independent (the indexer scores the given indexer keys; the new cache entry is read
+    only by the attention), so the append runs on a side stream while the indexer runs on
+    the main one; the attention waits for both."""
     main = stream if stream is not None else torch.cuda.current_stream()
+    if "CaI" in T:
+        _decode_append(T, D, main)
+        N.lightning_index(T["qI"], T.get("qI_scale"), T["w"], T["kI"], T.get("kI_scale"), T["n_entries"],
+                          T["q_pos"], D["k"], _ifmt(D), T["idx"], T["iws"], m=D["m"], stream=main)
+        attend(main)
+        return
     side = _side_stream(main.device)
     fork = torch.cuda.Event()
     fork.record(main)
@@ -111,8 +134,11 @@ def csa_decode_step(T, D, stream=None):
 
 def hca_decode_step(T, D, stream=None, prefix=""):
     """The fresh chunk's compression and the dense attention as one call (the attention
-    streams the other entries while the compression runs)."""
+    streams the other entries while the compression runs); the token's raw latent, when
+    given, goes into the window ring first."""
     p = prefix
+    if p + "raw_new" in T:
+        N.window_append(T[p + "raw_new"], T[p + "win"], T["win_slot"], stream=stream)
     N.hca_compress_attn_decode(T[p + "C"], T[p + "Z"], T[p + "bias"], T[p + "entry0"], T[p + "q"][:, 0],
                                T[p + "cache"], T[p + "n_entries"], T[p + "win"], T[p + "win_len"], T[p + "sink"],
                                D["sm_scale"], D["dv"], T[p + "out"][:, 0], T[p + "lse"][:, 0], T[p + "aws"],

@@ -175,6 +175,21 @@ def _csa_compressor_inputs(r: _Rng, B, T_new, d, m, gate_std, to_store):
     return t
 
 
+def _decode_fresh_inputs(r: _Rng, t: dict, dims: dict, B: int, dI: int, d: int, m: int, W: int, ifmt: str):
+    """What a decode token brings besides its query (drawn after every other tensor, so the
+    rest of the workload is unchanged): the indexer activations of the block it completes
+    (CaI .. prev_ZbI ~ N(0, 1), gates ~ N(0, 2), biases BaI, BbI ~ N(0, 0.1)), from which
+    the key of the fresh entry is produced in the step, and its raw latent raw_new ~ N(0, 1),
+    which the step writes into the window ring at slot q_pos0 mod W.  The workload's kI row
+    of the fresh entry and win row of that slot are stale inputs the step overwrites."""
+    ki = _csa_compressor_inputs(r, B, m, dI, m, 2.0, bf16_bits)
+    for k, v in ki.items():
+        t[k + "I"] = v
+    t["raw_new"] = bf16_bits(r.normal((B, d)))
+    dims["win_slot"] = dims["q_pos0"] % W
+    dims["key_fmt"] = ifmt
+
+
 def index_key_inputs(seed: int, B: int, T_new: int, d_I: int = 128, dtype: str = "bf16",
                      gate_std: float = 2.0, spread: float = 0.0) -> dict:
     """Indexer activations and gates for the indexer-key producer (the CSA pooling with
@@ -247,6 +262,7 @@ def make_workload(i: int, seed: int | None = None, scale: dict | None = None) ->
         t["kI"], t["kI_scale"] = quant_e4m3_rows(r.normal((B, N, dI)))
         t["w"] = fp32(r.uniform((B, 1, HI)))
         t["sink"] = fp32(r.normal((H,)))
+        _decode_fresh_inputs(r, t, dims, B, dI, d, m, W, "e4m3")
         return Workload(WORKLOADS[1], "csa_decode", dims, t)
 
     if i == 2:
@@ -263,6 +279,8 @@ def make_workload(i: int, seed: int | None = None, scale: dict | None = None) ->
         t["q"] = bf16_bits(r.normal((B, 1, H, d)))
         t["win"] = bf16_bits(r.normal((B, W, d)))
         t["sink"] = fp32(r.normal((H,)))
+        t["raw_new"] = bf16_bits(r.normal((B, d)))
+        dims["win_slot"] = (T - 1) % W
         return Workload(WORKLOADS[2], "hca_decode", dims, t)
 
     if i == 3:
@@ -308,6 +326,8 @@ def make_workload(i: int, seed: int | None = None, scale: dict | None = None) ->
         t["h_q"] = bf16_bits(r.normal((B, 1, H, d)))
         t["h_win"] = bf16_bits(r.normal((B, W, d)))
         t["h_sink"] = fp32(r.normal((H,)))
+        _decode_fresh_inputs(r, t, dims, B, dI, d, m, W, "mxfp4")
+        t["h_raw_new"] = bf16_bits(r.normal((B, d)))
         return Workload(WORKLOADS[4], "hybrid_pair", dims, t)
 
     raise ValueError(f"unknown workload {i}")

@@ -134,6 +134,37 @@ csa_status csa_compress_kv8(const void* Ca, const void* Cb, const void* Za, cons
                             int B, int T_new, int d, int m, int dtype, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * csa_decode_append — the cache and window appends of one decode step, in one launch.
+ * The current token completes block entry0[b] (m = 4) of sequence b; the call writes
+ *   - cache row entry0[b]: csa_compress of that block (Ca, Cb, Za, Zb [B, 4, d], the
+ *     previous block's b-series prev_Cb, prev_Zb [B, 4, d], biases Ba, Bb [4, d]);
+ *   - when CaI != NULL, indexer key row entry0[b] of kI / kI_scale: index_key_compress of
+ *     the block's indexer activations (CaI .. prev_ZbI [B, 4, d_I], BaI, BbI [4, d_I]) in
+ *     format ifmt ("FP4 с учётом квантования": the keys of compressed entries are cached);
+ *   - when raw_new != NULL, window row win_slot[b] of win [B, W, d]: the token's raw latent
+ *     raw_new [B, d] ("Гибридное внимание: CSA и HCA": the sliding window of uncompressed
+ *     entries).  The window is a ring: the token at position p goes to slot p mod W, and
+ *     the attention calls read its rows in any order.  A slot outside [0, W) is skipped
+ *     and sets CSA_DEVERR_WINDOW.
+ * Each part is the same arithmetic as its own call (csa_compress with T_new = 4,
+ * index_key_compress, a row copy).
+ * Supported: d / (8 for bf16, 4 for f32) <= 96; d_I as index_key_compress.
+ * ------------------------------------------------------------------------- */
+csa_status csa_decode_append(const void* Ca, const void* Cb, const void* Za, const void* Zb,
+                             const float* Ba, const float* Bb, const void* prev_Cb, const void* prev_Zb,
+                             const int32_t* entry0, void* cache, int64_t n_max, int d,
+                             const void* CaI, const void* CbI, const void* ZaI, const void* ZbI,
+                             const float* BaI, const float* BbI, const void* prev_CbI, const void* prev_ZbI,
+                             void* kI, void* kI_scale, int d_I, int ifmt,
+                             const void* raw_new, void* win, const int32_t* win_slot, int W,
+                             int B, int dtype, void* stream);
+
+/* window_append — the window part of csa_decode_append alone (for the HCA window):
+ * win[b, win_slot[b], :] = raw_new[b, :], raw_new [B, d], win [B, W, d].              */
+csa_status window_append(const void* raw_new, void* win, const int32_t* win_slot, int B, int W, int d,
+                         int dtype, void* stream);
+
+/* ---------------------------------------------------------------------------
  * hca_compress — HCA compression ("HCA: сжать в 128 раз, но смотреть на всё":
  * the same gated pooling with m' tokens per entry and no overlap).
  *

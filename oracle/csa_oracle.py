@@ -526,6 +526,17 @@ def run_csa_prefill(wl, rows=None):
     return res
 
 
+def _window(t, D, b, p, dt):
+    """The raw window rows of sequence b.  A decode token's own raw latent (raw_new, when the
+    workload gives it) goes into its ring slot win_slot = position mod W; the window is a set
+    of rows, so their order does not matter."""
+    win = load(t[p + "win"][b], dt)
+    if p + "raw_new" in t:
+        win = win.copy()
+        win[D["win_slot"]] = load(t[p + "raw_new"][b], dt)
+    return win
+
+
 def run_csa_decode(wl, batches=None, prefix=""):
     """CSA decode step (workload 1, CSA half of 4): compress the block completed
     by the current token into entry N-1, index, select top-k, attend."""
@@ -542,7 +553,17 @@ def run_csa_decode(wl, batches=None, prefix=""):
                            load(t["prev_Cb"][b], dt), load(t["prev_Zb"][b], dt), e0, m)
         entry = store(new, dt)
         ifmt = D["ifmt"]
-        I = indexer_scores(t["qI"][b], t["w"][b], t["kI"][b], ifmt, t["qI_scale"][b], t["kI_scale"][b])[0]
+        kI_b, kIs_b = t["kI"][b], t["kI_scale"][b]
+        if "CaI" in t:
+            # the key of the fresh entry comes from the block's indexer activations
+            codes, scales, _, _ = index_key_compress(
+                load(t["CaI"][b], dt), load(t["CbI"][b], dt), load(t["ZaI"][b], dt), load(t["ZbI"][b], dt),
+                load(t["BaI"], "f32"), load(t["BbI"], "f32"), ifmt, load(t["prev_CbI"][b], dt),
+                load(t["prev_ZbI"][b], dt), e0, m)
+            kI_b, kIs_b = kI_b.copy(), kIs_b.copy()
+            kI_b[e0:e0 + codes.shape[0]] = codes
+            kIs_b[e0:e0 + codes.shape[0]] = scales
+        I = indexer_scores(t["qI"][b], t["w"][b], kI_b, ifmt, t["qI_scale"][b], kIs_b)[0]
         sel = topk(I, n_eligible(pos, m, N), k)
         cache_b = t["cache"][b]
         rows_sel = load(cache_b[np.clip(sel[sel >= 0], 0, N - 1)], dt)
@@ -550,7 +571,7 @@ def run_csa_decode(wl, batches=None, prefix=""):
         for r_i, s in enumerate(sel[sel >= 0]):
             if e0 <= s < e0 + entry.shape[0]:
                 rows_sel[r_i] = entry[s - e0]
-        kv = np.concatenate([rows_sel, load(t["win"][b], dt)], axis=0)
+        kv = np.concatenate([rows_sel, _window(t, D, b, "", dt)], axis=0)
         o, lse = attention(load(t["q"][b][0], dt), kv, load(t["sink"], "f32"), D["sm_scale"], D["dv"])
         res["entry"][b] = entry
         res["idx"][b] = sel
@@ -577,7 +598,7 @@ def run_hca_decode(wl, batches=None, prefix=""):
         entry = store(new, dt)
         cache = load(t[p + "cache"][b], dt).copy()
         cache[e0:e0 + entry.shape[0]] = entry
-        kv = np.concatenate([cache[:N], load(t[p + "win"][b], dt)], axis=0)
+        kv = np.concatenate([cache[:N], _window(t, D, b, p, dt)], axis=0)
         o, lse = attention(load(t[p + "q"][b][0], dt), kv, load(t[p + "sink"], "f32"), D["sm_scale"], D["dv"])
         res["entry"][b] = entry
         res["out"][b] = o

@@ -262,3 +262,77 @@ def test_hca_decode_equals_csa_decode_with_every_entry():
     o, lse = O.attention(t["q"][0, 0], np.concatenate([cache[sel], t["win"][0]]), t["sink"], 1 / np.sqrt(8), 8)
     np.testing.assert_allclose(res["out"][0], o, rtol=0, atol=1e-13)
     np.testing.assert_allclose(res["lse"][0], lse, rtol=0, atol=1e-13)
+
+
+# -------------------------------------------------------------- fresh key and window ring
+
+def test_decode_fresh_key_and_ring_row_equal_a_prefill_row():
+    """A decode token brings its block's indexer activations and its raw latent: the pass
+    must produce the entry's key from the activations (the pinned index_key_compress) and
+    put the raw latent at ring slot position mod W.  The same sequence as a prefill (E4M3
+    indexer, the keys given as inputs, including the one the activations produce) must give
+    the same selection, output and lse for that token; the window ring holds positions
+    p - W + 1 .. p at slots pos mod W (in ring order, not position order)."""
+    W, k, m = 8, 3, 4
+    r = np.random.default_rng(31)
+    x = _tokens(48, 8, seed=31, **SIZES)
+    d, HI, dI = 8, 2, 32
+    # an E4M3 indexer: queries and keys quantised with per-row scales
+    qf = r.standard_normal((48, HI, dI))
+    x["qI8"], x["qIs"] = O.quantise_index_keys(qf.reshape(48 * HI, dI), "e4m3")[:2]
+    x["qI8"] = x["qI8"].reshape(48, HI, dI)
+    x["qIs"] = x["qIs"].reshape(48, HI)
+    kf = r.standard_normal((12, dI))
+    kI8, kIs = O.quantise_index_keys(kf, "e4m3")[:2]
+    act = {n: r.standard_normal((4, dI)) * (2.0 if n.startswith("Z") else 1.0) for n in ("Ca", "Cb", "Za", "Zb")}
+    act.update(prev_Cb=r.standard_normal((4, dI)), prev_Zb=2 * r.standard_normal((4, dI)),
+               Ba=0.1 * r.standard_normal((4, dI)), Bb=0.1 * r.standard_normal((4, dI)))
+    # the key of entry 11 as the activations give it
+    fresh8, fresh_s = O.index_key_compress(act["Ca"], act["Cb"], act["Za"], act["Zb"], act["Ba"], act["Bb"], "e4m3",
+                                           act["prev_Cb"], act["prev_Zb"], 11, m)[:2]
+    kI_full, kIs_full = kI8.copy(), kIs.copy()
+    kI_full[11], kIs_full[11] = fresh8[0], fresh_s[0]
+    # the prefill of all 48 tokens with the full key set
+    pre = _prefill_wl(x, 0, 48, None, W, k, H=2, HI=HI, dI=dI)
+    pre.dims["ifmt"] = "e4m3"
+    pre.tensors.update(qI=x["qI8"][None], qI_scale=x["qIs"][None], kI=kI_full[None], kI_scale=kIs_full[None])
+    full = O.run_csa_prefill(pre)
+    # the decode of token 47: stale key row 11 and stale ring slot 47 mod 8 = 7
+    ctx = O.run_csa_prefill(_prefill_wl(x, 0, 44, None, W, k, **SIZES))["cache"]
+    dec = _decode_wl(x, 47, ctx, W, k, H=2, HI=HI, dI=dI)
+    dec.dims.update(ifmt="e4m3", win_slot=47 % W)
+    ring = np.full((1, W, d), 5.0)
+    for pos in range(40, 47):
+        ring[0, pos % W] = x["raw"][pos]
+    stale_k = kI8.copy()
+    stale_k[11] = 0x38                                        # 1.0 everywhere: not the produced key
+    dec.tensors.update(qI=x["qI8"][None, 47:48], qI_scale=x["qIs"][None, 47:48], kI=stale_k[None],
+                       kI_scale=kIs[None], win=ring, raw_new=x["raw"][None, 47],
+                       **{n + "I": v[None] for n, v in act.items() if n not in ("Ba", "Bb")},
+                       BaI=act["Ba"], BbI=act["Bb"])
+    res = O.run_csa_decode(dec)
+    assert np.array_equal(res["idx"][0], full["idx"][47])
+    np.testing.assert_allclose(res["out"][0], full["out"][47], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(res["lse"][0], full["lse"][47], rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(res["scores"][0], full["scores"][47][:12])
+
+
+def test_hca_decode_ring_row():
+    """The HCA pass puts raw_new at ring slot win_slot: equal to the window with that row in place."""
+    wl = _hca_wl(4, 4, 6, stale=1.5, seed=8)
+    t = wl.tensors
+    ref = O.run_hca_decode(wl)
+    r = np.random.default_rng(9)
+    new = r.standard_normal((1, 8)).astype(np.float32)
+    wl2 = _hca_wl(4, 4, 6, stale=1.5, seed=8)
+    wl2.tensors["win"] = t["win"].copy()
+    wl2.tensors["win"][0, 3] = 99.0                           # stale
+    wl2.tensors["raw_new"] = new
+    wl2.dims["win_slot"] = 3
+    res = O.run_hca_decode(wl2)
+    wl3 = _hca_wl(4, 4, 6, stale=1.5, seed=8)
+    wl3.tensors["win"] = t["win"].copy()
+    wl3.tensors["win"][0, 3] = new[0]
+    exp = O.run_hca_decode(wl3)
+    np.testing.assert_array_equal(res["out"][0], exp["out"][0])
+    assert np.abs(res["out"][0] - ref["out"][0]).max() > 0       # the row mattered
