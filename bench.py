@@ -227,6 +227,15 @@ def main():
             run_ours(args, WORKLOADS[name], name)
 
 
+def check_device(csa, name, where):
+    """Raise if a kernel flagged an error (the library's device error word) since the last check."""
+    import torch
+    torch.cuda.synchronize()
+    e = csa.read_device_error()
+    if e:
+        raise RuntimeError(f"{name}: device error word 0x{e:x} after the {where}")
+
+
 def run_ours(args, wid, name):
     import numpy as np
     import torch
@@ -316,7 +325,7 @@ def run_ours(args, wid, name):
         f(T)
     launches_step = csa.launch_count() - n0
     torch.cuda.synchronize()
-    assert csa.read_device_error() == 0
+    check_device(csa, name, "eager warm-up")
     # the whole step as one CUDA graph per copy (the timed quantity), and one graph per ABI
     # call and copy (timed separately, for the per-call breakdown)
     active = {1: [1, 1, 1, 0], 2: [1, 0, 1, 0], 3: [1, 1, 1, 0], 4: [1, 1, 1, 1]}[wid]   # calls a step makes
@@ -352,7 +361,7 @@ def run_ours(args, wid, name):
             g_steps[c].replay()
         step_parts(mk(), w % n_copies)
     torch.cuda.synchronize()
-    assert csa.read_device_error() == 0
+    check_device(csa, name, "graph warm-up")
 
     clock_lines, stop = [], threading.Event()
     th = threading.Thread(target=sample_clocks, args=(stop, clock_lines), daemon=True)
@@ -384,7 +393,9 @@ def run_ours(args, wid, name):
     value = job_rate(tokens_per_step, world, ms_per_step)
 
     # ---- e2e through the public API with host buffers (max over ranks too)
+    check_device(csa, name, "timed steps")
     e2e_ms, h2d, d2h, h2d_gbs = measure_e2e(args, wid, wl, Ts, D, csa, steps)
+    check_device(csa, name, "e2e")
     e2e_ms = max_over_ranks(e2e_ms, world, "cuda")
     e2e = {"value": job_rate(tokens_per_step, world, e2e_ms), "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -429,6 +440,7 @@ def run_ours(args, wid, name):
                                    src)
         if kv:
             extra.update(kv)
+        check_device(csa, name, "rows beyond the step")
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -688,7 +700,7 @@ def measure_e2e(args, wid, wl, Ts, D, csa, steps):
     host_in = torch.empty(n_in, dtype=torch.uint8).pin_memory()
     for k, v in views(host_in, lay_in).items():
         v.copy_(T[k].cpu())
-    dev_in = [torch.empty(n_in, dtype=torch.uint8, device="cuda") for _ in range(2)]
+    dev_in = [host_in.to("cuda") for _ in range(2)]       # valid inputs for the warm-up and capture runs
     dev_out = [torch.empty(n_out, dtype=torch.uint8, device="cuda") for _ in range(2)]
     host_out = [torch.empty(n_out, dtype=torch.uint8).pin_memory() for _ in range(2)]
     io = [dict(views(dev_in[j], lay_in), **views(dev_out[j], lay_out)) for j in range(2)]

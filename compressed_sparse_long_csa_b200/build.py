@@ -11,7 +11,7 @@ CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libcsa_b200.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
-SOURCES = ["api.cu", "compress.cu", "indexer.cu", "indexer_tc.cu", "topk.cu", "select.cu", "select_hist.cu", "attention.cu", "attention_tc.cu", "noalloc.cu", "out_proj.cu", "shard.cu", "diag.cu"]
+SOURCES = ["api.cu", "compress.cu", "indexer.cu", "indexer_tc.cu", "topk.cu", "select.cu", "select_hist.cu", "select_row.cu", "attention.cu", "attention_tc.cu", "noalloc.cu", "out_proj.cu", "shard.cu", "diag.cu"]
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
          "-Xcompiler", "-fPIC", "-Xptxas", "-v"]
 

@@ -321,9 +321,13 @@ static csa_status run_lightning_index(const void* qI, const void* qI_scale, cons
   a.keyrange = (unsigned*)(ws + L.keyrange);
   a.idx_out = idx_out; a.score_out = score_out; a.err = err;
   a.score_bf16 = bf16_scores ? 1 : 0;
-  // the histogram-seeded selection: decode rows of the exact call (the bf16-key call
-  // selects on the stored keys with the plain top-k)
-  const bool hist_path = Tq <= kHistMaxTq && !bf16_scores;
+  // decode rows of the exact call (the bf16-key call selects on the stored keys with the
+  // plain top-k): rows that fit one CTA's shared memory take the one-CTA-per-row selection
+  // over the staged scores (no histograms); longer rows the histogram-seeded one
+  const bool decode_rows = Tq <= kHistMaxTq && !bf16_scores;
+  const bool row_path = decode_rows && (ifmt == CSA_IFMT_E4M3 || ifmt == CSA_IFMT_MXFP4) &&
+                        n_max <= indexer_select_row_max_entries();
+  const bool hist_path = decode_rows && !row_path;
   if (hist_path) {
     a.hist = (unsigned*)(ws + L.hist);
     a.fhist = (unsigned*)(ws + L.fhist);
@@ -331,7 +335,8 @@ static csa_status run_lightning_index(const void* qI, const void* qI_scale, cons
     a.bitmap = (unsigned*)(ws + L.bitmap);
     a.cand = ws + L.cand;
   }
-  cudaError_t e = cudaMemsetAsync(ws + L.knmax, 0, L.zero_end - L.knmax, S(stream));
+  // zeroed per call: knmax and the key ranges, and the histograms and counters when used
+  cudaError_t e = cudaMemsetAsync(ws + L.knmax, 0, (hist_path ? L.zero_end : L.hist) - L.knmax, S(stream));
   if (e != cudaSuccess) return CSA_ERR_CUDA;
   bool used_tc = false;
   if (tc_enabled()) {
@@ -350,6 +355,10 @@ static csa_status run_lightning_index(const void* qI, const void* qI_scale, cons
     RowCount rc;
     rc.q_pos = q_pos; rc.n_entries = n_entries; rc.m = m; rc.Tq = Tq;
     return cuda_status(launch_topk_select(a.scores, a.ld, rc, B * Tq, n_max, k, idx_out, S(stream), err));
+  }
+  if (row_path && used_tc) {
+    const cudaError_t er = launch_indexer_select_row(a, S(stream));
+    if (er != cudaErrorNotSupported) return cuda_status(er);
   }
   return cuda_status(launch_indexer_select(a, S(stream)));
 }
@@ -507,6 +516,7 @@ static csa_status sparse_decode(const void* q, const void* cache, const int32_t*
   a.q = q; a.cache = cache; a.idx = idx; a.k = k; a.n_seg_a = k; a.win = win; a.win_len = win_len;
   a.W = W; a.prefill = 0; a.sink = sink; a.B = B; a.Tq = 1; a.H = H; a.dk = d_k; a.dv = d_v; a.n_max = n_max;
   a.sm_scale = sm_scale; a.out = out; a.lse = lse; a.err = err; a.kv8 = kv8;
+  a.idx_late = 1;
   return run_attention(a, dtype, workspace, ws_bytes, true, S(stream));
 }
 

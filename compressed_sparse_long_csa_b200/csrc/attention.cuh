@@ -35,6 +35,9 @@ struct AttnArgs {
   const int32_t* dep_entry0;  // dense decode after a compression kernel in the same stream: it
   int dep_rows;               // writes rows dep_entry0[b] .. +dep_rows-1 (null: wait for it at once)
   int kv8;                    // cache rows are 656-byte FP8 rows (tensor-core kernel only)
+  int idx_late;               // sparse decode: only idx may come from the preceding kernel; each
+                              // split takes its tiles last to first (the window's first) and waits
+                              // for that kernel just before it resolves an index (tensor-core kernel)
   unsigned* err;
 };
 

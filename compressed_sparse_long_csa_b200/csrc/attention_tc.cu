@@ -201,7 +201,10 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
   // except after a compression kernel that writes known rows (dep_entry0): then only the
   // loader of a tile holding them waits, just before loading it.
   const bool dep_rows_only = a.dep_entry0 != nullptr;
-  if (!dep_rows_only) tc::griddep_wait();
+  const bool idx_late = a.idx_late != 0 && !dep_rows_only;
+  if (!dep_rows_only && !idx_late) tc::griddep_wait();
+  // the tile of a split's it-th step
+  auto tile_of = [&](int it) { return split + (idx_late ? n_t - 1 - it : it) * a.splits; };
   tc::griddep_launch_dependents();
   const uint32_t tmem = sm.tmem_base;
   // The sink logit, needed only at the end, is loaded now: with one split by every softmax
@@ -228,11 +231,16 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
     }
     // row coordinates of the next tile, resolved into registers before its stage is free
     int which = -1, y = 0;
+    bool idx_ready = !idx_late;
     auto coord = [&](int t) {
       which = -1;
       y = 0;
       if (lg < AT_ROWS) {
-        const int64_t v = (int64_t)(split + t * a.splits) * AT_ROWS + lg;
+        const int64_t v = (int64_t)tile_of(t) * AT_ROWS + lg;
+        if (!idx_ready && v < a.n_seg_a) {
+          tc::griddep_wait();                         // the indices come from the preceding kernel
+          idx_ready = true;
+        }
         if (v < nrows) which = attn_row_coord(a, row, (int)v, &y);
       }
     };
@@ -269,7 +277,7 @@ attn_tc_kernel(const __grid_constant__ AtMaps maps, AttnArgs a) {
       const int stop = *(volatile int*)&sm.ld_stop[g];
       if (stop != 0 && stop <= i + 1) break;
       if (!dep_done) {
-        const int64_t r0 = (int64_t)(split + it * a.splits) * AT_ROWS;   // the tile's cache rows
+        const int64_t r0 = (int64_t)tile_of(it) * AT_ROWS;   // the tile's cache rows
         if (r0 < dep1 && r0 + AT_ROWS > dep0) {
           tc::griddep_wait();                         // every thread of the group loads
           dep_done = true;

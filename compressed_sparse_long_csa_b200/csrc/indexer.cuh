@@ -114,6 +114,10 @@ cudaError_t launch_indexer_select_cluster(const IndexerArgs& a, cudaStream_t st)
 // Histogram-seeded selection of decode rows (select_hist.cu); cudaErrorNotSupported when
 // the scoring path wrote no histogram.
 cudaError_t launch_indexer_select_hist(const IndexerArgs& a, cudaStream_t st);
+// One-CTA-per-row selection of decode rows over the staged fp32 scores (select_row.cu);
+// cudaErrorNotSupported for other shapes.
+cudaError_t launch_indexer_select_row(const IndexerArgs& a, cudaStream_t st);
+int64_t indexer_select_row_max_entries();
 cudaError_t launch_topk_select_cluster(const float* scores, int64_t ld, RowCount rc, int R, int64_t n,
                                        int k, int32_t* idx_out, cudaStream_t st);
 

@@ -361,7 +361,11 @@ size_t attn_decode_workspace_size(int B, int H, int d_v, int64_t rows_max);
  *   win     device [B, W, d_k]: raw latents of the last win_len[b] positions
  *   win_len device [B] int32 (0..W)
  *   sink    device [H] fp32
- *   out     device [B, H, d_v];  lse device [B, H] fp32 or NULL                */
+ *   out     device [B, H, d_v];  lse device [B, H] fp32 or NULL
+ * Ordering: when the preceding kernel in the stream allows programmatic dependent
+ * launch (lightning_index's selection does), this call overlaps it and waits for it
+ * only before it reads idx: q, cache, win, win_len and sink must not be written by that
+ * kernel (they may be written by any earlier one).                                   */
 csa_status sparse_attn_decode(const void* q, const void* cache, const int32_t* idx,
                               const void* win, const int32_t* win_len, const float* sink,
                               int B, int H, int d_k, int d_v, int64_t n_max, int k, int W,

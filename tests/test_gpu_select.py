@@ -3,7 +3,9 @@
 tests do not reach: rows of different eligible counts, just above and at k; every key
 identical (all scores tie: the lowest indices win); scores packed into one narrow range
 (more candidates than the selection stages on chip); the exact scores returned with the
-selection.  Expected values come from the oracle only.
+selection; rows at the largest size one CTA stages in shared memory (24 576 entries, three
+bulk copies) and just above it (the multi-CTA selection).  Expected values come from the
+oracle only.
 """
 from __future__ import annotations
 
@@ -113,3 +115,17 @@ def test_score_out_is_the_exact_score_of_each_selected_entry(fmt):
         sel = idx[b][idx[b] >= 0]
         assert np.array_equal(so[b][:sel.size], I[sel].astype(np.float32))
         assert np.all(so[b][sel.size:] == 0)
+
+
+@pytest.mark.parametrize("N", [24576, 24577])
+def test_rows_at_and_above_the_staged_size(N):
+    g = torch.Generator().manual_seed(45)
+    B, k = 2, 1024
+    qI, qs = _keys("e4m3", torch.randn(B, 1, 64, 128, generator=g))
+    kI, ks = _keys("e4m3", torch.randn(B, N, 128, generator=g))
+    w = torch.rand(B, 1, 64, generator=g).numpy()
+    n_entries = np.array([N, N - 1000])
+    idx, _, err = _run(qI, qs, w, kI, ks, n_entries, 4 * n_entries - 1, k, "e4m3")
+    assert err == 0
+    for b in range(B):
+        _check_exact(idx[b], _oracle(qI, qs, w, kI, ks, b, n_entries[b], "e4m3"), n_entries[b], k)
