@@ -47,7 +47,7 @@ constexpr int SH_FINE = 16;              // fine bins (key >> 16) per coarse bin
 constexpr int SH_BLOC = 64;              // band entries one CTA re-scores
 constexpr int SH_BCAP = 4096;            // band entries the last CTA ranks in shared memory
 constexpr int SH_RB = 16;                // entries re-scored per batch
-constexpr int SH_KLD = 136;              // staged key row: 4 segments of 32 dims, 34 doubles apart
+constexpr int SH_KLD = 144;              // staged key row: 4 segments of 32 dims, 36 words apart
 constexpr int SH_BMW = 8192;             // bitmap words handled per output pass (262 144 entries)
 constexpr int SH_BINS2 = 2048;           // fallback refinement bins
 constexpr int SH_CTR0 = 4;               // row counters: [1] certain, [2] CTAs done, [3] overflow, [4 + p] band of CTA p
@@ -62,7 +62,8 @@ struct BandEnt {
 static_assert(sizeof(BandEnt) == 16, "band entries are 16-byte records");
 
 struct ShSmem {
-  double krow[SH_RB][SH_KLD];            // key rows of one re-scoring batch as fp64
+  alignas(16) int32_t krow[SH_RB][SH_KLD];   // key rows of one re-scoring batch as integers (E4M3: value * 2^9,
+                                            // FP4: value * 2), 32-dim segments 36 words apart
   double contrib[SH_RB][65];             // their per-head terms
   double rs_out[SH_RB];                  // their exact scores
   float ksc[SH_RB][4];                   // their scales (E4M3 row scale in [0], MXFP4 block scales)
@@ -137,15 +138,16 @@ struct KeySide {
 };
 
 // Exact fp64 scores of the entries sm.rid[0..cnt) (cnt <= SH_RB) of sequence b into
-// sm.rs_out, by the whole CTA (all threads call; barriers inside).  Thread t holds, in qr,
-// the query values of head j = t / 4 over dims [32 q, 32 q + 32), q = t % 4 (one MXFP4
-// scale block).  Its partial dot product with a key row is exact (FP8 / FP4 products are
-// exact in fp64 and every partial sum spans fewer than 53 bits, in any order); the four
-// partials of a head are combined as the definition does (E4M3: their exact sum times
-// sq * sk; MXFP4: the block terms (qs * ks) * P_b added in block order), each head's term
-// w_j * max(D_j, 0) is formed, and one thread per entry adds the terms in order.
+// sm.rs_out, by the whole CTA (all threads call; barriers inside).  Thread t holds, in qi,
+// the query codes of head j = t / 4 over dims [32 q, 32 q + 32), q = t % 4 (one MXFP4
+// scale block), as integers (E4M3: value * 2^9; FP4: value * 2).  Its partial dot product
+// with a key row is then an exact integer (E4M3: below 2^43 in 64 bits; FP4: below 2^13);
+// the four partials of a head are combined as the definition does (E4M3: their exact sum
+// * 2^-18 times sq * sk; MXFP4: the block terms (qs * ks) * P_b, P_b = partial * 2^-2,
+// added in block order), each head's term w_j * max(D_j, 0) is formed, and one thread per
+// entry adds the terms in order.
 template <int F>
-__device__ __forceinline__ void sh_rescore(const KeySide ks, ShSmem& sm, const double (&qr)[32], int b, int cnt) {
+__device__ __forceinline__ void sh_rescore(const KeySide ks, ShSmem& sm, const int (&qi)[32], int b, int cnt) {
   const int tid = threadIdx.x;
   const int j = tid >> 2, q = tid & 3;
   const int dI = ks.dI, nb = dI / 32, HI = ks.HI;
@@ -154,23 +156,17 @@ __device__ __forceinline__ void sh_rescore(const KeySide ks, ShSmem& sm, const d
     const int e = tid >> 3, seg = tid & 7;
     if (e < cnt && 16 * seg < dI) {
       const size_t koff = (size_t)b * ks.n_max + sm.rid[e];
-      double* kr = sm.krow[e];
+      int* kr = sm.krow[e] + 36 * (seg >> 1) + 16 * (seg & 1);
       if (F == CSA_IFMT_E4M3) {
         const uint4 v = *reinterpret_cast<const uint4*>((const uint8_t*)ks.kI + koff * dI + 16 * seg);
         const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int c = 16 * seg + i;
-          kr[34 * (c >> 5) + (c & 31)] = (double)e4m3_to_float((wd[i >> 2] >> (8 * (i & 3))) & 0xFFu);
-        }
+        for (int i = 0; i < 16; ++i) kr[i] = (int)(e4m3_to_float((wd[i >> 2] >> (8 * (i & 3))) & 0xFFu) * 512.f);
       } else {
         const uint2 v = *reinterpret_cast<const uint2*>((const uint8_t*)ks.kI + koff * (dI / 2) + 8 * seg);
         const uint32_t wd[2] = {v.x, v.y};
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int c = 16 * seg + i;
-          kr[34 * (c >> 5) + (c & 31)] = (double)e2m1_to_float((wd[i >> 3] >> (4 * (i & 7))) & 0xFu);
-        }
+        for (int i = 0; i < 16; ++i) kr[i] = (int)(e2m1_to_float((wd[i >> 3] >> (4 * (i & 7))) & 0xFu) * 2.f);
       }
     }
   } else if (tid < SH_RB * 8 + SH_RB * 4) {
@@ -184,34 +180,41 @@ __device__ __forceinline__ void sh_rescore(const KeySide ks, ShSmem& sm, const d
     sm.ksc[e2][q2] = v;
   }
   __syncthreads();
-  // ---- per-head terms, two entries at a time (key values read two doubles at a time)
+  // ---- per-head terms, two entries at a time
   const bool live = j < HI && 32 * q < dI;
   const double wj = (j < HI) ? (double)sm.w[j] : 0.0;
   for (int e0 = 0; e0 < cnt; e0 += 2) {
-    double acc[2][4];
+    long long acc[2] = {0, 0};
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      const double2* kr = reinterpret_cast<const double2*>(sm.krow[min(e0 + u, cnt - 1)] + 34 * q);
+      const int4* kr = reinterpret_cast<const int4*>(sm.krow[min(e0 + u, cnt - 1)] + 36 * q);
+      if (live) {
+        long long x = 0;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) acc[u][c] = 0.0;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const double2 kv = kr[i];
-        acc[u][(2 * i) & 3] = fma(qr[2 * i], kv.x, acc[u][(2 * i) & 3]);
-        acc[u][(2 * i + 1) & 3] = fma(qr[2 * i + 1], kv.y, acc[u][(2 * i + 1) & 3]);
+        for (int i = 0; i < 8; ++i) {
+          const int4 kv = kr[i];
+          if (F == CSA_IFMT_E4M3) {
+            x += (long long)qi[4 * i] * kv.x;
+            x += (long long)qi[4 * i + 1] * kv.y;
+            x += (long long)qi[4 * i + 2] * kv.z;
+            x += (long long)qi[4 * i + 3] * kv.w;
+          } else {
+            x += qi[4 * i] * kv.x + qi[4 * i + 1] * kv.y + qi[4 * i + 2] * kv.z + qi[4 * i + 3] * kv.w;
+          }
+        }
+        acc[u] = x;
       }
     }
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      const double part = (acc[u][0] + acc[u][1]) + (acc[u][2] + acc[u][3]);   // exact
       const int e = min(e0 + u, cnt - 1);
       double D;
       if (F == CSA_IFMT_E4M3) {
-        double raw = part + __shfl_xor_sync(0xffffffffu, part, 1);
-        raw += __shfl_xor_sync(0xffffffffu, raw, 2);                             // exact
-        D = live ? ((double)sm.qsc[j] * (double)sm.ksc[e][0]) * raw : 0.0;
+        long long raw = acc[u] + __shfl_xor_sync(0xffffffffu, acc[u], 1);
+        raw += __shfl_xor_sync(0xffffffffu, raw, 2);                                // exact
+        D = live ? ((double)sm.qsc[j] * (double)sm.ksc[e][0]) * ((double)raw * 3.814697265625e-06) : 0.0;   // 2^-18
       } else {
-        const double t = live ? ((double)sm.qsc[j * nb + q] * (double)sm.ksc[e][q]) * part : 0.0;
+        const double t = live ? ((double)sm.qsc[j * nb + q] * (double)sm.ksc[e][q]) * ((double)acc[u] * 0.25) : 0.0;
         const double t1 = __shfl_down_sync(0xffffffffu, t, 1);
         const double t2 = __shfl_down_sync(0xffffffffu, t, 2);
         const double t3 = __shfl_down_sync(0xffffffffu, t, 3);
@@ -265,29 +268,32 @@ indexer_select_hist_kernel(IndexerArgs a, int P, int chunk) {
       for (int q = 0; q < nb; ++q) sm.qsc[tid * nb + q] = ue8m0_to_float(((const uint8_t*)a.qI_scale)[((size_t)row * HI + tid) * nb + q]);
   }
   if (tid == 0) { sm.U = 0.f; sm.cnt = 0u; sm.ovf = 0u; }
-  double qr[32];
+  float qr[32];
+  int qi[32];
   {
     const int j = tid >> 2, q = tid & 3;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) qr[i] = 0.0;
+    for (int i = 0; i < 32; ++i) qr[i] = 0.f;
     if (j < HI && 32 * q < dI) {
       if (F == CSA_IFMT_E4M3) {
         const uint4* p = reinterpret_cast<const uint4*>((const uint8_t*)a.qI + qrow + (size_t)j * dI + 32 * q);
         const uint4 v0 = p[0], v1 = p[1];
         const uint32_t wds[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
-        for (int e = 0; e < 32; ++e) qr[e] = (double)e4m3_to_float((wds[e >> 2] >> (8 * (e & 3))) & 0xFFu);
+        for (int e = 0; e < 32; ++e) qr[e] = e4m3_to_float((wds[e >> 2] >> (8 * (e & 3))) & 0xFFu);
       } else {
         const uint4 v = *reinterpret_cast<const uint4*>((const uint8_t*)a.qI + (qrow + (size_t)j * dI + 32 * q) / 2);
         const uint32_t wds[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int e = 0; e < 32; ++e) qr[e] = (double)e2m1_to_float((wds[e >> 3] >> (4 * (e & 7))) & 0xFu);
+        for (int e = 0; e < 32; ++e) qr[e] = e2m1_to_float((wds[e >> 3] >> (4 * (e & 7))) & 0xFu);
       }
     }
     __syncthreads();                                         // w, scales, U = 0
     float ss = 0.f;
 #pragma unroll
-    for (int e = 0; e < 32; ++e) ss = fmaf((float)qr[e], (float)qr[e], ss);
+    for (int e = 0; e < 32; ++e) ss = fmaf(qr[e], qr[e], ss);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) qi[e] = (int)(qr[e] * (F == CSA_IFMT_E4M3 ? 512.f : 2.f));   // exact integers
     if (j < HI && 32 * q < dI) {
       const float sc = F == CSA_IFMT_E4M3 ? sm.qsc[j] : sm.qsc[j * nb + q];
       ss *= sc * sc;
@@ -310,7 +316,7 @@ indexer_select_hist_kernel(IndexerArgs a, int P, int chunk) {
           const int cnt = max(0, min(SH_RB, n - i0));
           if (tid < SH_RB) sm.rid[tid] = i0 + tid;
           __syncthreads();
-          if (cnt > 0) sh_rescore<F>(ks, sm, qr, b, cnt);
+          if (cnt > 0) sh_rescore<F>(ks, sm, qi, b, cnt);
           if (tid < SH_RB && i0 + tid < k) sout[i0 + tid] = tid < cnt ? (float)sm.rs_out[tid] : 0.f;
           __syncthreads();
         }
@@ -406,7 +412,7 @@ indexer_select_hist_kernel(IndexerArgs a, int P, int chunk) {
       const int cnt = (int)min((uint32_t)SH_RB, nb_mine - i0);
       if (tid < cnt) sm.rid[tid] = sm.band[i0 + tid].id;
       __syncthreads();
-      sh_rescore<F>(ks, sm, qr, b, cnt);
+      sh_rescore<F>(ks, sm, qi, b, cnt);
       if (tid < cnt) my_band[i0 + tid].s = sm.rs_out[tid];
     }
   } else if (tid == 0) {
@@ -585,7 +591,7 @@ indexer_select_hist_kernel(IndexerArgs a, int P, int chunk) {
       const int cnt = max(0, min(SH_RB, (int)written - i0));
       if (tid < SH_RB) sm.rid[tid] = (i0 + tid < k) ? __ldcg(out + i0 + tid) : 0;
       __syncthreads();
-      if (cnt > 0) sh_rescore<F>(ks, sm, qr, b, cnt);
+      if (cnt > 0) sh_rescore<F>(ks, sm, qi, b, cnt);
       if (tid < SH_RB && i0 + tid < k) sout[i0 + tid] = tid < cnt ? (float)sm.rs_out[tid] : 0.f;
       __syncthreads();
     }
