@@ -41,14 +41,17 @@ L2_BYTES = 126 * 1024 * 1024
 
 # DRAM bytes (read + write) per call of the dominant ABI call, summed over its kernels, from
 # the ncu captures summarised under profiles/ (None until a capture of the current kernels).
+TENSOR_PEAKS = {}   # measured once per single-GPU run (measure_tensor_peaks)
+
 TRAFFIC = {
-    # profiles/csa_decode_64k_dram_traffic.md: indexer_tc_kernel 34 768 896 + select 1 378 304 bytes
-    ("csa_decode_64k", "indexer"): 36147200,
-    # profiles/hybrid_pair_1m_launches.md: indexer_mxf4_kernel 144 098 816 + 7 310 592, select 8 669 952
-    ("hybrid_pair_1m", "indexer"): 160079360,
-    # profiles/hca_decode_1m_launches.md: attn_tc_kernel 38 996 736 (the combine's reads are L2 hits
-    # in the timed step; under ncu the caches are flushed before each kernel)
-    ("hca_decode_1m", "attention"): 38996736,
+    # profiles/csa_decode_64k_dram_traffic.md: indexer_tc_kernel<1,6> 34 770 688 + indexer_select_row 1 366 016
+    ("csa_decode_64k", "indexer"): 36136704,
+    # profiles/hybrid_pair_1m_dram_traffic.md: indexer_mxf4_kernel 143 312 128 read + 6 466 304 written
+    # (its histograms) + indexer_select_hist 8 931 328
+    ("hybrid_pair_1m", "indexer"): 158709760,
+    # profiles/hca_decode_1m_launches.md: attn_tc_kernel 39 008 896 read + 2 304 written (the combine's
+    # reads are L2 hits in the timed step; under ncu the caches are flushed before each kernel)
+    ("hca_decode_1m", "attention"): 39011200,
 }
 
 
@@ -98,6 +101,30 @@ def algorithmic_bytes(wid, D):
         return dict(compress=4 * Tq * d * 2, indexer=N * 132 + Tq * 64 * 132,
                     attention=Tq * H * d * 2 + Tq * H * dv * 2 + N * d * 2)
     raise ValueError(wid)
+
+
+def measure_tensor_peaks(csa):
+    """Dense MMA rate at the indexer's operand formats and shapes, measured by the library's
+    probe (operands resident in shared memory, one CTA per SM, CUDA events around three
+    launches after a warm-up), with the nominal dense figures beside it."""
+    import torch
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    res = {}
+    for name, fmt, n, iters, nominal in (("fp8_e4m3", csa.CSA_IFMT_E4M3, 256, 4000, 4500.0),
+                                         ("mxfp4", csa.CSA_IFMT_MXFP4, 64, 16000, 9000.0)):
+        csa.tensor_peak_probe(fmt, 100)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(3):
+            csa.tensor_peak_probe(fmt, iters)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / 3
+        flops = 2.0 * 128 * n * 128 * iters * sms
+        res[name] = {"tflops": flops / (ms * 1e-3) / 1e12, "nominal_tflops": nominal,
+                     "shape": f"M 128, N {n}, K 128 x {iters} per SM, {sms} SMs"}
+    return res
 
 
 def sample_clocks(stop, out):
@@ -249,6 +276,8 @@ def run_ours(args, wid, name):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
     import compressed_sparse_long_csa_b200 as csa
+    if world == 1 and "v" not in TENSOR_PEAKS:
+        TENSOR_PEAKS["v"] = measure_tensor_peaks(csa)
     from compressed_sparse_long_csa_b200 import steps
     import csa_inputs as CI
 
@@ -411,6 +440,7 @@ def run_ours(args, wid, name):
     src = "measured" if peaks else "fallback"
     hbm_peak = peaks.get("hbm_gbs", 6650.0)
     bf16_peak = peaks.get("bf16_tflops", 1590.0)
+    tpeaks = TENSOR_PEAKS.get("v") if world == 1 else None
     # the dominant ABI call by time; decode calls are HBM-bound, prefill calls tensor-bound
     # (the FP8 indexer against twice the measured bf16 peak, the nominal dense ratio)
     cand = [c for c in comp if c in ab]
@@ -418,15 +448,29 @@ def run_ours(args, wid, name):
     dom_ms = float(mean_ms[comp.index(dom)])
     fl = algorithmic_flops(wid, D)
     if wid == 3 and dom in fl:
-        peak = bf16_peak * (2.0 if dom == "indexer" else 1.0)
+        if dom == "indexer" and tpeaks:
+            peak, psrc = tpeaks["fp8_e4m3"]["tflops"], "measured fp8 MMA probe"
+        else:
+            peak = bf16_peak * (2.0 if dom == "indexer" else 1.0)
+            psrc = src + (" bf16 x 2 (fp8)" if dom == "indexer" else " bf16 burst")
         achieved = fl[dom] / (dom_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "peak_source": src + (" bf16 x 2 (fp8)" if dom == "indexer" else " bf16 burst"),
-                "traffic": TRAFFIC.get((name, dom))}
+                "frac": achieved / peak, "peak_source": psrc, "traffic": TRAFFIC.get((name, dom))}
     else:
         achieved = ab[dom] / (dom_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak, "peak_source": src, "traffic": TRAFFIC.get((name, dom))}
+    # the indexer's tensor-side fraction beside its HBM one: its dot-product FLOPs (every
+    # eligible entry x 64 heads x d_I) against the measured MMA rate of its format
+    idx_tensor = None
+    if tpeaks and wid in (1, 3, 4):
+        fmt_key = "fp8_e4m3" if D["ifmt"] == "e4m3" else "mxfp4"
+        if fmt_key in tpeaks:
+            idx_fl = fl.get("indexer") if wid == 3 else float(2 * D["HI"] * D["dI"] * D["N"] * D["B"])
+            a_tf = idx_fl / (float(mean_ms[comp.index("indexer")]) * 1e-3) / 1e12
+            idx_tensor = {"achieved": a_tf, "peak": tpeaks[fmt_key]["tflops"], "unit": "TFLOP/s",
+                          "frac": a_tf / tpeaks[fmt_key]["tflops"], "nominal_peak": tpeaks[fmt_key]["nominal_tflops"],
+                          "peak_source": "measured " + fmt_key + " MMA probe"}
     extra = None
     if world == 1:
         # the rows beyond the step, each timed alone on this GPU (single-GPU characterisations:
@@ -455,6 +499,10 @@ def run_ours(args, wid, name):
         "gpu_launches": launches_step * args.steps,
         "clocks": summarize_clocks(clock_lines),
     }
+    if idx_tensor:
+        line["indexer_tensor"] = idx_tensor
+    if tpeaks:
+        line["tensor_peaks"] = tpeaks
     if extra:
         line["next_rows"] = extra
     if rank == 0 and not args.no_cpu_baseline and world == 1:

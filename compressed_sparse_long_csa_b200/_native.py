@@ -23,6 +23,7 @@ _SIGS = {
     "csa_read_device_error": ([_vp, C.POINTER(C.c_uint32)], _i32),
     "csa_launch_count": ([], C.c_uint64),
     "csa_wait_probe": ([C.c_uint64, _vp], _i32),
+    "csa_tensor_peak_probe": ([_i32, _i32, _vp], _i32),
     "csa_compress": ([_vp] * 10 + [_i64, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
     "csa_compress_kv8": ([_vp] * 10 + [_i64, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
     "csa_decode_append": ([_vp] * 10 + [_i64, _i32] + [_vp] * 10 + [_i32, _i32, _vp, _vp, _vp, _i32, _i32, _i32, _vp], _i32),
@@ -107,6 +108,11 @@ def window_append(raw_new, win, win_slot, stream=None):
 def wait_probe(limit_ns: int, stream=None):
     """One kernel whose wait can never end, bounded by limit_ns (sets CSA_DEVERR_TIMEOUT)."""
     _check(lib.csa_wait_probe(int(limit_ns), _stream(stream)), "csa_wait_probe")
+
+
+def tensor_peak_probe(ifmt, iters, stream=None):
+    """Dense MMA rate probe at the indexer's operand formats (see csa_tensor_peak_probe)."""
+    _check(lib.csa_tensor_peak_probe(int(ifmt), int(iters), _stream(stream)), "csa_tensor_peak_probe")
 
 
 def launch_count() -> int:

@@ -25,6 +25,7 @@ cudaError_t launch_grouped_out_proj(const void* o, int T, int H, int dv, int g, 
                                     const void* W2, int d, void* u, void* y, float* part, size_t part_elems,
                                     cudaStream_t st, unsigned* err);
 cudaError_t launch_wait_probe(uint64_t limit_ns, cudaStream_t st, unsigned* err);
+cudaError_t launch_tensor_peak_probe(int ifmt, int iters, cudaStream_t st, unsigned* err);
 cudaError_t launch_decode_append(const void*, const void*, const void*, const void*, const float*, const float*,
                                  const void*, const void*, const int32_t*, void*, int64_t, int, const void*,
                                  const void*, const void*, const void*, const float*, const float*, const void*,
@@ -127,6 +128,14 @@ csa_status csa_read_device_error(void* stream, uint32_t* out) {
   if (e != cudaSuccess) return CSA_ERR_CUDA;
   *out = h;
   return CSA_OK;
+}
+
+csa_status csa_tensor_peak_probe(int ifmt, int iters, void* stream) {
+  REQUIRE(ifmt == CSA_IFMT_E4M3 || ifmt == CSA_IFMT_MXFP4, CSA_ERR_DTYPE);
+  REQUIRE(iters >= 1 && iters <= 1000000, CSA_ERR_SHAPE);
+  unsigned* err = device_error_word();
+  REQUIRE(err, CSA_ERR_CUDA);
+  return cuda_status(launch_tensor_peak_probe(ifmt, iters, S(stream), err));
 }
 
 csa_status csa_wait_probe(uint64_t limit_ns, void* stream) {

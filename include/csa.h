@@ -92,6 +92,17 @@ uint64_t csa_launch_count(void);
  * counterpart: it lets a caller check that a wait that cannot end returns an error. */
 csa_status csa_wait_probe(uint64_t limit_ns, void* stream);
 
+/* csa_tensor_peak_probe — the dense tensor-core rate at the indexer's operand formats,
+ * for the rooflines of the scoring kernels.  One CTA per SM issues iters x 128 of K of
+ * MMAs on operands resident in shared memory (nothing is read from or written to global
+ * memory except the error word): ifmt = CSA_IFMT_E4M3 runs kind::f8f6f4, M 128, N 256
+ * (2 * 128 * 256 * 128 * iters FLOP per SM); CSA_IFMT_MXFP4 runs kind::mxf4.block_scale,
+ * M 128, N 64 (2 * 128 * 64 * 128 * iters FLOP per SM).  Time it with events on the stream.
+ * iters in 1 .. 1e6 (CSA_ERR_SHAPE otherwise); other formats CSA_ERR_DTYPE.  A wait that
+ * gives up sets CSA_DEVERR_TIMEOUT.  The pages have no counterpart: it measures the GPU,
+ * not the method. */
+csa_status csa_tensor_peak_probe(int ifmt, int iters, void* stream);
+
 /* ---------------------------------------------------------------------------
  * csa_compress — CSA token-axis compression fused with the KV-cache append.
  * ("Гибридное внимание: CSA и HCA", CSA step 1: two KV series C^a, C^b and two
