@@ -271,7 +271,7 @@ constexpr size_t kHistCounters = 256;     // per row: certain count, CTAs done, 
 //   fhist [R][65536] | counters [R][256] | bitmap [R][ld/32] | band [R][ld] x 16 bytes
 // R = B * Tq.  knmax .. counters is one contiguous region, zeroed by one memset per call.
 struct IdxWs {
-  size_t scores, knmax, keyrange, hist, fhist, counters, bitmap, cand, end, zero_end;
+  size_t scores, knmax, keyrange, hist, fhist, counters, bitmap, cand, end, zero_end, scand, smeta;
 };
 static IdxWs idx_ws_layout(int B, int Tq, int64_t n_max) {
   const size_t R = (size_t)B * Tq, ld = (size_t)idx_ld(n_max);
@@ -288,6 +288,11 @@ static IdxWs idx_ws_layout(int B, int Tq, int64_t n_max) {
     L.bitmap = L.counters + round_up(R * kHistCounters * sizeof(unsigned), 256);
     L.cand = L.bitmap + round_up(R * (ld / 32) * sizeof(unsigned), 256);
     L.end = L.cand + round_up(R * ld * 16, 256);
+  } else {
+    // prefill rows: the streaming selection's candidate lists and their summaries
+    L.scand = L.hist;
+    L.smeta = L.scand + round_up(R * IDX_STREAM_CAP * sizeof(uint2), 256);
+    L.end = L.smeta + round_up(R * sizeof(uint4), 256);
   }
   return L;
 }
@@ -337,6 +342,14 @@ static csa_status run_lightning_index(const void* qI, const void* qI_scale, cons
   const bool row_path = decode_rows && (ifmt == CSA_IFMT_E4M3 || ifmt == CSA_IFMT_MXFP4) &&
                         n_max <= indexer_select_row_max_entries();
   const bool hist_path = decode_rows && !row_path;
+  // prefill rows that one CTA per four queries scores completely: the streaming selection
+  // (candidates instead of scores; nothing to zero)
+  if (Tq > kHistMaxTq && !bf16_scores && tc_enabled()) {
+    a.stream_cand = reinterpret_cast<uint2*>(ws + L.scand);
+    a.stream_meta = reinterpret_cast<uint4*>(ws + L.smeta);
+    if (!indexer_stream_applies(a)) a.stream_cand = nullptr, a.stream_meta = nullptr;
+  }
+  const bool stream_path = a.stream_cand != nullptr;
   if (hist_path) {
     a.hist = (unsigned*)(ws + L.hist);
     a.fhist = (unsigned*)(ws + L.fhist);
@@ -344,8 +357,11 @@ static csa_status run_lightning_index(const void* qI, const void* qI_scale, cons
     a.bitmap = (unsigned*)(ws + L.bitmap);
     a.cand = ws + L.cand;
   }
-  // zeroed per call: knmax and the key ranges, and the histograms and counters when used
-  cudaError_t e = cudaMemsetAsync(ws + L.knmax, 0, (hist_path ? L.zero_end : L.hist) - L.knmax, S(stream));
+  // zeroed per call: the key-norm bound and key ranges, and the histograms and counters when
+  // used; the streaming path needs only the bound (its pre-pass takes the keys' actual norms)
+  cudaError_t e = cudaMemsetAsync(ws + L.knmax, 0, (hist_path ? L.zero_end : stream_path ? L.keyrange : L.hist) - L.knmax,
+                                  S(stream));
+  if (e == cudaSuccess && stream_path) e = launch_key_norm_max(a, S(stream));
   if (e != cudaSuccess) return CSA_ERR_CUDA;
   bool used_tc = false;
   if (tc_enabled()) {
@@ -364,6 +380,10 @@ static csa_status run_lightning_index(const void* qI, const void* qI_scale, cons
     RowCount rc;
     rc.q_pos = q_pos; rc.n_entries = n_entries; rc.m = m; rc.Tq = Tq;
     return cuda_status(launch_topk_select(a.scores, a.ld, rc, B * Tq, n_max, k, idx_out, S(stream), err));
+  }
+  if (stream_path) {
+    if (!used_tc) return CSA_ERR_CUDA;                          // the streaming kernel always takes these rows
+    return cuda_status(launch_indexer_select_stream(a, S(stream)));
   }
   if (row_path && used_tc) {
     const cudaError_t er = launch_indexer_select_row(a, S(stream));

@@ -32,7 +32,14 @@ struct IndexerArgs {
   unsigned* counters;         // [B*Tq][256]: certain entries, CTAs done, overflow, per-CTA band counts; zeroed
   unsigned* bitmap;           // [B*Tq][ld/32] certain entries
   void* cand;                 // [B*Tq][ld] band entries, 16 bytes each (order key, entry id, exact score)
+  // prefill rows of the streaming selection (indexer_tc.cu, select_row.cu), else null:
+  uint2* stream_cand;         // [B*Tq][IDX_STREAM_CAP] (order key, entry id) of each row's candidates
+  uint4* stream_meta;         // [B*Tq]: candidates, threshold key, U (float bits), key-norm bound (float bits)
 };
+
+// Candidates one prefill row keeps while it is scored (the streaming selection).
+constexpr int IDX_STREAM_CAP = 2048;
+constexpr int IDX_STREAM_KMAX = 1024;        // largest k the streaming selection takes
 
 // Entries of one selection row: n_valid[row] (topk_select), else the indexer's
 // eligibility min(n_entries[b], (q_pos[row] + 1) / m) when q_pos is set, else n_cap;
@@ -117,6 +124,14 @@ cudaError_t launch_indexer_select_hist(const IndexerArgs& a, cudaStream_t st);
 // One-CTA-per-row selection of decode rows over the staged fp32 scores (select_row.cu);
 // cudaErrorNotSupported for other shapes.
 cudaError_t launch_indexer_select_row(const IndexerArgs& a, cudaStream_t st);
+// The exact selection of prefill rows from the candidates the streaming scoring kernel kept
+// (select_row.cu, one CTA per row).
+cudaError_t launch_indexer_select_stream(const IndexerArgs& a, cudaStream_t st);
+// Whether the streaming scoring + selection takes these rows (E4M3 keys of width 128, 64
+// heads, at least four queries per sequence, a grid that fills the GPU, k small enough).
+bool indexer_stream_applies(const IndexerArgs& a);
+// knmax[b] = the largest key norm of sequence b (E4M3 keys of width 128; knmax zeroed before).
+cudaError_t launch_key_norm_max(const IndexerArgs& a, cudaStream_t st);
 int64_t indexer_select_row_max_entries();
 cudaError_t launch_topk_select_cluster(const float* scores, int64_t ld, RowCount rc, int R, int64_t n,
                                        int k, int32_t* idx_out, cudaStream_t st);

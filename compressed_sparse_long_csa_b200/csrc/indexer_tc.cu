@@ -22,6 +22,7 @@
 #include "tc.cuh"
 
 #include <cudaTypedefs.h>
+#include <type_traits>
 
 namespace csa {
 
@@ -87,7 +88,39 @@ __device__ __forceinline__ void hist_flush(const uint32_t* fwin, uint32_t fbase,
   }
 }
 
-template <int G, int STAGES, bool HIST>
+// ---- the streaming selection of prefill rows --------------------------------------------
+// A CTA of the four-query kernel scores every eligible entry of its rows (one entry split),
+// so instead of writing the scores it keeps, per row, the entries whose order key is at
+// least a running threshold (IDX_STREAM_CAP of them in shared memory).  When a row's list has
+// less than two tiles' worth of room, the 256 epilogue threads compact it: the k-th largest
+// key of the list lies in a histogram bin [b_lo, ...]; the exact k-th largest score of the
+// row can only be larger, and an entry below it by more than the error band 2E can never be
+// selected, so the threshold rises to b_lo - 2E(b_lo) (rounded down; x - 2E(x) grows with x)
+// and the entries below it leave.  At the end the lists go to the workspace with the
+// threshold, U and the key-norm bound they used, and the selection kernel finishes each row
+// from its list (select_row.cu).  No score leaves the SM.
+constexpr int ST_T = 256;                  // epilogue threads (warps 4..11)
+constexpr int ST_HB = 2048;                // bins of the compaction histograms (all rows)
+constexpr int ST_PAIRS = 2;                // pairs of tiles between two meetings of the epilogue threads
+static_assert(IDX_STREAM_CAP - 2 * ST_PAIRS * IT_ROWS > IDX_STREAM_KMAX,
+              "a compacted list (about k entries) leaves room for the appends until the next meeting");
+
+template <int G>
+struct StreamBuf {
+  uint32_t ckey[G][IDX_STREAM_CAP];        // order keys of the kept entries
+  int32_t cid[G][IDX_STREAM_CAP];          // their indices
+  uint32_t hist[ST_HB];
+  unsigned long long ccnt;                  // the rows' list lengths, 16 bits each
+  uint32_t thr[G], ovf[G];
+  float U[G];
+  uint32_t kmaxbits;
+  uint32_t red[G][ST_T / 32];
+  uint32_t lo[G], hi[G], bin[G];
+};
+struct StreamNone {};
+static_assert(IDX_STREAM_CAP + 2 * 2 * 128 < 65536, "the packed 16-bit list lengths cannot carry");
+
+template <int G, int STAGES, bool HIST, bool STREAM = false>
 struct IdxSmem {
   alignas(1024) uint8_t q[G * 64 * IT_KB];
   alignas(1024) uint8_t k[STAGES][IT_TILE_BYTES];
@@ -105,13 +138,195 @@ struct IdxSmem {
   int n_elig[G];
   int row[G];
   alignas(16) float wq[G][64];
+  typename std::conditional<STREAM, StreamBuf<G>, StreamNone>::type st;
 };
 
-template <int G, int STAGES, bool HIST>
+// The weighted ReLU head sum of one entry (TMEM lane = the thread's entry) for query g of the
+// accumulator at column `col`: four partial sums over the heads (j mod 4).
+__device__ __forceinline__ float head_sum(uint32_t tmem_lane_col, const float* wq) {
+  float part[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int q16 = 0; q16 < 4; ++q16) {
+    uint32_t v[16];
+    tc::tmem_ld16(tmem_lane_col + q16 * 16, v);
+    // the 16 weights as four 16-byte loads, in flight with the TMEM load (one load per
+    // weight exposed its latency 64 times per tile)
+    const float4* w4p = reinterpret_cast<const float4*>(wq + q16 * 16);
+    float4 w4[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) w4[u] = w4p[u];
+    tc::tmem_ld_wait();
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      part[0] = fmaf(w4[u].x, fmaxf(__uint_as_float(v[4 * u]), 0.f), part[0]);
+      part[1] = fmaf(w4[u].y, fmaxf(__uint_as_float(v[4 * u + 1]), 0.f), part[1]);
+      part[2] = fmaf(w4[u].z, fmaxf(__uint_as_float(v[4 * u + 2]), 0.f), part[2]);
+      part[3] = fmaf(w4[u].w, fmaxf(__uint_as_float(v[4 * u + 3]), 0.f), part[3]);
+    }
+  }
+  return (part[0] + part[1]) + (part[2] + part[3]);
+}
+
+// Barrier of the 256 epilogue threads (named barrier 1; the producer and MMA warps go on).
+__device__ __forceinline__ void ep_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+// Length of row g's list (16 bits of the packed counts; a list that overflowed keeps counting
+// to at most IDX_STREAM_CAP + 2 * ST_PAIRS * 128 < 2^16).
+template <int G>
+__device__ __forceinline__ uint32_t st_count(const StreamBuf<G>& st, int g) {
+  return (uint32_t)((*(volatile const unsigned long long*)&st.ccnt >> (16 * g)) & 0xFFFFull);
+}
+
+// Exclusive scan of G values per epilogue thread at once; tot[g] = the sums.
+template <int G>
+__device__ __forceinline__ void ep_scan_g(const uint32_t (&v)[G], uint32_t (&excl)[G], uint32_t (&tot)[G],
+                                          uint32_t (*red)[ST_T / 32]) {
+  const int te = threadIdx.x - 128, lane = te & 31, w = te >> 5;
+  uint32_t incl[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    incl[g] = v[g];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t x = __shfl_up_sync(0xffffffffu, incl[g], o);
+      if (lane >= o) incl[g] += x;
+    }
+  }
+  ep_sync();
+  if (lane == 31)
+#pragma unroll
+    for (int g = 0; g < G; ++g) red[g][w] = incl[g];
+  ep_sync();
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    uint32_t pre = 0, t = 0;
+#pragma unroll
+    for (int i = 0; i < ST_T / 32; ++i) {
+      const uint32_t x = red[g][i];
+      pre += i < w ? x : 0u;
+      t += x;
+    }
+    excl[g] = pre + incl[g] - v[g];
+    tot[g] = t;
+  }
+}
+
+// Compact every row's list at once: raise each row's threshold to b_lo - 2E(b_lo), b_lo the
+// lower edge of the histogram bin (512 bins over the list's key range) that holds the list's
+// k-th largest key, and drop the entries below it.  A row with at most k entries keeps all.
+template <int G>
+__device__ __noinline__ void ep_compact_all(StreamBuf<G>& st, uint32_t k, const float (&EU)[G]) {
+  constexpr int HB = ST_HB / G;             // bins per row
+  const int te = threadIdx.x - 128, lane = te & 31;
+  uint32_t n[G], mn[G], mx[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    n[g] = min(st_count(st, g), (uint32_t)IDX_STREAM_CAP);
+    mn[g] = 0xFFFFFFFFu;
+    mx[g] = 0u;
+    for (uint32_t i = te; i < n[g]; i += ST_T) {
+      const uint32_t key = st.ckey[g][i];
+      mn[g] = min(mn[g], key);
+      mx[g] = max(mx[g], key);
+    }
+    mn[g] = __reduce_min_sync(0xffffffffu, mn[g]);
+    mx[g] = __reduce_max_sync(0xffffffffu, mx[g]);
+  }
+  if (te < G) { st.lo[te] = 0xFFFFFFFFu; st.hi[te] = 0u; st.bin[te] = 0u; }
+  for (int i = te; i < ST_HB; i += ST_T) st.hist[i] = 0u;
+  ep_sync();
+  if (lane == 0)
+#pragma unroll
+    for (int g = 0; g < G; ++g) { atomicMin(&st.lo[g], mn[g]); atomicMax(&st.hi[g], mx[g]); }
+  ep_sync();
+  int sh[G];
+  uint32_t lo[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    lo[g] = st.lo[g];
+    const uint64_t width = st.hi[g] >= lo[g] ? (uint64_t)(st.hi[g] - lo[g]) + 1u : 1u;
+    const int bits = width <= 1 ? 0 : 64 - __clzll((long long)(width - 1));
+    constexpr int LB = HB == 2048 ? 11 : HB == 1024 ? 10 : 9;
+    sh[g] = bits > LB ? bits - LB : 0;
+    for (uint32_t i = te; i < n[g]; i += ST_T) atomicAdd(&st.hist[g * HB + ((st.ckey[g][i] - lo[g]) >> sh[g])], 1u);
+  }
+  ep_sync();
+  // the bin of the k-th largest key of each row: thread t holds bins [HB/ST_T * t, +HB/ST_T)
+  constexpr int PER = HB / ST_T;
+  {
+    uint32_t c[G][PER], mine[G], excl[G], tot[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      mine[g] = 0u;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) { c[g][i] = st.hist[g * HB + PER * te + i]; mine[g] += c[g][i]; }
+    }
+    ep_scan_g<G>(mine, excl, tot, st.red);
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      uint32_t above = tot[g] - excl[g] - mine[g];
+#pragma unroll
+      for (int i = PER - 1; i >= 0; --i) {
+        if (above < k && k <= above + c[g][i]) st.bin[g] = (uint32_t)(PER * te + i);
+        above += c[g][i];
+      }
+    }
+  }
+  ep_sync();
+  uint32_t thr[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    thr[g] = st.thr[g];
+    if (n[g] > k) {
+      const float x = f32_from_order_key(lo[g] + (st.bin[g] << sh[g]));
+      const float E2 = 2.f * ((EU[g] + 1.52587890625e-05f * fabsf(x)) * 1.0002f);
+      thr[g] = max(thr[g], f32_order_key(__fsub_rd(x, E2)));
+    }
+  }
+  // in place: thread t keeps slots t, t + 256, ... of every row (conflict-free reads; the list's
+  // order does not matter)
+  constexpr int SL = IDX_STREAM_CAP / ST_T;
+  uint32_t kk[G][SL], keep[G], cnt[G], pos[G], tot2[G];
+  int32_t ii[G][SL];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    keep[g] = 0u;
+#pragma unroll
+    for (int u = 0; u < SL; ++u) {
+      const uint32_t i = te + ST_T * u;
+      const bool v = i < n[g];
+      kk[g][u] = v ? st.ckey[g][i] : 0u;
+      ii[g][u] = v ? st.cid[g][i] : 0;
+      keep[g] |= (v && kk[g][u] >= thr[g] ? 1u : 0u) << u;
+    }
+    cnt[g] = __popc(keep[g]);
+  }
+  ep_scan_g<G>(cnt, pos, tot2, st.red);                  // its barriers order the reads above before the writes
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+#pragma unroll
+    for (int u = 0; u < SL; ++u)
+      if ((keep[g] >> u) & 1u) {
+        st.ckey[g][pos[g]] = kk[g][u];
+        st.cid[g][pos[g]] = ii[g][u];
+        ++pos[g];
+      }
+    if (te == 0) st.thr[g] = thr[g];
+  }
+  if (te == 0) {
+    unsigned long long c = 0ull;
+#pragma unroll
+    for (int g = 0; g < G; ++g) c |= (unsigned long long)tot2[g] << (16 * g);
+    st.ccnt = c;
+  }
+  ep_sync();
+}
+
+template <int G, int STAGES, bool HIST, bool STREAM = false>
 __global__ void __launch_bounds__(IT_THREADS, G == 1 ? 2 : 1)
 indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ, IdxTcParams p) {
   extern __shared__ uint8_t smem_raw[];
-  using Sm = IdxSmem<G, STAGES, HIST>;
+  using Sm = IdxSmem<G, STAGES, HIST, STREAM>;
   Sm& sm = *reinterpret_cast<Sm*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const IndexerArgs& a = p.a;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -224,7 +439,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         if (last_issued >= 0) tc::mbar_wait(&sm.tfull[last_issued % NACC], (last_issued / NACC) & 1);
       }
     }
-  } else if (warp >= 4) {
+  } else if (warp >= 4 && !STREAM) {
     // epilogue warpgroup e takes tiles e, e+2, ...; quarter q = warp % 4 reads TMEM lanes 32q..32q+31
     const int e = (warp - 4) >> 2, quarter = warp & 3;
     const int r = quarter * 32 + lane;
@@ -249,29 +464,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
       const int s = (t_begin + it) * IT_ROWS + r;
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        // four partial sums over the heads (j mod 4)
-        float part[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int q16 = 0; q16 < 4; ++q16) {
-          uint32_t v[16];
-          const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + acc * N + g * 64 + q16 * 16;
-          tc::tmem_ld16(ta, v);
-          // the 16 weights as four 16-byte loads, in flight with the TMEM load (one load per
-          // weight exposed its latency 64 times per tile)
-          const float4* w4p = reinterpret_cast<const float4*>(&sm.wq[g][q16 * 16]);
-          float4 w4[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) w4[u] = w4p[u];
-          tc::tmem_ld_wait();
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            part[0] = fmaf(w4[u].x, fmaxf(__uint_as_float(v[4 * u]), 0.f), part[0]);
-            part[1] = fmaf(w4[u].y, fmaxf(__uint_as_float(v[4 * u + 1]), 0.f), part[1]);
-            part[2] = fmaf(w4[u].z, fmaxf(__uint_as_float(v[4 * u + 2]), 0.f), part[2]);
-            part[3] = fmaf(w4[u].w, fmaxf(__uint_as_float(v[4 * u + 3]), 0.f), part[3]);
-          }
-        }
-        const float val = (part[0] + part[1]) + (part[2] + part[3]);
+        const float val = head_sum(tmem + ((uint32_t)(quarter * 32) << 16) + acc * N + g * 64, sm.wq[g]);
         const bool valid = s < sm.n_elig[g];
         const float sc = a.score_bf16 ? round_bf16(val * sk) : val * sk;
         if (valid) {
@@ -290,6 +483,128 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     // |k8| <= 448 per element, so ||k_s|| <= sk * 448 * sqrt(d_I)
     kmax = warp_max(kmax);
     if (lane == 0 && kmax > 0.f) atomicMax(a.knmax + b, __float_as_uint(kmax * 448.f * 11.3137085f * 1.0001f));
+  } else if (warp >= 4) {
+    if constexpr (STREAM) {
+      // the streaming selection (see StreamBuf): candidates instead of scores
+      StreamBuf<G>& st = sm.st;
+      const int e = (warp - 4) >> 2, quarter = warp & 3;
+      const int r = quarter * 32 + lane, te = threadIdx.x - 128;
+      const float* kscale = (const float*)a.kI_scale;
+      if (te < G) { st.thr[te] = 0u; st.ovf[te] = 0u; st.U[te] = 0.f; }
+      if (te == 0) st.ccnt = 0ull;
+      if (te == 0) st.kmaxbits = 0u;
+      ep_sync();
+      // the sequence's key-norm bound (key_norm_max_kernel, before this kernel), and
+      // U = sum_j |w_j| ||q_j|| per row (thread te: head te / 4, dims [32 (te % 4), +32))
+      {
+        if (te == 0) st.kmaxbits = __ldcg(a.knmax + b);
+        const int j = te >> 2, q = te & 3;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const int t = qg * G + g;
+          float ss = 0.f;
+          if (t < a.Tq) {
+            const uint4* qp = reinterpret_cast<const uint4*>((const uint8_t*)a.qI +
+                                                             (((size_t)b * a.Tq + t) * 64 + j) * IT_KB + 32 * q);
+            const uint4 v0 = __ldg(qp), v1 = __ldg(qp + 1);
+            const uint32_t wd[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float x = e4m3_to_float((wd[i >> 2] >> (8 * (i & 3))) & 0xFFu);
+              ss = fmaf(x, x, ss);
+            }
+          }
+          ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+          ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+          float u = (q == 0 && t < a.Tq) ? fabsf(sm.wq[g][j]) * sqrtf(ss) : 0.f;   // wq = w * sq
+          u = warp_sum(u);
+          if (lane == 0) atomicAdd(&st.U[g], u);
+        }
+      }
+      ep_sync();
+      const float knmax = __uint_as_float(st.kmaxbits);
+      float EU[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) EU[g] = (a.eps_dot + 1.9073486328125e-06f) * st.U[g] * knmax * 1.0002f;
+      auto load_scale = [&](int it) {
+        const int s = (t_begin + it) * IT_ROWS + r;
+        return (it < n_t && s < a.n_max) ? __ldg(kscale + (size_t)b * a.n_max + s) : 0.f;
+      };
+      float sk_next = load_scale(e);
+      bool alive = true;
+      const int npairs = (n_t + 1) >> 1;
+      // the epilogue threads meet every ST_PAIRS pairs of tiles; a list with less room than
+      // those pairs can append is compacted there
+      for (int ip = 0; ip < npairs; ++ip) {
+        const int it = 2 * ip + e;
+        if (it < n_t && alive) {
+          const int acc = it % NACC;
+          const uint32_t aph = (it / NACC) & 1;
+          const float sk = sk_next;
+          sk_next = load_scale(it + 2);
+          bool ok = tc::mbar_wait(&sm.tfull[acc], aph) && !*(volatile int*)&sm.abort_flag;
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) {
+            atomicExch(&sm.abort_flag, 1);
+            alive = false;
+          } else {
+            tc::fence_after_sync();
+            const int s = (t_begin + it) * IT_ROWS + r;
+            // every row's entries first, then one shared-memory atomic per warp reserves the
+            // slots of all rows at once (the four row counts are 16-bit fields of one word)
+            uint32_t key[G], bt[G];
+            unsigned long long inc = 0ull;
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+              const float val = head_sum(tmem + ((uint32_t)(quarter * 32) << 16) + acc * N + g * 64, sm.wq[g]);
+              key[g] = f32_order_key(val * sk);
+              bt[g] = __ballot_sync(0xffffffffu, s < sm.n_elig[g] && key[g] >= st.thr[g]);
+              inc |= (unsigned long long)__popc(bt[g]) << (16 * g);
+            }
+            if (inc) {
+              unsigned long long old = 0ull;
+              if (lane == 0) old = atomicAdd(&st.ccnt, inc);
+              old = __shfl_sync(0xffffffffu, old, 0);
+#pragma unroll
+              for (int g = 0; g < G; ++g) {
+                if (!((bt[g] >> lane) & 1u)) continue;
+                const uint32_t off = (uint32_t)((old >> (16 * g)) & 0xFFFFull) + __popc(bt[g] & ((1u << lane) - 1u));
+                if (off < (uint32_t)IDX_STREAM_CAP) {
+                  st.ckey[g][off] = key[g];
+                  st.cid[g][off] = s;
+                } else {
+                  st.ovf[g] = 1u;
+                }
+              }
+            }
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&sm.tempty[acc]);
+          }
+        }
+        if (ip % ST_PAIRS == ST_PAIRS - 1 || ip == npairs - 1) {
+          ep_sync();
+          // (the decision reads shared memory after the barrier: every epilogue thread takes it alike)
+          bool full = false;
+#pragma unroll
+          for (int g = 0; g < G; ++g) full = full || st_count(st, g) > (uint32_t)(IDX_STREAM_CAP - 2 * ST_PAIRS * IT_ROWS);
+          if (full) ep_compact_all<G>(st, (uint32_t)a.k, EU);
+        }
+      }
+      // the lists, and what the selection needs to finish them
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const int t = qg * G + g;
+        if (t >= a.Tq) continue;
+        const size_t row = (size_t)b * a.Tq + t;
+        const uint32_t n = min(st_count(st, g), (uint32_t)IDX_STREAM_CAP);
+        for (uint32_t i = te; i < n; i += ST_T)
+          a.stream_cand[row * IDX_STREAM_CAP + i] = make_uint2(st.ckey[g][i], (uint32_t)st.cid[g][i]);
+        if (te == 0)
+          a.stream_meta[row] = make_uint4(n | (st.ovf[g] ? 0x80000000u : 0u), st.thr[g], __float_as_uint(st.U[g]),
+                                          __float_as_uint(knmax));
+      }
+    }
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -613,17 +928,18 @@ cudaError_t launch_mxf4(const IndexerArgs& a, cudaStream_t st, bool* used) {
   return cudaGetLastError();
 }
 
-template <int G, int STAGES, bool HIST>
+template <int G, int STAGES, bool HIST, bool STREAM = false>
 cudaError_t launch_g(const IndexerArgs& a, cudaStream_t st, bool* used) {
   IdxTcParams p{};
   p.a = a;
   p.n_qg = (a.Tq + G - 1) / G;
   p.tiles = (int)((a.n_max + IT_ROWS - 1) / IT_ROWS);
   // decode-like shapes: split the entry tiles so that the grid fills the SMs once
-  // (two CTAs per SM for the one-query variant, one for the four-query variant)
+  // (two CTAs per SM for the one-query variant, one for the four-query variant); the
+  // streaming selection keeps every entry of a row in one CTA
   const int64_t ctas = (int64_t)a.B * p.n_qg;
   const int64_t slots = G == 1 ? 2 * num_sms() : num_sms();
-  int splits = (int)(slots / ctas);
+  int splits = STREAM ? 1 : (int)(slots / ctas);
   if (splits > p.tiles) splits = p.tiles;
   if (splits < 1) splits = 1;
   p.tiles_per_split = (p.tiles + splits - 1) / splits;
@@ -631,18 +947,62 @@ cudaError_t launch_g(const IndexerArgs& a, cudaStream_t st, bool* used) {
   CUtensorMap mk, mq;
   if (!make_map_rows128(&mk, a.kI, (uint64_t)a.B * a.n_max, IT_ROWS)) return cudaSuccess;
   if (!make_map_rows128(&mq, a.qI, (uint64_t)a.B * a.Tq * 64, 64 * G)) return cudaSuccess;
-  const size_t smem = sizeof(IdxSmem<G, STAGES, HIST>) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<G, STAGES, HIST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  const size_t smem = sizeof(IdxSmem<G, STAGES, HIST, STREAM>) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<G, STAGES, HIST, STREAM>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(splits, p.n_qg, a.B);
   note_launch();
-  indexer_tc_kernel<G, STAGES, HIST><<<grid, IT_THREADS, smem, st>>>(mk, mq, p);
+  indexer_tc_kernel<G, STAGES, HIST, STREAM><<<grid, IT_THREADS, smem, st>>>(mk, mq, p);
   *used = true;
   return cudaGetLastError();
 }
 
 }  // namespace
+
+// The largest key norm of each sequence, for the streaming selection's error bound: one
+// thread per entry forms sk * sqrt(sum of its squared E4M3 codes) (fp32, times 1.0001 for the
+// rounding of 128 squares, the root and the product) and the warps' maxima go to knmax[b]
+// (zeroed by the caller) as float bits.  Tighter than the scale-only bound sk * 448 * sqrt(d_I)
+// by the ratio of a row's largest code to its root-mean-square code.
+__global__ void __launch_bounds__(256) key_norm_max_kernel(const uint8_t* __restrict__ kI, const float* __restrict__ ks,
+                                                           int64_t n_max, unsigned* knmax) {
+  const int b = blockIdx.y;
+  const int64_t s = (int64_t)blockIdx.x * 256 + threadIdx.x;
+  float nrm = 0.f;
+  if (s < n_max) {
+    const uint4* p = reinterpret_cast<const uint4*>(kI + ((size_t)b * n_max + s) * IT_KB);
+    float ss = 0.f;
+#pragma unroll
+    for (int v = 0; v < IT_KB / 16; ++v) {
+      const uint4 x = __ldg(p + v);
+      const uint32_t wd[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float c = e4m3_to_float((wd[i >> 2] >> (8 * (i & 3))) & 0xFFu);
+        ss = fmaf(c, c, ss);
+      }
+    }
+    nrm = __ldg(ks + (size_t)b * n_max + s) * sqrtf(ss) * 1.0001f;
+  }
+  nrm = warp_max(nrm);
+  if ((threadIdx.x & 31) == 0 && nrm > 0.f) atomicMax(knmax + b, __float_as_uint(nrm));
+}
+
+cudaError_t launch_key_norm_max(const IndexerArgs& a, cudaStream_t st) {
+  dim3 grid((unsigned)((a.n_max + 255) / 256), a.B);
+  note_launch();
+  key_norm_max_kernel<<<grid, 256, 0, st>>>((const uint8_t*)a.kI, (const float*)a.kI_scale, a.n_max, a.knmax);
+  return cudaGetLastError();
+}
+
+bool indexer_stream_applies(const IndexerArgs& a) {
+  if (a.ifmt != CSA_IFMT_E4M3 || a.H_I != 64 || a.d_I != 128 || a.Tq < 4 || a.score_bf16 || a.score_out) return false;
+  if (a.k > IDX_STREAM_KMAX || ((uintptr_t)a.kI & 15) || ((uintptr_t)a.qI & 15)) return false;
+  if ((int64_t)a.B * a.n_max > 0x7fffffffLL || (int64_t)a.B * a.Tq * 64 > 0x7fffffffLL) return false;
+  // one CTA per four queries holds all of their entries: enough of them to fill the GPU
+  return (int64_t)a.B * ((a.Tq + 3) / 4) >= num_sms();
+}
 
 // Tensor-core scores for E4M3 operands with 64 heads of width 128; other shapes
 // return *used = false and run on the CUDA-core path.
@@ -663,6 +1023,7 @@ cudaError_t launch_indexer_scores_tc(IndexerArgs& a, cudaStream_t st, bool* used
   // fp32 accumulation of exact products (128 * 2^-24 = 2^-17).  Measured on B200: <= 5e-9
   // relative to the bound's scale (test_indexer_fp32_score_error_within_band_bound).
   a.eps_dot = 1.0f / 131072.0f;
+  if (a.stream_cand) return launch_g<4, 6, false, true>(a, st, used);
   if (a.Tq >= 4) return launch_g<4, 6, false>(a, st, used);
   // decode rows: the score histogram for the selection (one fewer ring stage makes room
   // for it at two CTAs per SM)

@@ -51,9 +51,9 @@ constexpr int SR_CMAX = 8;                // CTAs per cluster
 constexpr int SR_HB = 4096;               // bins of the first histogram
 constexpr int SR_HB2 = 2048;              // bins of the refinements
 constexpr int SR_CCAP = 2048;             // candidates listed
-constexpr int SR_BCAP = 64;               // band entries re-scored exactly
+constexpr int SR_BCAP = 128;              // band entries re-scored exactly
 constexpr int SR_RB = 8;                  // entries re-scored at once
-constexpr int SR_NMAX = 32768;            // most scores a row stages in shared memory
+constexpr int SR_NMAX = 34816;            // most scores a row stages in shared memory (and bitmap bits)
 constexpr int SR_CHUNK = 16384;           // bytes per bulk copy (the first histogram starts on the first)
 constexpr int SR_KLD = 160;               // staged key row: dims 16 g .. 16 g + 15 at word 20 g (no bank conflicts)
 constexpr int SR_TLD = 66;                // per-head term row stride (the ordered sums read rows side by side)
@@ -75,7 +75,7 @@ struct SrSmem {
   float w[64];
   float qsc[64 * 4];
   uint32_t wred[SR_W];
-  alignas(8) uint64_t bar[SR_NMAX * 4 / SR_CHUNK];   // one per bulk copy
+  alignas(8) uint64_t bar[(SR_NMAX * 4 + SR_CHUNK - 1) / SR_CHUNK];   // one per bulk copy
   uint32_t bin, above, ccnt, bcnt, nsure, fail;
   float U;
   alignas(16) float sc[1];                // the row's scores (sized at launch)
@@ -291,7 +291,7 @@ indexer_select_row_kernel(IndexerArgs a) {
         sm.qsc[tid * nb + q] = ue8m0_to_float(((const uint8_t*)a.qI_scale)[((size_t)row * HI + tid) * nb + q]);
   }
   if (tid == 0) {
-    for (int c = 0; c < SR_NMAX * 4 / SR_CHUNK; ++c) tc::mbar_init(&sm.bar[c], 1);
+    for (int c = 0; c < (SR_NMAX * 4 + SR_CHUNK - 1) / SR_CHUNK; ++c) tc::mbar_init(&sm.bar[c], 1);
     tc::fence_mbar_init();
     sm.U = 0.f;
     sm.ccnt = 0u;
@@ -640,6 +640,197 @@ indexer_select_row_kernel(IndexerArgs a) {
   }
 }
 
+// The exact selection of a prefill row from the candidates the streaming scoring kernel kept
+// (indexer_tc.cu): every entry of the row whose order key is at least the list's threshold,
+// with the U and key-norm bound that threshold was computed from.  The k-th largest fp32 key
+// tau is at least the threshold, so it is the k-th largest of the list; the band
+// [tau - 2E, tau + 2E] (E from the same U and bound) lies above the threshold, so the list
+// holds all of it.  Then as the row selection: certain entries into the row's bitmap, the
+// band re-scored exactly and ranked, the bitmap written in ascending order.  One CTA per row.
+template <int F>
+__global__ void __launch_bounds__(SR_T, 1)
+indexer_select_stream_kernel(IndexerArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  SrSmem& sm = *reinterpret_cast<SrSmem*>(smem_raw);
+  const int row = blockIdx.x, b = row / a.Tq;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int k = a.k, HI = a.H_I, dI = a.d_I, nb = dI / 32;
+  int32_t* out = a.idx_out + (size_t)row * k;
+
+  // ---- prologue (inputs only): weights, query scales, the query codes as integers
+  if (tid < HI) {
+    sm.w[tid] = a.w[(size_t)row * HI + tid];
+    if (F == CSA_IFMT_E4M3) sm.qsc[tid] = ((const float*)a.qI_scale)[(size_t)row * HI + tid];
+    else
+      for (int q = 0; q < nb; ++q)
+        sm.qsc[tid * nb + q] = ue8m0_to_float(((const uint8_t*)a.qI_scale)[((size_t)row * HI + tid) * nb + q]);
+  }
+  if (tid == 0) { sm.bcnt = 0u; sm.nsure = 0u; sm.ccnt = 0u; }
+  const int qj = tid >> 3, qs = tid & 7;
+  const bool qlive = qj < HI && 16 * qs < dI;
+  int qi[16];
+  {
+    const size_t qrow = (size_t)row * HI * dI;
+    if (F == CSA_IFMT_E4M3) {
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (qlive) v = *reinterpret_cast<const uint4*>((const uint8_t*)a.qI + qrow + (size_t)qj * dI + 16 * qs);
+      const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 16; ++i) qi[i] = (int)(e4m3_to_float((wd[i >> 2] >> (8 * (i & 3))) & 0xFFu) * 512.f);
+    } else {
+      uint2 v = make_uint2(0u, 0u);
+      if (qlive) v = *reinterpret_cast<const uint2*>((const uint8_t*)a.qI + (qrow + (size_t)qj * dI + 16 * qs) / 2);
+      const uint32_t wd[2] = {v.x, v.y};
+#pragma unroll
+      for (int i = 0; i < 16; ++i) qi[i] = (int)(e2m1_to_float((wd[i >> 3] >> (4 * (i & 7))) & 0xFu) * 2.f);
+    }
+  }
+  const int n = row_eligible(a, row);
+  tc::griddep_wait();                                        // the candidate lists
+  tc::griddep_launch_dependents();
+  if (n <= k) {
+    for (int i = tid; i < k; i += SR_T) out[i] = i < n ? i : -1;
+    return;
+  }
+  const uint4 meta = __ldcg(a.stream_meta + row);
+  const uint32_t nc = min(meta.x & 0x7FFFFFFFu, (uint32_t)SR_CCAP);
+  const uint32_t thr = meta.y;
+  const float U = __uint_as_float(meta.z), knmax = __uint_as_float(meta.w);
+  if ((meta.x >> 31) && tid == 0) raise_err(a.err, CSA_DEVERR_BAND);      // a list overflowed: entries were lost
+  const uint2* cand = a.stream_cand + (size_t)row * IDX_STREAM_CAP;
+  for (uint32_t i = tid; i < nc; i += SR_T) {
+    const uint2 c = __ldcg(cand + i);
+    sm.ckey[i] = c.x;
+    sm.cid[i] = (int32_t)c.y;
+  }
+  const int nw = (n + 31) >> 5;
+  for (int w = tid; w < nw; w += SR_T) { sm.bm[w] = 0u; sm.tb[w] = 0u; }
+  for (int i = tid; i < SR_HB; i += SR_T) sm.hist[i] = 0u;
+  // the candidates' key range
+  uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+  __syncthreads();
+  for (uint32_t i = tid; i < nc; i += SR_T) { mn = min(mn, sm.ckey[i]); mx = max(mx, sm.ckey[i]); }
+  mn = __reduce_min_sync(0xffffffffu, mn);
+  mx = __reduce_max_sync(0xffffffffu, mx);
+  if (tid == 0) { sm.bin = 0xFFFFFFFFu; sm.above = 0u; }
+  __syncthreads();
+  if (lane == 0) { atomicMin(&sm.bin, mn); atomicMax(&sm.above, mx); }
+  __syncthreads();
+  const uint32_t lo = sm.bin, hi = max(sm.above, sm.bin);
+  // ---- the exact k-th largest key among the candidates
+  uint32_t want = (uint32_t)k, cur = lo;
+  uint64_t width = (uint64_t)(hi - lo) + 1u;
+  bool first = true;
+  while (width > 1) {
+    const int sh = sr_shift(width, first ? 12 : 11);
+    if (!first) {
+      for (int i = tid; i < SR_HB2; i += SR_T) sm.hist[i] = 0u;
+      __syncthreads();
+    }
+    for (uint32_t i = tid; i < nc; i += SR_T) {
+      const uint32_t key = sm.ckey[i];
+      if (key >= cur && (uint64_t)(key - cur) < width) atomicAdd(&sm.hist[(key - cur) >> sh], 1u);
+    }
+    __syncthreads();
+    if (first) sr_find_bin<SR_HB / SR_T>(sm, want);
+    else sr_find_bin<SR_HB2 / SR_T>(sm, want);
+    want -= sm.above;
+    cur += sm.bin << sh;
+    const uint64_t nwid = 1ull << sh;
+    width = nwid < width ? nwid : width;
+    first = false;
+  }
+  const uint32_t tkey = cur, quota = want;
+  const float tau = f32_from_order_key(tkey);
+  const float EU = (a.eps_dot + 1.9073486328125e-06f) * U * knmax * 1.0002f;
+  const float E2 = 2.f * ((EU + 1.52587890625e-05f * fabsf(tau)) * 1.0002f);
+  const float band_hi = __fadd_ru(tau, E2), band_lo = __fsub_rd(tau, E2);
+  if (f32_order_key(band_lo) < thr && tid == 0) raise_err(a.err, CSA_DEVERR_BAND);   // cannot happen: same U, bound
+  // ---- certain entries and the band
+  for (uint32_t i = tid; i < nc; i += SR_T) {
+    const int id = sm.cid[i];
+    const float s = f32_from_order_key(sm.ckey[i]);
+    if (s > band_hi) {
+      atomicOr(&sm.bm[id >> 5], 1u << (id & 31));
+      atomicAdd(&sm.nsure, 1u);
+    } else if (s >= band_lo) {
+      const uint32_t off = atomicAdd(&sm.bcnt, 1u);
+      if (off < (uint32_t)SR_BCAP) sm.bid_raw[off] = id;
+    }
+  }
+  __syncthreads();
+  const uint32_t nbnd = sm.bcnt;
+  if (nbnd <= (uint32_t)SR_BCAP) {
+    if (tid < (int)nbnd) {
+      const int id = sm.bid_raw[tid];
+      int pos = 0;
+      for (uint32_t j2 = 0; j2 < nbnd; ++j2) pos += sm.bid_raw[j2] < id ? 1 : 0;
+      sm.bid[pos] = id;
+    }
+    __syncthreads();
+    for (uint32_t i0 = 0; i0 < nbnd; i0 += SR_RB) {
+      const int cnt = (int)min((uint32_t)SR_RB, nbnd - i0);
+      if (tid < cnt) sm.rid[tid] = sm.bid[i0 + tid];
+      __syncthreads();
+      sr_rescore<F>(sm, a, b, cnt, qi);
+      if (tid < cnt) sm.bs[i0 + tid] = sm.rs[tid];
+    }
+    __syncthreads();
+    const uint32_t need = (uint32_t)k - sm.nsure;
+    for (uint32_t i = warp; i < nbnd; i += SR_W) {
+      const int id = sm.bid[i];
+      const double sc = sm.bs[i];
+      uint32_t rank = 0;
+      for (uint32_t j0 = 0; j0 < nbnd; j0 += 32) {
+        const uint32_t j2 = j0 + lane;
+        const bool better = j2 < nbnd && (sm.bs[j2] > sc || (sm.bs[j2] == sc && sm.bid[j2] < id));
+        rank += __popc(__ballot_sync(0xffffffffu, better));
+      }
+      if (lane == 0 && rank < need) atomicOr(&sm.bm[id >> 5], 1u << (id & 31));
+    }
+  } else {
+    // the fp32 order among the candidates: every key above tau, then the first `quota` equal
+    // to it by index
+    if (tid == 0) raise_err(a.err, CSA_DEVERR_BAND);
+    for (uint32_t i = tid; i < nc; i += SR_T) {
+      const int id = sm.cid[i];
+      const uint32_t key = sm.ckey[i];
+      if (key > tkey) atomicOr(&sm.bm[id >> 5], 1u << (id & 31));
+      else if (key == tkey) atomicOr(&sm.tb[id >> 5], 1u << (id & 31));
+    }
+    __syncthreads();
+    // (the certain entries marked above all have keys above tau, so the words hold exactly
+    // the keys above tau); now the first `quota` ties
+    const int wpt = (nw + SR_T - 1) / SR_T, a0 = tid * wpt, a1 = min(nw, a0 + wpt);
+    uint32_t c = 0;
+    for (int w = a0; w < a1; ++w) c += __popc(sm.tb[w]);
+    uint32_t tot;
+    uint32_t seen = sr_scan(c, sm.wred, &tot) - c;
+    for (int w = a0; w < a1; ++w) {
+      uint32_t keep = 0u;
+      for (uint32_t bits = sm.tb[w]; bits; bits &= bits - 1) {
+        if (seen < quota) keep |= bits & (0u - bits);
+        ++seen;
+      }
+      sm.bm[w] |= keep;
+    }
+  }
+  __syncthreads();
+  // ---- ascending write
+  const int wpt = (nw + SR_T - 1) / SR_T, a0 = tid * wpt, a1 = min(nw, a0 + wpt);
+  uint32_t c = 0;
+  for (int w = a0; w < a1; ++w) c += __popc(sm.bm[w]);
+  uint32_t written;
+  uint32_t pos = sr_scan(c, sm.wred, &written) - c;
+  for (int w = a0; w < a1; ++w)
+    for (uint32_t bits = sm.bm[w]; bits; bits &= bits - 1) {
+      if (pos < (uint32_t)k) out[pos] = 32 * w + __ffs(bits) - 1;
+      ++pos;
+    }
+  for (uint32_t i = written + tid; i < (uint32_t)k; i += SR_T) out[i] = -1;
+  if (written != (uint32_t)k && tid == 0) raise_err(a.err, CSA_DEVERR_BAND);
+}
+
 }  // namespace
 
 size_t indexer_select_row_smem(int64_t n_max) {
@@ -698,7 +889,31 @@ cudaError_t launch_indexer_select_row(const IndexerArgs& a, cudaStream_t st) {
 
 int64_t indexer_select_row_max_entries() { return SR_NMAX; }
 
+cudaError_t launch_indexer_select_stream(const IndexerArgs& a, cudaStream_t st) {
+  if (!a.stream_cand || !a.stream_meta || a.H_I > 64 || a.d_I > 128 || a.n_max > SR_NMAX || a.k > IDX_STREAM_KMAX ||
+      (a.ifmt != CSA_IFMT_E4M3 && a.ifmt != CSA_IFMT_MXFP4))
+    return cudaErrorNotSupported;
+  const size_t smem = offsetof(SrSmem, sc);
+  auto kern = a.ifmt == CSA_IFMT_E4M3 ? indexer_select_stream_kernel<CSA_IFMT_E4M3>
+                                      : indexer_select_stream_kernel<CSA_IFMT_MXFP4>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.B * a.Tq);
+  cfg.blockDim = dim3(SR_T);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  note_launch();
+  return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
 static_assert(offsetof(SrSmem, sc) % 16 == 0, "bulk copy destination");
 static_assert(offsetof(SrSmem, sc) + SR_NMAX * sizeof(float) <= 232448, "shared memory budget of one CTA (227 KB)");
+static_assert(SR_CCAP >= IDX_STREAM_CAP, "a streaming candidate list fits the candidate buffers");
 
 }  // namespace csa

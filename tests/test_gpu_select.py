@@ -129,3 +129,40 @@ def test_rows_at_and_above_the_staged_size(N):
     assert err == 0
     for b in range(B):
         _check_exact(idx[b], _oracle(qI, qs, w, kI, ks, b, n_entries[b], "e4m3"), n_entries[b], k)
+
+
+def _run_rows(qI, qs, w, kI, ks, n_entries, q_pos, k, fmt, m=4):
+    """lightning_index on prefill rows (Tq > 3): idx [B, Tq, k] and the device error word."""
+    B, Tq = qI.shape[0], qI.shape[1]
+    n_max = kI.shape[1]
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    idx = torch.empty(B, Tq, k, dtype=torch.int32, device="cuda")
+    ws = torch.empty(csa.lightning_index_workspace_size(B, Tq, n_max, k), dtype=torch.uint8, device="cuda")
+    ifmt = csa.CSA_IFMT_E4M3 if fmt == "e4m3" else csa.CSA_IFMT_MXFP4
+    csa.lightning_index(dev(qI), dev(qs), dev(w), dev(kI), dev(ks), dev(n_entries.astype(np.int32)),
+                        dev(q_pos.astype(np.int32)), k, ifmt, idx, ws, m=m)
+    torch.cuda.synchronize()
+    return idx.cpu().numpy(), csa.read_device_error()
+
+
+@pytest.mark.parametrize("k", [1024, 300])
+def test_prefill_rows_streaming_selection(k):
+    """640 query rows of one sequence (160 groups of four: the scoring kernel keeps candidate
+    lists instead of writing scores), rows whose eligible count is below and above k; the
+    selection of sampled rows equals the oracle's exact top-k."""
+    g = torch.Generator().manual_seed(46)
+    N, Tq = 8192, 640
+    qI, qs = _keys("e4m3", torch.randn(1, Tq, 64, 128, generator=g))
+    kI, ks = _keys("e4m3", torch.randn(1, N, 128, generator=g))
+    w = torch.rand(1, Tq, 64, generator=g).numpy()
+    n_entries = np.array([N])
+    q_pos = np.concatenate([np.arange(0, 4 * 2000, 4 * 2000 // 40)[:40],          # eligible 0 .. ~1950
+                            4 * N - Tq + 40 + np.arange(Tq - 40)])                 # eligible ~8000 .. N
+    q_pos = q_pos[None, :]
+    idx, err = _run_rows(qI, qs, w, kI, ks, n_entries, q_pos, k, "e4m3")
+    assert err == 0
+    rows = list(range(0, 40, 3)) + list(range(40, Tq, 37)) + [Tq - 1]
+    I = O.indexer_scores(qI[0][rows], w[0][rows], kI[0], "e4m3", qs[0][rows], ks[0])
+    for i, t in enumerate(rows):
+        n = O.n_eligible(int(q_pos[0, t]), 4, N)
+        _check_exact(idx[0, t], I[i][:n], n, k)
