@@ -270,6 +270,10 @@ constexpr size_t kHistCounters = 256;     // per row: certain count, CTAs done, 
 //   scores [R][ld] fp32 | knmax [B] | keyrange [R][2] | (decode rows:) hist [R][4096] |
 //   fhist [R][65536] | counters [R][256] | bitmap [R][ld/32] | band [R][ld] x 16 bytes
 // R = B * Tq.  knmax .. counters is one contiguous region, zeroed by one memset per call.
+// Decode rows that take the one-cluster-per-row selection use knmax and keyrange as
+// [R][kpart] partial slots (kpart <= kKpartCap(R)), written whole by the scoring kernel.
+constexpr int kKpartSlots = 512;          // at least two scoring CTAs per SM on any device
+static int kpart_cap(size_t R) { return R >= (size_t)kKpartSlots ? 1 : (int)(kKpartSlots / R); }
 struct IdxWs {
   size_t scores, knmax, keyrange, hist, fhist, counters, bitmap, cand, end, zero_end, scand, smeta;
 };
@@ -278,8 +282,9 @@ static IdxWs idx_ws_layout(int B, int Tq, int64_t n_max) {
   IdxWs L{};
   L.scores = 0;
   L.knmax = round_up(R * ld * sizeof(float), 256);
-  L.keyrange = L.knmax + round_up((size_t)B * sizeof(unsigned), 256);
-  L.hist = L.keyrange + round_up(R * 2 * sizeof(unsigned), 256);
+  const size_t slots = Tq <= kHistMaxTq ? R * kpart_cap(R) : R;
+  L.keyrange = L.knmax + round_up((slots > (size_t)B ? slots : (size_t)B) * sizeof(unsigned), 256);
+  L.hist = L.keyrange + round_up(slots * 2 * sizeof(unsigned), 256);
   L.fhist = L.counters = L.bitmap = L.cand = L.end = L.zero_end = L.hist;
   if (Tq <= kHistMaxTq) {
     L.fhist = L.hist + round_up(R * kHistBins * sizeof(unsigned), 256);
@@ -358,14 +363,25 @@ static csa_status run_lightning_index(const void* qI, const void* qI_scale, cons
     a.cand = ws + L.cand;
   }
   // zeroed per call: the key-norm bound and key ranges, and the histograms and counters when
-  // used; the streaming path needs only the bound (its pre-pass takes the keys' actual norms)
-  cudaError_t e = cudaMemsetAsync(ws + L.knmax, 0, (hist_path ? L.zero_end : stream_path ? L.keyrange : L.hist) - L.knmax,
-                                  S(stream));
+  // used; the streaming path needs only the bound (its pre-pass takes the keys' actual norms);
+  // the row path's scoring kernel writes per-split partial slots whole (nothing to zero) and
+  // starts by programmatic dependent launch (it waits for the preceding kernel before the
+  // tile of each row's newest entry and before its first write)
+  const size_t zero_bytes = (hist_path ? L.zero_end : stream_path ? L.keyrange : L.hist) - L.knmax;
+  cudaError_t e = cudaSuccess;
+  if (row_path && tc_enabled()) a.kpart = kpart_cap((size_t)B * Tq);
+  else e = cudaMemsetAsync(ws + L.knmax, 0, zero_bytes, S(stream));
   if (e == cudaSuccess && stream_path) e = launch_key_norm_max(a, S(stream));
   if (e != cudaSuccess) return CSA_ERR_CUDA;
   bool used_tc = false;
   if (tc_enabled()) {
-    e = launch_indexer_scores_tc(a, S(stream), &used_tc);       // sets a.eps_dot of its path
+    e = launch_indexer_scores_tc(a, S(stream), &used_tc);       // sets a.eps_dot (and a.kpart) of its path
+    if (e != cudaSuccess) return CSA_ERR_CUDA;
+  }
+  if (!used_tc && a.kpart > 0) {
+    // no tensor-core launch took these rows: the shared slots, zeroed, for the CUDA-core path
+    a.kpart = 0;
+    e = cudaMemsetAsync(ws + L.knmax, 0, zero_bytes, S(stream));
     if (e != cudaSuccess) return CSA_ERR_CUDA;
   }
   if (!used_tc) a.hist = a.fhist = nullptr;                    // the CUDA-core scores come without histograms

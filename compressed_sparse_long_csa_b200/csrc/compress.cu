@@ -305,6 +305,9 @@ decode_append_kernel(const T* __restrict__ Ca, const T* __restrict__ Cb, const T
                      void* __restrict__ kI_scale, int d_I,
                      const T* __restrict__ raw_new, T* __restrict__ win, const int32_t* __restrict__ win_slot, int W,
                      unsigned* err) {
+  // a dependent lightning_index may start now: it reads the key written here (each row's
+  // newest entry) only after waiting for this grid
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   constexpr int VEC = Elem<T>::VEC;
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

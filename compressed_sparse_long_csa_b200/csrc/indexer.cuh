@@ -21,6 +21,10 @@ struct IndexerArgs {
   int64_t ld;
   unsigned* knmax;            // workspace [B]: bits of max_s ||k_s||_2 (dequantised)
   unsigned* keyrange;         // workspace [B*Tq][2]: max order key, max of ~order key (= ~min) of the row's scores
+  int kpart;                  // > 0: knmax [B*Tq][kpart] and keyrange [B*Tq][kpart][2] hold one partial per
+                              // (row, entry split), each written by its scoring CTA (nothing to zero), and
+                              // the scoring kernel may overlap a preceding decode append (it waits for it
+                              // before the tile of each row's newest entry); 0: one atomic slot each
   int32_t* idx_out;           // [B*Tq, k]
   float* score_out;           // [B*Tq, k] or null
   unsigned* err;
@@ -65,6 +69,29 @@ struct RowCount {
 };
 
 __device__ __forceinline__ float round_bf16(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+
+// The key-norm bound of row `row` (sequence b) and its scores' order-key range (max key,
+// max of ~key), from the per-split partials when kpart > 0.
+__device__ __forceinline__ float load_knmax(const IndexerArgs& a, int row, int b) {
+  if (a.kpart == 0) return __uint_as_float(__ldcg(a.knmax + b));
+  uint32_t m = 0u;
+  for (int s = 0; s < a.kpart; ++s) m = max(m, __ldcg(a.knmax + (size_t)row * a.kpart + s));
+  return __uint_as_float(m);
+}
+__device__ __forceinline__ void load_keyrange(const IndexerArgs& a, int row, uint32_t* mx, uint32_t* nmn) {
+  if (a.kpart == 0) {
+    *mx = __ldcg(a.keyrange + 2 * (size_t)row);
+    *nmn = __ldcg(a.keyrange + 2 * (size_t)row + 1);
+    return;
+  }
+  uint32_t x = 0u, y = 0u;
+  for (int s = 0; s < a.kpart; ++s) {
+    x = max(x, __ldcg(a.keyrange + 2 * ((size_t)row * a.kpart + s)));
+    y = max(y, __ldcg(a.keyrange + 2 * ((size_t)row * a.kpart + s) + 1));
+  }
+  *mx = x;
+  *nmn = y;
+}
 
 // Number of entries visible to query row `row` (= b*Tq + t): all m sources <= pos.
 __device__ __forceinline__ int row_eligible(const IndexerArgs& a, int row) {

@@ -137,6 +137,8 @@ struct IdxSmem {
   int issued0;          // tile loads issued before the setup barrier
   int n_elig[G];
   int row[G];
+  int t_dep;            // tile of the row's newest entry (partial-slot mode), else -1
+  uint32_t part[3];     // the CTA's key range (max key, max ~key) and key-norm bound (partial-slot mode)
   alignas(16) float wq[G][64];
   typename std::conditional<STREAM, StreamBuf<G>, StreamNone>::type st;
 };
@@ -357,10 +359,15 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     if (t1 > t_lim) t1 = t_lim;
     sm.t_begin = t0;
     sm.t_end = t1 > t0 ? t1 : t0;
+    // partial-slot mode (one query per CTA): a preceding decode append may still be writing
+    // the row's newest key, so its tile is loaded only after waiting for that grid
+    sm.t_dep = (G == 1 && a.kpart > 0 && max_elig > 0) ? (max_elig - 1) / IT_ROWS : -1;
+    sm.part[0] = sm.part[1] = sm.part[2] = 0u;
     // the query tile and the first key tiles go out before the setup barrier (a stage's
     // first use needs no release)
-    const int n0 = sm.t_end - t0 < STAGES ? sm.t_end - t0 : STAGES;
-    if (n0 > 0) {
+    int n0 = sm.t_end - t0 < STAGES ? sm.t_end - t0 : STAGES;
+    if (sm.t_dep >= t0 && sm.t_dep < t0 + n0) n0 = sm.t_dep - t0;
+    if (sm.t_end > t0) {                      // (n0 may be 0: the first tile waits for the append)
       tc::mbar_arrive_expect_tx(&sm.qfull, G * 64 * IT_KB);
       tc::tma_load_2d(sm.q, &tmQ, &sm.qfull, 0, (b * a.Tq + qg * G) * 64);
       for (int it = 0; it < n0; ++it) {
@@ -400,6 +407,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         const uint32_t ph = (it / STAGES) & 1;
         if (!tc::mbar_wait(&sm.empty[st], ph ^ 1)) { atomicExch(&sm.abort_flag, 1); break; }
         if (*(volatile int*)&sm.abort_flag) break;
+        if (t_begin + it == sm.t_dep) tc::griddep_wait();
         tc::mbar_arrive_expect_tx(&sm.full[st], IT_TILE_BYTES);
         tc::tma_load_2d(sm.k[st], &tmK, &sm.full[st], 0, (int)(b * a.n_max) + (t_begin + it) * IT_ROWS);
         ++issued;
@@ -445,12 +453,17 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     const int r = quarter * 32 + lane;
     const float* kscale = (const float*)a.kI_scale;
     float kmax = 0.f;
+    const int t_dep = sm.t_dep;
     // the key scale of the group's next tile is loaded before waiting for the current accumulator
     auto load_scale = [&](int it) {
       const int s = (t_begin + it) * IT_ROWS + r;
-      return (it < n_t && s < a.n_max) ? __ldg(kscale + (size_t)b * a.n_max + s) : 0.f;
+      if (it < n_t && t_begin + it == t_dep) tc::griddep_wait();
+      return (it < n_t && s < a.n_max) ? __ldcg(kscale + (size_t)b * a.n_max + s) : 0.f;
     };
     float sk_next = load_scale(e);
+    // partial-slot mode: no global write before the preceding grid has finished (it may
+    // still read this workspace)
+    if (G == 1 && a.kpart > 0) tc::griddep_wait();
     KeyRange kr[G];
     for (int it = e; it < n_t; it += 2) {
       const int acc = it % NACC;
@@ -478,11 +491,21 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&sm.tempty[acc]);
     }
-#pragma unroll
-    for (int g = 0; g < G; ++g) flush_key_range(a.keyrange, sm.row[g], kr[g]);
     // |k8| <= 448 per element, so ||k_s|| <= sk * 448 * sqrt(d_I)
     kmax = warp_max(kmax);
-    if (lane == 0 && kmax > 0.f) atomicMax(a.knmax + b, __float_as_uint(kmax * 448.f * 11.3137085f * 1.0001f));
+    if (t_dep >= 0 || (G == 1 && a.kpart > 0)) {
+      // the CTA's partials, reduced in shared memory and written to its own slots at the end
+      const uint32_t mx = __reduce_max_sync(0xffffffffu, kr[0].mx), mn = __reduce_max_sync(0xffffffffu, kr[0].nmn);
+      if (lane == 0) {
+        atomicMax(&sm.part[0], mx);
+        atomicMax(&sm.part[1], mn);
+        if (kmax > 0.f) atomicMax(&sm.part[2], __float_as_uint(kmax * 448.f * 11.3137085f * 1.0001f));
+      }
+    } else {
+#pragma unroll
+      for (int g = 0; g < G; ++g) flush_key_range(a.keyrange, sm.row[g], kr[g]);
+      if (lane == 0 && kmax > 0.f) atomicMax(a.knmax + b, __float_as_uint(kmax * 448.f * 11.3137085f * 1.0001f));
+    }
   } else if (warp >= 4) {
     if constexpr (STREAM) {
       // the streaming selection (see StreamBuf): candidates instead of scores
@@ -613,6 +636,15 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, NCOLS);
   }
+  if (G == 1 && !STREAM && a.kpart > 0 && threadIdx.x == 0) {
+    // a CTA that never reached the newest tile still waits once, so that this grid ends
+    // after the append it may overlap (the kernels after it rely on that order)
+    tc::griddep_wait();
+    const size_t slot = (size_t)sm.row[0] * a.kpart + split;
+    a.keyrange[2 * slot] = sm.part[0];
+    a.keyrange[2 * slot + 1] = sm.part[1];
+    a.knmax[slot] = sm.part[2];
+  }
   if (HIST && a.hist) hist_flush(sm.fwin, sm.fbase, a, (size_t)sm.row[0]);
 }
 
@@ -645,6 +677,8 @@ struct MxSmem {
   int t_begin, t_end;
   int issued0;          // tile loads issued before the setup barrier
   int n_elig;
+  int t_dep;            // tile of the row's newest entry (partial-slot mode), else -1
+  uint32_t part[3];     // the CTA's key range (max key, max ~key) and key-norm bound (partial-slot mode)
   alignas(16) float w[64];
 };
 
@@ -686,9 +720,13 @@ indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     if (t1 > t_lim) t1 = t_lim;
     sm.t_begin = t0;
     sm.t_end = t1 > t0 ? t1 : t0;
+    // partial-slot mode: the tile of the row's newest entry waits for a preceding decode append
+    sm.t_dep = (a.kpart > 0 && ne > 0) ? (ne - 1) / IT_ROWS : -1;
+    sm.part[0] = sm.part[1] = sm.part[2] = 0u;
     // the query tile and the first key tiles go out before the setup barrier
-    const int n0 = sm.t_end - t0 < STAGES ? sm.t_end - t0 : STAGES;
-    if (n0 > 0) {
+    int n0 = sm.t_end - t0 < STAGES ? sm.t_end - t0 : STAGES;
+    if (sm.t_dep >= t0 && sm.t_dep < t0 + n0) n0 = sm.t_dep - t0;
+    if (sm.t_end > t0) {                      // (n0 may be 0: the first tile waits for the append)
       tc::mbar_arrive_expect_tx(&sm.qfull, 64 * MX_KB);
       tc::tma_load_2d(sm.q, &tmQ, &sm.qfull, 0, row * 64);
       for (int it = 0; it < n0; ++it) {
@@ -717,6 +755,7 @@ indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         const uint32_t ph = (it / STAGES) & 1;
         if (!tc::mbar_wait(&sm.empty[st], ph ^ 1)) { atomicExch(&sm.abort_flag, 1); break; }
         if (*(volatile int*)&sm.abort_flag) break;
+        if (t_begin + it == sm.t_dep) tc::griddep_wait();
         tc::mbar_arrive_expect_tx(&sm.full[st], MX_TILE_BYTES);
         tc::tma_load_2d(sm.k[st], &tmK, &sm.full[st], 0, (int)(b * a.n_max) + (t_begin + it) * IT_ROWS);
         ++issued;
@@ -766,10 +805,11 @@ indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     }
     auto load4 = [&](int it, uint32_t* v) {
       const int s0 = (t_begin + it) * IT_ROWS + lane;
+      if (it < n_t && t_begin + it == sm.t_dep) tc::griddep_wait();
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int s = s0 + 32 * c;
-        v[c] = (it < n_t && s < a.n_max) ? __ldg(ksc + (size_t)b * a.n_max + s) : 0u;
+        v[c] = (it < n_t && s < a.n_max) ? __ldcg(ksc + (size_t)b * a.n_max + s) : 0u;
       }
     };
     uint32_t nxt[4];
@@ -795,9 +835,11 @@ indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     float kb = 0.f;
     auto load_sc = [&](int it) {
       const int s = (t_begin + it) * IT_ROWS + r;
-      return (it < n_t && s < a.n_max) ? __ldg(ksc + (size_t)b * a.n_max + s) : 0u;
+      if (it < n_t && t_begin + it == sm.t_dep) tc::griddep_wait();
+      return (it < n_t && s < a.n_max) ? __ldcg(ksc + (size_t)b * a.n_max + s) : 0u;
     };
     uint32_t sc_next = load_sc(e);
+    if (a.kpart > 0) tc::griddep_wait();                   // no global write before the preceding grid ends
     KeyRange kr;
     for (int it = e; it < n_t; it += 2) {
       const int acc = it % MX_NACC;
@@ -848,9 +890,18 @@ indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&sm.tempty[acc]);
     }
-    flush_key_range(a.keyrange, row, kr);
     kb = warp_max(kb);
-    if (lane == 0 && kb > 0.f) atomicMax(a.knmax + b, __float_as_uint(kb * 1.0001f));
+    if (a.kpart > 0) {
+      const uint32_t mx = __reduce_max_sync(0xffffffffu, kr.mx), mn = __reduce_max_sync(0xffffffffu, kr.nmn);
+      if (lane == 0) {
+        atomicMax(&sm.part[0], mx);
+        atomicMax(&sm.part[1], mn);
+        if (kb > 0.f) atomicMax(&sm.part[2], __float_as_uint(kb * 1.0001f));
+      }
+    } else {
+      flush_key_range(a.keyrange, row, kr);
+      if (lane == 0 && kb > 0.f) atomicMax(a.knmax + b, __float_as_uint(kb * 1.0001f));
+    }
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -858,6 +909,13 @@ indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   if (warp == 1) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, MX_COLS);
+  }
+  if (a.kpart > 0 && threadIdx.x == 0) {
+    tc::griddep_wait();                                      // this grid ends after the append
+    const size_t slot = (size_t)row * a.kpart + split;
+    a.keyrange[2 * slot] = sm.part[0];
+    a.keyrange[2 * slot + 1] = sm.part[1];
+    a.knmax[slot] = sm.part[2];
   }
   if (a.hist) hist_flush(sm.fwin, sm.fbase, a, (size_t)row);
 }
@@ -902,7 +960,24 @@ bool make_map_rows64(CUtensorMap* m, const void* base, uint64_t rows, uint32_t b
   return r == CUDA_SUCCESS;
 }
 
-cudaError_t launch_mxf4(const IndexerArgs& a, cudaStream_t st, bool* used) {
+// A launch with programmatic stream serialization (the kernel may start while the previous
+// one in the stream runs; it waits for it with griddepcontrol.wait before dependent reads).
+template <typename K, typename... Args>
+cudaError_t launch_pdl(K kern, dim3 grid, int threads, size_t smem, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+cudaError_t launch_mxf4(const IndexerArgs& a, cudaStream_t st, bool* used, int* kpart_out) {
   constexpr int STAGES = 8;
   IdxTcParams p{};
   p.a = a;
@@ -910,6 +985,7 @@ cudaError_t launch_mxf4(const IndexerArgs& a, cudaStream_t st, bool* used) {
   p.tiles = (int)((a.n_max + IT_ROWS - 1) / IT_ROWS);
   const int64_t ctas = (int64_t)a.B * a.Tq;
   int splits = (int)(2 * num_sms() / ctas);         // one wave: two CTAs per SM
+  if (a.kpart > 0 && splits > a.kpart) splits = a.kpart;   // the partial slots a row has
   if (splits > p.tiles) splits = p.tiles;
   if (splits < 1) splits = 1;
   p.tiles_per_split = (p.tiles + splits - 1) / splits;
@@ -921,17 +997,23 @@ cudaError_t launch_mxf4(const IndexerArgs& a, cudaStream_t st, bool* used) {
   cudaError_t e = cudaFuncSetAttribute(indexer_mxf4_kernel<STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
+  if (a.kpart > 0) p.a.kpart = splits;
   dim3 grid(splits, a.Tq, a.B);
   note_launch();
-  indexer_mxf4_kernel<STAGES><<<grid, MX_THREADS, smem, st>>>(mk, mq, p);
   *used = true;
+  if (a.kpart > 0) {
+    *kpart_out = splits;
+    return launch_pdl(indexer_mxf4_kernel<STAGES>, grid, MX_THREADS, smem, st, mk, mq, p);
+  }
+  indexer_mxf4_kernel<STAGES><<<grid, MX_THREADS, smem, st>>>(mk, mq, p);
   return cudaGetLastError();
 }
 
 template <int G, int STAGES, bool HIST, bool STREAM = false>
-cudaError_t launch_g(const IndexerArgs& a, cudaStream_t st, bool* used) {
+cudaError_t launch_g(const IndexerArgs& a, cudaStream_t st, bool* used, int* kpart_out) {
   IdxTcParams p{};
   p.a = a;
+  if (G != 1) p.a.kpart = 0;
   p.n_qg = (a.Tq + G - 1) / G;
   p.tiles = (int)((a.n_max + IT_ROWS - 1) / IT_ROWS);
   // decode-like shapes: split the entry tiles so that the grid fills the SMs once
@@ -940,6 +1022,7 @@ cudaError_t launch_g(const IndexerArgs& a, cudaStream_t st, bool* used) {
   const int64_t ctas = (int64_t)a.B * p.n_qg;
   const int64_t slots = G == 1 ? 2 * num_sms() : num_sms();
   int splits = STREAM ? 1 : (int)(slots / ctas);
+  if (G == 1 && a.kpart > 0 && splits > a.kpart) splits = a.kpart;
   if (splits > p.tiles) splits = p.tiles;
   if (splits < 1) splits = 1;
   p.tiles_per_split = (p.tiles + splits - 1) / splits;
@@ -951,10 +1034,15 @@ cudaError_t launch_g(const IndexerArgs& a, cudaStream_t st, bool* used) {
   cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<G, STAGES, HIST, STREAM>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  if (G == 1 && a.kpart > 0) p.a.kpart = splits;
   dim3 grid(splits, p.n_qg, a.B);
   note_launch();
-  indexer_tc_kernel<G, STAGES, HIST, STREAM><<<grid, IT_THREADS, smem, st>>>(mk, mq, p);
   *used = true;
+  if (G == 1 && a.kpart > 0) {
+    *kpart_out = splits;
+    return launch_pdl(indexer_tc_kernel<G, STAGES, HIST, STREAM>, grid, IT_THREADS, smem, st, mk, mq, p);
+  }
+  indexer_tc_kernel<G, STAGES, HIST, STREAM><<<grid, IT_THREADS, smem, st>>>(mk, mq, p);
   return cudaGetLastError();
 }
 
@@ -1014,7 +1102,10 @@ cudaError_t launch_indexer_scores_tc(IndexerArgs& a, cudaStream_t st, bool* used
     if ((int64_t)a.B * a.n_max > 0x7fffffffLL || (int64_t)a.B * a.Tq * 64 > 0x7fffffffLL) return cudaSuccess;
     // same bound as the E4M3 kernel
     a.eps_dot = 1.0f / 131072.0f;
-    return launch_mxf4(a, st, used);
+    int kp = 0;
+    const cudaError_t e = launch_mxf4(a, st, used, &kp);
+    if (*used) a.kpart = kp;
+    return e;
   }
   if (a.ifmt != CSA_IFMT_E4M3 || a.H_I != 64 || a.d_I != 128) return cudaSuccess;
   if (((uintptr_t)a.kI & 15) || ((uintptr_t)a.qI & 15)) return cudaSuccess;
@@ -1023,12 +1114,17 @@ cudaError_t launch_indexer_scores_tc(IndexerArgs& a, cudaStream_t st, bool* used
   // fp32 accumulation of exact products (128 * 2^-24 = 2^-17).  Measured on B200: <= 5e-9
   // relative to the bound's scale (test_indexer_fp32_score_error_within_band_bound).
   a.eps_dot = 1.0f / 131072.0f;
-  if (a.stream_cand) return launch_g<4, 6, false, true>(a, st, used);
-  if (a.Tq >= 4) return launch_g<4, 6, false>(a, st, used);
+  // a.kpart on return: the partial slots per row the launch wrote (0: the shared atomic slots)
+  int kp = 0;
+  cudaError_t e;
+  if (a.stream_cand) e = launch_g<4, 6, false, true>(a, st, used, &kp);
+  else if (a.Tq >= 4) e = launch_g<4, 6, false>(a, st, used, &kp);
   // decode rows: the score histogram for the selection (one fewer ring stage makes room
   // for it at two CTAs per SM)
-  if (a.hist) return launch_g<1, 5, true>(a, st, used);
-  return launch_g<1, 6, false>(a, st, used);
+  else if (a.hist) e = launch_g<1, 5, true>(a, st, used, &kp);
+  else e = launch_g<1, 6, false>(a, st, used, &kp);
+  if (*used) a.kpart = kp;
+  return e;
 }
 
 }  // namespace csa

@@ -640,9 +640,11 @@ indexer_select_cluster_kernel(IndexerArgs a, int chunk) {
     }
   }
   if (n > k && tid < m - m4) sv[m4 + tid] = srow[m4 + tid];
-  const float knmax = __uint_as_float(a.knmax[b]);
+  const float knmax = load_knmax(a, row, b);
   // the key range the scoring kernel recorded (exact min / max over the row's eligible entries)
-  uint32_t lo_k = ~a.keyrange[2 * (size_t)row + 1], hi_k = a.keyrange[2 * (size_t)row];
+  uint32_t hi_k, lo_k;
+  load_keyrange(a, row, &hi_k, &lo_k);
+  lo_k = ~lo_k;
   if (tid < HI) {
     sh.w[tid] = w_r;
     if (F == CSA_IFMT_E4M3) sh.qsc[tid] = qs_r[0];

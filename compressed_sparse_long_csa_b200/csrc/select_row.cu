@@ -77,6 +77,7 @@ struct SrSmem {
   uint32_t wred[SR_W];
   alignas(8) uint64_t bar[(SR_NMAX * 4 + SR_CHUNK - 1) / SR_CHUNK];   // one per bulk copy
   uint32_t bin, above, ccnt, bcnt, nsure, fail;
+  uint32_t kr_mx, kr_nmn, kn;             // the row's key range and key-norm bound (reduced over partials)
   float U;
   alignas(16) float sc[1];                // the row's scores (sized at launch)
 };
@@ -379,9 +380,31 @@ indexer_select_row_kernel(IndexerArgs a) {
     }
   }
   for (int i = tid; i < SR_HB; i += SR_T) sm.hist[i] = 0u;
-  const uint32_t klo = ~__ldcg(a.keyrange + 2 * (size_t)row + 1), khi = __ldcg(a.keyrange + 2 * (size_t)row);
-  const float knmax = __uint_as_float(__ldcg(a.knmax + b));
+  if (warp == 0) {
+    // the scoring kernel's key range and key-norm bound: one value, or one per split
+    uint32_t x = 0u, y = 0u, z = 0u;
+    if (a.kpart == 0) {
+      if (lane == 0) {
+        x = __ldcg(a.keyrange + 2 * (size_t)row);
+        y = __ldcg(a.keyrange + 2 * (size_t)row + 1);
+        z = __ldcg(a.knmax + b);
+      }
+    } else {
+      for (int s = lane; s < a.kpart; s += 32) {
+        const size_t slot = (size_t)row * a.kpart + s;
+        x = max(x, __ldcg(a.keyrange + 2 * slot));
+        y = max(y, __ldcg(a.keyrange + 2 * slot + 1));
+        z = max(z, __ldcg(a.knmax + slot));
+      }
+    }
+    x = __reduce_max_sync(0xffffffffu, x);
+    y = __reduce_max_sync(0xffffffffu, y);
+    z = __reduce_max_sync(0xffffffffu, z);
+    if (lane == 0) sm.kr_mx = x, sm.kr_nmn = y, sm.kn = z;
+  }
   __syncthreads();
+  const uint32_t klo = ~sm.kr_nmn, khi = sm.kr_mx;
+  const float knmax = __uint_as_float(sm.kn);
   const float* sc = sm.sc;
   const float4* sc4 = reinterpret_cast<const float4*>(sc);
   const int nw = (n + 31) >> 5;

@@ -486,10 +486,12 @@ indexer_select_kernel(IndexerArgs a) {
   const float* S = a.scores + (size_t)row * a.ld;
   // the scoring kernel recorded this row's key range; the k-th largest fp32 score
   // lies in histogram bin [f_lo, f_hi]
-  const uint32_t kmax = a.keyrange[2 * (size_t)row], kmin = ~a.keyrange[2 * (size_t)row + 1];
+  uint32_t kmax, knmn;
+  load_keyrange(a, row, &kmax, &knmn);
+  const uint32_t kmin = ~knmn;
   const BinSel bs = hist_select(sh, n, k, [&](int i) { return f32_order_key(S[i]); }, kmin, kmax);
   const float f_lo = f32_from_order_key(bs.key_lo), f_hi = f32_from_order_key(bs.key_hi);
-  const float knmax = __uint_as_float(a.knmax[b]);
+  const float knmax = load_knmax(a, row, b);
   const float E = a.eps_dot * sh.U * knmax + 1.52587890625e-05f * fmaxf(fabsf(f_lo), fabsf(f_hi));  // 2^-16 |tau|
   // every score is within E of its exact value, so entries above f_hi + 2E are in and
   // entries below f_lo - 2E are out; the band between is re-scored exactly

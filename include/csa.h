@@ -293,7 +293,17 @@ csa_status grouped_out_proj(const void* o, int T, int H, int dv, int g, int d_mi
  * s < min(n_entries[b], (pos+1)/m) (all of an entry's tokens are <= pos).  The
  * k entries with the largest I are returned, ties to the lower index, in
  * ascending index order, padded with -1.  Selection is exact: tensor-core fp32
- * scores pick a candidate band which is re-scored in fp64 on CUDA cores.
+ * scores pick a candidate band which is re-scored exactly on CUDA cores
+ * (integer dot products of the E4M3 / MXFP4 codes, fp64 for F32 operands).
+ *
+ * Stream order: for decode rows (Tq <= 3, E4M3 or MXFP4) the scoring kernel is
+ * launched with programmatic dependent launch.  It may start while the kernel
+ * before it in the stream is still running, and it waits for that kernel to
+ * finish before it reads the key tile holding each row's newest eligible
+ * entry and before any write.  So the preceding kernel may produce only those
+ * newest keys (csa_decode_append does); every other input must be complete
+ * before it starts, as it is after any kernel that does not trigger its
+ * dependents early.
  *
  *   qI       device [B, Tq, H_I, d_I] (F32: fp32; E4M3: bytes; MXFP4: [.., d_I/2] bytes)
  *   qI_scale E4M3: device [B, Tq, H_I] fp32; MXFP4: [B, Tq, H_I, d_I/32] bytes; F32: NULL
