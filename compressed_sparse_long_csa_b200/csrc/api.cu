@@ -341,11 +341,13 @@ static csa_status run_lightning_index(const void* qI, const void* qI_scale, cons
   a.idx_out = idx_out; a.score_out = score_out; a.err = err;
   a.score_bf16 = bf16_scores ? 1 : 0;
   // decode rows of the exact call (the bf16-key call selects on the stored keys with the
-  // plain top-k): rows that fit one CTA's shared memory take the one-CTA-per-row selection
-  // over the staged scores (no histograms); longer rows the histogram-seeded one
+  // plain top-k): rows that fit one CTA's shared memory take the one-cluster-per-row selection
+  // over the staged scores, longer rows the same over chunks staged across a cluster (no
+  // histograms either way); rows beyond that the histogram-seeded one
   const bool decode_rows = Tq <= kHistMaxTq && !bf16_scores;
+  const bool row_fits = n_max <= indexer_select_row_max_entries();
   const bool row_path = decode_rows && (ifmt == CSA_IFMT_E4M3 || ifmt == CSA_IFMT_MXFP4) &&
-                        n_max <= indexer_select_row_max_entries();
+                        (row_fits || indexer_select_dist_clusters(a) > 0);
   const bool hist_path = decode_rows && !row_path;
   // prefill rows that one CTA per four queries scores completely: the streaming selection
   // (candidates instead of scores; nothing to zero)
@@ -402,7 +404,7 @@ static csa_status run_lightning_index(const void* qI, const void* qI_scale, cons
     return cuda_status(launch_indexer_select_stream(a, S(stream)));
   }
   if (row_path && used_tc) {
-    const cudaError_t er = launch_indexer_select_row(a, S(stream));
+    const cudaError_t er = row_fits ? launch_indexer_select_row(a, S(stream)) : launch_indexer_select_dist(a, S(stream));
     if (er != cudaErrorNotSupported) return cuda_status(er);
   }
   return cuda_status(launch_indexer_select(a, S(stream)));

@@ -160,6 +160,10 @@ bool indexer_stream_applies(const IndexerArgs& a);
 // knmax[b] = the largest key norm of sequence b (E4M3 keys of width 128; knmax zeroed before).
 cudaError_t launch_key_norm_max(const IndexerArgs& a, cudaStream_t st);
 int64_t indexer_select_row_max_entries();
+// Rows longer than one CTA stages: one cluster per row over chunks of it (select_row.cu).
+// indexer_select_dist_clusters: its cluster size for these rows, 0 when it does not apply.
+int indexer_select_dist_clusters(const IndexerArgs& a);
+cudaError_t launch_indexer_select_dist(const IndexerArgs& a, cudaStream_t st);
 cudaError_t launch_topk_select_cluster(const float* scores, int64_t ld, RowCount rc, int R, int64_t n,
                                        int k, int32_t* idx_out, cudaStream_t st);
 

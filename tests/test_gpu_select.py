@@ -3,9 +3,11 @@
 tests do not reach: rows of different eligible counts, just above and at k; every key
 identical (all scores tie: the lowest indices win); scores packed into one narrow range
 (more candidates than the selection stages on chip); the exact scores returned with the
-selection; rows at the largest size one CTA stages in shared memory (24 576 entries, three
-bulk copies) and just above it (the multi-CTA selection).  Expected values come from the
-oracle only.
+selection; rows around the sizes whose scores take several bulk copies; rows longer than one
+CTA stages (34 816 entries), which a cluster selects over chunks of the row: ragged eligible
+counts across the chunks, a row at or below k beside longer ones, all scores tied (the
+counted search of the k-th key and the fp32 order), the exact scores.  Expected values come
+from the oracle only.
 """
 from __future__ import annotations
 
@@ -129,6 +131,41 @@ def test_rows_at_and_above_the_staged_size(N):
     assert err == 0
     for b in range(B):
         _check_exact(idx[b], _oracle(qI, qs, w, kI, ks, b, n_entries[b], "e4m3"), n_entries[b], k)
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "mxfp4"])
+def test_rows_longer_than_one_cta_stages(fmt):
+    """Rows of 70 000 entries: chunks of one cluster; eligible counts that end inside a chunk,
+    on a chunk boundary region and far below the row's length, one at most k."""
+    g = torch.Generator().manual_seed(47)
+    B, N, k = 4, 70000, 1024
+    qI, qs = _keys(fmt, torch.randn(B, 1, 64, 128, generator=g))
+    kI, ks = _keys(fmt, torch.randn(B, N, 128, generator=g))
+    w = torch.rand(B, 1, 64, generator=g).numpy()
+    n_entries = np.array([N, 40001, 1000, 34817])
+    idx, so, err = _run(qI, qs, w, kI, ks, n_entries, 4 * n_entries - 1, k, fmt, score_out=True)
+    assert err == 0
+    for b in range(B):
+        I = _oracle(qI, qs, w, kI, ks, b, n_entries[b], fmt)
+        _check_exact(idx[b], I, n_entries[b], k)
+        sel = idx[b][idx[b] >= 0]
+        assert np.array_equal(so[b][:sel.size], I[sel].astype(np.float32))
+        assert np.all(so[b][sel.size:] == 0)
+
+
+def test_long_rows_all_scores_tie():
+    """Every key identical on rows a cluster selects in chunks: the k-th key comes from the
+    counted search, the band outgrows its buffer (flagged), and the k lowest indices win
+    across the chunks."""
+    g = torch.Generator().manual_seed(48)
+    B, N, k = 2, 50000, 512
+    qI, qs = _keys("e4m3", torch.randn(B, 1, 64, 128, generator=g))
+    kI, ks = _keys("e4m3", torch.randn(1, 1, 128, generator=g).expand(B, N, 128).contiguous())
+    w = torch.rand(B, 1, 64, generator=g).numpy()
+    n_entries = np.array([N, N - 3])
+    idx, _, err = _run(qI, qs, w, kI, ks, n_entries, 4 * n_entries - 1, k, "e4m3")
+    assert err & ~0x8 == 0                            # only CSA_DEVERR_BAND may be set
+    assert np.array_equal(idx, np.tile(np.arange(k), (B, 1)))
 
 
 def _run_rows(qI, qs, w, kI, ks, n_entries, q_pos, k, fmt, m=4):
