@@ -52,10 +52,11 @@ constexpr int SR_HB = 4096;               // bins of the first histogram
 constexpr int SR_HB2 = 2048;              // bins of the refinements
 constexpr int SR_CCAP = 2048;             // candidates listed
 constexpr int SR_BCAP = 512;              // band entries re-scored exactly (at most one per thread: the sort)
-constexpr int SR_RB = 8;                  // entries re-scored at once
+constexpr int SR_RB = 8;                  // entries re-scored at once (one per thread of a head's eight)
 constexpr int SR_NMAX = 34816;            // most scores a row stages in shared memory (and bitmap bits)
 constexpr int SR_CHUNK = 16384;           // bytes per bulk copy (the first histogram starts on the first)
 constexpr int SR_KLD = 160;               // staged key row: dims 16 g .. 16 g + 15 at word 20 g (no bank conflicts)
+static_assert(SR_RB == 8, "the re-scoring gives each of a head's eight threads one entry");
 constexpr int SR_TLD = 66;                // per-head term row stride (the ordered sums read rows side by side)
 constexpr int SD_CMAX = 16;               // CTAs per cluster of the chunked selection (above 8: non-portable size)
 constexpr int SD_LCAP = 1024;             // candidates (or band entries) one CTA of it lists
@@ -93,7 +94,7 @@ struct SrSmem {
   uint32_t kr_mx, kr_nmn, kn;             // the row's key range and key-norm bound (reduced over partials)
   float U;
   // chunked selection only
-  uint32_t hsum[SR_HB];                   // the cluster's histogram: this CTA's slice of it
+  uint32_t hsum[SR_HB / 2];               // the cluster's histogram: this CTA's slice of it (C >= 2)
   int32_t lid[SD_LCAP];                   // this chunk's candidates (row indices) and their keys
   uint32_t lkey[SD_LCAP];
   SdXchg x;
@@ -155,6 +156,17 @@ __device__ __forceinline__ void sr_find_bin(SrSmem& sm, uint32_t want) {
       sm.above = above;
     }
     above += c[i];
+  }
+  __syncthreads();
+}
+
+// The band's exact scores sm.bs[0, nbnd) replaced in place by monotone 64-bit keys (x + 0.0
+// folds -0 into +0; exact scores are never NaN), so that ranking compares integers instead of
+// running on the fp64 pipe.  All threads call (one barrier).
+__device__ __forceinline__ void sr_band_keys(SrSmem& sm, uint32_t nbnd) {
+  for (uint32_t i = threadIdx.x; i < nbnd; i += SR_T) {
+    const uint64_t u = (uint64_t)__double_as_longlong(sm.bs[i] + 0.0);
+    reinterpret_cast<uint64_t*>(sm.bs)[i] = (u >> 63) ? ~u : (u | 0x8000000000000000ull);
   }
   __syncthreads();
 }
@@ -235,14 +247,14 @@ __device__ __forceinline__ void sr_rescore(SrSmem& sm, const IndexerArgs& a, int
         acc[e] = x;
       }
     }
-    if (g == 0 && j < HI) {
-      const double wj = (double)sm.w[j], qs = (double)sm.qsc[j];
+    // every lane of the head holds the sums: thread g forms the term of entry g (the fp64
+    // pipe is narrow on this GPU, so the terms go to all lanes rather than one per head)
+    long long mine = 0;
 #pragma unroll
-      for (int e = 0; e < SR_RB; ++e)
-        if (e < cnt) {
-          const double D = (qs * (double)sm.ksc[e][0]) * ((double)acc[e] * 3.814697265625e-06);   // 2^-18
-          sm.term[e][j] = wj * fmax(D, 0.0);
-        }
+    for (int e = 0; e < SR_RB; ++e) mine = e == g ? acc[e] : mine;
+    if (j < HI && g < cnt) {
+      const double D = ((double)sm.qsc[j] * (double)sm.ksc[g][0]) * ((double)mine * 3.814697265625e-06);   // 2^-18
+      sm.term[g][j] = (double)sm.w[j] * fmax(D, 0.0);
     }
   } else {
     int acc[SR_RB];
@@ -260,26 +272,29 @@ __device__ __forceinline__ void sr_rescore(SrSmem& sm, const IndexerArgs& a, int
         }
       }
     }
+    // the 32-dim block q of a head sums lanes 2q and 2q + 1 of its eight; thread g takes the
+    // block sums of entry g and forms its term (blocks added in order)
+    int P[4] = {0, 0, 0, 0};
 #pragma unroll
     for (int e = 0; e < SR_RB; ++e) {
       if (e < cnt) {
-        const int x = acc[e] + __shfl_xor_sync(0xffffffffu, acc[e], 1);   // the 32-dim block of lanes g, g ^ 1
-        // the block partials at the head's first lane, in block order
-        const int p1 = __shfl_down_sync(0xffffffffu, x, 2);
-        const int p2 = __shfl_down_sync(0xffffffffu, x, 4);
-        const int p3 = __shfl_down_sync(0xffffffffu, x, 6);
-        if (g == 0 && j < HI) {
-          const int P[4] = {x, p1, p2, p3};
-          double D = 0.0;
+        const int x = acc[e] + __shfl_xor_sync(0xffffffffu, acc[e], 1);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            if (q >= nb) break;
-            const double t = ((double)sm.qsc[j * nb + q] * (double)sm.ksc[e][q]) * ((double)P[q] * 0.25);
-            D = q == 0 ? t : D + t;
-          }
-          sm.term[e][j] = (double)sm.w[j] * fmax(D, 0.0);
+        for (int q = 0; q < 4; ++q) {
+          const int pq = __shfl_sync(0xffffffffu, x, (lane & ~7) | (2 * q));
+          P[q] = e == g ? pq : P[q];
         }
       }
+    }
+    if (j < HI && g < cnt) {
+      double D = 0.0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (q >= nb) break;
+        const double t = ((double)sm.qsc[j * nb + q] * (double)sm.ksc[g][q]) * ((double)P[q] * 0.25);
+        D = q == 0 ? t : D + t;
+      }
+      sm.term[g][j] = (double)sm.w[j] * fmax(D, 0.0);
     }
   }
   __syncthreads();
@@ -655,13 +670,15 @@ indexer_select_row_kernel(IndexerArgs a) {
   if (band_ok) {
     // ---- 6. rank the band by (exact score desc, index asc); the first k - certain are chosen
     const uint32_t need = (uint32_t)k - sm.nsure;
+    sr_band_keys(sm, nbnd);
+    const uint64_t* bk = reinterpret_cast<const uint64_t*>(sm.bs);
     for (uint32_t i = warp; i < nbnd; i += SR_W) {
       const int id = sm.bid[i];
-      const double s = sm.bs[i];
+      const uint64_t s = bk[i];
       uint32_t rank = 0;
       for (uint32_t j0 = 0; j0 < nbnd; j0 += 32) {
         const uint32_t j2 = j0 + lane;
-        const bool better = j2 < nbnd && (sm.bs[j2] > s || (sm.bs[j2] == s && sm.bid[j2] < id));
+        const bool better = j2 < nbnd && (bk[j2] > s || (bk[j2] == s && sm.bid[j2] < id));
         rank += __popc(__ballot_sync(0xffffffffu, better));
       }
       if (lane == 0 && rank < need) atomicOr(&sm.bm[id >> 5], 1u << (id & 31));
@@ -833,13 +850,15 @@ indexer_select_stream_kernel(IndexerArgs a) {
     }
     __syncthreads();
     const uint32_t need = (uint32_t)k - sm.nsure;
+    sr_band_keys(sm, nbnd);
+    const uint64_t* bk = reinterpret_cast<const uint64_t*>(sm.bs);
     for (uint32_t i = warp; i < nbnd; i += SR_W) {
       const int id = sm.bid[i];
-      const double sc = sm.bs[i];
+      const uint64_t sc = bk[i];
       uint32_t rank = 0;
       for (uint32_t j0 = 0; j0 < nbnd; j0 += 32) {
         const uint32_t j2 = j0 + lane;
-        const bool better = j2 < nbnd && (sm.bs[j2] > sc || (sm.bs[j2] == sc && sm.bid[j2] < id));
+        const bool better = j2 < nbnd && (bk[j2] > sc || (bk[j2] == sc && sm.bid[j2] < id));
         rank += __popc(__ballot_sync(0xffffffffu, better));
       }
       if (lane == 0 && rank < need) atomicOr(&sm.bm[id >> 5], 1u << (id & 31));
@@ -1111,9 +1130,13 @@ indexer_select_dist_kernel(IndexerArgs a, int L) {
     uint32_t part = 0;
     for (int i = tid; i < S; i += SR_T) {
       const int bin = crank * S + i;
+      uint32_t r[SD_CMAX];
+#pragma unroll
+      for (int p = 0; p < SD_CMAX; ++p) r[p] = p < C ? *cluster.map_shared_rank(&sm.hist[bin], (unsigned)p) : 0u;
       uint32_t v = 0;
-      for (int p = 0; p < C; ++p) v += *cluster.map_shared_rank(&sm.hist[bin], (unsigned)p);
-      sm.hsum[bin] = v;
+#pragma unroll
+      for (int p = 0; p < SD_CMAX; ++p) v += r[p];
+      sm.hsum[i] = v;
       part += v;
     }
     uint32_t stot;
@@ -1130,7 +1153,7 @@ indexer_select_dist_kernel(IndexerArgs a, int L) {
   }
   {
     const uint32_t* oh = cluster.map_shared_rank(sm.hsum, (unsigned)ss);
-    for (int i = tid; i < SR_HB; i += SR_T) sm.hist[i] = i < S ? oh[ss * S + i] : 0u;
+    for (int i = tid; i < SR_HB; i += SR_T) sm.hist[i] = i < S ? oh[i] : 0u;
   }
   __syncthreads();
   if (S >= 2048) sr_find_bin<4>(sm, (uint32_t)k - above);
@@ -1211,17 +1234,13 @@ indexer_select_dist_kernel(IndexerArgs a, int L) {
   int rnd = 0;
   uint32_t tkey;
   if (listed) {
-    // every chunk's candidates, in chunk order
-    uint32_t off = 0;
-    for (int p = 0; p < C; ++p) {
-      const uint32_t cp = sm.x.ncand[p];
-      const int32_t* rid = cluster.map_shared_rank(sm.lid, (unsigned)p);
-      const uint32_t* rk = cluster.map_shared_rank(sm.lkey, (unsigned)p);
-      for (uint32_t i = tid; i < cp; i += SR_T) {
-        sm.cid[off + i] = rid[i];
-        sm.ckey[off + i] = rk[i];
-      }
-      off += cp;
+    // every chunk's candidates, in chunk order (each thread's remote loads independent)
+    for (uint32_t f = tid; f < ncand; f += SR_T) {
+      int p = 0;
+      uint32_t o = 0;
+      while (f >= o + sm.x.ncand[p]) o += sm.x.ncand[p++];
+      sm.cid[f] = cluster.map_shared_rank(sm.lid, (unsigned)p)[f - o];
+      sm.ckey[f] = cluster.map_shared_rank(sm.lkey, (unsigned)p)[f - o];
     }
     __syncthreads();
     // ---- the exact k-th largest key inside [blo, bhi]: by ranking the bin's candidates
@@ -1339,12 +1358,11 @@ indexer_select_dist_kernel(IndexerArgs a, int L) {
     band_ok = !bovf && nbt <= (uint32_t)SR_BCAP;
     __syncthreads();                                         // sm.bcnt read above
     if (band_ok) {
-      uint32_t off = 0;
-      for (int p = 0; p < C; ++p) {
-        const uint32_t cp = sm.x.nband[p];
-        const int32_t* rid = cluster.map_shared_rank(sm.lid, (unsigned)p);
-        for (uint32_t i = tid; i < cp; i += SR_T) sm.bid_raw[off + i] = rid[i];
-        off += cp;
+      for (uint32_t f = tid; f < nbt; f += SR_T) {
+        int p = 0;
+        uint32_t o = 0;
+        while (f >= o + sm.x.nband[p]) o += sm.x.nband[p++];
+        sm.bid_raw[f] = cluster.map_shared_rank(sm.lid, (unsigned)p)[f - o];
       }
     }
     if (tid == 0) sm.bcnt = nbt;
@@ -1375,13 +1393,15 @@ indexer_select_dist_kernel(IndexerArgs a, int L) {
     uint32_t nsure = 0;
     for (int p = 0; p < C; ++p) nsure += sm.sure[p];
     const uint32_t need = (uint32_t)k > nsure ? (uint32_t)k - nsure : 0u;
+    sr_band_keys(sm, nbnd);
+    const uint64_t* bk = reinterpret_cast<const uint64_t*>(sm.bs);
     for (uint32_t i = warp; i < nbnd; i += SR_W) {
       const int id = sm.bid[i];
-      const double s = sm.bs[i];
+      const uint64_t s = bk[i];
       uint32_t rank = 0;
       for (uint32_t j0 = 0; j0 < nbnd; j0 += 32) {
         const uint32_t j2 = j0 + lane;
-        const bool better = j2 < nbnd && (sm.bs[j2] > s || (sm.bs[j2] == s && sm.bid[j2] < id));
+        const bool better = j2 < nbnd && (bk[j2] > s || (bk[j2] == s && sm.bid[j2] < id));
         rank += __popc(__ballot_sync(0xffffffffu, better));
       }
       if (lane == 0 && rank < need) {
