@@ -99,6 +99,7 @@ __device__ __forceinline__ void hist_flush(const uint32_t* fwin, uint32_t fbase,
 // and the entries below it leave.  At the end the lists go to the workspace with the
 // threshold, U and the key-norm bound they used, and the selection kernel finishes each row
 // from its list (select_row.cu).  No score leaves the SM.
+constexpr int IT_PF = 4;                   // key scales fetched this many tiles (of a thread's own) ahead
 constexpr int ST_T = 256;                  // epilogue threads (warps 4..11)
 constexpr int ST_HB = 2048;                // bins of the compaction histograms (all rows)
 constexpr int ST_PAIRS = 2;                // pairs of tiles between two meetings of the epilogue threads
@@ -460,7 +461,11 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
       if (it < n_t && t_begin + it == t_dep) tc::griddep_wait();
       return (it < n_t && s < a.n_max) ? __ldcg(kscale + (size_t)b * a.n_max + s) : 0.f;
     };
-    float sk_next = load_scale(e);
+    // IT_PF of the group's tiles ahead: a scale fetched one group tile ahead tied the tile
+    // rate to the memory latency (about 0.5 us per tile whatever the ring depth)
+    float skq[IT_PF];
+#pragma unroll
+    for (int d = 0; d < IT_PF; ++d) skq[d] = load_scale(e + 2 * d);
     // partial-slot mode: no global write before the preceding grid has finished (it may
     // still read this workspace)
     if (G == 1 && a.kpart > 0) tc::griddep_wait();
@@ -468,8 +473,10 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     for (int it = e; it < n_t; it += 2) {
       const int acc = it % NACC;
       const uint32_t aph = (it / NACC) & 1;
-      const float sk = sk_next;
-      sk_next = load_scale(it + 2);
+      const float sk = skq[0];
+#pragma unroll
+      for (int d = 0; d + 1 < IT_PF; ++d) skq[d] = skq[d + 1];
+      skq[IT_PF - 1] = load_scale(it + 2 * IT_PF);
       bool ok = tc::mbar_wait(&sm.tfull[acc], aph) && !*(volatile int*)&sm.abort_flag;
       ok = __all_sync(0xffffffffu, ok);               // the TMEM loads below are warp-collective
       if (!ok) { atomicExch(&sm.abort_flag, 1); break; }
@@ -812,13 +819,19 @@ indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         v[c] = (it < n_t && s < a.n_max) ? __ldcg(ksc + (size_t)b * a.n_max + s) : 0u;
       }
     };
-    uint32_t nxt[4];
-    load4(0, nxt);
+    // the scales of IT_PF tiles ahead (one tile ahead tied the tile rate to the memory latency)
+    uint32_t nxt[IT_PF][4];
+#pragma unroll
+    for (int d = 0; d < IT_PF; ++d) load4(d, nxt[d]);
     for (int it = 0; it < n_t; ++it) {
       const int st = it % STAGES;
       const uint32_t ph = (it / STAGES) & 1;
-      uint32_t cur[4] = {nxt[0], nxt[1], nxt[2], nxt[3]};
-      load4(it + 1, nxt);
+      uint32_t cur[4] = {nxt[0][0], nxt[0][1], nxt[0][2], nxt[0][3]};
+#pragma unroll
+      for (int d = 0; d + 1 < IT_PF; ++d)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) nxt[d][c] = nxt[d + 1][c];
+      load4(it + IT_PF, nxt[IT_PF - 1]);
       bool ok = tc::mbar_wait(&sm.empty[st], ph ^ 1) && !*(volatile int*)&sm.abort_flag;
       if (!__all_sync(0xffffffffu, ok)) { atomicExch(&sm.abort_flag, 1); break; }
       tc::fence_after_sync();
@@ -838,7 +851,9 @@ indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       if (it < n_t && t_begin + it == sm.t_dep) tc::griddep_wait();
       return (it < n_t && s < a.n_max) ? __ldcg(ksc + (size_t)b * a.n_max + s) : 0u;
     };
-    uint32_t sc_next = load_sc(e);
+    uint32_t scq[IT_PF];
+#pragma unroll
+    for (int d = 0; d < IT_PF; ++d) scq[d] = load_sc(e + 2 * d);
     if (a.kpart > 0) tc::griddep_wait();                   // no global write before the preceding grid ends
     KeyRange kr;
     for (int it = e; it < n_t; it += 2) {
@@ -846,8 +861,10 @@ indexer_mxf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       const uint32_t aph = (it / MX_NACC) & 1;
       const int s = (t_begin + it) * IT_ROWS + r;
       const bool valid = s < sm.n_elig;
-      const uint32_t sc = sc_next;
-      sc_next = load_sc(it + 2);
+      const uint32_t sc = scq[0];
+#pragma unroll
+      for (int d = 0; d + 1 < IT_PF; ++d) scq[d] = scq[d + 1];
+      scq[IT_PF - 1] = load_sc(it + 2 * IT_PF);
       // ||k_s|| <= 6 * sqrt(32 * sum_b scale_b^2): |e2m1| <= 6
       if (valid) {
         float ss = 0.f;
