@@ -44,17 +44,17 @@ L2_BYTES = 126 * 1024 * 1024
 TENSOR_PEAKS = {}   # measured once per single-GPU run (measure_tensor_peaks)
 
 TRAFFIC = {
-    # profiles/csa_decode_64k_dram_traffic.md: indexer_tc_kernel<1,6> 34 771 200 + indexer_select_row 1 368 960
-    ("csa_decode_64k", "indexer"): 36140160,
-    # profiles/hybrid_pair_1m_dram_traffic.md: indexer_mxf4_kernel 142 688 512 read + 5 260 288 written (its
-    # scores) + indexer_select_dist 8 668 800
-    ("hybrid_pair_1m", "indexer"): 156617600,
+    # profiles/csa_decode_64k_dram_traffic.md: indexer_tc_kernel<1,6> 34 773 632 + indexer_select_row 1 369 984
+    ("csa_decode_64k", "indexer"): 36143616,
+    # profiles/hybrid_pair_1m_dram_traffic.md: indexer_mxf4_kernel 142 688 000 read + 5 062 784 written (its
+    # scores) + indexer_select_dist 8 670 080
+    ("hybrid_pair_1m", "indexer"): 156420864,
     # profiles/hca_decode_1m_launches.md: attn_tc_kernel 39 008 896 read + 2 304 written (the combine's
     # reads are L2 hits in the timed step; under ncu the caches are flushed before each kernel)
     ("hca_decode_1m", "attention"): 39011200,
-    # profiles/csa_prefill_4k_launches.md: attn_tc_kernel 829 513 216 read (cache rows, queries, raw
-    # window) + 511 258 624 written (the 537 MB bf16 output, partly still in L2 at the kernel's end)
-    ("csa_prefill_4k", "attention"): 1340771840,
+    # profiles/csa_prefill_4k_launches.md: attn_tc_kernel 831 254 272 read (cache rows, queries, raw
+    # window) + 513 781 248 written (the 537 MB bf16 output, partly still in L2 at the kernel's end)
+    ("csa_prefill_4k", "attention"): 1345035520,
 }
 
 
