@@ -445,7 +445,8 @@ def run_ours(args, wid, name):
     bf16_peak = peaks.get("bf16_tflops", 1590.0)
     tpeaks = TENSOR_PEAKS.get("v") if world == 1 else None
     # the dominant ABI call by time; decode calls are HBM-bound, prefill calls tensor-bound
-    # (the FP8 indexer against twice the measured bf16 peak, the nominal dense ratio)
+    # (the FP8 indexer against the measured FP8 MMA rate, else twice the measured bf16 peak,
+    # the nominal dense ratio)
     cand = [c for c in comp if c in ab]
     dom = max(cand, key=lambda c: mean_ms[comp.index(c)])
     dom_ms = float(mean_ms[comp.index(dom)])
@@ -496,6 +497,7 @@ def run_ours(args, wid, name):
                        l2=f"inputs rotated over {n_copies} copies ({n_copies * step_bytes / 1e6:.0f} MB, over 3x the "
                           f"126 MB L2 between reuses); no flush"),
         "hbm_gbs_step": sum(ab.values()) / (ms_per_step * 1e-3) / 1e9,
+        "hbm_frac_step": sum(ab.values()) / (ms_per_step * 1e-3) / 1e9 / hbm_peak,
         "breakdown_ms": {c: float(m) for c, m in zip(comp, mean_ms)},
         "roofline": roof,
         "e2e": e2e,
