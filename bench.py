@@ -587,7 +587,9 @@ def measure_bf16_index(wid, D, T, csa, steps, l2_flush, exact_ms, reps=20):
         return None
     exact = T["idx"].clone()
     idx = torch.empty_like(T["idx"])
-    ws = torch.empty_like(T["iws"])
+    # the bf16-key call writes its scores: the full workspace (the step's may omit that region)
+    ws = torch.empty(csa.lightning_index_workspace_size(D["B"], D["Tq"], D["n_max"], D["k"]), dtype=torch.uint8,
+                     device="cuda")
 
     def call():
         csa.lightning_index_bf16(T["qI"], T.get("qI_scale"), T["w"], T["kI"], T.get("kI_scale"), T["n_entries"],

@@ -35,6 +35,7 @@ _SIGS = {
     "grouped_out_proj": ([_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp], _i32),
     "hca_compress": ([_vp] * 5 + [_i64, _i32, _i32, _i32, _i32, _i32, _vp], _i32),
     "lightning_index_workspace_size": ([_i32, _i32, _i64, _i32], _sz),
+    "lightning_index_workspace_size_exact": ([_i32, _i32, _i64, _i32, _i32, _i32, _i32], _sz),
     "lightning_index": ([_vp] * 7 + [_i32, _i32, _i32, _i32, _i32, _i64, _i32, _i32, _vp, _vp, _vp, _sz, _vp], _i32),
     "lightning_index_bf16": ([_vp] * 7 + [_i32, _i32, _i32, _i32, _i32, _i64, _i32, _i32, _vp, _vp, _sz, _vp], _i32),
     "topk_select_workspace_size": ([_i32, _i64, _i32], _sz),
@@ -186,6 +187,10 @@ def hca_compress(C_, Z, bias, entry0, cache, m_prime=128, stream=None):
 
 def lightning_index_workspace_size(B, Tq, n_max, k):
     return int(lib.lightning_index_workspace_size(B, Tq, n_max, k))
+
+
+def lightning_index_workspace_size_exact(B, Tq, n_max, k, ifmt, H_I, d_I):
+    return int(lib.lightning_index_workspace_size_exact(B, Tq, n_max, k, ifmt, H_I, d_I))
 
 
 def lightning_index(qI, qI_scale, w, kI, kI_scale, n_entries, q_pos, k, ifmt, idx_out, workspace,

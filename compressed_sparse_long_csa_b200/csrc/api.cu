@@ -277,11 +277,12 @@ static int kpart_cap(size_t R) { return R >= (size_t)kKpartSlots ? 1 : (int)(kKp
 struct IdxWs {
   size_t scores, knmax, keyrange, hist, fhist, counters, bitmap, cand, end, zero_end, scand, smeta;
 };
-static IdxWs idx_ws_layout(int B, int Tq, int64_t n_max) {
+// with_scores = false (prefill rows of the streamed selection only): no score region.
+static IdxWs idx_ws_layout(int B, int Tq, int64_t n_max, bool with_scores = true) {
   const size_t R = (size_t)B * Tq, ld = (size_t)idx_ld(n_max);
   IdxWs L{};
   L.scores = 0;
-  L.knmax = round_up(R * ld * sizeof(float), 256);
+  L.knmax = with_scores ? round_up(R * ld * sizeof(float), 256) : 0;
   const size_t slots = Tq <= kHistMaxTq ? R * kpart_cap(R) : R;
   L.keyrange = L.knmax + round_up((slots > (size_t)B ? slots : (size_t)B) * sizeof(unsigned), 256);
   L.hist = L.keyrange + round_up(slots * 2 * sizeof(unsigned), 256);
@@ -308,6 +309,20 @@ size_t lightning_index_workspace_size(int B, int Tq, int64_t n_max, int k) {
   return idx_ws_layout(B, Tq, n_max).end;
 }
 
+// Prefill rows that the streamed selection takes (the exact call without score_out) need no
+// score region.  The same test decides the call's layout.
+static bool idx_streamed_shape(int B, int Tq, int64_t n_max, int k, int ifmt, int H_I, int d_I) {
+  if (!tc_enabled() || Tq <= kHistMaxTq) return false;
+  IndexerArgs a{};
+  a.B = B; a.Tq = Tq; a.n_max = n_max; a.k = k; a.ifmt = ifmt; a.H_I = H_I; a.d_I = d_I;
+  return indexer_stream_applies(a);
+}
+
+size_t lightning_index_workspace_size_exact(int B, int Tq, int64_t n_max, int k, int ifmt, int H_I, int d_I) {
+  if (B < 1 || Tq < 1 || n_max < 1) return 0;
+  return idx_ws_layout(B, Tq, n_max, !idx_streamed_shape(B, Tq, n_max, k, ifmt, H_I, d_I)).end;
+}
+
 static csa_status run_lightning_index(const void* qI, const void* qI_scale, const float* w, const void* kI,
                                       const void* kI_scale, const int32_t* n_entries, const int32_t* q_pos, int m,
                                       int B, int Tq, int H_I, int d_I, int64_t n_max, int k, int ifmt,
@@ -322,8 +337,10 @@ static csa_status run_lightning_index(const void* qI, const void* qI_scale, cons
   if (score_out) REQUIRE(aligned16(score_out), CSA_ERR_ALIGN);
   REQUIRE(aligned16(qI) && aligned16(kI), CSA_ERR_ALIGN);
   REQUIRE(n_entries && q_pos, CSA_ERR_NULL);
-  const size_t need = lightning_index_workspace_size(B, Tq, n_max, k);
-  REQUIRE(workspace && ws_bytes >= need, CSA_ERR_WORKSPACE);
+  // the streamed prefill selection writes no scores: its layout has no score region
+  const bool streamed = !bf16_scores && !score_out && idx_streamed_shape(B, Tq, n_max, k, ifmt, H_I, d_I);
+  const IdxWs L = idx_ws_layout(B, Tq, n_max, !streamed);
+  REQUIRE(workspace && ws_bytes >= L.end, CSA_ERR_WORKSPACE);
   REQUIRE(aligned16(workspace), CSA_ERR_ALIGN);
   unsigned* err = device_error_word();
   REQUIRE(err, CSA_ERR_CUDA);
@@ -333,7 +350,6 @@ static csa_status run_lightning_index(const void* qI, const void* qI_scale, cons
   a.n_entries = n_entries; a.q_pos = q_pos; a.m = m;
   a.B = B; a.Tq = Tq; a.H_I = H_I; a.d_I = d_I; a.n_max = n_max; a.k = k; a.ifmt = ifmt;
   a.ld = idx_ld(n_max);
-  const IdxWs L = idx_ws_layout(B, Tq, n_max);
   char* ws = (char*)workspace;
   a.scores = (float*)(ws + L.scores);
   a.knmax = (unsigned*)(ws + L.knmax);
@@ -351,10 +367,9 @@ static csa_status run_lightning_index(const void* qI, const void* qI_scale, cons
   const bool hist_path = decode_rows && !row_path;
   // prefill rows that one CTA per four queries scores completely: the streaming selection
   // (candidates instead of scores; nothing to zero)
-  if (Tq > kHistMaxTq && !bf16_scores && tc_enabled()) {
+  if (streamed) {
     a.stream_cand = reinterpret_cast<uint2*>(ws + L.scand);
     a.stream_meta = reinterpret_cast<uint4*>(ws + L.smeta);
-    if (!indexer_stream_applies(a)) a.stream_cand = nullptr, a.stream_meta = nullptr;
   }
   const bool stream_path = a.stream_cand != nullptr;
   if (hist_path) {

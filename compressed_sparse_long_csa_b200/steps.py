@@ -45,8 +45,9 @@ def upload(wl, device="cuda"):
         T["n_entries"] = torch.full((B,), D["N"], **i32)
         T["q_pos"] = (D["q_pos0"] + torch.arange(Tq, dtype=torch.int32)).repeat(B, 1).to(device)
         T["idx"] = torch.empty(B, Tq, D["k"], **i32)
-        T["iws"] = torch.empty(N.lightning_index_workspace_size(B, Tq, D["n_max"], D["k"]), dtype=torch.uint8,
-                               device=device)
+        # the exact call's own size: prefill rows that stream candidates need no score region
+        T["iws"] = torch.empty(N.lightning_index_workspace_size_exact(B, Tq, D["n_max"], D["k"], _ifmt(D), D["HI"],
+                                                                       D["dI"]), dtype=torch.uint8, device=device)
         T["out"] = torch.empty(B, Tq, D["H"], D["dv"], dtype=lat, device=device)
         T["lse"] = torch.empty(B, Tq, D["H"], dtype=torch.float32, device=device)
         if kind == "csa_prefill":

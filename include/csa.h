@@ -313,12 +313,20 @@ csa_status grouped_out_proj(const void* o, int T, int H, int dv, int g, int d_mi
  *   n_entries device [B] int32, q_pos device [B, Tq] int32
  *   idx_out  device [B, Tq, k] int32;  score_out device [B, Tq, k] fp32 or NULL
  *            (the fp64 score of each selected entry rounded to fp32; 0 for pads)
- *   workspace >= lightning_index_workspace_size(B, Tq, n_max, k) bytes
+ *   workspace >= lightning_index_workspace_size(B, Tq, n_max, k) bytes (or, with
+ *            score_out NULL, lightning_index_workspace_size_exact(...) bytes)
  * Supported: B*Tq <= 65535, H_I <= 64, d_I in {32, 64, 128}, k <= 2048,
  * n_max <= 2^24.  qI, kI, score_out and workspace must be 16-byte aligned
  * (CSA_ERR_ALIGN otherwise).
  * ------------------------------------------------------------------------- */
 size_t lightning_index_workspace_size(int B, int Tq, int64_t n_max, int k);
+/* The bytes lightning_index itself (score_out NULL) needs for these shapes on the current
+ * device: prefill rows whose selection streams candidates instead of scores (E4M3 keys,
+ * H_I 64, d_I 128, k <= 1024, Tq >= 4 and enough rows to fill the device) need no score
+ * region, about B*Tq*n_max*4 bytes less; otherwise the same as
+ * lightning_index_workspace_size.  A call with score_out, or lightning_index_bf16, needs
+ * lightning_index_workspace_size.  0 for empty shapes. */
+size_t lightning_index_workspace_size_exact(int B, int Tq, int64_t n_max, int k, int ifmt, int H_I, int d_I);
 csa_status lightning_index(const void* qI, const void* qI_scale, const float* w,
                            const void* kI, const void* kI_scale,
                            const int32_t* n_entries, const int32_t* q_pos, int m,

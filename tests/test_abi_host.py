@@ -285,3 +285,21 @@ def test_package_has_no_cpu_fallback():
     src = open(os.path.join(os.path.dirname(csa.__file__), "_native.py")).read() + \
         open(os.path.join(os.path.dirname(csa.__file__), "steps.py")).read()
     assert "oracle" not in src
+
+
+def test_exact_indexer_workspace_drops_the_score_region_only_for_streamed_prefill_rows():
+    """lightning_index_workspace_size_exact: the 4096-token prefill chunk (E4M3, 64 x 128,
+    k 1024) needs no [rows, n_max] fp32 score region; decode rows, MXFP4 keys, k above 1024
+    and too few query groups to fill the device keep the full size (host-side sizes only)."""
+    full = csa.lightning_index_workspace_size
+    exact = csa.lightning_index_workspace_size_exact
+    E, M = csa.CSA_IFMT_E4M3, csa.CSA_IFMT_MXFP4
+    B, Tq, N, k = 1, 4096, 33792, 1024
+    assert full(B, Tq, N, k) - exact(B, Tq, N, k, E, 64, 128) >= Tq * N * 4
+    assert exact(B, Tq, N, k, E, 64, 128) >= Tq * 2048 * 8          # the candidate lists stay
+    for args in [(16, 1, 16384, 512, E), (8, 1, 262144, 1024, M), (B, Tq, N, k, M), (B, Tq, N, 2048, E),
+                 (1, 8, N, k, E)]:
+        b, t, n, kk, f = args
+        assert exact(b, t, n, kk, f, 64, 128) == full(b, t, n, kk), args
+    assert exact(B, Tq, N, k, E, 32, 128) == full(B, Tq, N, k)
+    assert exact(0, Tq, N, k, E, 64, 128) == 0

@@ -168,22 +168,25 @@ def test_long_rows_all_scores_tie():
     assert np.array_equal(idx, np.tile(np.arange(k), (B, 1)))
 
 
-def _run_rows(qI, qs, w, kI, ks, n_entries, q_pos, k, fmt, m=4):
-    """lightning_index on prefill rows (Tq > 3): idx [B, Tq, k] and the device error word."""
+def _run_rows(qI, qs, w, kI, ks, n_entries, q_pos, k, fmt, m=4, exact_ws=False):
+    """lightning_index on prefill rows (Tq > 3): idx [B, Tq, k] and the device error word;
+    exact_ws: a workspace of exactly lightning_index_workspace_size_exact bytes."""
     B, Tq = qI.shape[0], qI.shape[1]
     n_max = kI.shape[1]
     dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
     idx = torch.empty(B, Tq, k, dtype=torch.int32, device="cuda")
-    ws = torch.empty(csa.lightning_index_workspace_size(B, Tq, n_max, k), dtype=torch.uint8, device="cuda")
     ifmt = csa.CSA_IFMT_E4M3 if fmt == "e4m3" else csa.CSA_IFMT_MXFP4
+    size = (csa.lightning_index_workspace_size_exact(B, Tq, n_max, k, ifmt, qI.shape[2], qI.shape[3]) if exact_ws
+            else csa.lightning_index_workspace_size(B, Tq, n_max, k))
+    ws = torch.empty(size, dtype=torch.uint8, device="cuda")
     csa.lightning_index(dev(qI), dev(qs), dev(w), dev(kI), dev(ks), dev(n_entries.astype(np.int32)),
                         dev(q_pos.astype(np.int32)), k, ifmt, idx, ws, m=m)
     torch.cuda.synchronize()
     return idx.cpu().numpy(), csa.read_device_error()
 
 
-@pytest.mark.parametrize("k", [1024, 300])
-def test_prefill_rows_streaming_selection(k):
+@pytest.mark.parametrize("k,exact_ws", [(1024, False), (300, False), (1024, True)])
+def test_prefill_rows_streaming_selection(k, exact_ws):
     """640 query rows of one sequence (160 groups of four: the scoring kernel keeps candidate
     lists instead of writing scores), rows whose eligible count is below and above k; the
     selection of sampled rows equals the oracle's exact top-k."""
@@ -196,7 +199,10 @@ def test_prefill_rows_streaming_selection(k):
     q_pos = np.concatenate([np.arange(0, 4 * 2000, 4 * 2000 // 40)[:40],          # eligible 0 .. ~1950
                             4 * N - Tq + 40 + np.arange(Tq - 40)])                 # eligible ~8000 .. N
     q_pos = q_pos[None, :]
-    idx, err = _run_rows(qI, qs, w, kI, ks, n_entries, q_pos, k, "e4m3")
+    if exact_ws:      # the streamed rows' workspace holds no score matrix
+        assert (csa.lightning_index_workspace_size(1, Tq, N, k) -
+                csa.lightning_index_workspace_size_exact(1, Tq, N, k, csa.CSA_IFMT_E4M3, 64, 128)) >= Tq * N * 4
+    idx, err = _run_rows(qI, qs, w, kI, ks, n_entries, q_pos, k, "e4m3", exact_ws=exact_ws)
     assert err == 0
     rows = list(range(0, 40, 3)) + list(range(40, Tq, 37)) + [Tq - 1]
     I = O.indexer_scores(qI[0][rows], w[0][rows], kI[0], "e4m3", qs[0][rows], ks[0])
