@@ -168,6 +168,38 @@ def test_long_rows_all_scores_tie():
     assert np.array_equal(idx, np.tile(np.arange(k), (B, 1)))
 
 
+def test_rows_beyond_the_chunked_cluster_size():
+    """600 000 entries, more than 16 chunks of 34 816 scores, so the histogram-seeded
+    selection (several CTAs per row, the last one finishes) takes the row.  Every key is a
+    power of two a_s (1, 2, 4 or 8) times one fixed key v with e2m1 values, so each MXFP4 key
+    decodes exactly to a_s v and every score is exactly a_s times the score of v (positive
+    head weights): the top-k is every entry of the highest level, then the lowest indices
+    of the next, with no oracle pass over 600 000 entries (ties flag CSA_DEVERR_BAND)."""
+    g = torch.Generator().manual_seed(49)
+    B, N, k = 1, 600000, 1024
+    n = N - 5
+    qI, qs = _keys("mxfp4", torch.randn(B, 1, 64, 128, generator=g))
+    e2m1 = torch.tensor([0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    v = e2m1[torch.randint(0, 7, (128,), generator=g)] * torch.where(torch.rand(128, generator=g) < 0.5, -1.0, 1.0)
+    level = torch.full((N,), 2.0)
+    level[torch.rand(N, generator=g) < 0.3] = 4.0
+    level[torch.rand(N, generator=g) < 0.2] = 1.0
+    top = torch.randperm(n, generator=g)[:700]
+    level[top] = 8.0
+    kI, ks = _keys("mxfp4", (level[:, None] * v[None, :])[None])
+    w = torch.rand(B, 1, 64, generator=g).numpy()
+    # the construction, checked on the oracle: the four levels score exactly 1, 2, 4, 8 times v's
+    kl, kls = _keys("mxfp4", (torch.tensor([1.0, 2.0, 4.0, 8.0])[:, None] * v[None, :])[None])
+    I_l = O.indexer_scores(qI[0], w[0], kl[0], "mxfp4", qs[0], kls[0])[0]
+    assert I_l[0] > 0 and np.array_equal(I_l / I_l[0], [1.0, 2.0, 4.0, 8.0])
+    lv = level[:n].numpy()
+    order = np.lexsort((np.arange(n), -lv))
+    exp = np.sort(order[:k])
+    idx, _, err = _run(qI, qs, w, kI, ks, np.array([n]), 4 * np.array([n]) - 1, k, "mxfp4")
+    assert err & ~0x8 == 0                            # only CSA_DEVERR_BAND may be set
+    assert np.array_equal(idx[0], exp)
+
+
 def _run_rows(qI, qs, w, kI, ks, n_entries, q_pos, k, fmt, m=4, exact_ws=False):
     """lightning_index on prefill rows (Tq > 3): idx [B, Tq, k] and the device error word;
     exact_ws: a workspace of exactly lightning_index_workspace_size_exact bytes."""
