@@ -303,3 +303,19 @@ def test_exact_indexer_workspace_drops_the_score_region_only_for_streamed_prefil
         assert exact(b, t, n, kk, f, 64, 128) == full(b, t, n, kk), args
     assert exact(B, Tq, N, k, E, 32, 128) == full(B, Tq, N, k)
     assert exact(0, Tq, N, k, E, 64, 128) == 0
+
+
+def test_exact_indexer_workspace_is_what_the_call_checks():
+    """The streamed prefill call accepts exactly lightning_index_workspace_size_exact bytes and
+    refuses one byte less; with score_out it needs the full size (both refusals happen
+    before any device work)."""
+    B, Tq, n_max, k, E = 1, 4096, 33792, 1024, csa.CSA_IFMT_E4M3
+    exact = csa.lightning_index_workspace_size_exact(B, Tq, n_max, k, E, 64, 128)
+    full = csa.lightning_index_workspace_size(B, Tq, n_max, k)
+
+    def call(wsb, so=None):
+        return N.lib.lightning_index(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, B, Tq, 64, 128, n_max, k, E, FAKE, so,
+                                     FAKE, wsb, None)
+    assert call(exact - 1) == ERR_WS
+    assert call(exact, so=FAKE) == ERR_WS        # score_out: the scores are written, so the full size
+    assert exact < full
